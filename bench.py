@@ -1,0 +1,404 @@
+"""Benchmark of the LSA decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config ctx500k] [--impl reference]
+
+One bench step is one tau window: a refresh decode step (full index scan,
+I >= 0.5 selection, cold-pool fetch, top-k, attention) followed by tau-1 = 63
+listed decode steps (re-score of the kept set, top-k, attention), i.e. every
+stage of the path.  `value` is decode steps/s of the whole job (all ranks);
+one decode step advances every sequence of the batch by one token.
+
+Inputs are resident in HBM (the cold pool in page-locked host memory) before
+the timed region.  L2: three replicas of the indexer keys, each with its own
+context and hot buffer, are rotated window by window (3 x 66 MB > 126 MB L2).
+`e2e` repeats the measurement through lsa_decode_step_host with the per-step
+inputs in page-locked host memory and the outputs copied back every step.
+
+Multi-GPU: every rank runs an independent batch (different seed), no data-path
+collective; the window time is the max over ranks (weak scaling).
+
+--impl reference runs the fp64 CPU oracle (the reference arm of this
+method-only build) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LSA decode steps/s at 500K ctx; indexer-scan HBM GB/s vs B200 peak"
+UNIT = "decode steps/s"
+FALLBACK_HBM_GBS = 6650.0
+REPLICAS = 3
+
+WORKLOAD_DESC = {
+    "ctx500k": "500K-token context decode: B=4, N=131072 compressed entries/seq, e4m3 indexer keys (per-row fp32 "
+               "scale) H_idx=64 d_idx=128, ~10% planted + 1% leakage, top-k 2048, bf16 MQA 128 heads x D=512 over "
+               "a latent KV head, 512 MB pinned host cold pool, hot buffer 20% of N",
+    "ctx128k": "128K-token context decode: B=1, N=32768, bf16 indexer keys H_idx=64 d_idx=128, 12% planted, "
+               "top-k 2048, bf16 MQA 128 heads x D=512",
+    "ragged": "ragged serving batch: 64 sequences of 16K-256K tokens (4:1), bf16 keys, planted 2-30%, top-k 2048",
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="ctx500k", choices=sorted(WORKLOAD_DESC))
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--hot-frac", type=float, default=0.2)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", FALLBACK_HBM_GBS)), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def scan_traffic_record():
+    """dram bytes per scan launch from the committed ncu summary, if it matches the current kernel source."""
+    import hashlib
+
+    rec = os.path.join(ROOT, "profiles", "scan_traffic.txt")
+    if not os.path.exists(rec):
+        return None
+    kv = {}
+    for line in open(rec):
+        if "=" in line and not line.startswith("#"):
+            a, b = line.strip().split("=", 1)
+            kv[a.strip()] = b.strip()
+    src = os.path.join(ROOT, "lookahead_sparse_kv_index_b200", "csrc", kv.get("kernel_file", "index_score_tc.cu"))
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if sha != kv.get("kernel_src_sha256"):
+        return None
+    try:
+        return float(kv["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.f = None
+
+    def start(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower().startswith("active")})
+        load = [s for s in sm if mx and s >= 0.5 * max(mx)] or sm
+        return {"sm_mhz": float(np.median(load)) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------- reference (oracle)
+
+def oracle_window_sample(wl, n_listed=1):
+    """Oracle time of one refresh step and `n_listed` listed steps; extrapolated tau-window time."""
+    import oracle
+    from oracle.stepper import OracleDecoder
+
+    dec = OracleDecoder(wl, tau=wl.tau)
+    t0 = time.perf_counter()
+    dec.step(0, *wl.step_inputs(0), with_gather=True)
+    t_ref = time.perf_counter() - t0
+    t_list = []
+    for t in range(1, 1 + n_listed):
+        inp = wl.step_inputs(t)
+        t0 = time.perf_counter()
+        dec.step(t, *inp)
+        t_list.append(time.perf_counter() - t0)
+    t_step = float(np.mean(t_list))
+    window = t_ref + (wl.tau - 1) * t_step
+    return wl.tau / window, dict(t_refresh_s=t_ref, t_listed_s=t_step, cores=oracle.num_threads())
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    import synth
+
+    wl = synth.CONFIGS[args.config](with_cold=True)
+    oracle.build()
+    vals = []
+    info = {}
+    for i in range(args.warmup + args.steps):
+        v, info = oracle_window_sample(wl)
+        if i >= args.warmup:
+            vals.append(v)
+    value = float(np.mean(vals))
+    sample = ("per bench step: 1 refresh decode step (full fp64 scan, selection, gather, top-k, attention) + 1 "
+              "listed decode step of the same workload on the host cores, extrapolated to a tau=64 window")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.tau / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD_DESC[args.config], "tau": wl.tau,
+                                         "bench_step": "one tau window = 64 decode steps"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": info.get("cores"), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------- CUDA arm
+
+def algorithmic_scan_bytes(wl):
+    n = wl.n_total
+    key_b = {"f32": 4, "bf16": 2, "e4m3": 1}[wl.key_dtype]
+    per_entry = wl.d * key_b + (4 if wl.k_scale is not None else 0) + 4   # key row (+ scale) + z out
+    per_seq = wl.H * wl.d * (2 if wl.q_dtype == "bf16" else 4) + wl.H * 4
+    return n * per_entry + wl.B * per_seq
+
+
+def run_cuda(args):
+    import torch
+
+    import synth
+    from lookahead_sparse_kv_index_b200 import lsa
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    pg = None
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
+        pg = dist
+
+    wl = synth.CONFIGS[args.config](seed={"ctx500k": 2, "ctx128k": 1, "ragged": 3}[args.config] + 1000 * rank)
+    dev = synth.to_torch(wl)
+    cap = max(wl.topk, int(args.hot_frac * wl.n_total))
+    ctxs, keys = [], []
+    for r in range(REPLICAS):
+        kr = dev["keys"].clone() if r else dev["keys"]
+        keys.append(kr)
+        ctxs.append(lsa.Context(B=wl.B, H=wl.H, d=wl.d, q_dtype=wl.q_dtype, k_dtype=wl.key_dtype, Hq=wl.Hq,
+                                D=wl.D, attn_dtype=wl.attn_dtype, topk=wl.topk, seq_off_host=wl.seq_off, keys=kr,
+                                k_scale=dev["k_scale"], cold_host=dev["cold"], row_bytes=wl.row_bytes,
+                                kv_row_stride=wl.row_stride, k_off=wl.k_off, v_off=wl.v_off, kept_capacity=cap,
+                                tau=wl.tau, scale=wl.scale))
+    tau = wl.tau
+    steps_in = [wl.step_inputs(t) for t in range(tau)]
+    q_d = [synth.raw_to_torch(s[0]) for s in steps_in]
+    w_d = [torch.from_numpy(np.ascontiguousarray(s[1])).cuda() for s in steps_in]
+    Q_d = [synth.raw_to_torch(s[2]) for s in steps_in]
+    odt = torch.int16 if wl.attn_dtype == "bf16" else torch.float32
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=odt, device="cuda")
+    lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def window(w):
+        ctx = ctxs[w % REPLICAS]
+        for t in range(tau):
+            ctx.step(t, q_d[t], w_d[t], Q_d[t], out, lse)
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    def max_over_ranks(x):
+        if pg is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up
+    for w in range(args.warmup):
+        window(w)
+    torch.cuda.synchronize()
+    for c in ctxs:
+        c.reset_counters()
+        c.set_timing(True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for w in range(args.steps):
+        window(args.warmup + w)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
+    launches = sum(c.launches() for c in ctxs)
+    stage = {}
+    for c in ctxs:
+        for k, (ms, calls) in c.stage_times().items():
+            a = stage.setdefault(k, [0.0, 0])
+            a[0] += ms
+            a[1] += calls
+        c.set_timing(False)
+    errs = [int(lsa.device_view(c.view().err, 1, torch.int32).item()) for c in ctxs]
+    ms_window = ms_total / args.steps
+    value = ws * tau * args.steps / (ms_total / 1e3)
+
+    # roofline of the index scan
+    peak, peak_src = measured_peaks()
+    scan_ms = stage["score"][0] / max(stage["score"][1], 1)
+    scan_bytes = algorithmic_scan_bytes(wl)
+    achieved = scan_bytes / (scan_ms / 1e3) / 1e9
+    traffic = scan_traffic_record()
+    gather_ms = stage["gather"][0] / max(stage["gather"][1], 1)
+    kept_total = int(lsa.device_view(ctxs[0].view().kept_off, wl.B + 1, torch.int64)[-1].item())
+    gather_bytes = min(kept_total, cap) * wl.row_bytes
+
+    # pinned host -> device peak of this machine (copy engine, 256 MB)
+    hsrc = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    ddst = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        ddst.copy_(hsrc, non_blocking=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(5):
+        ddst.copy_(hsrc, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    h2d_gbs = 5 * (256 << 20) / (e0.elapsed_time(e1) / 1e3) / 1e9
+    del hsrc, ddst
+
+    # end to end through the host-buffer entry point
+    q_h = [synth.raw_to_torch(s[0], "cpu").pin_memory() for s in steps_in]
+    w_h = [torch.from_numpy(np.ascontiguousarray(s[1])).pin_memory() for s in steps_in]
+    Q_h = [synth.raw_to_torch(s[2], "cpu").pin_memory() for s in steps_in]
+    out_h = torch.empty((wl.B, wl.Hq, wl.D), dtype=odt).pin_memory()
+    lse_h = torch.empty((wl.B, wl.Hq), dtype=torch.float32).pin_memory()
+
+    def window_host(w):
+        ctx = ctxs[w % REPLICAS]
+        for t in range(tau):
+            ctx.step_host(t, q_h[t], w_h[t], Q_h[t], out_h, lse_h)
+
+    for w in range(args.warmup):
+        window_host(w)
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for w in range(args.steps):
+        window_host(args.warmup + w)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    h2d = tau * (q_h[0].numel() * q_h[0].element_size() + w_h[0].numel() * 4 + Q_h[0].numel() * Q_h[0].element_size())
+    d2h = tau * (out_h.numel() * out_h.element_size() + lse_h.numel() * 4)
+
+    cpu_base = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        v, info = oracle_window_sample(wl)
+        cpu_base = {"value": v, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
+                    "sample": "1 refresh + 1 listed decode step of this workload (all 4 sequences) on the host "
+                              "cores, extrapolated to a tau=64 window: t_refresh=%.2fs t_listed=%.2fs"
+                              % (info["t_refresh_s"], info["t_listed_s"])}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_window, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32 accumulate (e4m3 keys, bf16 KV)", "data": "synthetic",
+            "config": {"workload": WORKLOAD_DESC[args.config], "tau": tau,
+                       "bench_step": "one tau window = 1 refresh + 63 listed decode steps",
+                       "decode_steps_per_bench_step": tau, "global_batch": wl.B * ws,
+                       "l2": "3 replicas of the indexer keys rotated per window (3 x %.0f MB > 126 MB L2)"
+                             % (scan_bytes / 1e6),
+                       "parallelism": f"independent batch per GPU x{ws}", "kept_capacity": cap},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "kernel": "lsa_index_score full scan",
+                         "algorithmic_bytes": scan_bytes, "avg_launch_ms": scan_ms, "peak_source": peak_src},
+            "cpu_baseline": cpu_base,
+            "e2e": {"value": ws * tau * args.steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "stages_ms_avg": {k: (v[0] / v[1] if v[1] else None) for k, v in stage.items()},
+            "host_link": {"gather_GBps": gather_bytes / (gather_ms / 1e3) / 1e9 if gather_ms else None,
+                          "gather_bytes": gather_bytes, "pinned_h2d_copy_GBps": h2d_gbs,
+                          "kept_entries": kept_total},
+            "device_errors": errs,
+        }
+        print(json.dumps(line), flush=True)
+    for c in ctxs:
+        c.close()
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_cuda(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

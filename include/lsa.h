@@ -1,0 +1,275 @@
+/*
+ * lsa.h -- C ABI of the Lookahead Sparse Attention (LSA) decode hot path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method ("FlashMemory-DeepSeek-V4: Lightning Index Ultra-Long Context via
+ * Lookahead Sparse Attention", gist.science technical summary, section 2.1):
+ *   - Periodic Triggering: every tau decode steps (tau = 64) the memory
+ *     indexer is evaluated on the current hidden state;
+ *   - Scoring Mechanism: a lookahead index score I_{t,s} between the current
+ *     indexer queries and every preceding compressed entry s, a head-fused
+ *     gated matching score through a sigmoid, fixed here as
+ *         I_{t,s} = sigmoid( sum_j w_{t,j} * ReLU(q_{t,j} . k_s) );
+ *   - Dynamic Fetching: every entry with I_{t,s} >= 0.5 is fetched from the
+ *     CPU cold pool into GPU memory (no rigid top-k at this stage);
+ *   - Tiered Selection: a fine-grained top-k inside that fetched subset feeds
+ *     the final core attention.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer unless its comment says host.
+ *     The caller owns every buffer; no entry point allocates or frees memory,
+ *     except lsa_ctx_create / lsa_ctx_destroy, which own the context's
+ *     internal buffers.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as
+ *     void*; NULL is the legacy default stream).  No entry point synchronises
+ *     the host, except where its comment says so.
+ *   - Argument validation happens on the host before anything is enqueued.  A
+ *     failed validation returns LSA_ERR_INVALID or LSA_ERR_UNSUPPORTED,
+ *     launches nothing and sets the message returned by lsa_last_error().
+ *   - Conditions only the device can see (kept entries beyond a buffer's
+ *     capacity, a bounded wait that gave up) are written to the caller's
+ *     device word `err` (int32, first error wins: LSA_ERR_CAPACITY or
+ *     LSA_ERR_TIMEOUT).  The caller zeroes it and reads it after the stream
+ *     has completed.  `err` may be NULL where the comment allows it.
+ *   - Ragged batches use CSR offsets: sequence b owns entries
+ *     [seq_off[b], seq_off[b+1]) of a flat entry axis of n_total entries.
+ *     Entry indices in kept and top-k lists are local to their sequence.
+ */
+#ifndef LSA_H
+#define LSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lsa_status {
+    LSA_OK = 0,
+    LSA_ERR_INVALID = 1,      /* bad argument: nothing was launched */
+    LSA_ERR_CUDA = 2,         /* a CUDA runtime call failed */
+    LSA_ERR_CAPACITY = 3,     /* more kept entries than the output can hold */
+    LSA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up */
+    LSA_ERR_UNSUPPORTED = 5   /* valid, but not a shape/dtype this library runs */
+} lsa_status;
+
+typedef enum lsa_dtype {
+    LSA_F32 = 0,   /* IEEE binary32 */
+    LSA_BF16 = 1,  /* bfloat16 */
+    LSA_E4M3 = 2   /* OCP FP8 E4M3 ("fn"): bias 7, no infinities, max 448 */
+} lsa_dtype;
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t lsa_version(void);
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char *lsa_last_error(void);
+
+/* Static name of a status code. */
+const char *lsa_status_name(lsa_status s);
+
+/* ------------------------------------------------------------------------
+ * lsa_index_score -- the lookahead index score (section 2.1, "Scoring
+ * Mechanism"; the interaction is a plain dot product, section 5).
+ *
+ *   z_s = sum_{j<H} w[b,j] * max(0, q[b,j,:] . k[s,:])     I_s = 1/(1+exp(-z_s))
+ *
+ * q        [B, H, d]   q_dtype LSA_F32 or LSA_BF16, row-major.
+ * w        [B, H]      fp32 gate weights (may be negative).
+ * k        [n_total, d] indexer keys K^{IComp}, row-major; k_dtype LSA_F32,
+ *                      LSA_BF16 or LSA_E4M3.  Rows start 16-byte aligned
+ *                      (d * element size is a multiple of 16).
+ * k_scale  [n_total]   fp32, one positive scale per row, required for E4M3
+ *                      keys (value = code * scale; rows of d <= 128), else NULL.
+ * seq_off  [B+1]       int64 CSR offsets; seq_off[B] == n_total (host value).
+ * Listed mode (idx != NULL): only entries idx[idx_off[b] .. idx_off[b+1])
+ *   of each sequence (indices local to the sequence) are scored, and z / I
+ *   are written at the list position.  idx_off [B+1] int64 on the device;
+ *   list_capacity (host) bounds idx_off[B].
+ * Full mode (idx == NULL): z / I are written for every entry, [n_total].
+ * z        fp32 output (required).   I  fp32 output or NULL.
+ * Shapes run: 1 <= H <= 64, d in {32, 64, 128} (d * element size % 16 == 0).
+ * ---------------------------------------------------------------------- */
+lsa_status lsa_index_score(const void *q, lsa_dtype q_dtype, const float *w,
+                           const void *k, lsa_dtype k_dtype, const float *k_scale,
+                           const int64_t *seq_off, int64_t n_total,
+                           const int32_t *idx, const int64_t *idx_off, int64_t list_capacity,
+                           int32_t B, int32_t H, int32_t d,
+                           float *z, float *I, void *stream);
+
+/* ------------------------------------------------------------------------
+ * lsa_select -- threshold selection (section 2.1, "Dynamic Fetching"):
+ * keep every entry with I >= 0.5.  The decision is taken as z >= 0, which
+ * is the same set in exact arithmetic (sigmoid is increasing, sigmoid(0) =
+ * 1/2) and cannot be moved by rounding of the sigmoid; -0.0 is kept, NaN is
+ * not.
+ *
+ * z         [n_total] fp32 scores (full mode of lsa_index_score).
+ * kept_idx  [capacity] int32 output: kept entries of each sequence, local
+ *           indices in ascending order, sequence after sequence.
+ * kept_off  [B+1] int64 output: CSR offsets into kept_idx.  kept_off[B] is the
+ *           true total even when it exceeds capacity; then only the first
+ *           `capacity` indices are written and *err = LSA_ERR_CAPACITY.
+ * mask      [ceil(n_total/32)] uint32 output or NULL: bit (s % 32) of word
+ *           s / 32 is set iff entry s (flat axis) is kept.
+ * workspace device scratch of at least lsa_select_workspace_size(n_total)
+ *           bytes, 16-byte aligned; contents need not be initialised.
+ * ---------------------------------------------------------------------- */
+size_t lsa_select_workspace_size(int64_t n_total);
+lsa_status lsa_select(const float *z, const int64_t *seq_off, int64_t n_total, int32_t B,
+                      int32_t *kept_idx, int64_t capacity, int64_t *kept_off, uint32_t *mask,
+                      void *workspace, size_t ws_bytes, int32_t *err, void *stream);
+
+/* ------------------------------------------------------------------------
+ * lsa_topk -- fine-grained top-k inside the kept set (section 2.1, "Tiered
+ * Selection").  Per sequence, the k kept entries with the largest z (the
+ * sigmoid is monotone, so ranking by z ranks by I); equal z goes to the lower
+ * entry index (-0.0 and +0.0 are equal).  The chosen set is written in
+ * ascending entry order; if a sequence keeps fewer than k entries, all of
+ * them are written and the rest of its row is -1.
+ *
+ * z            scores.  z_by_entry != 0: z is indexed on the flat entry axis,
+ *              z[seq_off[b] + kept_idx[p]] (scores of a full scan; seq_off
+ *              required).  z_by_entry == 0: z[p] is the score of kept
+ *              position p (a listed scan over the kept set).
+ * kept_idx, kept_off  the kept set, as produced by lsa_select.
+ * kept_capacity  number of valid kept_idx entries (the capacity given to
+ *              lsa_select); kept positions at or past it are ignored.
+ * topk_idx     [B, k] int32 output: local entry indices, ascending, -1 padded.
+ * topk_pos     [B, k] int32 output or NULL: the kept-list position p of each
+ *              chosen entry (= its hot-buffer row after lsa_gather), -1 padded.
+ * topk_cnt     [B] int32 output: min(k, kept count).
+ * Shapes run: 1 <= k <= 4096.  A sequence may keep any number of entries.
+ * ---------------------------------------------------------------------- */
+lsa_status lsa_topk(const float *z, int32_t z_by_entry, const int64_t *seq_off,
+                    const int32_t *kept_idx, const int64_t *kept_off, int64_t kept_capacity,
+                    int32_t B, int32_t k, int32_t *topk_idx, int32_t *topk_pos,
+                    int32_t *topk_cnt, void *stream);
+
+/* ------------------------------------------------------------------------
+ * lsa_gather -- cold-pool fetch (section 2.1, "Dynamic Fetching": kept
+ * entries are fetched from the CPU "Cold Pool" into GPU memory; blog page:
+ * "just in time").  Copies the cold row of every kept entry into the HBM hot
+ * buffer, in kept order: hot row kept_off[b] + i receives cold row
+ * seq_off[b] + kept_idx[kept_off[b] + i].
+ *
+ * cold_host   HOST pointer to the cold pool [n_total, row_bytes], page-locked
+ *             (cudaHostAlloc / cudaHostRegister, or torch pin_memory) so the
+ *             device can read it; it is read directly over the host link.
+ * row_bytes   bytes per row, a positive multiple of 16.
+ * hot         [hot_capacity, row_bytes] device output.  Rows past
+ *             hot_capacity are not written and *err = LSA_ERR_CAPACITY.
+ * slot_of     [n_total] int32 output or NULL: hot row of each entry, -1 for
+ *             entries not kept.
+ * ---------------------------------------------------------------------- */
+lsa_status lsa_gather(const void *cold_host, int64_t row_bytes, const int64_t *seq_off,
+                      int64_t n_total, const int32_t *kept_idx, const int64_t *kept_off, int32_t B,
+                      void *hot, int64_t hot_capacity, int32_t *slot_of, int32_t *err,
+                      void *stream);
+
+/* ------------------------------------------------------------------------
+ * lsa_sparse_attn -- core attention over the selected entries (section 2.1,
+ * "Tiered Selection": the top-k feeds "the final core attention
+ * computation").  Multi-query attention: all Hq query heads of a sequence
+ * attend over the same selected K/V rows.
+ *
+ *   a_i = scale * Q[b,h,:] . K_i     o[b,h,:] = sum_i softmax(a)_i V_i
+ *   lse[b,h] = log sum_i exp(a_i)     (no row selected: o = 0, lse = -inf)
+ *
+ * Q      [B, Hq, D] dtype LSA_F32 or LSA_BF16.   out  [B, Hq, D] same dtype.
+ * kv     rows of the hot buffer, same dtype; row r holds K at element
+ *        r * kv_row_stride + k_off and V at r * kv_row_stride + v_off (they
+ *        may alias: k_off == v_off for a latent head serving as K and V).
+ * rows   [B, k] int32 row indices into kv; negative entries are padding.
+ * lse    [B, Hq] fp32 output or NULL.
+ * workspace  at least lsa_sparse_attn_workspace_size(B, Hq, D, k) bytes.
+ * Shapes run: D % 32 == 0, D <= 512, 1 <= Hq <= 256, 1 <= k <= 4096.
+ * ---------------------------------------------------------------------- */
+size_t lsa_sparse_attn_workspace_size(int32_t B, int32_t Hq, int32_t D, int32_t k);
+lsa_status lsa_sparse_attn(const void *Q, lsa_dtype dtype, const void *kv, int64_t kv_row_stride,
+                           int64_t k_off, int64_t v_off, const int32_t *rows, int32_t B,
+                           int32_t Hq, int32_t D, int32_t k, float scale, void *out, float *lse,
+                           void *workspace, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Decode context and lsa_decode_step -- the tau cadence (section 2.1,
+ * "Periodic Triggering", tau = 64).
+ *
+ * At a refresh step (t % tau == 0): full index scan, selection, cold-pool
+ * fetch of the kept rows (on the context's side stream), top-k over the scan's
+ * scores, attention.  At every other step the kept set and hot buffer stay as
+ * they are; the kept entries are re-scored with that step's indexer query
+ * (listed scan), then top-k and attention.
+ * ---------------------------------------------------------------------- */
+typedef struct lsa_params {
+    int32_t B, H, d;             /* batch, indexer heads, indexer dim */
+    lsa_dtype q_dtype, k_dtype;  /* indexer query / key element types */
+    int32_t Hq, D;               /* attention query heads, head dim */
+    lsa_dtype attn_dtype;        /* Q, K/V rows and output element type */
+    int32_t topk;                /* k of the fine-grained top-k */
+    int32_t tau;                 /* refresh period; 0 means 64 */
+    float scale;                 /* softmax scale; 0 means 1/sqrt(D) */
+    int64_t n_total;             /* entries on the flat axis */
+    const int64_t *seq_off_host; /* HOST [B+1]; copied at creation */
+    const void *k_dev;           /* indexer keys [n_total, d] in HBM (caller-owned) */
+    const float *k_scale_dev;    /* [n_total] for E4M3 keys, else NULL */
+    const void *cold_host;       /* HOST page-locked cold pool [n_total, row_bytes] */
+    int64_t row_bytes;           /* bytes per cold row */
+    int64_t kv_row_stride;       /* elements per row (row_bytes / element size) */
+    int64_t k_off, v_off;        /* element offsets of K and V inside a row */
+    int64_t kept_capacity;       /* hot-buffer rows = max kept entries over the batch */
+} lsa_params;
+
+typedef struct lsa_ctx lsa_ctx;
+
+/* Allocates the context's device buffers (hot buffer, scores, kept list,
+ * top-k, workspaces, host staging) and its side stream.  Synchronous. */
+lsa_status lsa_ctx_create(const lsa_params *p, lsa_ctx **out);
+/* Synchronises the context's streams and frees everything it allocated. */
+lsa_status lsa_ctx_destroy(lsa_ctx *ctx);
+
+/* One decode step t >= 0 on device buffers: q [B,H,d], w [B,H], Q [B,Hq,D]
+ * in; out [B,Hq,D] and lse [B,Hq] (lse may be NULL) out. */
+lsa_status lsa_decode_step(lsa_ctx *ctx, int64_t t, const void *q, const float *w, const void *Q,
+                           void *out, float *lse, void *stream);
+
+/* The same step on HOST buffers (page-locked for asynchronous copies): the
+ * inputs are copied host->device, the step runs, out and lse are copied
+ * device->host, all on `stream`.  The host buffers must stay valid until the
+ * stream has completed. */
+lsa_status lsa_decode_step_host(lsa_ctx *ctx, int64_t t, const void *q_host, const float *w_host,
+                                const void *Q_host, void *out_host, float *lse_host, void *stream);
+
+/* Device pointers of the context's internal results, for inspection. */
+typedef struct lsa_ctx_view {
+    float *z;            /* [n_total] full-scan scores of the last refresh */
+    float *z_kept;       /* [kept_capacity] listed-scan scores of the last step */
+    int32_t *kept_idx;   /* [kept_capacity] */
+    int64_t *kept_off;   /* [B+1] */
+    int32_t *slot_of;    /* [n_total] */
+    void *hot;           /* [kept_capacity, row_bytes] */
+    int32_t *topk_idx;   /* [B, topk] */
+    int32_t *topk_pos;   /* [B, topk] */
+    int32_t *topk_cnt;   /* [B] */
+    int32_t *err;        /* device error word of the context */
+} lsa_ctx_view;
+lsa_status lsa_ctx_get_view(lsa_ctx *ctx, lsa_ctx_view *view);
+
+/* Stage timing.  When enabled, CUDA events bracket every stage on the stream
+ * it runs on; lsa_ctx_stage_times synchronises on them and returns the
+ * accumulated milliseconds and call counts per stage since the last reset
+ * (arrays of LSA_STAGE_COUNT).  lsa_ctx_launches returns the number of
+ * kernels the context has launched since the last reset. */
+enum { LSA_STAGE_SCORE = 0, LSA_STAGE_SELECT, LSA_STAGE_GATHER, LSA_STAGE_TOPK,
+       LSA_STAGE_ATTN, LSA_STAGE_RESCORE, LSA_STAGE_COUNT };
+lsa_status lsa_ctx_set_timing(lsa_ctx *ctx, int32_t enable);
+lsa_status lsa_ctx_stage_times(lsa_ctx *ctx, double *ms, int64_t *calls);
+lsa_status lsa_ctx_reset_counters(lsa_ctx *ctx);
+int64_t lsa_ctx_launches(lsa_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H */

@@ -1,0 +1,214 @@
+// Core attention over the selected entries ("FlashMemory-DeepSeek-V4 ...
+// Lookahead Sparse Attention", gist.science technical summary, section 2.1
+// "Tiered Selection": the top-k inside the fetched subset feeds the final core
+// attention).  Multi-query decode: every query head of a sequence attends
+// over the same selected K/V rows.
+//
+// Split-K over the selected rows: each block takes one sequence, one chunk of
+// kChunk selected rows and a group of kHeads query heads, stages the chunk's
+// K/V rows and the group's queries in shared memory, and writes a partial
+// (row max m, exp-sum l, unnormalised output o) per head.  A combine kernel
+// merges the chunks:  M = max m_c,  L = sum l_c e^{m_c - M},
+// o = sum o_c e^{m_c - M} / L,  lse = M + log L.
+//
+// This is the CUDA-core path (fp32 FMA), used for every supported shape and
+// both dtypes.
+#include "lsa_internal.cuh"
+
+namespace lsa {
+namespace {
+
+constexpr int kChunk = 64;          // selected rows per block
+constexpr int kHeads = 16;          // query heads per block
+constexpr int kAttnThreads = 256;   // 8 warps, 2 heads each
+constexpr int kMaxColsPerLane = 16; // D <= 512
+
+template <typename T>
+struct Elem;
+template <>
+struct Elem<float> {
+    static constexpr int kPad = 1;   // row stride D+1 words: conflict-free row-wise reads
+    __device__ static float get(const float *p, int i) { return p[i]; }
+    __device__ static float2 get2(const float *p, int i) { return make_float2(p[i], p[i + 1]); }
+    __device__ static void put(float *p, int64_t i, float v) { p[i] = v; }
+};
+template <>
+struct Elem<uint16_t> {
+    static constexpr int kPad = 2;   // row stride D+2 halves = odd number of words
+    __device__ static float get(const uint16_t *p, int i) { return bf16_to_f32(p[i]); }
+    __device__ static float2 get2(const uint16_t *p, int i) {
+        const uint32_t u = *reinterpret_cast<const uint32_t *>(p + i);
+        return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+    }
+    __device__ static void put(uint16_t *p, int64_t i, float v) {
+        __nv_bfloat16 h = __float2bfloat16_rn(v);
+        p[i] = *reinterpret_cast<uint16_t *>(&h);
+    }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kAttnThreads)
+attn_partial(const T *__restrict__ Q, const T *__restrict__ kv, int64_t stride, int64_t k_off,
+             int64_t v_off, const int32_t *__restrict__ rows, int Hq, int D, int k, float scale,
+             float *__restrict__ part) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int ld = D + Elem<T>::kPad;
+    const bool alias = k_off == v_off;
+    T *Ks = reinterpret_cast<T *>(smem_raw);
+    T *Vs = alias ? Ks : Ks + kChunk * ld;
+    float *Qs = reinterpret_cast<float *>(
+        smem_raw + align_up(size_t(kChunk) * ld * sizeof(T) * (alias ? 1 : 2), 16));
+    float *Ps = Qs + kHeads * D;
+    __shared__ int s_rows[kChunk];
+
+    const int chunk = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+    const int nchunks = gridDim.x;
+    const int h0 = hg * kHeads;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    if (threadIdx.x < kChunk) {
+        const int i = chunk * kChunk + threadIdx.x;
+        s_rows[threadIdx.x] = i < k ? rows[int64_t(b) * k + i] : -1;
+    }
+    __syncthreads();
+    // stage K (and V) rows: element-wise copy, zero for padding rows
+    for (int t = threadIdx.x; t < kChunk * D; t += kAttnThreads) {
+        const int i = t / D, c = t - i * D;
+        const int r = s_rows[i];
+        T kvv{}, vvv{};
+        if (r >= 0) {
+            kvv = kv[int64_t(r) * stride + k_off + c];
+            if (!alias) vvv = kv[int64_t(r) * stride + v_off + c];
+        }
+        Ks[i * ld + c] = kvv;
+        if (!alias) Vs[i * ld + c] = vvv;
+    }
+    for (int t = threadIdx.x; t < kHeads * D; t += kAttnThreads) {
+        const int hh = t / D, c = t - hh * D;
+        const int h = h0 + hh;
+        Qs[t] = h < Hq ? Elem<T>::get(Q, int((int64_t(b) * Hq + h) * D + c)) : 0.f;
+    }
+    __syncthreads();
+
+    const int ncols = D / 32;
+    for (int hh = warp; hh < kHeads; hh += kAttnThreads / 32) {
+        const int h = h0 + hh;
+        if (h >= Hq) break;
+        const float *qh = Qs + hh * D;
+        // logits for rows lane and lane + 32
+        float s0 = 0.f, s1 = 0.f;
+        for (int c = 0; c < D; c += 2) {
+            const float2 q2 = make_float2(qh[c], qh[c + 1]);
+            const float2 ka = Elem<T>::get2(Ks + lane * ld, c);
+            const float2 kb = Elem<T>::get2(Ks + (lane + 32) * ld, c);
+            s0 = fmaf(q2.x, ka.x, fmaf(q2.y, ka.y, s0));
+            s1 = fmaf(q2.x, kb.x, fmaf(q2.y, kb.y, s1));
+        }
+        const bool v0 = s_rows[lane] >= 0, v1 = s_rows[lane + 32] >= 0;
+        s0 = v0 ? s0 * scale : -INFINITY;
+        s1 = v1 ? s1 * scale : -INFINITY;
+        float m = fmaxf(s0, s1);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float p0 = v0 ? expf(s0 - m) : 0.f;
+        const float p1 = v1 ? expf(s1 - m) : 0.f;
+        float l = p0 + p1;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        float *ph = Ps + hh * kChunk;
+        ph[lane] = p0;
+        ph[lane + 32] = p1;
+        __syncwarp();
+        float acc[kMaxColsPerLane];
+#pragma unroll
+        for (int j = 0; j < kMaxColsPerLane; ++j) acc[j] = 0.f;
+        if (m != -INFINITY) {
+            for (int i = 0; i < kChunk; ++i) {
+                const float p = ph[i];
+                const T *vr = Vs + i * ld;
+#pragma unroll
+                for (int j = 0; j < kMaxColsPerLane; ++j)
+                    if (j < ncols) acc[j] = fmaf(p, Elem<T>::get(vr, lane + 32 * j), acc[j]);
+            }
+        }
+        float *dst = part + ((int64_t(b) * nchunks + chunk) * Hq + h) * (D + 2);
+#pragma unroll
+        for (int j = 0; j < kMaxColsPerLane; ++j)
+            if (j < ncols) dst[lane + 32 * j] = acc[j];
+        if (lane == 0) {
+            dst[D] = m;
+            dst[D + 1] = l;
+        }
+        __syncwarp();
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128)
+attn_combine(const float *__restrict__ part, int nchunks, int Hq, int D, T *__restrict__ out,
+             float *__restrict__ lse) {
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int64_t stride_c = int64_t(Hq) * (D + 2);
+    const float *base = part + (int64_t(b) * nchunks * Hq + h) * (D + 2);
+    float M = -INFINITY;
+    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, base[c * stride_c + D]);
+    float L = 0.f;
+    if (M != -INFINITY)
+        for (int c = 0; c < nchunks; ++c) {
+            const float m = base[c * stride_c + D];
+            if (m != -INFINITY) L += base[c * stride_c + D + 1] * expf(m - M);
+        }
+    const int64_t ob = (int64_t(b) * Hq + h) * D;
+    for (int col = threadIdx.x; col < D; col += blockDim.x) {
+        float o = 0.f;
+        if (M != -INFINITY) {
+            for (int c = 0; c < nchunks; ++c) {
+                const float m = base[c * stride_c + D];
+                if (m != -INFINITY) o = fmaf(base[c * stride_c + col], expf(m - M), o);
+            }
+            o /= L;
+        }
+        Elem<T>::put(out, ob + col, o);
+    }
+    if (threadIdx.x == 0 && lse) lse[int64_t(b) * Hq + h] = M == -INFINITY ? -INFINITY : M + logf(L);
+}
+
+template <typename T>
+lsa_status launch_t(const void *Q, const void *kv, int64_t stride, int64_t k_off, int64_t v_off,
+                    const int32_t *rows, int B, int Hq, int D, int k, float scale, void *out,
+                    float *lse, void *workspace, cudaStream_t st) {
+    const int nchunks = (k + kChunk - 1) / kChunk;
+    const int ld = D + Elem<T>::kPad;
+    const bool alias = k_off == v_off;
+    const size_t smem = align_up(size_t(kChunk) * ld * sizeof(T) * (alias ? 1 : 2), 16) +
+                        size_t(kHeads) * D * 4 + size_t(kHeads) * kChunk * 4;
+    auto kern = attn_partial<T>;
+    LSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    dim3 grid(nchunks, (Hq + kHeads - 1) / kHeads, B);
+    kern<<<grid, kAttnThreads, smem, st>>>(static_cast<const T *>(Q), static_cast<const T *>(kv), stride,
+                                           k_off, v_off, rows, Hq, D, k, scale,
+                                           static_cast<float *>(workspace));
+    LSA_LAUNCHED("attn_partial");
+    attn_combine<T><<<dim3(Hq, B), 128, 0, st>>>(static_cast<const float *>(workspace), nchunks, Hq, D,
+                                                 static_cast<T *>(out), lse);
+    LSA_LAUNCHED("attn_combine");
+    return LSA_OK;
+}
+
+}  // namespace
+
+size_t sparse_attn_workspace(int32_t B, int32_t Hq, int32_t D, int32_t k) {
+    const int nchunks = (k + kChunk - 1) / kChunk;
+    return size_t(B) * nchunks * Hq * (D + 2) * sizeof(float);
+}
+
+lsa_status launch_sparse_attn(const void *Q, lsa_dtype dtype, const void *kv, int64_t stride,
+                              int64_t k_off, int64_t v_off, const int32_t *rows, int32_t B,
+                              int32_t Hq, int32_t D, int32_t k, float scale, void *out, float *lse,
+                              void *workspace, cudaStream_t st) {
+    if (dtype == LSA_F32)
+        return launch_t<float>(Q, kv, stride, k_off, v_off, rows, B, Hq, D, k, scale, out, lse, workspace, st);
+    return launch_t<uint16_t>(Q, kv, stride, k_off, v_off, rows, B, Hq, D, k, scale, out, lse, workspace, st);
+}
+
+}  // namespace lsa

@@ -1,0 +1,356 @@
+// Decode context and the tau cadence ("FlashMemory-DeepSeek-V4 ...
+// Lookahead Sparse Attention", gist.science technical summary, section 2.1:
+// Periodic Triggering every tau = 64 steps; Scoring Mechanism; Dynamic
+// Fetching of every entry with I >= 0.5 from the CPU cold pool; Tiered
+// Selection of a fine-grained top-k inside the fetched subset for the core
+// attention).
+//
+// Refresh step (t % tau == 0):  score (full scan) -> select -> [side stream:
+// gather kept rows cold pool -> HBM] -> top-k over the scan's scores ->
+// wait for the gather -> attention over the hot buffer.
+// Other steps: listed re-score of the kept set with the step's indexer query
+// -> top-k -> attention.  The host never waits inside a step.
+#include <cmath>
+#include <vector>
+
+#include "lsa_internal.cuh"
+
+struct lsa_ctx {
+    lsa_params p{};
+    std::vector<int64_t> seq_off_h;
+    int device = 0;
+    int tau = 64;
+    float scale = 1.f;
+    const void *cold_dev = nullptr;
+    int64_t *seq_off_d = nullptr;
+    float *z = nullptr;
+    float *z_kept = nullptr;
+    int32_t *kept_idx = nullptr;
+    int64_t *kept_off = nullptr;
+    int32_t *slot_of = nullptr;
+    void *hot = nullptr;
+    int32_t *topk_idx = nullptr, *topk_pos = nullptr, *topk_cnt = nullptr;
+    int32_t *err = nullptr;
+    void *sel_ws = nullptr;
+    size_t sel_ws_bytes = 0;
+    void *attn_ws = nullptr;
+    size_t attn_ws_bytes = 0;
+    // staging for lsa_decode_step_host
+    void *q_d = nullptr, *Q_d = nullptr, *out_d = nullptr;
+    float *w_d = nullptr, *lse_d = nullptr;
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_sel = nullptr, ev_gather = nullptr;
+    bool refreshed = false;
+    // timing
+    bool timing = false;
+    struct Pending { int stage; cudaEvent_t a, b; };
+    std::vector<Pending> pending;
+    std::vector<cudaEvent_t> free_events;
+    double ms[LSA_STAGE_COUNT] = {0};
+    int64_t calls[LSA_STAGE_COUNT] = {0};
+    int64_t launches = 0;
+};
+
+namespace {
+
+using namespace lsa;
+
+void free_all(lsa_ctx *c) {
+    void *bufs[] = {c->seq_off_d, c->z, c->z_kept, c->kept_idx, c->kept_off, c->slot_of, c->hot,
+                    c->topk_idx, c->topk_pos, c->topk_cnt, c->err, c->sel_ws, c->attn_ws,
+                    c->q_d, c->Q_d, c->out_d, c->w_d, c->lse_d};
+    for (void *b : bufs)
+        if (b) cudaFree(b);
+    if (c->ev_sel) cudaEventDestroy(c->ev_sel);
+    if (c->ev_gather) cudaEventDestroy(c->ev_gather);
+    for (auto &pe : c->pending) { cudaEventDestroy(pe.a); cudaEventDestroy(pe.b); }
+    for (auto e : c->free_events) cudaEventDestroy(e);
+    if (c->side) cudaStreamDestroy(c->side);
+}
+
+cudaEvent_t take_event(lsa_ctx *c) {
+    if (!c->free_events.empty()) {
+        cudaEvent_t e = c->free_events.back();
+        c->free_events.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Brackets one stage with events when timing is on.
+struct StageTimer {
+    lsa_ctx *c;
+    int stage;
+    cudaStream_t st;
+    cudaEvent_t a = nullptr;
+    StageTimer(lsa_ctx *c_, int stage_, cudaStream_t st_) : c(c_), stage(stage_), st(st_) {
+        if (c->timing) {
+            a = take_event(c);
+            cudaEventRecord(a, st);
+        }
+    }
+    void done() {
+        if (a) {
+            cudaEvent_t b = take_event(c);
+            cudaEventRecord(b, st);
+            c->pending.push_back({stage, a, b});
+            a = nullptr;
+        }
+    }
+};
+
+#define LSA_TRY(call)                       \
+    do {                                    \
+        lsa_status s_ = (call);             \
+        if (s_ != LSA_OK) return s_;        \
+    } while (0)
+
+template <typename T>
+lsa_status alloc(T **p, size_t bytes) {
+    *p = nullptr;
+    if (bytes == 0) bytes = 16;
+    LSA_CUDA(cudaMalloc(reinterpret_cast<void **>(p), bytes));
+    return LSA_OK;
+}
+
+lsa_status run_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const void *Q, void *out,
+                    float *lse, cudaStream_t st) {
+    const lsa_params &p = c->p;
+    const int64_t launches0 = launch_count();
+    const bool refresh = (t % c->tau) == 0 || !c->refreshed;
+    const int64_t cap = p.kept_capacity;
+    if (refresh) {
+        StageTimer ts(c, LSA_STAGE_SCORE, st);
+        LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
+                                   p.n_total, nullptr, nullptr, 0, p.B, p.H, p.d, c->z, nullptr, st));
+        ts.done();
+        StageTimer tsel(c, LSA_STAGE_SELECT, st);
+        LSA_TRY(launch_select(c->z, c->seq_off_d, p.n_total, p.B, c->kept_idx, cap, c->kept_off,
+                              nullptr, c->sel_ws, c->err, st));
+        tsel.done();
+        LSA_CUDA(cudaEventRecord(c->ev_sel, st));
+        LSA_CUDA(cudaStreamWaitEvent(c->side, c->ev_sel, 0));
+        StageTimer tg(c, LSA_STAGE_GATHER, c->side);
+        LSA_TRY(launch_gather(c->cold_dev, p.row_bytes, c->seq_off_d, p.n_total, c->kept_idx,
+                              c->kept_off, p.B, c->hot, cap, c->slot_of, c->err, c->side));
+        tg.done();
+        LSA_CUDA(cudaEventRecord(c->ev_gather, c->side));
+        StageTimer tk(c, LSA_STAGE_TOPK, st);
+        LSA_TRY(launch_topk(c->z, 1, c->seq_off_d, c->kept_idx, c->kept_off, p.B, p.topk, cap,
+                            c->topk_idx, c->topk_pos, c->topk_cnt, st));
+        tk.done();
+        LSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
+        c->refreshed = true;
+    } else {
+        StageTimer tr(c, LSA_STAGE_RESCORE, st);
+        LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
+                                   p.n_total, c->kept_idx, c->kept_off, cap, p.B, p.H, p.d, c->z_kept,
+                                   nullptr, st));
+        tr.done();
+        StageTimer tk(c, LSA_STAGE_TOPK, st);
+        LSA_TRY(launch_topk(c->z_kept, 0, c->seq_off_d, c->kept_idx, c->kept_off, p.B, p.topk, cap,
+                            c->topk_idx, c->topk_pos, c->topk_cnt, st));
+        tk.done();
+    }
+    StageTimer ta(c, LSA_STAGE_ATTN, st);
+    LSA_TRY(launch_sparse_attn(Q, p.attn_dtype, c->hot, p.kv_row_stride, p.k_off, p.v_off, c->topk_pos,
+                               p.B, p.Hq, p.D, p.topk, c->scale, out, lse, c->attn_ws, st));
+    ta.done();
+    c->launches += launch_count() - launches0;
+    return LSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
+    clear_error();
+    LSA_CHECK_ARG(pp && out, "lsa_ctx_create: params and out are required");
+    *out = nullptr;
+    const lsa_params &p = *pp;
+    LSA_CHECK_ARG(p.B >= 1 && p.H >= 1 && p.d >= 1 && p.Hq >= 1 && p.D >= 1 && p.topk >= 1,
+                  "lsa_ctx_create: sizes must be positive");
+    LSA_CHECK_ARG(p.n_total >= 0 && p.n_total < (int64_t(1) << 31), "lsa_ctx_create: n_total out of range");
+    LSA_CHECK_ARG(p.seq_off_host && p.k_dev && p.cold_host, "lsa_ctx_create: seq_off_host, k_dev, cold_host required");
+    LSA_CHECK_ARG(p.tau >= 0, "lsa_ctx_create: tau < 0");
+    LSA_CHECK_ARG(p.kept_capacity >= 1, "lsa_ctx_create: kept_capacity must be >= 1");
+    LSA_CHECK_ARG(p.row_bytes > 0 && p.row_bytes % 16 == 0, "lsa_ctx_create: row_bytes must be a multiple of 16");
+    LSA_CHECK_ARG(p.kv_row_stride * int64_t(elem_size(p.attn_dtype)) == p.row_bytes,
+                  "lsa_ctx_create: kv_row_stride * element size must equal row_bytes");
+    LSA_CHECK_SUPPORTED(p.attn_dtype == LSA_F32 || p.attn_dtype == LSA_BF16, "lsa_ctx_create: attn dtype");
+    LSA_CHECK_SUPPORTED(p.q_dtype == LSA_F32 || p.q_dtype == LSA_BF16, "lsa_ctx_create: q dtype");
+    LSA_CHECK_ARG(valid_dtype(p.k_dtype) && ((p.k_dtype == LSA_E4M3) == (p.k_scale_dev != nullptr)),
+                  "lsa_ctx_create: k_scale_dev is required for E4M3 keys and only for them");
+    LSA_CHECK_SUPPORTED(p.H <= 64 && (p.d == 32 || p.d == 64 || p.d == 128), "lsa_ctx_create: H/d");
+    LSA_CHECK_SUPPORTED(p.D % 32 == 0 && p.D <= 512 && p.Hq <= 256 && p.topk <= 4096, "lsa_ctx_create: Hq/D/topk");
+    LSA_CHECK_ARG(p.k_off >= 0 && p.v_off >= 0 && p.k_off + p.D <= p.kv_row_stride && p.v_off + p.D <= p.kv_row_stride,
+                  "lsa_ctx_create: K/V must lie inside a row");
+    const int64_t *so = p.seq_off_host;
+    LSA_CHECK_ARG(so[0] == 0 && so[p.B] == p.n_total, "lsa_ctx_create: seq_off must run from 0 to n_total");
+    for (int b = 0; b < p.B; ++b)
+        LSA_CHECK_ARG(so[b + 1] >= so[b], "lsa_ctx_create: seq_off must be non-decreasing");
+
+    cudaPointerAttributes attr;
+    cudaError_t e = cudaPointerGetAttributes(&attr, p.cold_host);
+    if (e != cudaSuccess) cudaGetLastError();
+    LSA_CHECK_ARG(e == cudaSuccess && attr.type == cudaMemoryTypeHost && attr.devicePointer,
+                  "lsa_ctx_create: cold_host is not page-locked host memory mapped for the device");
+
+    lsa_ctx *c = new lsa_ctx();
+    c->p = p;
+    c->seq_off_h.assign(so, so + p.B + 1);
+    c->p.seq_off_host = c->seq_off_h.data();
+    c->tau = p.tau ? p.tau : 64;
+    c->scale = p.scale > 0.f ? p.scale : 1.f / std::sqrt(float(p.D));
+    c->cold_dev = attr.devicePointer;
+    cudaGetDevice(&c->device);
+
+    const int64_t cap = p.kept_capacity;
+    const size_t qbytes = size_t(p.B) * p.H * p.d * elem_size(p.q_dtype);
+    const size_t Qbytes = size_t(p.B) * p.Hq * p.D * elem_size(p.attn_dtype);
+    c->sel_ws_bytes = lsa_select_workspace_size(p.n_total);
+    c->attn_ws_bytes = sparse_attn_workspace(p.B, p.Hq, p.D, p.topk);
+    lsa_status s = LSA_OK;
+#define LSA_ALLOC(ptr, bytes) \
+    if (s == LSA_OK) s = alloc(&(ptr), (bytes))
+    LSA_ALLOC(c->seq_off_d, size_t(p.B + 1) * 8);
+    LSA_ALLOC(c->z, size_t(p.n_total) * 4);
+    LSA_ALLOC(c->z_kept, size_t(cap) * 4);
+    LSA_ALLOC(c->kept_idx, size_t(cap) * 4);
+    LSA_ALLOC(c->kept_off, size_t(p.B + 1) * 8);
+    LSA_ALLOC(c->slot_of, size_t(p.n_total) * 4);
+    LSA_ALLOC(c->hot, size_t(cap) * p.row_bytes);
+    LSA_ALLOC(c->topk_idx, size_t(p.B) * p.topk * 4);
+    LSA_ALLOC(c->topk_pos, size_t(p.B) * p.topk * 4);
+    LSA_ALLOC(c->topk_cnt, size_t(p.B) * 4);
+    LSA_ALLOC(c->err, 16);
+    LSA_ALLOC(c->sel_ws, c->sel_ws_bytes);
+    LSA_ALLOC(c->attn_ws, c->attn_ws_bytes);
+    LSA_ALLOC(c->q_d, qbytes);
+    LSA_ALLOC(c->w_d, size_t(p.B) * p.H * 4);
+    LSA_ALLOC(c->Q_d, Qbytes);
+    LSA_ALLOC(c->out_d, Qbytes);
+    LSA_ALLOC(c->lse_d, size_t(p.B) * p.Hq * 4);
+#undef LSA_ALLOC
+    if (s == LSA_OK) {
+        cudaError_t ce = cudaMemcpy(c->seq_off_d, so, size_t(p.B + 1) * 8, cudaMemcpyHostToDevice);
+        if (ce == cudaSuccess) ce = cudaMemset(c->err, 0, 16);
+        if (ce == cudaSuccess) ce = cudaMemset(c->hot, 0, size_t(cap) * p.row_bytes);
+        if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking);
+        if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_sel, cudaEventDisableTiming);
+        if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_gather, cudaEventDisableTiming);
+        if (ce != cudaSuccess) {
+            set_error("lsa_ctx_create: %s", cudaGetErrorString(ce));
+            s = LSA_ERR_CUDA;
+        }
+    }
+    if (s != LSA_OK) {
+        free_all(c);
+        delete c;
+        return s;
+    }
+    *out = c;
+    return LSA_OK;
+}
+
+lsa_status lsa_ctx_destroy(lsa_ctx *c) {
+    clear_error();
+    if (!c) return LSA_OK;
+    cudaDeviceSynchronize();
+    free_all(c);
+    delete c;
+    return LSA_OK;
+}
+
+lsa_status lsa_decode_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const void *Q, void *out,
+                           float *lse, void *stream) {
+    clear_error();
+    LSA_CHECK_ARG(c && q && w && Q && out, "lsa_decode_step: ctx, q, w, Q, out required");
+    LSA_CHECK_ARG(t >= 0, "lsa_decode_step: t < 0");
+    LSA_CHECK_ARG(aligned16(Q) && aligned16(out), "lsa_decode_step: Q and out must be 16-byte aligned");
+    return run_step(c, t, q, w, Q, out, lse, as_stream(stream));
+}
+
+lsa_status lsa_decode_step_host(lsa_ctx *c, int64_t t, const void *q_host, const float *w_host,
+                                const void *Q_host, void *out_host, float *lse_host, void *stream) {
+    clear_error();
+    LSA_CHECK_ARG(c && q_host && w_host && Q_host && out_host, "lsa_decode_step_host: ctx, q, w, Q, out required");
+    LSA_CHECK_ARG(t >= 0, "lsa_decode_step_host: t < 0");
+    const lsa_params &p = c->p;
+    cudaStream_t st = as_stream(stream);
+    const size_t qbytes = size_t(p.B) * p.H * p.d * elem_size(p.q_dtype);
+    const size_t Qbytes = size_t(p.B) * p.Hq * p.D * elem_size(p.attn_dtype);
+    LSA_CUDA(cudaMemcpyAsync(c->q_d, q_host, qbytes, cudaMemcpyHostToDevice, st));
+    LSA_CUDA(cudaMemcpyAsync(c->w_d, w_host, size_t(p.B) * p.H * 4, cudaMemcpyHostToDevice, st));
+    LSA_CUDA(cudaMemcpyAsync(c->Q_d, Q_host, Qbytes, cudaMemcpyHostToDevice, st));
+    lsa_status s = run_step(c, t, c->q_d, c->w_d, c->Q_d, c->out_d, c->lse_d, st);
+    if (s != LSA_OK) return s;
+    LSA_CUDA(cudaMemcpyAsync(out_host, c->out_d, Qbytes, cudaMemcpyDeviceToHost, st));
+    if (lse_host)
+        LSA_CUDA(cudaMemcpyAsync(lse_host, c->lse_d, size_t(p.B) * p.Hq * 4, cudaMemcpyDeviceToHost, st));
+    return LSA_OK;
+}
+
+lsa_status lsa_ctx_get_view(lsa_ctx *c, lsa_ctx_view *v) {
+    clear_error();
+    LSA_CHECK_ARG(c && v, "lsa_ctx_get_view: ctx and view required");
+    v->z = c->z;
+    v->z_kept = c->z_kept;
+    v->kept_idx = c->kept_idx;
+    v->kept_off = c->kept_off;
+    v->slot_of = c->slot_of;
+    v->hot = c->hot;
+    v->topk_idx = c->topk_idx;
+    v->topk_pos = c->topk_pos;
+    v->topk_cnt = c->topk_cnt;
+    v->err = c->err;
+    return LSA_OK;
+}
+
+lsa_status lsa_ctx_set_timing(lsa_ctx *c, int32_t enable) {
+    clear_error();
+    LSA_CHECK_ARG(c, "lsa_ctx_set_timing: ctx required");
+    c->timing = enable != 0;
+    return LSA_OK;
+}
+
+lsa_status lsa_ctx_stage_times(lsa_ctx *c, double *ms, int64_t *calls) {
+    clear_error();
+    LSA_CHECK_ARG(c && ms && calls, "lsa_ctx_stage_times: ctx, ms, calls required");
+    for (auto &pe : c->pending) {
+        LSA_CUDA(cudaEventSynchronize(pe.b));
+        float dt = 0.f;
+        LSA_CUDA(cudaEventElapsedTime(&dt, pe.a, pe.b));
+        c->ms[pe.stage] += dt;
+        c->calls[pe.stage] += 1;
+        c->free_events.push_back(pe.a);
+        c->free_events.push_back(pe.b);
+    }
+    c->pending.clear();
+    for (int i = 0; i < LSA_STAGE_COUNT; ++i) {
+        ms[i] = c->ms[i];
+        calls[i] = c->calls[i];
+    }
+    return LSA_OK;
+}
+
+lsa_status lsa_ctx_reset_counters(lsa_ctx *c) {
+    clear_error();
+    LSA_CHECK_ARG(c, "lsa_ctx_reset_counters: ctx required");
+    for (auto &pe : c->pending) {
+        cudaEventSynchronize(pe.b);
+        c->free_events.push_back(pe.a);
+        c->free_events.push_back(pe.b);
+    }
+    c->pending.clear();
+    for (int i = 0; i < LSA_STAGE_COUNT; ++i) { c->ms[i] = 0; c->calls[i] = 0; }
+    c->launches = 0;
+    return LSA_OK;
+}
+
+int64_t lsa_ctx_launches(lsa_ctx *c) { return c ? c->launches : -1; }
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+// Internal helpers shared by the CUDA translation units of liblsa.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdio>
+#include <string>
+
+#include "lsa.h"
+
+namespace lsa {
+
+// ---------------------------------------------------------------- host side
+
+void set_error(const char *fmt, ...);
+void clear_error();
+
+// Validation helper: returns LSA_ERR_INVALID with a message when cond fails.
+#define LSA_CHECK_ARG(cond, ...)              \
+    do {                                      \
+        if (!(cond)) {                        \
+            ::lsa::set_error(__VA_ARGS__);    \
+            return LSA_ERR_INVALID;           \
+        }                                     \
+    } while (0)
+
+#define LSA_CHECK_SUPPORTED(cond, ...)        \
+    do {                                      \
+        if (!(cond)) {                        \
+            ::lsa::set_error(__VA_ARGS__);    \
+            return LSA_ERR_UNSUPPORTED;       \
+        }                                     \
+    } while (0)
+
+#define LSA_CUDA(call)                                                              \
+    do {                                                                            \
+        cudaError_t e_ = (call);                                                    \
+        if (e_ != cudaSuccess) {                                                    \
+            ::lsa::set_error("%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), \
+                             __FILE__, __LINE__);                                   \
+            return LSA_ERR_CUDA;                                                    \
+        }                                                                           \
+    } while (0)
+
+// After a kernel launch: report launch-configuration errors.
+#define LSA_LAUNCHED(name)                                                             \
+    do {                                                                               \
+        cudaError_t e_ = cudaGetLastError();                                           \
+        if (e_ != cudaSuccess) {                                                       \
+            ::lsa::set_error("launch of %s failed: %s", name, cudaGetErrorString(e_)); \
+            return LSA_ERR_CUDA;                                                       \
+        }                                                                              \
+        ::lsa::count_launch();                                                         \
+    } while (0)
+
+// Per-thread kernel launch counter (read by the decode context).
+void count_launch();
+int64_t launch_count();
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t elem_size(lsa_dtype t) { return t == LSA_F32 ? 4 : t == LSA_BF16 ? 2 : 1; }
+inline bool valid_dtype(int t) { return t == LSA_F32 || t == LSA_BF16 || t == LSA_E4M3; }
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Internal launchers (each validates nothing; the public entry points do).
+lsa_status launch_index_score(const void *q, lsa_dtype q_dtype, const float *w, const void *k,
+                              lsa_dtype k_dtype, const float *k_scale, const int64_t *seq_off,
+                              int64_t n_total, const int32_t *idx, const int64_t *idx_off,
+                              int64_t list_capacity, int32_t B, int32_t H, int32_t d, float *z,
+                              float *I, cudaStream_t st);
+lsa_status launch_select(const float *z, const int64_t *seq_off, int64_t n_total, int32_t B,
+                         int32_t *kept_idx, int64_t capacity, int64_t *kept_off, uint32_t *mask,
+                         void *workspace, int32_t *err, cudaStream_t st);
+lsa_status launch_topk(const float *z, int32_t z_by_entry, const int64_t *seq_off,
+                       const int32_t *kept_idx, const int64_t *kept_off, int32_t B, int32_t k,
+                       int64_t kept_cap, int32_t *topk_idx, int32_t *topk_pos, int32_t *topk_cnt,
+                       cudaStream_t st);
+lsa_status launch_gather(const void *cold_dev, int64_t row_bytes, const int64_t *seq_off,
+                         int64_t n_total, const int32_t *kept_idx, const int64_t *kept_off,
+                         int32_t B, void *hot, int64_t hot_capacity, int32_t *slot_of,
+                         int32_t *err, cudaStream_t st);
+lsa_status launch_sparse_attn(const void *Q, lsa_dtype dtype, const void *kv, int64_t stride,
+                              int64_t k_off, int64_t v_off, const int32_t *rows, int32_t B,
+                              int32_t Hq, int32_t D, int32_t k, float scale, void *out, float *lse,
+                              void *workspace, cudaStream_t st);
+size_t sparse_attn_workspace(int32_t B, int32_t Hq, int32_t D, int32_t k);
+
+// ------------------------------------------------------------- device side
+
+// First error wins.
+__device__ __forceinline__ void raise_err(int32_t *err, int32_t code) {
+    if (err) atomicCAS(err, 0, code);
+}
+
+// Index of the sequence that owns position e of a CSR axis: the largest b
+// with off[b] <= e (off is non-decreasing, off[0] = 0, e < off[B]).
+__device__ __forceinline__ int seq_of(const int64_t *off, int B, int64_t e) {
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= e) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+}  // namespace lsa

@@ -1,0 +1,239 @@
+"""Thin ctypes binding of liblsa.so (include/lsa.h).
+
+Argument marshalling only: torch tensors supply device memory and streams,
+every step of the path runs in the library's CUDA kernels.  There is no CPU
+fallback: if liblsa.so is missing or cannot be loaded, importing this module
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblsa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m lookahead_sparse_kv_index_b200.build`")
+_L = ctypes.CDLL(LIB_PATH)
+
+P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+F32, BF16, E4M3 = 0, 1, 2
+DTYPE = {"f32": F32, "bf16": BF16, "e4m3": E4M3}
+STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID", 2: "LSA_ERR_CUDA", 3: "LSA_ERR_CAPACITY", 4: "LSA_ERR_TIMEOUT",
+          5: "LSA_ERR_UNSUPPORTED"}
+(STAGE_SCORE, STAGE_SELECT, STAGE_GATHER, STAGE_TOPK, STAGE_ATTN, STAGE_RESCORE) = range(6)
+STAGES = ["score", "select", "gather", "topk", "attn", "rescore"]
+N_STAGES = 6
+
+# every symbol include/lsa.h declares
+EXPORTS = [
+    "lsa_version", "lsa_last_error", "lsa_status_name", "lsa_index_score", "lsa_select_workspace_size",
+    "lsa_select", "lsa_topk", "lsa_gather", "lsa_sparse_attn_workspace_size", "lsa_sparse_attn",
+    "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
+    "lsa_ctx_set_timing", "lsa_ctx_stage_times", "lsa_ctx_reset_counters", "lsa_ctx_launches",
+]
+
+
+class LsaError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        msg = _L.lsa_last_error().decode()
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {msg}")
+
+
+class Params(ctypes.Structure):
+    _fields_ = [
+        ("B", i32), ("H", i32), ("d", i32), ("q_dtype", i32), ("k_dtype", i32),
+        ("Hq", i32), ("D", i32), ("attn_dtype", i32), ("topk", i32), ("tau", i32), ("scale", f32),
+        ("n_total", i64), ("seq_off_host", P), ("k_dev", P), ("k_scale_dev", P), ("cold_host", P),
+        ("row_bytes", i64), ("kv_row_stride", i64), ("k_off", i64), ("v_off", i64), ("kept_capacity", i64),
+    ]
+
+
+class View(ctypes.Structure):
+    _fields_ = [("z", P), ("z_kept", P), ("kept_idx", P), ("kept_off", P), ("slot_of", P), ("hot", P),
+                ("topk_idx", P), ("topk_pos", P), ("topk_cnt", P), ("err", P)]
+
+
+def _sig(name, res, args):
+    f = getattr(_L, name)
+    f.restype = res
+    f.argtypes = args
+
+
+_sig("lsa_version", i32, [])
+_sig("lsa_last_error", ctypes.c_char_p, [])
+_sig("lsa_status_name", ctypes.c_char_p, [i32])
+_sig("lsa_index_score", i32, [P, i32, P, P, i32, P, P, i64, P, P, i64, i32, i32, i32, P, P, P])
+_sig("lsa_select_workspace_size", sz, [i64])
+_sig("lsa_select", i32, [P, P, i64, i32, P, i64, P, P, P, sz, P, P])
+_sig("lsa_topk", i32, [P, i32, P, P, P, i64, i32, i32, P, P, P, P])
+_sig("lsa_gather", i32, [P, i64, P, i64, P, P, i32, P, i64, P, P, P])
+_sig("lsa_sparse_attn_workspace_size", sz, [i32, i32, i32, i32])
+_sig("lsa_sparse_attn", i32, [P, i32, P, i64, i64, i64, P, i32, i32, i32, i32, f32, P, P, P, sz, P])
+_sig("lsa_ctx_create", i32, [ctypes.POINTER(Params), ctypes.POINTER(P)])
+_sig("lsa_ctx_destroy", i32, [P])
+_sig("lsa_decode_step", i32, [P, i64, P, P, P, P, P, P])
+_sig("lsa_decode_step_host", i32, [P, i64, P, P, P, P, P, P])
+_sig("lsa_ctx_get_view", i32, [P, ctypes.POINTER(View)])
+_sig("lsa_ctx_set_timing", i32, [P, i32])
+_sig("lsa_ctx_stage_times", i32, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)])
+_sig("lsa_ctx_reset_counters", i32, [P])
+_sig("lsa_ctx_launches", i64, [P])
+
+lib = _L
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _check(status, where):
+    if status != 0:
+        raise LsaError(status, where)
+
+
+def version() -> int:
+    return int(_L.lsa_version())
+
+
+# ------------------------------------------------------------------ stages
+
+def index_score(q, q_dtype, w, k, k_dtype, k_scale, seq_off, n_total, H, d, z, I=None, idx=None, idx_off=None,
+                list_capacity=0, stream=None):
+    B = seq_off.numel() - 1
+    _check(_L.lsa_index_score(_ptr(q), DTYPE[q_dtype], _ptr(w), _ptr(k), DTYPE[k_dtype], _ptr(k_scale),
+                              _ptr(seq_off), n_total, _ptr(idx), _ptr(idx_off), list_capacity, B, H, d,
+                              _ptr(z), _ptr(I), _stream(stream)), "lsa_index_score")
+
+
+def select_workspace_size(n_total) -> int:
+    return int(_L.lsa_select_workspace_size(n_total))
+
+
+def select(z, seq_off, n_total, kept_idx, capacity, kept_off, mask, workspace, err, stream=None):
+    B = seq_off.numel() - 1
+    _check(_L.lsa_select(_ptr(z), _ptr(seq_off), n_total, B, _ptr(kept_idx), capacity, _ptr(kept_off), _ptr(mask),
+                         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(err),
+                         _stream(stream)), "lsa_select")
+
+
+def topk(z, z_by_entry, seq_off, kept_idx, kept_off, kept_capacity, k, topk_idx, topk_pos, topk_cnt, stream=None):
+    B = kept_off.numel() - 1
+    _check(_L.lsa_topk(_ptr(z), int(z_by_entry), _ptr(seq_off), _ptr(kept_idx), _ptr(kept_off), kept_capacity, B, k,
+                       _ptr(topk_idx), _ptr(topk_pos), _ptr(topk_cnt), _stream(stream)), "lsa_topk")
+
+
+def gather(cold_host, row_bytes, seq_off, n_total, kept_idx, kept_off, hot, hot_capacity, slot_of, err,
+           stream=None):
+    B = seq_off.numel() - 1
+    _check(_L.lsa_gather(_ptr(cold_host), row_bytes, _ptr(seq_off), n_total, _ptr(kept_idx), _ptr(kept_off), B,
+                         _ptr(hot), hot_capacity, _ptr(slot_of), _ptr(err), _stream(stream)), "lsa_gather")
+
+
+def sparse_attn_workspace_size(B, Hq, D, k) -> int:
+    return int(_L.lsa_sparse_attn_workspace_size(B, Hq, D, k))
+
+
+def sparse_attn(Q, dtype, kv, kv_row_stride, k_off, v_off, rows, B, Hq, D, k, scale, out, lse, workspace,
+                stream=None):
+    _check(_L.lsa_sparse_attn(_ptr(Q), DTYPE[dtype], _ptr(kv), kv_row_stride, k_off, v_off, _ptr(rows), B, Hq, D,
+                              k, float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream)), "lsa_sparse_attn")
+
+
+# ----------------------------------------------------------- decode context
+
+class Context:
+    """Owns an lsa_ctx: the tau-cadence decode loop over device-resident keys and a pinned cold pool.
+
+    The caller keeps `keys`, `k_scale` and `cold_host` alive for the context's lifetime.
+    """
+
+    def __init__(self, *, B, H, d, q_dtype, k_dtype, Hq, D, attn_dtype, topk, seq_off_host, keys, k_scale,
+                 cold_host, row_bytes, kv_row_stride, k_off, v_off, kept_capacity, tau=64, scale=0.0):
+        self._seq_off = torch.as_tensor(seq_off_host, dtype=torch.int64).contiguous()
+        n_total = int(self._seq_off[-1])
+        self.params = Params(B, H, d, DTYPE[q_dtype], DTYPE[k_dtype], Hq, D, DTYPE[attn_dtype], topk, tau,
+                             float(scale), n_total, self._seq_off.data_ptr(), _ptr(keys), _ptr(k_scale),
+                             _ptr(cold_host), row_bytes, kv_row_stride, k_off, v_off, kept_capacity)
+        self._keep = (keys, k_scale, cold_host)
+        h = P()
+        _check(_L.lsa_ctx_create(ctypes.byref(self.params), ctypes.byref(h)), "lsa_ctx_create")
+        self.handle = h
+        self.B, self.topk, self.n_total, self.kept_capacity = B, topk, n_total, kept_capacity
+
+    def close(self):
+        if self.handle:
+            _check(_L.lsa_ctx_destroy(self.handle), "lsa_ctx_destroy")
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def step(self, t, q, w, Q, out, lse=None, stream=None):
+        _check(_L.lsa_decode_step(self.handle, t, _ptr(q), _ptr(w), _ptr(Q), _ptr(out), _ptr(lse), _stream(stream)),
+               "lsa_decode_step")
+
+    def step_host(self, t, q_host, w_host, Q_host, out_host, lse_host=None, stream=None):
+        _check(_L.lsa_decode_step_host(self.handle, t, _ptr(q_host), _ptr(w_host), _ptr(Q_host), _ptr(out_host),
+                                       _ptr(lse_host), _stream(stream)), "lsa_decode_step_host")
+
+    def view(self) -> View:
+        v = View()
+        _check(_L.lsa_ctx_get_view(self.handle, ctypes.byref(v)), "lsa_ctx_get_view")
+        return v
+
+    def set_timing(self, on: bool):
+        _check(_L.lsa_ctx_set_timing(self.handle, int(on)), "lsa_ctx_set_timing")
+
+    def stage_times(self):
+        ms = (ctypes.c_double * N_STAGES)()
+        calls = (i64 * N_STAGES)()
+        _check(_L.lsa_ctx_stage_times(self.handle, ms, calls), "lsa_ctx_stage_times")
+        return {STAGES[i]: (ms[i], calls[i]) for i in range(N_STAGES)}
+
+    def reset_counters(self):
+        _check(_L.lsa_ctx_reset_counters(self.handle), "lsa_ctx_reset_counters")
+
+    def launches(self) -> int:
+        return int(_L.lsa_ctx_launches(self.handle))
+
+
+_cudart = None
+
+
+def device_view(ptr: int, numel: int, dtype: torch.dtype) -> torch.Tensor:
+    """Copy `numel` elements at a device address owned by a context into a new tensor (for inspection).
+
+    Synchronises the device first; uses the CUDA runtime torch already loaded.
+    """
+    global _cudart
+    if _cudart is None:
+        _cudart = ctypes.CDLL("libcudart.so.12")
+        _cudart.cudaMemcpy.restype = ctypes.c_int
+        _cudart.cudaMemcpy.argtypes = [P, P, sz, ctypes.c_int]
+    out = torch.empty(numel, dtype=dtype, device="cuda")
+    if numel:
+        torch.cuda.synchronize()
+        rc = _cudart.cudaMemcpy(out.data_ptr(), ptr, numel * out.element_size(), 3)  # device to device
+        if rc != 0:
+            raise RuntimeError(f"cudaMemcpy failed with error {rc}")
+    return out

@@ -270,3 +270,32 @@ CONFIGS = {
     "ctx500k": ctx500k,
     "ragged": ragged,
 }
+
+
+def to_torch(wl: Workload, device: str = "cuda", pin_cold: bool = True) -> dict:
+    """The workload's arrays as torch tensors: indexer inputs and attention queries on `device`,
+    the cold pool in page-locked host memory (when `pin_cold`).  Pure data movement."""
+    def raw(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            a = a.view(np.int16)
+        return torch.from_numpy(a)
+
+    t = dict(
+        seq_off=torch.from_numpy(wl.seq_off.copy()).to(device),
+        keys=raw(wl.keys).to(device),
+        k_scale=None if wl.k_scale is None else torch.from_numpy(np.ascontiguousarray(wl.k_scale[:, 0])).to(device),
+        q=raw(wl.q).to(device),
+        w=torch.from_numpy(np.ascontiguousarray(wl.w)).to(device),
+        Q=raw(wl.Q).to(device),
+    )
+    cold = raw(wl.cold)
+    t["cold"] = cold.pin_memory() if pin_cold else cold
+    return t
+
+
+def raw_to_torch(a: np.ndarray, device: str = "cuda") -> torch.Tensor:
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).to(device)

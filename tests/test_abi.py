@@ -1,0 +1,94 @@
+"""The C ABI boundary, checked without a GPU: the library loads, exports every
+symbol include/lsa.h declares, and rejects bad arguments on the host before
+launching anything (no CUDA call is reached on these paths)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lsa.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lsa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lsa():
+    from lookahead_sparse_kv_index_b200 import build
+
+    build.build()
+    from lookahead_sparse_kv_index_b200 import lsa as mod
+
+    return mod
+
+
+def test_every_declared_symbol_is_exported(lsa):
+    names = _declared()
+    assert len(names) >= 19
+    for n in names:
+        assert hasattr(lsa.lib, n), n
+    assert sorted(lsa.EXPORTS) == sorted(n for n in names)
+
+
+def test_version_and_status_names(lsa):
+    assert lsa.version() == 100
+    assert lsa.lib.lsa_status_name(0) == b"LSA_OK"
+    assert lsa.lib.lsa_status_name(3) == b"LSA_ERR_CAPACITY"
+
+
+def test_workspace_sizes(lsa):
+    assert lsa.select_workspace_size(0) == 0
+    assert lsa.select_workspace_size(1) >= 16
+    n = 4 * 131072
+    assert lsa.select_workspace_size(n) >= (n // 1024) * 12 + n // 8
+    assert lsa.sparse_attn_workspace_size(4, 128, 512, 2048) >= 4 * 128 * 514 * 4
+    assert lsa.sparse_attn_workspace_size(0, 128, 512, 2048) == 0
+
+
+def _score(lsa, **kw):
+    a = dict(q=1 << 20, qd=1, w=1 << 20, k=1 << 20, kd=1, ks=None, so=1 << 20, n=100, idx=None, idxo=None,
+             cap=0, B=1, H=64, d=128, z=1 << 20, I=None)
+    a.update(kw)
+    return lsa.lib.lsa_index_score(a["q"], a["qd"], a["w"], a["k"], a["kd"], a["ks"], a["so"], a["n"], a["idx"],
+                                   a["idxo"], a["cap"], a["B"], a["H"], a["d"], a["z"], a["I"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(z=None), 1), (dict(B=0), 1), (dict(H=65), 5), (dict(d=96), 5),
+    (dict(kd=2), 1), (dict(ks=1 << 20), 1), (dict(k=(1 << 20) + 8), 1), (dict(qd=2), 5), (dict(qd=7), 1),
+    (dict(idx=1 << 20), 1), (dict(n=-1), 1),
+])
+def test_index_score_rejects_bad_arguments(lsa, kw, status):
+    assert _score(lsa, **kw) == status
+    assert lsa.lib.lsa_last_error() != b""
+
+
+def test_other_entry_points_reject_bad_arguments(lsa):
+    L, big = lsa.lib, 1 << 20
+    assert L.lsa_select(None, big, 10, 1, big, 10, big, None, big, 1 << 20, None, None) == 1
+    assert L.lsa_select(big, big, 10, 1, big, 10, big, None, big, 1, None, None) == 1          # workspace
+    assert L.lsa_topk(big, 1, None, big, big, 10, 1, 32, big, None, big, None) == 1            # seq_off needed
+    assert L.lsa_topk(big, 0, None, big, big, 10, 1, 5000, big, None, big, None) == 5          # k too large
+    assert L.lsa_gather(big, 1000, big, 10, big, big, 1, big, 10, None, None, None) == 1       # row_bytes % 16
+    assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 48, 16, 1.0, big, None, big, 1 << 30, None) == 5
+    assert L.lsa_sparse_attn(big, 2, big, 512, 0, 0, big, 1, 128, 512, 16, 1.0, big, None, big, 1 << 30, None) == 5
+    assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 512, 16, -1.0, big, None, big, 1 << 30, None) == 1
+    assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 512, 16, 1.0, big, None, big, 16, None) == 1
+
+
+def test_ctx_create_rejects_bad_params(lsa):
+    import numpy as np
+
+    so = np.array([0, 10, 5], np.int64)
+    p = lsa.Params(2, 64, 128, 1, 1, 128, 512, 1, 2048, 64, 0.0, 5, so.ctypes.data, 1 << 20, None, 1 << 20,
+                   1024, 512, 0, 0, 100)
+    h = ctypes.c_void_p()
+    assert lsa.lib.lsa_ctx_create(ctypes.byref(p), ctypes.byref(h)) == 1   # seq_off decreasing
+    p.kv_row_stride = 256
+    assert lsa.lib.lsa_ctx_create(ctypes.byref(p), ctypes.byref(h)) == 1   # stride * 2 != row_bytes
+    assert h.value is None

@@ -1,0 +1,317 @@
+"""Parity of every CUDA stage with the fp64 oracle, called through the C ABI.
+
+Sizes span several tiles with ragged tails; the full-size workloads (128K and
+500K-token contexts, the ragged serving batch) run the decode steps in the same
+launch configuration the benchmark times.  Tolerances: see tests/gpu_cases.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_cases import (ATTN_TOL, I_TOL, Z_TOL, gpu_full_scores, gpu_select, in_mask_band, lsa_mod,
+                       rel_err_per_head, run_decode_and_check)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lsa():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    return lsa_mod()
+
+
+SCORE_CASES = {
+    "tiny": lambda: synth.tiny(),
+    "ragged_bf16": lambda: synth.small_ragged(key_dtype="bf16"),
+    "ragged_e4m3": lambda: synth.small_ragged(key_dtype="e4m3"),
+    "ragged_e4m3_d64_h16": lambda: synth.small_ragged(key_dtype="e4m3", H=16, d=64, lengths=(777, 129, 3000)),
+    "ragged_bf16_d64_h32": lambda: synth.small_ragged(key_dtype="bf16", H=32, d=64, lengths=(2048, 1, 999)),
+}
+
+
+# ------------------------------------------------------------------ score
+
+@pytest.mark.parametrize("name", sorted(SCORE_CASES))
+def test_index_score_full_matches_oracle(lsa, name):
+    wl = SCORE_CASES[name]()
+    dev = synth.to_torch(wl, pin_cold=False)
+    z, I = gpu_full_scores(wl, dev, lsa)
+    z_ref, I_ref = oracle.index_score(wl.q, wl.q_dtype, wl.w, wl.keys, wl.key_dtype, wl.k_scale, wl.seq_off,
+                                      wl.H, wl.d)
+    assert np.abs(z - z_ref).max() <= Z_TOL
+    assert np.abs(I - I_ref).max() <= I_TOL
+    # the arithmetic is fp32 accumulation of exactly representable products: far inside the tolerance
+    assert np.abs(z - z_ref).max() <= 1e-4 * max(1.0, np.abs(z_ref).max())
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_e4m3", "ragged_bf16"])
+def test_index_score_listed_matches_oracle(lsa, name):
+    wl = SCORE_CASES[name]()
+    dev = synth.to_torch(wl, pin_cold=False)
+    rng = np.random.default_rng(3)
+    lists = [np.sort(rng.choice(int(n), size=int(rng.integers(0, n + 1)), replace=False))
+             for n in np.diff(wl.seq_off)]
+    idx = np.concatenate(lists).astype(np.int32)
+    idx_off = np.concatenate([[0], np.cumsum([len(x) for x in lists])]).astype(np.int64)
+    cap = int(idx_off[-1]) + 5
+    z = torch.full((cap,), 123.0, dtype=torch.float32, device="cuda")
+    lsa.index_score(dev["q"], wl.q_dtype, dev["w"], dev["keys"], wl.key_dtype, dev["k_scale"], dev["seq_off"],
+                    wl.n_total, wl.H, wl.d, z, None, idx=torch.from_numpy(idx).cuda(),
+                    idx_off=torch.from_numpy(idx_off).cuda(), list_capacity=cap)
+    torch.cuda.synchronize()
+    z = z.cpu().numpy()
+    z_ref = oracle.index_score_list(wl.q, wl.q_dtype, wl.w, wl.keys, wl.key_dtype, wl.k_scale, wl.seq_off, idx,
+                                    idx_off, wl.H, wl.d)
+    n = int(idx_off[-1])
+    assert np.abs(z[:n] - z_ref).max() <= Z_TOL
+    assert (z[n:] == 123.0).all()          # nothing written past the list
+
+
+# --------------------------------------------------------------- select
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_bf16", "ragged_e4m3"])
+def test_select_stage_exact_and_vs_fp64(lsa, name):
+    wl = SCORE_CASES[name]()
+    dev = synth.to_torch(wl, pin_cold=False)
+    z, _ = gpu_full_scores(wl, dev, lsa, want_I=False)
+    kept, ko, mask, err = gpu_select(z, wl.seq_off, lsa)
+    assert err == 0
+    # stage-exact: the oracle's selection on the GPU's own fp32 scores
+    k_ref, ko_ref, m_ref = oracle.select(z.astype(np.float64), wl.seq_off)
+    assert np.array_equal(kept, k_ref) and np.array_equal(ko, ko_ref) and np.array_equal(mask, m_ref)
+    # against the fp64 scores: equal outside the 1e-5 band around I = 0.5
+    z64 = oracle.index_score(wl.q, wl.q_dtype, wl.w, wl.keys, wl.key_dtype, wl.k_scale, wl.seq_off, wl.H, wl.d,
+                             want_I=False)
+    m64 = z64 >= 0
+    band = in_mask_band(z64)
+    assert np.array_equal(mask[~band], m64[~band])
+
+
+SELECT_LENGTHS = [0, 1, 31, 32, 33, 1023, 1024, 1025, 0, 5000, 0]
+
+
+@pytest.mark.parametrize("pattern", ["random", "all", "none", "signed_zero"])
+def test_select_edge_cases(lsa, pattern):
+    seq_off = np.concatenate([[0], np.cumsum(SELECT_LENGTHS)]).astype(np.int64)
+    n = int(seq_off[-1])
+    rng = np.random.default_rng(7)
+    z = rng.normal(size=n).astype(np.float32)
+    if pattern == "all":
+        z = np.abs(z)
+    elif pattern == "none":
+        z = -np.abs(z) - 1e-3
+    elif pattern == "signed_zero":
+        z[::3] = -0.0
+        z[1::3] = 0.0
+        z[2::3] = -1e-30
+    kept, ko, mask, err = gpu_select(z, seq_off, lsa)
+    k_ref, ko_ref, m_ref = oracle.select(z.astype(np.float64), seq_off)
+    assert err == 0
+    assert np.array_equal(kept, k_ref) and np.array_equal(ko, ko_ref) and np.array_equal(mask, m_ref)
+
+
+def test_select_capacity_overflow(lsa):
+    seq_off = np.array([0, 3000, 3100, 9000], np.int64)
+    z = np.random.default_rng(8).normal(size=9000).astype(np.float32)
+    k_ref, ko_ref, _ = oracle.select(z.astype(np.float64), seq_off)
+    cap = len(k_ref) // 2
+    kept, ko, _, err = gpu_select(z, seq_off, lsa, capacity=cap)
+    assert err == 3                                       # LSA_ERR_CAPACITY
+    assert np.array_equal(ko, ko_ref)                     # true offsets even past capacity
+    assert np.array_equal(kept, k_ref[:cap])
+
+
+# ----------------------------------------------------------------- top-k
+
+def _topk_gpu(lsa, z, z_by_entry, seq_off, kept, ko, k, cap=None):
+    B = len(ko) - 1
+    cap = len(kept) if cap is None else cap
+    t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dt)).cuda()
+    idx = torch.full((B, k), -9, dtype=torch.int32, device="cuda")
+    pos = torch.full((B, k), -9, dtype=torch.int32, device="cuda")
+    cnt = torch.full((B,), -9, dtype=torch.int32, device="cuda")
+    lsa.topk(t(z, np.float32), z_by_entry, t(seq_off, np.int64), t(kept if len(kept) else [0], np.int32),
+             t(ko, np.int64), cap, k, idx, pos, cnt)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), pos.cpu().numpy(), cnt.cpu().numpy()
+
+
+@pytest.mark.parametrize("k", [1, 7, 32, 300, 2048])
+@pytest.mark.parametrize("ties", [False, True])
+def test_topk_stage_exact(lsa, k, ties):
+    rng = np.random.default_rng(k + 1000 * ties)
+    lens = [0, 5, 40, 999, 4096, 20000, 2048, 2049]
+    seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    n = int(seq_off[-1])
+    z = rng.normal(size=n).astype(np.float32)
+    if ties:
+        z = np.round(z * 4) / 4          # few distinct values: ties everywhere
+        z[::5] = -0.0
+        z[1::5] = 0.0
+    z = np.abs(z) * np.where(rng.random(n) < 0.8, 1, -1).astype(np.float32)   # ~80% kept
+    kept, ko, _ = oracle.select(z.astype(np.float64), seq_off)
+    b_of = np.repeat(np.arange(len(lens)), np.diff(ko))
+    zk = z[seq_off[:-1][b_of] + kept].astype(np.float64)
+    ref_idx, ref_cnt = oracle.topk(zk, kept, ko, k)
+    # by entry (refresh step) and by kept position (listed step)
+    for by_entry, zin in ((1, z), (0, zk.astype(np.float32))):
+        idx, pos, cnt = _topk_gpu(lsa, zin, by_entry, seq_off, kept, ko, k)
+        assert np.array_equal(cnt, ref_cnt)
+        assert np.array_equal(idx, ref_idx)
+        for b in range(len(lens)):
+            c = cnt[b]
+            assert (pos[b][c:] == -1).all()
+            assert np.array_equal(kept[pos[b][:c]], idx[b][:c])
+            assert ((pos[b][:c] >= ko[b]) & (pos[b][:c] < ko[b + 1])).all()
+
+
+def test_topk_respects_kept_capacity(lsa):
+    seq_off = np.array([0, 100, 300], np.int64)
+    z = np.linspace(1, 2, 300).astype(np.float32)
+    kept, ko, _ = oracle.select(z.astype(np.float64), seq_off)
+    idx, pos, cnt = _topk_gpu(lsa, z, 1, seq_off, kept[:150], ko, 64, cap=150)
+    assert cnt[0] == 64 and cnt[1] == 50                     # only positions < 150 are read
+    assert (idx[1][:50] == np.arange(50)).all()
+
+
+# ---------------------------------------------------------------- gather
+
+def test_gather_bytes_and_slots(lsa):
+    rng = np.random.default_rng(9)
+    lens = [1000, 0, 37, 4000]
+    seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    n = int(seq_off[-1])
+    row_bytes = 1024
+    cold = torch.from_numpy(rng.integers(0, 255, size=(n, row_bytes), dtype=np.uint8)).pin_memory()
+    z = rng.normal(size=n).astype(np.float32)
+    kept, ko, _ = oracle.select(z.astype(np.float64), seq_off)
+    hot_ref, slot_ref = oracle.gather(cold.numpy(), seq_off, kept, ko)
+    cap = len(kept) + 3
+    hot = torch.zeros((cap, row_bytes), dtype=torch.uint8, device="cuda")
+    slot = torch.zeros(n, dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dt)).cuda()
+    lsa.gather(cold, row_bytes, t(seq_off, np.int64), n, t(kept, np.int32), t(ko, np.int64), hot, cap, slot, err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert np.array_equal(hot[: len(kept)].cpu().numpy(), hot_ref)
+    assert (hot[len(kept):].cpu().numpy() == 0).all()
+    assert np.array_equal(slot.cpu().numpy(), slot_ref)
+    # capacity overflow: the first `cap` rows, error raised
+    hot2 = torch.zeros((10, row_bytes), dtype=torch.uint8, device="cuda")
+    lsa.gather(cold, row_bytes, t(seq_off, np.int64), n, t(kept, np.int32), t(ko, np.int64), hot2, 10, None, err)
+    torch.cuda.synchronize()
+    assert err.item() == 3
+    assert np.array_equal(hot2.cpu().numpy(), hot_ref[:10])
+
+
+def test_gather_rejects_pageable_cold_pool(lsa):
+    cold = torch.zeros((16, 64), dtype=torch.uint8)          # not page-locked
+    t0 = torch.zeros(2, dtype=torch.int64, device="cuda")
+    with pytest.raises(lsa.LsaError) as e:
+        lsa.gather(cold, 64, t0, 16, torch.zeros(1, dtype=torch.int32, device="cuda"), t0,
+                   torch.zeros((4, 64), dtype=torch.uint8, device="cuda"), 4, None, None)
+    assert e.value.status == 1
+
+
+# ------------------------------------------------------------- attention
+
+ATTN_CASES = [
+    # dtype, B, Hq, D, k, n_rows, separate K/V
+    ("f32", 1, 8, 64, 32, 512, True),
+    ("f32", 2, 5, 96, 70, 300, True),
+    ("bf16", 2, 128, 512, 2048, 6000, False),
+    ("bf16", 3, 16, 128, 100, 400, True),
+]
+
+
+@pytest.mark.parametrize("case", ATTN_CASES, ids=lambda c: f"{c[0]}-B{c[1]}-H{c[2]}-D{c[3]}-k{c[4]}")
+def test_sparse_attn_matches_oracle(lsa, case):
+    dt, B, Hq, D, k, n_rows, separate = case
+    g = torch.Generator().manual_seed(11)
+    stride = 2 * D if separate else D
+    to_raw = (lambda x: synth.to_raw(x, dt))
+    Q = to_raw(torch.randn(B, Hq, D, generator=g))
+    kv = to_raw(torch.randn(n_rows, stride, generator=g))
+    rng = np.random.default_rng(12)
+    rows = np.full((B, k), -1, np.int32)
+    counts = [k, k // 3, 0][:B] if B <= 3 else [k] * B
+    for b in range(B):
+        c = min(counts[b], n_rows)
+        rows[b, :c] = np.sort(rng.choice(n_rows, size=c, replace=False))
+    out = torch.empty((B, Hq, D), dtype=torch.float32 if dt == "f32" else torch.int16, device="cuda")
+    lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    ws = torch.empty(lsa.sparse_attn_workspace_size(B, Hq, D, k), dtype=torch.uint8, device="cuda")
+    scale = 1.0 / math.sqrt(D)
+    v_off = D if separate else 0
+    lsa.sparse_attn(synth.raw_to_torch(Q), dt, synth.raw_to_torch(kv), stride, 0, v_off,
+                    torch.from_numpy(rows).cuda(), B, Hq, D, k, scale, out, lse, ws)
+    torch.cuda.synchronize()
+    out_ref, lse_ref = oracle.sparse_attn(Q, dt, kv, dt, stride, 0, v_off, rows.astype(np.int64), scale)
+    o = out.cpu().numpy()
+    o = oracle.decode(o.view(np.uint16), "bf16") if dt == "bf16" else o.astype(np.float64)
+    rel = rel_err_per_head(o, out_ref)
+    assert rel <= ATTN_TOL[dt], rel
+    lg = lse.cpu().numpy()
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lg), fin)
+    assert np.abs(lg[fin] - lse_ref[fin]).max() <= (1e-5 if dt == "f32" else 1e-3)
+    empty = rows.max(axis=1) < 0
+    assert (o[empty] == 0).all()
+
+
+# ---------------------------------------------------------- decode steps
+
+@pytest.mark.parametrize("name,steps,tau", [
+    ("tiny", [0, 1, 2, 3, 4, 5], 4),
+    ("ragged_bf16", [0, 1, 3, 4, 7], 4),
+    ("ragged_e4m3", [0, 2, 4, 5], 4),
+])
+def test_decode_steps_small(lsa, name, steps, tau):
+    wl = SCORE_CASES[name]()
+    reps = run_decode_and_check(wl, steps, tau, lsa)
+    assert [r["t"] for r in reps] == steps
+
+
+def test_decode_step_host_equals_device(lsa):
+    wl = synth.small_ragged(key_dtype="e4m3")
+    from gpu_cases import make_context
+
+    dev = synth.to_torch(wl)
+    ctx_a = make_context(wl, dev, lsa, tau=4)
+    ctx_b = make_context(wl, dev, lsa, tau=4)
+    out_a = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.int16, device="cuda")
+    lse_a = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device="cuda")
+    out_b = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.int16).pin_memory()
+    lse_b = torch.empty((wl.B, wl.Hq), dtype=torch.float32).pin_memory()
+    for t in range(6):
+        q_t, w_t, Q_t = wl.step_inputs(t)
+        ctx_a.step(t, synth.raw_to_torch(q_t), torch.from_numpy(w_t).cuda(), synth.raw_to_torch(Q_t), out_a, lse_a)
+        qh = synth.raw_to_torch(q_t, "cpu").pin_memory()
+        wh = torch.from_numpy(np.ascontiguousarray(w_t)).pin_memory()
+        Qh = synth.raw_to_torch(Q_t, "cpu").pin_memory()
+        ctx_b.step_host(t, qh, wh, Qh, out_b, lse_b)
+        torch.cuda.synchronize()
+        assert torch.equal(out_a.cpu(), out_b)
+        assert torch.equal(lse_a.cpu(), lse_b)
+    assert ctx_a.launches() > 0
+    ctx_a.close()
+    ctx_b.close()
+
+
+@pytest.mark.parametrize("name", ["ctx128k", "ctx500k"])
+def test_decode_full_size(lsa, name):
+    wl = synth.CONFIGS[name]()
+    reps = run_decode_and_check(wl, [0, 1, 63], 64, lsa, kept_capacity=int(0.2 * wl.n_total))
+    print(name, reps)
+
+
+def test_decode_ragged_serving_batch(lsa):
+    wl = synth.ragged()
+    reps = run_decode_and_check(wl, [0, 1], 64, lsa)
+    print("ragged", reps)
