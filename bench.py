@@ -60,6 +60,8 @@ def parse_args():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--hot-frac", type=float, default=0.2)
+    ap.add_argument("--only", choices=["scan"], default=None,
+                    help="run one stage alone (W + K launches), for profiling; prints its mean time")
     return ap.parse_args()
 
 
@@ -393,10 +395,47 @@ def run_cuda(args):
     return 0
 
 
+def run_only_scan(args):
+    """The full index scan alone on the workload, rotating REPLICAS copies of the keys (> L2)."""
+    import torch
+
+    import synth
+    from lookahead_sparse_kv_index_b200 import lsa
+
+    wl = synth.CONFIGS[args.config](with_cold=False)
+    dev = synth.to_torch(wl, pin_cold=False)
+    keys = [dev["keys"]] + [dev["keys"].clone() for _ in range(REPLICAS - 1)]
+    n = wl.n_total
+    z = torch.empty(n, dtype=torch.float32, device="cuda")
+    ws = torch.empty(lsa.index_score_workspace_size(wl.B, wl.H, wl.d), dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def once(i):
+        lsa.index_score(dev["q"], wl.q_dtype, dev["w"], keys[i % REPLICAS], wl.key_dtype, dev["k_scale"],
+                        dev["seq_off"], n, wl.H, wl.d, z, None, workspace=ws, err=err)
+
+    for i in range(args.warmup):
+        once(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        once(args.warmup + i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    gbs = algorithmic_scan_bytes(wl) / (ms / 1e3) / 1e9
+    print(json.dumps({"only": "scan", "config": args.config, "ms_per_scan": ms, "GBps": gbs,
+                      "err": int(err.item())}), flush=True)
+    return 0 if err.item() == 0 else 1
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.only == "scan":
+        return run_only_scan(args)
     return run_cuda(args)
 
 

@@ -6,8 +6,8 @@
 // indexer queries staged in shared memory as fp32, per-head accumulators in
 // registers.  It runs every supported shape and dtype (fp32 keys included)
 // and the listed (gathered) variant used between refreshes.  Full scans of
-// bf16 / e4m3 keys with H % 16 == 0 go to the tensor-core kernel in
-// index_score_tc.cu when it is built for the shape.
+// bf16 / e4m3 keys of the shapes index_score_tc.cu supports go to the
+// tensor-core kernel when the caller provides its workspace.
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -182,23 +182,15 @@ lsa_status launch_kt(const void *q, lsa_dtype q_dtype, const float *w, const voi
 
 }  // namespace
 
-lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, lsa_dtype k_dtype,
-                                 const float *k_scale, const int64_t *seq_off, int64_t n_total,
-                                 int32_t B, int32_t H, int32_t d, float *z, float *I,
-                                 cudaStream_t st, bool *handled);
-
 lsa_status launch_index_score(const void *q, lsa_dtype q_dtype, const float *w, const void *k,
                               lsa_dtype k_dtype, const float *k_scale, const int64_t *seq_off,
                               int64_t n_total, const int32_t *idx, const int64_t *idx_off,
                               int64_t list_capacity, int32_t B, int32_t H, int32_t d, float *z,
-                              float *I, cudaStream_t st) {
+                              float *I, void *workspace, int32_t *err, cudaStream_t st) {
     const int64_t n_axis = idx ? list_capacity : n_total;
-    if (!idx && q_dtype == LSA_BF16 && k_dtype != LSA_F32) {
-        bool handled = false;
-        lsa_status s = launch_index_score_tc(q, w, k, k_dtype, k_scale, seq_off, n_total, B, H, d, z,
-                                             I, st, &handled);
-        if (handled || s != LSA_OK) return s;
-    }
+    if (!idx && workspace && index_score_tc_supported(q_dtype, k_dtype, n_total, B, H, d))
+        return launch_index_score_tc(q, w, k, k_dtype, k_scale, seq_off, n_total, B, H, d, z, I, workspace,
+                                     err, st);
     switch (k_dtype) {
     case LSA_F32:
         return launch_kt<LSA_F32>(q, q_dtype, w, k, k_scale, seq_off, n_axis, idx, idx_off, B, H, d, z, I, st);

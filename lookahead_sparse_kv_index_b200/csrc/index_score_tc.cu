@@ -1,14 +1,453 @@
-// Tensor-core (tcgen05) index scan -- placeholder until the kernel lands:
-// every shape falls through to the CUDA-core path.
+// Tensor-core index scan for sm_100a ("FlashMemory-DeepSeek-V4 ... Lookahead
+// Sparse Attention", gist.science technical summary, section 2.1 "Scoring
+// Mechanism"):  z_s = sum_j w_j ReLU(q_j . k_s) for every entry s.
+//
+// Per sequence the q.k block is a dense contraction [entries x d] x [d x H]
+// (H = 64 heads, d = 128: 16 Kflop per entry), so the scan is HBM-bound only
+// when the dot products run on the tensor cores.  Layout of the work:
+//   * persistent CTAs, one per SM, each streaming a contiguous range of
+//     128-entry tiles (tiles never straddle two sequences);
+//   * warp 0: TMA loads of key tiles (128-byte swizzle) into a smem ring,
+//     plus one bulk copy of the sequence's query operand on a sequence change;
+//   * warp 1: tcgen05.mma, M = 128 entries, N = H heads, into one of four
+//     TMEM accumulators (H fp32 columns each);
+//   * warps 2-5: epilogue, one TMEM lane (= one entry) per thread: ReLU, gate
+//     weights, head sum in registers, one coalesced fp32 store per entry.
+// bf16 keys use kind::f16 (bf16 x bf16).  e4m3 keys use kind::f8f6f4 against
+// an exact two-piece e4m3 split of the bf16 query (see scan_tc_prep), so the
+// keys go from HBM to the tensor core untouched; the per-row key scale and the
+// per-head power-of-two query scale are applied after the ReLU, which is
+// positively homogeneous.
+//
+// Every wait is bounded in time; a wait that gives up sets LSA_ERR_TIMEOUT in
+// the caller's error word, stops the CTA's loops, drains the issued MMAs and
+// frees TMEM before returning.
+#include <cuda.h>
+
 #include "lsa_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace lsa {
+namespace {
 
-lsa_status launch_index_score_tc(const void *, const float *, const void *, lsa_dtype, const float *,
-                                 const int64_t *, int64_t, int32_t, int32_t, int32_t, float *, float *,
-                                 cudaStream_t, bool *handled) {
-    *handled = false;
+using namespace ptx;
+
+enum Kind { BF16_D128 = 0, BF16_D64 = 1, E4M3_D128 = 2 };
+
+template <int KIND>
+struct Cfg;
+template <>
+struct Cfg<BF16_D128> {
+    static constexpr int kStageBytes = 32768;   // 128 rows x 128 bf16
+    static constexpr int kBoxes = 2;            // two 64-element (128-byte) column boxes
+    static constexpr int kQBytesPerHead = 256;
+    static constexpr int kStages = 5;
+};
+template <>
+struct Cfg<BF16_D64> {
+    static constexpr int kStageBytes = 16384;
+    static constexpr int kBoxes = 1;
+    static constexpr int kQBytesPerHead = 128;
+    static constexpr int kStages = 8;
+};
+template <>
+struct Cfg<E4M3_D128> {
+    static constexpr int kStageBytes = 16384;   // 128 rows x 128 e4m3
+    static constexpr int kBoxes = 1;
+    static constexpr int kQBytesPerHead = 256;  // two e4m3 pieces x 128
+    static constexpr int kStages = 8;
+};
+
+constexpr int kThreads = 192;
+constexpr int kRows = 128;
+constexpr int kAcc = 4;                  // TMEM accumulator stages
+constexpr int kMaxB = 512;               // sequences per launch on this path
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
+constexpr int kImgTail = 1024;           // bytes after the operand image: gate weights w'
+
+__host__ __device__ constexpr uint32_t tmem_cols(int H) {
+    return (kAcc * H) <= 32 ? 32 : (kAcc * H) <= 64 ? 64 : (kAcc * H) <= 128 ? 128 : 256;
+}
+
+template <int KIND, int H>
+__host__ __device__ constexpr int qimg_bytes() {
+    return Cfg<KIND>::kQBytesPerHead * H;
+}
+
+template <int KIND, int H>
+__host__ __device__ constexpr int img_stride() {
+    return qimg_bytes<KIND, H>() + kImgTail;
+}
+
+// ---------------------------------------------------------------------------
+// Query operand image, one per sequence, laid out exactly as the MMA reads it
+// from shared memory (K-major, 128-byte swizzle: 16-byte chunk c of row j is
+// stored at chunk c ^ (j % 8)), followed by the gate weights w'.
+//
+// bf16 keys: the bf16 query itself, w' = w.
+// e4m3 keys: per head j, a power-of-two scale 2^e_j brings max_c |q_jc| into
+// [128, 256); p1 = e4m3(q 2^e_j), p2 = e4m3(q 2^e_j - p1), both round to
+// nearest even.  A bf16 value has 8 significant bits, p1 carries 4 and the
+// remainder q 2^e_j - p1 is a multiple of the bf16 ulp no larger than 8 ulps,
+// so p2 holds it exactly whenever it is at least the e4m3 subnormal step 2^-9:
+// p1 + p2 == q 2^e_j for every element with |q| >= 2^-10 max_c |q_jc|, and
+// within 2^-10 of it (2^-17 max_c |q_jc| before scaling) otherwise.
+// w'_j = w_j 2^-e_j.
+// ---------------------------------------------------------------------------
+template <int KIND, int H>
+__global__ void __launch_bounds__(256)
+scan_tc_prep(const uint16_t *__restrict__ q, const float *__restrict__ w, int d, uint8_t *__restrict__ img) {
+    const int b = blockIdx.x;
+    uint8_t *dst = img + size_t(b) * img_stride<KIND, H>();
+    float *wp = reinterpret_cast<float *>(dst + qimg_bytes<KIND, H>());
+    const uint16_t *qb = q + size_t(b) * H * d;
+    if (KIND != E4M3_D128) {
+        const int cpr = d / 8;   // 16-byte chunks per row
+        for (int i = threadIdx.x; i < H * cpr; i += blockDim.x) {
+            const int j = i / cpr, c = i - j * cpr;
+            const int a = c >> 3, cc = c & 7;
+            const int off = a * (H * 128) + j * 128 + ((cc ^ (j & 7)) << 4);
+            *reinterpret_cast<uint4 *>(dst + off) = *reinterpret_cast<const uint4 *>(qb + j * d + c * 8);
+        }
+        for (int j = threadIdx.x; j < H; j += blockDim.x) wp[j] = w[size_t(b) * H + j];
+    } else {
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+        for (int j = warp; j < H; j += nw) {
+            float v[4];
+            float m = 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                v[u] = bf16_to_f32(qb[j * 128 + 4 * lane + u]);
+                m = fmaxf(m, fabsf(v[u]));
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            int e = 0;
+            if (m > 0.f) {
+                int E;
+                frexpf(m, &E);
+                e = 8 - E;
+            }
+            uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float s = ldexpf(v[u], e);
+                const __nv_fp8_storage_t p1 = __nv_cvt_float_to_fp8(s, __NV_SATFINITE, __NV_E4M3);
+                const __half_raw h1 = __nv_cvt_fp8_to_halfraw(p1, __NV_E4M3);
+                const float r = s - __half2float(__half(h1));
+                const __nv_fp8_storage_t p2 = __nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3);
+                w0 |= uint32_t(p1) << (8 * u);
+                w1 |= uint32_t(p2) << (8 * u);
+            }
+            const int off = j * 128 + (((lane >> 2) ^ (j & 7)) << 4) + (lane & 3) * 4;
+            *reinterpret_cast<uint32_t *>(dst + off) = w0;
+            *reinterpret_cast<uint32_t *>(dst + H * 128 + off) = w1;
+            if (lane == 0) wp[j] = ldexpf(w[size_t(b) * H + j], -e);
+        }
+    }
+}
+
+// Sequence and rows of tile t; `b` is a cursor that only moves forward.
+__device__ __forceinline__ void tile_info(const int64_t *s_toff, const int64_t *s_seq, int B, int64_t t, int &b,
+                                          int64_t &row0, int64_t &row_end) {
+    while (b < B - 1 && t >= s_toff[b + 1]) ++b;
+    row0 = s_seq[b] + (t - s_toff[b]) * kRows;
+    row_end = s_seq[b + 1];
+}
+
+template <int KIND, int H>
+__global__ void __launch_bounds__(kThreads, 1)
+scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ img,
+        const int64_t *__restrict__ seq_off, int B, const float *__restrict__ k_scale, float *__restrict__ z,
+        float *__restrict__ I, int32_t *err) {
+    using C = Cfg<KIND>;
+    constexpr int S = C::kStages;
+    constexpr int QIMG = qimg_bytes<KIND, H>();
+    constexpr int ISTRIDE = img_stride<KIND, H>();
+    constexpr uint32_t NCOL = tmem_cols(H);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *stages = smem;
+    uint8_t *qimg = stages + S * C::kStageBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(qimg + 2 * QIMG);
+    uint64_t *empty = full + S;
+    uint64_t *qfull = empty + S;
+    uint64_t *qempty = qfull + 2;
+    uint64_t *tfull = qempty + 2;
+    uint64_t *tempty = tfull + kAcc;
+    uint64_t *drain = tempty + kAcc;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+    float *wbuf = reinterpret_cast<float *>(tmem_slot + 4);      // [4 warps][H]
+    int64_t *s_seq = reinterpret_cast<int64_t *>(wbuf + 4 * H);  // [B+1]
+    int64_t *s_toff = s_seq + (B + 1);                           // [B+1]
+    __shared__ int64_t s_range[2];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int *abort_v = abort_flag;
+
+    if (threadIdx.x == 0) {
+        int64_t acc = 0;
+        for (int b = 0; b <= B; ++b) {
+            s_seq[b] = seq_off[b];
+            s_toff[b] = acc;
+            if (b < B) acc += (seq_off[b + 1] - seq_off[b] + kRows - 1) / kRows;
+        }
+        const int64_t T = acc;
+        s_range[0] = T * blockIdx.x / gridDim.x;
+        s_range[1] = T * (blockIdx.x + 1) / gridDim.x;
+        *abort_flag = 0;
+        for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < 2; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 1); }
+        for (int s = 0; s < kAcc; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 4); }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) prefetch_tmap(&tmap);
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, NCOL);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int64_t t0 = s_range[0], t1 = s_range[1];
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int b = 0, cur = -1, qn = 0, st = 0;
+            uint32_t ph = 0;
+            int64_t row0, row_end;
+            for (int64_t t = t0; t < t1; ++t) {
+                tile_info(s_toff, s_seq, B, t, b, row0, row_end);
+                if (b != cur) {
+                    const int slot = qn & 1;
+                    if (!mbar_wait(&qempty[slot], ((qn >> 1) & 1) ^ 1, abort_v, kWaitLimitNs)) break;
+                    mbar_arrive_expect_tx(&qfull[slot], QIMG);
+                    bulk_load(qimg + slot * QIMG, img + size_t(b) * ISTRIDE, QIMG, &qfull[slot]);
+                    cur = b;
+                    ++qn;
+                }
+                if (!mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs)) break;
+                mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+#pragma unroll
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                    tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64, int(row0));
+                if (++st == S) { st = 0; ph ^= 1; }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = KIND == E4M3_D128 ? idesc_e4m3(kRows, H) : idesc_bf16(kRows, H);
+            int b = 0, cur = -1, qn = 0, slot = 0, st = 0, acc = 0;
+            uint32_t ph = 0, aph = 0;
+            int64_t row0, row_end;
+            bool issued = false;
+            for (int64_t t = t0; t < t1; ++t) {
+                tile_info(s_toff, s_seq, B, t, b, row0, row_end);
+                int bn = -1;
+                if (t + 1 < t1) {
+                    int bb = b;
+                    int64_t r0, r1;
+                    tile_info(s_toff, s_seq, B, t + 1, bb, r0, r1);
+                    bn = bb;
+                }
+                if (b != cur) {
+                    slot = qn & 1;
+                    if (!mbar_wait(&qfull[slot], (qn >> 1) & 1, abort_v, kWaitLimitNs)) break;
+                    cur = b;
+                    ++qn;
+                }
+                if (!mbar_wait(&tempty[acc], aph ^ 1, abort_v, kWaitLimitNs)) break;
+                if (!mbar_wait(&full[st], ph, abort_v, kWaitLimitNs)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + uint32_t(acc * H);
+                const uint32_t a0 = smem_u32(stages + st * C::kStageBytes);
+                const uint32_t b0 = smem_u32(qimg + slot * QIMG);
+                if (KIND == BF16_D128) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_f16(d_tmem, desc_sw128(a0 + (kk >> 2) * 16384 + (kk & 3) * 32),
+                                desc_sw128(b0 + (kk >> 2) * (H * 128) + (kk & 3) * 32), IDESC, kk > 0);
+                } else if (KIND == BF16_D64) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), IDESC, kk > 0);
+                } else {
+#pragma unroll
+                    for (int p = 0; p < 2; ++p)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_f8(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + p * (H * 128) + kk * 32),
+                                   IDESC, (p | kk) != 0);
+                }
+                issued = true;
+                mma_commit(&empty[st]);
+                mma_commit(&tfull[acc]);
+                if (bn != b) mma_commit(&qempty[slot]);
+                if (++st == S) { st = 0; ph ^= 1; }
+                if (++acc == kAcc) { acc = 0; aph ^= 1; }
+            }
+            if (issued) {
+                // every issued MMA has finished before TMEM is released
+                mma_commit(drain);
+                volatile int no_abort = 0;
+                if (!mbar_wait(drain, 0, &no_abort, kWaitLimitNs)) *abort_v = 1;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;   // TMEM lanes 32*quarter .. +31
+        float *wq = wbuf + quarter * H;
+        int b = 0, cur = -1, acc = 0;
+        uint32_t aph = 0;
+        int64_t row0, row_end;
+        for (int64_t t = t0; t < t1; ++t) {
+            tile_info(s_toff, s_seq, B, t, b, row0, row_end);
+            if (b != cur) {
+                __syncwarp();
+                const float *wsrc = reinterpret_cast<const float *>(img + size_t(b) * ISTRIDE + QIMG);
+                for (int j = lane; j < H; j += 32) wq[j] = wsrc[j];
+                __syncwarp();
+                cur = b;
+            }
+            const bool ok = mbar_wait(&tfull[acc], aph, abort_v, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
+            tc_fence_after();
+            uint32_t r[H];
+            const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * H);
+#pragma unroll
+            for (int c = 0; c < H / 16; ++c)
+                tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[c * 16]));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            float zs = 0.f;
+#pragma unroll
+            for (int j = 0; j < H; ++j) zs = fmaf(wq[j], fmaxf(__uint_as_float(r[j]), 0.f), zs);
+            const int64_t row = row0 + quarter * 32 + lane;
+            if (row < row_end) {
+                if (KIND == E4M3_D128) zs *= k_scale[row];
+                z[row] = zs;
+                if (I) I[row] = 1.f / (1.f + expf(-zs));
+            }
+            if (++acc == kAcc) { acc = 0; aph ^= 1; }
+        }
+    }
+    __syncwarp();   // lanes that skipped a role loop wait for their lane 0 here
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, NCOL);
+    }
+    if (threadIdx.x == 0 && *abort_v) raise_err(err, LSA_ERR_TIMEOUT);
+}
+
+// ------------------------------------------------------------------- host
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+template <int KIND, int H>
+size_t smem_bytes(int B) {
+    using C = Cfg<KIND>;
+    return 1024 + size_t(C::kStages) * C::kStageBytes + 2 * qimg_bytes<KIND, H>() +
+           (2 * C::kStages + 4 + 2 * kAcc + 1) * 8 + 16 + 4 * H * 4 + size_t(B + 1) * 16 + 64;
+}
+
+template <int KIND, int H>
+lsa_status launch(const void *q, const float *w, const void *k, const float *k_scale, const int64_t *seq_off,
+                  int64_t n_total, int B, int d, float *z, float *I, void *workspace, int32_t *err,
+                  cudaStream_t st) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) {
+        set_error("lsa_index_score: cuTensorMapEncodeTiled is unavailable");
+        return LSA_ERR_CUDA;
+    }
+    CUtensorMap map;
+    const bool fp8 = KIND == E4M3_D128;
+    const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(n_total)};
+    const cuuint64_t strides[1] = {cuuint64_t(d) * (fp8 ? 1 : 2)};
+    const cuuint32_t box[2] = {cuuint32_t(fp8 ? 128 : 64), cuuint32_t(kRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("lsa_index_score: cuTensorMapEncodeTiled failed (%d)", int(r));
+        return LSA_ERR_CUDA;
+    }
+    uint8_t *img = static_cast<uint8_t *>(workspace);
+    scan_tc_prep<KIND, H><<<B, 256, 0, st>>>(static_cast<const uint16_t *>(q), w, d, img);
+    LSA_LAUNCHED("scan_tc_prep");
+    const size_t smem = smem_bytes<KIND, H>(B);
+    auto kern = scan_tc<KIND, H>;
+    LSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    const int64_t max_tiles = (n_total + kRows - 1) / kRows + B;
+    const int grid = int(max_tiles < sm_count() ? max_tiles : sm_count());
+    kern<<<grid, kThreads, smem, st>>>(map, img, seq_off, B, k_scale, z, I, err);
+    LSA_LAUNCHED("scan_tc");
     return LSA_OK;
+}
+
+template <int KIND>
+lsa_status launch_h(int H, const void *q, const float *w, const void *k, const float *k_scale,
+                    const int64_t *seq_off, int64_t n_total, int B, int d, float *z, float *I, void *ws,
+                    int32_t *err, cudaStream_t st) {
+    switch (H) {
+    case 16: return launch<KIND, 16>(q, w, k, k_scale, seq_off, n_total, B, d, z, I, ws, err, st);
+    case 32: return launch<KIND, 32>(q, w, k, k_scale, seq_off, n_total, B, d, z, I, ws, err, st);
+    default: return launch<KIND, 64>(q, w, k, k_scale, seq_off, n_total, B, d, z, I, ws, err, st);
+    }
+}
+
+}  // namespace
+
+size_t index_score_tc_workspace(int32_t B, int32_t H, int32_t d) {
+    // the largest image stride of the shapes this path runs (256 bytes per head + tail)
+    (void)d;
+    return size_t(B) * (size_t(256) * H + kImgTail) + 256;
+}
+
+bool index_score_tc_supported(lsa_dtype q_dtype, lsa_dtype k_dtype, int64_t n_total, int32_t B, int32_t H,
+                              int32_t d) {
+    if (q_dtype != LSA_BF16 || n_total < kRows || B > kMaxB) return false;
+    if (!(H == 16 || H == 32 || H == 64)) return false;
+    if (k_dtype == LSA_BF16) return d == 128 || d == 64;
+    if (k_dtype == LSA_E4M3) return d == 128;
+    return false;
+}
+
+lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, lsa_dtype k_dtype,
+                                 const float *k_scale, const int64_t *seq_off, int64_t n_total, int32_t B,
+                                 int32_t H, int32_t d, float *z, float *I, void *workspace, int32_t *err,
+                                 cudaStream_t st) {
+    if (k_dtype == LSA_E4M3)
+        return launch_h<E4M3_D128>(H, q, w, k, k_scale, seq_off, n_total, B, d, z, I, workspace, err, st);
+    if (d == 128)
+        return launch_h<BF16_D128>(H, q, w, k, k_scale, seq_off, n_total, B, d, z, I, workspace, err, st);
+    return launch_h<BF16_D64>(H, q, w, k, k_scale, seq_off, n_total, B, d, z, I, workspace, err, st);
 }
 
 }  // namespace lsa

@@ -31,7 +31,8 @@ N_STAGES = 6
 
 # every symbol include/lsa.h declares
 EXPORTS = [
-    "lsa_version", "lsa_last_error", "lsa_status_name", "lsa_index_score", "lsa_select_workspace_size",
+    "lsa_version", "lsa_last_error", "lsa_status_name", "lsa_index_score_workspace_size", "lsa_index_score",
+    "lsa_select_workspace_size",
     "lsa_select", "lsa_topk", "lsa_gather", "lsa_sparse_attn_workspace_size", "lsa_sparse_attn",
     "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
     "lsa_ctx_set_timing", "lsa_ctx_stage_times", "lsa_ctx_reset_counters", "lsa_ctx_launches",
@@ -68,7 +69,8 @@ def _sig(name, res, args):
 _sig("lsa_version", i32, [])
 _sig("lsa_last_error", ctypes.c_char_p, [])
 _sig("lsa_status_name", ctypes.c_char_p, [i32])
-_sig("lsa_index_score", i32, [P, i32, P, P, i32, P, P, i64, P, P, i64, i32, i32, i32, P, P, P])
+_sig("lsa_index_score_workspace_size", sz, [i32, i32, i32])
+_sig("lsa_index_score", i32, [P, i32, P, P, i32, P, P, i64, P, P, i64, i32, i32, i32, P, P, P, sz, P, P])
 _sig("lsa_select_workspace_size", sz, [i64])
 _sig("lsa_select", i32, [P, P, i64, i32, P, i64, P, P, P, sz, P, P])
 _sig("lsa_topk", i32, [P, i32, P, P, P, i64, i32, i32, P, P, P, P])
@@ -113,12 +115,18 @@ def version() -> int:
 
 # ------------------------------------------------------------------ stages
 
+def index_score_workspace_size(B, H, d) -> int:
+    return int(_L.lsa_index_score_workspace_size(B, H, d))
+
+
 def index_score(q, q_dtype, w, k, k_dtype, k_scale, seq_off, n_total, H, d, z, I=None, idx=None, idx_off=None,
-                list_capacity=0, stream=None):
+                list_capacity=0, workspace=None, err=None, stream=None):
     B = seq_off.numel() - 1
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_L.lsa_index_score(_ptr(q), DTYPE[q_dtype], _ptr(w), _ptr(k), DTYPE[k_dtype], _ptr(k_scale),
                               _ptr(seq_off), n_total, _ptr(idx), _ptr(idx_off), list_capacity, B, H, d,
-                              _ptr(z), _ptr(I), _stream(stream)), "lsa_index_score")
+                              _ptr(z), _ptr(I), _ptr(workspace), ws_bytes, _ptr(err), _stream(stream)),
+           "lsa_index_score")
 
 
 def select_workspace_size(n_total) -> int:

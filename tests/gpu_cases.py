@@ -43,13 +43,19 @@ def unpack_mask(words: np.ndarray, n: int) -> np.ndarray:
     return np.unpackbits(words.astype("<u4").view(np.uint8), bitorder="little")[:n].astype(bool)
 
 
-def gpu_full_scores(wl, dev, lsa, want_I=True):
+def gpu_full_scores(wl, dev, lsa, want_I=True, tc=False):
+    """Full scan; tc=True passes the workspace that enables the tensor-core kernel."""
     n = wl.n_total
-    z = torch.empty(max(n, 1), dtype=torch.float32, device="cuda")
+    z = torch.full((max(n, 1) + 64,), 77.0, dtype=torch.float32, device="cuda")
     I = torch.empty_like(z) if want_I else None
+    ws = (torch.empty(lsa.index_score_workspace_size(wl.B, wl.H, wl.d), dtype=torch.uint8, device="cuda")
+          if tc else None)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
     lsa.index_score(dev["q"], wl.q_dtype, dev["w"], dev["keys"], wl.key_dtype, dev["k_scale"], dev["seq_off"], n,
-                    wl.H, wl.d, z, I)
+                    wl.H, wl.d, z, I, workspace=ws, err=err)
     torch.cuda.synchronize()
+    assert err.item() == 0, f"device error {err.item()}"
+    assert (z[n:].cpu().numpy() == 77.0).all(), "scan wrote past the entry axis"
     return z[:n].cpu().numpy(), (I[:n].cpu().numpy() if want_I else None)
 
 
@@ -85,6 +91,8 @@ def decoded(raw: np.ndarray, dtype: str) -> np.ndarray:
 
 def make_context(wl, dev, lsa, kept_capacity=None, tau=64):
     cap = kept_capacity or max(64, int(0.4 * wl.n_total) + 64)
+    if wl.n_total <= 65536:
+        cap = kept_capacity or wl.n_total + 64   # small cases may keep more than half the entries
     return lsa.Context(B=wl.B, H=wl.H, d=wl.d, q_dtype=wl.q_dtype, k_dtype=wl.key_dtype, Hq=wl.Hq, D=wl.D,
                        attn_dtype=wl.attn_dtype, topk=wl.topk, seq_off_host=wl.seq_off, keys=dev["keys"],
                        k_scale=dev["k_scale"], cold_host=dev["cold"], row_bytes=wl.row_bytes,

@@ -31,16 +31,19 @@ SCORE_CASES = {
     "ragged_e4m3": lambda: synth.small_ragged(key_dtype="e4m3"),
     "ragged_e4m3_d64_h16": lambda: synth.small_ragged(key_dtype="e4m3", H=16, d=64, lengths=(777, 129, 3000)),
     "ragged_bf16_d64_h32": lambda: synth.small_ragged(key_dtype="bf16", H=32, d=64, lengths=(2048, 1, 999)),
+    "ragged_bf16_h16": lambda: synth.small_ragged(key_dtype="bf16", H=16, d=128, lengths=(1, 127, 128, 129, 4000)),
+    "ragged_e4m3_h32": lambda: synth.small_ragged(key_dtype="e4m3", H=32, d=128, lengths=(5000, 300, 0, 129)),
 }
 
 
 # ------------------------------------------------------------------ score
 
+@pytest.mark.parametrize("tc", [False, True], ids=["cuda_core", "tcgen05"])
 @pytest.mark.parametrize("name", sorted(SCORE_CASES))
-def test_index_score_full_matches_oracle(lsa, name):
+def test_index_score_full_matches_oracle(lsa, name, tc):
     wl = SCORE_CASES[name]()
     dev = synth.to_torch(wl, pin_cold=False)
-    z, I = gpu_full_scores(wl, dev, lsa)
+    z, I = gpu_full_scores(wl, dev, lsa, tc=tc)
     z_ref, I_ref = oracle.index_score(wl.q, wl.q_dtype, wl.w, wl.keys, wl.key_dtype, wl.k_scale, wl.seq_off,
                                       wl.H, wl.d)
     assert np.abs(z - z_ref).max() <= Z_TOL
@@ -78,7 +81,7 @@ def test_index_score_listed_matches_oracle(lsa, name):
 def test_select_stage_exact_and_vs_fp64(lsa, name):
     wl = SCORE_CASES[name]()
     dev = synth.to_torch(wl, pin_cold=False)
-    z, _ = gpu_full_scores(wl, dev, lsa, want_I=False)
+    z, _ = gpu_full_scores(wl, dev, lsa, want_I=False, tc=True)
     kept, ko, mask, err = gpu_select(z, wl.seq_off, lsa)
     assert err == 0
     # stage-exact: the oracle's selection on the GPU's own fp32 scores
