@@ -90,10 +90,11 @@ const char *lsa_status_name(lsa_status s);
  * Full mode (idx == NULL): z / I are written for every entry, [n_total].
  * z        fp32 output (required).   I  fp32 output or NULL.
  * workspace  device scratch of lsa_index_score_workspace_size(B, H, d) bytes,
- *          16-byte aligned, or NULL.  With a workspace, full scans of bf16 q
- *          over bf16 keys (d 64 or 128) or e4m3 keys (d 128) with H in
- *          {16, 32, 64} run on the tensor cores (tcgen05); every other case,
- *          and every call without a workspace, runs the CUDA-core kernel.
+ *          16-byte aligned, or NULL.  With a workspace, scans (full or
+ *          listed) of bf16 q over bf16 keys (d 64 or 128) or e4m3 keys
+ *          (d 128) with H in {16, 32, 64}, B <= 512 and n_total >= 128 run on
+ *          the tensor cores (tcgen05); every other case, and every call
+ *          without a workspace, runs the CUDA-core kernel.
  *          The workspace holds the per-sequence query operand between the two
  *          kernels of one call; calls that share a workspace must not overlap.
  * err      device error word or NULL (LSA_ERR_TIMEOUT if a bounded wait of the
@@ -194,14 +195,19 @@ lsa_status lsa_gather(const void *cold_host, int64_t row_bytes, const int64_t *s
  *        may alias: k_off == v_off for a latent head serving as K and V).
  * rows   [B, k] int32 row indices into kv; negative entries are padding.
  * lse    [B, Hq] fp32 output or NULL.
- * workspace  at least lsa_sparse_attn_workspace_size(B, Hq, D, k) bytes.
- * Shapes run: D % 32 == 0, D <= 512, 1 <= Hq <= 256, 1 <= k <= 4096.
+ * workspace  at least lsa_sparse_attn_workspace_size(B, Hq, D, k) bytes
+ *        (fp32 split-K partials); calls that share it must not overlap.
+ * err    device error word or NULL (LSA_ERR_TIMEOUT if a bounded wait of the
+ *        tensor-core kernel gave up).
+ * Shapes run: D % 32 == 0, D <= 512, 1 <= Hq <= 256, 1 <= k <= 4096.  bf16
+ * with Hq = 128, D = 512 and K aliasing V (a latent head) runs on the tensor
+ * cores (tcgen05); every other shape on the CUDA cores.
  * ---------------------------------------------------------------------- */
 size_t lsa_sparse_attn_workspace_size(int32_t B, int32_t Hq, int32_t D, int32_t k);
 lsa_status lsa_sparse_attn(const void *Q, lsa_dtype dtype, const void *kv, int64_t kv_row_stride,
                            int64_t k_off, int64_t v_off, const int32_t *rows, int32_t B,
                            int32_t Hq, int32_t D, int32_t k, float scale, void *out, float *lse,
-                           void *workspace, size_t ws_bytes, void *stream);
+                           void *workspace, size_t ws_bytes, int32_t *err, void *stream);
 
 /* ------------------------------------------------------------------------
  * Decode context and lsa_decode_step -- the tau cadence (section 2.1,

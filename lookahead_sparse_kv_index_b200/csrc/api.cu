@@ -155,7 +155,7 @@ size_t lsa_sparse_attn_workspace_size(int32_t B, int32_t Hq, int32_t D, int32_t 
 lsa_status lsa_sparse_attn(const void *Q, lsa_dtype dtype, const void *kv, int64_t kv_row_stride,
                            int64_t k_off, int64_t v_off, const int32_t *rows, int32_t B,
                            int32_t Hq, int32_t D, int32_t k, float scale, void *out, float *lse,
-                           void *workspace, size_t ws_bytes, void *stream) {
+                           void *workspace, size_t ws_bytes, int32_t *err, void *stream) {
     clear_error();
     LSA_CHECK_ARG(Q && kv && rows && out && workspace, "lsa_sparse_attn: Q, kv, rows, out, workspace required");
     LSA_CHECK_SUPPORTED(dtype == LSA_F32 || dtype == LSA_BF16, "lsa_sparse_attn: dtype must be F32 or BF16");
@@ -173,7 +173,7 @@ lsa_status lsa_sparse_attn(const void *Q, lsa_dtype dtype, const void *kv, int64
     LSA_CHECK_ARG(ws_bytes >= sparse_attn_workspace(B, Hq, D, k) && aligned16(workspace),
                   "lsa_sparse_attn: workspace of %zu bytes < %zu", ws_bytes, sparse_attn_workspace(B, Hq, D, k));
     return launch_sparse_attn(Q, dtype, kv, kv_row_stride, k_off, v_off, rows, B, Hq, D, k, scale, out,
-                              lse, workspace, as_stream(stream));
+                              lse, workspace, err, as_stream(stream));
 }
 
 }  // extern "C"

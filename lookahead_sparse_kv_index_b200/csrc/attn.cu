@@ -11,8 +11,9 @@
 // merges the chunks:  M = max m_c,  L = sum l_c e^{m_c - M},
 // o = sum o_c e^{m_c - M} / L,  lse = M + log L.
 //
-// This is the CUDA-core path (fp32 FMA), used for every supported shape and
-// both dtypes.
+// This file holds the CUDA-core partial kernel (fp32 FMA; every supported
+// shape, both dtypes) and the combine kernel; the 128-head x 512 latent bf16
+// shape runs its partials on the tensor cores (attn_tc.cu).
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -22,6 +23,7 @@ constexpr int kChunk = 64;          // selected rows per block
 constexpr int kHeads = 16;          // query heads per block
 constexpr int kAttnThreads = 256;   // 8 warps, 2 heads each
 constexpr int kMaxColsPerLane = 16; // D <= 512
+constexpr int kMaxChunks = 64;      // k <= 4096 rows in chunks of kChunk
 
 template <typename T>
 struct Elem;
@@ -50,7 +52,7 @@ template <typename T>
 __global__ void __launch_bounds__(kAttnThreads)
 attn_partial(const T *__restrict__ Q, const T *__restrict__ kv, int64_t stride, int64_t k_off,
              int64_t v_off, const int32_t *__restrict__ rows, int Hq, int D, int k, float scale,
-             float *__restrict__ part) {
+             float *__restrict__ part_o, float *__restrict__ part_ml) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int ld = D + Elem<T>::kPad;
     const bool alias = k_off == v_off;
@@ -131,66 +133,103 @@ attn_partial(const T *__restrict__ Q, const T *__restrict__ kv, int64_t stride, 
                     if (j < ncols) acc[j] = fmaf(p, Elem<T>::get(vr, lane + 32 * j), acc[j]);
             }
         }
-        float *dst = part + ((int64_t(b) * nchunks + chunk) * Hq + h) * (D + 2);
+        const int64_t pi = (int64_t(b) * nchunks + chunk) * Hq + h;
+        float *dst = part_o + pi * D;
 #pragma unroll
         for (int j = 0; j < kMaxColsPerLane; ++j)
             if (j < ncols) dst[lane + 32 * j] = acc[j];
         if (lane == 0) {
-            dst[D] = m;
-            dst[D + 1] = l;
+            part_ml[pi * 2] = m;
+            part_ml[pi * 2 + 1] = l;
         }
         __syncwarp();
     }
 }
 
+// Merge of the chunk partials of one (head, sequence):
+//   M = max_c m_c,  w_c = e^{m_c - M},  L = sum_c l_c w_c,  o = sum_c w_c o_c / L,
+//   lse = M + log L;  a chunk with m_c = -inf (no selected row) has weight 0.
 template <typename T>
 __global__ void __launch_bounds__(128)
-attn_combine(const float *__restrict__ part, int nchunks, int Hq, int D, T *__restrict__ out,
-             float *__restrict__ lse) {
+attn_combine(const float *__restrict__ part_o, const float *__restrict__ part_ml, int nchunks, int Hq, int D,
+             T *__restrict__ out, float *__restrict__ lse) {
+    __shared__ float s_w[kMaxChunks];
+    __shared__ float s_ML[2];
     const int h = blockIdx.x, b = blockIdx.y;
-    const int64_t stride_c = int64_t(Hq) * (D + 2);
-    const float *base = part + (int64_t(b) * nchunks * Hq + h) * (D + 2);
-    float M = -INFINITY;
-    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, base[c * stride_c + D]);
-    float L = 0.f;
-    if (M != -INFINITY)
-        for (int c = 0; c < nchunks; ++c) {
-            const float m = base[c * stride_c + D];
-            if (m != -INFINITY) L += base[c * stride_c + D + 1] * expf(m - M);
+    const int64_t p0 = int64_t(b) * nchunks * Hq + h;   // partial index of chunk 0; chunk c adds c * Hq
+    if (threadIdx.x < 32) {
+        float M = -INFINITY;
+        for (int c = threadIdx.x; c < nchunks; c += 32) M = fmaxf(M, part_ml[(p0 + int64_t(c) * Hq) * 2]);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f;
+        for (int c = threadIdx.x; c < nchunks; c += 32) {
+            const float m = part_ml[(p0 + int64_t(c) * Hq) * 2];
+            const float w = (m == -INFINITY) ? 0.f : expf(m - M);
+            s_w[c] = w;
+            L += w * part_ml[(p0 + int64_t(c) * Hq) * 2 + 1];
         }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (threadIdx.x == 0) { s_ML[0] = M; s_ML[1] = L; }
+    }
+    __syncthreads();
+    const float M = s_ML[0], L = s_ML[1];
+    const float inv = M == -INFINITY ? 0.f : 1.f / L;
     const int64_t ob = (int64_t(b) * Hq + h) * D;
-    for (int col = threadIdx.x; col < D; col += blockDim.x) {
-        float o = 0.f;
-        if (M != -INFINITY) {
+    for (int col = 4 * threadIdx.x; col < D; col += 4 * blockDim.x) {
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (M != -INFINITY)
             for (int c = 0; c < nchunks; ++c) {
-                const float m = base[c * stride_c + D];
-                if (m != -INFINITY) o = fmaf(base[c * stride_c + col], expf(m - M), o);
+                const float w = s_w[c];
+                if (w == 0.f) continue;
+                const float4 v = *reinterpret_cast<const float4 *>(part_o + (p0 + int64_t(c) * Hq) * D + col);
+                a.x = fmaf(w, v.x, a.x); a.y = fmaf(w, v.y, a.y);
+                a.z = fmaf(w, v.z, a.z); a.w = fmaf(w, v.w, a.w);
             }
-            o /= L;
-        }
-        Elem<T>::put(out, ob + col, o);
+        Elem<T>::put(out, ob + col, a.x * inv);
+        Elem<T>::put(out, ob + col + 1, a.y * inv);
+        Elem<T>::put(out, ob + col + 2, a.z * inv);
+        Elem<T>::put(out, ob + col + 3, a.w * inv);
     }
     if (threadIdx.x == 0 && lse) lse[int64_t(b) * Hq + h] = M == -INFINITY ? -INFINITY : M + logf(L);
 }
 
+// Partial workspace: o [B, nchunks, Hq, D] fp32, then (m, l) [B, nchunks, Hq, 2] fp32.
+struct Parts {
+    float *o, *ml;
+};
+Parts parts(void *workspace, int B, int Hq, int D, int nchunks) {
+    float *o = static_cast<float *>(workspace);
+    return {o, o + align_up(size_t(B) * nchunks * Hq * D, 64)};
+}
+
 template <typename T>
 lsa_status launch_t(const void *Q, const void *kv, int64_t stride, int64_t k_off, int64_t v_off,
-                    const int32_t *rows, int B, int Hq, int D, int k, float scale, void *out,
-                    float *lse, void *workspace, cudaStream_t st) {
-    const int nchunks = (k + kChunk - 1) / kChunk;
-    const int ld = D + Elem<T>::kPad;
-    const bool alias = k_off == v_off;
-    const size_t smem = align_up(size_t(kChunk) * ld * sizeof(T) * (alias ? 1 : 2), 16) +
-                        size_t(kHeads) * D * 4 + size_t(kHeads) * kChunk * 4;
-    auto kern = attn_partial<T>;
-    LSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-    dim3 grid(nchunks, (Hq + kHeads - 1) / kHeads, B);
-    kern<<<grid, kAttnThreads, smem, st>>>(static_cast<const T *>(Q), static_cast<const T *>(kv), stride,
-                                           k_off, v_off, rows, Hq, D, k, scale,
-                                           static_cast<float *>(workspace));
-    LSA_LAUNCHED("attn_partial");
-    attn_combine<T><<<dim3(Hq, B), 128, 0, st>>>(static_cast<const float *>(workspace), nchunks, Hq, D,
-                                                 static_cast<T *>(out), lse);
+                    const int32_t *rows, int B, int Hq, int D, int k, float scale, void *out, float *lse,
+                    void *workspace, int32_t *err, cudaStream_t st) {
+    int nchunks;
+    Parts pp;
+    if (sparse_attn_tc_supported(sizeof(T) == 2 ? LSA_BF16 : LSA_F32, k_off, v_off, Hq, D)) {
+        nchunks = (k + sparse_attn_tc_chunk() - 1) / sparse_attn_tc_chunk();
+        pp = parts(workspace, B, Hq, D, nchunks);
+        lsa_status s = launch_sparse_attn_tc(Q, kv, stride, k_off, rows, B, k, scale, pp.o, pp.ml, err, st);
+        if (s != LSA_OK) return s;
+    } else {
+        nchunks = (k + kChunk - 1) / kChunk;
+        pp = parts(workspace, B, Hq, D, nchunks);
+        const int ld = D + Elem<T>::kPad;
+        const bool alias = k_off == v_off;
+        const size_t smem = align_up(size_t(kChunk) * ld * sizeof(T) * (alias ? 1 : 2), 16) +
+                            size_t(kHeads) * D * 4 + size_t(kHeads) * kChunk * 4;
+        auto kern = attn_partial<T>;
+        LSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+        dim3 grid(nchunks, (Hq + kHeads - 1) / kHeads, B);
+        kern<<<grid, kAttnThreads, smem, st>>>(static_cast<const T *>(Q), static_cast<const T *>(kv), stride,
+                                               k_off, v_off, rows, Hq, D, k, scale, pp.o, pp.ml);
+        LSA_LAUNCHED("attn_partial");
+    }
+    attn_combine<T><<<dim3(Hq, B), 128, 0, st>>>(pp.o, pp.ml, nchunks, Hq, D, static_cast<T *>(out), lse);
     LSA_LAUNCHED("attn_combine");
     return LSA_OK;
 }
@@ -198,17 +237,17 @@ lsa_status launch_t(const void *Q, const void *kv, int64_t stride, int64_t k_off
 }  // namespace
 
 size_t sparse_attn_workspace(int32_t B, int32_t Hq, int32_t D, int32_t k) {
-    const int nchunks = (k + kChunk - 1) / kChunk;
-    return size_t(B) * nchunks * Hq * (D + 2) * sizeof(float);
+    const int nchunks = (k + kChunk - 1) / kChunk;   // the finer of the two chunkings
+    return (align_up(size_t(B) * nchunks * Hq * D, 64) + size_t(B) * nchunks * Hq * 2) * sizeof(float);
 }
 
 lsa_status launch_sparse_attn(const void *Q, lsa_dtype dtype, const void *kv, int64_t stride,
                               int64_t k_off, int64_t v_off, const int32_t *rows, int32_t B,
                               int32_t Hq, int32_t D, int32_t k, float scale, void *out, float *lse,
-                              void *workspace, cudaStream_t st) {
+                              void *workspace, int32_t *err, cudaStream_t st) {
     if (dtype == LSA_F32)
-        return launch_t<float>(Q, kv, stride, k_off, v_off, rows, B, Hq, D, k, scale, out, lse, workspace, st);
-    return launch_t<uint16_t>(Q, kv, stride, k_off, v_off, rows, B, Hq, D, k, scale, out, lse, workspace, st);
+        return launch_t<float>(Q, kv, stride, k_off, v_off, rows, B, Hq, D, k, scale, out, lse, workspace, err, st);
+    return launch_t<uint16_t>(Q, kv, stride, k_off, v_off, rows, B, Hq, D, k, scale, out, lse, workspace, err, st);
 }
 
 }  // namespace lsa

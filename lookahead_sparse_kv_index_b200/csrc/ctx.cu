@@ -150,7 +150,7 @@ lsa_status run_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const 
         StageTimer tr(c, LSA_STAGE_RESCORE, st);
         LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
                                    p.n_total, c->kept_idx, c->kept_off, cap, p.B, p.H, p.d, c->z_kept,
-                                   nullptr, nullptr, c->err, st));
+                                   nullptr, c->score_ws, c->err, st));
         tr.done();
         StageTimer tk(c, LSA_STAGE_TOPK, st);
         LSA_TRY(launch_topk(c->z_kept, 0, c->seq_off_d, c->kept_idx, c->kept_off, p.B, p.topk, cap,
@@ -159,7 +159,7 @@ lsa_status run_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const 
     }
     StageTimer ta(c, LSA_STAGE_ATTN, st);
     LSA_TRY(launch_sparse_attn(Q, p.attn_dtype, c->hot, p.kv_row_stride, p.k_off, p.v_off, c->topk_pos,
-                               p.B, p.Hq, p.D, p.topk, c->scale, out, lse, c->attn_ws, st));
+                               p.B, p.Hq, p.D, p.topk, c->scale, out, lse, c->attn_ws, c->err, st));
     ta.done();
     c->launches += launch_count() - launches0;
     return LSA_OK;

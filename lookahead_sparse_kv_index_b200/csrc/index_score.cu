@@ -5,8 +5,8 @@
 // This file holds the CUDA-core path: one thread per entry, the sequence's
 // indexer queries staged in shared memory as fp32, per-head accumulators in
 // registers.  It runs every supported shape and dtype (fp32 keys included)
-// and the listed (gathered) variant used between refreshes.  Full scans of
-// bf16 / e4m3 keys of the shapes index_score_tc.cu supports go to the
+// and the listed (gathered) variant used between refreshes.  Scans of bf16 /
+// e4m3 keys of the shapes index_score_tc.cu supports, full or listed, go to the
 // tensor-core kernel when the caller provides its workspace.
 #include "lsa_internal.cuh"
 
@@ -188,9 +188,9 @@ lsa_status launch_index_score(const void *q, lsa_dtype q_dtype, const float *w, 
                               int64_t list_capacity, int32_t B, int32_t H, int32_t d, float *z,
                               float *I, void *workspace, int32_t *err, cudaStream_t st) {
     const int64_t n_axis = idx ? list_capacity : n_total;
-    if (!idx && workspace && index_score_tc_supported(q_dtype, k_dtype, n_total, B, H, d))
-        return launch_index_score_tc(q, w, k, k_dtype, k_scale, seq_off, n_total, B, H, d, z, I, workspace,
-                                     err, st);
+    if (workspace && index_score_tc_supported(q_dtype, k_dtype, n_total, B, H, d))
+        return launch_index_score_tc(q, w, k, k_dtype, k_scale, seq_off, n_total, idx, idx_off, list_capacity, B,
+                                     H, d, z, I, workspace, err, st);
     switch (k_dtype) {
     case LSA_F32:
         return launch_kt<LSA_F32>(q, q_dtype, w, k, k_scale, seq_off, n_axis, idx, idx_off, B, H, d, z, I, st);

@@ -11,13 +11,20 @@
 //     plus one bulk copy of the sequence's query operand on a sequence change;
 //   * warp 1: tcgen05.mma, M = 128 entries, N = H heads, into one of four
 //     TMEM accumulators (H fp32 columns each);
-//   * warps 2-5: epilogue, one TMEM lane (= one entry) per thread: ReLU, gate
-//     weights, head sum in registers, one coalesced fp32 store per entry.
+//   * warps 2-9: two epilogue warpgroups taking alternate tiles, one TMEM lane
+//     (= one entry) per thread: ReLU, gate weights, head sum in registers, one
+//     coalesced fp32 store per entry; the row scale is fetched before the
+//     accumulator wait so its latency overlaps the MMA.
 // bf16 keys use kind::f16 (bf16 x bf16).  e4m3 keys use kind::f8f6f4 against
 // an exact two-piece e4m3 split of the bf16 query (see scan_tc_prep), so the
 // keys go from HBM to the tensor core untouched; the per-row key scale and the
 // per-head power-of-two query scale are applied after the ReLU, which is
 // positively homogeneous.
+//
+// The listed variant scores only the entries of a per-sequence index list (the
+// kept set, re-ranked every decode step): the producer warp gathers those key
+// rows with cp.async into the same swizzled layout, three tiles in flight per
+// lane.
 //
 // Every wait is bounded in time; a wait that gives up sets LSA_ERR_TIMEOUT in
 // the caller's error word, stops the CTA's loops, drains the issued MMAs and
@@ -58,7 +65,8 @@ struct Cfg<E4M3_D128> {
     static constexpr int kStages = 8;
 };
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;         // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue (2 warpgroups)
+constexpr int kEpiGroups = 2;
 constexpr int kRows = 128;
 constexpr int kAcc = 4;                  // TMEM accumulator stages
 constexpr int kMaxB = 512;               // sequences per launch on this path
@@ -97,22 +105,25 @@ __host__ __device__ constexpr int img_stride() {
 template <int KIND, int H>
 __global__ void __launch_bounds__(256)
 scan_tc_prep(const uint16_t *__restrict__ q, const float *__restrict__ w, int d, uint8_t *__restrict__ img) {
+    // grid (B, H / 8): block (b, g) prepares heads 8g .. 8g+7 of sequence b, one warp per head
     const int b = blockIdx.x;
     uint8_t *dst = img + size_t(b) * img_stride<KIND, H>();
     float *wp = reinterpret_cast<float *>(dst + qimg_bytes<KIND, H>());
     const uint16_t *qb = q + size_t(b) * H * d;
+    const int h0 = blockIdx.y * 8;
     if (KIND != E4M3_D128) {
         const int cpr = d / 8;   // 16-byte chunks per row
-        for (int i = threadIdx.x; i < H * cpr; i += blockDim.x) {
-            const int j = i / cpr, c = i - j * cpr;
+        for (int i = threadIdx.x; i < 8 * cpr; i += blockDim.x) {
+            const int j = h0 + i / cpr, c = i % cpr;
             const int a = c >> 3, cc = c & 7;
             const int off = a * (H * 128) + j * 128 + ((cc ^ (j & 7)) << 4);
             *reinterpret_cast<uint4 *>(dst + off) = *reinterpret_cast<const uint4 *>(qb + j * d + c * 8);
         }
-        for (int j = threadIdx.x; j < H; j += blockDim.x) wp[j] = w[size_t(b) * H + j];
+        if (threadIdx.x < 8) wp[h0 + threadIdx.x] = w[size_t(b) * H + h0 + threadIdx.x];
     } else {
-        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-        for (int j = warp; j < H; j += nw) {
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        {
+            const int j = h0 + warp;
             float v[4];
             float m = 0.f;
 #pragma unroll
@@ -155,11 +166,28 @@ __device__ __forceinline__ void tile_info(const int64_t *s_toff, const int64_t *
     row_end = s_seq[b + 1];
 }
 
-template <int KIND, int H>
+// cp.async of 16 bytes (zero-filled when src_bytes == 0) and its group controls.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+constexpr int kGatherDepth = 3;   // listed mode: tiles of row gathers in flight per producer lane
+
+// LISTED = false: every entry of every sequence (key tiles by TMA).
+// LISTED = true:  entries idx[idx_off[b] ..] of each sequence (rows gathered
+//                 by the producer warp with cp.async); z is written at the list
+//                 position.
+template <int KIND, int H, bool LISTED>
 __global__ void __launch_bounds__(kThreads, 1)
-scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ img,
-        const int64_t *__restrict__ seq_off, int B, const float *__restrict__ k_scale, float *__restrict__ z,
-        float *__restrict__ I, int32_t *err) {
+scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kbytes,
+        const uint8_t *__restrict__ img, const int64_t *__restrict__ seq_off, const int32_t *__restrict__ idx,
+        const int64_t *__restrict__ idx_off, int64_t list_cap, int B, const float *__restrict__ k_scale,
+        float *__restrict__ z, float *__restrict__ I, int32_t *err) {
     using C = Cfg<KIND>;
     constexpr int S = C::kStages;
     constexpr int QIMG = qimg_bytes<KIND, H>();
@@ -179,26 +207,36 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ im
     uint64_t *drain = tempty + kAcc;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-    float *wbuf = reinterpret_cast<float *>(tmem_slot + 4);      // [4 warps][H]
-    int64_t *s_seq = reinterpret_cast<int64_t *>(wbuf + 4 * H);  // [B+1]
+    float *wbuf = reinterpret_cast<float *>(tmem_slot + 4);      // [8 epilogue warps][H]
+    int64_t *s_seq = reinterpret_cast<int64_t *>(wbuf + 8 * H);  // [B+1]
     int64_t *s_toff = s_seq + (B + 1);                           // [B+1]
+    int64_t *s_base = s_toff + (B + 1);                          // [B+1] entry base (listed mode)
     __shared__ int64_t s_range[2];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort_v = abort_flag;
 
     if (threadIdx.x == 0) {
+        // tile axis: the entries (full mode) or the list positions (listed mode)
+        const int64_t *axis = LISTED ? idx_off : seq_off;
         int64_t acc = 0;
         for (int b = 0; b <= B; ++b) {
-            s_seq[b] = seq_off[b];
+            int64_t a = axis[b];
+            if (LISTED && a > list_cap) a = list_cap;
+            s_seq[b] = a;
+            s_base[b] = seq_off[b];
             s_toff[b] = acc;
-            if (b < B) acc += (seq_off[b + 1] - seq_off[b] + kRows - 1) / kRows;
+            if (b < B) {
+                int64_t a1 = axis[b + 1];
+                if (LISTED && a1 > list_cap) a1 = list_cap;
+                acc += (a1 > a ? a1 - a + kRows - 1 : 0) / kRows;
+            }
         }
         const int64_t T = acc;
         s_range[0] = T * blockIdx.x / gridDim.x;
         s_range[1] = T * (blockIdx.x + 1) / gridDim.x;
         *abort_flag = 0;
-        for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < S; ++s) { mbar_init(&full[s], LISTED ? 32 : 1); mbar_init(&empty[s], 1); }
         for (int s = 0; s < 2; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 1); }
         for (int s = 0; s < kAcc; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 4); }
         mbar_init(drain, 1);
@@ -217,26 +255,88 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ im
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
+        if (!LISTED) {
+            if (lane == 0) {
+                int b = 0, cur = -1, qn = 0, st = 0;
+                uint32_t ph = 0;
+                int64_t row0, row_end;
+                for (int64_t t = t0; t < t1; ++t) {
+                    tile_info(s_toff, s_seq, B, t, b, row0, row_end);
+                    if (b != cur) {
+                        const int slot = qn & 1;
+                        if (!mbar_wait(&qempty[slot], ((qn >> 1) & 1) ^ 1, abort_v, kWaitLimitNs)) break;
+                        mbar_arrive_expect_tx(&qfull[slot], QIMG);
+                        bulk_load(qimg + slot * QIMG, img + size_t(b) * ISTRIDE, QIMG, &qfull[slot]);
+                        cur = b;
+                        ++qn;
+                    }
+                    if (!mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs)) break;
+                    mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+#pragma unroll
+                    for (int bx = 0; bx < C::kBoxes; ++bx)
+                        tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64,
+                                    int(row0));
+                    if (++st == S) { st = 0; ph ^= 1; }
+                }
+            }
+        } else {
+            // all 32 lanes gather: lane owns rows lane, lane+32, lane+64, lane+96 of each tile
+            constexpr int RB = KIND == E4M3_D128 ? 128 : (KIND == BF16_D128 ? 256 : 128);   // row bytes
+            constexpr int CPR = RB / 16;
             int b = 0, cur = -1, qn = 0, st = 0;
             uint32_t ph = 0;
             int64_t row0, row_end;
+            int pend[kGatherDepth + 1];
+            int npend = 0, head = 0;
             for (int64_t t = t0; t < t1; ++t) {
                 tile_info(s_toff, s_seq, B, t, b, row0, row_end);
+                bool ok = true;
                 if (b != cur) {
-                    const int slot = qn & 1;
-                    if (!mbar_wait(&qempty[slot], ((qn >> 1) & 1) ^ 1, abort_v, kWaitLimitNs)) break;
-                    mbar_arrive_expect_tx(&qfull[slot], QIMG);
-                    bulk_load(qimg + slot * QIMG, img + size_t(b) * ISTRIDE, QIMG, &qfull[slot]);
+                    if (lane == 0) {
+                        const int slot = qn & 1;
+                        ok = mbar_wait(&qempty[slot], ((qn >> 1) & 1) ^ 1, abort_v, kWaitLimitNs);
+                        if (ok) {
+                            mbar_arrive_expect_tx(&qfull[slot], QIMG);
+                            bulk_load(qimg + slot * QIMG, img + size_t(b) * ISTRIDE, QIMG, &qfull[slot]);
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
                     cur = b;
                     ++qn;
                 }
-                if (!mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs)) break;
-                mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+                if (ok) ok = mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                const uint32_t stage_u32 = smem_u32(stages + st * C::kStageBytes);
 #pragma unroll
-                for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64, int(row0));
+                for (int rr = 0; rr < 4; ++rr) {
+                    const int r = lane + 32 * rr;
+                    const int64_t p = row0 + r;
+                    const bool valid = p < row_end;
+                    const int64_t e = valid ? s_base[b] + idx[p] : 0;
+                    const uint8_t *src = kbytes + e * RB;
+#pragma unroll
+                    for (int c = 0; c < CPR; ++c)
+                        cp_async_16(stage_u32 + (c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4),
+                                    src + c * 16, valid ? 16u : 0u);
+                }
+                cp_async_commit();
+                pend[(head + npend) % (kGatherDepth + 1)] = st;
+                ++npend;
+                if (npend > kGatherDepth) {
+                    cp_async_wait_group<kGatherDepth>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(&full[pend[head]]);
+                    head = (head + 1) % (kGatherDepth + 1);
+                    --npend;
+                }
                 if (++st == S) { st = 0; ph ^= 1; }
+            }
+            cp_async_wait_group<0>();
+            fence_proxy_async_smem();
+            while (npend > 0) {
+                mbar_arrive(&full[pend[head]]);
+                head = (head + 1) % (kGatherDepth + 1);
+                --npend;
             }
         }
     } else if (warp == 1) {
@@ -301,12 +401,16 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ im
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int quarter = warp & 3;   // TMEM lanes 32*quarter .. +31
-        float *wq = wbuf + quarter * H;
-        int b = 0, cur = -1, acc = 0;
-        uint32_t aph = 0;
+        const int ew = warp - 2;              // 0..7
+        const int grp = ew >> 2;              // warpgroup: takes tiles t0 + grp, t0 + grp + 2, ...
+        const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
+        float *wq = wbuf + ew * H;
+        int b = 0, cur = -1;
         int64_t row0, row_end;
-        for (int64_t t = t0; t < t1; ++t) {
+        for (int64_t t = t0 + grp; t < t1; t += kEpiGroups) {
+            const int64_t i = t - t0;         // local tile index: accumulator i % 4, its (i / 4)-th use
+            const int acc = int(i % kAcc);
+            const uint32_t aph = uint32_t((i / kAcc) & 1);
             tile_info(s_toff, s_seq, B, t, b, row0, row_end);
             if (b != cur) {
                 __syncwarp();
@@ -315,6 +419,10 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ im
                 __syncwarp();
                 cur = b;
             }
+            const int64_t row = row0 + quarter * 32 + lane;   // entry (full) or list position (listed)
+            float sc = 1.f;
+            if (KIND == E4M3_D128 && row < row_end)
+                sc = __ldg(k_scale + (LISTED ? s_base[b] + idx[row] : row));
             const bool ok = mbar_wait(&tfull[acc], aph, abort_v, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
             tc_fence_after();
@@ -329,14 +437,18 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ im
             if (lane == 0) mbar_arrive(&tempty[acc]);
             float zs = 0.f;
 #pragma unroll
-            for (int j = 0; j < H; ++j) zs = fmaf(wq[j], fmaxf(__uint_as_float(r[j]), 0.f), zs);
-            const int64_t row = row0 + quarter * 32 + lane;
+            for (int j = 0; j < H; j += 4) {
+                const float4 wv = *reinterpret_cast<const float4 *>(wq + j);
+                zs = fmaf(wv.x, fmaxf(__uint_as_float(r[j]), 0.f), zs);
+                zs = fmaf(wv.y, fmaxf(__uint_as_float(r[j + 1]), 0.f), zs);
+                zs = fmaf(wv.z, fmaxf(__uint_as_float(r[j + 2]), 0.f), zs);
+                zs = fmaf(wv.w, fmaxf(__uint_as_float(r[j + 3]), 0.f), zs);
+            }
             if (row < row_end) {
-                if (KIND == E4M3_D128) zs *= k_scale[row];
+                if (KIND == E4M3_D128) zs *= sc;
                 z[row] = zs;
                 if (I) I[row] = 1.f / (1.f + expf(-zs));
             }
-            if (++acc == kAcc) { acc = 0; aph ^= 1; }
         }
     }
     __syncwarp();   // lanes that skipped a role loop wait for their lane 0 here
@@ -372,13 +484,13 @@ template <int KIND, int H>
 size_t smem_bytes(int B) {
     using C = Cfg<KIND>;
     return 1024 + size_t(C::kStages) * C::kStageBytes + 2 * qimg_bytes<KIND, H>() +
-           (2 * C::kStages + 4 + 2 * kAcc + 1) * 8 + 16 + 4 * H * 4 + size_t(B + 1) * 16 + 64;
+           (2 * C::kStages + 4 + 2 * kAcc + 1) * 8 + 16 + 8 * H * 4 + size_t(B + 1) * 24 + 64;
 }
 
 template <int KIND, int H>
 lsa_status launch(const void *q, const float *w, const void *k, const float *k_scale, const int64_t *seq_off,
-                  int64_t n_total, int B, int d, float *z, float *I, void *workspace, int32_t *err,
-                  cudaStream_t st) {
+                  int64_t n_total, const int32_t *idx, const int64_t *idx_off, int64_t list_cap, int B, int d,
+                  float *z, float *I, void *workspace, int32_t *err, cudaStream_t st) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) {
         set_error("lsa_index_score: cuTensorMapEncodeTiled is unavailable");
@@ -399,26 +511,28 @@ lsa_status launch(const void *q, const float *w, const void *k, const float *k_s
         return LSA_ERR_CUDA;
     }
     uint8_t *img = static_cast<uint8_t *>(workspace);
-    scan_tc_prep<KIND, H><<<B, 256, 0, st>>>(static_cast<const uint16_t *>(q), w, d, img);
+    scan_tc_prep<KIND, H><<<dim3(B, H / 8), 256, 0, st>>>(static_cast<const uint16_t *>(q), w, d, img);
     LSA_LAUNCHED("scan_tc_prep");
     const size_t smem = smem_bytes<KIND, H>(B);
-    auto kern = scan_tc<KIND, H>;
+    auto kern = idx ? scan_tc<KIND, H, true> : scan_tc<KIND, H, false>;
     LSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
-    const int64_t max_tiles = (n_total + kRows - 1) / kRows + B;
+    const int64_t axis = idx ? list_cap : n_total;
+    const int64_t max_tiles = (axis + kRows - 1) / kRows + B;
     const int grid = int(max_tiles < sm_count() ? max_tiles : sm_count());
-    kern<<<grid, kThreads, smem, st>>>(map, img, seq_off, B, k_scale, z, I, err);
-    LSA_LAUNCHED("scan_tc");
+    kern<<<grid, kThreads, smem, st>>>(map, static_cast<const uint8_t *>(k), img, seq_off, idx, idx_off, list_cap,
+                                       B, k_scale, z, I, err);
+    LSA_LAUNCHED(idx ? "scan_tc_listed" : "scan_tc");
     return LSA_OK;
 }
 
 template <int KIND>
 lsa_status launch_h(int H, const void *q, const float *w, const void *k, const float *k_scale,
-                    const int64_t *seq_off, int64_t n_total, int B, int d, float *z, float *I, void *ws,
-                    int32_t *err, cudaStream_t st) {
+                    const int64_t *seq_off, int64_t n_total, const int32_t *idx, const int64_t *idx_off,
+                    int64_t list_cap, int B, int d, float *z, float *I, void *ws, int32_t *err, cudaStream_t st) {
     switch (H) {
-    case 16: return launch<KIND, 16>(q, w, k, k_scale, seq_off, n_total, B, d, z, I, ws, err, st);
-    case 32: return launch<KIND, 32>(q, w, k, k_scale, seq_off, n_total, B, d, z, I, ws, err, st);
-    default: return launch<KIND, 64>(q, w, k, k_scale, seq_off, n_total, B, d, z, I, ws, err, st);
+    case 16: return launch<KIND, 16>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, ws, err, st);
+    case 32: return launch<KIND, 32>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, ws, err, st);
+    default: return launch<KIND, 64>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, ws, err, st);
     }
 }
 
@@ -440,14 +554,18 @@ bool index_score_tc_supported(lsa_dtype q_dtype, lsa_dtype k_dtype, int64_t n_to
 }
 
 lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, lsa_dtype k_dtype,
-                                 const float *k_scale, const int64_t *seq_off, int64_t n_total, int32_t B,
+                                 const float *k_scale, const int64_t *seq_off, int64_t n_total,
+                                 const int32_t *idx, const int64_t *idx_off, int64_t list_cap, int32_t B,
                                  int32_t H, int32_t d, float *z, float *I, void *workspace, int32_t *err,
                                  cudaStream_t st) {
     if (k_dtype == LSA_E4M3)
-        return launch_h<E4M3_D128>(H, q, w, k, k_scale, seq_off, n_total, B, d, z, I, workspace, err, st);
+        return launch_h<E4M3_D128>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I,
+                                   workspace, err, st);
     if (d == 128)
-        return launch_h<BF16_D128>(H, q, w, k, k_scale, seq_off, n_total, B, d, z, I, workspace, err, st);
-    return launch_h<BF16_D64>(H, q, w, k, k_scale, seq_off, n_total, B, d, z, I, workspace, err, st);
+        return launch_h<BF16_D128>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I,
+                                   workspace, err, st);
+    return launch_h<BF16_D64>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I,
+                              workspace, err, st);
 }
 
 }  // namespace lsa

@@ -79,7 +79,8 @@ size_t index_score_tc_workspace(int32_t B, int32_t H, int32_t d);
 bool index_score_tc_supported(lsa_dtype q_dtype, lsa_dtype k_dtype, int64_t n_total, int32_t B, int32_t H,
                               int32_t d);
 lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, lsa_dtype k_dtype,
-                                 const float *k_scale, const int64_t *seq_off, int64_t n_total, int32_t B,
+                                 const float *k_scale, const int64_t *seq_off, int64_t n_total,
+                                 const int32_t *idx, const int64_t *idx_off, int64_t list_cap, int32_t B,
                                  int32_t H, int32_t d, float *z, float *I, void *workspace, int32_t *err,
                                  cudaStream_t st);
 lsa_status launch_select(const float *z, const int64_t *seq_off, int64_t n_total, int32_t B,
@@ -96,7 +97,12 @@ lsa_status launch_gather(const void *cold_dev, int64_t row_bytes, const int64_t 
 lsa_status launch_sparse_attn(const void *Q, lsa_dtype dtype, const void *kv, int64_t stride,
                               int64_t k_off, int64_t v_off, const int32_t *rows, int32_t B,
                               int32_t Hq, int32_t D, int32_t k, float scale, void *out, float *lse,
-                              void *workspace, cudaStream_t st);
+                              void *workspace, int32_t *err, cudaStream_t st);
+bool sparse_attn_tc_supported(lsa_dtype dtype, int64_t k_off, int64_t v_off, int32_t Hq, int32_t D);
+int sparse_attn_tc_chunk();
+lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, int64_t k_off,
+                                 const int32_t *rows, int32_t B, int32_t k, float scale, float *part_o,
+                                 float *part_ml, int32_t *err, cudaStream_t st);
 size_t sparse_attn_workspace(int32_t B, int32_t Hq, int32_t D, int32_t k);
 
 // ------------------------------------------------------------- device side

@@ -4,11 +4,17 @@
 //
 // One 1024-thread block per sequence.  Scores map to an order-preserving
 // 32-bit key (larger z -> larger key, -0.0 folded onto +0.0).  A most-
-// significant-digit radix select (4 passes of 8 bits, shared-memory
-// histograms) finds the key T of the k-th largest entry and how many entries
-// equal to T must be taken; a final ordered pass takes every key > T and the
-// lowest-index entries with key == T, and compacts them in kept-list order,
-// which is ascending entry order.
+// significant-digit radix select (4 passes of 8 bits) finds the key T of the
+// k-th largest entry and how many entries equal to T must be taken; a final
+// ordered pass takes every key > T and the lowest-index entries with key == T,
+// and compacts them in kept-list order, which is ascending entry order.
+//
+// Kept sets of up to kSmemKeys entries are staged once in shared memory; every warp keeps its own 256-bin histogram and lanes that hit the
+// same bin are merged with __match_any_sync before one atomic (the kept
+// entries' keys share their top byte, so a single histogram would serialise);
+// the final pass gives each thread a contiguous run of positions, so it needs
+// only two block scans.  Larger kept sets re-read the scores from global
+// memory in every pass instead of staging them.
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -50,66 +56,83 @@ __device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
     return res;
 }
 
+constexpr int kSmemKeys = 32768;   // keys staged in shared memory (128 KB)
+constexpr int kWarps = kTopkThreads / 32;
+
 __global__ void __launch_bounds__(kTopkThreads)
-topk_radix(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict__ seq_off,
-           const int32_t *__restrict__ kept_idx, const int64_t *__restrict__ kept_off,
-           int64_t kept_cap, int k, int32_t *__restrict__ topk_idx, int32_t *__restrict__ topk_pos,
-           int32_t *__restrict__ topk_cnt) {
-    __shared__ int hist[256];
+topk_smem(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict__ seq_off,
+          const int32_t *__restrict__ kept_idx, const int64_t *__restrict__ kept_off, int64_t kept_cap, int k,
+          int32_t *__restrict__ topk_idx, int32_t *__restrict__ topk_pos, int32_t *__restrict__ topk_cnt) {
+    extern __shared__ uint32_t s_keys[];                 // [n]
+    __shared__ int s_hist[kWarps][256];
     __shared__ int s_warp[32];
     __shared__ uint32_t s_want;
     __shared__ int s_kr;
 
     const int b = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t p0 = kept_off[b];
-    int64_t n = kept_off[b + 1] - p0;
-    if (p0 >= kept_cap) n = 0;
-    else if (p0 + n > kept_cap) n = kept_cap - p0;
-    if (n < 0) n = 0;
-    const int64_t sbase = z_by_entry ? seq_off[b] : 0;
+    int64_t n64 = kept_off[b + 1] - p0;
+    if (p0 >= kept_cap) n64 = 0;
+    else if (p0 + n64 > kept_cap) n64 = kept_cap - p0;
+    if (n64 < 0) n64 = 0;
+    const int n = int(n64);
     int32_t *out_idx = topk_idx + int64_t(b) * k;
     int32_t *out_pos = topk_pos ? topk_pos + int64_t(b) * k : nullptr;
 
-    auto key_at = [&](int64_t i) -> uint32_t {
-        const int64_t p = p0 + i;
-        return order_key(z_by_entry ? z[sbase + kept_idx[p]] : z[p]);
-    };
-
-    if (n <= k) {
-        for (int64_t i = threadIdx.x; i < k; i += kTopkThreads) {
+    if (n <= k) {   // everything kept is chosen
+        for (int i = threadIdx.x; i < k; i += kTopkThreads) {
             out_idx[i] = i < n ? kept_idx[p0 + i] : -1;
             if (out_pos) out_pos[i] = i < n ? int32_t(p0 + i) : -1;
         }
-        if (threadIdx.x == 0) topk_cnt[b] = int32_t(n);
+        if (threadIdx.x == 0) topk_cnt[b] = n;
         return;
     }
+    const int64_t sbase = z_by_entry ? seq_off[b] : 0;
+    const bool staged = n <= kSmemKeys;
+    auto key = [&](int i) -> uint32_t {
+        return staged ? s_keys[i] : order_key(z_by_entry ? z[sbase + kept_idx[p0 + i]] : z[p0 + i]);
+    };
+    if (staged)
+        for (int i = threadIdx.x; i < n; i += kTopkThreads)
+            s_keys[i] = order_key(z_by_entry ? z[sbase + kept_idx[p0 + i]] : z[p0 + i]);
 
     uint32_t want = 0, hmask = 0;
     int kr = k;
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
-        if (threadIdx.x < 256) hist[threadIdx.x] = 0;
+        for (int i = lane; i < 256; i += 32) s_hist[warp][i] = 0;
         __syncthreads();
-        for (int64_t i = threadIdx.x; i < n; i += kTopkThreads) {
-            const uint32_t u = key_at(i);
-            if ((u & hmask) == want) atomicAdd(&hist[(u >> shift) & 0xFFu], 1);
+        for (int i0 = warp * 32; i0 < n; i0 += kTopkThreads) {
+            const int i = i0 + lane;
+            const uint32_t u = i < n ? key(i) : 0u;
+            const bool in = i < n && (u & hmask) == want;
+            const int digit = in ? int((u >> shift) & 0xFFu) : -1;
+            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+            if (in && (__ffs(peers) - 1) == lane) atomicAdd(&s_hist[warp][digit], __popc(peers));
         }
         __syncthreads();
-        if (threadIdx.x < 32) {
-            const int lane = threadIdx.x;
+        if (threadIdx.x < 256) {   // fold the warp histograms into warp 0's row
+            int sum = 0;
+#pragma unroll 8
+            for (int w = 0; w < kWarps; ++w) sum += s_hist[w][threadIdx.x];
+            s_hist[0][threadIdx.x] = sum;
+        }
+        __syncthreads();
+        if (warp == 0) {
             int local = 0;
 #pragma unroll
-            for (int x = 0; x < 8; ++x) local += hist[8 * lane + x];
-            int suf = local;   // inclusive suffix sum over lanes >= lane
+            for (int x = 0; x < 8; ++x) local += s_hist[0][8 * lane + x];
+            int suf = local;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                int y = __shfl_down_sync(0xffffffffu, suf, o);
+                const int y = __shfl_down_sync(0xffffffffu, suf, o);
                 if (lane + o < 32) suf += y;
             }
-            int above = suf - local;  // entries in higher lanes' bins
+            int above = suf - local;
 #pragma unroll
             for (int x = 7; x >= 0; --x) {
-                const int h = hist[8 * lane + x];
+                const int h = s_hist[0][8 * lane + x];
                 if (above < kr && above + h >= kr) {
                     s_want = want | (uint32_t(8 * lane + x) << shift);
                     s_kr = kr - above;
@@ -121,26 +144,35 @@ topk_radix(const float *__restrict__ z, int z_by_entry, const int64_t *__restric
         want = s_want;
         kr = s_kr;
         hmask |= 0xFFu << shift;
-        __syncthreads();
     }
-    // want is the exact key of the k-th largest; take kr of the entries equal to it.
-    int tie_carry = 0, out_carry = 0;
-    for (int64_t c0 = 0; c0 < n; c0 += kTopkThreads) {
-        const int64_t i = c0 + threadIdx.x;
-        uint32_t u = 0;
-        const bool valid = i < n;
-        if (valid) u = key_at(i);
-        const bool gt = valid && u > want;
-        const bool eq = valid && u == want;
-        int tot;
-        const int eq_rank = block_excl_scan(eq ? 1 : 0, s_warp, &tot) + tie_carry;
-        tie_carry += tot;
-        const bool take = gt || (eq && eq_rank < kr);
-        const int r = block_excl_scan(take ? 1 : 0, s_warp, &tot) + out_carry;
-        out_carry += tot;
-        if (take && r < k) {
-            out_idx[r] = kept_idx[p0 + i];
-            if (out_pos) out_pos[r] = int32_t(p0 + i);
+    // ordered take: thread t owns positions [t*per, (t+1)*per)
+    const int per = (n + kTopkThreads - 1) / kTopkThreads;
+    const int lo = min(n, threadIdx.x * per), hi = min(n, lo + per);
+    int n_eq = 0;
+    for (int i = lo; i < hi; ++i) n_eq += key(i) == want;
+    int tot;
+    int eq_rank = block_excl_scan(n_eq, s_warp, &tot);
+    int n_take = 0;
+    {
+        int r = eq_rank;
+        for (int i = lo; i < hi; ++i) {
+            const uint32_t u = key(i);
+            if (u > want) ++n_take;
+            else if (u == want) { n_take += r < kr; ++r; }
+        }
+    }
+    int out = block_excl_scan(n_take, s_warp, &tot);
+    {
+        int r = eq_rank;
+        for (int i = lo; i < hi; ++i) {
+            const uint32_t u = key(i);
+            bool take = u > want;
+            if (u == want) { take = r < kr; ++r; }
+            if (take && out < k) {
+                out_idx[out] = kept_idx[p0 + i];
+                if (out_pos) out_pos[out] = int32_t(p0 + i);
+                ++out;
+            }
         }
     }
     if (threadIdx.x == 0) topk_cnt[b] = k;
@@ -152,9 +184,11 @@ lsa_status launch_topk(const float *z, int32_t z_by_entry, const int64_t *seq_of
                        const int32_t *kept_idx, const int64_t *kept_off, int32_t B, int32_t k,
                        int64_t kept_cap, int32_t *topk_idx, int32_t *topk_pos, int32_t *topk_cnt,
                        cudaStream_t st) {
-    topk_radix<<<B, kTopkThreads, 0, st>>>(z, z_by_entry, seq_off, kept_idx, kept_off, kept_cap, k,
-                                           topk_idx, topk_pos, topk_cnt);
-    LSA_LAUNCHED("topk_radix");
+    const size_t smem = size_t(kSmemKeys) * 4;
+    LSA_CUDA(cudaFuncSetAttribute(topk_smem, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    topk_smem<<<B, kTopkThreads, smem, st>>>(z, z_by_entry, seq_off, kept_idx, kept_off, kept_cap, k, topk_idx,
+                                             topk_pos, topk_cnt);
+    LSA_LAUNCHED("topk_smem");
     return LSA_OK;
 }
 

@@ -76,7 +76,7 @@ _sig("lsa_select", i32, [P, P, i64, i32, P, i64, P, P, P, sz, P, P])
 _sig("lsa_topk", i32, [P, i32, P, P, P, i64, i32, i32, P, P, P, P])
 _sig("lsa_gather", i32, [P, i64, P, i64, P, P, i32, P, i64, P, P, P])
 _sig("lsa_sparse_attn_workspace_size", sz, [i32, i32, i32, i32])
-_sig("lsa_sparse_attn", i32, [P, i32, P, i64, i64, i64, P, i32, i32, i32, i32, f32, P, P, P, sz, P])
+_sig("lsa_sparse_attn", i32, [P, i32, P, i64, i64, i64, P, i32, i32, i32, i32, f32, P, P, P, sz, P, P])
 _sig("lsa_ctx_create", i32, [ctypes.POINTER(Params), ctypes.POINTER(P)])
 _sig("lsa_ctx_destroy", i32, [P])
 _sig("lsa_decode_step", i32, [P, i64, P, P, P, P, P, P])
@@ -158,10 +158,11 @@ def sparse_attn_workspace_size(B, Hq, D, k) -> int:
 
 
 def sparse_attn(Q, dtype, kv, kv_row_stride, k_off, v_off, rows, B, Hq, D, k, scale, out, lse, workspace,
-                stream=None):
+                err=None, stream=None):
     _check(_L.lsa_sparse_attn(_ptr(Q), DTYPE[dtype], _ptr(kv), kv_row_stride, k_off, v_off, _ptr(rows), B, Hq, D,
                               k, float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
-                              workspace.numel() * workspace.element_size(), _stream(stream)), "lsa_sparse_attn")
+                              workspace.numel() * workspace.element_size(), _ptr(err), _stream(stream)),
+           "lsa_sparse_attn")
 
 
 # ----------------------------------------------------------- decode context

@@ -48,7 +48,7 @@ def test_workspace_sizes(lsa):
     assert lsa.select_workspace_size(1) >= 16
     n = 4 * 131072
     assert lsa.select_workspace_size(n) >= (n // 1024) * 12 + n // 8
-    assert lsa.sparse_attn_workspace_size(4, 128, 512, 2048) >= 4 * 128 * 514 * 4
+    assert lsa.sparse_attn_workspace_size(4, 128, 512, 2048) >= 4 * 32 * 128 * 514 * 4
     assert lsa.sparse_attn_workspace_size(0, 128, 512, 2048) == 0
 
 
@@ -78,10 +78,10 @@ def test_other_entry_points_reject_bad_arguments(lsa):
     assert L.lsa_topk(big, 1, None, big, big, 10, 1, 32, big, None, big, None) == 1            # seq_off needed
     assert L.lsa_topk(big, 0, None, big, big, 10, 1, 5000, big, None, big, None) == 5          # k too large
     assert L.lsa_gather(big, 1000, big, 10, big, big, 1, big, 10, None, None, None) == 1       # row_bytes % 16
-    assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 48, 16, 1.0, big, None, big, 1 << 30, None) == 5
-    assert L.lsa_sparse_attn(big, 2, big, 512, 0, 0, big, 1, 128, 512, 16, 1.0, big, None, big, 1 << 30, None) == 5
-    assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 512, 16, -1.0, big, None, big, 1 << 30, None) == 1
-    assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 512, 16, 1.0, big, None, big, 16, None) == 1
+    assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 48, 16, 1.0, big, None, big, 1 << 30, None, None) == 5
+    assert L.lsa_sparse_attn(big, 2, big, 512, 0, 0, big, 1, 128, 512, 16, 1.0, big, None, big, 1 << 30, None, None) == 5
+    assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 512, 16, -1.0, big, None, big, 1 << 30, None, None) == 1
+    assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 512, 16, 1.0, big, None, big, 16, None, None) == 1
 
 
 def test_ctx_create_rejects_bad_params(lsa):

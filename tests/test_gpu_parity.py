@@ -52,8 +52,9 @@ def test_index_score_full_matches_oracle(lsa, name, tc):
     assert np.abs(z - z_ref).max() <= 1e-4 * max(1.0, np.abs(z_ref).max())
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged_e4m3", "ragged_bf16"])
-def test_index_score_listed_matches_oracle(lsa, name):
+@pytest.mark.parametrize("tc", [False, True], ids=["cuda_core", "tcgen05"])
+@pytest.mark.parametrize("name", ["tiny", "ragged_e4m3", "ragged_bf16", "ragged_bf16_d64_h32", "ragged_e4m3_h32"])
+def test_index_score_listed_matches_oracle(lsa, name, tc):
     wl = SCORE_CASES[name]()
     dev = synth.to_torch(wl, pin_cold=False)
     rng = np.random.default_rng(3)
@@ -63,10 +64,15 @@ def test_index_score_listed_matches_oracle(lsa, name):
     idx_off = np.concatenate([[0], np.cumsum([len(x) for x in lists])]).astype(np.int64)
     cap = int(idx_off[-1]) + 5
     z = torch.full((cap,), 123.0, dtype=torch.float32, device="cuda")
+    ws = (torch.empty(lsa.index_score_workspace_size(wl.B, wl.H, wl.d), dtype=torch.uint8, device="cuda")
+          if tc else None)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx_d = torch.from_numpy(np.concatenate([idx, np.zeros(5, np.int32)])).cuda()   # list buffer of `cap` slots
     lsa.index_score(dev["q"], wl.q_dtype, dev["w"], dev["keys"], wl.key_dtype, dev["k_scale"], dev["seq_off"],
-                    wl.n_total, wl.H, wl.d, z, None, idx=torch.from_numpy(idx).cuda(),
-                    idx_off=torch.from_numpy(idx_off).cuda(), list_capacity=cap)
+                    wl.n_total, wl.H, wl.d, z, None, idx=idx_d, idx_off=torch.from_numpy(idx_off).cuda(),
+                    list_capacity=cap, workspace=ws, err=err)
     torch.cuda.synchronize()
+    assert err.item() == 0
     z = z.cpu().numpy()
     z_ref = oracle.index_score_list(wl.q, wl.q_dtype, wl.w, wl.keys, wl.key_dtype, wl.k_scale, wl.seq_off, idx,
                                     idx_off, wl.H, wl.d)
@@ -148,7 +154,7 @@ def _topk_gpu(lsa, z, z_by_entry, seq_off, kept, ko, k, cap=None):
 @pytest.mark.parametrize("ties", [False, True])
 def test_topk_stage_exact(lsa, k, ties):
     rng = np.random.default_rng(k + 1000 * ties)
-    lens = [0, 5, 40, 999, 4096, 20000, 2048, 2049]
+    lens = [0, 5, 40, 999, 4096, 20000, 2048, 2049, 50000]   # the last keeps > 32768: unstaged keys
     seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
     n = int(seq_off[-1])
     z = rng.normal(size=n).astype(np.float32)
@@ -230,6 +236,8 @@ ATTN_CASES = [
     ("f32", 2, 5, 96, 70, 300, True),
     ("bf16", 2, 128, 512, 2048, 6000, False),
     ("bf16", 3, 16, 128, 100, 400, True),
+    ("bf16", 3, 128, 512, 300, 1000, False),   # tensor-core path: partial chunk, an empty sequence
+    ("bf16", 1, 128, 512, 128, 128, False),    # exactly one full chunk
 ]
 
 
