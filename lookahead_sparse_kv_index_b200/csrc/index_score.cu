@@ -188,7 +188,9 @@ lsa_status launch_index_score(const void *q, lsa_dtype q_dtype, const float *w, 
                               int64_t list_capacity, int32_t B, int32_t H, int32_t d, float *z,
                               float *I, void *workspace, int32_t *err, cudaStream_t st) {
     const int64_t n_axis = idx ? list_capacity : n_total;
-    if (workspace && index_score_tc_supported(q_dtype, k_dtype, n_total, B, H, d))
+    // the tensor-core path reads q rows with 16-byte loads and the workspace as 16-byte chunks
+    if (workspace && aligned16(q) && aligned16(workspace) &&
+        index_score_tc_supported(q_dtype, k_dtype, n_total, B, H, d))
         return launch_index_score_tc(q, w, k, k_dtype, k_scale, seq_off, n_total, idx, idx_off, list_capacity, B,
                                      H, d, z, I, workspace, err, st);
     switch (k_dtype) {

@@ -207,7 +207,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     uint64_t *drain = tempty + kAcc;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-    float *wbuf = reinterpret_cast<float *>(tmem_slot + 4);      // [8 epilogue warps][H]
+    // [8 epilogue warps][H] gate weights, read as float4: 16-byte aligned
+    float *wbuf = reinterpret_cast<float *>((reinterpret_cast<uintptr_t>(tmem_slot + 4) + 15) & ~uintptr_t(15));
     int64_t *s_seq = reinterpret_cast<int64_t *>(wbuf + 8 * H);  // [B+1]
     int64_t *s_toff = s_seq + (B + 1);                           // [B+1]
     int64_t *s_base = s_toff + (B + 1);                          // [B+1] entry base (listed mode)
@@ -484,7 +485,7 @@ template <int KIND, int H>
 size_t smem_bytes(int B) {
     using C = Cfg<KIND>;
     return 1024 + size_t(C::kStages) * C::kStageBytes + 2 * qimg_bytes<KIND, H>() +
-           (2 * C::kStages + 4 + 2 * kAcc + 1) * 8 + 16 + 8 * H * 4 + size_t(B + 1) * 24 + 64;
+           (2 * C::kStages + 4 + 2 * kAcc + 1) * 8 + 16 + 16 + 8 * H * 4 + size_t(B + 1) * 24 + 64;
 }
 
 template <int KIND, int H>
