@@ -273,8 +273,17 @@ typedef struct lsa_ctx_view {
 } lsa_ctx_view;
 lsa_status lsa_ctx_get_view(lsa_ctx *ctx, lsa_ctx_view *view);
 
-/* Stage timing.  When enabled, CUDA events bracket every stage on the stream
- * it runs on; lsa_ctx_stage_times synchronises on them and returns the
+/* CUDA graphs (on by default): after one eager run of each step kind, a step
+ * is captured once per distinct (q, w, Q, out, lse) pointer set and replayed
+ * with a single graph launch on the caller's stream (at most 256 cached
+ * graphs; the cache is cleared when full).  Captured steps bake in their
+ * pointers: the buffers behind them must stay allocated while the context
+ * may replay them. */
+lsa_status lsa_ctx_set_graphs(lsa_ctx *ctx, int32_t enable);
+
+/* Stage timing.  When enabled, steps run eagerly (no graphs) and CUDA
+ * events bracket every stage on the stream it runs on; lsa_ctx_stage_times
+ * synchronises on them and returns the
  * accumulated milliseconds and call counts per stage since the last reset
  * (arrays of LSA_STAGE_COUNT).  lsa_ctx_launches returns the number of
  * kernels the context has launched since the last reset. */

@@ -2,6 +2,9 @@
 // Every entry point validates on the host and launches nothing on failure.
 #include <cstdarg>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "lsa_internal.cuh"
 
@@ -30,6 +33,20 @@ int sm_count() {
         cached[dev] = n > 0 ? n : 148;
     }
     return cached[dev];
+}
+
+cudaError_t ensure_smem_raw(const void *func, size_t bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, size_t> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    size_t &cur = done[{func, dev}];
+    if (cur >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+    if (e == cudaSuccess) cur = bytes;
+    return e;
 }
 
 }  // namespace lsa

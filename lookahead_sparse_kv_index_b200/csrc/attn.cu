@@ -223,7 +223,7 @@ lsa_status launch_t(const void *Q, const void *kv, int64_t stride, int64_t k_off
         const size_t smem = align_up(size_t(kChunk) * ld * sizeof(T) * (alias ? 1 : 2), 16) +
                             size_t(kHeads) * D * 4 + size_t(kHeads) * kChunk * 4;
         auto kern = attn_partial<T>;
-        LSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+        LSA_CUDA(ensure_smem(kern, size_t(int(smem))));
         dim3 grid(nchunks, (Hq + kHeads - 1) / kHeads, B);
         kern<<<grid, kAttnThreads, smem, st>>>(static_cast<const T *>(Q), static_cast<const T *>(kv), stride,
                                                k_off, v_off, rows, Hq, D, k, scale, pp.o, pp.ml);

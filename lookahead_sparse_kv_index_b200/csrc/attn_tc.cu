@@ -310,7 +310,7 @@ lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, 
         set_error("lsa_sparse_attn: cuTensorMapEncodeTiled failed (%d)", int(r));
         return LSA_ERR_CUDA;
     }
-    LSA_CUDA(cudaFuncSetAttribute(attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)));
+    LSA_CUDA(ensure_smem(attn_tc, size_t(int(kSmemBytes))));
     const int nchunks = (k + kRowsPerCta - 1) / kRowsPerCta;
     attn_tc<<<dim3(nchunks, B), kThreads, kSmemBytes, st>>>(qmap, static_cast<const uint16_t *>(kv), stride, k_off,
                                                             rows, k, scale, part_o, part_ml, err);

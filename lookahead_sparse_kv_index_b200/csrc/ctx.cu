@@ -10,10 +10,39 @@
 // wait for the gather -> attention over the hot buffer.
 // Other steps: listed re-score of the kept set with the step's indexer query
 // -> top-k -> attention.  The host never waits inside a step.
+//
+// CUDA graphs: after one eager run of each step kind (refresh / listed), a
+// step is captured once per distinct set of input and output pointers and
+// replayed with one graph launch; a decode loop that reuses its buffers runs
+// two graphs.  Stage timing runs the kernels eagerly.
 #include <cmath>
+#include <cstring>
+#include <unordered_map>
 #include <vector>
 
 #include "lsa_internal.cuh"
+
+struct GraphKey {
+    bool refresh;
+    const void *q, *w, *Q;
+    void *out;
+    float *lse;
+    bool operator==(const GraphKey &o) const {
+        return refresh == o.refresh && q == o.q && w == o.w && Q == o.Q && out == o.out && lse == o.lse;
+    }
+};
+struct GraphKeyHash {
+    size_t operator()(const GraphKey &k) const {
+        size_t h = k.refresh;
+        for (const void *p : {k.q, k.w, k.Q, static_cast<const void *>(k.out), static_cast<const void *>(k.lse)})
+            h = h * 1000003u ^ std::hash<const void *>()(p);
+        return h;
+    }
+};
+struct GraphEntry {
+    cudaGraphExec_t exec;
+    int64_t kernels;
+};
 
 struct lsa_ctx {
     lsa_params p{};
@@ -51,6 +80,11 @@ struct lsa_ctx {
     double ms[LSA_STAGE_COUNT] = {0};
     int64_t calls[LSA_STAGE_COUNT] = {0};
     int64_t launches = 0;
+    // graphs
+    bool use_graphs = true;
+    bool eager_done[2] = {false, false};
+    cudaStream_t cap = nullptr;
+    std::unordered_map<GraphKey, GraphEntry, GraphKeyHash> graphs;
 };
 
 namespace {
@@ -67,8 +101,13 @@ void free_all(lsa_ctx *c) {
     if (c->ev_gather) cudaEventDestroy(c->ev_gather);
     for (auto &pe : c->pending) { cudaEventDestroy(pe.a); cudaEventDestroy(pe.b); }
     for (auto e : c->free_events) cudaEventDestroy(e);
+    for (auto &g : c->graphs) cudaGraphExecDestroy(g.second.exec);
+    c->graphs.clear();
     if (c->side) cudaStreamDestroy(c->side);
+    if (c->cap) cudaStreamDestroy(c->cap);
 }
+
+constexpr size_t kMaxGraphs = 256;
 
 cudaEvent_t take_event(lsa_ctx *c) {
     if (!c->free_events.empty()) {
@@ -117,11 +156,9 @@ lsa_status alloc(T **p, size_t bytes) {
     return LSA_OK;
 }
 
-lsa_status run_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const void *Q, void *out,
-                    float *lse, cudaStream_t st) {
+lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w, const void *Q, void *out,
+                        float *lse, cudaStream_t st) {
     const lsa_params &p = c->p;
-    const int64_t launches0 = launch_count();
-    const bool refresh = (t % c->tau) == 0 || !c->refreshed;
     const int64_t cap = p.kept_capacity;
     if (refresh) {
         StageTimer ts(c, LSA_STAGE_SCORE, st);
@@ -145,7 +182,6 @@ lsa_status run_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const 
                             c->topk_idx, c->topk_pos, c->topk_cnt, st));
         tk.done();
         LSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
-        c->refreshed = true;
     } else {
         StageTimer tr(c, LSA_STAGE_RESCORE, st);
         LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
@@ -161,7 +197,50 @@ lsa_status run_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const 
     LSA_TRY(launch_sparse_attn(Q, p.attn_dtype, c->hot, p.kv_row_stride, p.k_off, p.v_off, c->topk_pos,
                                p.B, p.Hq, p.D, p.topk, c->scale, out, lse, c->attn_ws, c->err, st));
     ta.done();
-    c->launches += launch_count() - launches0;
+    return LSA_OK;
+}
+
+lsa_status run_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const void *Q, void *out,
+                    float *lse, cudaStream_t st) {
+    const bool refresh = (t % c->tau) == 0 || !c->refreshed;
+    if (c->use_graphs && !c->timing && c->eager_done[refresh]) {
+        const GraphKey key{refresh, q, w, Q, out, lse};
+        auto it = c->graphs.find(key);
+        if (it == c->graphs.end()) {
+            if (c->graphs.size() >= kMaxGraphs) {
+                for (auto &g : c->graphs) cudaGraphExecDestroy(g.second.exec);
+                c->graphs.clear();
+            }
+            LSA_CUDA(cudaStreamBeginCapture(c->cap, cudaStreamCaptureModeThreadLocal));
+            const int64_t l0 = launch_count();
+            const lsa_status s = enqueue_step(c, refresh, q, w, Q, out, lse, c->cap);
+            cudaGraph_t g = nullptr;
+            const cudaError_t e = cudaStreamEndCapture(c->cap, &g);
+            if (s != LSA_OK || e != cudaSuccess) {
+                if (g) cudaGraphDestroy(g);
+                cudaGetLastError();
+                if (s != LSA_OK) return s;
+                set_error("lsa_decode_step: stream capture failed: %s", cudaGetErrorString(e));
+                return LSA_ERR_CUDA;
+            }
+            cudaGraphExec_t exec = nullptr;
+            const cudaError_t ie = cudaGraphInstantiate(&exec, g, 0);
+            cudaGraphDestroy(g);
+            if (ie != cudaSuccess) {
+                set_error("lsa_decode_step: graph instantiation failed: %s", cudaGetErrorString(ie));
+                return LSA_ERR_CUDA;
+            }
+            it = c->graphs.emplace(key, GraphEntry{exec, launch_count() - l0}).first;
+        }
+        LSA_CUDA(cudaGraphLaunch(it->second.exec, st));
+        c->launches += it->second.kernels;
+    } else {
+        const int64_t l0 = launch_count();
+        LSA_TRY(enqueue_step(c, refresh, q, w, Q, out, lse, st));
+        c->launches += launch_count() - l0;
+        c->eager_done[refresh] = true;
+    }
+    if (refresh) c->refreshed = true;
     return LSA_OK;
 }
 
@@ -245,6 +324,7 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
         if (ce == cudaSuccess) ce = cudaMemset(c->err, 0, 16);
         if (ce == cudaSuccess) ce = cudaMemset(c->hot, 0, size_t(cap) * p.row_bytes);
         if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking);
+        if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking);
         if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_sel, cudaEventDisableTiming);
         if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_gather, cudaEventDisableTiming);
         if (ce != cudaSuccess) {
@@ -312,6 +392,13 @@ lsa_status lsa_ctx_get_view(lsa_ctx *c, lsa_ctx_view *v) {
     v->topk_pos = c->topk_pos;
     v->topk_cnt = c->topk_cnt;
     v->err = c->err;
+    return LSA_OK;
+}
+
+lsa_status lsa_ctx_set_graphs(lsa_ctx *c, int32_t enable) {
+    clear_error();
+    LSA_CHECK_ARG(c, "lsa_ctx_set_graphs: ctx required");
+    c->use_graphs = enable != 0;
     return LSA_OK;
 }
 

@@ -165,9 +165,7 @@ lsa_status launch_kt(const void *q, lsa_dtype q_dtype, const float *w, const voi
 #define LSA_SCORE_LAUNCH(HM)                                                                    \
     do {                                                                                        \
         auto kern = score_cuda_core<KT, HM>;                                                    \
-        if (smem > 48 * 1024)                                                                   \
-            LSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,    \
-                                          int(smem)));                                          \
+        if (smem > 48 * 1024) LSA_CUDA(ensure_smem(kern, smem));                                \
         kern<<<dim3(unsigned(grid)), kTile, smem, st>>>(q, qb, w, k, k_scale, seq_off, idx,     \
                                                          idx_off, n_axis, B, H, d, z, I);       \
     } while (0)

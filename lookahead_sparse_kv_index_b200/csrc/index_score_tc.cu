@@ -516,7 +516,7 @@ lsa_status launch(const void *q, const float *w, const void *k, const float *k_s
     LSA_LAUNCHED("scan_tc_prep");
     const size_t smem = smem_bytes<KIND, H>(B);
     auto kern = idx ? scan_tc<KIND, H, true> : scan_tc<KIND, H, false>;
-    LSA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    LSA_CUDA(ensure_smem(kern, size_t(int(smem))));
     const int64_t axis = idx ? list_cap : n_total;
     const int64_t max_tiles = (axis + kRows - 1) / kRows + B;
     const int grid = int(max_tiles < sm_count() ? max_tiles : sm_count());

@@ -69,6 +69,15 @@ inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// Raises a kernel's dynamic shared-memory limit on the current device to at
+// least `bytes`, once: later calls are a table lookup (no CUDA call), so
+// launches inside a stream capture make no attribute calls.
+cudaError_t ensure_smem_raw(const void *func, size_t bytes);
+template <typename F>
+inline cudaError_t ensure_smem(F *func, size_t bytes) {
+    return ensure_smem_raw(reinterpret_cast<const void *>(func), bytes);
+}
+
 // Internal launchers (each validates nothing; the public entry points do).
 lsa_status launch_index_score(const void *q, lsa_dtype q_dtype, const float *w, const void *k,
                               lsa_dtype k_dtype, const float *k_scale, const int64_t *seq_off,

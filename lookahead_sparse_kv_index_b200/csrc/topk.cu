@@ -185,7 +185,7 @@ lsa_status launch_topk(const float *z, int32_t z_by_entry, const int64_t *seq_of
                        int64_t kept_cap, int32_t *topk_idx, int32_t *topk_pos, int32_t *topk_cnt,
                        cudaStream_t st) {
     const size_t smem = size_t(kSmemKeys) * 4;
-    LSA_CUDA(cudaFuncSetAttribute(topk_smem, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
+    LSA_CUDA(ensure_smem(topk_smem, size_t(int(smem))));
     topk_smem<<<B, kTopkThreads, smem, st>>>(z, z_by_entry, seq_off, kept_idx, kept_off, kept_cap, k, topk_idx,
                                              topk_pos, topk_cnt);
     LSA_LAUNCHED("topk_smem");

@@ -35,7 +35,8 @@ EXPORTS = [
     "lsa_select_workspace_size",
     "lsa_select", "lsa_topk", "lsa_gather", "lsa_sparse_attn_workspace_size", "lsa_sparse_attn",
     "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
-    "lsa_ctx_set_timing", "lsa_ctx_stage_times", "lsa_ctx_reset_counters", "lsa_ctx_launches",
+    "lsa_ctx_set_graphs", "lsa_ctx_set_timing", "lsa_ctx_stage_times", "lsa_ctx_reset_counters",
+    "lsa_ctx_launches",
 ]
 
 
@@ -82,6 +83,7 @@ _sig("lsa_ctx_destroy", i32, [P])
 _sig("lsa_decode_step", i32, [P, i64, P, P, P, P, P, P])
 _sig("lsa_decode_step_host", i32, [P, i64, P, P, P, P, P, P])
 _sig("lsa_ctx_get_view", i32, [P, ctypes.POINTER(View)])
+_sig("lsa_ctx_set_graphs", i32, [P, i32])
 _sig("lsa_ctx_set_timing", i32, [P, i32])
 _sig("lsa_ctx_stage_times", i32, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)])
 _sig("lsa_ctx_reset_counters", i32, [P])
@@ -209,6 +211,9 @@ class Context:
         v = View()
         _check(_L.lsa_ctx_get_view(self.handle, ctypes.byref(v)), "lsa_ctx_get_view")
         return v
+
+    def set_graphs(self, on: bool):
+        _check(_L.lsa_ctx_set_graphs(self.handle, int(on)), "lsa_ctx_set_graphs")
 
     def set_timing(self, on: bool):
         _check(_L.lsa_ctx_set_timing(self.handle, int(on)), "lsa_ctx_set_timing")

@@ -315,6 +315,33 @@ def test_decode_step_host_equals_device(lsa):
     ctx_b.close()
 
 
+def test_decode_graph_replay_equals_eager(lsa):
+    """Steps replayed from captured CUDA graphs give the same bytes as eager steps, across
+    refreshes, with the output buffers alternating (two graphs per step kind)."""
+    from gpu_cases import make_context
+
+    wl = synth.small_ragged(key_dtype="bf16")
+    dev = synth.to_torch(wl)
+    ctx_g = make_context(wl, dev, lsa, tau=3)
+    ctx_e = make_context(wl, dev, lsa, tau=3)
+    ctx_e.set_graphs(False)
+    outs = [torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.int16, device="cuda") for _ in range(3)]
+    lses = [torch.empty((wl.B, wl.Hq), dtype=torch.float32, device="cuda") for _ in range(3)]
+    ins = [wl.step_inputs(t) for t in range(10)]
+    dins = [(synth.raw_to_torch(q), torch.from_numpy(np.ascontiguousarray(w)).cuda(), synth.raw_to_torch(Q))
+            for q, w, Q in ins]
+    for t in range(10):
+        o = t % 2
+        ctx_g.step(t, *dins[t], outs[o], lses[o])
+        ctx_e.step(t, *dins[t], outs[2], lses[2])
+        torch.cuda.synchronize()
+        assert torch.equal(outs[o], outs[2]), t
+        assert torch.equal(lses[o], lses[2]), t
+    assert ctx_g.launches() == ctx_e.launches()
+    ctx_g.close()
+    ctx_e.close()
+
+
 @pytest.mark.parametrize("name", ["ctx128k", "ctx500k"])
 def test_decode_full_size(lsa, name):
     wl = synth.CONFIGS[name]()
