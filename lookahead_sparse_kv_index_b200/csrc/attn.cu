@@ -155,6 +155,7 @@ attn_combine(const float *__restrict__ part_o, const float *__restrict__ part_ml
              T *__restrict__ out, float *__restrict__ lse) {
     __shared__ float s_w[kMaxChunks];
     __shared__ float s_ML[2];
+    pdl_wait();   // partials come from the preceding kernel
     const int h = blockIdx.x, b = blockIdx.y;
     const int64_t p0 = int64_t(b) * nchunks * Hq + h;   // partial index of chunk 0; chunk c adds c * Hq
     if (threadIdx.x < 32) {
@@ -180,12 +181,22 @@ attn_combine(const float *__restrict__ part_o, const float *__restrict__ part_ml
     for (int col = 4 * threadIdx.x; col < D; col += 4 * blockDim.x) {
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
         if (M != -INFINITY)
-            for (int c = 0; c < nchunks; ++c) {
-                const float w = s_w[c];
-                if (w == 0.f) continue;
-                const float4 v = *reinterpret_cast<const float4 *>(part_o + (p0 + int64_t(c) * Hq) * D + col);
-                a.x = fmaf(w, v.x, a.x); a.y = fmaf(w, v.y, a.y);
-                a.z = fmaf(w, v.z, a.z); a.w = fmaf(w, v.w, a.w);
+            for (int c0 = 0; c0 < nchunks; c0 += 4) {   // four independent loads in flight
+                float4 v[4];
+                float w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + u;
+                    w[u] = c < nchunks ? s_w[c] : 0.f;
+                    v[u] = w[u] != 0.f
+                               ? *reinterpret_cast<const float4 *>(part_o + (p0 + int64_t(c) * Hq) * D + col)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    a.x = fmaf(w[u], v[u].x, a.x); a.y = fmaf(w[u], v[u].y, a.y);
+                    a.z = fmaf(w[u], v[u].z, a.z); a.w = fmaf(w[u], v[u].w, a.w);
+                }
             }
         Elem<T>::put(out, ob + col, a.x * inv);
         Elem<T>::put(out, ob + col + 1, a.y * inv);
@@ -229,7 +240,8 @@ lsa_status launch_t(const void *Q, const void *kv, int64_t stride, int64_t k_off
                                                k_off, v_off, rows, Hq, D, k, scale, pp.o, pp.ml);
         LSA_LAUNCHED("attn_partial");
     }
-    attn_combine<T><<<dim3(Hq, B), 128, 0, st>>>(pp.o, pp.ml, nchunks, Hq, D, static_cast<T *>(out), lse);
+    LSA_CUDA(launch_pdl(attn_combine<T>, dim3(Hq, B), dim3(128), 0, st, static_cast<const float *>(pp.o),
+                        static_cast<const float *>(pp.ml), nchunks, Hq, D, static_cast<T *>(out), lse));
     LSA_LAUNCHED("attn_combine");
     return LSA_OK;
 }

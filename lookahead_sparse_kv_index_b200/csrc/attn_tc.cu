@@ -88,6 +88,7 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const uint16_t *__restrict__ k
     volatile int *abort_v = abort_flag;
     const int64_t pbase = (int64_t(b) * nchunks + chunk) * kHq;
 
+    pdl_launch_dependents();
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         *s_nvalid = 0;
@@ -99,6 +100,15 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const uint16_t *__restrict__ k
         fence_mbar_init();
     }
     __syncthreads();
+    if (warp == 5 && lane == 0) {
+        // Q does not depend on the preceding kernel: start streaming it now
+        prefetch_tmap(&qmap);
+        for (int kd = 0; kd < kQStages; ++kd) {
+            mbar_arrive_expect_tx(&qfull[kd], kQStageBytes);
+            tma_load_2d(qs + kd * kQStageBytes, &qmap, &qfull[kd], kd * 64, b * kHq);
+        }
+    }
+    pdl_wait();   // the selected rows (and the hot buffer) come from preceding kernels
     if (threadIdx.x < kRowsPerCta) {
         const int i = chunk * kRowsPerCta + threadIdx.x;
         const int r = i < k ? rows[int64_t(b) * k + i] : -1;
@@ -121,6 +131,8 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const uint16_t *__restrict__ k
             part_ml[(pbase + threadIdx.x) * 2] = -INFINITY;
             part_ml[(pbase + threadIdx.x) * 2 + 1] = 0.f;
         }
+        if (warp == 5 && lane == 0)   // let the early Q loads land before the CTA exits
+            for (int kd = 0; kd < kQStages; ++kd) mbar_wait(&qfull[kd], 0, abort_v, kWaitLimitNs);
     } else if (warp < 4) {
         const int t = threadIdx.x;   // 0..127
         // ---- 1. gather the chunk's rows: 128 rows x 64 sixteen-byte chunks
@@ -181,13 +193,15 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const uint16_t *__restrict__ k
                 tc_fence_after();
                 float *dst = part_o + (pbase + t) * kD;
 #pragma unroll 1
-                for (int c = 0; c < kD / 16; ++c) {
-                    uint32_t o[16];
-                    tmem_ld_32x32b_x16(taddr + c * 16, o);
+                for (int c = 0; c < kD / 64; ++c) {   // 64 columns per wait
+                    uint32_t o[64];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        tmem_ld_32x32b_x16(taddr + c * 64 + q4 * 16, *reinterpret_cast<uint32_t(*)[16]>(&o[q4 * 16]));
                     tmem_ld_wait();
 #pragma unroll
-                    for (int u = 0; u < 16; u += 4)
-                        *reinterpret_cast<float4 *>(dst + c * 16 + u) =
+                    for (int u = 0; u < 64; u += 4)
+                        *reinterpret_cast<float4 *>(dst + c * 64 + u) =
                             make_float4(__uint_as_float(o[u]), __uint_as_float(o[u + 1]),
                                         __uint_as_float(o[u + 2]), __uint_as_float(o[u + 3]));
                 }
@@ -239,12 +253,11 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const uint16_t *__restrict__ k
             (void)issued;
         }
     } else {
-        // ---- 2. Q producer
+        // ---- 2. Q producer (the first kQStages slices were issued before the dependency wait)
         if (lane == 0) {
-            prefetch_tmap(&qmap);
             int st = 0;
-            uint32_t ph = 0;
-            for (int kd = 0; kd < kD / 64; ++kd) {
+            uint32_t ph = 1;
+            for (int kd = kQStages; kd < kD / 64; ++kd) {
                 if (!mbar_wait(&qempty[st], ph ^ 1, abort_v, kWaitLimitNs)) break;
                 mbar_arrive_expect_tx(&qfull[st], kQStageBytes);
                 tma_load_2d(qs + st * kQStageBytes, &qmap, &qfull[st], kd * 64, b * kHq);
@@ -312,8 +325,8 @@ lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, 
     }
     LSA_CUDA(ensure_smem(attn_tc, size_t(int(kSmemBytes))));
     const int nchunks = (k + kRowsPerCta - 1) / kRowsPerCta;
-    attn_tc<<<dim3(nchunks, B), kThreads, kSmemBytes, st>>>(qmap, static_cast<const uint16_t *>(kv), stride, k_off,
-                                                            rows, k, scale, part_o, part_ml, err);
+    LSA_CUDA(launch_pdl(attn_tc, dim3(nchunks, B), dim3(kThreads), kSmemBytes, st, qmap,
+                        static_cast<const uint16_t *>(kv), stride, k_off, rows, k, scale, part_o, part_ml, err));
     LSA_LAUNCHED("attn_tc");
     return LSA_OK;
 }

@@ -105,6 +105,7 @@ __host__ __device__ constexpr int img_stride() {
 template <int KIND, int H>
 __global__ void __launch_bounds__(256)
 scan_tc_prep(const uint16_t *__restrict__ q, const float *__restrict__ w, int d, uint8_t *__restrict__ img) {
+    pdl_launch_dependents();   // the scan may start its prologue and key loads now
     // grid (B, H / 8): block (b, g) prepares heads 8g .. 8g+7 of sequence b, one warp per head
     const int b = blockIdx.x;
     uint8_t *dst = img + size_t(b) * img_stride<KIND, H>();
@@ -253,11 +254,13 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int64_t t0 = s_range[0], t1 = s_range[1];
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (!LISTED) {
             if (lane == 0) {
+                pdl_wait();   // the q image comes from the preceding prep kernel
                 int b = 0, cur = -1, qn = 0, st = 0;
                 uint32_t ph = 0;
                 int64_t row0, row_end;
@@ -282,6 +285,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             }
         } else {
             // all 32 lanes gather: lane owns rows lane, lane+32, lane+64, lane+96 of each tile
+            pdl_wait();
             constexpr int RB = KIND == E4M3_D128 ? 128 : (KIND == BF16_D128 ? 256 : 128);   // row bytes
             constexpr int CPR = RB / 16;
             int b = 0, cur = -1, qn = 0, st = 0;
@@ -408,6 +412,18 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         float *wq = wbuf + ew * H;
         int b = 0, cur = -1;
         int64_t row0, row_end;
+        // row scale of this thread's row in tile t (e4m3 keys), loaded one tile of this group ahead
+        auto scale_of = [&](int64_t t) -> float {
+            if (KIND != E4M3_D128 || t >= t1) return 1.f;
+            int bb = b;
+            int64_t r0, r1;
+            tile_info(s_toff, s_seq, B, t, bb, r0, r1);
+            const int64_t r = r0 + quarter * 32 + lane;
+            if (r >= r1) return 1.f;
+            return __ldg(k_scale + (LISTED ? s_base[bb] + idx[r] : r));
+        };
+        pdl_wait();   // gate weights come from the preceding prep kernel
+        float sc_next = scale_of(t0 + grp);
         for (int64_t t = t0 + grp; t < t1; t += kEpiGroups) {
             const int64_t i = t - t0;         // local tile index: accumulator i % 4, its (i / 4)-th use
             const int acc = int(i % kAcc);
@@ -421,9 +437,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 cur = b;
             }
             const int64_t row = row0 + quarter * 32 + lane;   // entry (full) or list position (listed)
-            float sc = 1.f;
-            if (KIND == E4M3_D128 && row < row_end)
-                sc = __ldg(k_scale + (LISTED ? s_base[b] + idx[row] : row));
+            const float sc = sc_next;
+            sc_next = scale_of(t + kEpiGroups);
             const bool ok = mbar_wait(&tfull[acc], aph, abort_v, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
             tc_fence_after();
@@ -520,8 +535,8 @@ lsa_status launch(const void *q, const float *w, const void *k, const float *k_s
     const int64_t axis = idx ? list_cap : n_total;
     const int64_t max_tiles = (axis + kRows - 1) / kRows + B;
     const int grid = int(max_tiles < sm_count() ? max_tiles : sm_count());
-    kern<<<grid, kThreads, smem, st>>>(map, static_cast<const uint8_t *>(k), img, seq_off, idx, idx_off, list_cap,
-                                       B, k_scale, z, I, err);
+    LSA_CUDA(launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, map, static_cast<const uint8_t *>(k),
+                        static_cast<const uint8_t *>(img), seq_off, idx, idx_off, list_cap, B, k_scale, z, I, err));
     LSA_LAUNCHED(idx ? "scan_tc_listed" : "scan_tc");
     return LSA_OK;
 }

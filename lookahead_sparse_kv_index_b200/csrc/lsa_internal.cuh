@@ -8,6 +8,7 @@
 
 #include <cstdio>
 #include <string>
+#include <utility>
 
 #include "lsa.h"
 
@@ -114,7 +115,32 @@ lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, 
                                  float *part_ml, int32_t *err, cudaStream_t st);
 size_t sparse_attn_workspace(int32_t B, int32_t Hq, int32_t D, int32_t k);
 
+// Launch with programmatic dependent launch: the kernel may be scheduled as
+// soon as the previous kernel on the stream signals griddepcontrol.
+// launch_dependents; it must execute pdl_wait() before touching anything the
+// previous kernel writes (pdl_wait returns once that kernel has completed and
+// its memory is visible).  Captured into CUDA graphs as programmatic edges.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ------------------------------------------------------------- device side
+
+// Programmatic dependent launch controls (no-ops for a kernel launched without it).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // First error wins.
 __device__ __forceinline__ void raise_err(int32_t *err, int32_t code) {
