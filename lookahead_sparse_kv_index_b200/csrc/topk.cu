@@ -2,25 +2,16 @@
 // Lookahead Sparse Attention", gist.science technical summary, section 2.1
 // "Tiered Selection").
 //
-// One 1024-thread block per sequence.  Scores map to an order-preserving
-// 32-bit key (larger z -> larger key, -0.0 folded onto +0.0).  A most-
-// significant-digit radix select (4 passes of 8 bits) finds the key T of the
-// k-th largest entry and how many entries equal to T must be taken; a final
-// ordered pass takes every key > T and the lowest-index entries with key == T,
+// One 512-thread block per sequence.  Scores map to an order-preserving 32-bit
+// key (larger z -> larger key, -0.0 folded onto +0.0).  A most-significant-
+// digit radix select (up to 4 passes of 8 bits) finds the digits of the k-th
+// largest key and how many entries sharing them must be taken; an ordered pass
+// then takes every key above and the lowest-index entries at the threshold,
 // and compacts them in kept-list order, which is ascending entry order.
-//
-// Kept sets of up to kSmemKeys entries are staged once in shared memory; every warp keeps its own 256-bin histogram and lanes that hit the
-// same bin are merged with __match_any_sync before one atomic (the kept
-// entries' keys share their top byte, so a single histogram would serialise);
-// the final pass gives each thread a contiguous run of positions, so it needs
-// only two block scans.  Larger kept sets re-read the scores from global
-// memory in every pass instead of staging them.
 #include "lsa_internal.cuh"
 
 namespace lsa {
 namespace {
-
-constexpr int kTopkThreads = 1024;
 
 __device__ __forceinline__ uint32_t order_key(float z) {
     uint32_t b = __float_as_uint(z);
@@ -28,165 +19,16 @@ __device__ __forceinline__ uint32_t order_key(float z) {
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Exclusive block-wide prefix sum of one int per thread (1024 threads);
-// returns the exclusive prefix, writes the block total to *total.
-__device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int s = s_warp[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int y = __shfl_up_sync(0xffffffffu, s, o);
-            if (lane >= o) s += y;
-        }
-        s_warp[lane] = s;
-    }
-    __syncthreads();
-    const int res = (warp ? s_warp[warp - 1] : 0) + x - v;
-    *total = s_warp[31];
-    __syncthreads();
-    return res;
-}
-
-constexpr int kSmemKeys = 32768;   // keys staged in shared memory (128 KB)
-constexpr int kWarps = kTopkThreads / 32;
-
-__global__ void __launch_bounds__(kTopkThreads)
-topk_smem(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict__ seq_off,
-          const int32_t *__restrict__ kept_idx, const int64_t *__restrict__ kept_off, int64_t kept_cap, int k,
-          int32_t *__restrict__ topk_idx, int32_t *__restrict__ topk_pos, int32_t *__restrict__ topk_cnt,
-          int min_n) {
-    extern __shared__ uint32_t s_keys[];                 // [n]
-    __shared__ int s_hist[kWarps][256];
-    __shared__ int s_warp[32];
-    __shared__ uint32_t s_want;
-    __shared__ int s_kr;
-
-    const int b = blockIdx.x;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t p0 = kept_off[b];
-    int64_t n64 = kept_off[b + 1] - p0;
-    if (p0 >= kept_cap) n64 = 0;
-    else if (p0 + n64 > kept_cap) n64 = kept_cap - p0;
-    if (n64 < 0) n64 = 0;
-    const int n = int(n64);
-    if (n < min_n) return;   // handled by topk_reg
-    int32_t *out_idx = topk_idx + int64_t(b) * k;
-    int32_t *out_pos = topk_pos ? topk_pos + int64_t(b) * k : nullptr;
-
-    if (n <= k) {   // everything kept is chosen
-        for (int i = threadIdx.x; i < k; i += kTopkThreads) {
-            out_idx[i] = i < n ? kept_idx[p0 + i] : -1;
-            if (out_pos) out_pos[i] = i < n ? int32_t(p0 + i) : -1;
-        }
-        if (threadIdx.x == 0) topk_cnt[b] = n;
-        return;
-    }
-    const int64_t sbase = z_by_entry ? seq_off[b] : 0;
-    const bool staged = n <= kSmemKeys;
-    auto key = [&](int i) -> uint32_t {
-        return staged ? s_keys[i] : order_key(z_by_entry ? z[sbase + kept_idx[p0 + i]] : z[p0 + i]);
-    };
-    if (staged)
-        for (int i = threadIdx.x; i < n; i += kTopkThreads)
-            s_keys[i] = order_key(z_by_entry ? z[sbase + kept_idx[p0 + i]] : z[p0 + i]);
-
-    uint32_t want = 0, hmask = 0;
-    int kr = k;
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int i = lane; i < 256; i += 32) s_hist[warp][i] = 0;
-        __syncthreads();
-        for (int i0 = warp * 32; i0 < n; i0 += kTopkThreads) {
-            const int i = i0 + lane;
-            const uint32_t u = i < n ? key(i) : 0u;
-            const bool in = i < n && (u & hmask) == want;
-            const int digit = in ? int((u >> shift) & 0xFFu) : -1;
-            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-            if (in && (__ffs(peers) - 1) == lane) atomicAdd(&s_hist[warp][digit], __popc(peers));
-        }
-        __syncthreads();
-        if (threadIdx.x < 256) {   // fold the warp histograms into warp 0's row
-            int sum = 0;
-#pragma unroll 8
-            for (int w = 0; w < kWarps; ++w) sum += s_hist[w][threadIdx.x];
-            s_hist[0][threadIdx.x] = sum;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            int local = 0;
-#pragma unroll
-            for (int x = 0; x < 8; ++x) local += s_hist[0][8 * lane + x];
-            int suf = local;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_down_sync(0xffffffffu, suf, o);
-                if (lane + o < 32) suf += y;
-            }
-            int above = suf - local;
-#pragma unroll
-            for (int x = 7; x >= 0; --x) {
-                const int h = s_hist[0][8 * lane + x];
-                if (above < kr && above + h >= kr) {
-                    s_want = want | (uint32_t(8 * lane + x) << shift);
-                    s_kr = kr - above;
-                }
-                above += h;
-            }
-        }
-        __syncthreads();
-        want = s_want;
-        kr = s_kr;
-        hmask |= 0xFFu << shift;
-    }
-    // ordered take: thread t owns positions [t*per, (t+1)*per)
-    const int per = (n + kTopkThreads - 1) / kTopkThreads;
-    const int lo = min(n, threadIdx.x * per), hi = min(n, lo + per);
-    int n_eq = 0;
-    for (int i = lo; i < hi; ++i) n_eq += key(i) == want;
-    int tot;
-    int eq_rank = block_excl_scan(n_eq, s_warp, &tot);
-    int n_take = 0;
-    {
-        int r = eq_rank;
-        for (int i = lo; i < hi; ++i) {
-            const uint32_t u = key(i);
-            if (u > want) ++n_take;
-            else if (u == want) { n_take += r < kr; ++r; }
-        }
-    }
-    int out = block_excl_scan(n_take, s_warp, &tot);
-    {
-        int r = eq_rank;
-        for (int i = lo; i < hi; ++i) {
-            const uint32_t u = key(i);
-            bool take = u > want;
-            if (u == want) { take = r < kr; ++r; }
-            if (take && out < k) {
-                out_idx[out] = kept_idx[p0 + i];
-                if (out_pos) out_pos[out] = int32_t(p0 + i);
-                ++out;
-            }
-        }
-    }
-    if (threadIdx.x == 0) topk_cnt[b] = k;
-}
-
-// Register-resident variant for kept sets of up to kRegThreads * kKpt entries:
-// thread t owns the contiguous positions [t*kKpt, (t+1)*kKpt) and loads their
+// Kept sets of up to kRegThreads * kKpt entries live in registers: thread t owns the contiguous positions [t*kKpt, (t+1)*kKpt) and loads their
 // scores and entry indices in one unrolled batch (independent loads in flight
 // instead of a chain of dependent ones); the radix passes count from
 // registers into per-warp histograms; the ordered take needs two block scans
-// and writes each thread's run in order.  Larger kept sets fall back to the
-// shared-memory kernel above.
+// and writes each thread's run in order.  Lanes of a warp that hit the same
+// histogram bin are merged with __match_any_sync before one shared atomic
+// (kept scores cluster in a few leading-digit bins, so unmerged atomics would
+// serialise), and the select stops as soon as the threshold bin holds exactly
+// the entries still needed.  Larger kept sets run the same select reading the
+// keys from global memory (topk_large).
 constexpr int kRegThreads = 512;
 constexpr int kKpt = 48;
 constexpr int kRegWarps = kRegThreads / 32;
@@ -215,6 +57,90 @@ __device__ __forceinline__ int block_excl_scan512(int v, int *s_warp, int *total
     *total = s_warp[kRegWarps - 1];
     __syncthreads();
     return res;
+}
+
+// Kept sets too large for the registers: the same radix select, reading the
+// keys from global memory in every pass.
+__device__ void topk_large(const float *__restrict__ z, int z_by_entry, int64_t sbase,
+                           const int32_t *__restrict__ kept_idx, int64_t p0, int n, int k,
+                           int32_t *__restrict__ out_idx, int32_t *__restrict__ out_pos,
+                           int (*s_hist)[256], int *s_warp, uint32_t *s_want, int *s_kr) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    auto key_at = [&](int i) -> uint32_t {
+        return order_key(z_by_entry ? z[sbase + kept_idx[p0 + i]] : z[p0 + i]);
+    };
+    uint32_t want = 0, hmask = 0;
+    int kr = k;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int i = lane; i < 256; i += 32) s_hist[warp][i] = 0;
+        __syncthreads();
+        for (int i0 = 0; i0 < n; i0 += kRegThreads) {
+            const int i = i0 + int(threadIdx.x);
+            const uint32_t u = i < n ? key_at(i) : 0u;
+            const bool in = i < n && (u & hmask) == want;
+            const int digit = in ? int((u >> shift) & 0xFFu) : -1;
+            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+            if (in && (__ffs(peers) - 1) == lane) atomicAdd(&s_hist[warp][digit], __popc(peers));
+        }
+        __syncthreads();
+        if (threadIdx.x < 256) {
+            int sum = 0;
+            for (int w = 0; w < kRegWarps; ++w) sum += s_hist[w][threadIdx.x];
+            s_hist[0][threadIdx.x] = sum;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int local = 0;
+            for (int x = 0; x < 8; ++x) local += s_hist[0][8 * lane + x];
+            int suf = local;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_down_sync(0xffffffffu, suf, o);
+                if (lane + o < 32) suf += y;
+            }
+            int above = suf - local;
+            for (int x = 7; x >= 0; --x) {
+                const int h = s_hist[0][8 * lane + x];
+                if (above < kr && above + h >= kr) {
+                    *s_want = want | (uint32_t(8 * lane + x) << shift);
+                    *s_kr = kr - above;
+                }
+                above += h;
+            }
+        }
+        __syncthreads();
+        want = *s_want;
+        kr = *s_kr;
+        hmask |= 0xFFu << shift;
+        __syncthreads();
+    }
+    const int per = (n + kRegThreads - 1) / kRegThreads;
+    const int lo = min(n, int(threadIdx.x) * per), hi = min(n, lo + per);
+    int n_eq = 0;
+    for (int i = lo; i < hi; ++i) n_eq += key_at(i) == want;
+    int tot;
+    const int eq_rank = block_excl_scan512(n_eq, s_warp, &tot);
+    int n_take = 0;
+    {
+        int r = eq_rank;
+        for (int i = lo; i < hi; ++i) {
+            const uint32_t u = key_at(i);
+            if (u > want) ++n_take;
+            else if (u == want) { n_take += r < kr; ++r; }
+        }
+    }
+    int out = block_excl_scan512(n_take, s_warp, &tot);
+    int r = eq_rank;
+    for (int i = lo; i < hi; ++i) {
+        const uint32_t u = key_at(i);
+        bool take = u > want;
+        if (u == want) { take = r < kr; ++r; }
+        if (take && out < k) {
+            out_idx[out] = kept_idx[p0 + i];
+            if (out_pos) out_pos[out] = int32_t(p0 + i);
+            ++out;
+        }
+    }
 }
 
 __global__ void __launch_bounds__(kRegThreads)
@@ -247,7 +173,12 @@ topk_reg(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict_
         if (threadIdx.x == 0) topk_cnt[b] = n;
         return;
     }
-    if (n > kRegThreads * kKpt) return;   // left to the shared-memory kernel
+    if (n > kRegThreads * kKpt) {
+        topk_large(z, z_by_entry, z_by_entry ? seq_off[b] : 0, kept_idx, p0, n, k, out_idx, out_pos, s_hist, s_warp,
+                   &s_want, &s_kr);
+        if (threadIdx.x == 0) topk_cnt[b] = k;
+        return;
+    }
     const int lo = threadIdx.x * kKpt;
     int32_t ids[kKpt];
     uint32_t key[kKpt];
@@ -260,13 +191,20 @@ topk_reg(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict_
 
     uint32_t want = 0, hmask = 0;
     int kr = k;
+    __shared__ int s_done;
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
         for (int i = lane; i < 256; i += 32) s_hist[warp][i] = 0;
         __syncthreads();
+        // kept scores cluster in a few bins of the leading digits: lanes that hit the same bin are
+        // merged first, so a warp issues one shared atomic per distinct bin
 #pragma unroll
-        for (int j = 0; j < kKpt; ++j)
-            if (lo + j < n && (key[j] & hmask) == want) atomicAdd(&s_hist[warp][(key[j] >> shift) & 0xFFu], 1);
+        for (int j = 0; j < kKpt; ++j) {
+            const bool in = lo + j < n && (key[j] & hmask) == want;
+            const int digit = in ? int((key[j] >> shift) & 0xFFu) : -1;
+            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+            if (in && (__ffs(peers) - 1) == lane) atomicAdd(&s_hist[warp][digit], __popc(peers));
+        }
         __syncthreads();
         if (threadIdx.x < 256) {
             int sum = 0;
@@ -292,6 +230,7 @@ topk_reg(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict_
                 if (above < kr && above + h >= kr) {
                     s_want = want | (uint32_t(8 * lane + x) << shift);
                     s_kr = kr - above;
+                    s_done = (above + h == kr);   // the whole bin is taken: no finer digit needed
                 }
                 above += h;
             }
@@ -300,10 +239,13 @@ topk_reg(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict_
         want = s_want;
         kr = s_kr;
         hmask |= 0xFFu << shift;
+        if (s_done) break;
+        __syncthreads();
     }
+    // take every key whose resolved digits exceed `want`, and the first kr whose digits equal it
     int n_eq = 0;
 #pragma unroll
-    for (int j = 0; j < kKpt; ++j) n_eq += (lo + j < n && key[j] == want);
+    for (int j = 0; j < kKpt; ++j) n_eq += (lo + j < n && (key[j] & hmask) == want);
     int tot;
     const int eq_rank = block_excl_scan512(n_eq, s_warp, &tot);
     uint64_t take = 0;   // per-position take flags (kKpt <= 64)
@@ -314,8 +256,9 @@ topk_reg(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict_
         for (int j = 0; j < kKpt; ++j) {
             bool t = false;
             if (lo + j < n) {
-                if (key[j] > want) t = true;
-                else if (key[j] == want) { t = r < kr; ++r; }
+                const uint32_t kk = key[j] & hmask;
+                if (kk > want) t = true;
+                else if (kk == want) { t = r < kr; ++r; }
             }
             if (t) {
                 ++n_take;
@@ -349,13 +292,6 @@ lsa_status launch_topk(const float *z, int32_t z_by_entry, const int64_t *seq_of
     LSA_CUDA(launch_pdl(topk_reg, dim3(B), dim3(kRegThreads), 0, st, z, z_by_entry, seq_off, kept_idx, kept_off,
                         kept_cap, k, topk_idx, topk_pos, topk_cnt));
     LSA_LAUNCHED("topk_reg");
-    if (kept_cap > int64_t(kRegThreads) * kKpt) {
-        const size_t smem = size_t(kSmemKeys) * 4;
-        LSA_CUDA(ensure_smem(topk_smem, smem));
-        topk_smem<<<B, kTopkThreads, smem, st>>>(z, z_by_entry, seq_off, kept_idx, kept_off, kept_cap, k, topk_idx,
-                                                 topk_pos, topk_cnt, kRegThreads * kKpt + 1);
-        LSA_LAUNCHED("topk_smem");
-    }
     return LSA_OK;
 }
 
