@@ -20,7 +20,9 @@
 //   5. warp 4 issues O = P V (M = 128, N = 2 x 256, K = 128) into TMEM columns
 //      0..511, reading the SAME smem rows as V through an MN-major descriptor
 //      (no transpose, no second copy of the rows);
-//   6. warps 0-3 read O and write the fp32 partial (o, m, l) of the chunk.
+//   6. warps 0-3 read O in 64-column blocks into the freed row buffer
+//      (128-byte swizzle) and write the fp32 partial with TMA stores; (m, l)
+//      per head.
 // The combine kernel (attn.cu) merges the chunks.  Every wait is bounded.
 #include <cuda.h>
 
@@ -44,6 +46,7 @@ constexpr int kKvBytes = kRowsPerCta * kD * 2;   // 128 KB: 8 blocks of [128 row
 constexpr int kKvBlock = kRowsPerCta * 128;      // 16 KB
 constexpr int kQStageBytes = kHq * 128;          // 16 KB: one 64-column slice of Q
 constexpr int kPBytes = kHq * kRowsPerCta * 2;   // 32 KB: 2 blocks of [128 heads x 128 B]
+constexpr int kOStageBytes = kHq * 64 * 4;       // 32 KB: [128 heads][64 fp32] staging of one O block
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -64,9 +67,9 @@ __device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t addr, uint32_t lbo) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_tc(const __grid_constant__ CUtensorMap qmap, const uint16_t *__restrict__ kv, int64_t stride, int64_t k_off,
-        const int32_t *__restrict__ rows, int k, float scale, float *__restrict__ part_o,
-        float *__restrict__ part_ml, int32_t *err) {
+attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap omap,
+        const uint16_t *__restrict__ kv, int64_t stride, int64_t k_off, const int32_t *__restrict__ rows, int k,
+        float scale, float *__restrict__ part_ml, int32_t *err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *kvs = smem;                         // 128 KB
@@ -152,7 +155,8 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const uint16_t *__restrict__ k
         const int quarter = warp;   // warps 0-3 -> TMEM lanes 32*warp ..
         bool ok = mbar_wait(s_full, 0, abort_v, kWaitLimitNs);
         float m = -INFINITY, l = 0.f;
-        if (__all_sync(0xffffffffu, ok)) {
+        // warps 0-3 take every branch below together (they meet at named barriers)
+        if (named_barrier_and(1, 128, ok)) {
             tc_fence_after();
             uint32_t sr[kRowsPerCta];
             const uint32_t taddr = tmem + (uint32_t(quarter * 32) << 16);
@@ -187,24 +191,44 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const uint16_t *__restrict__ k
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(p_full);
-            // ---- 6. read O and write the chunk's partial
+            // ---- 6. read O and write the chunk's partial: 64-column blocks staged in the (now free)
+            // row buffer, one TMA store per block; two staging buffers alternate
             ok = mbar_wait(o_full, 0, abort_v, kWaitLimitNs);
-            if (__all_sync(0xffffffffu, ok)) {
+            // the block loop below synchronises these 128 threads: agree on one outcome first
+            if (named_barrier_and(1, 128, ok)) {
                 tc_fence_after();
-                float *dst = part_o + (pbase + t) * kD;
 #pragma unroll 1
-                for (int c = 0; c < kD / 64; ++c) {   // 64 columns per wait
+                for (int c = 0; c < kD / 64; ++c) {
+                    float *sb = reinterpret_cast<float *>(kvs + (c & 1) * kOStageBytes);   // 2 x [128][32]
+                    if (c >= 2) {
+                        if (t == 0) bulk_wait_read<1>();   // the store issued two blocks ago has read its buffer
+                        named_barrier(1, 128);
+                    }
                     uint32_t o[64];
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
                         tmem_ld_32x32b_x16(taddr + c * 64 + q4 * 16, *reinterpret_cast<uint32_t(*)[16]>(&o[q4 * 16]));
                     tmem_ld_wait();
+                    // two [128 rows x 32 fp32] halves in the 128-byte-swizzled layout (16-byte chunk
+                    // u of row t at chunk u ^ (t % 8)): conflict-free writes, one TMA store per half
 #pragma unroll
-                    for (int u = 0; u < 64; u += 4)
-                        *reinterpret_cast<float4 *>(dst + c * 64 + u) =
-                            make_float4(__uint_as_float(o[u]), __uint_as_float(o[u + 1]),
-                                        __uint_as_float(o[u + 2]), __uint_as_float(o[u + 3]));
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            *reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(sb) + h * 16384 + t * 128 +
+                                                        ((u ^ (t & 7)) << 4)) =
+                                make_float4(__uint_as_float(o[h * 32 + 4 * u]), __uint_as_float(o[h * 32 + 4 * u + 1]),
+                                            __uint_as_float(o[h * 32 + 4 * u + 2]),
+                                            __uint_as_float(o[h * 32 + 4 * u + 3]));
+                    fence_proxy_async_smem();
+                    named_barrier(1, 128);
+                    if (t == 0) {
+                        tma_store_2d(&omap, sb, c * 64, int(pbase));
+                        tma_store_2d(&omap, reinterpret_cast<uint8_t *>(sb) + 16384, c * 64 + 32, int(pbase));
+                        bulk_commit();
+                    }
                 }
+                if (t == 0) bulk_wait_all();
                 part_ml[(pbase + t) * 2] = m;
                 part_ml[(pbase + t) * 2 + 1] = l;
             }
@@ -323,10 +347,22 @@ lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, 
         set_error("lsa_sparse_attn: cuTensorMapEncodeTiled failed (%d)", int(r));
         return LSA_ERR_CUDA;
     }
+    CUtensorMap omap;   // partial O [B * nchunks * 128 rows, 512] fp32, stored in swizzled [128 x 32] boxes
+    const int nchunks_o = (k + kRowsPerCta - 1) / kRowsPerCta;
+    const cuuint64_t odims[2] = {cuuint64_t(kD), cuuint64_t(B) * nchunks_o * kHq};
+    const cuuint64_t ostrides[1] = {cuuint64_t(kD) * 4};
+    const cuuint32_t obox[2] = {32, 128};
+    r = enc(&omap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, part_o, odims, ostrides, obox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("lsa_sparse_attn: cuTensorMapEncodeTiled (partials) failed (%d)", int(r));
+        return LSA_ERR_CUDA;
+    }
     LSA_CUDA(ensure_smem(attn_tc, size_t(int(kSmemBytes))));
     const int nchunks = (k + kRowsPerCta - 1) / kRowsPerCta;
-    LSA_CUDA(launch_pdl(attn_tc, dim3(nchunks, B), dim3(kThreads), kSmemBytes, st, qmap,
-                        static_cast<const uint16_t *>(kv), stride, k_off, rows, k, scale, part_o, part_ml, err));
+    LSA_CUDA(launch_pdl(attn_tc, dim3(nchunks, B), dim3(kThreads), kSmemBytes, st, qmap, omap,
+                        static_cast<const uint16_t *>(kv), stride, k_off, rows, k, scale, part_ml, err));
     LSA_LAUNCHED("attn_tc");
     return LSA_OK;
 }

@@ -4,7 +4,7 @@
 //
 // One 512-thread block per sequence.  Scores map to an order-preserving 32-bit
 // key (larger z -> larger key, -0.0 folded onto +0.0).  A most-significant-
-// digit radix select (up to 4 passes of 8 bits) finds the digits of the k-th
+// digit radix select (passes of 8 bits) finds the digits of the k-th
 // largest key and how many entries sharing them must be taken; an ordered pass
 // then takes every key above and the lowest-index entries at the threshold,
 // and compacts them in kept-list order, which is ascending entry order.
@@ -19,21 +19,12 @@ __device__ __forceinline__ uint32_t order_key(float z) {
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Kept sets of up to kRegThreads * kKpt entries live in registers: thread t owns the contiguous positions [t*kKpt, (t+1)*kKpt) and loads their
-// scores and entry indices in one unrolled batch (independent loads in flight
-// instead of a chain of dependent ones); the radix passes count from
-// registers into per-warp histograms; the ordered take needs two block scans
-// and writes each thread's run in order.  Lanes of a warp that hit the same
-// histogram bin are merged with __match_any_sync before one shared atomic
-// (kept scores cluster in a few leading-digit bins, so unmerged atomics would
-// serialise), and the select stops as soon as the threshold bin holds exactly
-// the entries still needed.  Larger kept sets run the same select reading the
-// keys from global memory (topk_large).
-constexpr int kRegThreads = 512;
-constexpr int kKpt = 48;
-constexpr int kRegWarps = kRegThreads / 32;
+// Block-wide reductions for 512 threads.
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kSmemKeys = 40960;   // keys staged in shared memory (160 KB)
 
-__device__ __forceinline__ int block_excl_scan512(int v, int *s_warp, int *total) {
+__device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
 #pragma unroll
@@ -44,113 +35,39 @@ __device__ __forceinline__ int block_excl_scan512(int v, int *s_warp, int *total
     if (lane == 31) s_warp[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int s = lane < kRegWarps ? s_warp[lane] : 0;
+        int s = lane < kWarps ? s_warp[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, s, o);
             if (lane >= o) s += y;
         }
-        if (lane < kRegWarps) s_warp[lane] = s;
+        if (lane < kWarps) s_warp[lane] = s;
     }
     __syncthreads();
     const int res = (warp ? s_warp[warp - 1] : 0) + x - v;
-    *total = s_warp[kRegWarps - 1];
+    *total = s_warp[kWarps - 1];
     __syncthreads();
     return res;
 }
 
-// Kept sets too large for the registers: the same radix select, reading the
-// keys from global memory in every pass.
-__device__ void topk_large(const float *__restrict__ z, int z_by_entry, int64_t sbase,
-                           const int32_t *__restrict__ kept_idx, int64_t p0, int n, int k,
-                           int32_t *__restrict__ out_idx, int32_t *__restrict__ out_pos,
-                           int (*s_hist)[256], int *s_warp, uint32_t *s_want, int *s_kr) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    auto key_at = [&](int i) -> uint32_t {
-        return order_key(z_by_entry ? z[sbase + kept_idx[p0 + i]] : z[p0 + i]);
-    };
-    uint32_t want = 0, hmask = 0;
-    int kr = k;
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int i = lane; i < 256; i += 32) s_hist[warp][i] = 0;
-        __syncthreads();
-        for (int i0 = 0; i0 < n; i0 += kRegThreads) {
-            const int i = i0 + int(threadIdx.x);
-            const uint32_t u = i < n ? key_at(i) : 0u;
-            const bool in = i < n && (u & hmask) == want;
-            const int digit = in ? int((u >> shift) & 0xFFu) : -1;
-            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-            if (in && (__ffs(peers) - 1) == lane) atomicAdd(&s_hist[warp][digit], __popc(peers));
-        }
-        __syncthreads();
-        if (threadIdx.x < 256) {
-            int sum = 0;
-            for (int w = 0; w < kRegWarps; ++w) sum += s_hist[w][threadIdx.x];
-            s_hist[0][threadIdx.x] = sum;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            int local = 0;
-            for (int x = 0; x < 8; ++x) local += s_hist[0][8 * lane + x];
-            int suf = local;
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_down_sync(0xffffffffu, suf, o);
-                if (lane + o < 32) suf += y;
-            }
-            int above = suf - local;
-            for (int x = 7; x >= 0; --x) {
-                const int h = s_hist[0][8 * lane + x];
-                if (above < kr && above + h >= kr) {
-                    *s_want = want | (uint32_t(8 * lane + x) << shift);
-                    *s_kr = kr - above;
-                }
-                above += h;
-            }
-        }
-        __syncthreads();
-        want = *s_want;
-        kr = *s_kr;
-        hmask |= 0xFFu << shift;
-        __syncthreads();
-    }
-    const int per = (n + kRegThreads - 1) / kRegThreads;
-    const int lo = min(n, int(threadIdx.x) * per), hi = min(n, lo + per);
-    int n_eq = 0;
-    for (int i = lo; i < hi; ++i) n_eq += key_at(i) == want;
-    int tot;
-    const int eq_rank = block_excl_scan512(n_eq, s_warp, &tot);
-    int n_take = 0;
-    {
-        int r = eq_rank;
-        for (int i = lo; i < hi; ++i) {
-            const uint32_t u = key_at(i);
-            if (u > want) ++n_take;
-            else if (u == want) { n_take += r < kr; ++r; }
-        }
-    }
-    int out = block_excl_scan512(n_take, s_warp, &tot);
-    int r = eq_rank;
-    for (int i = lo; i < hi; ++i) {
-        const uint32_t u = key_at(i);
-        bool take = u > want;
-        if (u == want) { take = r < kr; ++r; }
-        if (take && out < k) {
-            out_idx[out] = kept_idx[p0 + i];
-            if (out_pos) out_pos[out] = int32_t(p0 + i);
-            ++out;
-        }
-    }
-}
-
-__global__ void __launch_bounds__(kRegThreads)
-topk_reg(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict__ seq_off,
-         const int32_t *__restrict__ kept_idx, const int64_t *__restrict__ kept_off, int64_t kept_cap, int k,
-         int32_t *__restrict__ topk_idx, int32_t *__restrict__ topk_pos, int32_t *__restrict__ topk_cnt) {
-    __shared__ int s_hist[kRegWarps][256];
+// Kept sets of up to kSmemKeys entries are staged once in shared memory with
+// batched (independent) loads; larger ones re-read the scores from global
+// memory in every pass.  The radix digits start below the bits that every key
+// shares (the common prefix of the block's min and max key): kept scores sit
+// in a narrow positive range, so the leading bits are constant and a digit
+// there would say nothing while funnelling every key into one histogram bin.
+// Each warp counts into its own 256-bin histogram; each thread walks its own
+// contiguous run of positions, so the final ordered take needs two block scans.
+__global__ void __launch_bounds__(kThreads)
+topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict__ seq_off,
+            const int32_t *__restrict__ kept_idx, const int64_t *__restrict__ kept_off, int64_t kept_cap, int k,
+            int32_t *__restrict__ topk_idx, int32_t *__restrict__ topk_pos, int32_t *__restrict__ topk_cnt) {
+    extern __shared__ uint32_t s_keys[];
+    __shared__ int s_hist[kWarps][256];
     __shared__ int s_warp[32];
+    __shared__ uint32_t s_red[2][kWarps];
     __shared__ uint32_t s_want;
-    __shared__ int s_kr;
+    __shared__ int s_kr, s_done;
 
     pdl_launch_dependents();   // attention may stage its queries meanwhile
     pdl_wait();                // scores come from the preceding scan
@@ -165,51 +82,76 @@ topk_reg(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict_
     int32_t *out_idx = topk_idx + int64_t(b) * k;
     int32_t *out_pos = topk_pos ? topk_pos + int64_t(b) * k : nullptr;
 
-    if (n <= k) {
-        for (int i = threadIdx.x; i < k; i += kRegThreads) {
+    if (n <= k) {   // everything kept is chosen
+        for (int i = threadIdx.x; i < k; i += kThreads) {
             out_idx[i] = i < n ? kept_idx[p0 + i] : -1;
             if (out_pos) out_pos[i] = i < n ? int32_t(p0 + i) : -1;
         }
         if (threadIdx.x == 0) topk_cnt[b] = n;
         return;
     }
-    if (n > kRegThreads * kKpt) {
-        topk_large(z, z_by_entry, z_by_entry ? seq_off[b] : 0, kept_idx, p0, n, k, out_idx, out_pos, s_hist, s_warp,
-                   &s_want, &s_kr);
-        if (threadIdx.x == 0) topk_cnt[b] = k;
-        return;
-    }
-    const int lo = threadIdx.x * kKpt;
-    int32_t ids[kKpt];
-    uint32_t key[kKpt];
-#pragma unroll
-    for (int j = 0; j < kKpt; ++j) ids[j] = lo + j < n ? kept_idx[p0 + lo + j] : 0;
     const int64_t sbase = z_by_entry ? seq_off[b] : 0;
-#pragma unroll
-    for (int j = 0; j < kKpt; ++j)
-        key[j] = lo + j < n ? order_key(z_by_entry ? z[sbase + ids[j]] : z[p0 + lo + j]) : 0u;
+    const bool staged = n <= kSmemKeys;
+    auto load_key = [&](int i) -> uint32_t {
+        return order_key(z_by_entry ? z[sbase + kept_idx[p0 + i]] : z[p0 + i]);
+    };
+    auto key = [&](int i) -> uint32_t { return staged ? s_keys[i] : load_key(i); };
 
-    uint32_t want = 0, hmask = 0;
+    // thread t owns positions [lo, hi)
+    const int per = (n + kThreads - 1) / kThreads;
+    const int lo = min(n, int(threadIdx.x) * per), hi = min(n, lo + per);
+
+    // stage (8 loads in flight per thread) and reduce min / max
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int i0 = lo; i0 < hi; i0 += 8) {
+        uint32_t v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = i0 + u < hi ? load_key(i0 + u) : 0u;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (i0 + u < hi) {
+                if (staged) s_keys[i0 + u] = v[u];
+                kmin = min(kmin, v[u]);
+                kmax = max(kmax, v[u]);
+            }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    if (lane == 0) { s_red[0][warp] = kmin; s_red[1][warp] = kmax; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t a = 0xFFFFFFFFu, c = 0u;
+        for (int w = 0; w < kWarps; ++w) { a = min(a, s_red[0][w]); c = max(c, s_red[1][w]); }
+        s_red[0][0] = a;
+        s_red[1][0] = c;
+    }
+    __syncthreads();
+    const uint32_t diff = s_red[0][0] ^ s_red[1][0];
+    // bits above `top` are shared by every key
+    int top = diff ? 31 - __clz(diff) : -1;
+
+    uint32_t want = top >= 0 ? (s_red[0][0] & ~((2u << top) - 1u)) : s_red[0][0];
+    uint32_t hmask = top >= 0 ? ~((2u << top) - 1u) : 0xFFFFFFFFu;
+    if (top == 31) { want = 0; hmask = 0; }
     int kr = k;
-    __shared__ int s_done;
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
+    while (top >= 0) {
+        const int width = top + 1 < 8 ? top + 1 : 8;
+        const int shift = top + 1 - width;
+        const uint32_t dmask = (1u << width) - 1u;
         for (int i = lane; i < 256; i += 32) s_hist[warp][i] = 0;
         __syncthreads();
-        // kept scores cluster in a few bins of the leading digits: lanes that hit the same bin are
-        // merged first, so a warp issues one shared atomic per distinct bin
-#pragma unroll
-        for (int j = 0; j < kKpt; ++j) {
-            const bool in = lo + j < n && (key[j] & hmask) == want;
-            const int digit = in ? int((key[j] >> shift) & 0xFFu) : -1;
-            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-            if (in && (__ffs(peers) - 1) == lane) atomicAdd(&s_hist[warp][digit], __popc(peers));
+        for (int i = lo; i < hi; ++i) {
+            const uint32_t u = key(i);
+            if ((u & hmask) == want) atomicAdd(&s_hist[warp][(u >> shift) & dmask], 1);
         }
         __syncthreads();
         if (threadIdx.x < 256) {
             int sum = 0;
 #pragma unroll
-            for (int w = 0; w < kRegWarps; ++w) sum += s_hist[w][threadIdx.x];
+            for (int w = 0; w < kWarps; ++w) sum += s_hist[w][threadIdx.x];
             s_hist[0][threadIdx.x] = sum;
         }
         __syncthreads();
@@ -230,7 +172,7 @@ topk_reg(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict_
                 if (above < kr && above + h >= kr) {
                     s_want = want | (uint32_t(8 * lane + x) << shift);
                     s_kr = kr - above;
-                    s_done = (above + h == kr);   // the whole bin is taken: no finer digit needed
+                    s_done = (above + h == kr);   // the whole bin is taken
                 }
                 above += h;
             }
@@ -238,41 +180,35 @@ topk_reg(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict_
         __syncthreads();
         want = s_want;
         kr = s_kr;
-        hmask |= 0xFFu << shift;
+        hmask |= dmask << shift;
+        top = shift - 1;
         if (s_done) break;
         __syncthreads();
     }
-    // take every key whose resolved digits exceed `want`, and the first kr whose digits equal it
+    // take every key whose resolved bits exceed `want`, and the first kr equal to it
     int n_eq = 0;
-#pragma unroll
-    for (int j = 0; j < kKpt; ++j) n_eq += (lo + j < n && (key[j] & hmask) == want);
+    for (int i = lo; i < hi; ++i) n_eq += (key(i) & hmask) == want;
     int tot;
-    const int eq_rank = block_excl_scan512(n_eq, s_warp, &tot);
-    uint64_t take = 0;   // per-position take flags (kKpt <= 64)
+    const int eq_rank = block_excl_scan(n_eq, s_warp, &tot);
     int n_take = 0;
     {
         int r = eq_rank;
-#pragma unroll
-        for (int j = 0; j < kKpt; ++j) {
-            bool t = false;
-            if (lo + j < n) {
-                const uint32_t kk = key[j] & hmask;
-                if (kk > want) t = true;
-                else if (kk == want) { t = r < kr; ++r; }
-            }
-            if (t) {
-                ++n_take;
-                take |= uint64_t(1) << j;
-            }
+        for (int i = lo; i < hi; ++i) {
+            const uint32_t u = key(i) & hmask;
+            if (u > want) ++n_take;
+            else if (u == want) { n_take += r < kr; ++r; }
         }
     }
-    int out = block_excl_scan512(n_take, s_warp, &tot);
-#pragma unroll
-    for (int j = 0; j < kKpt; ++j) {
-        if ((take >> j) & 1u) {
+    int out = block_excl_scan(n_take, s_warp, &tot);
+    int r = eq_rank;
+    for (int i = lo; i < hi; ++i) {
+        const uint32_t u = key(i) & hmask;
+        bool take = u > want;
+        if (u == want) { take = r < kr; ++r; }
+        if (take) {
             if (out < k) {
-                out_idx[out] = ids[j];
-                if (out_pos) out_pos[out] = int32_t(p0 + lo + j);
+                out_idx[out] = kept_idx[p0 + i];
+                if (out_pos) out_pos[out] = int32_t(p0 + i);
             }
             ++out;
         }
@@ -286,12 +222,11 @@ lsa_status launch_topk(const float *z, int32_t z_by_entry, const int64_t *seq_of
                        const int32_t *kept_idx, const int64_t *kept_off, int32_t B, int32_t k,
                        int64_t kept_cap, int32_t *topk_idx, int32_t *topk_pos, int32_t *topk_cnt,
                        cudaStream_t st) {
-    // sequences whose kept set fits in registers (all of them at the decode step's shapes unless a
-    // sequence keeps more than 24576 entries) are done by topk_reg; the shared-memory kernel runs only
-    // when the kept capacity allows a larger set, and then only for such sequences.
-    LSA_CUDA(launch_pdl(topk_reg, dim3(B), dim3(kRegThreads), 0, st, z, z_by_entry, seq_off, kept_idx, kept_off,
+    const size_t smem = size_t(kSmemKeys) * 4;
+    LSA_CUDA(ensure_smem(topk_select, smem));
+    LSA_CUDA(launch_pdl(topk_select, dim3(B), dim3(kThreads), smem, st, z, z_by_entry, seq_off, kept_idx, kept_off,
                         kept_cap, k, topk_idx, topk_pos, topk_cnt));
-    LSA_LAUNCHED("topk_reg");
+    LSA_LAUNCHED("topk_select");
     return LSA_OK;
 }
 
