@@ -23,7 +23,6 @@ constexpr int kChunk = 64;          // selected rows per block
 constexpr int kHeads = 16;          // query heads per block
 constexpr int kAttnThreads = 256;   // 8 warps, 2 heads each
 constexpr int kMaxColsPerLane = 16; // D <= 512
-constexpr int kMaxChunks = 64;      // k <= 4096 rows in chunks of kChunk
 
 template <typename T>
 struct Elem;
@@ -149,53 +148,48 @@ attn_partial(const T *__restrict__ Q, const T *__restrict__ kv, int64_t stride, 
 // Merge of the chunk partials of one (head, sequence):
 //   M = max_c m_c,  w_c = e^{m_c - M},  L = sum_c l_c w_c,  o = sum_c w_c o_c / L,
 //   lse = M + log L;  a chunk with m_c = -inf (no selected row) has weight 0.
+// Every thread loads the (m, l) of all chunks and its four columns of every
+// chunk in batches of up to 16 independent loads, then reduces on its own (the
+// (m, l) are the same for the whole block), so no block synchronisation sits
+// between the loads and the arithmetic.
 template <typename T>
 __global__ void __launch_bounds__(128)
 attn_combine(const float *__restrict__ part_o, const float *__restrict__ part_ml, int nchunks, int Hq, int D,
              T *__restrict__ out, float *__restrict__ lse) {
-    __shared__ float s_w[kMaxChunks];
-    __shared__ float s_ML[2];
+    constexpr int kBatch = 16;
     pdl_wait();   // partials come from the preceding kernel
     const int h = blockIdx.x, b = blockIdx.y;
     const int64_t p0 = int64_t(b) * nchunks * Hq + h;   // partial index of chunk 0; chunk c adds c * Hq
-    if (threadIdx.x < 32) {
-        float M = -INFINITY;
-        for (int c = threadIdx.x; c < nchunks; c += 32) M = fmaxf(M, part_ml[(p0 + int64_t(c) * Hq) * 2]);
-#pragma unroll
-        for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float L = 0.f;
-        for (int c = threadIdx.x; c < nchunks; c += 32) {
+    float M = -INFINITY;
+    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, part_ml[(p0 + int64_t(c) * Hq) * 2]);
+    float L = 0.f;
+    if (M != -INFINITY)
+        for (int c = 0; c < nchunks; ++c) {
             const float m = part_ml[(p0 + int64_t(c) * Hq) * 2];
-            const float w = (m == -INFINITY) ? 0.f : expf(m - M);
-            s_w[c] = w;
-            L += w * part_ml[(p0 + int64_t(c) * Hq) * 2 + 1];
+            if (m != -INFINITY) L += part_ml[(p0 + int64_t(c) * Hq) * 2 + 1] * expf(m - M);
         }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-        if (threadIdx.x == 0) { s_ML[0] = M; s_ML[1] = L; }
-    }
-    __syncthreads();
-    const float M = s_ML[0], L = s_ML[1];
     const float inv = M == -INFINITY ? 0.f : 1.f / L;
     const int64_t ob = (int64_t(b) * Hq + h) * D;
     for (int col = 4 * threadIdx.x; col < D; col += 4 * blockDim.x) {
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
         if (M != -INFINITY)
-            for (int c0 = 0; c0 < nchunks; c0 += 4) {   // four independent loads in flight
-                float4 v[4];
-                float w[4];
+            for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
+                float4 v[kBatch];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < kBatch; ++u) {
                     const int c = c0 + u;
-                    w[u] = c < nchunks ? s_w[c] : 0.f;
-                    v[u] = w[u] != 0.f
-                               ? *reinterpret_cast<const float4 *>(part_o + (p0 + int64_t(c) * Hq) * D + col)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[u] = c < nchunks ? *reinterpret_cast<const float4 *>(part_o + (p0 + int64_t(c) * Hq) * D + col)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    a.x = fmaf(w[u], v[u].x, a.x); a.y = fmaf(w[u], v[u].y, a.y);
-                    a.z = fmaf(w[u], v[u].z, a.z); a.w = fmaf(w[u], v[u].w, a.w);
+                for (int u = 0; u < kBatch; ++u) {
+                    const int c = c0 + u;
+                    if (c >= nchunks) break;
+                    const float m = part_ml[(p0 + int64_t(c) * Hq) * 2];
+                    if (m == -INFINITY) continue;   // an empty chunk's o is never read into the sum
+                    const float w = expf(m - M);
+                    a.x = fmaf(w, v[u].x, a.x); a.y = fmaf(w, v[u].y, a.y);
+                    a.z = fmaf(w, v[u].z, a.z); a.w = fmaf(w, v[u].w, a.w);
                 }
             }
         Elem<T>::put(out, ob + col, a.x * inv);

@@ -154,7 +154,8 @@ def _topk_gpu(lsa, z, z_by_entry, seq_off, kept, ko, k, cap=None):
 @pytest.mark.parametrize("ties", [False, True])
 def test_topk_stage_exact(lsa, k, ties):
     rng = np.random.default_rng(k + 1000 * ties)
-    lens = [0, 5, 40, 999, 4096, 20000, 2048, 2049, 50000]   # the last keeps > 32768: unstaged keys
+    # the last two keep ~40K and ~144K entries: keys re-read from global memory, runs longer than 64
+    lens = [0, 5, 40, 999, 4096, 20000, 2048, 2049, 50000, 180000]
     seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
     n = int(seq_off[-1])
     z = rng.normal(size=n).astype(np.float32)
