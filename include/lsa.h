@@ -215,7 +215,10 @@ lsa_status lsa_sparse_attn(const void *Q, lsa_dtype dtype, const void *kv, int64
  *
  * At a refresh step (t % tau == 0): full index scan, selection, cold-pool
  * fetch of the kept rows (on the context's side stream), top-k over the scan's
- * scores, attention.  At every other step the kept set and hot buffer stay as
+ * scores, attention.  By default the hot buffer is a cache: a kept entry whose
+ * row is already resident keeps its slot and only the others cross the host
+ * link (rows no longer kept stay resident until their slot is reused).  The
+ * cold pool must not change while the context lives.  At every other step the kept set and hot buffer stay as
  * they are; the kept entries are re-scored with that step's indexer query
  * (listed scan), then top-k and attention.
  * ---------------------------------------------------------------------- */
@@ -236,6 +239,9 @@ typedef struct lsa_params {
     int64_t kv_row_stride;       /* elements per row (row_bytes / element size) */
     int64_t k_off, v_off;        /* element offsets of K and V inside a row */
     int64_t kept_capacity;       /* hot-buffer rows = max kept entries over the batch */
+    int32_t full_fetch;          /* 0: the hot buffer caches rows across refreshes and a refresh
+                                    fetches only entries not resident; nonzero: every refresh
+                                    fetches every kept row (lsa_gather) into kept order */
 } lsa_params;
 
 typedef struct lsa_ctx lsa_ctx;
@@ -264,12 +270,15 @@ typedef struct lsa_ctx_view {
     float *z_kept;       /* [kept_capacity] listed-scan scores of the last step */
     int32_t *kept_idx;   /* [kept_capacity] */
     int64_t *kept_off;   /* [B+1] */
-    int32_t *slot_of;    /* [n_total] */
+    int32_t *slot_of;    /* [n_total] hot slot of each entry, or -1 */
     void *hot;           /* [kept_capacity, row_bytes] */
     int32_t *topk_idx;   /* [B, topk] */
-    int32_t *topk_pos;   /* [B, topk] */
+    int32_t *topk_pos;   /* [B, topk] hot slot of each chosen entry, -1 padded */
     int32_t *topk_cnt;   /* [B] */
     int32_t *err;        /* device error word of the context */
+    int32_t *kept_slot;  /* [kept_capacity] hot slot of each kept position (NULL with full_fetch) */
+    int32_t *owner;      /* [kept_capacity] entry held by each hot slot, or -1 */
+    int64_t *fetched;    /* rows fetched from the cold pool by the last refresh */
 } lsa_ctx_view;
 lsa_status lsa_ctx_get_view(lsa_ctx *ctx, lsa_ctx_view *view);
 

@@ -139,7 +139,7 @@ lsa_status lsa_topk(const float *z, int32_t z_by_entry, const int64_t *seq_off,
     LSA_CHECK_ARG(B >= 1, "lsa_topk: B=%d", B);
     LSA_CHECK_SUPPORTED(k >= 1 && k <= 4096, "lsa_topk: k=%d not in [1, 4096]", k);
     LSA_CHECK_ARG(kept_capacity >= 0, "lsa_topk: kept_capacity < 0");
-    return launch_topk(z, z_by_entry, seq_off, kept_idx, kept_off, B, k, kept_capacity, topk_idx,
+    return launch_topk(z, z_by_entry, seq_off, kept_idx, kept_off, B, k, kept_capacity, nullptr, topk_idx,
                        topk_pos, topk_cnt, as_stream(stream));
 }
 

@@ -6,8 +6,9 @@
 // attention).
 //
 // Refresh step (t % tau == 0):  score (full scan) -> select -> [side stream:
-// gather kept rows cold pool -> HBM] -> top-k over the scan's scores ->
-// wait for the gather -> attention over the hot buffer.
+// fetch the newly kept rows cold pool -> HBM (fetch.cu; or every kept row with
+// full_fetch)] -> top-k over the scan's scores -> wait for the fetch ->
+// attention over the hot buffer.
 // Other steps: listed re-score of the kept set with the step's indexer query
 // -> top-k -> attention.  The host never waits inside a step.
 //
@@ -60,6 +61,12 @@ struct lsa_ctx {
     void *hot = nullptr;
     int32_t *topk_idx = nullptr, *topk_pos = nullptr, *topk_cnt = nullptr;
     int32_t *err = nullptr;
+    // hot-buffer cache (incremental fetch)
+    int32_t *owner = nullptr;       // [cap] entry held by each slot, or -1
+    int32_t *kept_slot = nullptr;   // [cap] hot slot of each kept position
+    int64_t *fetched = nullptr;     // rows fetched by the last refresh
+    void *fetch_ws = nullptr;
+    cudaEvent_t ev_assign = nullptr;
     void *sel_ws = nullptr;
     size_t sel_ws_bytes = 0;
     void *attn_ws = nullptr;
@@ -94,11 +101,13 @@ using namespace lsa;
 void free_all(lsa_ctx *c) {
     void *bufs[] = {c->seq_off_d, c->z, c->z_kept, c->kept_idx, c->kept_off, c->slot_of, c->hot,
                     c->topk_idx, c->topk_pos, c->topk_cnt, c->err, c->sel_ws, c->attn_ws, c->score_ws,
+                    c->owner, c->kept_slot, c->fetched, c->fetch_ws,
                     c->q_d, c->Q_d, c->out_d, c->w_d, c->lse_d};
     for (void *b : bufs)
         if (b) cudaFree(b);
     if (c->ev_sel) cudaEventDestroy(c->ev_sel);
     if (c->ev_gather) cudaEventDestroy(c->ev_gather);
+    if (c->ev_assign) cudaEventDestroy(c->ev_assign);
     for (auto &pe : c->pending) { cudaEventDestroy(pe.a); cudaEventDestroy(pe.b); }
     for (auto e : c->free_events) cudaEventDestroy(e);
     for (auto &g : c->graphs) cudaGraphExecDestroy(g.second.exec);
@@ -173,13 +182,21 @@ lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w,
         LSA_CUDA(cudaEventRecord(c->ev_sel, st));
         LSA_CUDA(cudaStreamWaitEvent(c->side, c->ev_sel, 0));
         StageTimer tg(c, LSA_STAGE_GATHER, c->side);
-        LSA_TRY(launch_gather(c->cold_dev, p.row_bytes, c->seq_off_d, p.n_total, c->kept_idx,
-                              c->kept_off, p.B, c->hot, cap, c->slot_of, c->err, c->side));
+        if (p.full_fetch) {
+            LSA_TRY(launch_gather(c->cold_dev, p.row_bytes, c->seq_off_d, p.n_total, c->kept_idx, c->kept_off, p.B,
+                                  c->hot, cap, c->slot_of, c->err, c->side));
+        } else {
+            LSA_TRY(launch_fetch(c->cold_dev, p.row_bytes, c->seq_off_d, c->kept_idx, c->kept_off, p.B, c->hot, cap,
+                                 c->slot_of, c->owner, c->kept_slot, c->fetched, c->fetch_ws, c->err, c->ev_assign,
+                                 c->side));
+        }
         tg.done();
         LSA_CUDA(cudaEventRecord(c->ev_gather, c->side));
+        // the top-k writes hot slots: with the cache it needs the slot assignment first
+        if (!p.full_fetch) LSA_CUDA(cudaStreamWaitEvent(st, c->ev_assign, 0));
         StageTimer tk(c, LSA_STAGE_TOPK, st);
         LSA_TRY(launch_topk(c->z, 1, c->seq_off_d, c->kept_idx, c->kept_off, p.B, p.topk, cap,
-                            c->topk_idx, c->topk_pos, c->topk_cnt, st));
+                            p.full_fetch ? nullptr : c->kept_slot, c->topk_idx, c->topk_pos, c->topk_cnt, st));
         tk.done();
         LSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
     } else {
@@ -190,7 +207,7 @@ lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w,
         tr.done();
         StageTimer tk(c, LSA_STAGE_TOPK, st);
         LSA_TRY(launch_topk(c->z_kept, 0, c->seq_off_d, c->kept_idx, c->kept_off, p.B, p.topk, cap,
-                            c->topk_idx, c->topk_pos, c->topk_cnt, st));
+                            p.full_fetch ? nullptr : c->kept_slot, c->topk_idx, c->topk_pos, c->topk_cnt, st));
         tk.done();
     }
     StageTimer ta(c, LSA_STAGE_ATTN, st);
@@ -313,6 +330,10 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     LSA_ALLOC(c->sel_ws, c->sel_ws_bytes);
     LSA_ALLOC(c->attn_ws, c->attn_ws_bytes);
     LSA_ALLOC(c->score_ws, c->score_ws_bytes);
+    LSA_ALLOC(c->owner, size_t(cap) * 4);
+    LSA_ALLOC(c->kept_slot, size_t(cap) * 4);
+    LSA_ALLOC(c->fetched, 16);
+    LSA_ALLOC(c->fetch_ws, fetch_workspace(cap));
     LSA_ALLOC(c->q_d, qbytes);
     LSA_ALLOC(c->w_d, size_t(p.B) * p.H * 4);
     LSA_ALLOC(c->Q_d, Qbytes);
@@ -323,10 +344,15 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
         cudaError_t ce = cudaMemcpy(c->seq_off_d, so, size_t(p.B + 1) * 8, cudaMemcpyHostToDevice);
         if (ce == cudaSuccess) ce = cudaMemset(c->err, 0, 16);
         if (ce == cudaSuccess) ce = cudaMemset(c->hot, 0, size_t(cap) * p.row_bytes);
+        // empty cache: no entry resident, no slot owned
+        if (ce == cudaSuccess) ce = cudaMemset(c->slot_of, 0xFF, size_t(p.n_total > 0 ? p.n_total : 1) * 4);
+        if (ce == cudaSuccess) ce = cudaMemset(c->owner, 0xFF, size_t(cap) * 4);
+        if (ce == cudaSuccess) ce = cudaMemset(c->fetched, 0, 16);
         if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking);
         if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking);
         if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_sel, cudaEventDisableTiming);
         if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_gather, cudaEventDisableTiming);
+        if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_assign, cudaEventDisableTiming);
         if (ce != cudaSuccess) {
             set_error("lsa_ctx_create: %s", cudaGetErrorString(ce));
             s = LSA_ERR_CUDA;
@@ -392,6 +418,9 @@ lsa_status lsa_ctx_get_view(lsa_ctx *c, lsa_ctx_view *v) {
     v->topk_pos = c->topk_pos;
     v->topk_cnt = c->topk_cnt;
     v->err = c->err;
+    v->kept_slot = c->p.full_fetch ? nullptr : c->kept_slot;
+    v->owner = c->p.full_fetch ? nullptr : c->owner;
+    v->fetched = c->fetched;
     return LSA_OK;
 }
 

@@ -260,6 +260,21 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         // ------------------------------------------------------------ producer
         if (!LISTED) {
             if (lane == 0) {
+                // the keys do not depend on the preceding prep kernel: fill the ring before waiting for it
+                const int64_t npre = (t1 - t0) < S ? (t1 - t0) : S;
+                {
+                    int bp = 0;
+                    int64_t r0, r1;
+                    for (int64_t t = t0; t < t0 + npre; ++t) {
+                        tile_info(s_toff, s_seq, B, t, bp, r0, r1);
+                        const int st = int(t - t0);
+                        mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+#pragma unroll
+                        for (int bx = 0; bx < C::kBoxes; ++bx)
+                            tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64,
+                                        int(r0));
+                    }
+                }
                 pdl_wait();   // the q image comes from the preceding prep kernel
                 int b = 0, cur = -1, qn = 0, st = 0;
                 uint32_t ph = 0;
@@ -274,12 +289,14 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                         cur = b;
                         ++qn;
                     }
-                    if (!mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs)) break;
-                    mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+                    if (t - t0 >= npre) {   // the first npre tiles were issued above
+                        if (!mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs)) break;
+                        mbar_arrive_expect_tx(&full[st], C::kStageBytes);
 #pragma unroll
-                    for (int bx = 0; bx < C::kBoxes; ++bx)
-                        tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64,
-                                    int(row0));
+                        for (int bx = 0; bx < C::kBoxes; ++bx)
+                            tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64,
+                                        int(row0));
+                    }
                     if (++st == S) { st = 0; ph ^= 1; }
                 }
             }

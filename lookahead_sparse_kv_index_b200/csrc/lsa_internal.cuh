@@ -96,10 +96,16 @@ lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, l
 lsa_status launch_select(const float *z, const int64_t *seq_off, int64_t n_total, int32_t B,
                          int32_t *kept_idx, int64_t capacity, int64_t *kept_off, uint32_t *mask,
                          void *workspace, int32_t *err, cudaStream_t st);
+// pos_map (nullable): topk_pos receives pos_map[p] instead of the kept position p.
 lsa_status launch_topk(const float *z, int32_t z_by_entry, const int64_t *seq_off,
                        const int32_t *kept_idx, const int64_t *kept_off, int32_t B, int32_t k,
-                       int64_t kept_cap, int32_t *topk_idx, int32_t *topk_pos, int32_t *topk_cnt,
-                       cudaStream_t st);
+                       int64_t kept_cap, const int32_t *pos_map, int32_t *topk_idx, int32_t *topk_pos,
+                       int32_t *topk_cnt, cudaStream_t st);
+size_t fetch_workspace(int64_t cap);
+lsa_status launch_fetch(const void *cold_dev, int64_t row_bytes, const int64_t *seq_off, const int32_t *kept_idx,
+                        const int64_t *kept_off, int32_t B, void *hot, int64_t cap, int32_t *slot_of,
+                        int32_t *owner, int32_t *kept_slot, int64_t *fetched, void *workspace, int32_t *err,
+                        cudaEvent_t assigned, cudaStream_t st);
 lsa_status launch_gather(const void *cold_dev, int64_t row_bytes, const int64_t *seq_off,
                          int64_t n_total, const int32_t *kept_idx, const int64_t *kept_off,
                          int32_t B, void *hot, int64_t hot_capacity, int32_t *slot_of,

@@ -69,7 +69,8 @@ __device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads)
 topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict__ seq_off,
             const int32_t *__restrict__ kept_idx, const int64_t *__restrict__ kept_off, int64_t kept_cap, int k,
-            int32_t *__restrict__ topk_idx, int32_t *__restrict__ topk_pos, int32_t *__restrict__ topk_cnt) {
+            const int32_t *__restrict__ pos_map, int32_t *__restrict__ topk_idx, int32_t *__restrict__ topk_pos,
+            int32_t *__restrict__ topk_cnt) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     __shared__ uint32_t s_keys[kStageKeys];
@@ -99,7 +100,7 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
     if (n <= k) {   // everything kept is chosen (uniform over the cluster: no cluster barrier is reached)
         for (int i = rank * kThreads + int(threadIdx.x); i < k; i += kCluster * kThreads) {
             out_idx[i] = i < n ? kept_idx[p0 + i] : -1;
-            if (out_pos) out_pos[i] = i < n ? int32_t(p0 + i) : -1;
+            if (out_pos) out_pos[i] = i < n ? (pos_map ? pos_map[p0 + i] : int32_t(p0 + i)) : -1;
         }
         if (rank == 0 && threadIdx.x == 0) topk_cnt[b] = n;
         return;
@@ -255,7 +256,10 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
                 if (u < nj) {
                     if (out < k) {
                         out_idx[out] = ids[u];
-                        if (out_pos) out_pos[out] = int32_t(p0 + c_lo + s0 + js[u]);
+                        if (out_pos) {
+                            const int64_t p = p0 + c_lo + s0 + js[u];
+                            out_pos[out] = pos_map ? pos_map[p] : int32_t(p);
+                        }
                     }
                     ++out;
                 }
@@ -269,10 +273,10 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
 
 lsa_status launch_topk(const float *z, int32_t z_by_entry, const int64_t *seq_off,
                        const int32_t *kept_idx, const int64_t *kept_off, int32_t B, int32_t k,
-                       int64_t kept_cap, int32_t *topk_idx, int32_t *topk_pos, int32_t *topk_cnt,
-                       cudaStream_t st) {
+                       int64_t kept_cap, const int32_t *pos_map, int32_t *topk_idx, int32_t *topk_pos,
+                       int32_t *topk_cnt, cudaStream_t st) {
     LSA_CUDA(launch_pdl(topk_select, dim3(kCluster, B), dim3(kThreads), 0, st, z, z_by_entry, seq_off, kept_idx,
-                        kept_off, kept_cap, k, topk_idx, topk_pos, topk_cnt));
+                        kept_off, kept_cap, k, pos_map, topk_idx, topk_pos, topk_cnt));
     LSA_LAUNCHED("topk_select");
     return LSA_OK;
 }

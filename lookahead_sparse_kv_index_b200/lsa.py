@@ -53,12 +53,14 @@ class Params(ctypes.Structure):
         ("Hq", i32), ("D", i32), ("attn_dtype", i32), ("topk", i32), ("tau", i32), ("scale", f32),
         ("n_total", i64), ("seq_off_host", P), ("k_dev", P), ("k_scale_dev", P), ("cold_host", P),
         ("row_bytes", i64), ("kv_row_stride", i64), ("k_off", i64), ("v_off", i64), ("kept_capacity", i64),
+        ("full_fetch", i32),
     ]
 
 
 class View(ctypes.Structure):
     _fields_ = [("z", P), ("z_kept", P), ("kept_idx", P), ("kept_off", P), ("slot_of", P), ("hot", P),
-                ("topk_idx", P), ("topk_pos", P), ("topk_cnt", P), ("err", P)]
+                ("topk_idx", P), ("topk_pos", P), ("topk_cnt", P), ("err", P), ("kept_slot", P), ("owner", P),
+                ("fetched", P)]
 
 
 def _sig(name, res, args):
@@ -176,17 +178,20 @@ class Context:
     """
 
     def __init__(self, *, B, H, d, q_dtype, k_dtype, Hq, D, attn_dtype, topk, seq_off_host, keys, k_scale,
-                 cold_host, row_bytes, kv_row_stride, k_off, v_off, kept_capacity, tau=64, scale=0.0):
+                 cold_host, row_bytes, kv_row_stride, k_off, v_off, kept_capacity, tau=64, scale=0.0,
+                 full_fetch=False):
         self._seq_off = torch.as_tensor(seq_off_host, dtype=torch.int64).contiguous()
         n_total = int(self._seq_off[-1])
         self.params = Params(B, H, d, DTYPE[q_dtype], DTYPE[k_dtype], Hq, D, DTYPE[attn_dtype], topk, tau,
                              float(scale), n_total, self._seq_off.data_ptr(), _ptr(keys), _ptr(k_scale),
-                             _ptr(cold_host), row_bytes, kv_row_stride, k_off, v_off, kept_capacity)
+                             _ptr(cold_host), row_bytes, kv_row_stride, k_off, v_off, kept_capacity,
+                             int(bool(full_fetch)))
         self._keep = (keys, k_scale, cold_host)
         h = P()
         _check(_L.lsa_ctx_create(ctypes.byref(self.params), ctypes.byref(h)), "lsa_ctx_create")
         self.handle = h
         self.B, self.topk, self.n_total, self.kept_capacity = B, topk, n_total, kept_capacity
+        self.row_bytes = row_bytes
 
     def close(self):
         if self.handle:
@@ -229,6 +234,10 @@ class Context:
 
     def launches(self) -> int:
         return int(_L.lsa_ctx_launches(self.handle))
+
+    def fetched(self) -> int:
+        """Rows the last refresh fetched from the cold pool (synchronises the device)."""
+        return int(device_view(self.view().fetched, 1, torch.int64).item())
 
 
 _cudart = None

@@ -89,7 +89,7 @@ def decoded(raw: np.ndarray, dtype: str) -> np.ndarray:
     return oracle.decode(raw, dtype)
 
 
-def make_context(wl, dev, lsa, kept_capacity=None, tau=64):
+def make_context(wl, dev, lsa, kept_capacity=None, tau=64, full_fetch=False):
     cap = kept_capacity or max(64, int(0.4 * wl.n_total) + 64)
     if wl.n_total <= 65536:
         cap = kept_capacity or wl.n_total + 64   # small cases may keep more than half the entries
@@ -97,7 +97,33 @@ def make_context(wl, dev, lsa, kept_capacity=None, tau=64):
                        attn_dtype=wl.attn_dtype, topk=wl.topk, seq_off_host=wl.seq_off, keys=dev["keys"],
                        k_scale=dev["k_scale"], cold_host=dev["cold"], row_bytes=wl.row_bytes,
                        kv_row_stride=wl.row_stride, k_off=wl.k_off, v_off=wl.v_off, kept_capacity=cap, tau=tau,
-                       scale=wl.scale)
+                       scale=wl.scale, full_fetch=full_fetch)
+
+
+def check_hot_cache(ctx, wl, lsa, gpu):
+    """The hot buffer after a refresh: every kept entry's row sits in its slot byte for byte,
+    slot_of and owner are inverse maps, and the top-k slots are the chosen entries' slots."""
+    v = ctx.view()
+    cap = ctx.kept_capacity
+    slot_of = lsa.device_view(v.slot_of, wl.n_total, torch.int32).cpu().numpy()
+    hot = lsa.device_view(v.hot, cap * ctx.row_bytes, torch.uint8).cpu().numpy().reshape(cap, ctx.row_bytes)
+    cold = np.ascontiguousarray(wl.cold).view(np.uint8).reshape(wl.n_total, ctx.row_bytes)
+    b_of = np.repeat(np.arange(wl.B), np.diff(gpu["kept_off"]))[: len(gpu["kept_idx"])]
+    ent = wl.seq_off[:-1][b_of] + gpu["kept_idx"]
+    slots = slot_of[ent]
+    assert (slots >= 0).all()
+    assert len(np.unique(slots)) == len(slots)
+    assert np.array_equal(hot[slots], cold[ent])
+    if v.owner:
+        owner = lsa.device_view(v.owner, cap, torch.int32).cpu().numpy()
+        assert np.array_equal(owner[slots], ent)
+        res = np.nonzero(slot_of >= 0)[0]
+        assert np.array_equal(owner[slot_of[res]], res)
+        assert np.array_equal(hot[slot_of[res]], cold[res])   # rows kept resident stay valid
+    for b in range(wl.B):
+        c = gpu["topk_cnt"][b]
+        e = wl.seq_off[b] + gpu["topk_idx"][b][:c]
+        assert np.array_equal(gpu["topk_pos"][b][:c], slot_of[e])
 
 
 def read_ctx(ctx, wl, lsa):
@@ -151,11 +177,6 @@ def check_decode_step(wl, t, q_t, w_t, Q_t, gpu, out_gpu, lse_gpu, z_refresh, re
             assert ok, (b, e, zb[e], z_k)
             n_swaps += 1
     report["topk_swaps"] = n_swaps
-    # top-k positions point at the right kept entries
-    for b in range(B):
-        for i in range(gpu["topk_cnt"][b]):
-            p = gpu["topk_pos"][b][i]
-            assert gpu["kept_idx"][p] == gpu["topk_idx"][b][i]
     # attention over the GPU's own top-k rows vs the oracle's attention on the same rows
     out_ref, lse_ref = oracle.sparse_attn(Q_t, wl.attn_dtype, wl.cold, wl.attn_dtype, wl.row_stride, wl.k_off,
                                           wl.v_off, oracle.local_to_global(gpu["topk_idx"], wl.seq_off), wl.scale)
@@ -173,12 +194,12 @@ def check_decode_step(wl, t, q_t, w_t, Q_t, gpu, out_gpu, lse_gpu, z_refresh, re
     return report
 
 
-def run_decode_and_check(wl, steps, tau, lsa, kept_capacity=None):
+def run_decode_and_check(wl, steps, tau, lsa, kept_capacity=None, full_fetch=False):
     """Drive the context and the oracle decoder over `steps`; check every listed step."""
     from oracle.stepper import OracleDecoder
 
     dev = synth.to_torch(wl)
-    ctx = make_context(wl, dev, lsa, kept_capacity=kept_capacity, tau=tau)
+    ctx = make_context(wl, dev, lsa, kept_capacity=kept_capacity, tau=tau, full_fetch=full_fetch)
     dec = OracleDecoder(wl, tau=tau)
     out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.float32 if wl.attn_dtype == "f32" else torch.int16,
                       device="cuda")
@@ -198,6 +219,7 @@ def run_decode_and_check(wl, steps, tau, lsa, kept_capacity=None):
         if t in steps:
             gpu = read_ctx(ctx, wl, lsa)
             assert gpu["err"] == 0
+            check_hot_cache(ctx, wl, lsa, gpu)
             rep = check_decode_step(wl, t, q_t, w_t, Q_t, gpu, out.cpu().numpy(), lse.cpu().numpy(), z_refresh,
                                     res_o)
             rep["t"] = t

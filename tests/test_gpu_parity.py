@@ -279,15 +279,50 @@ def test_sparse_attn_matches_oracle(lsa, case):
 
 # ---------------------------------------------------------- decode steps
 
+@pytest.mark.parametrize("full_fetch", [False, True], ids=["cached", "full_fetch"])
 @pytest.mark.parametrize("name,steps,tau", [
     ("tiny", [0, 1, 2, 3, 4, 5], 4),
-    ("ragged_bf16", [0, 1, 3, 4, 7], 4),
+    ("ragged_bf16", [0, 1, 3, 4, 7, 8], 4),
     ("ragged_e4m3", [0, 2, 4, 5], 4),
 ])
-def test_decode_steps_small(lsa, name, steps, tau):
+def test_decode_steps_small(lsa, name, steps, tau, full_fetch):
     wl = SCORE_CASES[name]()
-    reps = run_decode_and_check(wl, steps, tau, lsa)
+    reps = run_decode_and_check(wl, steps, tau, lsa, full_fetch=full_fetch)
     assert [r["t"] for r in reps] == steps
+
+
+def test_hot_cache_fetches_only_new_rows(lsa):
+    """A refresh that keeps the same set fetches nothing; one with a different query fetches exactly
+    the kept entries that are not resident; a small hot buffer evicts rows no longer kept."""
+    from gpu_cases import check_hot_cache, make_context, read_ctx
+
+    wl = synth.small_ragged(key_dtype="bf16", lengths=(3000, 1500))
+    dev = synth.to_torch(wl)
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.int16, device="cuda")
+    lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device="cuda")
+    ins = [wl.step_inputs(t) for t in (0, 5)]
+    dins = [(synth.raw_to_torch(q), torch.from_numpy(np.ascontiguousarray(w)).cuda(), synth.raw_to_torch(Q))
+            for q, w, Q in ins]
+    q1 = synth.raw_to_torch(synth.bf16_bits(torch.randn(wl.B, wl.H, wl.d) / 8))   # an unrelated query
+    z0 = oracle.index_score(ins[0][0], "bf16", ins[0][1], wl.keys, "bf16", None, wl.seq_off, wl.H, wl.d,
+                            want_I=False)
+    n0 = int((z0 >= 0).sum())
+    for cap in (wl.n_total, n0 + 40):   # roomy, and barely larger than the first kept set
+        ctx = make_context(wl, dev, lsa, kept_capacity=cap, tau=1)
+        ctx.step(0, *dins[0], out, lse)
+        assert ctx.fetched() == n0
+        resident = set(np.nonzero(lsa.device_view(ctx.view().slot_of, wl.n_total, torch.int32).cpu().numpy() >= 0)[0])
+        check_hot_cache(ctx, wl, lsa, read_ctx(ctx, wl, lsa))
+        ctx.step(1, *dins[0], out, lse)               # same query: same kept set
+        assert ctx.fetched() == 0
+        ctx.step(2, q1, dins[0][1], dins[0][2], out, lse)
+        g = read_ctx(ctx, wl, lsa)
+        assert g["err"] == 0
+        b_of = np.repeat(np.arange(wl.B), np.diff(g["kept_off"]))
+        ent = set((wl.seq_off[:-1][b_of] + g["kept_idx"]).tolist())
+        assert ctx.fetched() == len(ent - resident)
+        check_hot_cache(ctx, wl, lsa, g)
+        ctx.close()
 
 
 def test_decode_step_host_equals_device(lsa):
