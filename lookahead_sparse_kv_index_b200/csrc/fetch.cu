@@ -79,7 +79,8 @@ fetch_assign(const int64_t *__restrict__ seq_off, const int32_t *__restrict__ ke
              const int32_t *__restrict__ free_list, const int32_t *__restrict__ counts,
              int32_t *__restrict__ kept_slot, int32_t *__restrict__ slot_of, int32_t *__restrict__ owner,
              int64_t *__restrict__ fetched) {
-    const int n_new = counts[0];
+    // free >= new whenever the kept list fits the hot buffer; the clamp keeps every slot index in range
+    const int n_new = min(counts[0], counts[1]);
     if (blockIdx.x == 0 && threadIdx.x == 0) *fetched = n_new;
     for (int i = blockIdx.x * kThreads + threadIdx.x; i < n_new; i += gridDim.x * kThreads) {
         const int32_t p = new_list[i];
@@ -102,7 +103,7 @@ fetch_rows(const uint4 *__restrict__ cold, int64_t row_vec, const int64_t *__res
            const int32_t *__restrict__ kept_idx, const int64_t *__restrict__ kept_off, int B,
            const int32_t *__restrict__ new_list, const int32_t *__restrict__ counts,
            const int32_t *__restrict__ kept_slot, uint4 *__restrict__ hot) {
-    const int n_new = counts[0];
+    const int n_new = min(counts[0], counts[1]);
     const int lane = threadIdx.x & 31;
     const int64_t warp = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (int64_t(gridDim.x) * kThreads) >> 5;
