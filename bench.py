@@ -74,6 +74,30 @@ def dist_env():
     return ws, rank, local
 
 
+SEEDS = {"ctx500k": 2, "ctx128k": 1, "ragged": 3}
+
+
+def rank_seed(config: str, rank: int) -> int:
+    """Each rank runs an independent batch: the config's seed offset by the rank."""
+    return SEEDS[config] + 1000 * rank
+
+
+def max_over_ranks(x: float, pg, device="cpu") -> float:
+    """The slowest rank's time (all ranks take this collective step in the same order)."""
+    if pg is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_steps_per_s(world: int, tau: int, windows: int, ms_max: float) -> float:
+    """Decode steps/s of all ranks: every rank ran `windows` tau-windows in at most ms_max."""
+    return world * tau * windows / (ms_max / 1e3)
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -234,7 +258,7 @@ def run_cuda(args):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
         pg = dist
 
-    wl = synth.CONFIGS[args.config](seed={"ctx500k": 2, "ctx128k": 1, "ragged": 3}[args.config] + 1000 * rank)
+    wl = synth.CONFIGS[args.config](seed=rank_seed(args.config, rank))
     dev = synth.to_torch(wl)
     cap = max(wl.topk, int(args.hot_frac * wl.n_total))
     ctxs, keys = [], []
@@ -278,12 +302,6 @@ def run_cuda(args):
         if pg is not None:
             pg.barrier()
 
-    def max_over_ranks(x):
-        if pg is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
 
     # prime: two windows per context so that every step's graph is captured before timing
     # (a context runs each step kind eagerly once, then captures per pointer set)
@@ -308,12 +326,12 @@ def run_cuda(args):
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), pg, "cuda")
     launches = sum(c.launches() for c in ctxs)
     fetched_rows = [c.fetched() for c in ctxs]
     errs = [int(lsa.device_view(c.view().err, 1, torch.int32).item()) for c in ctxs]
     ms_window = ms_total / args.steps
-    value = ws * tau * args.steps / (ms_total / 1e3)
+    value = whole_job_steps_per_s(ws, tau, args.steps, ms_total)
 
     # stage breakdown: two more windows run eagerly with CUDA events around every stage
     # (these include launch gaps when the GPU waits for the host; not part of `value`)
@@ -401,7 +419,7 @@ def run_cuda(args):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, "cuda")
     h2d = tau * (q_h[0].numel() * q_h[0].element_size() + w_h[0].numel() * 4 + Q_h[0].numel() * Q_h[0].element_size())
     d2h = tau * (out_h.numel() * out_h.element_size() + lse_h.numel() * 4)
 
@@ -432,7 +450,7 @@ def run_cuda(args):
                          "in_window_stage_ms": stage["score"][0] / max(stage["score"][1], 1),
                          "peak_source": peak_src},
             "cpu_baseline": cpu_base,
-            "e2e": {"value": ws * tau * args.steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": whole_job_steps_per_s(ws, tau, args.steps, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "cuda_graphs": True,
