@@ -134,6 +134,25 @@ lsa_status lsa_select(const float *z, const int64_t *seq_off, int64_t n_total, i
                       void *workspace, size_t ws_bytes, int32_t *err, void *stream);
 
 /* ------------------------------------------------------------------------
+ * lsa_select_noalloc -- lsa_select without a caller workspace.  The pages
+ * have no counterpart: this is a calling convention for callers that cannot
+ * allocate device memory when they select (a stream capture that forbids
+ * allocation, a runtime whose pool owns all device memory, a plugin host that
+ * passes no workspace).  Same arguments and results as lsa_select, minus the
+ * workspace; the scratch is a static device array of the library (560 KB on
+ * every GPU that loads it, held until the process exits), so n_total is
+ * limited to lsa_select_noalloc_max_entries() (4,194,304); larger n_total is
+ * rejected with LSA_ERR_INVALID before anything is launched.  The first call
+ * on a device looks the array's device address up (cudaGetSymbolAddress) and
+ * should come before any stream capture.  No call allocates or frees memory.
+ * All calls on a device share the array: calls that overlap on the GPU race.
+ * ---------------------------------------------------------------------- */
+int64_t lsa_select_noalloc_max_entries(void);
+lsa_status lsa_select_noalloc(const float *z, const int64_t *seq_off, int64_t n_total, int32_t B,
+                              int32_t *kept_idx, int64_t capacity, int64_t *kept_off, uint32_t *mask,
+                              int32_t *err, void *stream);
+
+/* ------------------------------------------------------------------------
  * lsa_topk -- fine-grained top-k inside the kept set (section 2.1, "Tiered
  * Selection").  Per sequence, the k kept entries with the largest z (the
  * sigmoid is monotone, so ranking by z ranks by I); equal z goes to the lower

@@ -32,7 +32,7 @@ N_STAGES = 6
 # every symbol include/lsa.h declares
 EXPORTS = [
     "lsa_version", "lsa_last_error", "lsa_status_name", "lsa_index_score_workspace_size", "lsa_index_score",
-    "lsa_select_workspace_size",
+    "lsa_select_workspace_size", "lsa_select_noalloc_max_entries", "lsa_select_noalloc",
     "lsa_select", "lsa_topk", "lsa_gather", "lsa_sparse_attn_workspace_size", "lsa_sparse_attn",
     "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
     "lsa_ctx_set_graphs", "lsa_ctx_set_timing", "lsa_ctx_stage_times", "lsa_ctx_reset_counters",
@@ -76,6 +76,8 @@ _sig("lsa_index_score_workspace_size", sz, [i32, i32, i32])
 _sig("lsa_index_score", i32, [P, i32, P, P, i32, P, P, i64, P, P, i64, i32, i32, i32, P, P, P, sz, P, P])
 _sig("lsa_select_workspace_size", sz, [i64])
 _sig("lsa_select", i32, [P, P, i64, i32, P, i64, P, P, P, sz, P, P])
+_sig("lsa_select_noalloc_max_entries", i64, [])
+_sig("lsa_select_noalloc", i32, [P, P, i64, i32, P, i64, P, P, P, P])
 _sig("lsa_topk", i32, [P, i32, P, P, P, i64, i32, i32, P, P, P, P])
 _sig("lsa_gather", i32, [P, i64, P, i64, P, P, i32, P, i64, P, P, P])
 _sig("lsa_sparse_attn_workspace_size", sz, [i32, i32, i32, i32])
@@ -142,6 +144,17 @@ def select(z, seq_off, n_total, kept_idx, capacity, kept_off, mask, workspace, e
     _check(_L.lsa_select(_ptr(z), _ptr(seq_off), n_total, B, _ptr(kept_idx), capacity, _ptr(kept_off), _ptr(mask),
                          _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(err),
                          _stream(stream)), "lsa_select")
+
+
+def select_noalloc_max_entries() -> int:
+    return int(_L.lsa_select_noalloc_max_entries())
+
+
+def select_noalloc(z, seq_off, n_total, kept_idx, capacity, kept_off, mask, err, stream=None):
+    """lsa_select with the library's static scratch instead of a caller workspace."""
+    B = seq_off.numel() - 1
+    _check(_L.lsa_select_noalloc(_ptr(z), _ptr(seq_off), n_total, B, _ptr(kept_idx), capacity, _ptr(kept_off),
+                                 _ptr(mask), _ptr(err), _stream(stream)), "lsa_select_noalloc")
 
 
 def topk(z, z_by_entry, seq_off, kept_idx, kept_off, kept_capacity, k, topk_idx, topk_pos, topk_cnt, stream=None):
