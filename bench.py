@@ -208,7 +208,7 @@ def run_reference(args):
     import oracle
     import synth
 
-    wl = synth.CONFIGS[args.config](with_cold=True)
+    wl = synth.WORKLOADS[args.config](with_cold=True)
     oracle.build()
     vals = []
     info = {}
@@ -258,7 +258,7 @@ def run_cuda(args):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
         pg = dist
 
-    wl = synth.CONFIGS[args.config](seed=rank_seed(args.config, rank))
+    wl = synth.WORKLOADS[args.config](seed=rank_seed(args.config, rank))
     dev = synth.to_torch(wl)
     cap = max(wl.topk, int(args.hot_frac * wl.n_total))
     ctxs, keys = [], []
@@ -478,7 +478,7 @@ def run_only_scan(args):
     import synth
     from lookahead_sparse_kv_index_b200 import lsa
 
-    wl = synth.CONFIGS[args.config](with_cold=False)
+    wl = synth.WORKLOADS[args.config](with_cold=False)
     dev = synth.to_torch(wl, pin_cold=False)
     keys = [dev["keys"]] + [dev["keys"].clone() for _ in range(REPLICAS - 1)]
     n = wl.n_total

@@ -264,7 +264,7 @@ def small_ragged(seed: int = 5, key_dtype: str = "bf16", lengths=(1000, 4133, 25
                    topk=topk, Hq=Hq, D=D)
 
 
-CONFIGS = {
+WORKLOADS = {
     "tiny": tiny,
     "ctx128k": ctx128k,
     "ctx500k": ctx500k,

@@ -380,7 +380,7 @@ def test_decode_graph_replay_equals_eager(lsa):
 
 @pytest.mark.parametrize("name", ["ctx128k", "ctx500k"])
 def test_decode_full_size(lsa, name):
-    wl = synth.CONFIGS[name]()
+    wl = synth.WORKLOADS[name]()
     reps = run_decode_and_check(wl, [0, 1, 63], 64, lsa, kept_capacity=int(0.2 * wl.n_total))
     print(name, reps)
 
