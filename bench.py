@@ -351,12 +351,11 @@ def run_cuda(args):
     # the index scan alone, back to back on this stream over the rotating key replicas
     # (queries of step 0): its launch duration without host gaps
     zs = torch.empty(wl.n_total, dtype=torch.float32, device="cuda")
-    sws = torch.empty(lsa.index_score_workspace_size(wl.B, wl.H, wl.d), dtype=torch.uint8, device="cuda")
     serr = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     def scan_once(i):
         lsa.index_score(q_d[0], wl.q_dtype, w_d[0], keys[i % REPLICAS], wl.key_dtype, dev["k_scale"],
-                        dev["seq_off"], wl.n_total, wl.H, wl.d, zs, None, workspace=sws, err=serr)
+                        dev["seq_off"], wl.n_total, wl.H, wl.d, zs, None, err=serr)
 
     for i in range(3):
         scan_once(i)
@@ -444,7 +443,7 @@ def run_cuda(args):
                        "parallelism": f"independent batch per GPU x{ws}", "kept_capacity": cap},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "lsa_index_score full scan (scan_tc_prep + scan_tc), %d back-to-back launches "
+                         "kernel": "lsa_index_score full scan (scan_tc), %d back-to-back launches "
                                    "on the bench stream over 3 rotating key replicas" % n_scan,
                          "algorithmic_bytes": scan_bytes, "avg_launch_ms": scan_ms,
                          "in_window_stage_ms": stage["score"][0] / max(stage["score"][1], 1),
@@ -483,12 +482,11 @@ def run_only_scan(args):
     keys = [dev["keys"]] + [dev["keys"].clone() for _ in range(REPLICAS - 1)]
     n = wl.n_total
     z = torch.empty(n, dtype=torch.float32, device="cuda")
-    ws = torch.empty(lsa.index_score_workspace_size(wl.B, wl.H, wl.d), dtype=torch.uint8, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     def once(i):
         lsa.index_score(dev["q"], wl.q_dtype, dev["w"], keys[i % REPLICAS], wl.key_dtype, dev["k_scale"],
-                        dev["seq_off"], n, wl.H, wl.d, z, None, workspace=ws, err=err)
+                        dev["seq_off"], n, wl.H, wl.d, z, None, err=err)
 
     for i in range(args.warmup):
         once(i)

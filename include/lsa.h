@@ -89,26 +89,22 @@ const char *lsa_status_name(lsa_status s);
  *   list_capacity (host) bounds idx_off[B].
  * Full mode (idx == NULL): z / I are written for every entry, [n_total].
  * z        fp32 output (required).   I  fp32 output or NULL.
- * workspace  device scratch of lsa_index_score_workspace_size(B, H, d) bytes,
- *          16-byte aligned, or NULL.  With a workspace, scans (full or
- *          listed) of bf16 q over bf16 keys (d 64 or 128) or e4m3 keys
- *          (d 128) with H in {16, 32, 64}, B <= 512 and n_total >= 128 run on
- *          the tensor cores (tcgen05); every other case, and every call
- *          without a workspace, runs the CUDA-core kernel.
- *          The workspace holds the per-sequence query operand between the two
- *          kernels of one call; calls that share a workspace must not overlap.
+ * flags    0, or LSA_SCORE_CUDA_CORE.  Scans (full or listed) of bf16 q (16-byte
+ *          aligned) over bf16 keys (d 64 or 128) or e4m3 keys (d 128) with H in
+ *          {16, 32, 64}, B <= 512 and n_total >= 128 run on the tensor cores
+ *          (tcgen05); every other case, and every call with
+ *          LSA_SCORE_CUDA_CORE, runs the CUDA-core kernel.
  * err      device error word or NULL (LSA_ERR_TIMEOUT if a bounded wait of the
  *          tensor-core kernel gave up).
  * Shapes run: 1 <= H <= 64, d in {32, 64, 128} (d * element size % 16 == 0).
  * ---------------------------------------------------------------------- */
-size_t lsa_index_score_workspace_size(int32_t B, int32_t H, int32_t d);
+enum { LSA_SCORE_CUDA_CORE = 1 };
 lsa_status lsa_index_score(const void *q, lsa_dtype q_dtype, const float *w,
                            const void *k, lsa_dtype k_dtype, const float *k_scale,
                            const int64_t *seq_off, int64_t n_total,
                            const int32_t *idx, const int64_t *idx_off, int64_t list_capacity,
                            int32_t B, int32_t H, int32_t d,
-                           float *z, float *I, void *workspace, size_t ws_bytes,
-                           int32_t *err, void *stream);
+                           float *z, float *I, int32_t flags, int32_t *err, void *stream);
 
 /* ------------------------------------------------------------------------
  * lsa_select -- threshold selection (section 2.1, "Dynamic Fetching"):

@@ -71,16 +71,11 @@ const char *lsa_status_name(lsa_status s) {
     return "LSA_ERR_UNKNOWN";
 }
 
-size_t lsa_index_score_workspace_size(int32_t B, int32_t H, int32_t d) {
-    if (B < 1 || H < 1 || d < 1) return 0;
-    return index_score_tc_workspace(B, H, d);
-}
-
 lsa_status lsa_index_score(const void *q, lsa_dtype q_dtype, const float *w, const void *k,
                            lsa_dtype k_dtype, const float *k_scale, const int64_t *seq_off,
                            int64_t n_total, const int32_t *idx, const int64_t *idx_off,
                            int64_t list_capacity, int32_t B, int32_t H, int32_t d, float *z,
-                           float *I, void *workspace, size_t ws_bytes, int32_t *err, void *stream) {
+                           float *I, int32_t flags, int32_t *err, void *stream) {
     clear_error();
     LSA_CHECK_ARG(q && w && k && seq_off && z, "lsa_index_score: q, w, k, seq_off and z are required");
     LSA_CHECK_ARG(B >= 1 && H >= 1 && d >= 1, "lsa_index_score: B=%d H=%d d=%d must be positive", B, H, d);
@@ -99,12 +94,10 @@ lsa_status lsa_index_score(const void *q, lsa_dtype q_dtype, const float *w, con
                   "lsa_index_score: idx and idx_off go together");
     LSA_CHECK_ARG(idx == nullptr || (list_capacity >= 0 && list_capacity < (int64_t(1) << 31)),
                   "lsa_index_score: bad list_capacity");
-    LSA_CHECK_ARG(workspace == nullptr ||
-                      (aligned16(workspace) && ws_bytes >= lsa_index_score_workspace_size(B, H, d)),
-                  "lsa_index_score: workspace of %zu bytes < %zu", ws_bytes, lsa_index_score_workspace_size(B, H, d));
+    LSA_CHECK_ARG((flags & ~LSA_SCORE_CUDA_CORE) == 0, "lsa_index_score: unknown flags 0x%x", flags);
     if ((idx ? list_capacity : n_total) == 0) return LSA_OK;
     return launch_index_score(q, q_dtype, w, k, k_dtype, k_scale, seq_off, n_total, idx, idx_off,
-                              list_capacity, B, H, d, z, I, workspace, err, as_stream(stream));
+                              list_capacity, B, H, d, z, I, flags, err, as_stream(stream));
 }
 
 size_t lsa_select_workspace_size(int64_t n_total) {

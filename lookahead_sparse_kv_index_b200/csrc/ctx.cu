@@ -71,8 +71,6 @@ struct lsa_ctx {
     size_t sel_ws_bytes = 0;
     void *attn_ws = nullptr;
     size_t attn_ws_bytes = 0;
-    void *score_ws = nullptr;
-    size_t score_ws_bytes = 0;
     // staging for lsa_decode_step_host
     void *q_d = nullptr, *Q_d = nullptr, *out_d = nullptr;
     float *w_d = nullptr, *lse_d = nullptr;
@@ -100,7 +98,7 @@ using namespace lsa;
 
 void free_all(lsa_ctx *c) {
     void *bufs[] = {c->seq_off_d, c->z, c->z_kept, c->kept_idx, c->kept_off, c->slot_of, c->hot,
-                    c->topk_idx, c->topk_pos, c->topk_cnt, c->err, c->sel_ws, c->attn_ws, c->score_ws,
+                    c->topk_idx, c->topk_pos, c->topk_cnt, c->err, c->sel_ws, c->attn_ws,
                     c->owner, c->kept_slot, c->fetched, c->fetch_ws,
                     c->q_d, c->Q_d, c->out_d, c->w_d, c->lse_d};
     for (void *b : bufs)
@@ -172,8 +170,8 @@ lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w,
     if (refresh) {
         StageTimer ts(c, LSA_STAGE_SCORE, st);
         LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
-                                   p.n_total, nullptr, nullptr, 0, p.B, p.H, p.d, c->z, nullptr,
-                                   c->score_ws, c->err, st));
+                                   p.n_total, nullptr, nullptr, 0, p.B, p.H, p.d, c->z, nullptr, 0,
+                                   c->err, st));
         ts.done();
         StageTimer tsel(c, LSA_STAGE_SELECT, st);
         LSA_TRY(launch_select(c->z, c->seq_off_d, p.n_total, p.B, c->kept_idx, cap, c->kept_off,
@@ -203,7 +201,7 @@ lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w,
         StageTimer tr(c, LSA_STAGE_RESCORE, st);
         LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
                                    p.n_total, c->kept_idx, c->kept_off, cap, p.B, p.H, p.d, c->z_kept,
-                                   nullptr, c->score_ws, c->err, st));
+                                   nullptr, 0, c->err, st));
         tr.done();
         StageTimer tk(c, LSA_STAGE_TOPK, st);
         LSA_TRY(launch_topk(c->z_kept, 0, c->seq_off_d, c->kept_idx, c->kept_off, p.B, p.topk, cap,
@@ -312,7 +310,6 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     const size_t Qbytes = size_t(p.B) * p.Hq * p.D * elem_size(p.attn_dtype);
     c->sel_ws_bytes = lsa_select_workspace_size(p.n_total);
     c->attn_ws_bytes = sparse_attn_workspace(p.B, p.Hq, p.D, p.topk);
-    c->score_ws_bytes = index_score_tc_workspace(p.B, p.H, p.d);
     lsa_status s = LSA_OK;
 #define LSA_ALLOC(ptr, bytes) \
     if (s == LSA_OK) s = alloc(&(ptr), (bytes))
@@ -329,7 +326,6 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     LSA_ALLOC(c->err, 16);
     LSA_ALLOC(c->sel_ws, c->sel_ws_bytes);
     LSA_ALLOC(c->attn_ws, c->attn_ws_bytes);
-    LSA_ALLOC(c->score_ws, c->score_ws_bytes);
     LSA_ALLOC(c->owner, size_t(cap) * 4);
     LSA_ALLOC(c->kept_slot, size_t(cap) * 4);
     LSA_ALLOC(c->fetched, 16);

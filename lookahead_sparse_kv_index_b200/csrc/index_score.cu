@@ -7,7 +7,7 @@
 // registers.  It runs every supported shape and dtype (fp32 keys included)
 // and the listed (gathered) variant used between refreshes.  Scans of bf16 /
 // e4m3 keys of the shapes index_score_tc.cu supports, full or listed, go to the
-// tensor-core kernel when the caller provides its workspace.
+// tensor-core kernel unless the caller asks for this path.
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -184,13 +184,12 @@ lsa_status launch_index_score(const void *q, lsa_dtype q_dtype, const float *w, 
                               lsa_dtype k_dtype, const float *k_scale, const int64_t *seq_off,
                               int64_t n_total, const int32_t *idx, const int64_t *idx_off,
                               int64_t list_capacity, int32_t B, int32_t H, int32_t d, float *z,
-                              float *I, void *workspace, int32_t *err, cudaStream_t st) {
+                              float *I, int32_t flags, int32_t *err, cudaStream_t st) {
     const int64_t n_axis = idx ? list_capacity : n_total;
-    // the tensor-core path reads q rows with 16-byte loads and the workspace as 16-byte chunks
-    if (workspace && aligned16(q) && aligned16(workspace) &&
-        index_score_tc_supported(q_dtype, k_dtype, n_total, B, H, d))
+    // the tensor-core kernel reads query rows with 16-byte loads
+    if (!(flags & LSA_SCORE_CUDA_CORE) && aligned16(q) && index_score_tc_supported(q_dtype, k_dtype, n_total, B, H, d))
         return launch_index_score_tc(q, w, k, k_dtype, k_scale, seq_off, n_total, idx, idx_off, list_capacity, B,
-                                     H, d, z, I, workspace, err, st);
+                                     H, d, z, I, err, st);
     switch (k_dtype) {
     case LSA_F32:
         return launch_kt<LSA_F32>(q, q_dtype, w, k, k_scale, seq_off, n_axis, idx, idx_off, B, H, d, z, I, st);

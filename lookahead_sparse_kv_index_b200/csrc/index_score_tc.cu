@@ -4,31 +4,36 @@
 //
 // Per sequence the q.k block is a dense contraction [entries x d] x [d x H]
 // (H = 64 heads, d = 128: 16 Kflop per entry), so the scan is HBM-bound only
-// when the dot products run on the tensor cores.  Layout of the work:
-//   * persistent CTAs, one per SM, each streaming a contiguous range of
-//     128-entry tiles (tiles never straddle two sequences);
-//   * warp 0: TMA loads of key tiles (128-byte swizzle) into a smem ring,
-//     plus one bulk copy of the sequence's query operand on a sequence change;
-//   * warp 1: tcgen05.mma, M = 128 entries, N = H heads, into one of four
-//     TMEM accumulators (H fp32 columns each);
+// when the dot products run on the tensor cores.  One kernel, persistent CTAs
+// (one per SM), each streaming a contiguous range of 128-entry tiles (tiles
+// never straddle two sequences):
+//   * warp 0 (producer): TMA loads of key tiles (128-byte swizzle) into a smem
+//     ring -- the first ring's worth before anything else -- and, on every
+//     sequence change, builds that sequence's query operand and gate weights
+//     in one of two smem slots (no separate preparation kernel);
+//   * warp 1: tcgen05.mma, M = 128 entries, N = H heads (bf16 keys) or 2H
+//     (e4m3 keys: both query pieces at once), into one of four TMEM
+//     accumulators;
 //   * warps 2-9: two epilogue warpgroups taking alternate tiles, one TMEM lane
 //     (= one entry) per thread: ReLU, gate weights, head sum in registers, one
-//     coalesced fp32 store per entry; the row scale is fetched before the
-//     accumulator wait so its latency overlaps the MMA.
+//     coalesced fp32 store per entry; the row scale is fetched one tile ahead.
 // bf16 keys use kind::f16 (bf16 x bf16).  e4m3 keys use kind::f8f6f4 against
-// an exact two-piece e4m3 split of the bf16 query (see scan_tc_prep), so the
-// keys go from HBM to the tensor core untouched; the per-row key scale and the
-// per-head power-of-two query scale are applied after the ReLU, which is
-// positively homogeneous.
+// an exact two-piece e4m3 split of the bf16 query, so the keys go from HBM to
+// the tensor core untouched; the per-row key scale and the per-head
+// power-of-two query scale are applied after the ReLU, which is positively
+// homogeneous.
 //
 // The listed variant scores only the entries of a per-sequence index list (the
 // kept set, re-ranked every decode step): the producer warp gathers those key
 // rows with cp.async into the same swizzled layout, three tiles in flight per
 // lane.
 //
-// Every wait is bounded in time; a wait that gives up sets LSA_ERR_TIMEOUT in
-// the caller's error word, stops the CTA's loops, drains the issued MMAs and
-// frees TMEM before returning.
+// A query slot is rewritten only after the MMA and all eight epilogue warps
+// have released the sequence that used it (release barriers indexed by the
+// sequence's ordinal mod 8, so a warp running ahead never completes an older
+// phase).  Every wait is bounded in time; a wait that gives up sets
+// LSA_ERR_TIMEOUT in the caller's error word, stops the CTA's loops, drains the
+// issued MMAs and frees TMEM before returning.
 #include <cuda.h>
 
 #include "lsa_internal.cuh"
@@ -65,106 +70,32 @@ struct Cfg<E4M3_D128> {
     static constexpr int kStages = 8;
 };
 
-constexpr int kThreads = 320;         // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue (2 warpgroups)
+constexpr int kThreads = 320;         // warp 0 producer, warp 1 MMA, warps 2-9 epilogue (2 warpgroups)
 constexpr int kEpiGroups = 2;
+constexpr int kEpiWarps = 8;
+constexpr int kRel = 8;               // query-slot release barriers, by sequence ordinal mod kRel
 constexpr int kRows = 128;
-constexpr int kAcc = 4;                  // TMEM accumulator stages
-constexpr int kMaxB = 512;               // sequences per launch on this path
+constexpr int kAcc = 4;               // TMEM accumulator stages
+constexpr int kMaxB = 512;            // sequences per launch on this path
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
-constexpr int kImgTail = 1024;           // bytes after the operand image: gate weights w'
+constexpr int kGatherDepth = 3;       // listed mode: tiles of row gathers in flight per producer lane
 
-__host__ __device__ constexpr uint32_t tmem_cols(int H) {
-    return (kAcc * H) <= 32 ? 32 : (kAcc * H) <= 64 ? 64 : (kAcc * H) <= 128 ? 128 : 256;
+// Accumulator width in TMEM columns: H for bf16 keys; 2H for e4m3 keys, whose MMA
+// multiplies by both query pieces at once (piece 1 -> columns [0,H), piece 2 ->
+// [H,2H)) and whose epilogue adds the two halves before the ReLU.
+__host__ __device__ constexpr int acc_cols(int KIND, int H) { return KIND == 2 ? 2 * H : H; }
+
+__host__ __device__ constexpr uint32_t tmem_cols(int cols) {
+    return (kAcc * cols) <= 32    ? 32
+           : (kAcc * cols) <= 64  ? 64
+           : (kAcc * cols) <= 128 ? 128
+           : (kAcc * cols) <= 256 ? 256
+                                  : 512;
 }
 
 template <int KIND, int H>
 __host__ __device__ constexpr int qimg_bytes() {
     return Cfg<KIND>::kQBytesPerHead * H;
-}
-
-template <int KIND, int H>
-__host__ __device__ constexpr int img_stride() {
-    return qimg_bytes<KIND, H>() + kImgTail;
-}
-
-// ---------------------------------------------------------------------------
-// Query operand image, one per sequence, laid out exactly as the MMA reads it
-// from shared memory (K-major, 128-byte swizzle: 16-byte chunk c of row j is
-// stored at chunk c ^ (j % 8)), followed by the gate weights w'.
-//
-// bf16 keys: the bf16 query itself, w' = w.
-// e4m3 keys: per head j, a power-of-two scale 2^e_j brings max_c |q_jc| into
-// [128, 256); p1 = e4m3(q 2^e_j), p2 = e4m3(q 2^e_j - p1), both round to
-// nearest even.  A bf16 value has 8 significant bits, p1 carries 4 and the
-// remainder q 2^e_j - p1 is a multiple of the bf16 ulp no larger than 8 ulps,
-// so p2 holds it exactly whenever it is at least the e4m3 subnormal step 2^-9:
-// p1 + p2 == q 2^e_j for every element with |q| >= 2^-10 max_c |q_jc|, and
-// within 2^-10 of it (2^-17 max_c |q_jc| before scaling) otherwise.
-// w'_j = w_j 2^-e_j.
-// ---------------------------------------------------------------------------
-template <int KIND, int H>
-__global__ void __launch_bounds__(256)
-scan_tc_prep(const uint16_t *__restrict__ q, const float *__restrict__ w, int d, uint8_t *__restrict__ img) {
-    pdl_launch_dependents();   // the scan may start its prologue and key loads now
-    // grid (B, H / 8): block (b, g) prepares heads 8g .. 8g+7 of sequence b, one warp per head
-    const int b = blockIdx.x;
-    uint8_t *dst = img + size_t(b) * img_stride<KIND, H>();
-    float *wp = reinterpret_cast<float *>(dst + qimg_bytes<KIND, H>());
-    const uint16_t *qb = q + size_t(b) * H * d;
-    const int h0 = blockIdx.y * 8;
-    if (KIND != E4M3_D128) {
-        const int cpr = d / 8;   // 16-byte chunks per row
-        for (int i = threadIdx.x; i < 8 * cpr; i += blockDim.x) {
-            const int j = h0 + i / cpr, c = i % cpr;
-            const int a = c >> 3, cc = c & 7;
-            const int off = a * (H * 128) + j * 128 + ((cc ^ (j & 7)) << 4);
-            *reinterpret_cast<uint4 *>(dst + off) = *reinterpret_cast<const uint4 *>(qb + j * d + c * 8);
-        }
-        if (threadIdx.x < 8) wp[h0 + threadIdx.x] = w[size_t(b) * H + h0 + threadIdx.x];
-    } else {
-        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-        {
-            const int j = h0 + warp;
-            float v[4];
-            float m = 0.f;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                v[u] = bf16_to_f32(qb[j * 128 + 4 * lane + u]);
-                m = fmaxf(m, fabsf(v[u]));
-            }
-#pragma unroll
-            for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            int e = 0;
-            if (m > 0.f) {
-                int E;
-                frexpf(m, &E);
-                e = 8 - E;
-            }
-            uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float s = ldexpf(v[u], e);
-                const __nv_fp8_storage_t p1 = __nv_cvt_float_to_fp8(s, __NV_SATFINITE, __NV_E4M3);
-                const __half_raw h1 = __nv_cvt_fp8_to_halfraw(p1, __NV_E4M3);
-                const float r = s - __half2float(__half(h1));
-                const __nv_fp8_storage_t p2 = __nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3);
-                w0 |= uint32_t(p1) << (8 * u);
-                w1 |= uint32_t(p2) << (8 * u);
-            }
-            const int off = j * 128 + (((lane >> 2) ^ (j & 7)) << 4) + (lane & 3) * 4;
-            *reinterpret_cast<uint32_t *>(dst + off) = w0;
-            *reinterpret_cast<uint32_t *>(dst + H * 128 + off) = w1;
-            if (lane == 0) wp[j] = ldexpf(w[size_t(b) * H + j], -e);
-        }
-    }
-}
-
-// Sequence and rows of tile t; `b` is a cursor that only moves forward.
-__device__ __forceinline__ void tile_info(const int64_t *s_toff, const int64_t *s_seq, int B, int64_t t, int &b,
-                                          int64_t &row0, int64_t &row_end) {
-    while (b < B - 1 && t >= s_toff[b + 1]) ++b;
-    row0 = s_seq[b] + (t - s_toff[b]) * kRows;
-    row_end = s_seq[b + 1];
 }
 
 // cp.async of 16 bytes (zero-filled when src_bytes == 0) and its group controls.
@@ -177,7 +108,98 @@ __device__ __forceinline__ void cp_async_wait_group() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-constexpr int kGatherDepth = 3;   // listed mode: tiles of row gathers in flight per producer lane
+// ---------------------------------------------------------------------------
+// Query operand of one sequence, built by the 32 lanes of the producer warp
+// straight into a shared-memory slot, laid out exactly as the MMA reads it
+// (K-major, 128-byte swizzle: 16-byte chunk c of row j at chunk c ^ (j % 8)),
+// plus the gate weights w' the epilogue applies.
+//
+// bf16 keys: the bf16 query itself, w' = w.
+// e4m3 keys: per head j, a power-of-two scale 2^e_j brings max_c |q_jc| into
+// [128, 256); p1 = e4m3(q 2^e_j), p2 = e4m3(q 2^e_j - p1), both round to
+// nearest even.  A bf16 value has 8 significant bits, p1 carries 4 and the
+// remainder q 2^e_j - p1 is a multiple of the bf16 ulp no larger than 8 ulps,
+// so p2 holds it exactly whenever it is at least the e4m3 subnormal step 2^-9:
+// p1 + p2 == q 2^e_j for every element with |q| >= 2^-10 max_c |q_jc|, and
+// within 2^-10 of it (2^-17 max_c |q_jc| before scaling) otherwise.  The two
+// pieces are rows [0, H) and [H, 2H) of one operand.  w'_j = w_j 2^-e_j.
+// ---------------------------------------------------------------------------
+template <int KIND, int H>
+__device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, const float *__restrict__ wb, int d,
+                                            uint8_t *slot, float *wsm, int lane) {
+    if (KIND != E4M3_D128) {
+        const int cpr = d / 8;   // 16-byte chunks per row
+        const uint32_t s_u32 = smem_u32(slot);
+        for (int i0 = 0; i0 < H * cpr; i0 += 32 * 8) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u * 32 + lane;
+                if (i < H * cpr) {
+                    const int j = i / cpr, c = i % cpr;
+                    v[u] = *reinterpret_cast<const uint4 *>(qb + j * d + c * 8);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u * 32 + lane;
+                if (i < H * cpr) {
+                    const int j = i / cpr, c = i % cpr;
+                    const uint32_t dst = s_u32 + (c >> 3) * (H * 128) + j * 128 + (((c & 7) ^ (j & 7)) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[u].x), "r"(v[u].y),
+                                 "r"(v[u].z), "r"(v[u].w)
+                                 : "memory");
+                }
+            }
+        }
+        for (int j = lane; j < H; j += 32) wsm[j] = wb[j];
+    } else {
+        // lane owns channels 4*lane .. 4*lane+3 of every head; 8 heads per batch of loads
+        for (int j0 = 0; j0 < H; j0 += 8) {
+            uint2 raw[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) raw[u] = *reinterpret_cast<const uint2 *>(qb + (j0 + u) * 128 + 4 * lane);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + u;
+                const float v[4] = {__uint_as_float(raw[u].x << 16), __uint_as_float(raw[u].x & 0xFFFF0000u),
+                                    __uint_as_float(raw[u].y << 16), __uint_as_float(raw[u].y & 0xFFFF0000u)};
+                float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+                for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                int e = 0;
+                if (m > 0.f) {
+                    int E;
+                    frexpf(m, &E);
+                    e = 8 - E;
+                }
+                uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float s = ldexpf(v[c], e);
+                    const __nv_fp8_storage_t p1 = __nv_cvt_float_to_fp8(s, __NV_SATFINITE, __NV_E4M3);
+                    const __half_raw h1 = __nv_cvt_fp8_to_halfraw(p1, __NV_E4M3);
+                    const float r = s - __half2float(__half(h1));
+                    const __nv_fp8_storage_t p2 = __nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3);
+                    w0 |= uint32_t(p1) << (8 * c);
+                    w1 |= uint32_t(p2) << (8 * c);
+                }
+                const int off = j * 128 + (((lane >> 2) ^ (j & 7)) << 4) + (lane & 3) * 4;
+                *reinterpret_cast<uint32_t *>(slot + off) = w0;
+                *reinterpret_cast<uint32_t *>(slot + H * 128 + off) = w1;
+                if (lane == 0) wsm[j] = ldexpf(wb[j], -e);
+            }
+        }
+    }
+}
+
+// Sequence and rows of tile t; `b` is a cursor that only moves forward.
+__device__ __forceinline__ void tile_info(const int64_t *s_toff, const int64_t *s_seq, int B, int64_t t, int &b,
+                                          int64_t &row0, int64_t &row_end) {
+    while (b < B - 1 && t >= s_toff[b + 1]) ++b;
+    row0 = s_seq[b] + (t - s_toff[b]) * kRows;
+    row_end = s_seq[b + 1];
+}
 
 // LISTED = false: every entry of every sequence (key tiles by TMA).
 // LISTED = true:  entries idx[idx_off[b] ..] of each sequence (rows gathered
@@ -186,32 +208,33 @@ constexpr int kGatherDepth = 3;   // listed mode: tiles of row gathers in flight
 template <int KIND, int H, bool LISTED>
 __global__ void __launch_bounds__(kThreads, 1)
 scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kbytes,
-        const uint8_t *__restrict__ img, const int64_t *__restrict__ seq_off, const int32_t *__restrict__ idx,
-        const int64_t *__restrict__ idx_off, int64_t list_cap, int B, const float *__restrict__ k_scale,
-        float *__restrict__ z, float *__restrict__ I, int32_t *err) {
+        const uint16_t *__restrict__ q, const float *__restrict__ w, int d, const int64_t *__restrict__ seq_off,
+        const int32_t *__restrict__ idx, const int64_t *__restrict__ idx_off, int64_t list_cap, int B,
+        const float *__restrict__ k_scale, float *__restrict__ z, float *__restrict__ I, int32_t *err) {
     using C = Cfg<KIND>;
     constexpr int S = C::kStages;
     constexpr int QIMG = qimg_bytes<KIND, H>();
-    constexpr int ISTRIDE = img_stride<KIND, H>();
-    constexpr uint32_t NCOL = tmem_cols(H);
+    constexpr int AC = acc_cols(KIND, H);
+    constexpr uint32_t NCOL = tmem_cols(AC);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stages = smem;
-    uint8_t *qimg = stages + S * C::kStageBytes;
+    uint8_t *qimg = stages + S * C::kStageBytes;                  // 2 query slots
     uint64_t *full = reinterpret_cast<uint64_t *>(qimg + 2 * QIMG);
     uint64_t *empty = full + S;
-    uint64_t *qfull = empty + S;
-    uint64_t *qempty = qfull + 2;
-    uint64_t *tfull = qempty + 2;
+    uint64_t *qfull = empty + S;                                  // [2] by slot
+    uint64_t *qrel = qfull + 2;                                   // [kRel] by sequence ordinal
+    uint64_t *tfull = qrel + kRel;
     uint64_t *tempty = tfull + kAcc;
     uint64_t *drain = tempty + kAcc;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-    // [8 epilogue warps][H] gate weights, read as float4: 16-byte aligned
-    float *wbuf = reinterpret_cast<float *>((reinterpret_cast<uintptr_t>(tmem_slot + 4) + 15) & ~uintptr_t(15));
-    int64_t *s_seq = reinterpret_cast<int64_t *>(wbuf + 8 * H);  // [B+1]
-    int64_t *s_toff = s_seq + (B + 1);                           // [B+1]
+    int *s_nord = abort_flag + 1;                                 // sequences (ordinals) in this CTA's range
+    // gate weights of the two slots, read as float4: 16-byte aligned
+    float *wsm = reinterpret_cast<float *>((reinterpret_cast<uintptr_t>(tmem_slot + 4) + 15) & ~uintptr_t(15));
+    int64_t *s_seq = reinterpret_cast<int64_t *>(wsm + 2 * H);   // [B+1] tile-axis offsets
+    int64_t *s_toff = s_seq + (B + 1);                           // [B+1] first tile of each sequence
     int64_t *s_base = s_toff + (B + 1);                          // [B+1] entry base (listed mode)
     __shared__ int64_t s_range[2];
 
@@ -235,11 +258,17 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             }
         }
         const int64_t T = acc;
-        s_range[0] = T * blockIdx.x / gridDim.x;
-        s_range[1] = T * (blockIdx.x + 1) / gridDim.x;
+        const int64_t t0 = T * blockIdx.x / gridDim.x, t1 = T * (blockIdx.x + 1) / gridDim.x;
+        s_range[0] = t0;
+        s_range[1] = t1;
+        int nord = 0;   // sequences that own tiles in [t0, t1)
+        for (int b = 0; b < B; ++b)
+            if (s_toff[b + 1] > s_toff[b] && s_toff[b + 1] > t0 && s_toff[b] < t1) ++nord;
+        *s_nord = nord;
         *abort_flag = 0;
         for (int s = 0; s < S; ++s) { mbar_init(&full[s], LISTED ? 32 : 1); mbar_init(&empty[s], 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 1); }
+        for (int s = 0; s < 2; ++s) mbar_init(&qfull[s], 1);
+        for (int s = 0; s < kRel; ++s) mbar_init(&qrel[s], 1 + kEpiWarps);
         for (int s = 0; s < kAcc; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 4); }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -254,51 +283,67 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int64_t t0 = s_range[0], t1 = s_range[1];
+    const int nord = *s_nord;
     pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        // builds the query operand of a new sequence (ordinal o) into slot o & 1
+        auto next_query = [&](int b, int o) -> bool {
+            bool ok = true;
+            if (o >= 2)   // slot o & 1 last served ordinal o - 2: wait until every reader released it
+                ok = mbar_wait(&qrel[(o - 2) % kRel], uint32_t(((o - 2) / kRel) & 1), abort_v, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) return false;
+            build_query<KIND, H>(q + size_t(b) * H * d, w + size_t(b) * H, d, qimg + (o & 1) * QIMG,
+                                 wsm + (o & 1) * H, lane);
+            fence_proxy_async_smem();   // generic-proxy smem writes -> tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&qfull[o & 1]);
+            return true;
+        };
         if (!LISTED) {
+            // the keys do not depend on the preceding kernel: fill the ring first
+            const int64_t npre = (t1 - t0) < S ? (t1 - t0) : S;
             if (lane == 0) {
-                // the keys do not depend on the preceding prep kernel: fill the ring before waiting for it
-                const int64_t npre = (t1 - t0) < S ? (t1 - t0) : S;
-                {
-                    int bp = 0;
-                    int64_t r0, r1;
-                    for (int64_t t = t0; t < t0 + npre; ++t) {
-                        tile_info(s_toff, s_seq, B, t, bp, r0, r1);
-                        const int st = int(t - t0);
-                        mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+                int bp = 0;
+                int64_t r0, r1;
+                for (int64_t t = t0; t < t0 + npre; ++t) {
+                    tile_info(s_toff, s_seq, B, t, bp, r0, r1);
+                    const int st = int(t - t0);
+                    mbar_arrive_expect_tx(&full[st], C::kStageBytes);
 #pragma unroll
-                        for (int bx = 0; bx < C::kBoxes; ++bx)
-                            tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64,
-                                        int(r0));
-                    }
+                    for (int bx = 0; bx < C::kBoxes; ++bx)
+                        tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64,
+                                    int(r0));
                 }
-                pdl_wait();   // the q image comes from the preceding prep kernel
-                int b = 0, cur = -1, qn = 0, st = 0;
-                uint32_t ph = 0;
-                int64_t row0, row_end;
-                for (int64_t t = t0; t < t1; ++t) {
-                    tile_info(s_toff, s_seq, B, t, b, row0, row_end);
-                    if (b != cur) {
-                        const int slot = qn & 1;
-                        if (!mbar_wait(&qempty[slot], ((qn >> 1) & 1) ^ 1, abort_v, kWaitLimitNs)) break;
-                        mbar_arrive_expect_tx(&qfull[slot], QIMG);
-                        bulk_load(qimg + slot * QIMG, img + size_t(b) * ISTRIDE, QIMG, &qfull[slot]);
-                        cur = b;
-                        ++qn;
-                    }
-                    if (t - t0 >= npre) {   // the first npre tiles were issued above
-                        if (!mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs)) break;
-                        mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+            }
+            pdl_wait();
+            int b = 0, cur = -1, qn = 0, st = 0;
+            uint32_t ph = 0;
+            int64_t row0, row_end;
+            for (int64_t t = t0; t < t1; ++t) {
+                tile_info(s_toff, s_seq, B, t, b, row0, row_end);
+                if (b != cur) {
+                    if (!next_query(b, qn)) break;
+                    cur = b;
+                    ++qn;
+                }
+                bool ok = true;
+                if (t - t0 >= npre) {   // the first npre tiles were issued above
+                    if (lane == 0) {
+                        ok = mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs);
+                        if (ok) {
+                            mbar_arrive_expect_tx(&full[st], C::kStageBytes);
 #pragma unroll
-                        for (int bx = 0; bx < C::kBoxes; ++bx)
-                            tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64,
-                                        int(row0));
+                            for (int bx = 0; bx < C::kBoxes; ++bx)
+                                tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64,
+                                            int(row0));
+                        }
                     }
-                    if (++st == S) { st = 0; ph ^= 1; }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
                 }
+                if (!ok) break;
+                if (++st == S) { st = 0; ph ^= 1; }
             }
         } else {
             // all 32 lanes gather: lane owns rows lane, lane+32, lane+64, lane+96 of each tile
@@ -312,21 +357,12 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             int npend = 0, head = 0;
             for (int64_t t = t0; t < t1; ++t) {
                 tile_info(s_toff, s_seq, B, t, b, row0, row_end);
-                bool ok = true;
                 if (b != cur) {
-                    if (lane == 0) {
-                        const int slot = qn & 1;
-                        ok = mbar_wait(&qempty[slot], ((qn >> 1) & 1) ^ 1, abort_v, kWaitLimitNs);
-                        if (ok) {
-                            mbar_arrive_expect_tx(&qfull[slot], QIMG);
-                            bulk_load(qimg + slot * QIMG, img + size_t(b) * ISTRIDE, QIMG, &qfull[slot]);
-                        }
-                    }
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!next_query(b, qn)) break;
                     cur = b;
                     ++qn;
                 }
-                if (ok) ok = mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs);
+                const bool ok = mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 const uint32_t stage_u32 = smem_u32(stages + st * C::kStageBytes);
 #pragma unroll
@@ -364,7 +400,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC = KIND == E4M3_D128 ? idesc_e4m3(kRows, H) : idesc_bf16(kRows, H);
+            constexpr uint32_t IDESC = KIND == E4M3_D128 ? idesc_e4m3(kRows, AC) : idesc_bf16(kRows, AC);
             int b = 0, cur = -1, qn = 0, slot = 0, st = 0, acc = 0;
             uint32_t ph = 0, aph = 0;
             int64_t row0, row_end;
@@ -387,7 +423,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 if (!mbar_wait(&tempty[acc], aph ^ 1, abort_v, kWaitLimitNs)) break;
                 if (!mbar_wait(&full[st], ph, abort_v, kWaitLimitNs)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + uint32_t(acc * H);
+                const uint32_t d_tmem = tmem_base + uint32_t(acc * AC);
                 const uint32_t a0 = smem_u32(stages + st * C::kStageBytes);
                 const uint32_t b0 = smem_u32(qimg + slot * QIMG);
                 if (KIND == BF16_D128) {
@@ -400,17 +436,15 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                     for (int kk = 0; kk < 4; ++kk)
                         mma_f16(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), IDESC, kk > 0);
                 } else {
+                    // B = the two query pieces stacked as 2H rows (adjacent in the slot)
 #pragma unroll
-                    for (int p = 0; p < 2; ++p)
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_f8(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + p * (H * 128) + kk * 32),
-                                   IDESC, (p | kk) != 0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f8(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), IDESC, kk != 0);
                 }
                 issued = true;
                 mma_commit(&empty[st]);
                 mma_commit(&tfull[acc]);
-                if (bn != b) mma_commit(&qempty[slot]);
+                if (bn != b) mma_commit(&qrel[(qn - 1) % kRel]);   // this sequence's operand is no longer read
                 if (++st == S) { st = 0; ph ^= 1; }
                 if (++acc == kAcc) { acc = 0; aph ^= 1; }
             }
@@ -426,8 +460,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         const int ew = warp - 2;              // 0..7
         const int grp = ew >> 2;              // warpgroup: takes tiles t0 + grp, t0 + grp + 2, ...
         const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
-        float *wq = wbuf + ew * H;
-        int b = 0, cur = -1;
+        int b = 0, cur = -1, ord = -1, released = 0;
         int64_t row0, row_end;
         // row scale of this thread's row in tile t (e4m3 keys), loaded one tile of this group ahead
         auto scale_of = [&](int64_t t) -> float {
@@ -439,32 +472,57 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             if (r >= r1) return 1.f;
             return __ldg(k_scale + (LISTED ? s_base[bb] + idx[r] : r));
         };
-        pdl_wait();   // gate weights come from the preceding prep kernel
+        // a sequence ordinal this warp will not read again frees its slot (1 of the 8 epilogue arrivals)
+        auto release_to = [&](int upto) {
+            for (; released < upto; ++released)
+                if (lane == 0) mbar_arrive(&qrel[released % kRel]);
+        };
         float sc_next = scale_of(t0 + grp);
+        // ordinal of each tile: count the sequence changes over every tile of the range (both groups')
+        int ob = 0, ocur = -1, onum = -1;
+        int64_t orow0, orow1, u_next = t0;
+        bool ok = true;
         for (int64_t t = t0 + grp; t < t1; t += kEpiGroups) {
             const int64_t i = t - t0;         // local tile index: accumulator i % 4, its (i / 4)-th use
             const int acc = int(i % kAcc);
             const uint32_t aph = uint32_t((i / kAcc) & 1);
+            for (; u_next <= t; ++u_next) {
+                tile_info(s_toff, s_seq, B, u_next, ob, orow0, orow1);
+                if (ob != ocur) { ocur = ob; ++onum; }
+            }
             tile_info(s_toff, s_seq, B, t, b, row0, row_end);
             if (b != cur) {
-                __syncwarp();
-                const float *wsrc = reinterpret_cast<const float *>(img + size_t(b) * ISTRIDE + QIMG);
-                for (int j = lane; j < H; j += 32) wq[j] = wsrc[j];
-                __syncwarp();
                 cur = b;
+                ord = onum;
+                release_to(ord);   // earlier sequences: this warp is done with them
+                // the gate weights of this sequence were written before the producer's arrival
+                ok = mbar_wait(&qfull[ord & 1], uint32_t((ord >> 1) & 1), abort_v, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) break;
             }
+            const float *wq = wsm + (ord & 1) * H;
             const int64_t row = row0 + quarter * 32 + lane;   // entry (full) or list position (listed)
             const float sc = sc_next;
             sc_next = scale_of(t + kEpiGroups);
-            const bool ok = mbar_wait(&tfull[acc], aph, abort_v, kWaitLimitNs);
+            ok = mbar_wait(&tfull[acc], aph, abort_v, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
             tc_fence_after();
             uint32_t r[H];
-            const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * H);
+            const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * AC);
 #pragma unroll
             for (int c = 0; c < H / 16; ++c)
                 tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[c * 16]));
             tmem_ld_wait();
+            if (KIND == E4M3_D128) {   // add the second piece's products, 16 columns at a time
+#pragma unroll
+                for (int c = 0; c < H / 16; ++c) {
+                    uint32_t r2[16];
+                    tmem_ld_32x32b_x16(taddr + H + c * 16, r2);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int u = 0; u < 16; ++u)
+                        r[c * 16 + u] = __float_as_uint(__uint_as_float(r[c * 16 + u]) + __uint_as_float(r2[u]));
+                }
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -483,6 +541,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 if (I) I[row] = 1.f / (1.f + expf(-zs));
             }
         }
+        release_to(nord);   // every sequence of the range
     }
     __syncwarp();   // lanes that skipped a role loop wait for their lane 0 here
     __syncthreads();
@@ -517,13 +576,13 @@ template <int KIND, int H>
 size_t smem_bytes(int B) {
     using C = Cfg<KIND>;
     return 1024 + size_t(C::kStages) * C::kStageBytes + 2 * qimg_bytes<KIND, H>() +
-           (2 * C::kStages + 4 + 2 * kAcc + 1) * 8 + 16 + 16 + 8 * H * 4 + size_t(B + 1) * 24 + 64;
+           (2 * C::kStages + 2 + kRel + 2 * kAcc + 1) * 8 + 16 + 16 + 2 * H * 4 + size_t(B + 1) * 24 + 64;
 }
 
 template <int KIND, int H>
 lsa_status launch(const void *q, const float *w, const void *k, const float *k_scale, const int64_t *seq_off,
                   int64_t n_total, const int32_t *idx, const int64_t *idx_off, int64_t list_cap, int B, int d,
-                  float *z, float *I, void *workspace, int32_t *err, cudaStream_t st) {
+                  float *z, float *I, int32_t *err, cudaStream_t st) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) {
         set_error("lsa_index_score: cuTensorMapEncodeTiled is unavailable");
@@ -543,17 +602,15 @@ lsa_status launch(const void *q, const float *w, const void *k, const float *k_s
         set_error("lsa_index_score: cuTensorMapEncodeTiled failed (%d)", int(r));
         return LSA_ERR_CUDA;
     }
-    uint8_t *img = static_cast<uint8_t *>(workspace);
-    scan_tc_prep<KIND, H><<<dim3(B, H / 8), 256, 0, st>>>(static_cast<const uint16_t *>(q), w, d, img);
-    LSA_LAUNCHED("scan_tc_prep");
     const size_t smem = smem_bytes<KIND, H>(B);
     auto kern = idx ? scan_tc<KIND, H, true> : scan_tc<KIND, H, false>;
-    LSA_CUDA(ensure_smem(kern, size_t(int(smem))));
+    LSA_CUDA(ensure_smem(kern, smem));
     const int64_t axis = idx ? list_cap : n_total;
     const int64_t max_tiles = (axis + kRows - 1) / kRows + B;
     const int grid = int(max_tiles < sm_count() ? max_tiles : sm_count());
     LSA_CUDA(launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, map, static_cast<const uint8_t *>(k),
-                        static_cast<const uint8_t *>(img), seq_off, idx, idx_off, list_cap, B, k_scale, z, I, err));
+                        static_cast<const uint16_t *>(q), w, d, seq_off, idx, idx_off, list_cap, B, k_scale, z, I,
+                        err));
     LSA_LAUNCHED(idx ? "scan_tc_listed" : "scan_tc");
     return LSA_OK;
 }
@@ -561,21 +618,15 @@ lsa_status launch(const void *q, const float *w, const void *k, const float *k_s
 template <int KIND>
 lsa_status launch_h(int H, const void *q, const float *w, const void *k, const float *k_scale,
                     const int64_t *seq_off, int64_t n_total, const int32_t *idx, const int64_t *idx_off,
-                    int64_t list_cap, int B, int d, float *z, float *I, void *ws, int32_t *err, cudaStream_t st) {
+                    int64_t list_cap, int B, int d, float *z, float *I, int32_t *err, cudaStream_t st) {
     switch (H) {
-    case 16: return launch<KIND, 16>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, ws, err, st);
-    case 32: return launch<KIND, 32>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, ws, err, st);
-    default: return launch<KIND, 64>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, ws, err, st);
+    case 16: return launch<KIND, 16>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err, st);
+    case 32: return launch<KIND, 32>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err, st);
+    default: return launch<KIND, 64>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err, st);
     }
 }
 
 }  // namespace
-
-size_t index_score_tc_workspace(int32_t B, int32_t H, int32_t d) {
-    // the largest image stride of the shapes this path runs (256 bytes per head + tail)
-    (void)d;
-    return size_t(B) * (size_t(256) * H + kImgTail) + 256;
-}
 
 bool index_score_tc_supported(lsa_dtype q_dtype, lsa_dtype k_dtype, int64_t n_total, int32_t B, int32_t H,
                               int32_t d) {
@@ -589,16 +640,14 @@ bool index_score_tc_supported(lsa_dtype q_dtype, lsa_dtype k_dtype, int64_t n_to
 lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, lsa_dtype k_dtype,
                                  const float *k_scale, const int64_t *seq_off, int64_t n_total,
                                  const int32_t *idx, const int64_t *idx_off, int64_t list_cap, int32_t B,
-                                 int32_t H, int32_t d, float *z, float *I, void *workspace, int32_t *err,
-                                 cudaStream_t st) {
+                                 int32_t H, int32_t d, float *z, float *I, int32_t *err, cudaStream_t st) {
     if (k_dtype == LSA_E4M3)
-        return launch_h<E4M3_D128>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I,
-                                   workspace, err, st);
+        return launch_h<E4M3_D128>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err,
+                                   st);
     if (d == 128)
-        return launch_h<BF16_D128>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I,
-                                   workspace, err, st);
-    return launch_h<BF16_D64>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I,
-                              workspace, err, st);
+        return launch_h<BF16_D128>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err,
+                                   st);
+    return launch_h<BF16_D64>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err, st);
 }
 
 }  // namespace lsa

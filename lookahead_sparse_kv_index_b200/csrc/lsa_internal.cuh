@@ -84,15 +84,13 @@ lsa_status launch_index_score(const void *q, lsa_dtype q_dtype, const float *w, 
                               lsa_dtype k_dtype, const float *k_scale, const int64_t *seq_off,
                               int64_t n_total, const int32_t *idx, const int64_t *idx_off,
                               int64_t list_capacity, int32_t B, int32_t H, int32_t d, float *z,
-                              float *I, void *workspace, int32_t *err, cudaStream_t st);
-size_t index_score_tc_workspace(int32_t B, int32_t H, int32_t d);
+                              float *I, int32_t flags, int32_t *err, cudaStream_t st);
 bool index_score_tc_supported(lsa_dtype q_dtype, lsa_dtype k_dtype, int64_t n_total, int32_t B, int32_t H,
                               int32_t d);
 lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, lsa_dtype k_dtype,
                                  const float *k_scale, const int64_t *seq_off, int64_t n_total,
                                  const int32_t *idx, const int64_t *idx_off, int64_t list_cap, int32_t B,
-                                 int32_t H, int32_t d, float *z, float *I, void *workspace, int32_t *err,
-                                 cudaStream_t st);
+                                 int32_t H, int32_t d, float *z, float *I, int32_t *err, cudaStream_t st);
 lsa_status launch_select(const float *z, const int64_t *seq_off, int64_t n_total, int32_t B,
                          int32_t *kept_idx, int64_t capacity, int64_t *kept_off, uint32_t *mask,
                          void *workspace, int32_t *err, cudaStream_t st);

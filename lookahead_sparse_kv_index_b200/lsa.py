@@ -31,7 +31,7 @@ N_STAGES = 6
 
 # every symbol include/lsa.h declares
 EXPORTS = [
-    "lsa_version", "lsa_last_error", "lsa_status_name", "lsa_index_score_workspace_size", "lsa_index_score",
+    "lsa_version", "lsa_last_error", "lsa_status_name", "lsa_index_score",
     "lsa_select_workspace_size", "lsa_select_noalloc_max_entries", "lsa_select_noalloc",
     "lsa_select", "lsa_topk", "lsa_gather", "lsa_sparse_attn_workspace_size", "lsa_sparse_attn",
     "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
@@ -72,8 +72,8 @@ def _sig(name, res, args):
 _sig("lsa_version", i32, [])
 _sig("lsa_last_error", ctypes.c_char_p, [])
 _sig("lsa_status_name", ctypes.c_char_p, [i32])
-_sig("lsa_index_score_workspace_size", sz, [i32, i32, i32])
-_sig("lsa_index_score", i32, [P, i32, P, P, i32, P, P, i64, P, P, i64, i32, i32, i32, P, P, P, sz, P, P])
+_sig("lsa_index_score", i32, [P, i32, P, P, i32, P, P, i64, P, P, i64, i32, i32, i32, P, P, i32, P, P])
+SCORE_CUDA_CORE = 1
 _sig("lsa_select_workspace_size", sz, [i64])
 _sig("lsa_select", i32, [P, P, i64, i32, P, i64, P, P, P, sz, P, P])
 _sig("lsa_select_noalloc_max_entries", i64, [])
@@ -121,17 +121,13 @@ def version() -> int:
 
 # ------------------------------------------------------------------ stages
 
-def index_score_workspace_size(B, H, d) -> int:
-    return int(_L.lsa_index_score_workspace_size(B, H, d))
-
-
 def index_score(q, q_dtype, w, k, k_dtype, k_scale, seq_off, n_total, H, d, z, I=None, idx=None, idx_off=None,
-                list_capacity=0, workspace=None, err=None, stream=None):
+                list_capacity=0, cuda_core=False, err=None, stream=None):
+    """Lookahead index score; cuda_core=True forces the CUDA-core kernel (else tcgen05 where supported)."""
     B = seq_off.numel() - 1
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_L.lsa_index_score(_ptr(q), DTYPE[q_dtype], _ptr(w), _ptr(k), DTYPE[k_dtype], _ptr(k_scale),
                               _ptr(seq_off), n_total, _ptr(idx), _ptr(idx_off), list_capacity, B, H, d,
-                              _ptr(z), _ptr(I), _ptr(workspace), ws_bytes, _ptr(err), _stream(stream)),
+                              _ptr(z), _ptr(I), SCORE_CUDA_CORE if cuda_core else 0, _ptr(err), _stream(stream)),
            "lsa_index_score")
 
 

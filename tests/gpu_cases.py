@@ -44,15 +44,13 @@ def unpack_mask(words: np.ndarray, n: int) -> np.ndarray:
 
 
 def gpu_full_scores(wl, dev, lsa, want_I=True, tc=False):
-    """Full scan; tc=True passes the workspace that enables the tensor-core kernel."""
+    """Full scan; tc=False forces the CUDA-core kernel (tc=True: tcgen05 where the shape is supported)."""
     n = wl.n_total
     z = torch.full((max(n, 1) + 64,), 77.0, dtype=torch.float32, device="cuda")
     I = torch.empty_like(z) if want_I else None
-    ws = (torch.empty(lsa.index_score_workspace_size(wl.B, wl.H, wl.d), dtype=torch.uint8, device="cuda")
-          if tc else None)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     lsa.index_score(dev["q"], wl.q_dtype, dev["w"], dev["keys"], wl.key_dtype, dev["k_scale"], dev["seq_off"], n,
-                    wl.H, wl.d, z, I, workspace=ws, err=err)
+                    wl.H, wl.d, z, I, cuda_core=not tc, err=err)
     torch.cuda.synchronize()
     assert err.item() == 0, f"device error {err.item()}"
     assert (z[n:].cpu().numpy() == 77.0).all(), "scan wrote past the entry axis"

@@ -42,8 +42,6 @@ def test_version_and_status_names(lsa):
 
 
 def test_workspace_sizes(lsa):
-    assert lsa.index_score_workspace_size(4, 64, 128) >= 4 * (64 * 256 + 64 * 4)
-    assert lsa.index_score_workspace_size(0, 64, 128) == 0
     assert lsa.select_workspace_size(0) == 0
     assert lsa.select_workspace_size(1) >= 16
     n = 4 * 131072
@@ -54,17 +52,17 @@ def test_workspace_sizes(lsa):
 
 def _score(lsa, **kw):
     a = dict(q=1 << 20, qd=1, w=1 << 20, k=1 << 20, kd=1, ks=None, so=1 << 20, n=100, idx=None, idxo=None,
-             cap=0, B=1, H=64, d=128, z=1 << 20, I=None, ws=None, wsb=0)
+             cap=0, B=1, H=64, d=128, z=1 << 20, I=None, flags=0)
     a.update(kw)
     return lsa.lib.lsa_index_score(a["q"], a["qd"], a["w"], a["k"], a["kd"], a["ks"], a["so"], a["n"], a["idx"],
-                                   a["idxo"], a["cap"], a["B"], a["H"], a["d"], a["z"], a["I"], a["ws"],
-                                   a["wsb"], None, None)
+                                   a["idxo"], a["cap"], a["B"], a["H"], a["d"], a["z"], a["I"], a["flags"], None,
+                                   None)
 
 
 @pytest.mark.parametrize("kw,status", [
     (dict(q=None), 1), (dict(z=None), 1), (dict(B=0), 1), (dict(H=65), 5), (dict(d=96), 5),
     (dict(kd=2), 1), (dict(ks=1 << 20), 1), (dict(k=(1 << 20) + 8), 1), (dict(qd=2), 5), (dict(qd=7), 1),
-    (dict(idx=1 << 20), 1), (dict(n=-1), 1), (dict(ws=1 << 20, wsb=100), 1), (dict(ws=(1 << 20) + 4, wsb=1 << 20), 1),
+    (dict(idx=1 << 20), 1), (dict(n=-1), 1), (dict(flags=2), 1), (dict(flags=-1), 1),
 ])
 def test_index_score_rejects_bad_arguments(lsa, kw, status):
     assert _score(lsa, **kw) == status

@@ -64,13 +64,11 @@ def test_index_score_listed_matches_oracle(lsa, name, tc):
     idx_off = np.concatenate([[0], np.cumsum([len(x) for x in lists])]).astype(np.int64)
     cap = int(idx_off[-1]) + 5
     z = torch.full((cap,), 123.0, dtype=torch.float32, device="cuda")
-    ws = (torch.empty(lsa.index_score_workspace_size(wl.B, wl.H, wl.d), dtype=torch.uint8, device="cuda")
-          if tc else None)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     idx_d = torch.from_numpy(np.concatenate([idx, np.zeros(5, np.int32)])).cuda()   # list buffer of `cap` slots
     lsa.index_score(dev["q"], wl.q_dtype, dev["w"], dev["keys"], wl.key_dtype, dev["k_scale"], dev["seq_off"],
                     wl.n_total, wl.H, wl.d, z, None, idx=idx_d, idx_off=torch.from_numpy(idx_off).cuda(),
-                    list_capacity=cap, workspace=ws, err=err)
+                    list_capacity=cap, cuda_core=not tc, err=err)
     torch.cuda.synchronize()
     assert err.item() == 0
     z = z.cpu().numpy()
