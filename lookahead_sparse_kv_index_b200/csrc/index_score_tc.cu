@@ -9,8 +9,10 @@
 // never straddle two sequences):
 //   * warp 0 (producer): TMA loads of key tiles (128-byte swizzle) into a smem
 //     ring -- the first ring's worth before anything else -- and, on every
-//     sequence change, builds that sequence's query operand and gate weights
-//     in one of two smem slots (no separate preparation kernel);
+//     sequence change from the third sequence on, builds that sequence's query
+//     operand and gate weights in one of two smem slots (the first two are
+//     built by the epilogue warps while the first keys load; no separate
+//     preparation kernel);
 //   * warp 1: tcgen05.mma, M = 128 entries, N = H heads (bf16 keys) or 2H
 //     (e4m3 keys: both query pieces at once), into one of four TMEM
 //     accumulators;
@@ -126,23 +128,25 @@ __device__ __forceinline__ void cp_async_wait_group() {
 // ---------------------------------------------------------------------------
 template <int KIND, int H>
 __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, const float *__restrict__ wb, int d,
-                                            uint8_t *slot, float *wsm, int lane) {
+                                            uint8_t *slot, float *wsm, int wi, int nw, int lane) {
     if (KIND != E4M3_D128) {
-        const int cpr = d / 8;   // 16-byte chunks per row
+        // 16-byte chunks, all of a thread's loads in flight before its stores
+        const int cpr = d / 8;
+        const int tid = wi * 32 + lane, nthr = nw * 32;
         const uint32_t s_u32 = smem_u32(slot);
-        for (int i0 = 0; i0 < H * cpr; i0 += 32 * 8) {
-            uint4 v[8];
+        for (int i0 = 0; i0 < H * cpr; i0 += nthr * 16) {
+            uint4 v[16];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = i0 + u * 32 + lane;
+            for (int u = 0; u < 16; ++u) {
+                const int i = i0 + u * nthr + tid;
                 if (i < H * cpr) {
                     const int j = i / cpr, c = i % cpr;
                     v[u] = *reinterpret_cast<const uint4 *>(qb + j * d + c * 8);
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = i0 + u * 32 + lane;
+            for (int u = 0; u < 16; ++u) {
+                const int i = i0 + u * nthr + tid;
                 if (i < H * cpr) {
                     const int j = i / cpr, c = i % cpr;
                     const uint32_t dst = s_u32 + (c >> 3) * (H * 128) + j * 128 + (((c & 7) ^ (j & 7)) << 4);
@@ -152,16 +156,20 @@ __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, con
                 }
             }
         }
-        for (int j = lane; j < H; j += 32) wsm[j] = wb[j];
+        for (int j = wi * 32 + lane; j < H; j += nw * 32) wsm[j] = wb[j];
     } else {
-        // lane owns channels 4*lane .. 4*lane+3 of every head; 8 heads per batch of loads
-        for (int j0 = 0; j0 < H; j0 += 8) {
+        // warp wi owns heads wi, wi + nw, ...; lane owns channels 4*lane .. 4*lane+3; 8 heads per batch
+        for (int j0 = wi; j0 < H; j0 += 8 * nw) {
             uint2 raw[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) raw[u] = *reinterpret_cast<const uint2 *>(qb + (j0 + u) * 128 + 4 * lane);
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + u * nw;
+                if (j < H) raw[u] = *reinterpret_cast<const uint2 *>(qb + j * 128 + 4 * lane);
+            }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int j = j0 + u;
+                const int j = j0 + u * nw;
+                if (j >= H) break;
                 const float v[4] = {__uint_as_float(raw[u].x << 16), __uint_as_float(raw[u].x & 0xFFFF0000u),
                                     __uint_as_float(raw[u].y << 16), __uint_as_float(raw[u].y & 0xFFFF0000u)};
                 float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
@@ -176,10 +184,10 @@ __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, con
                 uint32_t w0 = 0, w1 = 0;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const float s = ldexpf(v[c], e);
-                    const __nv_fp8_storage_t p1 = __nv_cvt_float_to_fp8(s, __NV_SATFINITE, __NV_E4M3);
+                    const float sv = ldexpf(v[c], e);
+                    const __nv_fp8_storage_t p1 = __nv_cvt_float_to_fp8(sv, __NV_SATFINITE, __NV_E4M3);
                     const __half_raw h1 = __nv_cvt_fp8_to_halfraw(p1, __NV_E4M3);
-                    const float r = s - __half2float(__half(h1));
+                    const float r = sv - __half2float(__half(h1));
                     const __nv_fp8_storage_t p2 = __nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3);
                     w0 |= uint32_t(p1) << (8 * c);
                     w1 |= uint32_t(p2) << (8 * c);
@@ -289,13 +297,15 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         // builds the query operand of a new sequence (ordinal o) into slot o & 1
+        // (ordinals 0 and 1 are built by the epilogue warps, idle at kernel start)
         auto next_query = [&](int b, int o) -> bool {
+            if (o < 2) return true;
             bool ok = true;
             if (o >= 2)   // slot o & 1 last served ordinal o - 2: wait until every reader released it
                 ok = mbar_wait(&qrel[(o - 2) % kRel], uint32_t(((o - 2) / kRel) & 1), abort_v, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) return false;
             build_query<KIND, H>(q + size_t(b) * H * d, w + size_t(b) * H, d, qimg + (o & 1) * QIMG,
-                                 wsm + (o & 1) * H, lane);
+                                 wsm + (o & 1) * H, 0, 1, lane);
             fence_proxy_async_smem();   // generic-proxy smem writes -> tensor core
             __syncwarp();
             if (lane == 0) mbar_arrive(&qfull[o & 1]);
@@ -401,19 +411,17 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC = KIND == E4M3_D128 ? idesc_e4m3(kRows, AC) : idesc_bf16(kRows, AC);
+            // descriptors of stage 0 and slot 0; the others differ only in the start address field
+            const uint64_t a_desc0 = desc_sw128(smem_u32(stages));
+            const uint64_t b_desc0 = desc_sw128(smem_u32(qimg));
             int b = 0, cur = -1, qn = 0, slot = 0, st = 0, acc = 0;
             uint32_t ph = 0, aph = 0;
             int64_t row0, row_end;
             bool issued = false;
             for (int64_t t = t0; t < t1; ++t) {
                 tile_info(s_toff, s_seq, B, t, b, row0, row_end);
-                int bn = -1;
-                if (t + 1 < t1) {
-                    int bb = b;
-                    int64_t r0, r1;
-                    tile_info(s_toff, s_seq, B, t + 1, bb, r0, r1);
-                    bn = bb;
-                }
+                // the next tile starts a new sequence when it is the first tile of a later one
+                const bool last_of_seq = (t + 1 >= t1) || (t + 1 >= s_toff[b + 1]);
                 if (b != cur) {
                     slot = qn & 1;
                     if (!mbar_wait(&qfull[slot], (qn >> 1) & 1, abort_v, kWaitLimitNs)) break;
@@ -424,27 +432,30 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 if (!mbar_wait(&full[st], ph, abort_v, kWaitLimitNs)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + uint32_t(acc * AC);
-                const uint32_t a0 = smem_u32(stages + st * C::kStageBytes);
-                const uint32_t b0 = smem_u32(qimg + slot * QIMG);
+                // start-address field advances in 16-byte units
+                const uint64_t a_desc = a_desc0 + uint64_t((st * C::kStageBytes) >> 4);
+                const uint64_t b_desc = b_desc0 + uint64_t((slot * QIMG) >> 4);
                 if (KIND == BF16_D128) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_f16(d_tmem, desc_sw128(a0 + (kk >> 2) * 16384 + (kk & 3) * 32),
-                                desc_sw128(b0 + (kk >> 2) * (H * 128) + (kk & 3) * 32), IDESC, kk > 0);
+                        mma_f16(d_tmem, a_desc + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                                b_desc + uint64_t(((kk >> 2) * (H * 128) + (kk & 3) * 32) >> 4), IDESC, kk > 0);
                 } else if (KIND == BF16_D64) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f16(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), IDESC, kk > 0);
+                        mma_f16(d_tmem, a_desc + uint64_t((kk * 32) >> 4), b_desc + uint64_t((kk * 32) >> 4), IDESC,
+                                kk > 0);
                 } else {
                     // B = the two query pieces stacked as 2H rows (adjacent in the slot)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f8(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), IDESC, kk != 0);
+                        mma_f8(d_tmem, a_desc + uint64_t((kk * 32) >> 4), b_desc + uint64_t((kk * 32) >> 4), IDESC,
+                               kk != 0);
                 }
                 issued = true;
                 mma_commit(&empty[st]);
                 mma_commit(&tfull[acc]);
-                if (bn != b) mma_commit(&qrel[(qn - 1) % kRel]);   // this sequence's operand is no longer read
+                if (last_of_seq) mma_commit(&qrel[(qn - 1) % kRel]);   // this sequence's operand is no longer read
                 if (++st == S) { st = 0; ph ^= 1; }
                 if (++acc == kAcc) { acc = 0; aph ^= 1; }
             }
@@ -477,6 +488,25 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             for (; released < upto; ++released)
                 if (lane == 0) mbar_arrive(&qrel[released % kRel]);
         };
+        if (nord > 0) {
+            // the query operands of ordinals 0 and 1 (slots 0 and 1), built by all 8 epilogue warps
+            // while the first keys load, so that no CTA's producer stalls at its first sequence change
+            int bo = 0;
+            int64_t r0, r1;
+            tile_info(s_toff, s_seq, B, t0, bo, r0, r1);
+            pdl_wait();   // the query and gate weights may come from the preceding kernel
+            for (int o = 0; o < 2 && o < nord; ++o) {
+                if (o == 1) {   // the next sequence that owns tiles
+                    ++bo;
+                    while (bo < B - 1 && s_toff[bo + 1] == s_toff[bo]) ++bo;
+                }
+                build_query<KIND, H>(q + size_t(bo) * H * d, w + size_t(bo) * H, d, qimg + o * QIMG, wsm + o * H,
+                                     ew, kEpiWarps, lane);
+                fence_proxy_async_smem();
+                named_barrier(2, kEpiWarps * 32);
+                if (ew == 0 && lane == 0) mbar_arrive(&qfull[o]);
+            }
+        }
         float sc_next = scale_of(t0 + grp);
         // ordinal of each tile: count the sequence changes over every tile of the range (both groups')
         int ob = 0, ocur = -1, onum = -1;
@@ -506,34 +536,52 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             ok = mbar_wait(&tfull[acc], aph, abort_v, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
             tc_fence_after();
-            uint32_t r[H];
             const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * AC);
-#pragma unroll
-            for (int c = 0; c < H / 16; ++c)
-                tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[c * 16]));
-            tmem_ld_wait();
-            if (KIND == E4M3_D128) {   // add the second piece's products, 16 columns at a time
-#pragma unroll
-                for (int c = 0; c < H / 16; ++c) {
-                    uint32_t r2[16];
-                    tmem_ld_32x32b_x16(taddr + H + c * 16, r2);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int u = 0; u < 16; ++u)
-                        r[c * 16 + u] = __float_as_uint(__uint_as_float(r[c * 16 + u]) + __uint_as_float(r2[u]));
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
             float zs = 0.f;
+            if (KIND != E4M3_D128) {
+                uint32_t r[H];
 #pragma unroll
-            for (int j = 0; j < H; j += 4) {
-                const float4 wv = *reinterpret_cast<const float4 *>(wq + j);
-                zs = fmaf(wv.x, fmaxf(__uint_as_float(r[j]), 0.f), zs);
-                zs = fmaf(wv.y, fmaxf(__uint_as_float(r[j + 1]), 0.f), zs);
-                zs = fmaf(wv.z, fmaxf(__uint_as_float(r[j + 2]), 0.f), zs);
-                zs = fmaf(wv.w, fmaxf(__uint_as_float(r[j + 3]), 0.f), zs);
+                for (int c = 0; c < H / 16; ++c)
+                    tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[c * 16]));
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+#pragma unroll
+                for (int j = 0; j < H; j += 4) {
+                    const float4 wv = *reinterpret_cast<const float4 *>(wq + j);
+                    zs = fmaf(wv.x, fmaxf(__uint_as_float(r[j]), 0.f), zs);
+                    zs = fmaf(wv.y, fmaxf(__uint_as_float(r[j + 1]), 0.f), zs);
+                    zs = fmaf(wv.z, fmaxf(__uint_as_float(r[j + 2]), 0.f), zs);
+                    zs = fmaf(wv.w, fmaxf(__uint_as_float(r[j + 3]), 0.f), zs);
+                }
+            } else {
+                // heads in halves of H/2: both pieces' columns of a half in one round trip
+                constexpr int HH = H / 2;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r1[HH], r2[HH];
+#pragma unroll
+                    for (int c = 0; c < HH / 16; ++c) {
+                        tmem_ld_32x32b_x16(taddr + half * HH + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&r1[c * 16]));
+                        tmem_ld_32x32b_x16(taddr + H + half * HH + c * 16,
+                                           *reinterpret_cast<uint32_t(*)[16]>(&r2[c * 16]));
+                    }
+                    tmem_ld_wait();
+                    if (half == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[acc]);
+                    }
+#pragma unroll
+                    for (int j = 0; j < HH; j += 4) {
+                        const float4 wv = *reinterpret_cast<const float4 *>(wq + half * HH + j);
+                        zs = fmaf(wv.x, fmaxf(__uint_as_float(r1[j]) + __uint_as_float(r2[j]), 0.f), zs);
+                        zs = fmaf(wv.y, fmaxf(__uint_as_float(r1[j + 1]) + __uint_as_float(r2[j + 1]), 0.f), zs);
+                        zs = fmaf(wv.z, fmaxf(__uint_as_float(r1[j + 2]) + __uint_as_float(r2[j + 2]), 0.f), zs);
+                        zs = fmaf(wv.w, fmaxf(__uint_as_float(r1[j + 3]) + __uint_as_float(r2[j + 3]), 0.f), zs);
+                    }
+                }
             }
             if (row < row_end) {
                 if (KIND == E4M3_D128) zs *= sc;
