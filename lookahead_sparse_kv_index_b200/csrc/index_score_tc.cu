@@ -5,20 +5,26 @@
 // Per sequence the q.k block is a dense contraction [entries x d] x [d x H]
 // (H = 64 heads, d = 128: 16 Kflop per entry), so the scan is HBM-bound only
 // when the dot products run on the tensor cores.  One kernel, persistent CTAs
-// (one per SM), each streaming a contiguous range of 128-entry tiles (tiles
-// never straddle two sequences):
+// (one per SM), each streaming a contiguous range of tiles (128 entries for
+// bf16 keys, 256 for e4m3 keys; tiles never straddle two sequences):
 //   * warp 0 (producer): TMA loads of key tiles (128-byte swizzle) into a smem
 //     ring -- the first ring's worth before anything else -- and, on every
 //     sequence change from the third sequence on, builds that sequence's query
 //     operand and gate weights in one of two smem slots (the first two are
 //     built by the epilogue warps while the first keys load; no separate
 //     preparation kernel);
-//   * warp 1: tcgen05.mma, M = 128 entries, N = H heads (bf16 keys) or 2H
-//     (e4m3 keys: both query pieces at once), into one of four TMEM
-//     accumulators;
-//   * warps 2-9: two epilogue warpgroups taking alternate tiles, one TMEM lane
-//     (= one entry) per thread: ReLU, gate weights, head sum in registers, one
-//     coalesced fp32 store per entry; the row scale is fetched one tile ahead.
+//   * warp 1: tcgen05.mma, M = 128 entries per instruction, into a ring of
+//     TMEM accumulators.  bf16 keys: N = H heads, the MMAs of two tiles issued
+//     interleaved.  e4m3 keys: N = 2H (both query pieces), the two 128-entry
+//     halves of a tile issued interleaved.  Issuing an MMA and passing a tile
+//     boundary both cost the single issuing thread far more than the small
+//     MMAs take on the tensor core, so the layout keeps MMAs per byte and
+//     tiles per byte low: 8 MMAs per 32 KB of keys in both cases;
+//   * warps 2-9: two epilogue warpgroups (alternate tiles for bf16 keys, the
+//     two halves of every tile for e4m3 keys), one TMEM lane (= one entry)
+//     per thread: the two pieces' products added (e4m3), ReLU, gate weights,
+//     head sum in registers, one coalesced fp32 store per entry; the row
+//     scale is fetched one tile ahead.
 // bf16 keys use kind::f16 (bf16 x bf16).  e4m3 keys use kind::f8f6f4 against
 // an exact two-piece e4m3 split of the bf16 query, so the keys go from HBM to
 // the tensor core untouched; the per-row key scale and the per-head
@@ -50,49 +56,80 @@ enum Kind { BF16_D128 = 0, BF16_D64 = 1, E4M3_D128 = 2 };
 
 template <int KIND>
 struct Cfg;
+// Per key type: a tile is kSub sub-tiles of 128 rows (one MMA row block each);
+// a stage holds one tile, loaded as kBoxes TMA boxes of 128 bytes x kBoxRows
+// rows; the query operand has kPieces x H rows (N of the MMA).
 template <>
 struct Cfg<BF16_D128> {
+    static constexpr int kSub = 1;
     static constexpr int kStageBytes = 32768;   // 128 rows x 128 bf16
     static constexpr int kBoxes = 2;            // two 64-element (128-byte) column boxes
+    static constexpr int kBoxRows = 128;
+    static constexpr int kPieces = 1;
     static constexpr int kQBytesPerHead = 256;
     static constexpr int kStages = 5;
 };
 template <>
 struct Cfg<BF16_D64> {
+    static constexpr int kSub = 1;
     static constexpr int kStageBytes = 16384;
     static constexpr int kBoxes = 1;
+    static constexpr int kBoxRows = 128;
+    static constexpr int kPieces = 1;
     static constexpr int kQBytesPerHead = 128;
     static constexpr int kStages = 8;
 };
 template <>
 struct Cfg<E4M3_D128> {
-    static constexpr int kStageBytes = 16384;   // 128 rows x 128 e4m3
+    static constexpr int kSub = 2;              // 256-row tiles: half as many tile steps per byte
+    static constexpr int kStageBytes = 32768;   // 256 rows x 128 e4m3
     static constexpr int kBoxes = 1;
+    static constexpr int kBoxRows = 256;
+    static constexpr int kPieces = 2;           // both query pieces in one N = 2H operand
     static constexpr int kQBytesPerHead = 256;  // two e4m3 pieces x 128
-    static constexpr int kStages = 8;
+    static constexpr int kStages = 5;
 };
 
 constexpr int kThreads = 320;         // warp 0 producer, warp 1 MMA, warps 2-9 epilogue (2 warpgroups)
 constexpr int kEpiGroups = 2;
 constexpr int kEpiWarps = 8;
 constexpr int kRel = 8;               // query-slot release barriers, by sequence ordinal mod kRel
-constexpr int kRows = 128;
-constexpr int kAcc = 4;               // TMEM accumulator stages
+constexpr int kRows = 128;            // rows of one MMA (M) and of a sub-tile
+constexpr int kAccMax = 8;            // TMEM accumulator stages at most
 constexpr int kMaxB = 512;            // sequences per launch on this path
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
 constexpr int kGatherDepth = 3;       // listed mode: tiles of row gathers in flight per producer lane
 
-// Accumulator width in TMEM columns: H for bf16 keys; 2H for e4m3 keys, whose MMA
-// multiplies by both query pieces at once (piece 1 -> columns [0,H), piece 2 ->
-// [H,2H)) and whose epilogue adds the two halves before the ReLU.
-__host__ __device__ constexpr int acc_cols(int KIND, int H) { return KIND == 2 ? 2 * H : H; }
-
+template <int KIND>
+__host__ __device__ constexpr int tile_rows() {
+    return kRows * Cfg<KIND>::kSub;
+}
+// TMEM columns of one sub-tile's accumulator (fp32, one per head and query
+// piece: e4m3 keys give columns [0, H) for piece 1 and [H, 2H) for piece 2,
+// added by the epilogue before the ReLU) and of one tile's.
+template <int KIND, int H>
+__host__ __device__ constexpr int sub_cols() {
+    return H * Cfg<KIND>::kPieces;
+}
+template <int KIND, int H>
+__host__ __device__ constexpr int tile_cols() {
+    return sub_cols<KIND, H>() * Cfg<KIND>::kSub;
+}
+// Tile accumulators held in TMEM (512 columns per SM).
+template <int KIND, int H>
+__host__ __device__ constexpr int acc_tiles() {
+    return 512 / tile_cols<KIND, H>() < kAccMax ? 512 / tile_cols<KIND, H>() : kAccMax;
+}
+// Tiles whose MMAs are issued together, interleaved so that consecutive MMAs
+// write different accumulators: a chain of MMAs into one accumulator waits on
+// each accumulation, independent chains overlap in the tensor pipe.  The two
+// halves of a 256-row tile already give two chains.
+template <int KIND, int H>
+__host__ __device__ constexpr int mma_group() {
+    return Cfg<KIND>::kSub == 2 ? 1 : 2;
+}
 __host__ __device__ constexpr uint32_t tmem_cols(int cols) {
-    return (kAcc * cols) <= 32    ? 32
-           : (kAcc * cols) <= 64  ? 64
-           : (kAcc * cols) <= 128 ? 128
-           : (kAcc * cols) <= 256 ? 256
-                                  : 512;
+    return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
 }
 
 template <int KIND, int H>
@@ -111,8 +148,9 @@ __device__ __forceinline__ void cp_async_wait_group() {
 }
 
 // ---------------------------------------------------------------------------
-// Query operand of one sequence, built by the 32 lanes of the producer warp
-// straight into a shared-memory slot, laid out exactly as the MMA reads it
+// Query operand of one sequence, built by nw warps (the 8 epilogue warps at
+// kernel start, the producer warp later) straight into a shared-memory slot,
+// laid out exactly as the MMA reads it
 // (K-major, 128-byte swizzle: 16-byte chunk c of row j at chunk c ^ (j % 8)),
 // plus the gate weights w' the epilogue applies.
 //
@@ -126,6 +164,23 @@ __device__ __forceinline__ void cp_async_wait_group() {
 // within 2^-10 of it (2^-17 max_c |q_jc| before scaling) otherwise.  The two
 // pieces are rows [0, H) and [H, 2H) of one operand.  w'_j = w_j 2^-e_j.
 // ---------------------------------------------------------------------------
+// 2^e as a float, for -126 <= e <= 127.
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float(uint32_t(e + 127) << 23); }
+// v * 2^e with a single rounding (like ldexpf), for -126 <= e <= 254.
+__device__ __forceinline__ float scale_pow2(float v, int e) {
+    if (e > 127) {   // exact: v * 2^127 stays finite because |v| < 2^(8 - e) here
+        v *= pow2f(127);
+        e -= 127;
+    }
+    return v * pow2f(e);
+}
+// The exponent E of m > 0 in the frexp sense: m = f * 2^E with 0.5 <= f < 1.
+__device__ __forceinline__ int frexp_exponent(float m) {
+    const uint32_t bits = __float_as_uint(m);
+    const int ex = int(bits >> 23);
+    return ex ? ex - 126 : (32 - __clz(int(bits & 0x7FFFFFu))) - 149;
+}
+
 template <int KIND, int H>
 __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, const float *__restrict__ wb, int d,
                                             uint8_t *slot, float *wsm, int wi, int nw, int lane) {
@@ -161,10 +216,14 @@ __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, con
         // warp wi owns heads wi, wi + nw, ...; lane owns channels 4*lane .. 4*lane+3; 8 heads per batch
         for (int j0 = wi; j0 < H; j0 += 8 * nw) {
             uint2 raw[8];
+            float wr[8];   // gate weights, loaded with the query rows (not one round trip per head)
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int j = j0 + u * nw;
-                if (j < H) raw[u] = *reinterpret_cast<const uint2 *>(qb + j * 128 + 4 * lane);
+                if (j < H) {
+                    raw[u] = *reinterpret_cast<const uint2 *>(qb + j * 128 + 4 * lane);
+                    wr[u] = wb[j];
+                }
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -175,37 +234,33 @@ __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, con
                 float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
 #pragma unroll
                 for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                int e = 0;
-                if (m > 0.f) {
-                    int E;
-                    frexpf(m, &E);
-                    e = 8 - E;
-                }
+                const int e = m > 0.f ? 8 - frexp_exponent(m) : 0;   // m 2^e in [128, 256)
                 uint32_t w0 = 0, w1 = 0;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float sv = ldexpf(v[c], e);
-                    const __nv_fp8_storage_t p1 = __nv_cvt_float_to_fp8(sv, __NV_SATFINITE, __NV_E4M3);
-                    const __half_raw h1 = __nv_cvt_fp8_to_halfraw(p1, __NV_E4M3);
-                    const float r = sv - __half2float(__half(h1));
-                    const __nv_fp8_storage_t p2 = __nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3);
+                for (int c = 0; c < 4; c += 2) {   // two channels per conversion (.x -> low byte)
+                    const float2 sv = make_float2(scale_pow2(v[c], e), scale_pow2(v[c + 1], e));
+                    const __nv_fp8x2_storage_t p1 = __nv_cvt_float2_to_fp8x2(sv, __NV_SATFINITE, __NV_E4M3);
+                    const float2 h1 = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(p1, __NV_E4M3)));
+                    const __nv_fp8x2_storage_t p2 =
+                        __nv_cvt_float2_to_fp8x2(make_float2(sv.x - h1.x, sv.y - h1.y), __NV_SATFINITE, __NV_E4M3);
                     w0 |= uint32_t(p1) << (8 * c);
                     w1 |= uint32_t(p2) << (8 * c);
                 }
                 const int off = j * 128 + (((lane >> 2) ^ (j & 7)) << 4) + (lane & 3) * 4;
                 *reinterpret_cast<uint32_t *>(slot + off) = w0;
                 *reinterpret_cast<uint32_t *>(slot + H * 128 + off) = w1;
-                if (lane == 0) wsm[j] = ldexpf(wb[j], -e);
+                if (lane == 0) wsm[j] = ldexpf(wr[u], -e);
             }
         }
     }
 }
 
 // Sequence and rows of tile t; `b` is a cursor that only moves forward.
+template <int TR>
 __device__ __forceinline__ void tile_info(const int64_t *s_toff, const int64_t *s_seq, int B, int64_t t, int &b,
                                           int64_t &row0, int64_t &row_end) {
     while (b < B - 1 && t >= s_toff[b + 1]) ++b;
-    row0 = s_seq[b] + (t - s_toff[b]) * kRows;
+    row0 = s_seq[b] + (t - s_toff[b]) * TR;
     row_end = s_seq[b + 1];
 }
 
@@ -222,8 +277,14 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     using C = Cfg<KIND>;
     constexpr int S = C::kStages;
     constexpr int QIMG = qimg_bytes<KIND, H>();
-    constexpr int AC = acc_cols(KIND, H);
-    constexpr uint32_t NCOL = tmem_cols(AC);
+    constexpr int TR = tile_rows<KIND>();          // rows per tile
+    constexpr int SUBC = sub_cols<KIND, H>();      // accumulator columns per 128-row sub-tile (MMA N)
+    constexpr int TILEC = tile_cols<KIND, H>();    // accumulator columns per tile
+    constexpr int KACC = acc_tiles<KIND, H>();     // tile accumulators
+    constexpr int G = mma_group<KIND, H>();
+    constexpr uint32_t NCOL = tmem_cols(KACC * TILEC);
+    static_assert(G >= 1 && G <= KACC / 2, "the epilogue must own accumulators while a group is issued");
+    static_assert(S >= G, "a group waits for G filled stages");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -234,8 +295,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     uint64_t *qfull = empty + S;                                  // [2] by slot
     uint64_t *qrel = qfull + 2;                                   // [kRel] by sequence ordinal
     uint64_t *tfull = qrel + kRel;
-    uint64_t *tempty = tfull + kAcc;
-    uint64_t *drain = tempty + kAcc;
+    uint64_t *tempty = tfull + kAccMax;
+    uint64_t *drain = tempty + kAccMax;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     int *s_nord = abort_flag + 1;                                 // sequences (ordinals) in this CTA's range
@@ -249,20 +310,26 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort_v = abort_flag;
 
-    if (threadIdx.x == 0) {
-        // tile axis: the entries (full mode) or the list positions (listed mode)
+    // tile axis: the entries (full mode) or the list positions (listed mode); all offsets are
+    // loaded at once, the tile prefix is then summed from shared memory
+    {
+        if (LISTED) pdl_wait();   // the list offsets come from an earlier kernel
         const int64_t *axis = LISTED ? idx_off : seq_off;
-        int64_t acc = 0;
-        for (int b = 0; b <= B; ++b) {
+        for (int b = threadIdx.x; b <= B; b += kThreads) {
             int64_t a = axis[b];
             if (LISTED && a > list_cap) a = list_cap;
             s_seq[b] = a;
             s_base[b] = seq_off[b];
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int64_t acc = 0;
+        for (int b = 0; b <= B; ++b) {
             s_toff[b] = acc;
             if (b < B) {
-                int64_t a1 = axis[b + 1];
-                if (LISTED && a1 > list_cap) a1 = list_cap;
-                acc += (a1 > a ? a1 - a + kRows - 1 : 0) / kRows;
+                const int64_t a = s_seq[b], a1 = s_seq[b + 1];
+                acc += (a1 > a ? a1 - a + TR - 1 : 0) / TR;
             }
         }
         const int64_t T = acc;
@@ -277,7 +344,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         for (int s = 0; s < S; ++s) { mbar_init(&full[s], LISTED ? 32 : 1); mbar_init(&empty[s], 1); }
         for (int s = 0; s < 2; ++s) mbar_init(&qfull[s], 1);
         for (int s = 0; s < kRel; ++s) mbar_init(&qrel[s], 1 + kEpiWarps);
-        for (int s = 0; s < kAcc; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 4); }
+        // an accumulator is released by the warps that read it: one warpgroup per 128-row sub-tile
+        for (int s = 0; s < KACC; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 4 * C::kSub); }
         mbar_init(drain, 1);
         fence_mbar_init();
     }
@@ -318,7 +386,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 int bp = 0;
                 int64_t r0, r1;
                 for (int64_t t = t0; t < t0 + npre; ++t) {
-                    tile_info(s_toff, s_seq, B, t, bp, r0, r1);
+                    tile_info<TR>(s_toff, s_seq, B, t, bp, r0, r1);
                     const int st = int(t - t0);
                     mbar_arrive_expect_tx(&full[st], C::kStageBytes);
 #pragma unroll
@@ -332,7 +400,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             uint32_t ph = 0;
             int64_t row0, row_end;
             for (int64_t t = t0; t < t1; ++t) {
-                tile_info(s_toff, s_seq, B, t, b, row0, row_end);
+                tile_info<TR>(s_toff, s_seq, B, t, b, row0, row_end);
                 if (b != cur) {
                     if (!next_query(b, qn)) break;
                     cur = b;
@@ -356,7 +424,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 if (++st == S) { st = 0; ph ^= 1; }
             }
         } else {
-            // all 32 lanes gather: lane owns rows lane, lane+32, lane+64, lane+96 of each tile
+            // all 32 lanes gather: lane owns rows lane, lane + 32, ... of each tile
             pdl_wait();
             constexpr int RB = KIND == E4M3_D128 ? 128 : (KIND == BF16_D128 ? 256 : 128);   // row bytes
             constexpr int CPR = RB / 16;
@@ -365,18 +433,32 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             int64_t row0, row_end;
             int pend[kGatherDepth + 1];
             int npend = 0, head = 0;
+            // completes every gather still held back and signals its stage: done before any
+            // wait whose end may depend on the MMA consuming one of those stages
+            auto flush = [&]() {
+                if (npend == 0) return;
+                cp_async_wait_group<0>();
+                fence_proxy_async_smem();
+                while (npend > 0) {
+                    mbar_arrive(&full[pend[head]]);
+                    head = (head + 1) % (kGatherDepth + 1);
+                    --npend;
+                }
+            };
             for (int64_t t = t0; t < t1; ++t) {
-                tile_info(s_toff, s_seq, B, t, b, row0, row_end);
+                tile_info<TR>(s_toff, s_seq, B, t, b, row0, row_end);
                 if (b != cur) {
+                    if (qn >= 2) flush();   // the slot's release needs the MMA to finish the older sequence
                     if (!next_query(b, qn)) break;
                     cur = b;
                     ++qn;
                 }
+                if (!__all_sync(0xffffffffu, mbar_test_wait(&empty[st], ph ^ 1))) flush();
                 const bool ok = mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 const uint32_t stage_u32 = smem_u32(stages + st * C::kStageBytes);
 #pragma unroll
-                for (int rr = 0; rr < 4; ++rr) {
+                for (int rr = 0; rr < TR / 32; ++rr) {
                     const int r = lane + 32 * rr;
                     const int64_t p = row0 + r;
                     const bool valid = p < row_end;
@@ -399,65 +481,91 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 }
                 if (++st == S) { st = 0; ph ^= 1; }
             }
-            cp_async_wait_group<0>();
-            fence_proxy_async_smem();
-            while (npend > 0) {
-                mbar_arrive(&full[pend[head]]);
-                head = (head + 1) % (kGatherDepth + 1);
-                --npend;
-            }
+            flush();
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC = KIND == E4M3_D128 ? idesc_e4m3(kRows, AC) : idesc_bf16(kRows, AC);
+            constexpr uint32_t IDESC = KIND == E4M3_D128 ? idesc_e4m3(kRows, SUBC) : idesc_bf16(kRows, SUBC);
             // descriptors of stage 0 and slot 0; the others differ only in the start address field
             const uint64_t a_desc0 = desc_sw128(smem_u32(stages));
             const uint64_t b_desc0 = desc_sw128(smem_u32(qimg));
             int b = 0, cur = -1, qn = 0, slot = 0, st = 0, acc = 0;
             uint32_t ph = 0, aph = 0;
             int64_t row0, row_end;
-            bool issued = false;
-            for (int64_t t = t0; t < t1; ++t) {
-                tile_info(s_toff, s_seq, B, t, b, row0, row_end);
-                // the next tile starts a new sequence when it is the first tile of a later one
-                const bool last_of_seq = (t + 1 >= t1) || (t + 1 >= s_toff[b + 1]);
-                if (b != cur) {
-                    slot = qn & 1;
-                    if (!mbar_wait(&qfull[slot], (qn >> 1) & 1, abort_v, kWaitLimitNs)) break;
-                    cur = b;
-                    ++qn;
+            bool issued = false, ok = true;
+            // A group never continues past a sequence change: the query of a new sequence is
+            // waited for only at the start of a group, once every earlier release is committed.
+            for (int64_t tg = t0; tg < t1;) {
+                const int gmax = int(t1 - tg < G ? t1 - tg : G);
+                int gn = 0;
+                uint64_t a_d[G], b_d[G];
+                uint32_t d_t[G];
+                int st_of[G], acc_of[G], rel_of[G];
+#pragma unroll
+                for (int u = 0; u < G; ++u) {
+                    if (u >= gmax) break;
+                    const int64_t t = tg + u;
+                    tile_info<TR>(s_toff, s_seq, B, t, b, row0, row_end);
+                    if (b != cur) {
+                        if (u > 0) break;
+                        slot = qn & 1;
+                        if (!mbar_wait(&qfull[slot], (qn >> 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+                        cur = b;
+                        ++qn;
+                    }
+                    if (!mbar_wait(&tempty[acc], aph ^ 1, abort_v, kWaitLimitNs)) { ok = false; break; }
+                    if (!mbar_wait(&full[st], ph, abort_v, kWaitLimitNs)) { ok = false; break; }
+                    // start-address fields advance in 16-byte units
+                    a_d[u] = a_desc0 + uint64_t((st * C::kStageBytes) >> 4);
+                    b_d[u] = b_desc0 + uint64_t((slot * QIMG) >> 4);
+                    d_t[u] = tmem_base + uint32_t(acc * TILEC);
+                    st_of[u] = st;
+                    acc_of[u] = acc;
+                    // the next tile starts a new sequence when it is the first tile of a later one
+                    rel_of[u] = ((t + 1 >= t1) || (t + 1 >= s_toff[b + 1])) ? (qn - 1) % kRel : -1;
+                    if (++st == S) { st = 0; ph ^= 1; }
+                    if (++acc == KACC) { acc = 0; aph ^= 1; }
+                    ++gn;
                 }
-                if (!mbar_wait(&tempty[acc], aph ^ 1, abort_v, kWaitLimitNs)) break;
-                if (!mbar_wait(&full[st], ph, abort_v, kWaitLimitNs)) break;
+                if (!ok) break;
+                tg += gn;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + uint32_t(acc * AC);
-                // start-address field advances in 16-byte units
-                const uint64_t a_desc = a_desc0 + uint64_t((st * C::kStageBytes) >> 4);
-                const uint64_t b_desc = b_desc0 + uint64_t((slot * QIMG) >> 4);
                 if (KIND == BF16_D128) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_f16(d_tmem, a_desc + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                                b_desc + uint64_t(((kk >> 2) * (H * 128) + (kk & 3) * 32) >> 4), IDESC, kk > 0);
+#pragma unroll
+                        for (int u = 0; u < G; ++u)
+                            if (u < gn)
+                                mma_f16(d_t[u], a_d[u] + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                                        b_d[u] + uint64_t(((kk >> 2) * (H * 128) + (kk & 3) * 32) >> 4), IDESC,
+                                        kk > 0);
                 } else if (KIND == BF16_D64) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f16(d_tmem, a_desc + uint64_t((kk * 32) >> 4), b_desc + uint64_t((kk * 32) >> 4), IDESC,
-                                kk > 0);
+#pragma unroll
+                        for (int u = 0; u < G; ++u)
+                            if (u < gn)
+                                mma_f16(d_t[u], a_d[u] + uint64_t((kk * 32) >> 4), b_d[u] + uint64_t((kk * 32) >> 4),
+                                        IDESC, kk > 0);
                 } else {
-                    // B = the two query pieces stacked as 2H rows (adjacent in the slot)
+                    // the two 128-row halves of the tile (16 KB apart in the stage) into their own
+                    // column blocks, chains interleaved; N = 2H covers both query pieces
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f8(d_tmem, a_desc + uint64_t((kk * 32) >> 4), b_desc + uint64_t((kk * 32) >> 4), IDESC,
-                               kk != 0);
+#pragma unroll
+                        for (int sub = 0; sub < 2; ++sub)
+                            mma_f8(d_t[0] + uint32_t(sub * SUBC), a_d[0] + uint64_t((sub * 16384 + kk * 32) >> 4),
+                                   b_d[0] + uint64_t((kk * 32) >> 4), IDESC, kk > 0);
                 }
                 issued = true;
-                mma_commit(&empty[st]);
-                mma_commit(&tfull[acc]);
-                if (last_of_seq) mma_commit(&qrel[(qn - 1) % kRel]);   // this sequence's operand is no longer read
-                if (++st == S) { st = 0; ph ^= 1; }
-                if (++acc == kAcc) { acc = 0; aph ^= 1; }
+#pragma unroll
+                for (int u = 0; u < G; ++u) {
+                    if (u >= gn) break;
+                    mma_commit(&empty[st_of[u]]);
+                    mma_commit(&tfull[acc_of[u]]);
+                    if (rel_of[u] >= 0) mma_commit(&qrel[rel_of[u]]);   // this sequence's operand is no longer read
+                }
             }
             if (issued) {
                 // every issued MMA has finished before TMEM is released
@@ -469,8 +577,13 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     } else {
         // ------------------------------------------------------------ epilogue
         const int ew = warp - 2;              // 0..7
-        const int grp = ew >> 2;              // warpgroup: takes tiles t0 + grp, t0 + grp + 2, ...
+        const int grp = ew >> 2;              // warpgroup
         const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
+        // 128-row tiles: the warpgroups take alternate tiles; 256-row tiles: every tile, warpgroup g
+        // its sub-tile g
+        constexpr int kStep = C::kSub == 2 ? 1 : kEpiGroups;
+        const int sub = C::kSub == 2 ? grp : 0;
+        const int64_t tfirst = C::kSub == 2 ? t0 : t0 + grp;
         int b = 0, cur = -1, ord = -1, released = 0;
         int64_t row0, row_end;
         // row scale of this thread's row in tile t (e4m3 keys), loaded one tile of this group ahead
@@ -478,8 +591,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             if (KIND != E4M3_D128 || t >= t1) return 1.f;
             int bb = b;
             int64_t r0, r1;
-            tile_info(s_toff, s_seq, B, t, bb, r0, r1);
-            const int64_t r = r0 + quarter * 32 + lane;
+            tile_info<TR>(s_toff, s_seq, B, t, bb, r0, r1);
+            const int64_t r = r0 + sub * kRows + quarter * 32 + lane;
             if (r >= r1) return 1.f;
             return __ldg(k_scale + (LISTED ? s_base[bb] + idx[r] : r));
         };
@@ -493,7 +606,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             // while the first keys load, so that no CTA's producer stalls at its first sequence change
             int bo = 0;
             int64_t r0, r1;
-            tile_info(s_toff, s_seq, B, t0, bo, r0, r1);
+            tile_info<TR>(s_toff, s_seq, B, t0, bo, r0, r1);
             pdl_wait();   // the query and gate weights may come from the preceding kernel
             for (int o = 0; o < 2 && o < nord; ++o) {
                 if (o == 1) {   // the next sequence that owns tiles
@@ -507,20 +620,20 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 if (ew == 0 && lane == 0) mbar_arrive(&qfull[o]);
             }
         }
-        float sc_next = scale_of(t0 + grp);
+        float sc_next = scale_of(tfirst);
         // ordinal of each tile: count the sequence changes over every tile of the range (both groups')
         int ob = 0, ocur = -1, onum = -1;
         int64_t orow0, orow1, u_next = t0;
         bool ok = true;
-        for (int64_t t = t0 + grp; t < t1; t += kEpiGroups) {
-            const int64_t i = t - t0;         // local tile index: accumulator i % 4, its (i / 4)-th use
-            const int acc = int(i % kAcc);
-            const uint32_t aph = uint32_t((i / kAcc) & 1);
+        for (int64_t t = tfirst; t < t1; t += kStep) {
+            const int64_t i = t - t0;         // local tile index: accumulator i % KACC, its (i / KACC)-th use
+            const int acc = int(i % KACC);
+            const uint32_t aph = uint32_t((i / KACC) & 1);
             for (; u_next <= t; ++u_next) {
-                tile_info(s_toff, s_seq, B, u_next, ob, orow0, orow1);
+                tile_info<TR>(s_toff, s_seq, B, u_next, ob, orow0, orow1);
                 if (ob != ocur) { ocur = ob; ++onum; }
             }
-            tile_info(s_toff, s_seq, B, t, b, row0, row_end);
+            tile_info<TR>(s_toff, s_seq, B, t, b, row0, row_end);
             if (b != cur) {
                 cur = b;
                 ord = onum;
@@ -530,15 +643,16 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 if (!__all_sync(0xffffffffu, ok)) break;
             }
             const float *wq = wsm + (ord & 1) * H;
-            const int64_t row = row0 + quarter * 32 + lane;   // entry (full) or list position (listed)
+            const int64_t row = row0 + sub * kRows + quarter * 32 + lane;   // entry (full) or list position
             const float sc = sc_next;
-            sc_next = scale_of(t + kEpiGroups);
+            sc_next = scale_of(t + kStep);
             ok = mbar_wait(&tfull[acc], aph, abort_v, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
             tc_fence_after();
-            const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * AC);
-            float zs = 0.f;
-            if (KIND != E4M3_D128) {
+            const uint32_t taddr =
+                tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * TILEC + sub * SUBC);
+            float za = 0.f, zb = 0.f, zc = 0.f, zd = 0.f;   // four short dependency chains
+            if (C::kPieces == 1) {
                 uint32_t r[H];
 #pragma unroll
                 for (int c = 0; c < H / 16; ++c)
@@ -550,39 +664,32 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
 #pragma unroll
                 for (int j = 0; j < H; j += 4) {
                     const float4 wv = *reinterpret_cast<const float4 *>(wq + j);
-                    zs = fmaf(wv.x, fmaxf(__uint_as_float(r[j]), 0.f), zs);
-                    zs = fmaf(wv.y, fmaxf(__uint_as_float(r[j + 1]), 0.f), zs);
-                    zs = fmaf(wv.z, fmaxf(__uint_as_float(r[j + 2]), 0.f), zs);
-                    zs = fmaf(wv.w, fmaxf(__uint_as_float(r[j + 3]), 0.f), zs);
+                    za = fmaf(wv.x, fmaxf(__uint_as_float(r[j]), 0.f), za);
+                    zb = fmaf(wv.y, fmaxf(__uint_as_float(r[j + 1]), 0.f), zb);
+                    zc = fmaf(wv.z, fmaxf(__uint_as_float(r[j + 2]), 0.f), zc);
+                    zd = fmaf(wv.w, fmaxf(__uint_as_float(r[j + 3]), 0.f), zd);
                 }
             } else {
-                // heads in halves of H/2: both pieces' columns of a half in one round trip
-                constexpr int HH = H / 2;
+                // both pieces' columns in one round trip, so that the accumulator is released
+                // before any arithmetic (only two tile accumulators fit in TMEM)
+                uint32_t r[2 * H];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r1[HH], r2[HH];
+                for (int c = 0; c < 2 * H / 16; ++c)
+                    tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[c * 16]));
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
 #pragma unroll
-                    for (int c = 0; c < HH / 16; ++c) {
-                        tmem_ld_32x32b_x16(taddr + half * HH + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&r1[c * 16]));
-                        tmem_ld_32x32b_x16(taddr + H + half * HH + c * 16,
-                                           *reinterpret_cast<uint32_t(*)[16]>(&r2[c * 16]));
-                    }
-                    tmem_ld_wait();
-                    if (half == 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&tempty[acc]);
-                    }
-#pragma unroll
-                    for (int j = 0; j < HH; j += 4) {
-                        const float4 wv = *reinterpret_cast<const float4 *>(wq + half * HH + j);
-                        zs = fmaf(wv.x, fmaxf(__uint_as_float(r1[j]) + __uint_as_float(r2[j]), 0.f), zs);
-                        zs = fmaf(wv.y, fmaxf(__uint_as_float(r1[j + 1]) + __uint_as_float(r2[j + 1]), 0.f), zs);
-                        zs = fmaf(wv.z, fmaxf(__uint_as_float(r1[j + 2]) + __uint_as_float(r2[j + 2]), 0.f), zs);
-                        zs = fmaf(wv.w, fmaxf(__uint_as_float(r1[j + 3]) + __uint_as_float(r2[j + 3]), 0.f), zs);
-                    }
+                for (int j = 0; j < H; j += 4) {
+                    const float4 wv = *reinterpret_cast<const float4 *>(wq + j);
+                    za = fmaf(wv.x, fmaxf(__uint_as_float(r[j]) + __uint_as_float(r[H + j]), 0.f), za);
+                    zb = fmaf(wv.y, fmaxf(__uint_as_float(r[j + 1]) + __uint_as_float(r[H + j + 1]), 0.f), zb);
+                    zc = fmaf(wv.z, fmaxf(__uint_as_float(r[j + 2]) + __uint_as_float(r[H + j + 2]), 0.f), zc);
+                    zd = fmaf(wv.w, fmaxf(__uint_as_float(r[j + 3]) + __uint_as_float(r[H + j + 3]), 0.f), zd);
                 }
             }
+            float zs = (za + zb) + (zc + zd);
             if (row < row_end) {
                 if (KIND == E4M3_D128) zs *= sc;
                 z[row] = zs;
@@ -624,7 +731,7 @@ template <int KIND, int H>
 size_t smem_bytes(int B) {
     using C = Cfg<KIND>;
     return 1024 + size_t(C::kStages) * C::kStageBytes + 2 * qimg_bytes<KIND, H>() +
-           (2 * C::kStages + 2 + kRel + 2 * kAcc + 1) * 8 + 16 + 16 + 2 * H * 4 + size_t(B + 1) * 24 + 64;
+           (2 * C::kStages + 2 + kRel + 2 * kAccMax + 1) * 8 + 16 + 16 + 2 * H * 4 + size_t(B + 1) * 24 + 64;
 }
 
 template <int KIND, int H>
@@ -640,7 +747,7 @@ lsa_status launch(const void *q, const float *w, const void *k, const float *k_s
     const bool fp8 = KIND == E4M3_D128;
     const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(n_total)};
     const cuuint64_t strides[1] = {cuuint64_t(d) * (fp8 ? 1 : 2)};
-    const cuuint32_t box[2] = {cuuint32_t(fp8 ? 128 : 64), cuuint32_t(kRows)};
+    const cuuint32_t box[2] = {cuuint32_t(fp8 ? 128 : 64), cuuint32_t(Cfg<KIND>::kBoxRows)};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                      const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -654,7 +761,7 @@ lsa_status launch(const void *q, const float *w, const void *k, const float *k_s
     auto kern = idx ? scan_tc<KIND, H, true> : scan_tc<KIND, H, false>;
     LSA_CUDA(ensure_smem(kern, smem));
     const int64_t axis = idx ? list_cap : n_total;
-    const int64_t max_tiles = (axis + kRows - 1) / kRows + B;
+    const int64_t max_tiles = (axis + tile_rows<KIND>() - 1) / tile_rows<KIND>() + B;
     const int grid = int(max_tiles < sm_count() ? max_tiles : sm_count());
     LSA_CUDA(launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, map, static_cast<const uint8_t *>(k),
                         static_cast<const uint16_t *>(q), w, d, seq_off, idx, idx_off, list_cap, B, k_scale, z, I,
@@ -678,7 +785,9 @@ lsa_status launch_h(int H, const void *q, const float *w, const void *k, const f
 
 bool index_score_tc_supported(lsa_dtype q_dtype, lsa_dtype k_dtype, int64_t n_total, int32_t B, int32_t H,
                               int32_t d) {
-    if (q_dtype != LSA_BF16 || n_total < kRows || B > kMaxB) return false;
+    // (a TMA box never exceeds the key matrix: at least one tile of rows)
+    if (q_dtype != LSA_BF16 || B > kMaxB) return false;
+    if (n_total < (k_dtype == LSA_E4M3 ? tile_rows<E4M3_D128>() : kRows)) return false;
     if (!(H == 16 || H == 32 || H == 64)) return false;
     if (k_dtype == LSA_BF16) return d == 128 || d == 64;
     if (k_dtype == LSA_E4M3) return d == 128;
