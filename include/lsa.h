@@ -318,6 +318,27 @@ lsa_status lsa_ctx_stage_times(lsa_ctx *ctx, double *ms, int64_t *calls);
 lsa_status lsa_ctx_reset_counters(lsa_ctx *ctx);
 int64_t lsa_ctx_launches(lsa_ctx *ctx);
 
+/* ------------------------------------------------------------------------
+ * lsa_selftest_bounded_wait -- checks, on the GPU, the expiry path of the
+ * bounded device-side waits that every tcgen05 kernel here uses (the pages
+ * have no counterpart: this is failure-handling infrastructure).  One CTA
+ * waits on a shared-memory mbarrier that nothing arrives at:
+ *   - warp 0 waits with a limit of limit_ns (%globaltimer); when it runs out
+ *     the kernel writes LSA_ERR_TIMEOUT into *err (first error wins) and
+ *     waited_ns[0] = the time it waited;
+ *   - warp 1 waits on the same barrier with a limit of 4 * limit_ns and
+ *     returns as soon as warp 0 raises the CTA's abort flag: waited_ns[1] =
+ *     its wait (about limit_ns, well below 4 * limit_ns), waited_ns[2] = 1 if
+ *     its wait reported success (it must not: 0).
+ * The kernel always returns; no fault, trap or hang is involved.
+ *
+ * limit_ns   1,000 .. 100,000,000 (1 us .. 100 ms), else LSA_ERR_INVALID
+ * err        device int32 error word (the caller zeroes it first)
+ * waited_ns  device int64[3], written by the kernel
+ * stream     cudaStream_t or NULL
+ * ---------------------------------------------------------------------- */
+lsa_status lsa_selftest_bounded_wait(int64_t limit_ns, int32_t *err, int64_t *waited_ns, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,7 +8,9 @@
 // rows):
 //   1. warps 0-3 gather the chunk's 128 rows (1 KB each, arbitrary hot-buffer
 //      rows) with cp.async straight into the 128-byte-swizzled K-major layout
-//      the tensor core reads (8 column blocks of 64 elements); padding rows are
+//      the tensor core reads (8 column blocks of 64 elements), block by block,
+//      each block signalled as soon as it lands so that the S MMAs of block 0
+//      start while the others are still in flight; padding rows are
 //      zero-filled;
 //   2. warp 5 streams Q[b] (128 x 512 bf16) by TMA in 8 slices of 64 columns
 //      through a 3-stage ring;
@@ -21,8 +23,8 @@
 //      0..511, reading the SAME smem rows as V through an MN-major descriptor
 //      (no transpose, no second copy of the rows);
 //   6. warps 0-3 read O in 64-column blocks into the freed row buffer
-//      (128-byte swizzle) and write the fp32 partial with TMA stores; (m, l)
-//      per head.
+//      (128-byte swizzle, four staging buffers) and write the fp32 partial
+//      with TMA stores; (m, l) per head.
 // The combine kernel (attn.cu) merges the chunks.  Every wait is bounded.
 #include <cuda.h>
 
@@ -51,7 +53,11 @@ constexpr int kOStageBytes = kHq * 64 * 4;       // 32 KB: [128 heads][64 fp32] 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
 // 64-element (128-byte) blocks along MN `lbo` bytes apart, 8-row groups along
@@ -77,8 +83,8 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
     uint8_t *ps = qs + kQStages * kQStageBytes;  // 32 KB
     uint64_t *qfull = reinterpret_cast<uint64_t *>(ps + kPBytes);
     uint64_t *qempty = qfull + kQStages;
-    uint64_t *kv_full = qempty + kQStages;
-    uint64_t *s_full = kv_full + 1;
+    uint64_t *kv_full = qempty + kQStages;       // [kD / 64] column blocks of the rows
+    uint64_t *s_full = kv_full + kD / 64;
     uint64_t *p_full = s_full + 1;
     uint64_t *o_full = p_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_full + 1);
@@ -96,7 +102,7 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
         *abort_flag = 0;
         *s_nvalid = 0;
         for (int s = 0; s < kQStages; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 1); }
-        mbar_init(kv_full, 128);
+        for (int kb = 0; kb < kD / 64; ++kb) mbar_init(&kv_full[kb], 128);
         mbar_init(s_full, 1);
         mbar_init(p_full, 128);
         mbar_init(o_full, 1);
@@ -138,18 +144,31 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
             for (int kd = 0; kd < kQStages; ++kd) mbar_wait(&qfull[kd], 0, abort_v, kWaitLimitNs);
     } else if (warp < 4) {
         const int t = threadIdx.x;   // 0..127
-        // ---- 1. gather the chunk's rows: 128 rows x 64 sixteen-byte chunks
+        // ---- 1. gather the chunk's rows: 8 column blocks of 128 rows x 8 sixteen-byte chunks, one
+        // cp.async group per block (8 consecutive threads read one row's 128 contiguous bytes)
         const uint32_t kv_u32 = smem_u32(kvs);
-        for (int i = t; i < kRowsPerCta * 64; i += 128) {
-            const int r = i >> 6, c = i & 63;
-            const int row = s_rows[r];
-            const uint32_t dst = kv_u32 + (c >> 3) * kKvBlock + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-            const uint16_t *src = kv + (row >= 0 ? int64_t(row) * stride + k_off + c * 8 : 0);
-            cp_async_16(dst, src, row >= 0 ? 16u : 0u);
+#pragma unroll
+        for (int kb = 0; kb < kD / 64; ++kb) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = t + 128 * u;
+                const int r = i >> 3, c = kb * 8 + (i & 7);
+                const int row = s_rows[r];
+                const uint32_t dst = kv_u32 + kb * kKvBlock + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+                const uint16_t *src = kv + (row >= 0 ? int64_t(row) * stride + k_off + c * 8 : 0);
+                cp_async_16(dst, src, row >= 0 ? 16u : 0u);
+            }
+            cp_async_commit();
         }
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(kv_full);
+        // block kb has landed once at most 7 - kb younger groups are pending
+        cp_async_wait_group<7>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[0]);
+        cp_async_wait_group<6>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[1]);
+        cp_async_wait_group<5>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[2]);
+        cp_async_wait_group<4>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[3]);
+        cp_async_wait_group<3>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[4]);
+        cp_async_wait_group<2>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[5]);
+        cp_async_wait_group<1>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[6]);
+        cp_async_wait_group<0>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[7]);
 
         // ---- 4. softmax of the chunk: thread t owns head t (TMEM lane t)
         const int quarter = warp;   // warps 0-3 -> TMEM lanes 32*warp ..
@@ -192,16 +211,16 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
             tc_fence_before();
             mbar_arrive(p_full);
             // ---- 6. read O and write the chunk's partial: 64-column blocks staged in the (now free)
-            // row buffer, one TMA store per block; two staging buffers alternate
+            // row buffer, one TMA store per block; four staging buffers rotate
             ok = mbar_wait(o_full, 0, abort_v, kWaitLimitNs);
             // the block loop below synchronises these 128 threads: agree on one outcome first
             if (named_barrier_and(1, 128, ok)) {
                 tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < kD / 64; ++c) {
-                    float *sb = reinterpret_cast<float *>(kvs + (c & 1) * kOStageBytes);   // 2 x [128][32]
-                    if (c >= 2) {
-                        if (t == 0) bulk_wait_read<1>();   // the store issued two blocks ago has read its buffer
+                    float *sb = reinterpret_cast<float *>(kvs + (c & 3) * kOStageBytes);   // 2 halves of [128][32]
+                    if (c >= 4) {
+                        if (t == 0) bulk_wait_read<3>();   // the store issued four blocks ago has read its buffer
                         named_barrier(1, 128);
                     }
                     uint32_t o[64];
@@ -239,13 +258,14 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128);
             constexpr uint32_t IDESC_O = idesc_bf16(128, 256) | (1u << 16);   // B (V) is MN-major
             bool issued = false;
-            if (mbar_wait(kv_full, 0, abort_v, kWaitLimitNs)) {
+            {
                 const uint32_t kv_u32 = smem_u32(kvs);
                 int st = 0;
                 uint32_t ph = 0;
                 bool ok = true;
                 for (int kd = 0; kd < kD / 64 && ok; ++kd) {
-                    ok = mbar_wait(&qfull[st], ph, abort_v, kWaitLimitNs);
+                    ok = mbar_wait(&kv_full[kd], 0, abort_v, kWaitLimitNs) &&
+                         mbar_wait(&qfull[st], ph, abort_v, kWaitLimitNs);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t q_u32 = smem_u32(qs + st * kQStageBytes);
@@ -317,7 +337,7 @@ EncodeTiledFn encode_fn() {
 }
 
 constexpr size_t kSmemBytes = 1024 + size_t(kKvBytes) + size_t(kQStages) * kQStageBytes + kPBytes +
-                              (2 * kQStages + 4) * 8 + 16 + (kRowsPerCta + 2) * 4 + 64;
+                              (2 * kQStages + kD / 64 + 3) * 8 + 16 + (kRowsPerCta + 2) * 4 + 64;
 
 }  // namespace
 

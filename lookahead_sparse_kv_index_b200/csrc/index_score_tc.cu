@@ -87,7 +87,7 @@ struct Cfg<E4M3_D128> {
     static constexpr int kBoxRows = 256;
     static constexpr int kPieces = 2;           // both query pieces in one N = 2H operand
     static constexpr int kQBytesPerHead = 256;  // two e4m3 pieces x 128
-    static constexpr int kStages = 5;
+    static constexpr int kStages = 4;           // at most twice the tile accumulators (2)
 };
 
 constexpr int kThreads = 320;         // warp 0 producer, warp 1 MMA, warps 2-9 epilogue (2 warpgroups)
@@ -96,6 +96,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kRel = 8;               // query-slot release barriers, by sequence ordinal mod kRel
 constexpr int kRows = 128;            // rows of one MMA (M) and of a sub-tile
 constexpr int kAccMax = 8;            // TMEM accumulator stages at most
+constexpr int kScaleSlotsMax = 16;    // row-scale ring slots at most (stages + accumulators)
 constexpr int kMaxB = 512;            // sequences per launch on this path
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
 constexpr int kGatherDepth = 3;       // listed mode: tiles of row gathers in flight per producer lane
@@ -140,6 +141,15 @@ __host__ __device__ constexpr int qimg_bytes() {
 // cp.async of 16 bytes (zero-filled when src_bytes == 0) and its group controls.
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// 4-byte cp.async (zero-filled when src_bytes == 0).
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// Arrive on `bar` once every cp.async this thread has issued so far has completed (the barrier's
+// expected count includes this arrival).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -285,19 +295,32 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     constexpr uint32_t NCOL = tmem_cols(KACC * TILEC);
     static_assert(G >= 1 && G <= KACC / 2, "the epilogue must own accumulators while a group is issued");
     static_assert(S >= G, "a group waits for G filled stages");
+    // a stage is free again when the MMA of the tile it held has completed, which the producer learns
+    // from that tile's accumulator barrier; a parity wait on it is unambiguous while the barrier
+    // cannot run two phases ahead, i.e. while S <= 2 * KACC
+    static_assert(S <= 2 * KACC, "stage reuse is tracked on the accumulator barriers");
+    // e4m3 keys: the per-row scales of each tile go to a shared-memory ring by cp.async (the
+    // producer warp), never through a register load of an epilogue warp, whose wait on its TMEM
+    // loads would otherwise also wait for that HBM load.  Slot j % RS holds tile j's scales; it is
+    // rewritten for tile j + RS only after the MMA of tile j + KACC, i.e. after the epilogue of tile
+    // j released its accumulator, which it does after reading the scales.
+    constexpr bool kScales = KIND == E4M3_D128;
+    constexpr int RS = S + KACC;
+    static_assert(!kScales || RS <= kScaleSlotsMax, "row-scale ring");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stages = smem;
     uint8_t *qimg = stages + S * C::kStageBytes;                  // 2 query slots
-    uint64_t *full = reinterpret_cast<uint64_t *>(qimg + 2 * QIMG);
-    uint64_t *empty = full + S;
-    uint64_t *qfull = empty + S;                                  // [2] by slot
+    uint64_t *full = reinterpret_cast<uint64_t *>(qimg + 2 * QIMG);  // [S] stage loaded
+    uint64_t *qfull = full + S;                                   // [2] query slot built
     uint64_t *qrel = qfull + 2;                                   // [kRel] by sequence ordinal
-    uint64_t *tfull = qrel + kRel;
-    uint64_t *tempty = tfull + kAccMax;
+    // [KACC] the MMAs of a tile completed: its accumulator is ready and its stage is free
+    uint64_t *tdone = qrel + kRel;
+    uint64_t *tempty = tdone + kAccMax;                           // [KACC] accumulator read by the epilogue
     uint64_t *drain = tempty + kAccMax;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *sfull = drain + 1;                                  // [RS] row scales of a tile landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfull + kScaleSlotsMax);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     int *s_nord = abort_flag + 1;                                 // sequences (ordinals) in this CTA's range
     // gate weights of the two slots, read as float4: 16-byte aligned
@@ -305,6 +328,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     int64_t *s_seq = reinterpret_cast<int64_t *>(wsm + 2 * H);   // [B+1] tile-axis offsets
     int64_t *s_toff = s_seq + (B + 1);                           // [B+1] first tile of each sequence
     int64_t *s_base = s_toff + (B + 1);                          // [B+1] entry base (listed mode)
+    float *s_scale = reinterpret_cast<float *>((reinterpret_cast<uintptr_t>(s_base + (B + 1)) + 15) & ~uintptr_t(15));
     __shared__ int64_t s_range[2];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -341,12 +365,14 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             if (s_toff[b + 1] > s_toff[b] && s_toff[b + 1] > t0 && s_toff[b] < t1) ++nord;
         *s_nord = nord;
         *abort_flag = 0;
-        for (int s = 0; s < S; ++s) { mbar_init(&full[s], LISTED ? 32 : 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < S; ++s) mbar_init(&full[s], LISTED ? 32 : 1);
         for (int s = 0; s < 2; ++s) mbar_init(&qfull[s], 1);
         for (int s = 0; s < kRel; ++s) mbar_init(&qrel[s], 1 + kEpiWarps);
         // an accumulator is released by the warps that read it: one warpgroup per 128-row sub-tile
-        for (int s = 0; s < KACC; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 4 * C::kSub); }
+        for (int s = 0; s < KACC; ++s) { mbar_init(&tdone[s], 1); mbar_init(&tempty[s], 4 * C::kSub); }
         mbar_init(drain, 1);
+        if (kScales)
+            for (int s = 0; s < RS; ++s) mbar_init(&sfull[s], 32);   // one cp.async arrival per producer lane
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) prefetch_tmap(&tmap);
@@ -365,6 +391,40 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         // builds the query operand of a new sequence (ordinal o) into slot o & 1
+        // local tile j may be loaded once the MMA of tile j - S (same stage) has completed
+        auto stage_free_test = [&](int64_t j) -> bool {
+            return j < S || mbar_test_wait(&tdone[(j - S) % KACC], uint32_t(((j - S) / KACC) & 1));
+        };
+        auto stage_free_wait = [&](int64_t j) -> bool {
+            return j < S || mbar_wait(&tdone[(j - S) % KACC], uint32_t(((j - S) / KACC) & 1), abort_v, kWaitLimitNs);
+        };
+        // row scales of local tile j (rows [row0, row_end) of the entry axis), all 32 lanes.  A span
+        // that starts 16-byte aligned and has a multiple of 4 rows goes by one bulk copy (the copy
+        // engine, like the keys); any other by 4-byte cp.async.  Global loads through the SM's L1 path
+        // held the tensor pipe back by a factor of about four here, so the bulk path is the rule: it
+        // takes every tile when the sequence offsets are multiples of 4.
+        auto load_scales = [&](int64_t j, int64_t row0, int64_t row_end) {
+            if (!kScales) return;
+            const int slot = int(j % RS);
+            const int64_t nvalid = (row_end - row0) < TR ? (row_end - row0) : TR;
+            if ((row0 & 3) == 0 && (nvalid & 3) == 0 && (reinterpret_cast<uintptr_t>(k_scale) & 15) == 0) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sfull[slot], uint32_t(nvalid * 4));
+                    bulk_load(s_scale + slot * TR, k_scale + row0, uint32_t(nvalid * 4), &sfull[slot]);
+                } else {
+                    mbar_arrive(&sfull[slot]);
+                }
+                return;
+            }
+            const uint32_t dst = smem_u32(s_scale + slot * TR);
+#pragma unroll
+            for (int k = 0; k < TR / 32; ++k) {
+                const int r = lane + 32 * k;
+                const bool valid = row0 + r < row_end;
+                cp_async_4(dst + r * 4, k_scale + (valid ? row0 + r : 0), valid ? 4u : 0u);
+            }
+            cp_async_arrive_noinc(&sfull[slot]);
+        };
         // (ordinals 0 and 1 are built by the epilogue warps, idle at kernel start)
         auto next_query = [&](int b, int o) -> bool {
             if (o < 2) return true;
@@ -382,17 +442,20 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         if (!LISTED) {
             // the keys do not depend on the preceding kernel: fill the ring first
             const int64_t npre = (t1 - t0) < S ? (t1 - t0) : S;
-            if (lane == 0) {
+            {
                 int bp = 0;
                 int64_t r0, r1;
                 for (int64_t t = t0; t < t0 + npre; ++t) {
                     tile_info<TR>(s_toff, s_seq, B, t, bp, r0, r1);
                     const int st = int(t - t0);
-                    mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&full[st], C::kStageBytes);
 #pragma unroll
-                    for (int bx = 0; bx < C::kBoxes; ++bx)
-                        tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64,
-                                    int(r0));
+                        for (int bx = 0; bx < C::kBoxes; ++bx)
+                            tma_load_2d(stages + st * C::kStageBytes + bx * 16384, &tmap, &full[st], bx * 64,
+                                        int(r0));
+                    }
+                    load_scales(t - t0, r0, r1);
                 }
             }
             pdl_wait();
@@ -409,7 +472,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 bool ok = true;
                 if (t - t0 >= npre) {   // the first npre tiles were issued above
                     if (lane == 0) {
-                        ok = mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs);
+                        ok = stage_free_wait(t - t0);
                         if (ok) {
                             mbar_arrive_expect_tx(&full[st], C::kStageBytes);
 #pragma unroll
@@ -419,6 +482,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                         }
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (ok) load_scales(t - t0, row0, row_end);
                 }
                 if (!ok) break;
                 if (++st == S) { st = 0; ph ^= 1; }
@@ -453,8 +517,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                     cur = b;
                     ++qn;
                 }
-                if (!__all_sync(0xffffffffu, mbar_test_wait(&empty[st], ph ^ 1))) flush();
-                const bool ok = mbar_wait(&empty[st], ph ^ 1, abort_v, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, stage_free_test(t - t0))) flush();
+                const bool ok = stage_free_wait(t - t0);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 const uint32_t stage_u32 = smem_u32(stages + st * C::kStageBytes);
 #pragma unroll
@@ -468,7 +532,10 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                     for (int c = 0; c < CPR; ++c)
                         cp_async_16(stage_u32 + (c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4),
                                     src + c * 16, valid ? 16u : 0u);
+                    if (kScales)
+                        cp_async_4(smem_u32(s_scale + int((t - t0) % RS) * TR + r), k_scale + e, valid ? 4u : 0u);
                 }
+                if (kScales) cp_async_arrive_noinc(&sfull[int((t - t0) % RS)]);
                 cp_async_commit();
                 pend[(head + npend) % (kGatherDepth + 1)] = st;
                 ++npend;
@@ -488,48 +555,44 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         if (lane == 0) {
             constexpr uint32_t IDESC = KIND == E4M3_D128 ? idesc_e4m3(kRows, SUBC) : idesc_bf16(kRows, SUBC);
             // descriptors of stage 0 and slot 0; the others differ only in the start address field
+            // (16-byte units), advanced incrementally: this thread's per-tile work is the tensor pipe's idle time
             const uint64_t a_desc0 = desc_sw128(smem_u32(stages));
             const uint64_t b_desc0 = desc_sw128(smem_u32(qimg));
-            int b = 0, cur = -1, qn = 0, slot = 0, st = 0, acc = 0;
+            constexpr uint64_t kStageStep = uint64_t(C::kStageBytes >> 4);
+            int b = 0, qn = -1, st = 0, acc = 0;
             uint32_t ph = 0, aph = 0;
-            int64_t row0, row_end;
+            int64_t row0, row_end, seq_end = t0;   // seq_end: first tile of the next sequence
+            uint64_t a_cur = a_desc0, b_cur = b_desc0;
             bool issued = false, ok = true;
-            // A group never continues past a sequence change: the query of a new sequence is
-            // waited for only at the start of a group, once every earlier release is committed.
-            for (int64_t tg = t0; tg < t1;) {
-                const int gmax = int(t1 - tg < G ? t1 - tg : G);
-                int gn = 0;
-                uint64_t a_d[G], b_d[G];
+            // A group of up to G tiles never continues past a sequence change: the query of a new
+            // sequence is waited for only at the start of a group, once every earlier release is committed.
+            for (int64_t t = t0; t < t1;) {
+                if (t == seq_end) {   // first tile of a sequence (ordinal qn + 1)
+                    tile_info<TR>(s_toff, s_seq, B, t, b, row0, row_end);
+                    seq_end = s_toff[b + 1];
+                    ++qn;
+                    b_cur = b_desc0 + uint64_t(((qn & 1) * QIMG) >> 4);
+                    if (!mbar_wait(&qfull[qn & 1], uint32_t((qn >> 1) & 1), abort_v, kWaitLimitNs)) break;
+                }
+                const int64_t gend = (seq_end < t1 ? seq_end : t1);
+                const int gn = int(gend - t < G ? gend - t : G);
+                uint64_t a_d[G];
                 uint32_t d_t[G];
-                int st_of[G], acc_of[G], rel_of[G];
+                int acc_of[G];
 #pragma unroll
                 for (int u = 0; u < G; ++u) {
-                    if (u >= gmax) break;
-                    const int64_t t = tg + u;
-                    tile_info<TR>(s_toff, s_seq, B, t, b, row0, row_end);
-                    if (b != cur) {
-                        if (u > 0) break;
-                        slot = qn & 1;
-                        if (!mbar_wait(&qfull[slot], (qn >> 1) & 1, abort_v, kWaitLimitNs)) { ok = false; break; }
-                        cur = b;
-                        ++qn;
-                    }
+                    if (u >= gn) break;
                     if (!mbar_wait(&tempty[acc], aph ^ 1, abort_v, kWaitLimitNs)) { ok = false; break; }
                     if (!mbar_wait(&full[st], ph, abort_v, kWaitLimitNs)) { ok = false; break; }
-                    // start-address fields advance in 16-byte units
-                    a_d[u] = a_desc0 + uint64_t((st * C::kStageBytes) >> 4);
-                    b_d[u] = b_desc0 + uint64_t((slot * QIMG) >> 4);
+                    a_d[u] = a_cur;
                     d_t[u] = tmem_base + uint32_t(acc * TILEC);
-                    st_of[u] = st;
                     acc_of[u] = acc;
-                    // the next tile starts a new sequence when it is the first tile of a later one
-                    rel_of[u] = ((t + 1 >= t1) || (t + 1 >= s_toff[b + 1])) ? (qn - 1) % kRel : -1;
-                    if (++st == S) { st = 0; ph ^= 1; }
+                    a_cur += kStageStep;
+                    if (++st == S) { st = 0; ph ^= 1; a_cur = a_desc0; }
                     if (++acc == KACC) { acc = 0; aph ^= 1; }
-                    ++gn;
                 }
                 if (!ok) break;
-                tg += gn;
+                t += gn;
                 tc_fence_after();
                 if (KIND == BF16_D128) {
 #pragma unroll
@@ -538,7 +601,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                         for (int u = 0; u < G; ++u)
                             if (u < gn)
                                 mma_f16(d_t[u], a_d[u] + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                                        b_d[u] + uint64_t(((kk >> 2) * (H * 128) + (kk & 3) * 32) >> 4), IDESC,
+                                        b_cur + uint64_t(((kk >> 2) * (H * 128) + (kk & 3) * 32) >> 4), IDESC,
                                         kk > 0);
                 } else if (KIND == BF16_D64) {
 #pragma unroll
@@ -546,7 +609,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
 #pragma unroll
                         for (int u = 0; u < G; ++u)
                             if (u < gn)
-                                mma_f16(d_t[u], a_d[u] + uint64_t((kk * 32) >> 4), b_d[u] + uint64_t((kk * 32) >> 4),
+                                mma_f16(d_t[u], a_d[u] + uint64_t((kk * 32) >> 4), b_cur + uint64_t((kk * 32) >> 4),
                                         IDESC, kk > 0);
                 } else {
                     // the two 128-row halves of the tile (16 KB apart in the stage) into their own
@@ -556,16 +619,13 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
 #pragma unroll
                         for (int sub = 0; sub < 2; ++sub)
                             mma_f8(d_t[0] + uint32_t(sub * SUBC), a_d[0] + uint64_t((sub * 16384 + kk * 32) >> 4),
-                                   b_d[0] + uint64_t((kk * 32) >> 4), IDESC, kk > 0);
+                                   b_cur + uint64_t((kk * 32) >> 4), IDESC, kk > 0);
                 }
                 issued = true;
 #pragma unroll
-                for (int u = 0; u < G; ++u) {
-                    if (u >= gn) break;
-                    mma_commit(&empty[st_of[u]]);
-                    mma_commit(&tfull[acc_of[u]]);
-                    if (rel_of[u] >= 0) mma_commit(&qrel[rel_of[u]]);   // this sequence's operand is no longer read
-                }
+                for (int u = 0; u < G; ++u)
+                    if (u < gn) mma_commit(&tdone[acc_of[u]]);   // accumulator ready, stage free
+                if (t == gend) mma_commit(&qrel[qn % kRel]);      // this sequence's operand is no longer read
             }
             if (issued) {
                 // every issued MMA has finished before TMEM is released
@@ -586,16 +646,6 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         const int64_t tfirst = C::kSub == 2 ? t0 : t0 + grp;
         int b = 0, cur = -1, ord = -1, released = 0;
         int64_t row0, row_end;
-        // row scale of this thread's row in tile t (e4m3 keys), loaded one tile of this group ahead
-        auto scale_of = [&](int64_t t) -> float {
-            if (KIND != E4M3_D128 || t >= t1) return 1.f;
-            int bb = b;
-            int64_t r0, r1;
-            tile_info<TR>(s_toff, s_seq, B, t, bb, r0, r1);
-            const int64_t r = r0 + sub * kRows + quarter * 32 + lane;
-            if (r >= r1) return 1.f;
-            return __ldg(k_scale + (LISTED ? s_base[bb] + idx[r] : r));
-        };
         // a sequence ordinal this warp will not read again frees its slot (1 of the 8 epilogue arrivals)
         auto release_to = [&](int upto) {
             for (; released < upto; ++released)
@@ -620,7 +670,6 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 if (ew == 0 && lane == 0) mbar_arrive(&qfull[o]);
             }
         }
-        float sc_next = scale_of(tfirst);
         // ordinal of each tile: count the sequence changes over every tile of the range (both groups')
         int ob = 0, ocur = -1, onum = -1;
         int64_t orow0, orow1, u_next = t0;
@@ -644,11 +693,12 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             }
             const float *wq = wsm + (ord & 1) * H;
             const int64_t row = row0 + sub * kRows + quarter * 32 + lane;   // entry (full) or list position
-            const float sc = sc_next;
-            sc_next = scale_of(t + kStep);
-            ok = mbar_wait(&tfull[acc], aph, abort_v, kWaitLimitNs);
+            ok = mbar_wait(&tdone[acc], aph, abort_v, kWaitLimitNs);
+            // the row scales landed long before (loaded with the keys); read before the release
+            if (kScales) ok = ok && mbar_wait(&sfull[i % RS], uint32_t((i / RS) & 1), abort_v, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
             tc_fence_after();
+            const float sc = kScales ? s_scale[int(i % RS) * TR + sub * kRows + quarter * 32 + lane] : 1.f;
             const uint32_t taddr =
                 tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * TILEC + sub * SUBC);
             float za = 0.f, zb = 0.f, zc = 0.f, zd = 0.f;   // four short dependency chains
@@ -731,7 +781,9 @@ template <int KIND, int H>
 size_t smem_bytes(int B) {
     using C = Cfg<KIND>;
     return 1024 + size_t(C::kStages) * C::kStageBytes + 2 * qimg_bytes<KIND, H>() +
-           (2 * C::kStages + 2 + kRel + 2 * kAccMax + 1) * 8 + 16 + 16 + 2 * H * 4 + size_t(B + 1) * 24 + 64;
+           (C::kStages + 2 + kRel + 2 * kAccMax + 1 + kScaleSlotsMax) * 8 + 16 + 16 + 2 * H * 4 +
+           size_t(B + 1) * 24 + 16 + (KIND == E4M3_D128 ? size_t(C::kStages + acc_tiles<KIND, H>()) * tile_rows<KIND>() * 4 : 0) +
+           64;
 }
 
 template <int KIND, int H>

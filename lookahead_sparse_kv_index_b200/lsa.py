@@ -36,7 +36,7 @@ EXPORTS = [
     "lsa_select", "lsa_topk", "lsa_gather", "lsa_sparse_attn_workspace_size", "lsa_sparse_attn",
     "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
     "lsa_ctx_set_graphs", "lsa_ctx_set_timing", "lsa_ctx_stage_times", "lsa_ctx_reset_counters",
-    "lsa_ctx_launches",
+    "lsa_ctx_launches", "lsa_selftest_bounded_wait",
 ]
 
 
@@ -92,6 +92,7 @@ _sig("lsa_ctx_set_timing", i32, [P, i32])
 _sig("lsa_ctx_stage_times", i32, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)])
 _sig("lsa_ctx_reset_counters", i32, [P])
 _sig("lsa_ctx_launches", i64, [P])
+_sig("lsa_selftest_bounded_wait", i32, [i64, P, P, P])
 
 lib = _L
 
@@ -151,6 +152,12 @@ def select_noalloc(z, seq_off, n_total, kept_idx, capacity, kept_off, mask, err,
     B = seq_off.numel() - 1
     _check(_L.lsa_select_noalloc(_ptr(z), _ptr(seq_off), n_total, B, _ptr(kept_idx), capacity, _ptr(kept_off),
                                  _ptr(mask), _ptr(err), _stream(stream)), "lsa_select_noalloc")
+
+
+def selftest_bounded_wait(limit_ns, err, waited_ns, stream=None):
+    """Runs a bounded device wait on a barrier nothing arrives at (see lsa.h)."""
+    _check(_L.lsa_selftest_bounded_wait(int(limit_ns), _ptr(err), _ptr(waited_ns), _stream(stream)),
+           "lsa_selftest_bounded_wait")
 
 
 def topk(z, z_by_entry, seq_off, kept_idx, kept_off, kept_capacity, k, topk_idx, topk_pos, topk_cnt, stream=None):

@@ -80,6 +80,9 @@ def test_other_entry_points_reject_bad_arguments(lsa):
     assert L.lsa_sparse_attn(big, 2, big, 512, 0, 0, big, 1, 128, 512, 16, 1.0, big, None, big, 1 << 30, None, None) == 5
     assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 512, 16, -1.0, big, None, big, 1 << 30, None, None) == 1
     assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 512, 16, 1.0, big, None, big, 16, None, None) == 1
+    assert L.lsa_selftest_bounded_wait(10, big, big, None) == 1              # limit below 1 us
+    assert L.lsa_selftest_bounded_wait(1 << 40, big, big, None) == 1         # limit above 100 ms
+    assert L.lsa_selftest_bounded_wait(1000000, None, big, None) == 1        # no error word
 
 
 def test_ctx_create_rejects_bad_params(lsa):
