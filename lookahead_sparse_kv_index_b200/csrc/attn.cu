@@ -147,11 +147,13 @@ attn_partial(const T *__restrict__ Q, const T *__restrict__ kv, int64_t stride, 
 
 // Merge of the chunk partials of one (head, sequence):
 //   M = max_c m_c,  w_c = e^{m_c - M},  L = sum_c l_c w_c,  o = sum_c w_c o_c / L,
-//   lse = M + log L;  a chunk with m_c = -inf (no selected row) has weight 0.
-// Every thread loads the (m, l) of all chunks and its four columns of every
-// chunk in batches of up to 16 independent loads, then reduces on its own (the
-// (m, l) are the same for the whole block), so no block synchronisation sits
-// between the loads and the arithmetic.
+//   lse = M + log L;  a chunk with m_c = -inf (no selected row) has weight 0 and
+// its o is never read into the sum.
+// The kernel is a chain of dependent L2 round trips unless the loads go out
+// together: with up to 16 chunks every thread issues the (m, l) of all chunks
+// and its four columns of every chunk at once, then reduces on its own (the
+// (m, l) are the same for the whole block, so no block synchronisation sits
+// between the loads and the arithmetic).  More chunks: the same in batches.
 template <typename T>
 __global__ void __launch_bounds__(128)
 attn_combine(const float *__restrict__ part_o, const float *__restrict__ part_ml, int nchunks, int Hq, int D,
@@ -160,34 +162,88 @@ attn_combine(const float *__restrict__ part_o, const float *__restrict__ part_ml
     pdl_wait();   // partials come from the preceding kernel
     const int h = blockIdx.x, b = blockIdx.y;
     const int64_t p0 = int64_t(b) * nchunks * Hq + h;   // partial index of chunk 0; chunk c adds c * Hq
+    const float2 *ml = reinterpret_cast<const float2 *>(part_ml);
+    const int64_t ob = (int64_t(b) * Hq + h) * D;
+    const int col0 = 4 * threadIdx.x;
+    if (nchunks <= kBatch) {
+        float2 mlv[kBatch];
+        float4 v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            mlv[u] = u < nchunks ? ml[p0 + int64_t(u) * Hq] : make_float2(-INFINITY, 0.f);
+            v[u] = (u < nchunks && col0 < D) ? *reinterpret_cast<const float4 *>(part_o + (p0 + int64_t(u) * Hq) * D + col0)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) M = fmaxf(M, mlv[u].x);
+        float wgt[kBatch], L = 0.f;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            wgt[u] = mlv[u].x == -INFINITY ? 0.f : expf(mlv[u].x - M);
+            L += mlv[u].y * wgt[u];
+        }
+        const float inv = M == -INFINITY ? 0.f : 1.f / L;
+        for (int col = col0; col < D; col += 4 * blockDim.x) {
+            if (col != col0) {
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u)
+                    if (u < nchunks) v[u] = *reinterpret_cast<const float4 *>(part_o + (p0 + int64_t(u) * Hq) * D + col);
+            }
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                if (mlv[u].x == -INFINITY) continue;   // includes u >= nchunks
+                a.x = fmaf(wgt[u], v[u].x, a.x); a.y = fmaf(wgt[u], v[u].y, a.y);
+                a.z = fmaf(wgt[u], v[u].z, a.z); a.w = fmaf(wgt[u], v[u].w, a.w);
+            }
+            Elem<T>::put(out, ob + col, a.x * inv);
+            Elem<T>::put(out, ob + col + 1, a.y * inv);
+            Elem<T>::put(out, ob + col + 2, a.z * inv);
+            Elem<T>::put(out, ob + col + 3, a.w * inv);
+        }
+        if (threadIdx.x == 0 && lse) lse[int64_t(b) * Hq + h] = M == -INFINITY ? -INFINITY : M + logf(L);
+        return;
+    }
+    // more chunks than one batch: (m, l) in batches, then the columns in batches
     float M = -INFINITY;
-    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, part_ml[(p0 + int64_t(c) * Hq) * 2]);
+    for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
+        float2 mlv[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+            mlv[u] = c0 + u < nchunks ? ml[p0 + int64_t(c0 + u) * Hq] : make_float2(-INFINITY, 0.f);
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) M = fmaxf(M, mlv[u].x);
+    }
     float L = 0.f;
     if (M != -INFINITY)
-        for (int c = 0; c < nchunks; ++c) {
-            const float m = part_ml[(p0 + int64_t(c) * Hq) * 2];
-            if (m != -INFINITY) L += part_ml[(p0 + int64_t(c) * Hq) * 2 + 1] * expf(m - M);
+        for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
+            float2 mlv[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                mlv[u] = c0 + u < nchunks ? ml[p0 + int64_t(c0 + u) * Hq] : make_float2(-INFINITY, 0.f);
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                if (mlv[u].x != -INFINITY) L += mlv[u].y * expf(mlv[u].x - M);
         }
     const float inv = M == -INFINITY ? 0.f : 1.f / L;
-    const int64_t ob = (int64_t(b) * Hq + h) * D;
-    for (int col = 4 * threadIdx.x; col < D; col += 4 * blockDim.x) {
+    for (int col = col0; col < D; col += 4 * blockDim.x) {
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
         if (M != -INFINITY)
             for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
                 float4 v[kBatch];
+                float2 mlv[kBatch];
 #pragma unroll
                 for (int u = 0; u < kBatch; ++u) {
                     const int c = c0 + u;
+                    mlv[u] = c < nchunks ? ml[p0 + int64_t(c) * Hq] : make_float2(-INFINITY, 0.f);
                     v[u] = c < nchunks ? *reinterpret_cast<const float4 *>(part_o + (p0 + int64_t(c) * Hq) * D + col)
                                        : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
 #pragma unroll
                 for (int u = 0; u < kBatch; ++u) {
-                    const int c = c0 + u;
-                    if (c >= nchunks) break;
-                    const float m = part_ml[(p0 + int64_t(c) * Hq) * 2];
-                    if (m == -INFINITY) continue;   // an empty chunk's o is never read into the sum
-                    const float w = expf(m - M);
+                    if (mlv[u].x == -INFINITY) continue;   // an empty chunk's o is never read into the sum
+                    const float w = expf(mlv[u].x - M);
                     a.x = fmaf(w, v[u].x, a.x); a.y = fmaf(w, v[u].y, a.y);
                     a.z = fmaf(w, v[u].z, a.z); a.w = fmaf(w, v[u].w, a.w);
                 }
