@@ -13,7 +13,7 @@
 //      start while the others are still in flight; padding rows are
 //      zero-filled;
 //   2. warp 5 streams Q[b] (128 x 512 bf16) by TMA in 8 slices of 64 columns
-//      through a 3-stage ring;
+//      through a 5-stage ring (P later reuses its memory);
 //   3. warp 4 issues S = Q K^T (M = 128 heads, N = 128 rows, K = 512) into
 //      TMEM columns 0..127;
 //   4. warps 0-3 (one head per thread) read S, compute the chunk's row max m,
@@ -39,7 +39,7 @@ using namespace ptx;
 constexpr int kHq = 128;
 constexpr int kD = 512;
 constexpr int kRowsPerCta = 128;
-constexpr int kQStages = 3;
+constexpr int kQStages = 5;   // 5 x 16 KB of Q in flight; P reuses this ring once S is done
 constexpr int kThreads = 192;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kTmemCols = 512;
@@ -79,9 +79,12 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *kvs = smem;                         // 128 KB
-    uint8_t *qs = kvs + kKvBytes;                // 3 x 16 KB
-    uint8_t *ps = qs + kQStages * kQStageBytes;  // 32 KB
-    uint64_t *qfull = reinterpret_cast<uint64_t *>(ps + kPBytes);
+    uint8_t *qs = kvs + kKvBytes;                // kQStages x 16 KB
+    // P (32 KB) overwrites the Q ring: it is written only after every S MMA has completed, and by then
+    // every Q load has landed (each was waited for by an S MMA)
+    uint8_t *ps = qs;
+    static_assert(kQStages * kQStageBytes >= kPBytes, "P lives in the Q ring");
+    uint64_t *qfull = reinterpret_cast<uint64_t *>(qs + kQStages * kQStageBytes);
     uint64_t *qempty = qfull + kQStages;
     uint64_t *kv_full = qempty + kQStages;       // [kD / 64] column blocks of the rows
     uint64_t *s_full = kv_full + kD / 64;
@@ -91,6 +94,7 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     int *s_rows = abort_flag + 1;                // [128]
     int *s_nvalid = s_rows + kRowsPerCta;
+    uint32_t *s_valid = reinterpret_cast<uint32_t *>(s_nvalid + 1);   // [4] bit j % 32 of word j / 32: row j selected
 
     const int chunk = blockIdx.x, b = blockIdx.y, nchunks = gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -123,6 +127,8 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
         const int r = i < k ? rows[int64_t(b) * k + i] : -1;
         s_rows[threadIdx.x] = r;
         if (r >= 0) atomicAdd(s_nvalid, 1);
+        const uint32_t bal = __ballot_sync(0xffffffffu, r >= 0);   // threads 0..127: whole warps
+        if ((threadIdx.x & 31) == 0) s_valid[threadIdx.x >> 5] = bal;
     }
     if (warp == 4) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -177,36 +183,54 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
         // warps 0-3 take every branch below together (they meet at named barriers)
         if (named_barrier_and(1, 128, ok)) {
             tc_fence_after();
-            uint32_t sr[kRowsPerCta];
             const uint32_t taddr = tmem + (uint32_t(quarter * 32) << 16);
+            // S is read from TMEM 16 columns at a time, in two passes (row max, then weights): rolled
+            // loops keep this phase's code and registers small.  Selected rows come from a bit mask; a
+            // full chunk (the common case) skips the tests.  Max and sum run as four chains.
+            const bool all_valid = (s_valid[0] & s_valid[1] & s_valid[2] & s_valid[3]) == 0xffffffffu;
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+            for (int c = 0; c < kRowsPerCta / 16; ++c) {
+                uint32_t r16[16];
+                tmem_ld_32x32b_x16(taddr + c * 16, r16);
+                tmem_ld_wait();
+                const uint32_t vb = all_valid ? 0xffffu : (s_valid[c >> 1] >> ((c & 1) * 16)) & 0xffffu;
 #pragma unroll
-            for (int c = 0; c < kRowsPerCta / 16; ++c)
-                tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c * 16]));
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < kRowsPerCta; ++j)
-                if (s_rows[j] >= 0) m = fmaxf(m, scale * __uint_as_float(sr[j]));
+                for (int u = 0; u < 16; ++u)
+                    if ((vb >> u) & 1u) mq[u & 3] = fmaxf(mq[u & 3], scale * __uint_as_float(r16[u]));
+            }
+            m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+            float lq[4] = {0.f, 0.f, 0.f, 0.f};
             // P in bf16, K-major swizzled: block (j / 64), row t, 16-byte chunk (j % 64) / 8
             const uint32_t p_u32 = smem_u32(ps);
+#pragma unroll 1
+            for (int c = 0; c < kRowsPerCta / 16; ++c) {
+                uint32_t r16[16];
+                tmem_ld_32x32b_x16(taddr + c * 16, r16);
+                tmem_ld_wait();
+                const uint32_t vb = all_valid ? 0xffffu : (s_valid[c >> 1] >> ((c & 1) * 16)) & 0xffffu;
+                uint32_t packed[8];
 #pragma unroll
-            for (int c = 0; c < kRowsPerCta / 8; ++c) {
-                uint32_t packed[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int j0 = c * 8 + 2 * u, j1 = j0 + 1;
-                    const float p0 = s_rows[j0] >= 0 ? __expf(scale * __uint_as_float(sr[j0]) - m) : 0.f;
-                    const float p1 = s_rows[j1] >= 0 ? __expf(scale * __uint_as_float(sr[j1]) - m) : 0.f;
+                for (int u = 0; u < 8; ++u) {
+                    const int j0 = 2 * u, j1 = j0 + 1;
+                    const float p0 = ((vb >> j0) & 1u) ? __expf(scale * __uint_as_float(r16[j0]) - m) : 0.f;
+                    const float p1 = ((vb >> j1) & 1u) ? __expf(scale * __uint_as_float(r16[j1]) - m) : 0.f;
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                     // the normaliser sums the bf16-rounded weights the MMA actually uses
                     const float2 back = __bfloat1622float2(h2);
-                    l += back.x + back.y;
+                    lq[u & 3] += back.x + back.y;
                     packed[u] = *reinterpret_cast<const uint32_t *>(&h2);
                 }
-                const uint32_t dst = p_u32 + (c >> 3) * (kHq * 128) + t * 128 + (((c & 7) ^ (t & 7)) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(packed[0]), "r"(packed[1]),
-                             "r"(packed[2]), "r"(packed[3])
-                             : "memory");
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int cc = 2 * c + h;   // 16-byte chunk of the row (8 weights)
+                    const uint32_t dst = p_u32 + (cc >> 3) * (kHq * 128) + t * 128 + (((cc & 7) ^ (t & 7)) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(packed[4 * h]),
+                                 "r"(packed[4 * h + 1]), "r"(packed[4 * h + 2]), "r"(packed[4 * h + 3])
+                                 : "memory");
+                }
             }
+            l = (lq[0] + lq[1]) + (lq[2] + lq[3]);
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(p_full);
@@ -336,8 +360,8 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-constexpr size_t kSmemBytes = 1024 + size_t(kKvBytes) + size_t(kQStages) * kQStageBytes + kPBytes +
-                              (2 * kQStages + kD / 64 + 3) * 8 + 16 + (kRowsPerCta + 2) * 4 + 64;
+constexpr size_t kSmemBytes = 1024 + size_t(kKvBytes) + size_t(kQStages) * kQStageBytes +
+                              (2 * kQStages + kD / 64 + 3) * 8 + 16 + (kRowsPerCta + 2) * 4 + 16 + 64;
 
 }  // namespace
 
