@@ -154,9 +154,17 @@ attn_partial(const T *__restrict__ Q, const T *__restrict__ kv, int64_t stride, 
 // and its four columns of every chunk at once, then reduces on its own (the
 // (m, l) are the same for the whole block, so no block synchronisation sits
 // between the loads and the arithmetic).  More chunks: the same in batches.
-template <typename T>
+// four consecutive partial values as fp32 (partials in fp32 or bf16)
+__device__ __forceinline__ float4 load4(const float *p, int64_t i) { return *reinterpret_cast<const float4 *>(p + i); }
+__device__ __forceinline__ float4 load4(const uint16_t *p, int64_t i) {
+    const uint2 w = *reinterpret_cast<const uint2 *>(p + i);
+    return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u), __uint_as_float(w.y << 16),
+                       __uint_as_float(w.y & 0xFFFF0000u));
+}
+
+template <typename T, typename TP>
 __global__ void __launch_bounds__(128)
-attn_combine(const float *__restrict__ part_o, const float *__restrict__ part_ml, int nchunks, int Hq, int D,
+attn_combine(const TP *__restrict__ part_o, const float *__restrict__ part_ml, int nchunks, int Hq, int D,
              T *__restrict__ out, float *__restrict__ lse) {
     constexpr int kBatch = 16;
     pdl_wait();   // partials come from the preceding kernel
@@ -171,7 +179,7 @@ attn_combine(const float *__restrict__ part_o, const float *__restrict__ part_ml
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             mlv[u] = u < nchunks ? ml[p0 + int64_t(u) * Hq] : make_float2(-INFINITY, 0.f);
-            v[u] = (u < nchunks && col0 < D) ? *reinterpret_cast<const float4 *>(part_o + (p0 + int64_t(u) * Hq) * D + col0)
+            v[u] = (u < nchunks && col0 < D) ? load4(part_o, (p0 + int64_t(u) * Hq) * D + col0)
                                              : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         float M = -INFINITY;
@@ -188,7 +196,7 @@ attn_combine(const float *__restrict__ part_o, const float *__restrict__ part_ml
             if (col != col0) {
 #pragma unroll
                 for (int u = 0; u < kBatch; ++u)
-                    if (u < nchunks) v[u] = *reinterpret_cast<const float4 *>(part_o + (p0 + int64_t(u) * Hq) * D + col);
+                    if (u < nchunks) v[u] = load4(part_o, (p0 + int64_t(u) * Hq) * D + col);
             }
             float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -237,8 +245,7 @@ attn_combine(const float *__restrict__ part_o, const float *__restrict__ part_ml
                 for (int u = 0; u < kBatch; ++u) {
                     const int c = c0 + u;
                     mlv[u] = c < nchunks ? ml[p0 + int64_t(c) * Hq] : make_float2(-INFINITY, 0.f);
-                    v[u] = c < nchunks ? *reinterpret_cast<const float4 *>(part_o + (p0 + int64_t(c) * Hq) * D + col)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[u] = c < nchunks ? load4(part_o, (p0 + int64_t(c) * Hq) * D + col) : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
 #pragma unroll
                 for (int u = 0; u < kBatch; ++u) {
@@ -256,7 +263,8 @@ attn_combine(const float *__restrict__ part_o, const float *__restrict__ part_ml
     if (threadIdx.x == 0 && lse) lse[int64_t(b) * Hq + h] = M == -INFINITY ? -INFINITY : M + logf(L);
 }
 
-// Partial workspace: o [B, nchunks, Hq, D] fp32, then (m, l) [B, nchunks, Hq, 2] fp32.
+// Partial workspace: o [B, nchunks, Hq, D] fp32 (bf16 from the tensor-core chunks, which use the
+// first half), then (m, l) [B, nchunks, Hq, 2] fp32.
 struct Parts {
     float *o, *ml;
 };
@@ -272,10 +280,14 @@ lsa_status launch_t(const void *Q, const void *kv, int64_t stride, int64_t k_off
     int nchunks;
     Parts pp;
     if (sparse_attn_tc_supported(sizeof(T) == 2 ? LSA_BF16 : LSA_F32, k_off, v_off, Hq, D)) {
+        // tensor-core chunks write bf16 partials (the fp32 workspace has room for them)
         nchunks = (k + sparse_attn_tc_chunk() - 1) / sparse_attn_tc_chunk();
         pp = parts(workspace, B, Hq, D, nchunks);
         lsa_status s = launch_sparse_attn_tc(Q, kv, stride, k_off, rows, B, k, scale, pp.o, pp.ml, err, st);
         if (s != LSA_OK) return s;
+        LSA_CUDA(launch_pdl(attn_combine<T, uint16_t>, dim3(Hq, B), dim3(128), 0, st,
+                            reinterpret_cast<const uint16_t *>(pp.o), static_cast<const float *>(pp.ml), nchunks,
+                            Hq, D, static_cast<T *>(out), lse));
     } else {
         nchunks = (k + kChunk - 1) / kChunk;
         pp = parts(workspace, B, Hq, D, nchunks);
@@ -289,9 +301,9 @@ lsa_status launch_t(const void *Q, const void *kv, int64_t stride, int64_t k_off
         kern<<<grid, kAttnThreads, smem, st>>>(static_cast<const T *>(Q), static_cast<const T *>(kv), stride,
                                                k_off, v_off, rows, Hq, D, k, scale, pp.o, pp.ml);
         LSA_LAUNCHED("attn_partial");
+        LSA_CUDA(launch_pdl(attn_combine<T, float>, dim3(Hq, B), dim3(128), 0, st, static_cast<const float *>(pp.o),
+                            static_cast<const float *>(pp.ml), nchunks, Hq, D, static_cast<T *>(out), lse));
     }
-    LSA_CUDA(launch_pdl(attn_combine<T>, dim3(Hq, B), dim3(128), 0, st, static_cast<const float *>(pp.o),
-                        static_cast<const float *>(pp.ml), nchunks, Hq, D, static_cast<T *>(out), lse));
     LSA_LAUNCHED("attn_combine");
     return LSA_OK;
 }

@@ -23,8 +23,8 @@
 //      0..511, reading the SAME smem rows as V through an MN-major descriptor
 //      (no transpose, no second copy of the rows);
 //   6. warps 0-3 read O in 64-column blocks into the freed row buffer
-//      (128-byte swizzle, four staging buffers) and write the fp32 partial
-//      with TMA stores; (m, l) per head.
+//      (128-byte swizzle, one staging buffer per block) and write the
+//      partial in bf16 with TMA stores; (m, l) per head in fp32.
 // The combine kernel (attn.cu) merges the chunks.  Every wait is bounded.
 #include <cuda.h>
 
@@ -48,7 +48,8 @@ constexpr int kKvBytes = kRowsPerCta * kD * 2;   // 128 KB: 8 blocks of [128 row
 constexpr int kKvBlock = kRowsPerCta * 128;      // 16 KB
 constexpr int kQStageBytes = kHq * 128;          // 16 KB: one 64-column slice of Q
 constexpr int kPBytes = kHq * kRowsPerCta * 2;   // 32 KB: 2 blocks of [128 heads x 128 B]
-constexpr int kOStageBytes = kHq * 64 * 4;       // 32 KB: [128 heads][64 fp32] staging of one O block
+constexpr int kOStageBytes = kHq * 64 * 2;       // 16 KB: [128 heads][64 bf16] staging of one O block
+static_assert((kD / 64) * kOStageBytes <= kKvBytes, "every O block has its own staging buffer in the row buffer");
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -184,37 +185,39 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
         if (named_barrier_and(1, 128, ok)) {
             tc_fence_after();
             const uint32_t taddr = tmem + (uint32_t(quarter * 32) << 16);
-            // S is read from TMEM 16 columns at a time, in two passes (row max, then weights): rolled
+            // S is read from TMEM 32 columns at a time, in two passes (row max, then weights): rolled
             // loops keep this phase's code and registers small.  Selected rows come from a bit mask; a
             // full chunk (the common case) skips the tests.  Max and sum run as four chains.
             const bool all_valid = (s_valid[0] & s_valid[1] & s_valid[2] & s_valid[3]) == 0xffffffffu;
             float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-            for (int c = 0; c < kRowsPerCta / 16; ++c) {
-                uint32_t r16[16];
-                tmem_ld_32x32b_x16(taddr + c * 16, r16);
+            for (int c = 0; c < kRowsPerCta / 32; ++c) {
+                uint32_t r32[32];
+                tmem_ld_32x32b_x16(taddr + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&r32[0]));
+                tmem_ld_32x32b_x16(taddr + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r32[16]));
                 tmem_ld_wait();
-                const uint32_t vb = all_valid ? 0xffffu : (s_valid[c >> 1] >> ((c & 1) * 16)) & 0xffffu;
+                const uint32_t vb = all_valid ? 0xffffffffu : s_valid[c];
 #pragma unroll
-                for (int u = 0; u < 16; ++u)
-                    if ((vb >> u) & 1u) mq[u & 3] = fmaxf(mq[u & 3], scale * __uint_as_float(r16[u]));
+                for (int u = 0; u < 32; ++u)
+                    if ((vb >> u) & 1u) mq[u & 3] = fmaxf(mq[u & 3], scale * __uint_as_float(r32[u]));
             }
             m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
             float lq[4] = {0.f, 0.f, 0.f, 0.f};
             // P in bf16, K-major swizzled: block (j / 64), row t, 16-byte chunk (j % 64) / 8
             const uint32_t p_u32 = smem_u32(ps);
 #pragma unroll 1
-            for (int c = 0; c < kRowsPerCta / 16; ++c) {
-                uint32_t r16[16];
-                tmem_ld_32x32b_x16(taddr + c * 16, r16);
+            for (int c = 0; c < kRowsPerCta / 32; ++c) {
+                uint32_t r32[32];
+                tmem_ld_32x32b_x16(taddr + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&r32[0]));
+                tmem_ld_32x32b_x16(taddr + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r32[16]));
                 tmem_ld_wait();
-                const uint32_t vb = all_valid ? 0xffffu : (s_valid[c >> 1] >> ((c & 1) * 16)) & 0xffffu;
-                uint32_t packed[8];
+                const uint32_t vb = all_valid ? 0xffffffffu : s_valid[c];
+                uint32_t packed[16];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 16; ++u) {
                     const int j0 = 2 * u, j1 = j0 + 1;
-                    const float p0 = ((vb >> j0) & 1u) ? __expf(scale * __uint_as_float(r16[j0]) - m) : 0.f;
-                    const float p1 = ((vb >> j1) & 1u) ? __expf(scale * __uint_as_float(r16[j1]) - m) : 0.f;
+                    const float p0 = ((vb >> j0) & 1u) ? __expf(scale * __uint_as_float(r32[j0]) - m) : 0.f;
+                    const float p1 = ((vb >> j1) & 1u) ? __expf(scale * __uint_as_float(r32[j1]) - m) : 0.f;
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                     // the normaliser sums the bf16-rounded weights the MMA actually uses
                     const float2 back = __bfloat1622float2(h2);
@@ -222,8 +225,8 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
                     packed[u] = *reinterpret_cast<const uint32_t *>(&h2);
                 }
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int cc = 2 * c + h;   // 16-byte chunk of the row (8 weights)
+                for (int h = 0; h < 4; ++h) {
+                    const int cc = 4 * c + h;   // 16-byte chunk of the row (8 weights)
                     const uint32_t dst = p_u32 + (cc >> 3) * (kHq * 128) + t * 128 + (((cc & 7) ^ (t & 7)) << 4);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(packed[4 * h]),
                                  "r"(packed[4 * h + 1]), "r"(packed[4 * h + 2]), "r"(packed[4 * h + 3])
@@ -234,40 +237,40 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(p_full);
-            // ---- 6. read O and write the chunk's partial: 64-column blocks staged in the (now free)
-            // row buffer, one TMA store per block; four staging buffers rotate
+            // ---- 6. read O and write the chunk's partial (bf16): 64-column blocks staged in the (now
+            // free) row buffer, each in its own 16 KB buffer, one TMA store per block
             ok = mbar_wait(o_full, 0, abort_v, kWaitLimitNs);
             // the block loop below synchronises these 128 threads: agree on one outcome first
             if (named_barrier_and(1, 128, ok)) {
                 tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < kD / 64; ++c) {
-                    float *sb = reinterpret_cast<float *>(kvs + (c & 3) * kOStageBytes);   // 2 halves of [128][32]
-                    if (c >= 4) {
-                        if (t == 0) bulk_wait_read<3>();   // the store issued four blocks ago has read its buffer
-                        named_barrier(1, 128);
-                    }
+                    uint8_t *sb = kvs + c * kOStageBytes;   // [128 rows x 128 B]
                     uint32_t o[64];
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
                         tmem_ld_32x32b_x16(taddr + c * 64 + q4 * 16, *reinterpret_cast<uint32_t(*)[16]>(&o[q4 * 16]));
                     tmem_ld_wait();
-                    // two [128 rows x 32 fp32] halves in the 128-byte-swizzled layout (16-byte chunk
-                    // u of row t at chunk u ^ (t % 8)): conflict-free writes, one TMA store per half
+                    // [128 rows x 64 bf16] in the 128-byte-swizzled layout (16-byte chunk u of row t at
+                    // chunk u ^ (t % 8)): conflict-free writes
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
+                    for (int u = 0; u < 8; ++u) {
+                        uint32_t w4[4];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            *reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(sb) + h * 16384 + t * 128 +
-                                                        ((u ^ (t & 7)) << 4)) =
-                                make_float4(__uint_as_float(o[h * 32 + 4 * u]), __uint_as_float(o[h * 32 + 4 * u + 1]),
-                                            __uint_as_float(o[h * 32 + 4 * u + 2]),
-                                            __uint_as_float(o[h * 32 + 4 * u + 3]));
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[8 * u + 2 * e]),
+                                                                            __uint_as_float(o[8 * u + 2 * e + 1]));
+                            w4[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                        }
+                        const uint32_t dst = smem_u32(sb) + t * 128 + ((u ^ (t & 7)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w4[0]), "r"(w4[1]),
+                                     "r"(w4[2]), "r"(w4[3])
+                                     : "memory");
+                    }
                     fence_proxy_async_smem();
                     named_barrier(1, 128);
                     if (t == 0) {
                         tma_store_2d(&omap, sb, c * 64, int(pbase));
-                        tma_store_2d(&omap, reinterpret_cast<uint8_t *>(sb) + 16384, c * 64 + 32, int(pbase));
                         bulk_commit();
                     }
                 }
@@ -372,7 +375,7 @@ bool sparse_attn_tc_supported(lsa_dtype dtype, int64_t k_off, int64_t v_off, int
 int sparse_attn_tc_chunk() { return kRowsPerCta; }
 
 lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, int64_t k_off,
-                                 const int32_t *rows, int32_t B, int32_t k, float scale, float *part_o,
+                                 const int32_t *rows, int32_t B, int32_t k, float scale, void *part_o,
                                  float *part_ml, int32_t *err, cudaStream_t st) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) {
@@ -391,12 +394,12 @@ lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, 
         set_error("lsa_sparse_attn: cuTensorMapEncodeTiled failed (%d)", int(r));
         return LSA_ERR_CUDA;
     }
-    CUtensorMap omap;   // partial O [B * nchunks * 128 rows, 512] fp32, stored in swizzled [128 x 32] boxes
+    CUtensorMap omap;   // partial O [B * nchunks * 128 rows, 512] bf16, stored in swizzled [128 x 64] boxes
     const int nchunks_o = (k + kRowsPerCta - 1) / kRowsPerCta;
     const cuuint64_t odims[2] = {cuuint64_t(kD), cuuint64_t(B) * nchunks_o * kHq};
-    const cuuint64_t ostrides[1] = {cuuint64_t(kD) * 4};
-    const cuuint32_t obox[2] = {32, 128};
-    r = enc(&omap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, part_o, odims, ostrides, obox, estr,
+    const cuuint64_t ostrides[1] = {cuuint64_t(kD) * 2};
+    const cuuint32_t obox[2] = {64, 128};
+    r = enc(&omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, part_o, odims, ostrides, obox, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {

@@ -115,7 +115,7 @@ lsa_status launch_sparse_attn(const void *Q, lsa_dtype dtype, const void *kv, in
 bool sparse_attn_tc_supported(lsa_dtype dtype, int64_t k_off, int64_t v_off, int32_t Hq, int32_t D);
 int sparse_attn_tc_chunk();
 lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, int64_t k_off,
-                                 const int32_t *rows, int32_t B, int32_t k, float scale, float *part_o,
+                                 const int32_t *rows, int32_t B, int32_t k, float scale, void *part_o,
                                  float *part_ml, int32_t *err, cudaStream_t st);
 size_t sparse_attn_workspace(int32_t B, int32_t Hq, int32_t D, int32_t k);
 
