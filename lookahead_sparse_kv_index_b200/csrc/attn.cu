@@ -145,122 +145,143 @@ attn_partial(const T *__restrict__ Q, const T *__restrict__ kv, int64_t stride, 
     }
 }
 
+// Raw partial values, converted where they are used (bf16 partials stay packed: two registers per
+// chunk in flight instead of four).
+template <typename TP>
+struct Raw4;
+template <>
+struct Raw4<float> {
+    using type = float4;
+    __device__ static type load(const float *p, int64_t i) { return *reinterpret_cast<const float4 *>(p + i); }
+    __device__ static float4 f(const type &v) { return v; }
+    __device__ static type zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+};
+template <>
+struct Raw4<uint16_t> {
+    using type = uint2;
+    __device__ static type load(const uint16_t *p, int64_t i) { return *reinterpret_cast<const uint2 *>(p + i); }
+    __device__ static float4 f(const type &w) {
+        return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u), __uint_as_float(w.y << 16),
+                           __uint_as_float(w.y & 0xFFFF0000u));
+    }
+    __device__ static type zero() { return make_uint2(0u, 0u); }
+};
+
+template <typename T>
+__device__ __forceinline__ void put4(T *out, int64_t i, float4 a, float inv) {
+    Elem<T>::put(out, i, a.x * inv);
+    Elem<T>::put(out, i + 1, a.y * inv);
+    Elem<T>::put(out, i + 2, a.z * inv);
+    Elem<T>::put(out, i + 3, a.w * inv);
+}
+
 // Merge of the chunk partials of one (head, sequence):
 //   M = max_c m_c,  w_c = e^{m_c - M},  L = sum_c l_c w_c,  o = sum_c w_c o_c / L,
 //   lse = M + log L;  a chunk with m_c = -inf (no selected row) has weight 0 and
 // its o is never read into the sum.
 // The kernel is a chain of dependent L2 round trips unless the loads go out
-// together: with up to 16 chunks every thread issues the (m, l) of all chunks
-// and its four columns of every chunk at once, then reduces on its own (the
-// (m, l) are the same for the whole block, so no block synchronisation sits
-// between the loads and the arithmetic).  More chunks: the same in batches.
-// four consecutive partial values as fp32 (partials in fp32 or bf16)
-__device__ __forceinline__ float4 load4(const float *p, int64_t i) { return *reinterpret_cast<const float4 *>(p + i); }
-__device__ __forceinline__ float4 load4(const uint16_t *p, int64_t i) {
-    const uint2 w = *reinterpret_cast<const uint2 *>(p + i);
-    return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u), __uint_as_float(w.y << 16),
-                       __uint_as_float(w.y & 0xFFFF0000u));
+// together.  Up to 16 chunks: every thread issues its four columns of every
+// chunk at once; the (m, l) of the chunks, the same for the whole block, go
+// through shared memory meanwhile.
+template <typename T, typename TP>
+__global__ void __launch_bounds__(128, 4)   // 4 CTAs per SM: the whole grid (Hq x B) resident at once
+attn_combine16(const TP *__restrict__ part_o, const float *__restrict__ part_ml, int nchunks, int Hq, int D,
+               T *__restrict__ out, float *__restrict__ lse) {
+    constexpr int kMax = 16;
+    using PR = Raw4<TP>;
+    __shared__ float2 s_ml[kMax];
+    pdl_wait();   // partials come from the preceding kernel
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int64_t p0 = int64_t(b) * nchunks * Hq + h;   // partial index of chunk 0; chunk c adds c * Hq
+    const int64_t ob = (int64_t(b) * Hq + h) * D;
+    if (threadIdx.x < kMax)
+        s_ml[threadIdx.x] = int(threadIdx.x) < nchunks
+                                ? reinterpret_cast<const float2 *>(part_ml)[p0 + int64_t(threadIdx.x) * Hq]
+                                : make_float2(-INFINITY, 0.f);
+    const int64_t cstride = int64_t(Hq) * D;
+    for (int col0 = 0; col0 < D; col0 += 4 * int(blockDim.x)) {   // uniform trip count: barrier inside
+        const int col = col0 + 4 * int(threadIdx.x);
+        const bool act = col < D;
+        typename PR::type v[kMax];
+        const TP *base = part_o + p0 * D + col;
+#pragma unroll
+        for (int u = 0; u < kMax; ++u) v[u] = (act && u < nchunks) ? PR::load(base, int64_t(u) * cstride) : PR::zero();
+        __syncthreads();
+        float M = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kMax; ++u) M = fmaxf(M, s_ml[u].x);
+        float L = 0.f;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < kMax; ++u) {
+            const float2 x = s_ml[u];
+            if (x.x == -INFINITY) continue;   // empty chunk (or u >= nchunks): its o is never read
+            const float w = expf(x.x - M);
+            L = fmaf(x.y, w, L);
+            const float4 o = PR::f(v[u]);
+            a.x = fmaf(w, o.x, a.x); a.y = fmaf(w, o.y, a.y);
+            a.z = fmaf(w, o.z, a.z); a.w = fmaf(w, o.w, a.w);
+        }
+        if (act) put4(out, ob + col, a, M == -INFINITY ? 0.f : 1.f / L);
+        if (col == 0 && lse) lse[int64_t(b) * Hq + h] = M == -INFINITY ? -INFINITY : M + logf(L);
+    }
 }
 
+// Any number of chunks: (m, l) in batches, then the columns in batches of 16 chunks.
 template <typename T, typename TP>
 __global__ void __launch_bounds__(128)
 attn_combine(const TP *__restrict__ part_o, const float *__restrict__ part_ml, int nchunks, int Hq, int D,
              T *__restrict__ out, float *__restrict__ lse) {
     constexpr int kBatch = 16;
+    using PR = Raw4<TP>;
     pdl_wait();   // partials come from the preceding kernel
     const int h = blockIdx.x, b = blockIdx.y;
-    const int64_t p0 = int64_t(b) * nchunks * Hq + h;   // partial index of chunk 0; chunk c adds c * Hq
+    const int64_t p0 = int64_t(b) * nchunks * Hq + h;
     const float2 *ml = reinterpret_cast<const float2 *>(part_ml);
     const int64_t ob = (int64_t(b) * Hq + h) * D;
-    const int col0 = 4 * threadIdx.x;
-    if (nchunks <= kBatch) {
-        float2 mlv[kBatch];
-        float4 v[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            mlv[u] = u < nchunks ? ml[p0 + int64_t(u) * Hq] : make_float2(-INFINITY, 0.f);
-            v[u] = (u < nchunks && col0 < D) ? load4(part_o, (p0 + int64_t(u) * Hq) * D + col0)
-                                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        float M = -INFINITY;
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) M = fmaxf(M, mlv[u].x);
-        float wgt[kBatch], L = 0.f;
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            wgt[u] = mlv[u].x == -INFINITY ? 0.f : expf(mlv[u].x - M);
-            L += mlv[u].y * wgt[u];
-        }
-        const float inv = M == -INFINITY ? 0.f : 1.f / L;
-        for (int col = col0; col < D; col += 4 * blockDim.x) {
-            if (col != col0) {
-#pragma unroll
-                for (int u = 0; u < kBatch; ++u)
-                    if (u < nchunks) v[u] = load4(part_o, (p0 + int64_t(u) * Hq) * D + col);
-            }
-            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                if (mlv[u].x == -INFINITY) continue;   // includes u >= nchunks
-                a.x = fmaf(wgt[u], v[u].x, a.x); a.y = fmaf(wgt[u], v[u].y, a.y);
-                a.z = fmaf(wgt[u], v[u].z, a.z); a.w = fmaf(wgt[u], v[u].w, a.w);
-            }
-            Elem<T>::put(out, ob + col, a.x * inv);
-            Elem<T>::put(out, ob + col + 1, a.y * inv);
-            Elem<T>::put(out, ob + col + 2, a.z * inv);
-            Elem<T>::put(out, ob + col + 3, a.w * inv);
-        }
-        if (threadIdx.x == 0 && lse) lse[int64_t(b) * Hq + h] = M == -INFINITY ? -INFINITY : M + logf(L);
-        return;
-    }
-    // more chunks than one batch: (m, l) in batches, then the columns in batches
     float M = -INFINITY;
-    for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
-        float2 mlv[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-            mlv[u] = c0 + u < nchunks ? ml[p0 + int64_t(c0 + u) * Hq] : make_float2(-INFINITY, 0.f);
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) M = fmaxf(M, mlv[u].x);
-    }
+    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, ml[p0 + int64_t(c) * Hq].x);
     float L = 0.f;
     if (M != -INFINITY)
-        for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
-            float2 mlv[kBatch];
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u)
-                mlv[u] = c0 + u < nchunks ? ml[p0 + int64_t(c0 + u) * Hq] : make_float2(-INFINITY, 0.f);
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u)
-                if (mlv[u].x != -INFINITY) L += mlv[u].y * expf(mlv[u].x - M);
+        for (int c = 0; c < nchunks; ++c) {
+            const float2 x = ml[p0 + int64_t(c) * Hq];
+            if (x.x != -INFINITY) L += x.y * expf(x.x - M);
         }
     const float inv = M == -INFINITY ? 0.f : 1.f / L;
-    for (int col = col0; col < D; col += 4 * blockDim.x) {
+    for (int col = 4 * int(threadIdx.x); col < D; col += 4 * blockDim.x) {
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
         if (M != -INFINITY)
             for (int c0 = 0; c0 < nchunks; c0 += kBatch) {
-                float4 v[kBatch];
-                float2 mlv[kBatch];
+                typename PR::type v[kBatch];
+                float mv[kBatch];
 #pragma unroll
                 for (int u = 0; u < kBatch; ++u) {
                     const int c = c0 + u;
-                    mlv[u] = c < nchunks ? ml[p0 + int64_t(c) * Hq] : make_float2(-INFINITY, 0.f);
-                    v[u] = c < nchunks ? load4(part_o, (p0 + int64_t(c) * Hq) * D + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    mv[u] = c < nchunks ? ml[p0 + int64_t(c) * Hq].x : -INFINITY;
+                    v[u] = c < nchunks ? PR::load(part_o, (p0 + int64_t(c) * Hq) * D + col) : PR::zero();
                 }
 #pragma unroll
                 for (int u = 0; u < kBatch; ++u) {
-                    if (mlv[u].x == -INFINITY) continue;   // an empty chunk's o is never read into the sum
-                    const float w = expf(mlv[u].x - M);
-                    a.x = fmaf(w, v[u].x, a.x); a.y = fmaf(w, v[u].y, a.y);
-                    a.z = fmaf(w, v[u].z, a.z); a.w = fmaf(w, v[u].w, a.w);
+                    if (mv[u] == -INFINITY) continue;   // an empty chunk's o is never read into the sum
+                    const float w = expf(mv[u] - M);
+                    const float4 o = PR::f(v[u]);
+                    a.x = fmaf(w, o.x, a.x); a.y = fmaf(w, o.y, a.y);
+                    a.z = fmaf(w, o.z, a.z); a.w = fmaf(w, o.w, a.w);
                 }
             }
-        Elem<T>::put(out, ob + col, a.x * inv);
-        Elem<T>::put(out, ob + col + 1, a.y * inv);
-        Elem<T>::put(out, ob + col + 2, a.z * inv);
-        Elem<T>::put(out, ob + col + 3, a.w * inv);
+        put4(out, ob + col, a, inv);
     }
     if (threadIdx.x == 0 && lse) lse[int64_t(b) * Hq + h] = M == -INFINITY ? -INFINITY : M + logf(L);
+}
+
+template <typename T, typename TP>
+lsa_status launch_combine(const TP *part_o, const float *part_ml, int nchunks, int B, int Hq, int D, void *out,
+                          float *lse, cudaStream_t st) {
+    auto kern = nchunks <= 16 ? attn_combine16<T, TP> : attn_combine<T, TP>;
+    LSA_CUDA(launch_pdl(kern, dim3(Hq, B), dim3(128), 0, st, part_o, part_ml, nchunks, Hq, D, static_cast<T *>(out),
+                        lse));
+    LSA_LAUNCHED("attn_combine");
+    return LSA_OK;
 }
 
 // Partial workspace: o [B, nchunks, Hq, D] fp32 (bf16 from the tensor-core chunks, which use the
@@ -285,9 +306,8 @@ lsa_status launch_t(const void *Q, const void *kv, int64_t stride, int64_t k_off
         pp = parts(workspace, B, Hq, D, nchunks);
         lsa_status s = launch_sparse_attn_tc(Q, kv, stride, k_off, rows, B, k, scale, pp.o, pp.ml, err, st);
         if (s != LSA_OK) return s;
-        LSA_CUDA(launch_pdl(attn_combine<T, uint16_t>, dim3(Hq, B), dim3(128), 0, st,
-                            reinterpret_cast<const uint16_t *>(pp.o), static_cast<const float *>(pp.ml), nchunks,
-                            Hq, D, static_cast<T *>(out), lse));
+        return launch_combine<T, uint16_t>(reinterpret_cast<const uint16_t *>(pp.o), pp.ml, nchunks, B, Hq, D, out,
+                                           lse, st);
     } else {
         nchunks = (k + kChunk - 1) / kChunk;
         pp = parts(workspace, B, Hq, D, nchunks);
@@ -301,11 +321,8 @@ lsa_status launch_t(const void *Q, const void *kv, int64_t stride, int64_t k_off
         kern<<<grid, kAttnThreads, smem, st>>>(static_cast<const T *>(Q), static_cast<const T *>(kv), stride,
                                                k_off, v_off, rows, Hq, D, k, scale, pp.o, pp.ml);
         LSA_LAUNCHED("attn_partial");
-        LSA_CUDA(launch_pdl(attn_combine<T, float>, dim3(Hq, B), dim3(128), 0, st, static_cast<const float *>(pp.o),
-                            static_cast<const float *>(pp.ml), nchunks, Hq, D, static_cast<T *>(out), lse));
+        return launch_combine<T, float>(pp.o, pp.ml, nchunks, B, Hq, D, out, lse, st);
     }
-    LSA_LAUNCHED("attn_combine");
-    return LSA_OK;
 }
 
 }  // namespace
