@@ -26,6 +26,7 @@ __device__ __forceinline__ uint32_t order_key(float z) {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kStageKeys = 40960;   // keys staged in shared memory (160 KB)
+constexpr int kMaxK = 4096;          // the largest k (the entry points check it); positions of the chosen in smem
 constexpr int kDigit = 11;
 constexpr int kBins = 1 << kDigit;   // 2048: two bins per thread
 
@@ -52,8 +53,31 @@ __device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
     __syncthreads();
     const int res = (warp ? s_warp[warp - 1] : 0) + x - v;
     *total = s_warp[kWarps - 1];
+    return res;   // s_warp is rewritten only after the caller's next barrier
+}
+
+// Exclusive block-wide prefix sum of a 64-bit value (two counters packed as hi:lo 32-bit halves).
+__device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t *s_warp64) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint64_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp64[warp] = x;
     __syncthreads();
-    return res;
+    if (warp == 0) {
+        uint64_t t = s_warp64[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint64_t y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        s_warp64[lane] = t;
+    }
+    __syncthreads();
+    return (warp ? s_warp64[warp - 1] : 0) + x - v;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -61,9 +85,11 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
             const int32_t *__restrict__ kept_idx, const int64_t *__restrict__ kept_off, int64_t kept_cap, int k,
             const int32_t *__restrict__ pos_map, int32_t *__restrict__ topk_idx, int32_t *__restrict__ topk_pos,
             int32_t *__restrict__ topk_cnt) {
-    extern __shared__ uint32_t s_keys[];   // [kStageKeys]
+    extern __shared__ uint32_t s_keys[];   // [kStageKeys] keys, then [kMaxK] positions of the chosen
+    int *s_pos = reinterpret_cast<int *>(s_keys + kStageKeys);
     __shared__ int s_hist[kBins];
     __shared__ int s_warp[kWarps];
+    __shared__ uint64_t s_warp64[kWarps];
     __shared__ uint32_t s_red[2][kWarps];
     __shared__ uint32_t s_want;
     __shared__ int s_kr, s_done;
@@ -135,13 +161,13 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
     uint32_t hmask = top >= 31 ? 0u : (top >= 0 ? ~((2u << top) - 1u) : 0xFFFFFFFFu);
     uint32_t want = gmin & hmask;
     int kr = k;
+    s_hist[threadIdx.x] = 0;   // each pass's reader zeroes its bins for the next pass
+    s_hist[threadIdx.x + kThreads] = 0;
+    __syncthreads();
     while (top >= 0) {
         const int width = top + 1 < kDigit ? top + 1 : kDigit;
         const int shift = top + 1 - width;
         const uint32_t dmask = (1u << width) - 1u;
-        s_hist[threadIdx.x] = 0;
-        s_hist[threadIdx.x + kThreads] = 0;
-        __syncthreads();
         for (int i = lo; i < hi; ++i) {
             const uint32_t u = key(i);
             if ((u & hmask) == want) atomicAdd(&s_hist[(u >> shift) & dmask], 1);
@@ -150,6 +176,8 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
         {   // thread t owns bins 2047 - 2t and 2046 - 2t (descending key order); suffix counts by a block scan
             const int bh = kBins - 1 - 2 * int(threadIdx.x);
             const int h0 = s_hist[bh], h1 = s_hist[bh - 1];
+            s_hist[bh] = 0;   // only this thread reads these two bins
+            s_hist[bh - 1] = 0;
             int tot;
             int above = block_excl_scan(h0 + h1, s_warp, &tot);   // entries in bins above bh
             if (above < kr && above + h0 >= kr) {
@@ -169,34 +197,35 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
         top = shift - 1;
         if (s_done) break;   // uniform: read after the barrier, rewritten only after the next barrier
     }
-    // ordered take: keys whose resolved bits exceed `want`, then the first kr equal to it
-    int n_eq = 0;
-    for (int i = lo; i < hi; ++i) n_eq += (key(i) & hmask) == want;
-    int tot;
-    const int eq_rank = block_excl_scan(n_eq, s_warp, &tot);
-    int n_take = 0;
-    {
-        int r = eq_rank;
-        for (int i = lo; i < hi; ++i) {
-            const uint32_t u = key(i) & hmask;
-            if (u > want) ++n_take;
-            else if (u == want) { n_take += r < kr; ++r; }
-        }
+    // ordered take: keys whose resolved bits exceed `want`, then the first kr equal to it (in kept-list
+    // order).  One scan of the packed counts (equal : above) gives both this thread's rank among the
+    // equal keys and the number of keys above before it.
+    int n_eq = 0, n_above = 0;
+    for (int i = lo; i < hi; ++i) {
+        const uint32_t u = key(i) & hmask;
+        n_eq += u == want;
+        n_above += u > want;
     }
-    int out = block_excl_scan(n_take, s_warp, &tot);
+    const uint64_t pre = block_excl_scan64((uint64_t(n_eq) << 32) | uint32_t(n_above), s_warp64);
+    const int eq_rank = int(pre >> 32);
+    int out = int(uint32_t(pre)) + min(eq_rank, kr);
+    // the take records the position of each output slot; the entry indices are then fetched with
+    // independent loads, two slots per thread (a dependent load per taken key serialised the tail)
     int r = eq_rank;
     for (int i = lo; i < hi; ++i) {
         const uint32_t u = key(i) & hmask;
         bool t = u > want;
         if (u == want) { t = r < kr; ++r; }
         if (t) {
-            if (out < k) {
-                const int64_t p = p0 + i;
-                out_idx[out] = kept_idx[p];
-                if (out_pos) out_pos[out] = pos_map ? pos_map[p] : int32_t(p);
-            }
+            if (out < k) s_pos[out] = i;
             ++out;
         }
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < k; j += kThreads) {
+        const int64_t p = p0 + s_pos[j];
+        out_idx[j] = kept_idx[p];
+        if (out_pos) out_pos[j] = pos_map ? pos_map[p] : int32_t(p);
     }
     if (threadIdx.x == 0) topk_cnt[b] = k;
 }
@@ -207,7 +236,7 @@ lsa_status launch_topk(const float *z, int32_t z_by_entry, const int64_t *seq_of
                        const int32_t *kept_idx, const int64_t *kept_off, int32_t B, int32_t k,
                        int64_t kept_cap, const int32_t *pos_map, int32_t *topk_idx, int32_t *topk_pos,
                        int32_t *topk_cnt, cudaStream_t st) {
-    const size_t smem = size_t(kStageKeys) * 4;
+    const size_t smem = size_t(kStageKeys) * 4 + size_t(kMaxK) * 4;
     LSA_CUDA(ensure_smem(topk_select, smem));
     LSA_CUDA(launch_pdl(topk_select, dim3(B), dim3(kThreads), smem, st, z, z_by_entry, seq_off, kept_idx, kept_off,
                         kept_cap, k, pos_map, topk_idx, topk_pos, topk_cnt));
