@@ -223,44 +223,42 @@ __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, con
         }
         for (int j = wi * 32 + lane; j < H; j += nw * 32) wsm[j] = wb[j];
     } else {
-        // warp wi owns heads wi, wi + nw, ...; lane owns channels 4*lane .. 4*lane+3; 8 heads per batch
-        for (int j0 = wi; j0 < H; j0 += 8 * nw) {
-            uint2 raw[8];
-            float wr[8];   // gate weights, loaded with the query rows (not one round trip per head)
+        // eight threads per head, thread g of a head owns channels 16g .. 16g+15 (one 16-byte chunk of
+        // each piece): the head's max is a 3-step shuffle and each thread converts 16 channels
+        const int tid = wi * 32 + lane, nthr = nw * 32;
+        const int g = tid & 7;
+        for (int j = tid >> 3; j < H; j += nthr >> 3) {   // every lane of a warp takes the same trip count
+            const uint4 *src = reinterpret_cast<const uint4 *>(qb + j * 128 + 16 * g);
+            const uint4 ra = src[0], rb = src[1];
+            const float wj = wb[j];
+            const uint32_t wds[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+            float v[16];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int j = j0 + u * nw;
-                if (j < H) {
-                    raw[u] = *reinterpret_cast<const uint2 *>(qb + j * 128 + 4 * lane);
-                    wr[u] = wb[j];
-                }
+            for (int c = 0; c < 8; ++c) {
+                v[2 * c] = __uint_as_float(wds[c] << 16);
+                v[2 * c + 1] = __uint_as_float(wds[c] & 0xFFFF0000u);
             }
+            float m = 0.f;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int j = j0 + u * nw;
-                if (j >= H) break;
-                const float v[4] = {__uint_as_float(raw[u].x << 16), __uint_as_float(raw[u].x & 0xFFFF0000u),
-                                    __uint_as_float(raw[u].y << 16), __uint_as_float(raw[u].y & 0xFFFF0000u)};
-                float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+            for (int c = 0; c < 16; ++c) m = fmaxf(m, fabsf(v[c]));
 #pragma unroll
-                for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                const int e = m > 0.f ? 8 - frexp_exponent(m) : 0;   // m 2^e in [128, 256)
-                uint32_t w0 = 0, w1 = 0;
+            for (int o = 4; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            const int e = m > 0.f ? 8 - frexp_exponent(m) : 0;   // m 2^e in [128, 256)
+            uint32_t p1w[4] = {0u, 0u, 0u, 0u}, p2w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-                for (int c = 0; c < 4; c += 2) {   // two channels per conversion (.x -> low byte)
-                    const float2 sv = make_float2(scale_pow2(v[c], e), scale_pow2(v[c + 1], e));
-                    const __nv_fp8x2_storage_t p1 = __nv_cvt_float2_to_fp8x2(sv, __NV_SATFINITE, __NV_E4M3);
-                    const float2 h1 = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(p1, __NV_E4M3)));
-                    const __nv_fp8x2_storage_t p2 =
-                        __nv_cvt_float2_to_fp8x2(make_float2(sv.x - h1.x, sv.y - h1.y), __NV_SATFINITE, __NV_E4M3);
-                    w0 |= uint32_t(p1) << (8 * c);
-                    w1 |= uint32_t(p2) << (8 * c);
-                }
-                const int off = j * 128 + (((lane >> 2) ^ (j & 7)) << 4) + (lane & 3) * 4;
-                *reinterpret_cast<uint32_t *>(slot + off) = w0;
-                *reinterpret_cast<uint32_t *>(slot + H * 128 + off) = w1;
-                if (lane == 0) wsm[j] = ldexpf(wr[u], -e);
+            for (int c = 0; c < 16; c += 2) {   // two channels per conversion (.x -> low byte)
+                const float2 sv = make_float2(scale_pow2(v[c], e), scale_pow2(v[c + 1], e));
+                const __nv_fp8x2_storage_t p1 = __nv_cvt_float2_to_fp8x2(sv, __NV_SATFINITE, __NV_E4M3);
+                const float2 h1 = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(p1, __NV_E4M3)));
+                const __nv_fp8x2_storage_t p2 =
+                    __nv_cvt_float2_to_fp8x2(make_float2(sv.x - h1.x, sv.y - h1.y), __NV_SATFINITE, __NV_E4M3);
+                p1w[c >> 2] |= uint32_t(p1) << (8 * (c & 3));
+                p2w[c >> 2] |= uint32_t(p2) << (8 * (c & 3));
             }
+            const int off = j * 128 + ((g ^ (j & 7)) << 4);
+            *reinterpret_cast<uint4 *>(slot + off) = make_uint4(p1w[0], p1w[1], p1w[2], p1w[3]);
+            *reinterpret_cast<uint4 *>(slot + H * 128 + off) = make_uint4(p2w[0], p2w[1], p2w[2], p2w[3]);
+            if (g == 0) wsm[j] = ldexpf(wj, -e);
         }
     }
 }
