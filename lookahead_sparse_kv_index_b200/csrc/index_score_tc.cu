@@ -99,7 +99,6 @@ constexpr int kAccMax = 8;            // TMEM accumulator stages at most
 constexpr int kScaleSlotsMax = 16;    // row-scale ring slots at most (stages + accumulators)
 constexpr int kMaxB = 512;            // sequences per launch on this path
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
-constexpr int kGatherDepth = 3;       // listed mode: tiles of row gathers in flight per producer lane
 
 template <int KIND>
 __host__ __device__ constexpr int tile_rows() {
@@ -138,7 +137,7 @@ __host__ __device__ constexpr int qimg_bytes() {
     return Cfg<KIND>::kQBytesPerHead * H;
 }
 
-// cp.async of 16 bytes (zero-filled when src_bytes == 0) and its group controls.
+// cp.async of 16 bytes (zero-filled when src_bytes == 0).
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
@@ -151,11 +150,7 @@ __device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src, uint32
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // Query operand of one sequence, built by nw warps (the 8 epilogue warps at
@@ -486,36 +481,21 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 if (++st == S) { st = 0; ph ^= 1; }
             }
         } else {
-            // all 32 lanes gather: lane owns rows lane, lane + 32, ... of each tile
+            // all 32 lanes gather: lane owns rows lane, lane + 32, ... of each tile; a stage (and its row
+            // scales) is signalled by cp.async-tracked arrivals, one per lane
             pdl_wait();
             constexpr int RB = KIND == E4M3_D128 ? 128 : (KIND == BF16_D128 ? 256 : 128);   // row bytes
             constexpr int CPR = RB / 16;
             int b = 0, cur = -1, qn = 0, st = 0;
             uint32_t ph = 0;
             int64_t row0, row_end;
-            int pend[kGatherDepth + 1];
-            int npend = 0, head = 0;
-            // completes every gather still held back and signals its stage: done before any
-            // wait whose end may depend on the MMA consuming one of those stages
-            auto flush = [&]() {
-                if (npend == 0) return;
-                cp_async_wait_group<0>();
-                fence_proxy_async_smem();
-                while (npend > 0) {
-                    mbar_arrive(&full[pend[head]]);
-                    head = (head + 1) % (kGatherDepth + 1);
-                    --npend;
-                }
-            };
             for (int64_t t = t0; t < t1; ++t) {
                 tile_info<TR>(s_toff, s_seq, B, t, b, row0, row_end);
                 if (b != cur) {
-                    if (qn >= 2) flush();   // the slot's release needs the MMA to finish the older sequence
                     if (!next_query(b, qn)) break;
                     cur = b;
                     ++qn;
                 }
-                if (!__all_sync(0xffffffffu, stage_free_test(t - t0))) flush();
                 const bool ok = stage_free_wait(t - t0);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 const uint32_t stage_u32 = smem_u32(stages + st * C::kStageBytes);
@@ -533,20 +513,13 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                     if (kScales)
                         cp_async_4(smem_u32(s_scale + int((t - t0) % RS) * TR + r), k_scale + e, valid ? 4u : 0u);
                 }
+                // each lane's arrival fires when its copies so far have landed: the stage is signalled as
+                // soon as its own rows are in, while the next tile's gathers are already being issued
+                cp_async_arrive_noinc(&full[st]);
                 if (kScales) cp_async_arrive_noinc(&sfull[int((t - t0) % RS)]);
-                cp_async_commit();
-                pend[(head + npend) % (kGatherDepth + 1)] = st;
-                ++npend;
-                if (npend > kGatherDepth) {
-                    cp_async_wait_group<kGatherDepth>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(&full[pend[head]]);
-                    head = (head + 1) % (kGatherDepth + 1);
-                    --npend;
-                }
                 if (++st == S) { st = 0; ph ^= 1; }
             }
-            flush();
+            cp_async_wait_all();   // no copy into this CTA's shared memory outlives the loop
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
