@@ -364,8 +364,10 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         // an accumulator is released by the warps that read it: one warpgroup per 128-row sub-tile
         for (int s = 0; s < KACC; ++s) { mbar_init(&tdone[s], 1); mbar_init(&tempty[s], 4 * C::kSub); }
         mbar_init(drain, 1);
+        // full mode: one arrival (the bulk copy's expect_tx, or lane 0 after the copies landed); listed
+        // mode: one cp.async-tracked arrival per producer lane
         if (kScales)
-            for (int s = 0; s < RS; ++s) mbar_init(&sfull[s], 32);   // one cp.async arrival per producer lane
+            for (int s = 0; s < RS; ++s) mbar_init(&sfull[s], LISTED ? 32 : 1);
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) prefetch_tmap(&tmap);
@@ -401,11 +403,9 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             const int slot = int(j % RS);
             const int64_t nvalid = (row_end - row0) < TR ? (row_end - row0) : TR;
             if ((row0 & 3) == 0 && (nvalid & 3) == 0 && (reinterpret_cast<uintptr_t>(k_scale) & 15) == 0) {
-                if (lane == 0) {
+                if (lane == 0) {   // the barrier's only arrival (no per-lane arrivals next to the MMA's reads)
                     mbar_arrive_expect_tx(&sfull[slot], uint32_t(nvalid * 4));
                     bulk_load(s_scale + slot * TR, k_scale + row0, uint32_t(nvalid * 4), &sfull[slot]);
-                } else {
-                    mbar_arrive(&sfull[slot]);
                 }
                 return;
             }
@@ -416,7 +416,9 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 const bool valid = row0 + r < row_end;
                 cp_async_4(dst + r * 4, k_scale + (valid ? row0 + r : 0), valid ? 4u : 0u);
             }
-            cp_async_arrive_noinc(&sfull[slot]);
+            cp_async_wait_all();   // unaligned spans only: the copies land, then one arrival
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sfull[slot]);
         };
         // (ordinals 0 and 1 are built by the epilogue warps, idle at kernel start)
         auto next_query = [&](int b, int o) -> bool {
