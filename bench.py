@@ -60,8 +60,9 @@ def parse_args():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--hot-frac", type=float, default=0.2)
-    ap.add_argument("--only", choices=["scan"], default=None,
-                    help="run one stage alone (W + K launches), for profiling; prints its mean time")
+    ap.add_argument("--only", choices=["scan", "union"], default=None,
+                    help="run one stage alone (W + K launches), for profiling; prints its mean time. "
+                         "union: the OR-mode union of three indexer layers (three full scans, the union, select)")
     return ap.parse_args()
 
 
@@ -515,12 +516,63 @@ def run_only_scan(args):
     return 0 if err.item() == 0 else 1
 
 
+def run_only_union(args):
+    """Three indexer layers (independent queries, gates and keys) over the workload's entry axis: the
+    union kernel alone, and the refresh-side scoring of the three layers (three full scans, the union,
+    select).  The union kernel reads 3 x 4 B and writes 4 B per entry."""
+    import torch
+
+    import synth
+    from lookahead_sparse_kv_index_b200 import lsa
+
+    layers = [synth.WORKLOADS[args.config](seed=100 + l, with_cold=False) for l in range(3)]
+    devs = [synth.to_torch(wl, pin_cold=False) for wl in layers]
+    wl = layers[0]
+    n = wl.n_total
+    zs = [torch.empty(n, dtype=torch.float32, device="cuda") for _ in layers]
+    zu = torch.empty(n, dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cap = n
+    kept_idx = torch.empty(cap, dtype=torch.int32, device="cuda")
+    kept_off = torch.empty(wl.B + 1, dtype=torch.int64, device="cuda")
+    mask = torch.empty((n + 31) // 32, dtype=torch.int32, device="cuda")
+    ws = torch.empty(lsa.select_workspace_size(n), dtype=torch.uint8, device="cuda")
+
+    def scans():
+        for l, (lw, dv) in enumerate(zip(layers, devs)):
+            lsa.index_score(dv["q"], lw.q_dtype, dv["w"], dv["keys"], lw.key_dtype, dv["k_scale"], dv["seq_off"],
+                            n, lw.H, lw.d, zs[l], None, err=err)
+
+    def union():
+        lsa.index_union(zs, n, zu)
+
+    def refresh():
+        scans()
+        union()
+        lsa.select(zu, devs[0]["seq_off"], n, kept_idx, cap, kept_off, mask, ws, err)
+
+    union_ms = graph_launch_ms(lambda i: union(), max(args.steps, 3))
+    refresh_ms = graph_launch_ms(lambda i: refresh(), max(args.steps, 3))
+    torch.cuda.synchronize()
+    union_bytes = 16 * n
+    peak, peak_src = measured_peaks()
+    kept = int(kept_off[-1].item())
+    print(json.dumps({"only": "union", "config": args.config, "layers": 3, "entries": n,
+                      "union_ms": union_ms, "union_GBps": union_bytes / (union_ms / 1e3) / 1e9,
+                      "union_frac_of_peak": union_bytes / (union_ms / 1e3) / 1e9 / peak, "peak_source": peak_src,
+                      "three_layer_refresh_scoring_ms": refresh_ms, "union_kept": kept,
+                      "union_kept_fraction": kept / n, "err": int(err.item())}), flush=True)
+    return 0 if err.item() == 0 else 1
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.only == "scan":
         return run_only_scan(args)
+    if args.only == "union":
+        return run_only_union(args)
     return run_cuda(args)
 
 

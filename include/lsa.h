@@ -149,6 +149,26 @@ lsa_status lsa_select_noalloc(const float *z, const int64_t *seq_off, int64_t n_
                               int32_t *err, void *stream);
 
 /* ------------------------------------------------------------------------
+ * lsa_index_union -- OR-mode union of several indexer layers (section 2.4,
+ * "Optimal Configuration": independent Memory Indexers on three layers whose
+ * predictions are united at inference to decide what is fetched).  Layer l
+ * keeps entry s when z_l[s] >= 0 (I >= 0.5); the union keeps s when any layer
+ * does, i.e. when max_l z_l[s] >= 0.  Writes z_union[s] = max_l z_l[s] (exact;
+ * a NaN counts as "not kept" by its layer), so lsa_select on z_union gives the
+ * union's kept set, and z_union is the union's ranking score for lsa_topk.
+ *
+ * z_layers   HOST array of n_layers DEVICE pointers, each to n_total fp32
+ *            scores on one entry axis (the layers share seq_off)
+ * n_layers   1 .. 8
+ * n_total    entries (0: nothing is launched)
+ * z_union    device fp32 [n_total]; may alias one of the layers' arrays
+ * stream     cudaStream_t or NULL
+ * Errors: LSA_ERR_INVALID for a null pointer or n_layers outside [1, 8].
+ * ---------------------------------------------------------------------- */
+lsa_status lsa_index_union(const float *const *z_layers, int32_t n_layers, int64_t n_total, float *z_union,
+                           void *stream);
+
+/* ------------------------------------------------------------------------
  * lsa_topk -- fine-grained top-k inside the kept set (section 2.1, "Tiered
  * Selection").  Per sequence, the k kept entries with the largest z (the
  * sigmoid is monotone, so ranking by z ranks by I); equal z goes to the lower

@@ -36,7 +36,7 @@ EXPORTS = [
     "lsa_select", "lsa_topk", "lsa_gather", "lsa_sparse_attn_workspace_size", "lsa_sparse_attn",
     "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
     "lsa_ctx_set_graphs", "lsa_ctx_set_timing", "lsa_ctx_stage_times", "lsa_ctx_reset_counters",
-    "lsa_ctx_launches", "lsa_selftest_bounded_wait",
+    "lsa_ctx_launches", "lsa_selftest_bounded_wait", "lsa_index_union",
 ]
 
 
@@ -93,6 +93,7 @@ _sig("lsa_ctx_stage_times", i32, [P, ctypes.POINTER(ctypes.c_double), ctypes.POI
 _sig("lsa_ctx_reset_counters", i32, [P])
 _sig("lsa_ctx_launches", i64, [P])
 _sig("lsa_selftest_bounded_wait", i32, [i64, P, P, P])
+_sig("lsa_index_union", i32, [ctypes.POINTER(P), i32, i64, P, P])
 
 lib = _L
 
@@ -152,6 +153,12 @@ def select_noalloc(z, seq_off, n_total, kept_idx, capacity, kept_off, mask, err,
     B = seq_off.numel() - 1
     _check(_L.lsa_select_noalloc(_ptr(z), _ptr(seq_off), n_total, B, _ptr(kept_idx), capacity, _ptr(kept_off),
                                  _ptr(mask), _ptr(err), _stream(stream)), "lsa_select_noalloc")
+
+
+def index_union(z_layers, n_total, z_union, stream=None):
+    """OR-mode union of indexer layers: z_union = max over the layers' scores (see lsa.h)."""
+    arr = (P * len(z_layers))(*[_ptr(z) for z in z_layers])
+    _check(_L.lsa_index_union(arr, len(z_layers), n_total, _ptr(z_union), _stream(stream)), "lsa_index_union")
 
 
 def selftest_bounded_wait(limit_ns, err, waited_ns, stream=None):

@@ -64,6 +64,7 @@ def lib():
         L.orc_select.restype = i64
         L.orc_select.argtypes = [P, P, i32, P, P, P]
         L.orc_topk.argtypes = [P, P, P, i32, i32, P, P]
+        L.orc_index_union.argtypes = [P, i32, i64, P, P]
         L.orc_gather.argtypes = [P, i64, P, P, P, i32, P, P]
         L.orc_sparse_attn.argtypes = [P, i32, P, i32, i64, i64, i64, P, i32, i32, i32, i32, dbl, P, P]
         L.orc_num_threads.restype = i32
@@ -136,6 +137,18 @@ def select(z, seq_off):
     mask = np.empty(int(seq_off[-1]), np.uint8)
     n = lib().orc_select(_p(z), _p(seq_off), B, _p(kept_idx), _p(kept_off), _p(mask))
     return kept_idx[:n].copy(), kept_off, mask.astype(bool)
+
+
+def index_union(z_layers):
+    """OR-mode union of indexer layers: (keep, score); keep[s] = any layer has z >= 0, score = the largest
+    non-NaN z of the layers (NaN when every layer's is NaN)."""
+    zs = [_c(z, np.float64) for z in z_layers]
+    n = len(zs[0])
+    arr = (ctypes.c_void_p * len(zs))(*[z.ctypes.data for z in zs])
+    keep = np.empty(max(n, 1), np.uint8)
+    score = np.empty(max(n, 1), np.float64)
+    lib().orc_index_union(ctypes.cast(arr, ctypes.c_void_p), len(zs), n, _p(keep), _p(score))
+    return keep[:n].astype(bool), score[:n]
 
 
 def topk(zk, kept_idx, kept_off, k):

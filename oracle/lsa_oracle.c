@@ -205,6 +205,37 @@ int64_t orc_select(const double *z, const int64_t *seq_off, int B,
 }
 
 /* ------------------------------------------------------------------ */
+/* OR-mode union of indexer layers (section 2.4 "Optimal              */
+/* Configuration": independent Memory Indexers on three layers, whose */
+/* predictions are united at inference to decide what is fetched).    */
+/* Each layer l predicts "fetch s" exactly when z_l[s] >= 0; the union */
+/* fetches s when any layer does.  The union's ranking score is taken  */
+/* as the largest z of the layers (the pages give none): a NaN score   */
+/* is no prediction and no score.                                     */
+/* ------------------------------------------------------------------ */
+
+void orc_index_union(const double *const *z, int n_layers, int64_t n, uint8_t *keep, double *score)
+{
+    int64_t s;
+    for (s = 0; s < n; s++) {
+        int l, any = 0, have = 0;
+        double best = NAN;
+        for (l = 0; l < n_layers; l++) {
+            double v = z[l][s];
+            if (v >= 0.0)
+                any = 1;
+            if (v == v) {
+                if (!have || v > best)
+                    best = v;
+                have = 1;
+            }
+        }
+        keep[s] = (uint8_t)any;
+        score[s] = best;
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* Fine-grained top-k inside the kept subset (section 2.1 "Tiered      */
 /* Selection").  Ranking is by z (the sigmoid is monotone), larger    */
 /* first, equal z broken towards the lower entry index.  The chosen   */

@@ -83,6 +83,14 @@ def test_other_entry_points_reject_bad_arguments(lsa):
     assert L.lsa_selftest_bounded_wait(10, big, big, None) == 1              # limit below 1 us
     assert L.lsa_selftest_bounded_wait(1 << 40, big, big, None) == 1         # limit above 100 ms
     assert L.lsa_selftest_bounded_wait(1000000, None, big, None) == 1        # no error word
+    arr = (ctypes.c_void_p * 3)(big, big, big)
+    assert L.lsa_index_union(None, 3, 10, big, None) == 1                     # no layers
+    assert L.lsa_index_union(arr, 0, 10, big, None) == 1                      # n_layers < 1
+    assert L.lsa_index_union(arr, 9, 10, big, None) == 1                      # n_layers > 8
+    assert L.lsa_index_union(arr, 3, -1, big, None) == 1                      # n_total < 0
+    assert L.lsa_index_union(arr, 3, 10, None, None) == 1                     # no output
+    arr[1] = None
+    assert L.lsa_index_union(arr, 3, 10, big, None) == 1                      # a layer without scores
 
 
 def test_ctx_create_rejects_bad_params(lsa):

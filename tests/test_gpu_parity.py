@@ -187,6 +187,61 @@ def test_topk_respects_kept_capacity(lsa):
     assert (idx[1][:50] == np.arange(50)).all()
 
 
+# ------------------------------------------------------------ layer union
+
+def test_index_union_of_three_scanned_layers(lsa):
+    # three independent indexer layers (own q, w and keys) over one ragged entry axis
+    lengths = (1000, 4133, 257, 64)
+    wls = [synth.small_ragged(seed=30 + l, key_dtype="e4m3", lengths=lengths) for l in range(3)]
+    n = wls[0].n_total
+    seq_off = wls[0].seq_off
+    zs = []
+    for wl in wls:
+        z, _ = gpu_full_scores(wl, synth.to_torch(wl, pin_cold=False), lsa, want_I=False, tc=True)
+        zs.append(z.astype(np.float32))
+    zd = [torch.from_numpy(z).cuda() for z in zs]
+    zu = torch.full((n + 8,), 77.0, dtype=torch.float32, device="cuda")
+    lsa.index_union(zd, n, zu)
+    torch.cuda.synchronize()
+    keep_ref, score_ref = oracle.index_union([z.astype(np.float64) for z in zs])
+    got = zu[:n].cpu().numpy()
+    assert np.array_equal(got, score_ref.astype(np.float32))      # the maximum is exact
+    assert (zu[n:].cpu().numpy() == 77.0).all()
+    # the union's kept set: select on the union score equals the OR of the layers' predictions
+    kept, ko, mask, err = gpu_select(got, seq_off, lsa)
+    assert err == 0 and np.array_equal(mask, keep_ref)
+    # top-k of the union ranks by the union score (stage-exact against the oracle on the same fp32 values)
+    k = 256
+    kept_o, ko_o, _ = oracle.select(score_ref, seq_off)
+    assert np.array_equal(kept, kept_o) and np.array_equal(ko, ko_o)
+    b_of = np.repeat(np.arange(len(lengths)), np.diff(ko))
+    zk = got[seq_off[:-1][b_of] + kept].astype(np.float64)
+    ref_idx, ref_cnt = oracle.topk(zk, kept, ko, k)
+    idx, pos, cnt = _topk_gpu(lsa, got, 1, seq_off, kept, ko, k)
+    assert np.array_equal(cnt, ref_cnt) and np.array_equal(idx, ref_idx)
+
+
+@pytest.mark.parametrize("n,offset", [(1 << 20, 0), (1000003, 0), (4096, 1)], ids=["vec4", "ragged_n", "unaligned"])
+def test_index_union_random_with_nans(lsa, n, offset):
+    rng = np.random.default_rng(n)
+    zs = []
+    for l in range(3):
+        z = rng.normal(size=n + offset).astype(np.float32)
+        z[rng.random(n + offset) < 0.01] = np.nan
+        z[rng.random(n + offset) < 0.01] = -0.0
+        zs.append(z)
+    zd = [torch.from_numpy(z).cuda()[offset:] for z in zs]      # offset 1: 4-byte aligned only (scalar path)
+    zu = torch.empty(n, dtype=torch.float32, device="cuda")
+    lsa.index_union(zd, n, zu)
+    torch.cuda.synchronize()
+    keep_ref, score_ref = oracle.index_union([z[offset:].astype(np.float64) for z in zs])
+    got = zu.cpu().numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(score_ref))
+    fin = ~np.isnan(score_ref)
+    assert np.array_equal(got[fin], score_ref[fin].astype(np.float32))
+    assert np.array_equal(got >= 0, keep_ref)
+
+
 # ---------------------------------------------------------------- gather
 
 def test_gather_bytes_and_slots(lsa):

@@ -149,6 +149,43 @@ def test_select_is_the_half_threshold_rule():
         assert ki.tolist() == local.tolist()
 
 
+# ------------------------------------------------------------- layer union
+
+def test_union_handworked():
+    # three layers x six entries, chosen by hand: the union fetches what any layer fetches (z >= 0,
+    # -0.0 included); a NaN is no prediction and no score
+    nan = float("nan")
+    z = [np.array([1.5, -1.0, nan, -0.0, -2.0, nan]),
+         np.array([-2.0, -3.0, nan, -5.0, -0.5, nan]),
+         np.array([-1.0, 2.25, -7.0, nan, -4.0, nan])]
+    keep, score = oracle.index_union(z)
+    assert keep.tolist() == [True, True, False, True, False, False]
+    assert score[:5].tolist() == [1.5, 2.25, -7.0, 0.0, -0.5] and np.signbit(score[3])
+    assert np.isnan(score[5])
+
+
+def test_union_is_the_or_of_the_layers_selections():
+    seq_off = np.array([0, 300, 300, 1000], np.int64)
+    layers = []
+    for l in range(3):
+        q, w, k, _ = _rand_case(20 + l, lens=(300, 0, 700))
+        z, _ = oracle.index_score(q, "f32", w, k, "f32", None, seq_off, 5, 7)
+        layers.append(z)
+    keep, score = oracle.index_union(layers)
+    masks = [oracle.select(z, seq_off)[2] for z in layers]
+    assert np.array_equal(keep, masks[0] | masks[1] | masks[2])
+    assert np.array_equal(keep, score >= 0)                       # the score decides the same set
+    stacked = np.stack(layers)
+    assert np.all((stacked == score).any(axis=0))                 # the score is one of the layers' scores
+    assert np.all(stacked <= score)
+    # one layer: the union is that layer
+    keep1, score1 = oracle.index_union([layers[1]])
+    assert np.array_equal(keep1, masks[1]) and np.array_equal(score1, layers[1])
+    # the union's kept set is what select keeps on the union score
+    kept_idx, kept_off, mask = oracle.select(score, seq_off)
+    assert np.array_equal(mask, keep)
+
+
 # ------------------------------------------------------------------- top-k
 
 def _brute_topk(zk, idx, k):
