@@ -65,6 +65,7 @@ def lib():
         L.orc_select.argtypes = [P, P, i32, P, P, P]
         L.orc_topk.argtypes = [P, P, P, i32, i32, P, P]
         L.orc_index_union.argtypes = [P, i32, i64, P, P]
+        L.orc_query_encode.argtypes = [P, i32, i32, i32, P, P, P, i32, i32, i32, i32, P, P, P]
         L.orc_gather.argtypes = [P, i64, P, P, P, i32, P, P]
         L.orc_sparse_attn.argtypes = [P, i32, P, i32, i64, i64, i64, P, i32, i32, i32, i32, dbl, P, P]
         L.orc_num_threads.restype = i32
@@ -149,6 +150,23 @@ def index_union(z_layers):
     score = np.empty(max(n, 1), np.float64)
     lib().orc_index_union(ctypes.cast(arr, ctypes.c_void_p), len(zs), n, _p(keep), _p(score))
     return keep[:n].astype(bool), score[:n]
+
+
+def query_encode(h, h_dtype, W_dq, W_uq, W_w, w_dtype, H, d):
+    """Indexer query encoder: (c, q, w) with c = W_dq h [B,rank], q = W_uq c viewed as [B,H,d] and
+    w = W_w h [B,H], all fp64.  h: raw [B,hidden]; W_dq raw [rank,hidden]; W_uq raw [H*d,rank];
+    W_w raw [H,hidden]."""
+    h = np.ascontiguousarray(h)
+    W_dq, W_uq, W_w = (np.ascontiguousarray(a) for a in (W_dq, W_uq, W_w))
+    B, hidden = h.shape
+    rank = W_dq.shape[0]
+    assert W_dq.shape == (rank, hidden) and W_uq.shape == (H * d, rank) and W_w.shape == (H, hidden)
+    c = np.empty((B, rank), np.float64)
+    q = np.empty((B, H, d), np.float64)
+    w = np.empty((B, H), np.float64)
+    lib().orc_query_encode(_p(h), _NP_CODE[h_dtype], B, hidden, _p(W_dq), _p(W_uq), _p(W_w), _NP_CODE[w_dtype],
+                           rank, H, d, _p(c), _p(q), _p(w))
+    return c, q, w
 
 
 def topk(zk, kept_idx, kept_off, k):

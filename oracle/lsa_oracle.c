@@ -236,6 +236,49 @@ void orc_index_union(const double *const *z, int n_layers, int64_t n, uint8_t *k
 }
 
 /* ------------------------------------------------------------------ */
+/* Indexer query encoder (section 2.1 "Memory Indexer": the current    */
+/* query token's hidden state h_t is mapped to low-rank indexer        */
+/* queries; section 2.3 "Query Optimization": what the encoder trains  */
+/* are its low-rank projection matrices).  Read as a rank-r            */
+/* factorisation with the head weights taken from h_t directly:        */
+/*   c   = W_dq h            (W_dq [rank, hidden])                     */
+/*   q_j = (W_uq c)[j*d .. j*d+d-1]   (W_uq [H*d, rank])               */
+/*   w   = W_w h             (W_w [H, hidden])                         */
+/* with no norm, activation or positional term (the pages name none).  */
+/* Matrices are row-major [out, in]; every product and sum in fp64.    */
+/* ------------------------------------------------------------------ */
+
+void orc_query_encode(const void *h, int h_dtype, int B, int hidden,
+                      const void *W_dq, const void *W_uq, const void *W_w, int w_dtype,
+                      int rank, int H, int d, double *c, double *q, double *w)
+{
+    int b;
+#pragma omp parallel for schedule(static)
+    for (b = 0; b < B; b++) {
+        const int64_t hb = (int64_t)b * hidden;
+        int i, n, j, k;
+        for (i = 0; i < rank; i++) {
+            double acc = 0.0;
+            for (k = 0; k < hidden; k++)
+                acc += load_elem(W_dq, w_dtype, (int64_t)i * hidden + k) * load_elem(h, h_dtype, hb + k);
+            c[(int64_t)b * rank + i] = acc;
+        }
+        for (n = 0; n < H * d; n++) {
+            double acc = 0.0;
+            for (i = 0; i < rank; i++)
+                acc += load_elem(W_uq, w_dtype, (int64_t)n * rank + i) * c[(int64_t)b * rank + i];
+            q[(int64_t)b * H * d + n] = acc;
+        }
+        for (j = 0; j < H; j++) {
+            double acc = 0.0;
+            for (k = 0; k < hidden; k++)
+                acc += load_elem(W_w, w_dtype, (int64_t)j * hidden + k) * load_elem(h, h_dtype, hb + k);
+            w[(int64_t)b * H + j] = acc;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* Fine-grained top-k inside the kept subset (section 2.1 "Tiered      */
 /* Selection").  Ranking is by z (the sigmoid is monotone), larger    */
 /* first, equal z broken towards the lower entry index.  The chosen   */

@@ -186,6 +186,55 @@ def test_union_is_the_or_of_the_layers_selections():
     assert np.array_equal(mask, keep)
 
 
+# ------------------------------------------------------------ query encoder
+
+def test_query_encode_handworked():
+    with open(os.path.join(GOLDEN, "query_encode_handworked.json")) as f:
+        g = json.load(f)
+    arr = {k: np.array(g[k], np.float32) for k in ("h", "W_dq", "W_uq", "W_w")}
+    c, q, w = oracle.query_encode(arr["h"], "f32", arr["W_dq"], arr["W_uq"], arr["W_w"], "f32", g["H"], g["d"])
+    assert np.array_equal(c, np.array(g["c"], np.float64))
+    assert np.array_equal(q, np.array(g["q"], np.float64))
+    assert np.array_equal(w, np.array(g["w"], np.float64))
+
+
+def test_query_encode_matches_numpy_matmul_on_bf16_operands():
+    """Random bf16 operands: the oracle's loops equal numpy's fp64 matrix products of the decoded operands
+    (every product of two bf16 values is exact in fp64, so only the summation order differs)."""
+    g = torch.Generator().manual_seed(5)
+    B, hidden, rank, H, d = 3, 40, 24, 4, 8
+    h = synth.bf16_bits(torch.randn(B, hidden, generator=g))
+    W_dq = synth.bf16_bits(torch.randn(rank, hidden, generator=g) / 6)
+    W_uq = synth.bf16_bits(torch.randn(H * d, rank, generator=g) / 5)
+    W_w = synth.bf16_bits(torch.randn(H, hidden, generator=g) / 6)
+    c, q, w = oracle.query_encode(h, "bf16", W_dq, W_uq, W_w, "bf16", H, d)
+    hd, Dq, Uq, Ww = (oracle.decode(a, "bf16") for a in (h, W_dq, W_uq, W_w))
+    np.testing.assert_allclose(c, hd @ Dq.T, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(q.reshape(B, H * d), (hd @ Dq.T) @ Uq.T, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(w, hd @ Ww.T, rtol=1e-13, atol=1e-13)
+    # head j of q is the j-th block of d rows of W_uq applied to c (no transposed head/channel order)
+    j = 2
+    np.testing.assert_allclose(q[:, j, :], c @ Uq[j * d:(j + 1) * d].T, rtol=1e-12, atol=1e-12)
+
+
+def test_query_encode_is_low_rank_in_h():
+    """The map h -> q factors through the rank-r latent: over the one-hot hidden states its image has rank
+    exactly r (generic weights), and q is linear in h."""
+    g = torch.Generator().manual_seed(6)
+    hidden, rank, H, d = 24, 5, 3, 4
+    W_dq = torch.randn(rank, hidden, generator=g).numpy().astype(np.float32)
+    W_uq = torch.randn(H * d, rank, generator=g).numpy().astype(np.float32)
+    W_w = torch.randn(H, hidden, generator=g).numpy().astype(np.float32)
+    eye = np.eye(hidden, dtype=np.float32)
+    _, q, w = oracle.query_encode(eye, "f32", W_dq, W_uq, W_w, "f32", H, d)
+    assert np.linalg.matrix_rank(q.reshape(hidden, H * d), tol=1e-9) == rank
+    np.testing.assert_allclose(w, W_w.T.astype(np.float64), rtol=0, atol=0)   # w of e_k is column k of W_w
+    h2 = torch.randn(2, hidden, generator=g).numpy().astype(np.float32)
+    _, q2, _ = oracle.query_encode(h2, "f32", W_dq, W_uq, W_w, "f32", H, d)
+    lin = np.tensordot(h2.astype(np.float64), q, axes=(1, 0))           # sum_k h_k q(e_k)
+    np.testing.assert_allclose(q2, lin, rtol=1e-10, atol=1e-10)
+
+
 # ------------------------------------------------------------------- top-k
 
 def _brute_topk(zk, idx, k):
