@@ -292,10 +292,17 @@ lsa_status lsa_ctx_destroy(lsa_ctx *ctx);
 lsa_status lsa_decode_step(lsa_ctx *ctx, int64_t t, const void *q, const float *w, const void *Q,
                            void *out, float *lse, void *stream);
 
-/* The same step on HOST buffers (page-locked for asynchronous copies): the
- * inputs are copied host->device, the step runs, out and lse are copied
- * device->host, all on `stream`.  The host buffers must stay valid until the
- * stream has completed. */
+/* The same step on HOST buffers (page-locked for asynchronous copies).
+ * The inputs are copied host->device on an internal copy stream into one of
+ * two device staging slots (alternating per call), so a call's input copies
+ * overlap the kernels of the call before it; the step's kernels run on
+ * `stream` after its inputs have landed, and out and lse are copied
+ * device->host before `stream` completes.  Ordering: the input copies are NOT
+ * ordered after earlier work on `stream` -- the input host buffers must hold
+ * the step's values when the call is made (host program order) and stay
+ * unchanged, like out_host and lse_host stay untouched, until `stream` has
+ * completed this call's work; out_host and lse_host hold the results once
+ * `stream` has completed. */
 lsa_status lsa_decode_step_host(lsa_ctx *ctx, int64_t t, const void *q_host, const float *w_host,
                                 const void *Q_host, void *out_host, float *lse_host, void *stream);
 

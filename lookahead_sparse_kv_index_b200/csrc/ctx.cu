@@ -71,9 +71,17 @@ struct lsa_ctx {
     size_t sel_ws_bytes = 0;
     void *attn_ws = nullptr;
     size_t attn_ws_bytes = 0;
-    // staging for lsa_decode_step_host
-    void *q_d = nullptr, *Q_d = nullptr, *out_d = nullptr;
-    float *w_d = nullptr, *lse_d = nullptr;
+    // staging for lsa_decode_step_host: two slots, so that the inputs of one
+    // step cross the host link while the previous step's kernels run
+    struct Staging {
+        void *q = nullptr, *Q = nullptr, *out = nullptr;
+        float *w = nullptr, *lse = nullptr;
+        cudaEvent_t in_ready = nullptr;   // the slot's inputs have landed (copy stream)
+        cudaEvent_t used = nullptr;       // the slot's step has run (caller's stream)
+        cudaEvent_t lse_done = nullptr;   // the slot's lse has reached the host
+    } stage[2];
+    int64_t host_calls = 0;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
     cudaStream_t side = nullptr;
     cudaEvent_t ev_sel = nullptr, ev_gather = nullptr;
     bool refreshed = false;
@@ -99,10 +107,17 @@ using namespace lsa;
 void free_all(lsa_ctx *c) {
     void *bufs[] = {c->seq_off_d, c->z, c->z_kept, c->kept_idx, c->kept_off, c->slot_of, c->hot,
                     c->topk_idx, c->topk_pos, c->topk_cnt, c->err, c->sel_ws, c->attn_ws,
-                    c->owner, c->kept_slot, c->fetched, c->fetch_ws,
-                    c->q_d, c->Q_d, c->out_d, c->w_d, c->lse_d};
+                    c->owner, c->kept_slot, c->fetched, c->fetch_ws};
     for (void *b : bufs)
         if (b) cudaFree(b);
+    for (auto &sg : c->stage) {
+        for (void *b : {sg.q, sg.Q, sg.out, static_cast<void *>(sg.w), static_cast<void *>(sg.lse)})
+            if (b) cudaFree(b);
+        for (cudaEvent_t e : {sg.in_ready, sg.used, sg.lse_done})
+            if (e) cudaEventDestroy(e);
+    }
+    if (c->h2d) cudaStreamDestroy(c->h2d);
+    if (c->d2h) cudaStreamDestroy(c->d2h);
     if (c->ev_sel) cudaEventDestroy(c->ev_sel);
     if (c->ev_gather) cudaEventDestroy(c->ev_gather);
     if (c->ev_assign) cudaEventDestroy(c->ev_assign);
@@ -330,11 +345,13 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     LSA_ALLOC(c->kept_slot, size_t(cap) * 4);
     LSA_ALLOC(c->fetched, 16);
     LSA_ALLOC(c->fetch_ws, fetch_workspace(cap));
-    LSA_ALLOC(c->q_d, qbytes);
-    LSA_ALLOC(c->w_d, size_t(p.B) * p.H * 4);
-    LSA_ALLOC(c->Q_d, Qbytes);
-    LSA_ALLOC(c->out_d, Qbytes);
-    LSA_ALLOC(c->lse_d, size_t(p.B) * p.Hq * 4);
+    for (auto &sg : c->stage) {
+        LSA_ALLOC(sg.q, qbytes);
+        LSA_ALLOC(sg.w, size_t(p.B) * p.H * 4);
+        LSA_ALLOC(sg.Q, Qbytes);
+        LSA_ALLOC(sg.out, Qbytes);
+        LSA_ALLOC(sg.lse, size_t(p.B) * p.Hq * 4);
+    }
 #undef LSA_ALLOC
     if (s == LSA_OK) {
         cudaError_t ce = cudaMemcpy(c->seq_off_d, so, size_t(p.B + 1) * 8, cudaMemcpyHostToDevice);
@@ -349,6 +366,11 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
         if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_sel, cudaEventDisableTiming);
         if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_gather, cudaEventDisableTiming);
         if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_assign, cudaEventDisableTiming);
+        if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->h2d, cudaStreamNonBlocking);
+        if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->d2h, cudaStreamNonBlocking);
+        for (auto &sg : c->stage)
+            for (cudaEvent_t *e : {&sg.in_ready, &sg.used, &sg.lse_done})
+                if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(e, cudaEventDisableTiming);
         if (ce != cudaSuccess) {
             set_error("lsa_ctx_create: %s", cudaGetErrorString(ce));
             s = LSA_ERR_CUDA;
@@ -390,14 +412,28 @@ lsa_status lsa_decode_step_host(lsa_ctx *c, int64_t t, const void *q_host, const
     cudaStream_t st = as_stream(stream);
     const size_t qbytes = size_t(p.B) * p.H * p.d * elem_size(p.q_dtype);
     const size_t Qbytes = size_t(p.B) * p.Hq * p.D * elem_size(p.attn_dtype);
-    LSA_CUDA(cudaMemcpyAsync(c->q_d, q_host, qbytes, cudaMemcpyHostToDevice, st));
-    LSA_CUDA(cudaMemcpyAsync(c->w_d, w_host, size_t(p.B) * p.H * 4, cudaMemcpyHostToDevice, st));
-    LSA_CUDA(cudaMemcpyAsync(c->Q_d, Q_host, Qbytes, cudaMemcpyHostToDevice, st));
-    lsa_status s = run_step(c, t, c->q_d, c->w_d, c->Q_d, c->out_d, c->lse_d, st);
+    auto &sg = c->stage[c->host_calls & 1];
+    // inputs on the copy stream, once the slot's previous step has read them;
+    // they overlap the kernels of the step enqueued before this one
+    LSA_CUDA(cudaStreamWaitEvent(c->h2d, sg.used, 0));
+    LSA_CUDA(cudaMemcpyAsync(sg.q, q_host, qbytes, cudaMemcpyHostToDevice, c->h2d));
+    LSA_CUDA(cudaMemcpyAsync(sg.w, w_host, size_t(p.B) * p.H * 4, cudaMemcpyHostToDevice, c->h2d));
+    LSA_CUDA(cudaMemcpyAsync(sg.Q, Q_host, Qbytes, cudaMemcpyHostToDevice, c->h2d));
+    LSA_CUDA(cudaEventRecord(sg.in_ready, c->h2d));
+    LSA_CUDA(cudaStreamWaitEvent(st, sg.in_ready, 0));
+    lsa_status s = run_step(c, t, sg.q, sg.w, sg.Q, sg.out, sg.lse, st);
     if (s != LSA_OK) return s;
-    LSA_CUDA(cudaMemcpyAsync(out_host, c->out_d, Qbytes, cudaMemcpyDeviceToHost, st));
-    if (lse_host)
-        LSA_CUDA(cudaMemcpyAsync(lse_host, c->lse_d, size_t(p.B) * p.Hq * 4, cudaMemcpyDeviceToHost, st));
+    LSA_CUDA(cudaEventRecord(sg.used, st));
+    ++c->host_calls;
+    // outputs: out on the caller's stream, lse beside it on the second copy
+    // stream; the caller's stream joins both before it completes
+    LSA_CUDA(cudaMemcpyAsync(out_host, sg.out, Qbytes, cudaMemcpyDeviceToHost, st));
+    if (lse_host) {
+        LSA_CUDA(cudaStreamWaitEvent(c->d2h, sg.used, 0));
+        LSA_CUDA(cudaMemcpyAsync(lse_host, sg.lse, size_t(p.B) * p.Hq * 4, cudaMemcpyDeviceToHost, c->d2h));
+        LSA_CUDA(cudaEventRecord(sg.lse_done, c->d2h));
+        LSA_CUDA(cudaStreamWaitEvent(st, sg.lse_done, 0));
+    }
     return LSA_OK;
 }
 

@@ -404,6 +404,39 @@ def test_decode_step_host_equals_device(lsa):
     ctx_b.close()
 
 
+def test_decode_step_host_pipelined_equals_device(lsa):
+    """Host steps issued back to back with no synchronisation in between (the input copies
+    of each call overlap the previous call's kernels through the two staging slots) give the
+    same bytes as device steps, for every step, across refreshes."""
+    wl = synth.small_ragged(key_dtype="e4m3")
+    from gpu_cases import make_context, read_ctx
+
+    dev = synth.to_torch(wl)
+    ctx_a = make_context(wl, dev, lsa, tau=4)
+    ctx_b = make_context(wl, dev, lsa, tau=4)
+    n = 11
+    ins = [wl.step_inputs(t) for t in range(n)]
+    host_in = [(synth.raw_to_torch(q, "cpu").pin_memory(), torch.from_numpy(np.ascontiguousarray(w)).pin_memory(),
+                synth.raw_to_torch(Q, "cpu").pin_memory()) for q, w, Q in ins]
+    outs_b = [torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.int16).pin_memory() for _ in range(n)]
+    lses_b = [torch.empty((wl.B, wl.Hq), dtype=torch.float32).pin_memory() for _ in range(n)]
+    torch.cuda.synchronize()
+    for t in range(n):
+        ctx_b.step_host(t, *host_in[t], outs_b[t], lses_b[t])
+    torch.cuda.synchronize()
+    out_a = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.int16, device="cuda")
+    lse_a = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device="cuda")
+    for t in range(n):
+        q_t, w_t, Q_t = ins[t]
+        ctx_a.step(t, synth.raw_to_torch(q_t), torch.from_numpy(w_t).cuda(), synth.raw_to_torch(Q_t), out_a, lse_a)
+        torch.cuda.synchronize()
+        assert torch.equal(out_a.cpu(), outs_b[t]), t
+        assert torch.equal(lse_a.cpu(), lses_b[t]), t
+    assert int(read_ctx(ctx_b, wl, lsa)["err"]) == 0
+    ctx_a.close()
+    ctx_b.close()
+
+
 def test_decode_graph_replay_equals_eager(lsa):
     """Steps replayed from captured CUDA graphs give the same bytes as eager steps, across
     refreshes, with the output buffers alternating (two graphs per step kind)."""
