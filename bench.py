@@ -60,8 +60,8 @@ def parse_args():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--hot-frac", type=float, default=0.2)
-    ap.add_argument("--only", choices=["scan", "union"], default=None,
-                    help="run one stage alone (W + K launches), for profiling; prints its mean time. "
+    ap.add_argument("--only", choices=["scan", "union", "encoder"], default=None,
+                    help="run one stage alone (W + K launches), for profiling; prints its mean time. encoder: the indexer query encoder h -> (q, w). "
                          "union: the OR-mode union of three indexer layers (three full scans, the union, select)")
     return ap.parse_args()
 
@@ -565,6 +565,51 @@ def run_only_union(args):
     return 0 if err.item() == 0 else 1
 
 
+def run_only_encoder(args):
+    """The indexer query encoder h -> (q, w) at the default shape (hidden 7168, rank 1536, the workload's
+    H and d) for the workload's batch: both passes, PDL-chained, timed as back-to-back launches in one
+    CUDA graph over 4 rotating weight replicas (4 x 48 MB > 126 MB L2, so the weights stream from HBM)."""
+    import torch
+
+    import synth
+    from lookahead_sparse_kv_index_b200 import lsa
+
+    wl = synth.WORKLOADS[args.config](with_cold=False)
+    B, H, d = wl.B, wl.H, wl.d
+    hidden, rank = synth.ENCODER_HIDDEN, synth.ENCODER_RANK
+    reps = 4
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda()
+
+    weights = []
+    for r in range(reps):
+        ew = synth.encoder_weights(200 + r, H, d, hidden=hidden, rank=rank)
+        weights.append((dev(ew.W_dq), dev(ew.W_uq), dev(ew.W_w)))
+    h = dev(synth.hidden_states(200, B, hidden=hidden))
+    q = torch.empty((B, H, d), dtype=torch.int16, device="cuda")
+    w = torch.empty((B, H), dtype=torch.float32, device="cuda")
+    c = torch.empty((B, rank), dtype=torch.float32, device="cuda")
+
+    def encode(i):
+        W_dq, W_uq, W_w = weights[i % reps]
+        lsa.query_encode(h, W_dq, W_uq, W_w, H, d, q, "bf16", w, c)
+
+    n = max(args.steps, 3) * reps
+    ms = graph_launch_ms(encode, n)
+    torch.cuda.synchronize()
+    weight_bytes = 2 * (rank * hidden + H * hidden + H * d * rank)
+    act_bytes = 2 * B * hidden + 2 * 4 * B * rank + 2 * B * H * d + 4 * B * H
+    total = weight_bytes + act_bytes
+    peak, peak_src = measured_peaks()
+    print(json.dumps({"only": "encoder", "config": args.config, "B": B, "hidden": hidden, "rank": rank, "H": H,
+                      "d": d, "launches_timed": n, "encode_ms": ms, "algorithmic_bytes": total,
+                      "GBps": total / (ms / 1e3) / 1e9, "frac_of_peak": total / (ms / 1e3) / 1e9 / peak,
+                      "peak_source": peak_src, "l2": "4 rotating weight replicas (%.0f MB each)" % (weight_bytes / 1e6)}),
+          flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -573,6 +618,8 @@ def main():
         return run_only_scan(args)
     if args.only == "union":
         return run_only_union(args)
+    if args.only == "encoder":
+        return run_only_encoder(args)
     return run_cuda(args)
 
 

@@ -169,6 +169,36 @@ lsa_status lsa_index_union(const float *const *z_layers, int32_t n_layers, int64
                            void *stream);
 
 /* ------------------------------------------------------------------------
+ * lsa_query_encode -- the indexer's query encoder (section 2.1 "Memory
+ * Indexer": the current query token's hidden state h_t is mapped to low-rank
+ * indexer queries; section 2.3 "Query Optimization": the encoder's trained
+ * part is its low-rank projection matrices).  Read as a rank-r factorisation
+ * with the head weights taken from h_t directly, and no norm, activation or
+ * positional term (the pages name none):
+ *     c = W_dq h,   q_j = rows j*d .. j*d+d-1 of W_uq c,   w = W_w h.
+ * Its outputs are lsa_index_score's q and w.
+ *
+ * h       device bf16 [B, hidden] hidden states
+ * W_dq    device bf16 [rank, hidden] down-projection, row-major [out, in]
+ * W_uq    device bf16 [H*d, rank] up-projection (rows of head j: j*d .. j*d+d-1)
+ * W_w     device bf16 [H, hidden] head-weight projection
+ * q_out   device [B, H, d] in q_dtype (BF16: rounded to nearest even from the
+ *         fp32 sum; F32)
+ * w_out   device fp32 [B, H]
+ * c_out   device fp32 [B, rank]: the latent, written by the first pass and
+ *         read by the second (the caller's buffer; nothing is allocated)
+ * Every sum is an fp32 accumulation of exact bf16 x bf16 (or bf16 x fp32)
+ * products; the summation order is fixed, so results are deterministic.
+ * Layout rules: hidden and rank multiples of 8 (>= 8); h, the three weight
+ * matrices and c_out 16-byte aligned.  Two kernel launches on `stream`.
+ * Errors: LSA_ERR_INVALID for a null pointer, a size or an alignment outside
+ * these rules; LSA_ERR_UNSUPPORTED for a q_dtype other than BF16 / F32.
+ * ---------------------------------------------------------------------- */
+lsa_status lsa_query_encode(const void *h, int32_t B, int32_t hidden, const void *W_dq, int32_t rank,
+                            const void *W_uq, int32_t H, int32_t d, const void *W_w, void *q_out,
+                            lsa_dtype q_dtype, float *w_out, float *c_out, void *stream);
+
+/* ------------------------------------------------------------------------
  * lsa_topk -- fine-grained top-k inside the kept set (section 2.1, "Tiered
  * Selection").  Per sequence, the k kept entries with the largest z (the
  * sigmoid is monotone, so ranking by z ranks by I); equal z goes to the lower

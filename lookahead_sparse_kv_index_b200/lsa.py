@@ -36,7 +36,7 @@ EXPORTS = [
     "lsa_select", "lsa_topk", "lsa_gather", "lsa_sparse_attn_workspace_size", "lsa_sparse_attn",
     "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
     "lsa_ctx_set_graphs", "lsa_ctx_set_timing", "lsa_ctx_stage_times", "lsa_ctx_reset_counters",
-    "lsa_ctx_launches", "lsa_selftest_bounded_wait", "lsa_index_union",
+    "lsa_ctx_launches", "lsa_selftest_bounded_wait", "lsa_index_union", "lsa_query_encode",
 ]
 
 
@@ -94,6 +94,7 @@ _sig("lsa_ctx_reset_counters", i32, [P])
 _sig("lsa_ctx_launches", i64, [P])
 _sig("lsa_selftest_bounded_wait", i32, [i64, P, P, P])
 _sig("lsa_index_union", i32, [ctypes.POINTER(P), i32, i64, P, P])
+_sig("lsa_query_encode", i32, [P, i32, i32, P, i32, P, i32, i32, P, P, i32, P, P, P])
 
 lib = _L
 
@@ -159,6 +160,15 @@ def index_union(z_layers, n_total, z_union, stream=None):
     """OR-mode union of indexer layers: z_union = max over the layers' scores (see lsa.h)."""
     arr = (P * len(z_layers))(*[_ptr(z) for z in z_layers])
     _check(_L.lsa_index_union(arr, len(z_layers), n_total, _ptr(z_union), _stream(stream)), "lsa_index_union")
+
+
+def query_encode(h, W_dq, W_uq, W_w, H, d, q_out, q_dtype, w_out, c_out, stream=None):
+    """Indexer query encoder: c = W_dq h, q = W_uq c as [B,H,d], w = W_w h (see lsa.h).  h: bf16 [B,hidden];
+    W_dq [rank,hidden], W_uq [H*d,rank], W_w [H,hidden] bf16 (any 2-byte tensors holding bf16 bits)."""
+    B, hidden = h.shape
+    rank = W_dq.shape[0]
+    _check(_L.lsa_query_encode(_ptr(h), B, hidden, _ptr(W_dq), rank, _ptr(W_uq), H, d, _ptr(W_w), _ptr(q_out),
+                               DTYPE[q_dtype], _ptr(w_out), _ptr(c_out), _stream(stream)), "lsa_query_encode")
 
 
 def selftest_bounded_wait(limit_ns, err, waited_ns, stream=None):

@@ -299,3 +299,40 @@ def raw_to_torch(a: np.ndarray, device: str = "cuda") -> torch.Tensor:
     if a.dtype == np.uint16:
         a = a.view(np.int16)
     return torch.from_numpy(a).to(device)
+
+
+# ------------------------------------------------------------ query encoder
+# Seeded stand-ins for the indexer's query encoder (trained weights are not
+# available): hidden states h ~ N(0, 1) and projection matrices with
+# variance-preserving scales, W_dq ~ N(0, 1/hidden), W_w ~ N(0, 1/hidden)/H,
+# W_uq ~ N(0, 1/rank)/sqrt(d) (so c ~ N(0, 1), q_j ~ N(0, I/d), |w_j| ~ 1/H,
+# the magnitudes of the planted-chunk recipe's queries and gates).  All bf16,
+# row-major [out, in].  Default sizes: hidden 7168, rank 1536.
+
+ENCODER_HIDDEN = 7168
+ENCODER_RANK = 1536
+
+
+@dataclass
+class EncoderWeights:
+    hidden: int
+    rank: int
+    H: int
+    d: int
+    W_dq: np.ndarray   # bf16 bits [rank, hidden]
+    W_uq: np.ndarray   # bf16 bits [H*d, rank]
+    W_w: np.ndarray    # bf16 bits [H, hidden]
+
+
+def encoder_weights(seed: int, H: int, d: int, hidden: int = ENCODER_HIDDEN, rank: int = ENCODER_RANK):
+    g = torch.Generator().manual_seed(seed * 7919 + 17)
+    W_dq = bf16_bits(torch.randn(rank, hidden, generator=g) / math.sqrt(hidden))
+    W_uq = bf16_bits(torch.randn(H * d, rank, generator=g) / math.sqrt(rank * d))
+    W_w = bf16_bits(torch.randn(H, hidden, generator=g) / (math.sqrt(hidden) * H))
+    return EncoderWeights(hidden, rank, H, d, W_dq, W_uq, W_w)
+
+
+def hidden_states(seed: int, B: int, hidden: int = ENCODER_HIDDEN, t: int = 0) -> np.ndarray:
+    """bf16 bits [B, hidden]: the decode-step-t hidden states of B sequences."""
+    g = torch.Generator().manual_seed(seed * 1000003 + 31 + t)
+    return bf16_bits(torch.randn(B, hidden, generator=g))
