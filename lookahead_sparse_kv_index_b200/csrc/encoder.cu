@@ -13,12 +13,16 @@
 //   pass 1: the rows of W_dq and W_w (stacked) against h  -> c, w (fp32)
 //   pass 2: the rows of W_uq against c                    -> q (bf16 / fp32)
 // A warp owns 4 weight rows and a strided set of 256-element chunks of their
-// K range; each lane loads 16 bytes of each row per chunk (coalesced 512-byte
-// row segments per warp, L1 bypassed) with the next chunk's loads issued
-// before the current chunk's FMAs.  The warps of a CTA split K when there are
-// too few row groups to fill the GPU; their partial sums are added in a fixed
-// order, so results are deterministic.  Batch rows beyond 4 are further
-// grid rows that read the same weights (mostly from L2).
+// K range; each lane streams 16 bytes of each row per chunk (coalesced
+// 512-byte row segments per warp) into its own slots of a 4-deep shared-memory
+// ring with cp.async, so four chunks per warp are in flight without holding
+// registers, and reads back only what it copied itself (no barriers).  The
+// warps of a CTA split K when there are too few row groups to fill the GPU;
+// their partial sums are added in a fixed order, so results are
+// deterministic.  The grid is sized to one wave.  Pass 1 also prefetches
+// W_uq into L2 (a bulk prefetch per CTA), so both passes' weights share one
+// HBM stream and pass 2 reads its weights from L2.  Batch rows beyond 4 are
+// further grid rows that read the same weights.
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -29,12 +33,21 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kRows = 4;      // weight rows per warp
 constexpr int kChunk = 256;   // K elements per warp chunk: 32 lanes x 8
 
-__device__ __forceinline__ uint4 ld_weights(const uint16_t *p) {
-    uint4 v;
-    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-        : "l"(p));
-    return v;
+// Chunks in flight per warp: three keep ~144 KB per SM in flight at three
+// CTAs per SM (measured: two to four stages time the same at batch 4).
+constexpr int kDepth = 3;
+constexpr int kStageU4 = kRows * 32;     // 16-byte slots of one warp stage (4 rows x 32 lanes)
+constexpr size_t kRingBytes = size_t(kWarps) * kDepth * kStageU4 * 16;   // 48 KB per CTA
+constexpr int kMinCtasPerSm = 3;
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *src) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
@@ -67,12 +80,14 @@ __device__ __forceinline__ void load_x8(const void *x, int64_t off, float *f) {
 
 // y[b, n] = sum_k W_n[k] x[b, k] for the stacked rows n < n0 (W0, into y0) and
 // n0 <= n < n0 + n1 (W1, into y1).  Warp w of a CTA takes row group
-// w / ks and K split w % ks; grid.y runs over groups of NB batch rows.
+// w / ks and K split w % ks; grid.y runs over groups of NB batch rows.  When
+// pf is set, blockIdx.y == 0 CTAs bulk-prefetch their share of pf_bytes
+// bytes at pf into L2.
 template <int NB, bool X_F32, bool OUT_BF16>
-__global__ void __launch_bounds__(kThreads) encode_rows(const uint16_t *__restrict__ W0, int n0,
-                                                        const uint16_t *__restrict__ W1, int n1, int K, int ks,
-                                                        const void *x, int B, void *y0, float *y1,
-                                                        int prefetch) {
+__global__ void __launch_bounds__(kThreads, kMinCtasPerSm)
+    encode_rows(const uint16_t *__restrict__ W0, int n0, const uint16_t *__restrict__ W1, int n1, int K, int ks,
+                const void *x, int B, void *y0, float *y1, const uint8_t *pf, int64_t pf_bytes) {
+    extern __shared__ uint4 ring[];
     __shared__ float red[kWarps][kRows * NB];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int groups_per_cta = kWarps / ks;
@@ -87,11 +102,32 @@ __global__ void __launch_bounds__(kThreads) encode_rows(const uint16_t *__restri
         const int n = min(row0 + r, nrows - 1);   // rows past the end re-read the last row; not written
         wrow[r] = n < n0 ? W0 + int64_t(n) * K : W1 + int64_t(n - n0) * K;
     }
+    uint4 *mine = ring + size_t(warp) * kDepth * kStageU4 + lane;   // this lane's slot, stage 0, row 0
+    const int nch = (K + kChunk - 1) / kChunk;
+    const int count = split < nch ? (nch - split + ks - 1) / ks : 0;   // chunks of this warp
+
+    // chunk i of this warp -> stage i % kDepth; one commit group per chunk (empty past the end)
+    auto issue = [&](int i) {
+        if (i < count) {
+            const int k0 = (split + i * ks) * kChunk + lane * 8;
+            if (k0 < K) {
+                uint4 *st = mine + (i % kDepth) * kStageU4;
+#pragma unroll
+                for (int r = 0; r < kRows; ++r) cp_async16(st + r * 32, wrow[r] + k0);
+            }
+        }
+        cp_async_commit();
+    };
+
     pdl_launch_dependents();
-    // the weights depend on no earlier kernel: start them towards L2 before waiting
-    if (prefetch && split == 0 && lane < kRows && row0 + lane < nrows) {
-        const int n = row0 + lane;
-        prefetch_l2(n < n0 ? W0 + int64_t(n) * K : W1 + int64_t(n - n0) * K, uint32_t(K) * 2u);
+    // the weights depend on no earlier kernel: start streaming them before waiting
+#pragma unroll
+    for (int i = 0; i < kDepth; ++i) issue(i);
+    if (pf && blockIdx.y == 0 && threadIdx.x == 0) {
+        const int64_t share = ((pf_bytes + gridDim.x - 1) / gridDim.x + 15) / 16 * 16;
+        const int64_t end = min(pf_bytes, int64_t(blockIdx.x + 1) * share);
+        for (int64_t o = int64_t(blockIdx.x) * share; o < end; o += 65536)
+            prefetch_l2(pf + o, uint32_t(min(int64_t(65536), end - o)));
     }
     pdl_wait();
 
@@ -105,34 +141,30 @@ __global__ void __launch_bounds__(kThreads) encode_rows(const uint16_t *__restri
 #pragma unroll
     for (int bb = 0; bb < NB; ++bb) xoff[bb] = int64_t(min(b0 + bb, B - 1)) * K;   // rows past B: not written
 
-    const int nch = (K + kChunk - 1) / kChunk;
-    uint4 cur[kRows], nxt[kRows];
-    auto load_chunk = [&](int ch, uint4 *dst) {
-        const int k0 = ch * kChunk + lane * 8;
+    for (int i = 0; i < count; ++i) {
+        const int k0 = (split + i * ks) * kChunk + lane * 8;
+        const bool live = k0 < K;
+        float xf[NB][8];
+        if (live) {
 #pragma unroll
-        for (int r = 0; r < kRows; ++r) dst[r] = k0 < K ? ld_weights(wrow[r] + k0) : make_uint4(0, 0, 0, 0);
-    };
-    if (split < nch) load_chunk(split, cur);
-    for (int ch = split; ch < nch; ch += ks) {
-        if (ch + ks < nch) load_chunk(ch + ks, nxt);
-        const int k0 = ch * kChunk + lane * 8;
-        if (k0 < K) {
-            float wf[kRows][8];
+            for (int bb = 0; bb < NB; ++bb) load_x8<X_F32>(x, xoff[bb] + k0, xf[bb]);
+        }
+        cp_async_wait<kDepth - 1>();   // chunk i's group has landed (groups complete in order)
+        if (live) {
+            const uint4 *st = mine + (i % kDepth) * kStageU4;
 #pragma unroll
-            for (int r = 0; r < kRows; ++r) widen8(cur[r], wf[r]);
+            for (int r = 0; r < kRows; ++r) {
+                float wf[8];
+                widen8(st[r * 32], wf);
 #pragma unroll
-            for (int bb = 0; bb < NB; ++bb) {
-                float xf[8];
-                load_x8<X_F32>(x, xoff[bb] + k0, xf);
+                for (int bb = 0; bb < NB; ++bb)
 #pragma unroll
-                for (int r = 0; r < kRows; ++r)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[r][bb] = fmaf(wf[r][e], xf[e], acc[r][bb]);
+                    for (int e = 0; e < 8; ++e) acc[r][bb] = fmaf(wf[e], xf[bb][e], acc[r][bb]);
             }
         }
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) cur[r] = nxt[r];
+        issue(i + kDepth);   // refills the stage just read (this lane's own slots)
     }
+    cp_async_wait<0>();
 
     // lanes -> warp total (butterfly: every lane ends with the sum), then the K splits in order
 #pragma unroll
@@ -165,34 +197,46 @@ __global__ void __launch_bounds__(kThreads) encode_rows(const uint16_t *__restri
     }
 }
 
-// K splits per row group: enough warps to keep HBM busy (16 per SM), at most
-// one split per chunk, at most the 8 warps of a CTA.
-int pick_splits(int nrows, int K) {
-    const int groups = (nrows + kRows - 1) / kRows;
+// K splits per row group: as many as fit the grid in one wave of resident
+// CTAs (more warps in flight), at most one split per chunk, at most the 8
+// warps of a CTA.
+int pick_splits(int nrows, int K, int batch_groups, int slots) {
+    const int64_t groups = (nrows + kRows - 1) / kRows;
     const int nch = (K + kChunk - 1) / kChunk;
-    const int64_t target = int64_t(sm_count()) * 16;
     int ks = 1;
-    while (ks < kWarps && int64_t(groups) * ks < target && ks * 2 <= nch) ks *= 2;
+    while (ks < kWarps && ks * 2 <= nch && (groups * ks * 2 + kWarps - 1) / kWarps * batch_groups <= slots) ks *= 2;
     return ks;
+}
+
+template <int NB, bool X_F32, bool OUT_BF16>
+cudaError_t launch_nb(const uint16_t *W0, int n0, const uint16_t *W1, int n1, int K, const void *x, int B,
+                      void *y0, float *y1, const void *pf, int64_t pf_bytes, cudaStream_t st) {
+    auto kern = encode_rows<NB, X_F32, OUT_BF16>;
+    cudaError_t e = ensure_smem(kern, kRingBytes);   // per device
+    if (e != cudaSuccess) return e;
+    static int per_sm = -1;   // resident CTAs per SM of this instance (one GPU model per process)
+    if (per_sm < 0) {
+        int n = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, kRingBytes);
+        if (e != cudaSuccess) return e;
+        per_sm = n < 1 ? 1 : n;
+    }
+    const int nrows = n0 + n1;
+    const int bgroups = (B + NB - 1) / NB;
+    const int ks = pick_splits(nrows, K, bgroups, per_sm * sm_count());
+    const int gpc = kWarps / ks;
+    const int groups = (nrows + kRows - 1) / kRows;
+    const dim3 grid((groups + gpc - 1) / gpc, bgroups);
+    return launch_pdl(kern, grid, dim3(kThreads), kRingBytes, st, W0, n0, W1, n1, K, ks, x, B, y0, y1,
+                      static_cast<const uint8_t *>(pf), pf_bytes);
 }
 
 template <bool X_F32, bool OUT_BF16>
 cudaError_t launch_pass(const uint16_t *W0, int n0, const uint16_t *W1, int n1, int K, const void *x, int B,
-                        void *y0, float *y1, int prefetch, cudaStream_t st) {
-    const int nrows = n0 + n1;
-    const int ks = pick_splits(nrows, K);
-    const int gpc = kWarps / ks;
-    const int groups = (nrows + kRows - 1) / kRows;
-    const int nb = B == 1 ? 1 : B == 2 ? 2 : 4;
-    const dim3 grid((groups + gpc - 1) / gpc, (B + nb - 1) / nb);
-    if (nb == 1)
-        return launch_pdl(encode_rows<1, X_F32, OUT_BF16>, grid, dim3(kThreads), 0, st, W0, n0, W1, n1, K, ks, x,
-                          B, y0, y1, prefetch);
-    if (nb == 2)
-        return launch_pdl(encode_rows<2, X_F32, OUT_BF16>, grid, dim3(kThreads), 0, st, W0, n0, W1, n1, K, ks, x,
-                          B, y0, y1, prefetch);
-    return launch_pdl(encode_rows<4, X_F32, OUT_BF16>, grid, dim3(kThreads), 0, st, W0, n0, W1, n1, K, ks, x, B,
-                      y0, y1, prefetch);
+                        void *y0, float *y1, const void *pf, int64_t pf_bytes, cudaStream_t st) {
+    if (B == 1) return launch_nb<1, X_F32, OUT_BF16>(W0, n0, W1, n1, K, x, B, y0, y1, pf, pf_bytes, st);
+    if (B == 2) return launch_nb<2, X_F32, OUT_BF16>(W0, n0, W1, n1, K, x, B, y0, y1, pf, pf_bytes, st);
+    return launch_nb<4, X_F32, OUT_BF16>(W0, n0, W1, n1, K, x, B, y0, y1, pf, pf_bytes, st);
 }
 
 }  // namespace
@@ -219,12 +263,13 @@ extern "C" lsa_status lsa_query_encode(const void *h, int32_t B, int32_t hidden,
     const auto *Wd = static_cast<const uint16_t *>(W_dq);
     const auto *Ww = static_cast<const uint16_t *>(W_w);
     const auto *Wu = static_cast<const uint16_t *>(W_uq);
-    LSA_CUDA((launch_pass<false, false>(Wd, rank, Ww, H, hidden, h, B, c_out, w_out, 0, st)));
+    const int64_t uq_bytes = int64_t(H) * d * rank * 2;
+    LSA_CUDA((launch_pass<false, false>(Wd, rank, Ww, H, hidden, h, B, c_out, w_out, Wu, uq_bytes, st)));
     LSA_LAUNCHED("encode_rows (W_dq | W_w)");
     if (q_dtype == LSA_BF16)
-        LSA_CUDA((launch_pass<true, true>(Wu, H * d, nullptr, 0, rank, c_out, B, q_out, nullptr, 1, st)));
+        LSA_CUDA((launch_pass<true, true>(Wu, H * d, nullptr, 0, rank, c_out, B, q_out, nullptr, nullptr, 0, st)));
     else
-        LSA_CUDA((launch_pass<true, false>(Wu, H * d, nullptr, 0, rank, c_out, B, q_out, nullptr, 1, st)));
+        LSA_CUDA((launch_pass<true, false>(Wu, H * d, nullptr, 0, rank, c_out, B, q_out, nullptr, nullptr, 0, st)));
     LSA_LAUNCHED("encode_rows (W_uq)");
     return LSA_OK;
 }
