@@ -214,6 +214,39 @@ def sparse_attn(Q, q_dtype, kv, kv_dtype, row_stride, k_off, v_off, sel_global, 
     return out, lse
 
 
+def attention_set(topk_idx, seq_off, window, hca_off=None):
+    """The rows one sequence attends when the always-resident context is merged into the core attention
+    (technical summary, section 2.1 "Architectural Design": all HCA chunks, 128:1 compressed, are retained
+    for global awareness; section 1 "Problem Statement": the most recent 8K tokens alone answer most long
+    requests).  Read as the
+    set union, per sequence b, of
+      * the top-k entries (topk_idx[b], local indices, -1 padded),
+      * the last `window` entries of the sequence (all of them when it is shorter), and
+      * every HCA row of the sequence (hca_off[b] .. hca_off[b+1]-1; none when hca_off is None),
+    each row counted once.  Rows are global indices into the concatenation [entries (n_total rows); HCA
+    rows], listed as: top-k entries outside the window (ascending), HCA rows (ascending), window entries
+    (ascending); -1 padded to a common width.  Returns (rows int64 [B, width], count int64 [B])."""
+    seq_off = np.asarray(seq_off, np.int64)
+    B = len(seq_off) - 1
+    n_total = int(seq_off[-1])
+    lists = []
+    for b in range(B):
+        n_b = int(seq_off[b + 1] - seq_off[b])
+        w_b = min(int(window), n_b)
+        win = set(range(n_b - w_b, n_b))
+        top = set(int(e) for e in np.asarray(topk_idx[b]) if e >= 0)
+        hca = [] if hca_off is None else list(range(int(hca_off[b]), int(hca_off[b + 1])))
+        rows = ([int(seq_off[b]) + e for e in sorted(top - win)] + [n_total + j for j in hca]
+                + [int(seq_off[b]) + e for e in sorted(win)])
+        assert len(rows) == len(set(rows))
+        lists.append(rows)
+    width = max(1, max(len(r) for r in lists))
+    out = np.full((B, width), -1, np.int64)
+    for b, r in enumerate(lists):
+        out[b, :len(r)] = r
+    return out, np.array([len(r) for r in lists], np.int64)
+
+
 def local_to_global(idx, seq_off):
     """Turn a [B,k] array of per-sequence entry indices (-1 padded) into global entry indices."""
     idx = np.asarray(idx, np.int64)

@@ -235,6 +235,70 @@ def test_query_encode_is_low_rank_in_h():
     np.testing.assert_allclose(q2, lin, rtol=1e-10, atol=1e-10)
 
 
+# ------------------------------------------- merged attention set (window + HCA)
+
+def test_attention_set_handworked():
+    """Two sequences of 10 and 4 entries, window 3, HCA rows 2 and 1.  Sequence 0: top-k {1, 5, 8}; 8 lies in
+    the window {7, 8, 9} and is counted once -> {1, 5} + HCA {0, 1} + {7, 8, 9}.  Sequence 1 (entries 10..13):
+    top-k {0, 2} (local) -> 2 lies in the window {1, 2, 3} -> {0} + HCA {2} + {1, 2, 3}.  HCA rows come after
+    the 14 entries in the concatenated row space (14, 15, 16)."""
+    seq_off = np.array([0, 10, 14])
+    topk = np.array([[1, 5, 8], [0, 2, -1]])
+    rows, cnt = oracle.attention_set(topk, seq_off, 3, hca_off=np.array([0, 2, 3]))
+    assert cnt.tolist() == [7, 5]
+    assert rows[0].tolist() == [1, 5, 14, 15, 7, 8, 9]
+    assert rows[1].tolist() == [10, 16, 11, 12, 13, -1, -1]
+    # no window, no HCA: the top-k set itself
+    rows0, cnt0 = oracle.attention_set(topk, seq_off, 0)
+    assert cnt0.tolist() == [3, 2] and rows0[1].tolist() == [10, 12, -1]
+    # a window longer than the sequence covers all of it
+    rows1, cnt1 = oracle.attention_set(topk, seq_off, 50)
+    assert cnt1.tolist() == [10, 4] and rows1[1].tolist() == [10, 11, 12, 13] + [-1] * 6
+
+
+def _lse_merge(parts):
+    """Softmax attention over a disjoint union from the parts' (out, lse): the log-sum-exp identity."""
+    lses = np.stack([p[1] for p in parts])
+    lse = np.logaddexp.reduce(lses, axis=0)
+    out = sum(np.exp(p[1] - lse)[..., None] * p[0] for p in parts)
+    return out, lse
+
+
+def test_merged_attention_is_softmax_over_the_union():
+    """Attention over the merged set equals the log-sum-exp combination of attention over its three disjoint
+    parts (top-k outside the window, HCA rows, window), and differs from attention that counts a top-k entry
+    inside the window twice."""
+    g = torch.Generator().manual_seed(17)
+    B, Hq, D, stride = 2, 4, 32, 32
+    seq_off = np.array([0, 300, 420])
+    n_total = 420
+    hca_off = np.array([0, 3, 5])
+    kv = torch.randn(n_total + 5, stride, generator=g).numpy().astype(np.float32)
+    Q = torch.randn(B, Hq, D, generator=g).numpy().astype(np.float32)
+    topk = np.array([[3, 40, 41, 290, 299, -1], [0, 7, 100, 110, 115, 119]])
+    window = 16
+    rows, cnt = oracle.attention_set(topk, seq_off, window, hca_off=hca_off)
+    scale = 0.2
+    out, lse = oracle.sparse_attn(Q, "f32", kv, "f32", stride, 0, 0, rows, scale)
+    parts = []
+    for sel in ("top", "hca", "win"):
+        part = np.full_like(rows, -1)
+        for b in range(B):
+            r = [x for x in rows[b, :cnt[b]]
+                 if (sel == "hca") == (x >= n_total) and
+                 (sel == "hca" or ((x - seq_off[b] >= seq_off[b + 1] - seq_off[b] - window) == (sel == "win")))]
+            part[b, :len(r)] = r
+        parts.append(oracle.sparse_attn(Q, "f32", kv, "f32", stride, 0, 0, part, scale))
+    m_out, m_lse = _lse_merge(parts)
+    np.testing.assert_allclose(out, m_out, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, m_lse, rtol=1e-12, atol=1e-12)
+    # counting entry 290 (in sequence 0's window) a second time changes the result
+    dup = np.concatenate([rows, np.full((B, 1), -1)], axis=1)
+    dup[0, cnt[0]] = 290
+    out_d, _ = oracle.sparse_attn(Q, "f32", kv, "f32", stride, 0, 0, dup, scale)
+    assert np.max(np.abs(out_d[0] - out[0])) > 1e-6
+
+
 # ------------------------------------------------------------------- top-k
 
 def _brute_topk(zk, idx, k):
