@@ -60,8 +60,8 @@ def parse_args():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--hot-frac", type=float, default=0.2)
-    ap.add_argument("--only", choices=["scan", "union", "encoder"], default=None,
-                    help="run one stage alone (W + K launches), for profiling; prints its mean time. encoder: the indexer query encoder h -> (q, w). "
+    ap.add_argument("--only", choices=["scan", "union", "encoder", "merged"], default=None,
+                    help="run one stage alone (W + K launches), for profiling; prints its mean time. encoder: the indexer query encoder h -> (q, w). merged: decode with the recent window and HCA rows merged into the attention set. "
                          "union: the OR-mode union of three indexer layers (three full scans, the union, select)")
     return ap.parse_args()
 
@@ -610,6 +610,84 @@ def run_only_encoder(args):
     return 0
 
 
+def run_only_merged(args):
+    """Decode windows with the always-resident context merged into the attention set: a recent window of
+    8K tokens (2048 entries) and the HCA rows (one per 128 tokens) per sequence, against the same decode
+    without them.  Same loop as the headline (tau-step windows, 3 context replicas over cloned keys, CUDA
+    graphs); reports decode steps/s of both and the merged step's eager stage times."""
+    import torch
+
+    import synth
+    from lookahead_sparse_kv_index_b200 import lsa
+
+    wl = synth.WORKLOADS[args.config]()
+    dev = synth.to_torch(wl)
+    hca, hca_off = synth.hca_rows(wl)
+    hca_t = torch.from_numpy(hca.view(np.int16)).cuda()
+    window_entries = synth.RECENT_TOKENS // synth.ENTRY_RATIO
+    cap = max(wl.topk, int(args.hot_frac * wl.n_total))
+    tau = wl.tau
+    steps_in = [wl.step_inputs(t) for t in range(tau)]
+    q_d = [synth.raw_to_torch(s[0]) for s in steps_in]
+    w_d = [torch.from_numpy(np.ascontiguousarray(s[1])).cuda() for s in steps_in]
+    Q_d = [synth.raw_to_torch(s[2]) for s in steps_in]
+    q_ref = [synth.raw_to_torch(wl.step_inputs(tau * (w + 1))[0]) for w in range(8)]
+    odt = torch.int16 if wl.attn_dtype == "bf16" else torch.float32
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=odt, device="cuda")
+    lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device="cuda")
+    keys = [dev["keys"]] + [dev["keys"].clone() for _ in range(REPLICAS - 1)]
+    res = {}
+    for mode in ("topk_only", "merged"):
+        extra = dict(window=window_entries, hca_rows=hca_t, hca_off_host=hca_off) if mode == "merged" else {}
+        ctxs = [lsa.Context(B=wl.B, H=wl.H, d=wl.d, q_dtype=wl.q_dtype, k_dtype=wl.key_dtype, Hq=wl.Hq, D=wl.D,
+                            attn_dtype=wl.attn_dtype, topk=wl.topk, seq_off_host=wl.seq_off, keys=keys[r],
+                            k_scale=dev["k_scale"], cold_host=dev["cold"], row_bytes=wl.row_bytes,
+                            kv_row_stride=wl.row_stride, k_off=wl.k_off, v_off=wl.v_off, kept_capacity=cap,
+                            tau=tau, scale=wl.scale, **extra) for r in range(REPLICAS)]
+        q0 = q_d[0].clone()
+        qs = [q0] + q_d[1:]
+        counter = [0]
+
+        def window(w):
+            q0.copy_(q_ref[counter[0] % len(q_ref)], non_blocking=True)
+            counter[0] += 1
+            for t in range(tau):
+                ctxs[w % REPLICAS].step(t, qs[t], w_d[t], Q_d[t], out, lse)
+
+        for w in range(2 * REPLICAS + args.warmup):
+            window(w)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for w in range(args.steps):
+            window(w)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        errs = [int(lsa.device_view(c.view().err, 1, torch.int32).item()) for c in ctxs]
+        entry = {"decode_steps_per_s": tau * args.steps / (ms / 1e3), "ms_per_window": ms / args.steps,
+                 "device_errors": errs}
+        if mode == "merged":
+            v = ctxs[0].view()
+            entry["attn_rows_per_sequence_cap"] = int(v.attn_row_cap)
+            entry["window_entries"] = window_entries
+            entry["hca_rows_per_sequence"] = np.diff(hca_off).tolist()
+            ctxs[0].reset_counters()
+            ctxs[0].set_timing(True)
+            window(0)
+            torch.cuda.synchronize()
+            st = ctxs[0].stage_times()
+            entry["stages_ms_avg_eager"] = {k: (v_[0] / v_[1] if v_[1] else None) for k, v_ in st.items()}
+            ctxs[0].set_timing(False)
+        res[mode] = entry
+        for c in ctxs:
+            c.close()
+        torch.cuda.synchronize()
+    print(json.dumps({"only": "merged", "config": args.config, "tau": tau, "windows_timed": args.steps, **res}),
+          flush=True)
+    return 0 if all(e == 0 for r in res.values() for e in r["device_errors"]) else 1
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -620,6 +698,8 @@ def main():
         return run_only_union(args)
     if args.only == "encoder":
         return run_only_encoder(args)
+    if args.only == "merged":
+        return run_only_merged(args)
     return run_cuda(args)
 
 

@@ -61,6 +61,9 @@ typedef enum lsa_dtype {
 } lsa_dtype;
 
 /* Library version, major*10000 + minor*100 + patch. */
+/* sizeof(lsa_params) for which = 0, sizeof(lsa_ctx_view) for 1, else -1: lets a
+ * binding that mirrors the structs check its layout.  Needs no GPU. */
+int64_t lsa_struct_size(int32_t which);
 int32_t lsa_version(void);
 
 /* Message of the last failing call on this host thread ("" if none). */
@@ -199,6 +202,34 @@ lsa_status lsa_query_encode(const void *h, int32_t B, int32_t hidden, const void
                             lsa_dtype q_dtype, float *w_out, float *c_out, void *stream);
 
 /* ------------------------------------------------------------------------
+ * lsa_attn_set_merge -- the merged attention set (section 2.1 "Architectural
+ * Design": every Heavily Compressed Attention chunk, 128:1, stays resident for
+ * global awareness; section 1 "Problem Statement": the most recent 8K tokens
+ * alone answer most long requests).  Per sequence b the core attention runs
+ * over the set union of its top-k entries, its last `window` entries and its
+ * HCA rows, each row once (a top-k entry inside the window is attended through
+ * the window's row).  Writes, per sequence, the row list for lsa_sparse_attn
+ * over one KV arena: the top-k slots of entries below the window (ascending
+ * entry order), then rows hca_base + hca_off[b] .. hca_base + hca_off[b+1]-1,
+ * then rows win_base + b*window + t for t < min(window, N_b) (row t holding
+ * entry N_b - min(window, N_b) + t), then -1 up to row_cap.
+ *
+ * topk_idx, topk_pos, topk_cnt   device, as written by lsa_topk ([B, k], [B, k], [B])
+ * seq_off    device int64 [B+1]
+ * hca_off    device int64 [B+1] offsets of each sequence's HCA rows, or NULL (none)
+ * rows       device int32 [B, row_cap]; count device int32 [B] (rows used) or NULL
+ * err        device error word or NULL: LSA_ERR_CAPACITY when a sequence needs more than
+ *            row_cap rows (its list is cut at row_cap)
+ * One launch (a CTA per sequence) on `stream`.  Row indices are int32: the
+ * caller keeps hca_base + hca_off[B] and win_base + B*window below 2^31.
+ * Errors: LSA_ERR_INVALID for a null pointer or a negative size.
+ * ---------------------------------------------------------------------- */
+lsa_status lsa_attn_set_merge(const int32_t *topk_idx, const int32_t *topk_pos, const int32_t *topk_cnt,
+                              const int64_t *seq_off, int32_t B, int32_t k, int32_t window, int32_t win_base,
+                              const int64_t *hca_off, int32_t hca_base, int32_t *rows, int32_t row_cap,
+                              int32_t *count, int32_t *err, void *stream);
+
+/* ------------------------------------------------------------------------
  * lsa_topk -- fine-grained top-k inside the kept set (section 2.1, "Tiered
  * Selection").  Per sequence, the k kept entries with the largest z (the
  * sigmoid is monotone, so ranking by z ranks by I); equal z goes to the lower
@@ -264,7 +295,7 @@ lsa_status lsa_gather(const void *cold_host, int64_t row_bytes, const int64_t *s
  *        (fp32 split-K partials); calls that share it must not overlap.
  * err    device error word or NULL (LSA_ERR_TIMEOUT if a bounded wait of the
  *        tensor-core kernel gave up).
- * Shapes run: D % 32 == 0, D <= 512, 1 <= Hq <= 256, 1 <= k <= 4096.  bf16
+ * Shapes run: D % 32 == 0, D <= 512, 1 <= Hq <= 256, 1 <= k <= 65536.  bf16
  * with Hq = 128, D = 512 and K aliasing V (a latent head) runs on the tensor
  * cores (tcgen05); every other shape on the CUDA cores.
  * ---------------------------------------------------------------------- */
@@ -307,6 +338,14 @@ typedef struct lsa_params {
     int32_t full_fetch;          /* 0: the hot buffer caches rows across refreshes and a refresh
                                     fetches only entries not resident; nonzero: every refresh
                                     fetches every kept row (lsa_gather) into kept order */
+    /* Always-resident context merged into the core attention (lsa_attn_set_merge):
+     * with window > 0 or hca_rows set, every step attends over the union of its
+     * top-k, the last `window` entries of its sequence and the sequence's HCA rows.
+     * The context copies both into HBM at creation (window rows from cold_host). */
+    int32_t window;              /* recent-window entries per sequence (0: none) */
+    const void *hca_rows;        /* HCA rows [hca_off_host[B], row_bytes], host or device memory, same
+                                    row format as the cold pool; NULL: none */
+    const int64_t *hca_off_host; /* HOST [B+1] offsets of each sequence's HCA rows (with hca_rows) */
 } lsa_params;
 
 typedef struct lsa_ctx lsa_ctx;
@@ -343,7 +382,8 @@ typedef struct lsa_ctx_view {
     int32_t *kept_idx;   /* [kept_capacity] */
     int64_t *kept_off;   /* [B+1] */
     int32_t *slot_of;    /* [n_total] hot slot of each entry, or -1 */
-    void *hot;           /* [kept_capacity, row_bytes] */
+    void *hot;           /* [kept_capacity + B * window + HCA rows, row_bytes]: the hot buffer,
+                            then the window rows, then the HCA rows */
     int32_t *topk_idx;   /* [B, topk] */
     int32_t *topk_pos;   /* [B, topk] hot slot of each chosen entry, -1 padded */
     int32_t *topk_cnt;   /* [B] */
@@ -351,6 +391,11 @@ typedef struct lsa_ctx_view {
     int32_t *kept_slot;  /* [kept_capacity] hot slot of each kept position (NULL with full_fetch) */
     int32_t *owner;      /* [kept_capacity] entry held by each hot slot, or -1 */
     int64_t *fetched;    /* rows fetched from the cold pool by the last refresh */
+    int32_t *attn_rows;  /* [B, attn_row_cap] merged attention rows into `hot` (NULL without
+                            window / HCA rows): see lsa_attn_set_merge */
+    int64_t attn_row_cap;
+    int64_t win_base;    /* arena row of sequence 0's first window row (sequence b: + b * window) */
+    int64_t hca_base;    /* arena row of the first HCA row */
 } lsa_ctx_view;
 lsa_status lsa_ctx_get_view(lsa_ctx *ctx, lsa_ctx_view *view);
 

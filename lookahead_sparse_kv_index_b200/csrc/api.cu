@@ -57,6 +57,10 @@ extern "C" {
 
 int32_t lsa_version(void) { return 100; }
 
+int64_t lsa_struct_size(int32_t which) {
+    return which == 0 ? int64_t(sizeof(lsa_params)) : which == 1 ? int64_t(sizeof(lsa_ctx_view)) : -1;
+}
+
 const char *lsa_last_error(void) { return lsa::g_msg; }
 
 const char *lsa_status_name(lsa_status s) {
@@ -172,7 +176,7 @@ lsa_status lsa_sparse_attn(const void *Q, lsa_dtype dtype, const void *kv, int64
     LSA_CHECK_ARG(B >= 1, "lsa_sparse_attn: B=%d", B);
     LSA_CHECK_SUPPORTED(D % 32 == 0 && D >= 32 && D <= 512, "lsa_sparse_attn: D=%d", D);
     LSA_CHECK_SUPPORTED(Hq >= 1 && Hq <= 256, "lsa_sparse_attn: Hq=%d", Hq);
-    LSA_CHECK_SUPPORTED(k >= 1 && k <= 4096, "lsa_sparse_attn: k=%d", k);
+    LSA_CHECK_SUPPORTED(k >= 1 && k <= 65536, "lsa_sparse_attn: k=%d not in [1, 65536]", k);
     LSA_CHECK_ARG(kv_row_stride >= D && k_off >= 0 && v_off >= 0 && k_off + D <= kv_row_stride &&
                       v_off + D <= kv_row_stride,
                   "lsa_sparse_attn: K/V must lie inside a row");

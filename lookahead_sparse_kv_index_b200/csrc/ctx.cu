@@ -16,6 +16,7 @@
 // step is captured once per distinct set of input and output pointers and
 // replayed with one graph launch; a decode loop that reuses its buffers runs
 // two graphs.  Stage timing runs the kernels eagerly.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <unordered_map>
@@ -67,6 +68,11 @@ struct lsa_ctx {
     int64_t *fetched = nullptr;     // rows fetched by the last refresh
     void *fetch_ws = nullptr;
     cudaEvent_t ev_assign = nullptr;
+    // merged attention set: window and HCA rows live in the arena after the hot buffer
+    bool merged = false;
+    int64_t win_base = 0, hca_base = 0, row_cap = 0;
+    int64_t *hca_off_d = nullptr;
+    int32_t *attn_rows = nullptr;
     void *sel_ws = nullptr;
     size_t sel_ws_bytes = 0;
     void *attn_ws = nullptr;
@@ -107,7 +113,7 @@ using namespace lsa;
 void free_all(lsa_ctx *c) {
     void *bufs[] = {c->seq_off_d, c->z, c->z_kept, c->kept_idx, c->kept_off, c->slot_of, c->hot,
                     c->topk_idx, c->topk_pos, c->topk_cnt, c->err, c->sel_ws, c->attn_ws,
-                    c->owner, c->kept_slot, c->fetched, c->fetch_ws};
+                    c->owner, c->kept_slot, c->fetched, c->fetch_ws, c->hca_off_d, c->attn_rows};
     for (void *b : bufs)
         if (b) cudaFree(b);
     for (auto &sg : c->stage) {
@@ -224,8 +230,16 @@ lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w,
         tk.done();
     }
     StageTimer ta(c, LSA_STAGE_ATTN, st);
-    LSA_TRY(launch_sparse_attn(Q, p.attn_dtype, c->hot, p.kv_row_stride, p.k_off, p.v_off, c->topk_pos,
-                               p.B, p.Hq, p.D, p.topk, c->scale, out, lse, c->attn_ws, c->err, st));
+    if (c->merged) {
+        LSA_TRY(launch_merge_rows(c->topk_idx, c->topk_pos, c->topk_cnt, c->seq_off_d, p.B, p.topk, p.window,
+                                  int32_t(c->win_base), c->hca_off_d, int32_t(c->hca_base), c->attn_rows,
+                                  int32_t(c->row_cap), nullptr, c->err, st));
+        LSA_TRY(launch_sparse_attn(Q, p.attn_dtype, c->hot, p.kv_row_stride, p.k_off, p.v_off, c->attn_rows, p.B,
+                                   p.Hq, p.D, int32_t(c->row_cap), c->scale, out, lse, c->attn_ws, c->err, st));
+    } else {
+        LSA_TRY(launch_sparse_attn(Q, p.attn_dtype, c->hot, p.kv_row_stride, p.k_off, p.v_off, c->topk_pos,
+                                   p.B, p.Hq, p.D, p.topk, c->scale, out, lse, c->attn_ws, c->err, st));
+    }
     ta.done();
     return LSA_OK;
 }
@@ -304,6 +318,23 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     LSA_CHECK_ARG(so[0] == 0 && so[p.B] == p.n_total, "lsa_ctx_create: seq_off must run from 0 to n_total");
     for (int b = 0; b < p.B; ++b)
         LSA_CHECK_ARG(so[b + 1] >= so[b], "lsa_ctx_create: seq_off must be non-decreasing");
+    LSA_CHECK_ARG(p.window >= 0, "lsa_ctx_create: window < 0");
+    LSA_CHECK_ARG(!p.hca_rows || p.hca_off_host, "lsa_ctx_create: hca_rows needs hca_off_host");
+    int64_t n_hca = 0, max_hca = 0;
+    if (p.hca_rows) {
+        const int64_t *ho = p.hca_off_host;
+        LSA_CHECK_ARG(ho[0] == 0, "lsa_ctx_create: hca_off_host[0] must be 0");
+        for (int b = 0; b < p.B; ++b) {
+            LSA_CHECK_ARG(ho[b + 1] >= ho[b], "lsa_ctx_create: hca_off_host must be non-decreasing");
+            max_hca = std::max(max_hca, ho[b + 1] - ho[b]);
+        }
+        n_hca = ho[p.B];
+    }
+    const bool merged = p.window > 0 || n_hca > 0;
+    const int64_t row_cap = merged ? int64_t(p.topk) + p.window + max_hca : p.topk;
+    const int64_t arena_rows = p.kept_capacity + (merged ? int64_t(p.B) * p.window + n_hca : 0);
+    LSA_CHECK_SUPPORTED(row_cap <= 65536, "lsa_ctx_create: topk + window + HCA rows per sequence > 65536");
+    LSA_CHECK_ARG(arena_rows < (int64_t(1) << 31), "lsa_ctx_create: hot buffer, window and HCA rows exceed 2^31");
 
     cudaPointerAttributes attr;
     cudaError_t e = cudaPointerGetAttributes(&attr, p.cold_host);
@@ -324,7 +355,11 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     const size_t qbytes = size_t(p.B) * p.H * p.d * elem_size(p.q_dtype);
     const size_t Qbytes = size_t(p.B) * p.Hq * p.D * elem_size(p.attn_dtype);
     c->sel_ws_bytes = lsa_select_workspace_size(p.n_total);
-    c->attn_ws_bytes = sparse_attn_workspace(p.B, p.Hq, p.D, p.topk);
+    c->attn_ws_bytes = sparse_attn_workspace(p.B, p.Hq, p.D, int32_t(row_cap));
+    c->merged = merged;
+    c->row_cap = row_cap;
+    c->win_base = cap;
+    c->hca_base = cap + int64_t(p.B) * p.window;
     lsa_status s = LSA_OK;
 #define LSA_ALLOC(ptr, bytes) \
     if (s == LSA_OK) s = alloc(&(ptr), (bytes))
@@ -334,7 +369,11 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     LSA_ALLOC(c->kept_idx, size_t(cap) * 4);
     LSA_ALLOC(c->kept_off, size_t(p.B + 1) * 8);
     LSA_ALLOC(c->slot_of, size_t(p.n_total) * 4);
-    LSA_ALLOC(c->hot, size_t(cap) * p.row_bytes);
+    LSA_ALLOC(c->hot, size_t(arena_rows) * p.row_bytes);
+    if (merged) {
+        LSA_ALLOC(c->hca_off_d, size_t(p.B + 1) * 8);
+        LSA_ALLOC(c->attn_rows, size_t(p.B) * row_cap * 4);
+    }
     LSA_ALLOC(c->topk_idx, size_t(p.B) * p.topk * 4);
     LSA_ALLOC(c->topk_pos, size_t(p.B) * p.topk * 4);
     LSA_ALLOC(c->topk_cnt, size_t(p.B) * 4);
@@ -356,7 +395,25 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     if (s == LSA_OK) {
         cudaError_t ce = cudaMemcpy(c->seq_off_d, so, size_t(p.B + 1) * 8, cudaMemcpyHostToDevice);
         if (ce == cudaSuccess) ce = cudaMemset(c->err, 0, 16);
-        if (ce == cudaSuccess) ce = cudaMemset(c->hot, 0, size_t(cap) * p.row_bytes);
+        if (ce == cudaSuccess) ce = cudaMemset(c->hot, 0, size_t(arena_rows) * p.row_bytes);
+        if (merged) {
+            // always-resident context: the last `window` entries of each sequence, then the HCA rows
+            char *arena = static_cast<char *>(c->hot);
+            const char *cold = static_cast<const char *>(p.cold_host);
+            for (int b = 0; b < p.B && ce == cudaSuccess; ++b) {
+                const int64_t w_b = std::min<int64_t>(p.window, so[b + 1] - so[b]);
+                if (w_b > 0)
+                    ce = cudaMemcpy(arena + (c->win_base + int64_t(b) * p.window) * p.row_bytes,
+                                    cold + (so[b + 1] - w_b) * p.row_bytes, size_t(w_b) * p.row_bytes,
+                                    cudaMemcpyDefault);
+            }
+            if (ce == cudaSuccess && n_hca > 0)
+                ce = cudaMemcpy(arena + c->hca_base * p.row_bytes, p.hca_rows, size_t(n_hca) * p.row_bytes,
+                                cudaMemcpyDefault);
+            std::vector<int64_t> ho(p.B + 1, 0);
+            if (p.hca_rows) ho.assign(p.hca_off_host, p.hca_off_host + p.B + 1);
+            if (ce == cudaSuccess) ce = cudaMemcpy(c->hca_off_d, ho.data(), ho.size() * 8, cudaMemcpyHostToDevice);
+        }
         // empty cache: no entry resident, no slot owned
         if (ce == cudaSuccess) ce = cudaMemset(c->slot_of, 0xFF, size_t(p.n_total > 0 ? p.n_total : 1) * 4);
         if (ce == cudaSuccess) ce = cudaMemset(c->owner, 0xFF, size_t(cap) * 4);
@@ -453,6 +510,10 @@ lsa_status lsa_ctx_get_view(lsa_ctx *c, lsa_ctx_view *v) {
     v->kept_slot = c->p.full_fetch ? nullptr : c->kept_slot;
     v->owner = c->p.full_fetch ? nullptr : c->owner;
     v->fetched = c->fetched;
+    v->attn_rows = c->attn_rows;
+    v->attn_row_cap = c->row_cap;
+    v->win_base = c->win_base;
+    v->hca_base = c->hca_base;
     return LSA_OK;
 }
 

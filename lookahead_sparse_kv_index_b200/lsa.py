@@ -37,6 +37,7 @@ EXPORTS = [
     "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
     "lsa_ctx_set_graphs", "lsa_ctx_set_timing", "lsa_ctx_stage_times", "lsa_ctx_reset_counters",
     "lsa_ctx_launches", "lsa_selftest_bounded_wait", "lsa_index_union", "lsa_query_encode",
+    "lsa_attn_set_merge", "lsa_struct_size",
 ]
 
 
@@ -53,14 +54,14 @@ class Params(ctypes.Structure):
         ("Hq", i32), ("D", i32), ("attn_dtype", i32), ("topk", i32), ("tau", i32), ("scale", f32),
         ("n_total", i64), ("seq_off_host", P), ("k_dev", P), ("k_scale_dev", P), ("cold_host", P),
         ("row_bytes", i64), ("kv_row_stride", i64), ("k_off", i64), ("v_off", i64), ("kept_capacity", i64),
-        ("full_fetch", i32),
+        ("full_fetch", i32), ("window", i32), ("hca_rows", P), ("hca_off_host", P),
     ]
 
 
 class View(ctypes.Structure):
     _fields_ = [("z", P), ("z_kept", P), ("kept_idx", P), ("kept_off", P), ("slot_of", P), ("hot", P),
                 ("topk_idx", P), ("topk_pos", P), ("topk_cnt", P), ("err", P), ("kept_slot", P), ("owner", P),
-                ("fetched", P)]
+                ("fetched", P), ("attn_rows", P), ("attn_row_cap", i64), ("win_base", i64), ("hca_base", i64)]
 
 
 def _sig(name, res, args):
@@ -70,6 +71,7 @@ def _sig(name, res, args):
 
 
 _sig("lsa_version", i32, [])
+_sig("lsa_struct_size", i64, [i32])
 _sig("lsa_last_error", ctypes.c_char_p, [])
 _sig("lsa_status_name", ctypes.c_char_p, [i32])
 _sig("lsa_index_score", i32, [P, i32, P, P, i32, P, P, i64, P, P, i64, i32, i32, i32, P, P, i32, P, P])
@@ -95,6 +97,7 @@ _sig("lsa_ctx_launches", i64, [P])
 _sig("lsa_selftest_bounded_wait", i32, [i64, P, P, P])
 _sig("lsa_index_union", i32, [ctypes.POINTER(P), i32, i64, P, P])
 _sig("lsa_query_encode", i32, [P, i32, i32, P, i32, P, i32, i32, P, P, i32, P, P, P])
+_sig("lsa_attn_set_merge", i32, [P, P, P, P, i32, i32, i32, i32, P, i32, P, i32, P, P, P])
 
 lib = _L
 
@@ -171,6 +174,15 @@ def query_encode(h, W_dq, W_uq, W_w, H, d, q_out, q_dtype, w_out, c_out, stream=
                                DTYPE[q_dtype], _ptr(w_out), _ptr(c_out), _stream(stream)), "lsa_query_encode")
 
 
+def attn_set_merge(topk_idx, topk_pos, topk_cnt, seq_off, k, window, win_base, hca_off, hca_base, rows, row_cap,
+                   count=None, err=None, stream=None):
+    """Merged attention set: per sequence the row list top-k (outside the window) + HCA rows + window rows."""
+    B = seq_off.numel() - 1
+    _check(_L.lsa_attn_set_merge(_ptr(topk_idx), _ptr(topk_pos), _ptr(topk_cnt), _ptr(seq_off), B, k, window,
+                                 win_base, _ptr(hca_off), hca_base, _ptr(rows), row_cap, _ptr(count), _ptr(err),
+                                 _stream(stream)), "lsa_attn_set_merge")
+
+
 def selftest_bounded_wait(limit_ns, err, waited_ns, stream=None):
     """Runs a bounded device wait on a barrier nothing arrives at (see lsa.h)."""
     _check(_L.lsa_selftest_bounded_wait(int(limit_ns), _ptr(err), _ptr(waited_ns), _stream(stream)),
@@ -212,13 +224,17 @@ class Context:
 
     def __init__(self, *, B, H, d, q_dtype, k_dtype, Hq, D, attn_dtype, topk, seq_off_host, keys, k_scale,
                  cold_host, row_bytes, kv_row_stride, k_off, v_off, kept_capacity, tau=64, scale=0.0,
-                 full_fetch=False):
+                 full_fetch=False, window=0, hca_rows=None, hca_off_host=None):
+        """window / hca_rows / hca_off_host: the always-resident context merged into the attention set
+        (see lsa_attn_set_merge); hca_rows is a host or device tensor of HCA rows in the cold-pool row format."""
         self._seq_off = torch.as_tensor(seq_off_host, dtype=torch.int64).contiguous()
+        self._hca_off = None if hca_off_host is None else torch.as_tensor(hca_off_host, dtype=torch.int64).contiguous()
         n_total = int(self._seq_off[-1])
         self.params = Params(B, H, d, DTYPE[q_dtype], DTYPE[k_dtype], Hq, D, DTYPE[attn_dtype], topk, tau,
                              float(scale), n_total, self._seq_off.data_ptr(), _ptr(keys), _ptr(k_scale),
                              _ptr(cold_host), row_bytes, kv_row_stride, k_off, v_off, kept_capacity,
-                             int(bool(full_fetch)))
+                             int(bool(full_fetch)), int(window), _ptr(hca_rows),
+                             None if self._hca_off is None else self._hca_off.data_ptr())
         self._keep = (keys, k_scale, cold_host)
         h = P()
         _check(_L.lsa_ctx_create(ctypes.byref(self.params), ctypes.byref(h)), "lsa_ctx_create")

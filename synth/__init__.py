@@ -336,3 +336,24 @@ def hidden_states(seed: int, B: int, hidden: int = ENCODER_HIDDEN, t: int = 0) -
     """bf16 bits [B, hidden]: the decode-step-t hidden states of B sequences."""
     g = torch.Generator().manual_seed(seed * 1000003 + 31 + t)
     return bf16_bits(torch.randn(B, hidden, generator=g))
+
+
+# -------------------------------------------------- always-resident context
+# HCA rows (heavily compressed attention, 128 tokens per row) for the merged
+# attention set: a sequence of N_b compressed entries at 4:1 covers 4 N_b
+# tokens, so it has ceil(4 N_b / 128) = ceil(N_b / 32) HCA rows.  Rows follow
+# the cold pool's row format and distribution (N(0, 1) latent rows).
+HCA_RATIO = 128
+ENTRY_RATIO = 4
+RECENT_TOKENS = 8192   # the recent window of 8K tokens = 2048 compressed entries at 4:1
+
+
+def hca_rows(wl: Workload, seed: int = 0):
+    """(rows raw [sum_b n_hca_b, row_stride], hca_off int64 [B+1]) in the workload's cold-row format."""
+    n_b = np.diff(wl.seq_off)
+    n_hca = (n_b * ENTRY_RATIO + HCA_RATIO - 1) // HCA_RATIO
+    hca_off = np.concatenate([[0], np.cumsum(n_hca)]).astype(np.int64)
+    g = torch.Generator().manual_seed(wl.seed * 7907 + 3 + seed)
+    dtype = "bf16" if wl.cold.dtype == np.uint16 else "f32"
+    rows = _randn_chunked(g, int(hca_off[-1]), wl.row_stride, dtype)
+    return rows, hca_off

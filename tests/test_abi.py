@@ -93,6 +93,41 @@ def test_other_entry_points_reject_bad_arguments(lsa):
     assert L.lsa_index_union(arr, 3, 10, big, None) == 1                      # a layer without scores
 
 
+def test_struct_mirrors_match_the_header(lsa):
+    assert lsa.lib.lsa_struct_size(0) == ctypes.sizeof(lsa.Params)
+    assert lsa.lib.lsa_struct_size(1) == ctypes.sizeof(lsa.View)
+    assert lsa.lib.lsa_struct_size(2) == -1
+
+
+def test_encoder_and_merge_reject_bad_arguments(lsa):
+    L, big = lsa.lib, 1 << 20
+    ok = dict(h=big, B=4, hidden=7168, W_dq=big, rank=1536, W_uq=big, H=64, d=128, W_w=big, q=big, qdt=1, w=big,
+              c=big)
+
+    def enc(**kw):
+        a = dict(ok, **kw)
+        return L.lsa_query_encode(a["h"], a["B"], a["hidden"], a["W_dq"], a["rank"], a["W_uq"], a["H"], a["d"],
+                                  a["W_w"], a["q"], a["qdt"], a["w"], a["c"], None)
+
+    assert enc(h=None) == 1
+    assert enc(c=None) == 1
+    assert enc(B=0) == 1
+    assert enc(hidden=7164) == 1          # not a multiple of 8
+    assert enc(rank=4) == 1
+    assert enc(H=0) == 1
+    assert enc(W_uq=big + 2) == 1         # unaligned
+    assert enc(qdt=2) == 5                # E4M3 queries are not produced
+    # merge: topk_idx, topk_pos, topk_cnt, seq_off, B, k, window, win_base, hca_off, hca_base, rows, row_cap, ...
+    assert L.lsa_attn_set_merge(None, big, big, big, 2, 32, 16, 0, None, 0, big, 64, None, None, None) == 1
+    assert L.lsa_attn_set_merge(big, big, big, big, 2, 0, 16, 0, None, 0, big, 64, None, None, None) == 1
+    assert L.lsa_attn_set_merge(big, big, big, big, 2, 32, -1, 0, None, 0, big, 64, None, None, None) == 1
+    assert L.lsa_attn_set_merge(big, big, big, big, 2, 32, 16, 0, None, 0, big, 0, None, None, None) == 1
+    assert L.lsa_attn_set_merge(big, big, big, big, 2, 32, 1 << 30, 1 << 30, None, 0, big, 64, None, None,
+                                None) == 1                                              # rows overflow int32
+    assert L.lsa_sparse_attn(big, 1, big, 512, 0, 0, big, 1, 128, 512, 70000, 1.0, big, None, big, 1 << 40, None,
+                             None) == 5                                                 # k above 65536
+
+
 def test_ctx_create_rejects_bad_params(lsa):
     import numpy as np
 
@@ -103,4 +138,11 @@ def test_ctx_create_rejects_bad_params(lsa):
     assert lsa.lib.lsa_ctx_create(ctypes.byref(p), ctypes.byref(h)) == 1   # seq_off decreasing
     p.kv_row_stride = 256
     assert lsa.lib.lsa_ctx_create(ctypes.byref(p), ctypes.byref(h)) == 1   # stride * 2 != row_bytes
+    so[:] = [0, 3, 5]
+    p.kv_row_stride = 512
+    p.window = -1
+    assert lsa.lib.lsa_ctx_create(ctypes.byref(p), ctypes.byref(h)) == 1   # negative window
+    p.window = 16
+    p.hca_rows = 1 << 20
+    assert lsa.lib.lsa_ctx_create(ctypes.byref(p), ctypes.byref(h)) == 1   # HCA rows without offsets
     assert h.value is None
