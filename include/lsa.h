@@ -346,6 +346,14 @@ typedef struct lsa_params {
     const void *hca_rows;        /* HCA rows [hca_off_host[B], row_bytes], host or device memory, same
                                     row format as the cold pool; NULL: none */
     const int64_t *hca_off_host; /* HOST [B+1] offsets of each sequence's HCA rows (with hca_rows) */
+    /* OR-mode union of indexer layers in the cadence (lsa_index_union): with n_layers >= 2 every
+     * refresh scores each layer's keys with that layer's (q, w) and selects and ranks on the union
+     * score max_l z_l; listed steps re-score the kept set in every layer and rank on the union.
+     * q and w then carry a leading layer dimension: q [n_layers, B, H, d], w [n_layers, B, H]. */
+    int32_t n_layers;                   /* 0 or 1: one layer (k_dev); 2 .. 8: layers 0 .. n_layers-1 */
+    const void *const *k_dev_layers;    /* HOST array [n_layers-1] of DEVICE key pointers of layers
+                                           1 .. n_layers-1 (layer 0 is k_dev); same dtype and shape */
+    const float *const *k_scale_layers; /* HOST array [n_layers-1] of their E4M3 row scales (else NULL) */
 } lsa_params;
 
 typedef struct lsa_ctx lsa_ctx;
@@ -357,7 +365,8 @@ lsa_status lsa_ctx_create(const lsa_params *p, lsa_ctx **out);
 lsa_status lsa_ctx_destroy(lsa_ctx *ctx);
 
 /* One decode step t >= 0 on device buffers: q [B,H,d], w [B,H], Q [B,Hq,D]
- * in; out [B,Hq,D] and lse [B,Hq] (lse may be NULL) out. */
+ * in ([n_layers, B, H, d] and [n_layers, B, H] with n_layers >= 2); out
+ * [B,Hq,D] and lse [B,Hq] (lse may be NULL) out. */
 lsa_status lsa_decode_step(lsa_ctx *ctx, int64_t t, const void *q, const float *w, const void *Q,
                            void *out, float *lse, void *stream);
 

@@ -68,6 +68,12 @@ struct lsa_ctx {
     int64_t *fetched = nullptr;     // rows fetched by the last refresh
     void *fetch_ws = nullptr;
     cudaEvent_t ev_assign = nullptr;
+    // indexer layers (OR-mode union): keys and scales per layer, per-layer scores
+    int n_layers = 1;
+    const void *k_layer[lsa::kMaxUnionLayers] = {};
+    const float *ks_layer[lsa::kMaxUnionLayers] = {};
+    float *z_layers = nullptr;    // [n_layers, n_total] full-scan scores (n_layers >= 2)
+    float *zk_layers = nullptr;   // [n_layers, kept_capacity] listed scores (n_layers >= 2)
     // merged attention set: window and HCA rows live in the arena after the hot buffer
     bool merged = false;
     int64_t win_base = 0, hca_base = 0, row_cap = 0;
@@ -113,7 +119,8 @@ using namespace lsa;
 void free_all(lsa_ctx *c) {
     void *bufs[] = {c->seq_off_d, c->z, c->z_kept, c->kept_idx, c->kept_off, c->slot_of, c->hot,
                     c->topk_idx, c->topk_pos, c->topk_cnt, c->err, c->sel_ws, c->attn_ws,
-                    c->owner, c->kept_slot, c->fetched, c->fetch_ws, c->hca_off_d, c->attn_rows};
+                    c->owner, c->kept_slot, c->fetched, c->fetch_ws, c->hca_off_d, c->attn_rows, c->z_layers,
+                    c->zk_layers};
     for (void *b : bufs)
         if (b) cudaFree(b);
     for (auto &sg : c->stage) {
@@ -188,11 +195,25 @@ lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w,
                         float *lse, cudaStream_t st) {
     const lsa_params &p = c->p;
     const int64_t cap = p.kept_capacity;
+    const size_t q_layer = size_t(p.B) * p.H * p.d * elem_size(p.q_dtype);   // bytes of one layer's q
+    const size_t w_layer = size_t(p.B) * p.H;                                 // floats of one layer's w
     if (refresh) {
         StageTimer ts(c, LSA_STAGE_SCORE, st);
-        LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
-                                   p.n_total, nullptr, nullptr, 0, p.B, p.H, p.d, c->z, nullptr, 0,
-                                   c->err, st));
+        if (c->n_layers == 1) {
+            LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
+                                       p.n_total, nullptr, nullptr, 0, p.B, p.H, p.d, c->z, nullptr, 0,
+                                       c->err, st));
+        } else {
+            const float *zl[kMaxUnionLayers];
+            for (int l = 0; l < c->n_layers; ++l) {
+                float *z_l = c->z_layers + size_t(l) * p.n_total;
+                LSA_TRY(launch_index_score(static_cast<const char *>(q) + l * q_layer, p.q_dtype, w + l * w_layer,
+                                           c->k_layer[l], p.k_dtype, c->ks_layer[l], c->seq_off_d, p.n_total,
+                                           nullptr, nullptr, 0, p.B, p.H, p.d, z_l, nullptr, 0, c->err, st));
+                zl[l] = z_l;
+            }
+            LSA_TRY(launch_union(zl, c->n_layers, p.n_total, c->z, st));
+        }
         ts.done();
         StageTimer tsel(c, LSA_STAGE_SELECT, st);
         LSA_TRY(launch_select(c->z, c->seq_off_d, p.n_total, p.B, c->kept_idx, cap, c->kept_off,
@@ -220,9 +241,24 @@ lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w,
         LSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
     } else {
         StageTimer tr(c, LSA_STAGE_RESCORE, st);
-        LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
-                                   p.n_total, c->kept_idx, c->kept_off, cap, p.B, p.H, p.d, c->z_kept,
-                                   nullptr, 0, c->err, st));
+        if (c->n_layers == 1) {
+            LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
+                                       p.n_total, c->kept_idx, c->kept_off, cap, p.B, p.H, p.d, c->z_kept,
+                                       nullptr, 0, c->err, st));
+        } else {
+            // every layer re-scores the kept set; the ranking score is their union (positions past the
+            // kept total hold stale values that the top-k never reads)
+            const float *zl[kMaxUnionLayers];
+            for (int l = 0; l < c->n_layers; ++l) {
+                float *z_l = c->zk_layers + size_t(l) * cap;
+                LSA_TRY(launch_index_score(static_cast<const char *>(q) + l * q_layer, p.q_dtype, w + l * w_layer,
+                                           c->k_layer[l], p.k_dtype, c->ks_layer[l], c->seq_off_d, p.n_total,
+                                           c->kept_idx, c->kept_off, cap, p.B, p.H, p.d, z_l, nullptr, 0, c->err,
+                                           st));
+                zl[l] = z_l;
+            }
+            LSA_TRY(launch_union(zl, c->n_layers, cap, c->z_kept, st));
+        }
         tr.done();
         StageTimer tk(c, LSA_STAGE_TOPK, st);
         LSA_TRY(launch_topk(c->z_kept, 0, c->seq_off_d, c->kept_idx, c->kept_off, p.B, p.topk, cap,
@@ -319,6 +355,17 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     for (int b = 0; b < p.B; ++b)
         LSA_CHECK_ARG(so[b + 1] >= so[b], "lsa_ctx_create: seq_off must be non-decreasing");
     LSA_CHECK_ARG(p.window >= 0, "lsa_ctx_create: window < 0");
+    const int n_layers = p.n_layers <= 1 ? 1 : p.n_layers;
+    LSA_CHECK_ARG(n_layers <= kMaxUnionLayers, "lsa_ctx_create: n_layers=%d > %d", p.n_layers, kMaxUnionLayers);
+    if (n_layers > 1) {
+        LSA_CHECK_ARG(p.k_dev_layers, "lsa_ctx_create: n_layers >= 2 needs k_dev_layers");
+        LSA_CHECK_ARG(p.k_dtype != LSA_E4M3 || p.k_scale_layers, "lsa_ctx_create: E4M3 layers need k_scale_layers");
+        for (int l = 1; l < n_layers; ++l) {
+            LSA_CHECK_ARG(p.k_dev_layers[l - 1], "lsa_ctx_create: layer %d has no keys", l);
+            LSA_CHECK_ARG((p.k_dtype == LSA_E4M3) == (p.k_scale_layers && p.k_scale_layers[l - 1] != nullptr),
+                          "lsa_ctx_create: layer %d: a row-scale pointer for E4M3 keys and only for them", l);
+        }
+    }
     LSA_CHECK_ARG(!p.hca_rows || p.hca_off_host, "lsa_ctx_create: hca_rows needs hca_off_host");
     int64_t n_hca = 0, max_hca = 0;
     if (p.hca_rows) {
@@ -357,6 +404,15 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     c->sel_ws_bytes = lsa_select_workspace_size(p.n_total);
     c->attn_ws_bytes = sparse_attn_workspace(p.B, p.Hq, p.D, int32_t(row_cap));
     c->merged = merged;
+    c->n_layers = n_layers;
+    c->k_layer[0] = p.k_dev;
+    c->ks_layer[0] = p.k_scale_dev;
+    for (int l = 1; l < n_layers; ++l) {
+        c->k_layer[l] = p.k_dev_layers[l - 1];
+        c->ks_layer[l] = p.k_scale_layers ? p.k_scale_layers[l - 1] : nullptr;
+    }
+    c->p.k_dev_layers = nullptr;     // the caller's arrays are not kept
+    c->p.k_scale_layers = nullptr;
     c->row_cap = row_cap;
     c->win_base = cap;
     c->hca_base = cap + int64_t(p.B) * p.window;
@@ -370,6 +426,10 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     LSA_ALLOC(c->kept_off, size_t(p.B + 1) * 8);
     LSA_ALLOC(c->slot_of, size_t(p.n_total) * 4);
     LSA_ALLOC(c->hot, size_t(arena_rows) * p.row_bytes);
+    if (n_layers > 1) {
+        LSA_ALLOC(c->z_layers, size_t(n_layers) * p.n_total * 4);
+        LSA_ALLOC(c->zk_layers, size_t(n_layers) * cap * 4);
+    }
     if (merged) {
         LSA_ALLOC(c->hca_off_d, size_t(p.B + 1) * 8);
         LSA_ALLOC(c->attn_rows, size_t(p.B) * row_cap * 4);
@@ -385,8 +445,8 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     LSA_ALLOC(c->fetched, 16);
     LSA_ALLOC(c->fetch_ws, fetch_workspace(cap));
     for (auto &sg : c->stage) {
-        LSA_ALLOC(sg.q, qbytes);
-        LSA_ALLOC(sg.w, size_t(p.B) * p.H * 4);
+        LSA_ALLOC(sg.q, qbytes * n_layers);
+        LSA_ALLOC(sg.w, size_t(n_layers) * p.B * p.H * 4);
         LSA_ALLOC(sg.Q, Qbytes);
         LSA_ALLOC(sg.out, Qbytes);
         LSA_ALLOC(sg.lse, size_t(p.B) * p.Hq * 4);
@@ -473,8 +533,8 @@ lsa_status lsa_decode_step_host(lsa_ctx *c, int64_t t, const void *q_host, const
     // inputs on the copy stream, once the slot's previous step has read them;
     // they overlap the kernels of the step enqueued before this one
     LSA_CUDA(cudaStreamWaitEvent(c->h2d, sg.used, 0));
-    LSA_CUDA(cudaMemcpyAsync(sg.q, q_host, qbytes, cudaMemcpyHostToDevice, c->h2d));
-    LSA_CUDA(cudaMemcpyAsync(sg.w, w_host, size_t(p.B) * p.H * 4, cudaMemcpyHostToDevice, c->h2d));
+    LSA_CUDA(cudaMemcpyAsync(sg.q, q_host, qbytes * c->n_layers, cudaMemcpyHostToDevice, c->h2d));
+    LSA_CUDA(cudaMemcpyAsync(sg.w, w_host, size_t(c->n_layers) * p.B * p.H * 4, cudaMemcpyHostToDevice, c->h2d));
     LSA_CUDA(cudaMemcpyAsync(sg.Q, Q_host, Qbytes, cudaMemcpyHostToDevice, c->h2d));
     LSA_CUDA(cudaEventRecord(sg.in_ready, c->h2d));
     LSA_CUDA(cudaStreamWaitEvent(st, sg.in_ready, 0));

@@ -288,10 +288,20 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     constexpr uint32_t NCOL = tmem_cols(KACC * TILEC);
     static_assert(G >= 1 && G <= KACC / 2, "the epilogue must own accumulators while a group is issued");
     static_assert(S >= G, "a group waits for G filled stages");
-    // a stage is free again when the MMA of the tile it held has completed, which the producer learns
-    // from that tile's accumulator barrier; a parity wait on it is unambiguous while the barrier
-    // cannot run two phases ahead, i.e. while S <= 2 * KACC
-    static_assert(S <= 2 * KACC, "stage reuse is tracked on the accumulator barriers");
+    // One commit per tile tells both the epilogue (accumulator ready) and the producer (stage free)
+    // that the tile's MMAs completed.  A parity wait is only unambiguous while the barrier cannot
+    // complete a second phase past the one waited for.  Per accumulator (S <= KACC): the next tile
+    // on the same accumulator needs this tile's epilogue release, and the producer's wait for tile
+    // j - S sees no other tile of that accumulator before j.  With more stages than accumulators
+    // (e4m3 keys: 4 stages, 2 accumulators) tile j - S + KACC shares the accumulator and could
+    // complete while a slow producer (listed gathers) has not yet polled for tile j - S: there the
+    // barrier is per stage, whose next use is the producer's own load; the epilogue's wait stays
+    // unambiguous because tile i + S needs every epilogue warp's release of tile i + S - KACC >= i.
+    constexpr bool kStageDone = S > KACC;
+    constexpr int NDONE = kStageDone ? S : KACC;
+    static_assert(NDONE <= kAccMax, "completion barriers");
+    static_assert(!kStageDone || (S % KACC == 0 && C::kSub == 2),
+                  "per-stage completion needs every epilogue warp on every tile, in order");
     // e4m3 keys: the per-row scales of each tile go to a shared-memory ring by cp.async (the
     // producer warp), never through a register load of an epilogue warp, whose wait on its TMEM
     // loads would otherwise also wait for that HBM load.  Slot j % RS holds tile j's scales; it is
@@ -308,7 +318,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     uint64_t *full = reinterpret_cast<uint64_t *>(qimg + 2 * QIMG);  // [S] stage loaded
     uint64_t *qfull = full + S;                                   // [2] query slot built
     uint64_t *qrel = qfull + 2;                                   // [kRel] by sequence ordinal
-    // [KACC] the MMAs of a tile completed: its accumulator is ready and its stage is free
+    // [NDONE] the MMAs of a tile completed (per accumulator, or per stage when S > KACC): its
+    // accumulator is ready and its stage is free
     uint64_t *tdone = qrel + kRel;
     uint64_t *tempty = tdone + kAccMax;                           // [KACC] accumulator read by the epilogue
     uint64_t *drain = tempty + kAccMax;
@@ -362,7 +373,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         for (int s = 0; s < 2; ++s) mbar_init(&qfull[s], 1);
         for (int s = 0; s < kRel; ++s) mbar_init(&qrel[s], 1 + kEpiWarps);
         // an accumulator is released by the warps that read it: one warpgroup per 128-row sub-tile
-        for (int s = 0; s < KACC; ++s) { mbar_init(&tdone[s], 1); mbar_init(&tempty[s], 4 * C::kSub); }
+        for (int s = 0; s < NDONE; ++s) mbar_init(&tdone[s], 1);
+        for (int s = 0; s < KACC; ++s) mbar_init(&tempty[s], 4 * C::kSub);
         mbar_init(drain, 1);
         // full mode: one arrival (the bulk copy's expect_tx, or lane 0 after the copies landed); listed
         // mode: one cp.async-tracked arrival per producer lane
@@ -387,11 +399,14 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         // ------------------------------------------------------------ producer
         // builds the query operand of a new sequence (ordinal o) into slot o & 1
         // local tile j may be loaded once the MMA of tile j - S (same stage) has completed
+        // completion barrier and parity of local tile i
+        auto done_bar = [&](int64_t i) -> uint64_t * { return &tdone[int(i % NDONE)]; };
+        auto done_par = [&](int64_t i) -> uint32_t { return uint32_t((i / NDONE) & 1); };
         auto stage_free_test = [&](int64_t j) -> bool {
-            return j < S || mbar_test_wait(&tdone[(j - S) % KACC], uint32_t(((j - S) / KACC) & 1));
+            return j < S || mbar_test_wait(done_bar(j - S), done_par(j - S));
         };
         auto stage_free_wait = [&](int64_t j) -> bool {
-            return j < S || mbar_wait(&tdone[(j - S) % KACC], uint32_t(((j - S) / KACC) & 1), abort_v, kWaitLimitNs);
+            return j < S || mbar_wait(done_bar(j - S), done_par(j - S), abort_v, kWaitLimitNs);
         };
         // row scales of local tile j (rows [row0, row_end) of the entry axis), all 32 lanes.  A span
         // that starts 16-byte aligned and has a multiple of 4 rows goes by one bulk copy (the copy
@@ -551,7 +566,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 const int gn = int(gend - t < G ? gend - t : G);
                 uint64_t a_d[G];
                 uint32_t d_t[G];
-                int acc_of[G];
+                int done_of[G];   // completion barrier of each tile of the group
 #pragma unroll
                 for (int u = 0; u < G; ++u) {
                     if (u >= gn) break;
@@ -559,7 +574,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                     if (!mbar_wait(&full[st], ph, abort_v, kWaitLimitNs)) { ok = false; break; }
                     a_d[u] = a_cur;
                     d_t[u] = tmem_base + uint32_t(acc * TILEC);
-                    acc_of[u] = acc;
+                    done_of[u] = kStageDone ? st : acc;
                     a_cur += kStageStep;
                     if (++st == S) { st = 0; ph ^= 1; a_cur = a_desc0; }
                     if (++acc == KACC) { acc = 0; aph ^= 1; }
@@ -597,7 +612,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 issued = true;
 #pragma unroll
                 for (int u = 0; u < G; ++u)
-                    if (u < gn) mma_commit(&tdone[acc_of[u]]);   // accumulator ready, stage free
+                    if (u < gn) mma_commit(&tdone[done_of[u]]);   // accumulator ready, stage free
                 if (t == gend) mma_commit(&qrel[qn % kRel]);      // this sequence's operand is no longer read
             }
             if (issued) {
@@ -666,7 +681,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             }
             const float *wq = wsm + (ord & 1) * H;
             const int64_t row = row0 + sub * kRows + quarter * 32 + lane;   // entry (full) or list position
-            ok = mbar_wait(&tdone[acc], aph, abort_v, kWaitLimitNs);
+            ok = kStageDone ? mbar_wait(&tdone[int(i % S)], uint32_t((i / S) & 1), abort_v, kWaitLimitNs)
+                            : mbar_wait(&tdone[acc], aph, abort_v, kWaitLimitNs);
             // the row scales landed long before (loaded with the keys); read before the release
             if (kScales) ok = ok && mbar_wait(&sfull[i % RS], uint32_t((i / RS) & 1), abort_v, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld

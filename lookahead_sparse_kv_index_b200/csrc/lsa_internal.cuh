@@ -118,6 +118,9 @@ lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, 
                                  const int32_t *rows, int32_t B, int32_t k, float scale, void *part_o,
                                  float *part_ml, int32_t *err, cudaStream_t st);
 size_t sparse_attn_workspace(int32_t B, int32_t Hq, int32_t D, int32_t k);
+constexpr int kMaxUnionLayers = 8;
+lsa_status launch_union(const float *const *z_layers, int32_t n_layers, int64_t n_total, float *z_union,
+                        cudaStream_t st);
 lsa_status launch_merge_rows(const int32_t *topk_idx, const int32_t *topk_pos, const int32_t *topk_cnt,
                              const int64_t *seq_off, int32_t B, int32_t k, int32_t window, int32_t win_base,
                              const int64_t *hca_off, int32_t hca_base, int32_t *rows, int32_t row_cap,

@@ -14,7 +14,7 @@
 namespace lsa {
 namespace {
 
-constexpr int kMaxLayers = 8;
+constexpr int kMaxLayers = kMaxUnionLayers;
 constexpr int kThreads = 256;
 
 struct LayerPtrs {
@@ -47,6 +47,25 @@ __global__ void __launch_bounds__(kThreads) union_max(LayerPtrs zs, int n_layers
 }
 
 }  // namespace
+
+lsa_status launch_union(const float *const *z_layers, int32_t n_layers, int64_t n_total, float *z_union,
+                        cudaStream_t st) {
+    LayerPtrs zs = {};
+    bool aligned = (reinterpret_cast<uintptr_t>(z_union) & 15) == 0 && n_total % 4 == 0;
+    for (int l = 0; l < n_layers; ++l) {
+        zs.p[l] = z_layers[l];
+        aligned = aligned && (reinterpret_cast<uintptr_t>(z_layers[l]) & 15) == 0;
+    }
+    if (n_total == 0) return LSA_OK;
+    const int64_t units = aligned ? n_total / 4 : n_total;
+    const int64_t want = (units + kThreads - 1) / kThreads;
+    const int grid = int(want < int64_t(sm_count()) * 8 ? want : int64_t(sm_count()) * 8);
+    LSA_CUDA(launch_pdl(union_max, dim3(grid), dim3(kThreads), 0, st, zs, int(n_layers), n_total, int(aligned),
+                        z_union));
+    LSA_LAUNCHED("union_max");
+    return LSA_OK;
+}
+
 }  // namespace lsa
 
 using namespace lsa;
@@ -58,19 +77,6 @@ extern "C" lsa_status lsa_index_union(const float *const *z_layers, int32_t n_la
     LSA_CHECK_ARG(n_layers >= 1 && n_layers <= kMaxLayers, "lsa_index_union: n_layers=%d not in [1, %d]", n_layers,
                   kMaxLayers);
     LSA_CHECK_ARG(n_total >= 0, "lsa_index_union: n_total=%lld < 0", (long long)n_total);
-    LayerPtrs zs = {};
-    bool aligned = (reinterpret_cast<uintptr_t>(z_union) & 15) == 0 && n_total % 4 == 0;
-    for (int l = 0; l < n_layers; ++l) {
-        LSA_CHECK_ARG(z_layers[l], "lsa_index_union: layer %d has no scores", l);
-        zs.p[l] = z_layers[l];
-        aligned = aligned && (reinterpret_cast<uintptr_t>(z_layers[l]) & 15) == 0;
-    }
-    if (n_total == 0) return LSA_OK;
-    const int64_t units = aligned ? n_total / 4 : n_total;
-    const int64_t want = (units + kThreads - 1) / kThreads;
-    const int grid = int(want < int64_t(sm_count()) * 8 ? want : int64_t(sm_count()) * 8);
-    LSA_CUDA(launch_pdl(union_max, dim3(grid), dim3(kThreads), 0, as_stream(stream), zs, int(n_layers), n_total,
-                        int(aligned), z_union));
-    LSA_LAUNCHED("union_max");
-    return LSA_OK;
+    for (int l = 0; l < n_layers; ++l) LSA_CHECK_ARG(z_layers[l], "lsa_index_union: layer %d has no scores", l);
+    return launch_union(z_layers, n_layers, n_total, z_union, as_stream(stream));
 }

@@ -55,6 +55,7 @@ class Params(ctypes.Structure):
         ("n_total", i64), ("seq_off_host", P), ("k_dev", P), ("k_scale_dev", P), ("cold_host", P),
         ("row_bytes", i64), ("kv_row_stride", i64), ("k_off", i64), ("v_off", i64), ("kept_capacity", i64),
         ("full_fetch", i32), ("window", i32), ("hca_rows", P), ("hca_off_host", P),
+        ("n_layers", i32), ("k_dev_layers", P), ("k_scale_layers", P),
     ]
 
 
@@ -224,9 +225,11 @@ class Context:
 
     def __init__(self, *, B, H, d, q_dtype, k_dtype, Hq, D, attn_dtype, topk, seq_off_host, keys, k_scale,
                  cold_host, row_bytes, kv_row_stride, k_off, v_off, kept_capacity, tau=64, scale=0.0,
-                 full_fetch=False, window=0, hca_rows=None, hca_off_host=None):
+                 full_fetch=False, window=0, hca_rows=None, hca_off_host=None, layers=None):
         """window / hca_rows / hca_off_host: the always-resident context merged into the attention set
-        (see lsa_attn_set_merge); hca_rows is a host or device tensor of HCA rows in the cold-pool row format."""
+        (see lsa_attn_set_merge); hca_rows is a host or device tensor of HCA rows in the cold-pool row format.
+        layers: [(keys, k_scale), ...] of indexer layers 1 .. L-1 (layer 0 is keys / k_scale) for the OR-mode
+        union in the cadence; steps then take q [L, B, H, d] and w [L, B, H]."""
         self._seq_off = torch.as_tensor(seq_off_host, dtype=torch.int64).contiguous()
         self._hca_off = None if hca_off_host is None else torch.as_tensor(hca_off_host, dtype=torch.int64).contiguous()
         n_total = int(self._seq_off[-1])
@@ -235,7 +238,15 @@ class Context:
                              _ptr(cold_host), row_bytes, kv_row_stride, k_off, v_off, kept_capacity,
                              int(bool(full_fetch)), int(window), _ptr(hca_rows),
                              None if self._hca_off is None else self._hca_off.data_ptr())
-        self._keep = (keys, k_scale, cold_host)
+        self.n_layers = 1
+        if layers:
+            self.n_layers = 1 + len(layers)
+            self._karr = (P * len(layers))(*[_ptr(k) for k, _ in layers])
+            self._sarr = (P * len(layers))(*[_ptr(s) for _, s in layers])
+            self.params.n_layers = self.n_layers
+            self.params.k_dev_layers = ctypes.cast(self._karr, P)
+            self.params.k_scale_layers = ctypes.cast(self._sarr, P) if k_scale is not None else None
+        self._keep = (keys, k_scale, cold_host, layers)
         h = P()
         _check(_L.lsa_ctx_create(ctypes.byref(self.params), ctypes.byref(h)), "lsa_ctx_create")
         self.handle = h

@@ -10,27 +10,46 @@ fine-grained top-k inside the fetched subset feeds core attention (Tiered
 Selection).  Between refreshes the kept set stays fixed; each step re-ranks it
 with that step's indexer query (the reading used for "fine-grained Top-k
 selection within this restricted boundary").
+
+With several indexer layers (section 2.4 "Optimal Configuration": the layers'
+predictions are united at inference) each layer scores with its own keys and
+query, an entry is kept when any layer keeps it, and the ranking score is the
+union score max_l z_l (index_union).
 """
 from __future__ import annotations
 
 import numpy as np
 
-from . import TAU, gather, index_score, index_score_list, local_to_global, select, sparse_attn, topk
+from . import TAU, gather, index_score, index_score_list, index_union, local_to_global, select, sparse_attn, topk
 
 
 class OracleDecoder:
     """Plain sequential driver over the oracle stages; holds the kept set between refreshes."""
 
-    def __init__(self, wl, tau: int = TAU):
+    def __init__(self, wl, tau: int = TAU, layers=None):
+        """layers: [(keys, k_scale), ...] of indexer layers 1 .. L-1 (layer 0 is the workload's keys); with
+        layers, step() takes q [L, B, H, d] and w [L, B, H]."""
         self.wl = wl
         self.tau = tau
+        self.layers = [(wl.keys, wl.k_scale)] + list(layers or [])
         self.kept_idx = None
         self.kept_off = None
         self.slot_of = None
 
+    def _per_layer(self, q, w):
+        if len(self.layers) == 1:
+            return [(q, w, self.layers[0])]
+        return [(q[l], w[l], self.layers[l]) for l in range(len(self.layers))]
+
     def refresh(self, q, w):
         wl = self.wl
-        z, I = index_score(q, wl.q_dtype, w, wl.keys, wl.key_dtype, wl.k_scale, wl.seq_off, wl.H, wl.d)
+        if len(self.layers) == 1:
+            z, I = index_score(q, wl.q_dtype, w, wl.keys, wl.key_dtype, wl.k_scale, wl.seq_off, wl.H, wl.d)
+        else:
+            zs = [index_score(ql, wl.q_dtype, wl_, keys, wl.key_dtype, ks, wl.seq_off, wl.H, wl.d, want_I=False)
+                  for ql, wl_, (keys, ks) in self._per_layer(q, w)]
+            z = index_union(zs)[1]
+            I = 1.0 / (1.0 + np.exp(-z))   # the union's probability: that of its most confident layer
         kept_idx, kept_off, mask = select(z, wl.seq_off)
         self.kept_idx, self.kept_off = kept_idx, kept_off
         return z, I, mask
@@ -48,8 +67,9 @@ class OracleDecoder:
                 hot, slot_of = gather(wl.cold, wl.seq_off, self.kept_idx, self.kept_off)
                 res.update(hot=hot, slot_of=slot_of)
         else:
-            zk = index_score_list(q, wl.q_dtype, w, wl.keys, wl.key_dtype, wl.k_scale, wl.seq_off,
-                                  self.kept_idx, self.kept_off, wl.H, wl.d)
+            zks = [index_score_list(ql, wl.q_dtype, wl_, keys, wl.key_dtype, ks, wl.seq_off, self.kept_idx,
+                                    self.kept_off, wl.H, wl.d) for ql, wl_, (keys, ks) in self._per_layer(q, w)]
+            zk = zks[0] if len(zks) == 1 else index_union(zks)[1]
         tk, cnt = topk(zk, self.kept_idx, self.kept_off, wl.topk)
         out, lse = sparse_attn(Q, wl.attn_dtype, wl.cold, wl.attn_dtype, wl.row_stride, wl.k_off, wl.v_off,
                                local_to_global(tk, wl.seq_off), wl.scale)

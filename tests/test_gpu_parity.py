@@ -79,6 +79,39 @@ def test_index_score_listed_matches_oracle(lsa, name, tc):
     assert (z[n:] == 123.0).all()          # nothing written past the list
 
 
+def test_index_score_listed_e4m3_stage_reuse(lsa):
+    """Listed e4m3 scan with enough rows that every CTA reuses its stages (about 4 tiles of 256 rows per
+    CTA): 40K listed entries per sequence of the 500K-context workload.  The listed scores equal the full
+    scan's scores of the same entries (same arithmetic), a sample matches the oracle, and no bounded wait
+    gives up (a stage-free wait that misread a barrier two phases ahead used to time out here)."""
+    wl = synth.ctx500k(with_cold=False)
+    dev = synth.to_torch(wl, pin_cold=False)
+    z_full, _ = gpu_full_scores(wl, dev, lsa, want_I=False, tc=True)
+    rng = np.random.default_rng(9)
+    lists = [np.sort(rng.choice(int(n), size=40000, replace=False)) for n in np.diff(wl.seq_off)]
+    idx = np.concatenate(lists).astype(np.int32)
+    idx_off = np.concatenate([[0], np.cumsum([len(x) for x in lists])]).astype(np.int64)
+    cap = int(idx_off[-1])
+    z = torch.full((cap,), 123.0, dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        lsa.index_score(dev["q"], wl.q_dtype, dev["w"], dev["keys"], wl.key_dtype, dev["k_scale"], dev["seq_off"],
+                        wl.n_total, wl.H, wl.d, z, None, idx=torch.from_numpy(idx).cuda(),
+                        idx_off=torch.from_numpy(idx_off).cuda(), list_capacity=cap, err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    z = z.cpu().numpy()
+    b_of = np.repeat(np.arange(wl.B), np.diff(idx_off))
+    glob = wl.seq_off[:-1][b_of] + idx
+    assert np.abs(z - z_full[glob]).max() <= 1e-6 * max(1.0, np.abs(z_full).max())
+    pick = np.sort(rng.choice(cap, size=3000, replace=False))
+    sub = [idx[pick][b_of[pick] == b] for b in range(wl.B)]
+    sub_off = np.concatenate([[0], np.cumsum([len(x) for x in sub])]).astype(np.int64)
+    z_ref = oracle.index_score_list(wl.q, wl.q_dtype, wl.w, wl.keys, wl.key_dtype, wl.k_scale, wl.seq_off,
+                                    np.concatenate(sub).astype(np.int32), sub_off, wl.H, wl.d)
+    assert np.abs(z[pick] - z_ref).max() <= Z_TOL
+
+
 # --------------------------------------------------------------- select
 
 @pytest.mark.parametrize("name", ["tiny", "ragged_bf16", "ragged_e4m3"])
