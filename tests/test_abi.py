@@ -145,4 +145,16 @@ def test_ctx_create_rejects_bad_params(lsa):
     p.window = 16
     p.hca_rows = 1 << 20
     assert lsa.lib.lsa_ctx_create(ctypes.byref(p), ctypes.byref(h)) == 1   # HCA rows without offsets
+    p.hca_rows = None
+    p.window = 0
+    def rejected(why):
+        return lsa.lib.lsa_ctx_create(ctypes.byref(p), ctypes.byref(h)) == 1 and why in lsa.lib.lsa_last_error().decode()
+
+    p.n_layers = 9
+    assert rejected("n_layers=9")                    # more than 8 indexer layers
+    p.n_layers = 3
+    assert rejected("needs k_dev_layers")            # layers without their keys
+    arr = (ctypes.c_void_p * 2)(1 << 20, None)
+    p.k_dev_layers = ctypes.cast(arr, ctypes.c_void_p)
+    assert rejected("layer 2 has no keys")
     assert h.value is None
