@@ -380,7 +380,11 @@ lsa_status lsa_decode_step(lsa_ctx *ctx, int64_t t, const void *q, const float *
  * the step's values when the call is made (host program order) and stay
  * unchanged, like out_host and lse_host stay untouched, until `stream` has
  * completed this call's work; out_host and lse_host hold the results once
- * `stream` has completed. */
+ * `stream` has completed.  When out_host (and lse_host, if given) are
+ * page-locked host memory mapped for the device (cudaHostAlloc, or
+ * pinned tensors, on a UVA system), the step's attention writes them
+ * directly over the host link; other host memory goes through a device
+ * staging buffer and a copy. */
 lsa_status lsa_decode_step_host(lsa_ctx *ctx, int64_t t, const void *q_host, const float *w_host,
                                 const void *Q_host, void *out_host, float *lse_host, void *stream);
 

@@ -144,6 +144,16 @@ void free_all(lsa_ctx *c) {
 
 constexpr size_t kMaxGraphs = 256;
 
+// The device address of page-locked host memory mapped for the device, else nullptr.
+void *mapped_host(const void *p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
 cudaEvent_t take_event(lsa_ctx *c) {
     if (!c->free_events.empty()) {
         cudaEvent_t e = c->free_events.back();
@@ -538,11 +548,18 @@ lsa_status lsa_decode_step_host(lsa_ctx *c, int64_t t, const void *q_host, const
     LSA_CUDA(cudaMemcpyAsync(sg.Q, Q_host, Qbytes, cudaMemcpyHostToDevice, c->h2d));
     LSA_CUDA(cudaEventRecord(sg.in_ready, c->h2d));
     LSA_CUDA(cudaStreamWaitEvent(st, sg.in_ready, 0));
-    lsa_status s = run_step(c, t, sg.q, sg.w, sg.Q, sg.out, sg.lse, st);
+    // outputs in page-locked host memory mapped for the device: the attention writes them there
+    // directly (posted writes over the host link), with no staging buffer and no copy
+    void *out_map = mapped_host(out_host);
+    float *lse_map = lse_host ? static_cast<float *>(mapped_host(lse_host)) : nullptr;
+    const bool direct = out_map && aligned16(out_map) && (!lse_host || lse_map);
+    lsa_status s = direct ? run_step(c, t, sg.q, sg.w, sg.Q, out_map, lse_map, st)
+                          : run_step(c, t, sg.q, sg.w, sg.Q, sg.out, sg.lse, st);
     if (s != LSA_OK) return s;
     LSA_CUDA(cudaEventRecord(sg.used, st));
     ++c->host_calls;
-    // outputs: out on the caller's stream, lse beside it on the second copy
+    if (direct) return LSA_OK;
+    // otherwise out on the caller's stream, lse beside it on the second copy
     // stream; the caller's stream joins both before it completes
     LSA_CUDA(cudaMemcpyAsync(out_host, sg.out, Qbytes, cudaMemcpyDeviceToHost, st));
     if (lse_host) {
