@@ -453,6 +453,35 @@ def test_decoder_tau_cadence_and_kept_superset():
     assert "z" in r4                                       # refresh again at t = tau
 
 
+def test_layered_decoder_reduces_to_one_layer_and_keeps_the_or():
+    """Three copies of one indexer layer give exactly the one-layer decode (the union of equal scores is
+    that score); with three different layers every layer's own kept set lies inside the union's, and the
+    union's top-k ranks by the largest layer score."""
+    wl = synth.small_ragged(lengths=(300, 700), topk=64, Hq=4, D=64)
+    one = OracleDecoder(wl, tau=4)
+    three = OracleDecoder(wl, tau=4, layers=[(wl.keys, wl.k_scale)] * 2)
+    for t in (0, 1, 4):
+        q, w, Q = wl.step_inputs(t)
+        a = one.step(t, q, w, Q)
+        b = three.step(t, np.stack([q] * 3), np.stack([w] * 3), Q)
+        for key in ("kept_idx", "kept_off", "topk_idx", "topk_cnt", "out", "lse", "zk"):
+            assert np.array_equal(a[key], b[key]), (t, key)
+    others = [synth.small_ragged(seed=5 + 10 * l, lengths=(300, 700), topk=64, Hq=4, D=64) for l in (1, 2)]
+    mixed = OracleDecoder(wl, tau=4, layers=[(o.keys, o.k_scale) for o in others])
+    ins = [wl.step_inputs(0)] + [o.step_inputs(0) for o in others]
+    r = mixed.step(0, np.stack([i[0] for i in ins]), np.stack([i[1] for i in ins]), ins[0][2])
+    kept = set(zip(np.repeat(np.arange(wl.B), np.diff(r["kept_off"])).tolist(), r["kept_idx"].tolist()))
+    zs = []
+    for l, src in enumerate([wl] + others):
+        z_l = oracle.index_score(ins[l][0], wl.q_dtype, ins[l][1], src.keys, src.key_dtype, src.k_scale,
+                                 wl.seq_off, wl.H, wl.d, want_I=False)
+        zs.append(z_l)
+        idx, off, _ = oracle.select(z_l, wl.seq_off)
+        own = set(zip(np.repeat(np.arange(wl.B), np.diff(off)).tolist(), idx.tolist()))
+        assert own <= kept
+    assert np.array_equal(r["z"], np.max(np.stack(zs), axis=0))
+
+
 # ----------------------------------------------------- synthetic workloads
 
 def test_gate_calibration_reproduces_background_leakage():
