@@ -12,6 +12,16 @@
 // Other steps: listed re-score of the kept set with the step's indexer query
 // -> top-k -> attention.  The host never waits inside a step.
 //
+// Options.  Several indexer layers (section 2.4 "Optimal Configuration"): each
+// scan runs once per layer with that layer's keys and (q, w), and the union
+// score max_l z_l (union.cu) feeds select and the top-k.  Merged attention set
+// (section 2.1 "Architectural Design", HCA chunks retained; section 1, the
+// recent tokens): the window and HCA rows live after the hot buffer in one KV
+// arena, and a row-list merge (attn_set.cu) precedes the attention.
+// Host-buffer steps: inputs through two staging slots on a copy stream (a
+// call's copies overlap the previous call's kernels); outputs written straight
+// into mapped pinned host memory, else staged and copied.
+//
 // CUDA graphs: after one eager run of each step kind (refresh / listed), a
 // step is captured once per distinct set of input and output pointers and
 // replayed with one graph launch; a decode loop that reuses its buffers runs
