@@ -390,8 +390,9 @@ lsa_status lsa_decode_step_host(lsa_ctx *ctx, int64_t t, const void *q_host, con
 
 /* Device pointers of the context's internal results, for inspection. */
 typedef struct lsa_ctx_view {
-    float *z;            /* [n_total] full-scan scores of the last refresh */
-    float *z_kept;       /* [kept_capacity] listed-scan scores of the last step */
+    float *z;            /* [n_total] full-scan scores of the last refresh (the union score
+                            max_l z_l with n_layers >= 2) */
+    float *z_kept;       /* [kept_capacity] listed-scan scores of the last step (union likewise) */
     int32_t *kept_idx;   /* [kept_capacity] */
     int64_t *kept_off;   /* [B+1] */
     int32_t *slot_of;    /* [n_total] hot slot of each entry, or -1 */

@@ -433,6 +433,8 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     }
     c->p.k_dev_layers = nullptr;     // the caller's arrays are not kept
     c->p.k_scale_layers = nullptr;
+    c->p.hca_rows = nullptr;         // copied into the arena below
+    c->p.hca_off_host = nullptr;
     c->row_cap = row_cap;
     c->win_base = cap;
     c->hca_base = cap + int64_t(p.B) * p.window;
