@@ -142,8 +142,12 @@ lsa_status lsa_select(const float *z, const int64_t *seq_off, int64_t n_total, i
  * every GPU that loads it, held until the process exits), so n_total is
  * limited to lsa_select_noalloc_max_entries() (4,194,304); larger n_total is
  * rejected with LSA_ERR_INVALID before anything is launched.  The first call
- * on a device looks the array's device address up (cudaGetSymbolAddress) and
- * should come before any stream capture.  No call allocates or frees memory.
+ * on a device is its set-up: it looks the array's device address up
+ * (cudaGetSymbolAddress, cached per device and CUDA context) and, with lazy
+ * module loading (the CUDA 12 default), loads the library's device code, which
+ * creates the array in device memory.  Make that first call early: before any
+ * stream capture and before a runtime claims the rest of the device's memory.
+ * After it, no call allocates or frees memory (no cudaMalloc, no cudaFree).
  * All calls on a device share the array: calls that overlap on the GPU race.
  * ---------------------------------------------------------------------- */
 int64_t lsa_select_noalloc_max_entries(void);

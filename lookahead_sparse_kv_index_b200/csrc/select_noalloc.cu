@@ -12,11 +12,18 @@
 //
 // The array's name is only a host-side stand-in in host code; its device
 // address is looked up with cudaGetSymbolAddress on the first call made on
-// each device (with that device current) and cached.  That first call should
-// come before any stream capture.  Every call on a device shares the one
-// array, so calls that overlap on the GPU (different streams, no ordering
-// between them) race on it.  Nothing in it needs to start at zero: each call
-// writes every scratch word it reads before reading it.
+// each device (with that device current) and cached with the CUDA context it
+// belongs to: after a device reset the next call finds a new context and looks
+// the address up again.  With lazy module loading (the CUDA 12 default) that
+// first call also loads the library's device code, which creates the array in
+// device memory; so the first call on a device is the set-up call: make it
+// before any stream capture and before a runtime claims the rest of the
+// device's memory.  Every call on a device shares the one array, so calls that
+// overlap on the GPU (different streams, no ordering between them) race on it.
+// Nothing in it needs to start at zero: each call writes every scratch word it
+// reads before reading it.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "lsa_internal.cuh"
@@ -35,9 +42,32 @@ constexpr size_t kScratchBytes = align256(size_t((kNoallocMaxEntries + 1023) / 1
 __device__ __align__(256) uint8_t g_select_scratch[kScratchBytes];
 
 std::mutex g_mu;
-void *g_addr[64] = {nullptr};
+struct Cached {
+    CUcontext ctx;   // the context the address was looked up in
+    void *addr;
+};
+Cached g_addr[64] = {};
 
-// Device address of the scratch on the current device (looked up once per device).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+// The driver's cuCtxGetCurrent, through the runtime's entry-point query (the
+// library links no driver import library).
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// Device address of the scratch on the current device, looked up once per
+// device and context.
 lsa_status scratch_address(void **out) {
     int dev = 0;
     LSA_CUDA(cudaGetDevice(&dev));
@@ -46,12 +76,18 @@ lsa_status scratch_address(void **out) {
         return LSA_ERR_UNSUPPORTED;
     }
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev]) {
+    CtxGetCurrentFn get = ctx_get_current();
+    CUcontext ctx = nullptr;
+    if (get && get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+    // no context current yet on this thread (or no way to ask): the lookup itself makes the device's primary
+    // context current; the address is cached only together with a known context
+    if (ctx == nullptr || !g_addr[dev].addr || g_addr[dev].ctx != ctx) {
         void *p = nullptr;
         LSA_CUDA(cudaGetSymbolAddress(&p, g_select_scratch));
-        g_addr[dev] = p;
+        if (get && get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+        g_addr[dev] = {ctx, p};
     }
-    *out = g_addr[dev];
+    *out = g_addr[dev].addr;
     return LSA_OK;
 }
 
