@@ -57,7 +57,12 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", default="ctx500k", choices=sorted(WORKLOAD_DESC))
+    ap.add_argument("--config", default="ctx500k", choices=sorted(WORKLOAD_DESC) + ["sweep"],
+                    help="sweep: the indexer-only sweep (lsa_index_score + I >= 0.5 compaction over B x N x H x d x "
+                         "key dtype) and the 1-64 MB cold-pool fetch sweep; one JSON line per point")
+    ap.add_argument("--sweep-grid", default="full", choices=["full", "quick"],
+                    help="full: every point of the grid; quick: the B x N edges at H=64, d=128 and the H / d / dtype "
+                         "points at B=4, N=128K")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--hot-frac", type=float, default=0.2)
@@ -749,10 +754,139 @@ def run_only_merged(args):
     return 0 if all(e == 0 for r in res.values() for e in r["device_errors"]) else 1
 
 
+def sweep_points(grid):
+    import synth
+
+    pts = []
+    if grid == "full":
+        for B in synth.SWEEP_B:
+            for N in synth.SWEEP_N:
+                for H in synth.SWEEP_H:
+                    for d in synth.SWEEP_D:
+                        for dt in synth.SWEEP_DTYPES:
+                            pts.append((B, N, H, d, dt))
+    else:
+        for dt in synth.SWEEP_DTYPES:
+            for B, N in ((1, 8192), (1, 262144), (4, 131072), (32, 8192), (32, 262144)):
+                pts.append((B, N, 64, 128, dt))
+            for H in synth.SWEEP_H:
+                for d in synth.SWEEP_D:
+                    if (H, d) != (64, 128):
+                        pts.append((4, 131072, H, d, dt))
+    return pts
+
+
+def run_sweep(args):
+    """Indexer-only sweep: per grid point, lsa_index_score (full scan) followed by lsa_select (I >= 0.5
+    compaction), timed as back-to-back launches in one CUDA graph over enough key replicas that the rotation
+    exceeds twice the L2 (at most 128); then the cold-pool fetch sweep, 1-64 MB of 1 KB latent rows gathered
+    from page-locked host memory by lsa_gather, in 64-entry runs and as scattered rows, against the pinned
+    host-to-device copy rate of the same run.  One JSON line per point."""
+    import torch
+
+    import synth
+    from lookahead_sparse_kv_index_b200 import lsa
+
+    torch.cuda.set_device(0)
+    peak, peak_src = measured_peaks()
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    n_ok = 0
+    for (B, N, H, d, dt) in sweep_points(args.sweep_grid):
+        dv = synth.sweep_device(B, N, H, d, dt, synth.sweep_seed(B, N, H, d, dt))
+        n = dv["n_total"]
+        kb = 1 if dt == "e4m3" else 2
+        key_bytes = n * d * kb + (4 * n if dt == "e4m3" else 0)
+        reps = int(min(128, max(1, math.ceil(2 * l2 / key_bytes))))
+        keys = [dv["keys"]] + [dv["keys"].clone() for _ in range(reps - 1)]
+        scales = [dv["k_scale"]] + [dv["k_scale"].clone() if dv["k_scale"] is not None else None
+                                    for _ in range(reps - 1)]
+        z = torch.empty(n, dtype=torch.float32, device="cuda")
+        kept = torch.empty(n, dtype=torch.int32, device="cuda")
+        ko = torch.empty(B + 1, dtype=torch.int64, device="cuda")
+        ws = torch.empty(lsa.select_workspace_size(n), dtype=torch.uint8, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+        def scan(i):
+            lsa.index_score(dv["q"], "bf16", dv["w"], keys[i % reps], dt, scales[i % reps], dv["seq_off"], n, H, d,
+                            z, None, err=err)
+
+        def scan_select(i):
+            scan(i)
+            lsa.select(z, dv["seq_off"], n, kept, n, ko, None, ws, err)
+
+        n_launch = max(reps, 6)
+        scan(0)
+        kernel = lsa.last_kernel()
+        ms_scan = graph_launch_ms(scan, n_launch)
+        ms_both = graph_launch_ms(scan_select, n_launch)
+        torch.cuda.synchronize()
+        kept_n = int(ko[-1].item())
+        e = int(err.item())
+        scan_bytes = n * (d * kb + (4 if dt == "e4m3" else 0) + 4) + B * (H * d * 2 + H * 4)
+        both_bytes = scan_bytes + 4 * kept_n   # fused compaction: 4 B per kept entry out
+        gbs = both_bytes / (ms_both / 1e3) / 1e9
+        print(json.dumps({
+            "sweep": "index", "B": B, "N": N, "H": H, "d": d, "key_dtype": dt, "kernel": kernel,
+            "entries": n, "kept_fraction": kept_n / n, "replicas": reps, "l2_resident": reps * key_bytes < l2,
+            "ms_scan": ms_scan, "ms_scan_select": ms_both,
+            "scan_GBps": scan_bytes / (ms_scan / 1e3) / 1e9, "GBps": gbs,
+            "frac_of_measured": gbs / peak, "frac_of_nominal_8000": gbs / NOMINAL_HBM_GBS,
+            "algorithmic_bytes": both_bytes, "peak_source": peak_src, "device_error": e}), flush=True)
+        n_ok += e == 0
+        del keys, scales, dv, z, kept, ws
+        torch.cuda.empty_cache()
+
+    # cold-pool fetch sweep: rows of 1 KB (512 bf16 latent), a pool of 256K rows (256 MB page-locked)
+    row_bytes, n_pool = 1024, 1 << 18
+    g = torch.Generator().manual_seed(4)
+    cold = torch.randint(-32768, 32767, (n_pool, row_bytes // 2), generator=g, dtype=torch.int16).pin_memory()
+    hsrc = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    ddst = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ddst.copy_(hsrc, non_blocking=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        ddst.copy_(hsrc, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    h2d_gbs = 3 * (256 << 20) / (e0.elapsed_time(e1) / 1e3) / 1e9
+    del hsrc
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device="cuda")
+    seq_off = torch.tensor([0, n_pool], dtype=torch.int64, device="cuda")
+    for mb in (1, 2, 4, 8, 16, 32, 64):
+        for layout in ("runs", "scattered"):
+            rows = synth.sweep_fetch_rows(n_pool, mb * 1024, layout, seed=mb * 10 + (layout == "runs"))
+            kept_idx = torch.from_numpy(rows).cuda()
+            ko = torch.tensor([0, len(rows)], dtype=torch.int64, device="cuda")
+            hot = torch.empty((len(rows), row_bytes), dtype=torch.uint8, device="cuda")
+            err = torch.zeros(1, dtype=torch.int32, device="cuda")
+            times = []
+            for it in range(6):
+                flush.zero_()   # nothing of the pool or the hot rows left in L2
+                e0.record()
+                lsa.gather(cold, row_bytes, seq_off, n_pool, kept_idx, ko, hot, len(rows), None, err)
+                e1.record()
+                torch.cuda.synchronize()
+                if it:
+                    times.append(e0.elapsed_time(e1))
+            ms = float(np.median(times))
+            nbytes = len(rows) * row_bytes
+            ok = bool(torch.equal(hot[:: max(1, len(rows) // 64)].cpu(),
+                                  cold.view(torch.uint8)[torch.from_numpy(rows[:: max(1, len(rows) // 64)]).long()]))
+            print(json.dumps({"sweep": "fetch", "MB": mb, "layout": layout, "rows": len(rows), "ms": ms,
+                              "GBps": nbytes / (ms / 1e3) / 1e9, "pinned_h2d_copy_GBps": h2d_gbs,
+                              "frac_of_pinned_copy": nbytes / (ms / 1e3) / 1e9 / h2d_gbs,
+                              "path": "zero-copy reads of page-locked host rows by the gather kernel",
+                              "sampled_rows_equal": ok, "device_error": int(err.item())}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.config == "sweep":
+        return run_sweep(args)
     if args.only == "scan":
         return run_only_scan(args)
     if args.only == "union":

@@ -72,6 +72,12 @@ const char *lsa_last_error(void);
 /* Static name of a status code. */
 const char *lsa_status_name(lsa_status s);
 
+/* Name of the last kernel this host thread launched through the library ("" if
+ * none), e.g. "scan_tc e4m3 d64" for the tensor-core index scan of e4m3 keys
+ * with d = 64: lets a caller or a test see which implementation ran.  A static
+ * string; it needs no GPU to call. */
+const char *lsa_last_kernel(void);
+
 /* ------------------------------------------------------------------------
  * lsa_index_score -- the lookahead index score (section 2.1, "Scoring
  * Mechanism"; the interaction is a plain dot product, section 5).
@@ -93,10 +99,11 @@ const char *lsa_status_name(lsa_status s);
  * Full mode (idx == NULL): z / I are written for every entry, [n_total].
  * z        fp32 output (required).   I  fp32 output or NULL.
  * flags    0, or LSA_SCORE_CUDA_CORE.  Scans (full or listed) of bf16 q (16-byte
- *          aligned) over bf16 keys (d 64 or 128) or e4m3 keys (d 128) with H in
- *          {16, 32, 64}, B <= 512 and n_total >= 128 run on the tensor cores
- *          (tcgen05); every other case, and every call with
- *          LSA_SCORE_CUDA_CORE, runs the CUDA-core kernel.
+ *          aligned) over bf16 or e4m3 keys with d in {64, 128} and H in
+ *          {16, 32, 64}, B <= 512 and n_total >= 128 (bf16) or >= 256 (e4m3)
+ *          run on the tensor cores (tcgen05); every other case, and every call
+ *          with LSA_SCORE_CUDA_CORE, runs the CUDA-core kernel
+ *          (lsa_last_kernel names the one that ran).
  * err      device error word or NULL (LSA_ERR_TIMEOUT if a bounded wait of the
  *          tensor-core kernel gave up).
  * Shapes run: 1 <= H <= 64, d in {32, 64, 128} (d * element size % 16 == 0).

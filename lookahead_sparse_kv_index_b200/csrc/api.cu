@@ -12,6 +12,7 @@ namespace lsa {
 
 static thread_local char g_msg[512] = "";
 static thread_local int64_t g_launches = 0;
+static thread_local const char *g_last_kernel = "";
 
 void set_error(const char *fmt, ...) {
     va_list ap;
@@ -20,7 +21,10 @@ void set_error(const char *fmt, ...) {
     va_end(ap);
 }
 void clear_error() { g_msg[0] = 0; }
-void count_launch() { ++g_launches; }
+void count_launch(const char *name) {
+    ++g_launches;
+    g_last_kernel = name;
+}
 int64_t launch_count() { return g_launches; }
 
 int sm_count() {
@@ -62,6 +66,8 @@ int64_t lsa_struct_size(int32_t which) {
 }
 
 const char *lsa_last_error(void) { return lsa::g_msg; }
+
+const char *lsa_last_kernel(void) { return lsa::g_last_kernel; }
 
 const char *lsa_status_name(lsa_status s) {
     switch (s) {

@@ -5,26 +5,29 @@
 //
 // Shape run here: 128 query heads over one latent KV head of dim 512 (the same
 // bf16 row serves as K and V).  One CTA per (sequence, chunk of 128 selected
-// rows):
-//   1. warps 0-3 gather the chunk's 128 rows (1 KB each, arbitrary hot-buffer
-//      rows) with cp.async straight into the 128-byte-swizzled K-major layout
-//      the tensor core reads (8 column blocks of 64 elements), block by block,
-//      each block signalled as soon as it lands so that the S MMAs of block 0
-//      start while the others are still in flight; padding rows are
-//      zero-filled;
-//   2. warp 5 streams Q[b] (128 x 512 bf16) by TMA in 8 slices of 64 columns
-//      through a 5-stage ring (P later reuses its memory);
-//   3. warp 4 issues S = Q K^T (M = 128 heads, N = 128 rows, K = 512) into
-//      TMEM columns 0..127;
-//   4. warps 0-3 (one head per thread) read S, compute the chunk's row max m,
-//      p = exp(scale*s - m), l = sum p, and write P as bf16 in the K-major
-//      swizzled layout;
-//   5. warp 4 issues O = P V (M = 128, N = 2 x 256, K = 128) into TMEM columns
-//      0..511, reading the SAME smem rows as V through an MN-major descriptor
-//      (no transpose, no second copy of the rows);
-//   6. warps 0-3 read O in 64-column blocks into the freed row buffer
-//      (128-byte swizzle, one staging buffer per block) and write the
-//      partial in bf16 with TMA stores; (m, l) per head in fp32.
+// rows), ten warps:
+//   * warp 9 (loads): streams Q[b] (128 x 512 bf16) by TMA in 8 slices of 64
+//     columns through a 5-stage ring, the first five before the dependency on
+//     the preceding kernel is resolved; reads the chunk's row indices;
+//   * warps 0-7 first gather the chunk's rows (1 KB each, arbitrary hot-buffer
+//     rows) with cp.async straight into the 128-byte-swizzled K-major layout
+//     the tensor core reads, 8 column blocks of 64 elements, each signalled on
+//     its own barrier as soon as it lands so that the S MMAs of block 0 start
+//     while the others are in flight; padding rows are zero-filled.  (A TMA
+//     row gather, tile::gather4, moved the same rows at about a third of this
+//     rate: its instructions are serialised through the SM's one TMA unit.);
+//   * warp 8 (MMA): S = Q K^T (M = 128 heads, N = 128 rows, K = 512) into TMEM
+//     columns 0..127; then O = P V (M = 128, N = 2 x 256, K = 128) into TMEM
+//     columns 0..511, reading the SAME shared rows as V through an MN-major
+//     descriptor (no transpose, no second copy);
+//   * warps 0-7 (then softmax, epilogue): warp w owns TMEM lanes 32 (w % 4) ..
+//     (heads) and the 64 chunk rows 64 (w / 4) ..; S stays in registers from
+//     the row max to the weights; the two warps of a head meet in shared
+//     memory for its max and sum; P goes to shared memory as bf16 in the
+//     K-major layout (one 64-row block per warp half, over the Q ring); after
+//     O, each half converts 256 output columns to bf16 in 64-column blocks
+//     staged in the freed row buffer and writes them with TMA stores; (m, l)
+//     per head in fp32.
 // The combine kernel (attn.cu) merges the chunks.  Every wait is bounded.
 #include <cuda.h>
 
@@ -40,7 +43,10 @@ constexpr int kHq = 128;
 constexpr int kD = 512;
 constexpr int kRowsPerCta = 128;
 constexpr int kQStages = 5;   // 5 x 16 KB of Q in flight; P reuses this ring once S is done
-constexpr int kThreads = 192;
+constexpr int kSoftWarps = 8;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr int kThreads = 32 * (kSoftWarps + 2);
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kTmemCols = 512;
 
@@ -50,14 +56,21 @@ constexpr int kQStageBytes = kHq * 128;          // 16 KB: one 64-column slice o
 constexpr int kPBytes = kHq * kRowsPerCta * 2;   // 32 KB: 2 blocks of [128 heads x 128 B]
 constexpr int kOStageBytes = kHq * 64 * 2;       // 16 KB: [128 heads][64 bf16] staging of one O block
 static_assert((kD / 64) * kOStageBytes <= kKvBytes, "every O block has its own staging buffer in the row buffer");
+static_assert(kQStages * kQStageBytes >= kPBytes, "P lives in the Q ring");
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// Arrive on `bar` once every cp.async this thread has issued so far has landed (counted in the barrier's
+// expected arrivals).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// 2^x (the hardware approximation, as the fast exponential uses).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
@@ -75,8 +88,8 @@ __device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t addr, uint32_t lbo) {
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap omap,
-        const uint16_t *__restrict__ kv, int64_t stride, int64_t k_off, const int32_t *__restrict__ rows, int k,
-        float scale, float *__restrict__ part_ml, int32_t *err) {
+        const uint16_t *__restrict__ kv, int64_t stride, const int32_t *__restrict__ rows, int k, float scale,
+        float *__restrict__ part_ml, int32_t *err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *kvs = smem;                         // 128 KB
@@ -84,7 +97,6 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
     // P (32 KB) overwrites the Q ring: it is written only after every S MMA has completed, and by then
     // every Q load has landed (each was waited for by an S MMA)
     uint8_t *ps = qs;
-    static_assert(kQStages * kQStageBytes >= kPBytes, "P lives in the Q ring");
     uint64_t *qfull = reinterpret_cast<uint64_t *>(qs + kQStages * kQStageBytes);
     uint64_t *qempty = qfull + kQStages;
     uint64_t *kv_full = qempty + kQStages;       // [kD / 64] column blocks of the rows
@@ -93,9 +105,12 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
     uint64_t *o_full = p_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_full + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
-    int *s_rows = abort_flag + 1;                // [128]
-    int *s_nvalid = s_rows + kRowsPerCta;
+    int *s_nvalid = abort_flag + 1;
     uint32_t *s_valid = reinterpret_cast<uint32_t *>(s_nvalid + 1);   // [4] bit j % 32 of word j / 32: row j selected
+    float *s_max = reinterpret_cast<float *>(s_valid + 4);             // [128 heads][2 halves]
+    float *s_sum = s_max + 2 * kHq;                                    // [128 heads][2 halves]
+    // [128] the chunk's rows (-1: padding), written as int4: 16-byte aligned
+    int *s_rows = reinterpret_cast<int *>((reinterpret_cast<uintptr_t>(s_sum + 2 * kHq) + 15) & ~uintptr_t(15));
 
     const int chunk = blockIdx.x, b = blockIdx.y, nchunks = gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -105,36 +120,55 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
     pdl_launch_dependents();
     if (threadIdx.x == 0) {
         *abort_flag = 0;
-        *s_nvalid = 0;
         for (int s = 0; s < kQStages; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 1); }
-        for (int kb = 0; kb < kD / 64; ++kb) mbar_init(&kv_full[kb], 128);
+        for (int kb = 0; kb < kD / 64; ++kb) mbar_init(&kv_full[kb], 32 * kSoftWarps);
         mbar_init(s_full, 1);
-        mbar_init(p_full, 128);
+        mbar_init(p_full, kSoftWarps);
         mbar_init(o_full, 1);
         fence_mbar_init();
     }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
     __syncthreads();
-    if (warp == 5 && lane == 0) {
+    if (warp == kLoadWarp && lane == 0) {
         // Q does not depend on the preceding kernel: start streaming it now
         prefetch_tmap(&qmap);
-        for (int kd = 0; kd < kQStages; ++kd) {
+            for (int kd = 0; kd < kQStages; ++kd) {
             mbar_arrive_expect_tx(&qfull[kd], kQStageBytes);
             tma_load_2d(qs + kd * kQStageBytes, &qmap, &qfull[kd], kd * 64, b * kHq);
         }
     }
     pdl_wait();   // the selected rows (and the hot buffer) come from preceding kernels
-    if (threadIdx.x < kRowsPerCta) {
-        const int i = chunk * kRowsPerCta + threadIdx.x;
-        const int r = i < k ? rows[int64_t(b) * k + i] : -1;
-        s_rows[threadIdx.x] = r;
-        if (r >= 0) atomicAdd(s_nvalid, 1);
-        const uint32_t bal = __ballot_sync(0xffffffffu, r >= 0);   // threads 0..127: whole warps
-        if ((threadIdx.x & 31) == 0) s_valid[threadIdx.x >> 5] = bal;
-    }
-    if (warp == 4) {
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
-        tc_fence_before();
+    if (warp == kLoadWarp) {
+        // lane l owns chunk rows 4l .. 4l+3
+        int r[4];
+        uint32_t nib = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = chunk * kRowsPerCta + 4 * lane + j;
+            r[j] = i < k ? rows[int64_t(b) * k + i] : -1;
+            if (r[j] < 0) r[j] = -1;   // any negative index is padding
+            nib |= uint32_t(r[j] >= 0) << j;
+        }
+        const int nvalid = __reduce_add_sync(0xffffffffu, __popc(nib));
+        // word w of the row mask = rows 32w .. 32w+31 = the nibbles of lanes 8w .. 8w+7
+        uint32_t words[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) word |= __shfl_sync(0xffffffffu, nib, 8 * w + j) << (4 * j);
+            words[w] = word;
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) s_valid[w] = words[w];
+            *s_nvalid = nvalid;
+        }
+        *reinterpret_cast<int4 *>(s_rows + 4 * lane) = make_int4(r[0], r[1], r[2], r[3]);
     }
     __syncthreads();
     tc_fence_after();
@@ -147,109 +181,105 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
             part_ml[(pbase + threadIdx.x) * 2] = -INFINITY;
             part_ml[(pbase + threadIdx.x) * 2 + 1] = 0.f;
         }
-        if (warp == 5 && lane == 0)   // let the early Q loads land before the CTA exits
+        if (warp == kLoadWarp && lane == 0)   // let the early Q loads land before the CTA exits
             for (int kd = 0; kd < kQStages; ++kd) mbar_wait(&qfull[kd], 0, abort_v, kWaitLimitNs);
-    } else if (warp < 4) {
-        const int t = threadIdx.x;   // 0..127
-        // ---- 1. gather the chunk's rows: 8 column blocks of 128 rows x 8 sixteen-byte chunks, one
-        // cp.async group per block (8 consecutive threads read one row's 128 contiguous bytes)
-        const uint32_t kv_u32 = smem_u32(kvs);
+    } else if (warp < kSoftWarps) {
+        // ---- the row gather: thread t copies 16-byte chunk t % 8 of each 128-byte piece of rows
+        // t / 8 + 32 j (j < 4), column block by column block; a column block is signalled once every
+        // thread's copies into it have landed (cp.async-tracked arrivals)
+        {
+            const int t = threadIdx.x, c = t & 7;
+            const uint32_t kv_u32 = smem_u32(kvs);
+            const uint16_t *src[4];
+            uint32_t nbytes[4], dst[4];
 #pragma unroll
-        for (int kb = 0; kb < kD / 64; ++kb) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = t + 128 * u;
-                const int r = i >> 3, c = kb * 8 + (i & 7);
-                const int row = s_rows[r];
-                const uint32_t dst = kv_u32 + kb * kKvBlock + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-                const uint16_t *src = kv + (row >= 0 ? int64_t(row) * stride + k_off + c * 8 : 0);
-                cp_async_16(dst, src, row >= 0 ? 16u : 0u);
+            for (int j = 0; j < 4; ++j) {
+                const int rr = (t >> 3) + 32 * j;
+                const int row = s_rows[rr];
+                src[j] = kv + (row >= 0 ? int64_t(row) * stride : 0) + c * 8;
+                nbytes[j] = row >= 0 ? 16u : 0u;
+                dst[j] = kv_u32 + rr * 128 + ((c ^ (rr & 7)) << 4);
             }
-            cp_async_commit();
+#pragma unroll
+            for (int kb = 0; kb < kD / 64; ++kb) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) cp_async_16(dst[j] + kb * kKvBlock, src[j] + kb * 64, nbytes[j]);
+                cp_async_arrive_noinc(&kv_full[kb]);
+            }
         }
-        // block kb has landed once at most 7 - kb younger groups are pending
-        cp_async_wait_group<7>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[0]);
-        cp_async_wait_group<6>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[1]);
-        cp_async_wait_group<5>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[2]);
-        cp_async_wait_group<4>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[3]);
-        cp_async_wait_group<3>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[4]);
-        cp_async_wait_group<2>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[5]);
-        cp_async_wait_group<1>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[6]);
-        cp_async_wait_group<0>(); fence_proxy_async_smem(); mbar_arrive(&kv_full[7]);
-
-        // ---- 4. softmax of the chunk: thread t owns head t (TMEM lane t)
-        const int quarter = warp;   // warps 0-3 -> TMEM lanes 32*warp ..
+        // ---- softmax: thread (quarter, lane) owns head 32 * quarter + lane (its TMEM lane) and chunk rows
+        // 64 * half .. 64 * half + 63 (TMEM columns)
+        const int quarter = warp & 3, half = warp >> 2;
+        const int head = 32 * quarter + lane;
+        const uint32_t taddr = tmem + (uint32_t(quarter * 32) << 16);
         bool ok = mbar_wait(s_full, 0, abort_v, kWaitLimitNs);
         float m = -INFINITY, l = 0.f;
-        // warps 0-3 take every branch below together (they meet at named barriers)
-        if (named_barrier_and(1, 128, ok)) {
+        // the softmax warps take every branch below together (they meet at named barriers)
+        if (named_barrier_and(1, 32 * kSoftWarps, ok)) {
             tc_fence_after();
-            const uint32_t taddr = tmem + (uint32_t(quarter * 32) << 16);
-            // S is read from TMEM 32 columns at a time, in two passes (row max, then weights): rolled
-            // loops keep this phase's code and registers small.  Selected rows come from a bit mask; a
-            // full chunk (the common case) skips the tests.  Max and sum run as four chains.
-            const bool all_valid = (s_valid[0] & s_valid[1] & s_valid[2] & s_valid[3]) == 0xffffffffu;
+            uint32_t sv[64];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tmem_ld_32x32b_x16(taddr + half * 64 + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[c * 16]));
+            tmem_ld_wait();
+            const uint32_t v0 = s_valid[2 * half], v1 = s_valid[2 * half + 1];
+            const bool all_valid = (v0 & v1) == 0xffffffffu;
             float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-            for (int c = 0; c < kRowsPerCta / 32; ++c) {
-                uint32_t r32[32];
-                tmem_ld_32x32b_x16(taddr + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&r32[0]));
-                tmem_ld_32x32b_x16(taddr + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r32[16]));
-                tmem_ld_wait();
-                const uint32_t vb = all_valid ? 0xffffffffu : s_valid[c];
 #pragma unroll
-                for (int u = 0; u < 32; ++u)
-                    if ((vb >> u) & 1u) mq[u & 3] = fmaxf(mq[u & 3], scale * __uint_as_float(r32[u]));
+            for (int u = 0; u < 64; ++u) {
+                const bool valid = all_valid || (((u < 32 ? v0 : v1) >> (u & 31)) & 1u);
+                if (valid) mq[u & 3] = fmaxf(mq[u & 3], scale * __uint_as_float(sv[u]));
             }
-            m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+            s_max[2 * head + half] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+            named_barrier(1, 32 * kSoftWarps);
+            m = fmaxf(s_max[2 * head], s_max[2 * head + 1]);   // a head with a valid row has m > -inf
+            // exp(scale s - m) = 2^(scale log2(e) s - m log2(e)): one FFMA and one ex2 per weight
+            const float c1 = scale * 1.4426950408889634f, c0 = -m * 1.4426950408889634f;
+            // P in bf16, K-major swizzled: block `half` (rows 64 half ..), row `head`, 16-byte chunk c
             float lq[4] = {0.f, 0.f, 0.f, 0.f};
-            // P in bf16, K-major swizzled: block (j / 64), row t, 16-byte chunk (j % 64) / 8
-            const uint32_t p_u32 = smem_u32(ps);
-#pragma unroll 1
-            for (int c = 0; c < kRowsPerCta / 32; ++c) {
-                uint32_t r32[32];
-                tmem_ld_32x32b_x16(taddr + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&r32[0]));
-                tmem_ld_32x32b_x16(taddr + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r32[16]));
-                tmem_ld_wait();
-                const uint32_t vb = all_valid ? 0xffffffffu : s_valid[c];
-                uint32_t packed[16];
+            const uint32_t p_u32 = smem_u32(ps) + half * (kHq * 128) + head * 128;
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int j0 = 2 * u, j1 = j0 + 1;
-                    const float p0 = ((vb >> j0) & 1u) ? __expf(scale * __uint_as_float(r32[j0]) - m) : 0.f;
-                    const float p1 = ((vb >> j1) & 1u) ? __expf(scale * __uint_as_float(r32[j1]) - m) : 0.f;
+            for (int c = 0; c < 8; ++c) {
+                uint32_t packed[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j0 = 8 * c + 2 * e, j1 = j0 + 1;
+                    const uint32_t vb = c < 4 ? v0 : v1;
+                    const bool ok0 = all_valid || ((vb >> (j0 & 31)) & 1u);
+                    const bool ok1 = all_valid || ((vb >> (j1 & 31)) & 1u);
+                    const float p0 = ok0 ? ex2_approx(fmaf(c1, __uint_as_float(sv[j0]), c0)) : 0.f;
+                    const float p1 = ok1 ? ex2_approx(fmaf(c1, __uint_as_float(sv[j1]), c0)) : 0.f;
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                     // the normaliser sums the bf16-rounded weights the MMA actually uses
                     const float2 back = __bfloat1622float2(h2);
-                    lq[u & 3] += back.x + back.y;
-                    packed[u] = *reinterpret_cast<const uint32_t *>(&h2);
+                    lq[e] += back.x + back.y;
+                    packed[e] = *reinterpret_cast<const uint32_t *>(&h2);
                 }
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int cc = 4 * c + h;   // 16-byte chunk of the row (8 weights)
-                    const uint32_t dst = p_u32 + (cc >> 3) * (kHq * 128) + t * 128 + (((cc & 7) ^ (t & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(packed[4 * h]),
-                                 "r"(packed[4 * h + 1]), "r"(packed[4 * h + 2]), "r"(packed[4 * h + 3])
-                                 : "memory");
-                }
+                const uint32_t dst = p_u32 + ((c ^ (head & 7)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(packed[0]), "r"(packed[1]),
+                             "r"(packed[2]), "r"(packed[3])
+                             : "memory");
             }
-            l = (lq[0] + lq[1]) + (lq[2] + lq[3]);
+            s_sum[2 * head + half] = (lq[0] + lq[1]) + (lq[2] + lq[3]);
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(p_full);
-            // ---- 6. read O and write the chunk's partial (bf16): 64-column blocks staged in the (now
-            // free) row buffer, each in its own 16 KB buffer, one TMA store per block
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+            // ---- O: each half converts its 256 columns, 64-column blocks staged in the (now free) row
+            // buffer, each in its own 16 KB buffer, one TMA store per block
             ok = mbar_wait(o_full, 0, abort_v, kWaitLimitNs);
-            // the block loop below synchronises these 128 threads: agree on one outcome first
-            if (named_barrier_and(1, 128, ok)) {
+            // the block loop below synchronises these 256 threads: agree on one outcome first
+            if (named_barrier_and(1, 32 * kSoftWarps, ok)) {
                 tc_fence_after();
+                l = s_sum[2 * head] + s_sum[2 * head + 1];
 #pragma unroll 1
-                for (int c = 0; c < kD / 64; ++c) {
-                    uint8_t *sb = kvs + c * kOStageBytes;   // [128 rows x 128 B]
+                for (int c = 0; c < 4; ++c) {
+                    const int cb = 4 * half + c;                   // output column block
+                    uint8_t *sb = kvs + cb * kOStageBytes;        // [128 rows x 128 B]
                     uint32_t o[64];
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
-                        tmem_ld_32x32b_x16(taddr + c * 64 + q4 * 16, *reinterpret_cast<uint32_t(*)[16]>(&o[q4 * 16]));
+                        tmem_ld_32x32b_x16(taddr + cb * 64 + q4 * 16, *reinterpret_cast<uint32_t(*)[16]>(&o[q4 * 16]));
                     tmem_ld_wait();
                     // [128 rows x 64 bf16] in the 128-byte-swizzled layout (16-byte chunk u of row t at
                     // chunk u ^ (t % 8)): conflict-free writes
@@ -262,69 +292,72 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
                                                                             __uint_as_float(o[8 * u + 2 * e + 1]));
                             w4[e] = *reinterpret_cast<const uint32_t *>(&h2);
                         }
-                        const uint32_t dst = smem_u32(sb) + t * 128 + ((u ^ (t & 7)) << 4);
+                        const uint32_t dst = smem_u32(sb) + head * 128 + ((u ^ (head & 7)) << 4);
                         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w4[0]), "r"(w4[1]),
                                      "r"(w4[2]), "r"(w4[3])
                                      : "memory");
                     }
                     fence_proxy_async_smem();
-                    named_barrier(1, 128);
-                    if (t == 0) {
-                        tma_store_2d(&omap, sb, c * 64, int(pbase));
+                    named_barrier(2 + half, 128);   // the four warps of this half
+                    if (quarter == 0 && lane == 0) {
+                        tma_store_2d(&omap, sb, cb * 64, int(pbase));
                         bulk_commit();
                     }
                 }
-                if (t == 0) bulk_wait_all();
-                part_ml[(pbase + t) * 2] = m;
-                part_ml[(pbase + t) * 2 + 1] = l;
+                if (quarter == 0 && lane == 0) bulk_wait_all();
+                if (half == 0) {
+                    part_ml[(pbase + head) * 2] = m;
+                    part_ml[(pbase + head) * 2 + 1] = l;
+                }
             }
         }
-    } else if (warp == 4) {
-        // ---- 3./5. MMA issuer
+    } else if (warp == kMmaWarp) {
+        // ---- MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(128, 128);
             constexpr uint32_t IDESC_O = idesc_bf16(128, 256) | (1u << 16);   // B (V) is MN-major
-            bool issued = false;
-            {
-                const uint32_t kv_u32 = smem_u32(kvs);
-                int st = 0;
-                uint32_t ph = 0;
-                bool ok = true;
-                for (int kd = 0; kd < kD / 64 && ok; ++kd) {
-                    ok = mbar_wait(&kv_full[kd], 0, abort_v, kWaitLimitNs) &&
-                         mbar_wait(&qfull[st], ph, abort_v, kWaitLimitNs);
-                    if (!ok) break;
+            const uint32_t kv_u32 = smem_u32(kvs);
+            int st = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int kd = 0; kd < kD / 64 && ok; ++kd) {
+                ok = mbar_wait(&kv_full[kd], 0, abort_v, kWaitLimitNs) &&
+                     mbar_wait(&qfull[st], ph, abort_v, kWaitLimitNs);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t q_u32 = smem_u32(qs + st * kQStageBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16(tmem, desc_sw128(q_u32 + kk * 32), desc_sw128(kv_u32 + kd * kKvBlock + kk * 32), IDESC_S,
+                            (kd | kk) != 0);
+                mma_commit(&qempty[st]);
+                if (++st == kQStages) { st = 0; ph ^= 1; }
+            }
+            if (ok) {
+                mma_commit(s_full);
+                if (mbar_wait(p_full, 0, abort_v, kWaitLimitNs)) {
                     tc_fence_after();
-                    const uint32_t q_u32 = smem_u32(qs + st * kQStageBytes);
+                    const uint32_t p_u32 = smem_u32(ps);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f16(tmem, desc_sw128(q_u32 + kk * 32), desc_sw128(kv_u32 + kd * kKvBlock + kk * 32),
-                                IDESC_S, (kd | kk) != 0);
-                    issued = true;
-                    mma_commit(&qempty[st]);
-                    if (++st == kQStages) { st = 0; ph ^= 1; }
-                }
-                if (ok) {
-                    mma_commit(s_full);
-                    if (mbar_wait(p_full, 0, abort_v, kWaitLimitNs)) {
-                        tc_fence_after();
-                        const uint32_t p_u32 = smem_u32(ps);
+                    for (int half = 0; half < 2; ++half)
 #pragma unroll
-                        for (int half = 0; half < 2; ++half)
-#pragma unroll
-                            for (int kk = 0; kk < kRowsPerCta / 16; ++kk)
-                                mma_f16(tmem + half * 256,
-                                        desc_sw128(p_u32 + (kk >> 2) * (kHq * 128) + (kk & 3) * 32),
-                                        desc_sw128_mn(kv_u32 + half * 4 * kKvBlock + kk * 2048, kKvBlock),
-                                        IDESC_O, kk != 0);
-                        mma_commit(o_full);
-                    }
+                        for (int kk = 0; kk < kRowsPerCta / 16; ++kk)
+                            mma_f16(tmem + half * 256, desc_sw128(p_u32 + (kk >> 2) * (kHq * 128) + (kk & 3) * 32),
+                                    desc_sw128_mn(kv_u32 + half * 4 * kKvBlock + kk * 2048, kKvBlock), IDESC_O,
+                                    kk != 0);
+                    mma_commit(o_full);
                 }
             }
-            (void)issued;
+            if (!ok) {
+                // let the row gathers land before the CTA exits
+                for (int kb = 0; kb < kD / 64; ++kb) {
+                    volatile int no_abort = 0;
+                    mbar_wait(&kv_full[kb], 0, &no_abort, kWaitLimitNs);
+                }
+            }
         }
     } else {
-        // ---- 2. Q producer (the first kQStages slices were issued before the dependency wait)
+        // ---- Q producer (the first kQStages slices were issued before the dependency wait)
         if (lane == 0) {
             int st = 0;
             uint32_t ph = 1;
@@ -338,7 +371,7 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
     }
     __syncwarp();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -364,7 +397,7 @@ EncodeTiledFn encode_fn() {
 }
 
 constexpr size_t kSmemBytes = 1024 + size_t(kKvBytes) + size_t(kQStages) * kQStageBytes +
-                              (2 * kQStages + kD / 64 + 3) * 8 + 16 + (kRowsPerCta + 2) * 4 + 16 + 64;
+                              (2 * kQStages + kD / 64 + 3) * 8 + 16 + 16 + 4 * kHq * 4 + 16 + kRowsPerCta * 4 + 64;
 
 }  // namespace
 
@@ -382,11 +415,11 @@ lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, 
         set_error("lsa_sparse_attn: cuTensorMapEncodeTiled is unavailable");
         return LSA_ERR_CUDA;
     }
+    const cuuint32_t estr[2] = {1, 1};
     CUtensorMap qmap;
     const cuuint64_t dims[2] = {cuuint64_t(kD), cuuint64_t(B) * kHq};
     const cuuint64_t strides[1] = {cuuint64_t(kD) * 2};
     const cuuint32_t box[2] = {64, 128};
-    const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(Q), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -395,8 +428,8 @@ lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, 
         return LSA_ERR_CUDA;
     }
     CUtensorMap omap;   // partial O [B * nchunks * 128 rows, 512] bf16, stored in swizzled [128 x 64] boxes
-    const int nchunks_o = (k + kRowsPerCta - 1) / kRowsPerCta;
-    const cuuint64_t odims[2] = {cuuint64_t(kD), cuuint64_t(B) * nchunks_o * kHq};
+    const int nchunks = (k + kRowsPerCta - 1) / kRowsPerCta;
+    const cuuint64_t odims[2] = {cuuint64_t(kD), cuuint64_t(B) * nchunks * kHq};
     const cuuint64_t ostrides[1] = {cuuint64_t(kD) * 2};
     const cuuint32_t obox[2] = {64, 128};
     r = enc(&omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, part_o, odims, ostrides, obox, estr,
@@ -407,9 +440,8 @@ lsa_status launch_sparse_attn_tc(const void *Q, const void *kv, int64_t stride, 
         return LSA_ERR_CUDA;
     }
     LSA_CUDA(ensure_smem(attn_tc, size_t(int(kSmemBytes))));
-    const int nchunks = (k + kRowsPerCta - 1) / kRowsPerCta;
     LSA_CUDA(launch_pdl(attn_tc, dim3(nchunks, B), dim3(kThreads), kSmemBytes, st, qmap, omap,
-                        static_cast<const uint16_t *>(kv), stride, k_off, rows, k, scale, part_ml, err));
+                        static_cast<const uint16_t *>(kv) + k_off, stride, rows, k, scale, part_ml, err));
     LSA_LAUNCHED("attn_tc");
     return LSA_OK;
 }

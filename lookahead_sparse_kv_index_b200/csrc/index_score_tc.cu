@@ -52,7 +52,9 @@ namespace {
 
 using namespace ptx;
 
-enum Kind { BF16_D128 = 0, BF16_D64 = 1, E4M3_D128 = 2 };
+enum Kind { BF16_D128 = 0, BF16_D64 = 1, E4M3_D128 = 2, E4M3_D64 = 3 };
+
+__host__ __device__ constexpr bool is_e4m3(int kind) { return kind == E4M3_D128 || kind == E4M3_D64; }
 
 template <int KIND>
 struct Cfg;
@@ -89,6 +91,38 @@ struct Cfg<E4M3_D128> {
     static constexpr int kQBytesPerHead = 256;  // two e4m3 pieces x 128
     static constexpr int kStages = 4;           // at most twice the tile accumulators (2)
 };
+// e4m3 keys with d = 64: 64-byte rows in the 64-byte-swizzled K-major layout (the
+// 128-byte swizzle needs 128-byte rows); 256-row tiles of 16 KB, each sub-tile
+// two K = 32 MMAs, so again 8 MMAs per 32 KB of keys; twice the stages of the
+// d = 128 ring for the same bytes in flight.
+template <>
+struct Cfg<E4M3_D64> {
+    static constexpr int kSub = 2;
+    static constexpr int kStageBytes = 16384;   // 256 rows x 64 e4m3
+    static constexpr int kBoxes = 1;
+    static constexpr int kBoxRows = 256;
+    static constexpr int kPieces = 2;
+    static constexpr int kQBytesPerHead = 128;  // two e4m3 pieces x 64
+    static constexpr int kStages = 8;           // a multiple of the tile accumulators (2, 4 or 8)
+};
+
+// Key row bytes, and where 16-byte chunk c of row r of a stage sits: the TMA
+// writes a stage in this layout and the MMA descriptors read it.  128-byte rows
+// use the 128-byte swizzle (bf16 d = 128 keys are two such column boxes, 16 KB
+// apart); 64-byte rows the 64-byte swizzle.
+template <int KIND>
+__host__ __device__ constexpr int row_bytes() {
+    return KIND == BF16_D128 ? 256 : KIND == E4M3_D64 ? 64 : 128;
+}
+template <int KIND>
+__device__ __forceinline__ uint32_t stage_chunk_off(int r, int c) {
+    if (KIND == E4M3_D64) return uint32_t(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+    return uint32_t((c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+template <int KIND>
+__device__ __forceinline__ uint64_t kdesc(uint32_t addr) {
+    return KIND == E4M3_D64 ? desc_sw64(addr) : desc_sw128(addr);
+}
 
 constexpr int kThreads = 320;         // warp 0 producer, warp 1 MMA, warps 2-9 epilogue (2 warpgroups)
 constexpr int kEpiGroups = 2;
@@ -189,7 +223,7 @@ __device__ __forceinline__ int frexp_exponent(float m) {
 template <int KIND, int H>
 __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, const float *__restrict__ wb, int d,
                                             uint8_t *slot, float *wsm, int wi, int nw, int lane) {
-    if (KIND != E4M3_D128) {
+    if (!is_e4m3(KIND)) {
         // 16-byte chunks, all of a thread's loads in flight before its stores
         const int cpr = d / 8;
         const int tid = wi * 32 + lane, nthr = nw * 32;
@@ -218,12 +252,17 @@ __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, con
         }
         for (int j = wi * 32 + lane; j < H; j += nw * 32) wsm[j] = wb[j];
     } else {
-        // eight threads per head, thread g of a head owns channels 16g .. 16g+15 (one 16-byte chunk of
-        // each piece): the head's max is a 3-step shuffle and each thread converts 16 channels
+        // d / 16 threads per head (8 for d = 128, 4 for d = 64), thread g of a head owns channels
+        // 16g .. 16g+15 (one 16-byte chunk of each piece): the head's max is a 3- or 2-step shuffle and
+        // each thread converts 16 channels
+        constexpr int DK = KIND == E4M3_D64 ? 64 : 128;
+        constexpr int TPH = DK / 16;   // threads per head
+        constexpr int LOG_TPH = TPH == 8 ? 3 : 2;
         const int tid = wi * 32 + lane, nthr = nw * 32;
-        const int g = tid & 7;
-        for (int j = tid >> 3; j < H; j += nthr >> 3) {   // every lane of a warp takes the same trip count
-            const uint4 *src = reinterpret_cast<const uint4 *>(qb + j * 128 + 16 * g);
+        const int g = tid & (TPH - 1);
+        // every lane of a warp takes the same trip count (32 / TPH heads per warp, H a multiple of 16)
+        for (int j = tid >> LOG_TPH; j < H; j += nthr >> LOG_TPH) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(qb + j * DK + 16 * g);
             const uint4 ra = src[0], rb = src[1];
             const float wj = wb[j];
             const uint32_t wds[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
@@ -237,7 +276,7 @@ __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, con
 #pragma unroll
             for (int c = 0; c < 16; ++c) m = fmaxf(m, fabsf(v[c]));
 #pragma unroll
-            for (int o = 4; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            for (int o = TPH / 2; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             const int e = m > 0.f ? 8 - frexp_exponent(m) : 0;   // m 2^e in [128, 256)
             uint32_t p1w[4] = {0u, 0u, 0u, 0u}, p2w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
@@ -250,9 +289,11 @@ __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, con
                 p1w[c >> 2] |= uint32_t(p1) << (8 * (c & 3));
                 p2w[c >> 2] |= uint32_t(p2) << (8 * (c & 3));
             }
-            const int off = j * 128 + ((g ^ (j & 7)) << 4);
+            // the query operand in the keys' layout: row j (piece 1) and row H + j (piece 2); H is a
+            // multiple of 8, so both rows have the same swizzle phase
+            const int off = DK == 128 ? j * 128 + ((g ^ (j & 7)) << 4) : j * 64 + ((g ^ ((j >> 1) & 3)) << 4);
             *reinterpret_cast<uint4 *>(slot + off) = make_uint4(p1w[0], p1w[1], p1w[2], p1w[3]);
-            *reinterpret_cast<uint4 *>(slot + H * 128 + off) = make_uint4(p2w[0], p2w[1], p2w[2], p2w[3]);
+            *reinterpret_cast<uint4 *>(slot + H * DK + off) = make_uint4(p2w[0], p2w[1], p2w[2], p2w[3]);
             if (g == 0) wsm[j] = ldexpf(wj, -e);
         }
     }
@@ -307,7 +348,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     // loads would otherwise also wait for that HBM load.  Slot j % RS holds tile j's scales; it is
     // rewritten for tile j + RS only after the MMA of tile j + KACC, i.e. after the epilogue of tile
     // j released its accumulator, which it does after reading the scales.
-    constexpr bool kScales = KIND == E4M3_D128;
+    constexpr bool kScales = is_e4m3(KIND);
     constexpr int RS = S + KACC;
     static_assert(!kScales || RS <= kScaleSlotsMax, "row-scale ring");
 
@@ -501,7 +542,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             // all 32 lanes gather: lane owns rows lane, lane + 32, ... of each tile; a stage (and its row
             // scales) is signalled by cp.async-tracked arrivals, one per lane
             pdl_wait();
-            constexpr int RB = KIND == E4M3_D128 ? 128 : (KIND == BF16_D128 ? 256 : 128);   // row bytes
+            constexpr int RB = row_bytes<KIND>();
             constexpr int CPR = RB / 16;
             int b = 0, cur = -1, qn = 0, st = 0;
             uint32_t ph = 0;
@@ -525,8 +566,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                     const uint8_t *src = kbytes + e * RB;
 #pragma unroll
                     for (int c = 0; c < CPR; ++c)
-                        cp_async_16(stage_u32 + (c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4),
-                                    src + c * 16, valid ? 16u : 0u);
+                        cp_async_16(stage_u32 + stage_chunk_off<KIND>(r, c), src + c * 16, valid ? 16u : 0u);
                     if (kScales)
                         cp_async_4(smem_u32(s_scale + int((t - t0) % RS) * TR + r), k_scale + e, valid ? 4u : 0u);
                 }
@@ -541,11 +581,11 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC = KIND == E4M3_D128 ? idesc_e4m3(kRows, SUBC) : idesc_bf16(kRows, SUBC);
+            constexpr uint32_t IDESC = is_e4m3(KIND) ? idesc_e4m3(kRows, SUBC) : idesc_bf16(kRows, SUBC);
             // descriptors of stage 0 and slot 0; the others differ only in the start address field
             // (16-byte units), advanced incrementally: this thread's per-tile work is the tensor pipe's idle time
-            const uint64_t a_desc0 = desc_sw128(smem_u32(stages));
-            const uint64_t b_desc0 = desc_sw128(smem_u32(qimg));
+            const uint64_t a_desc0 = kdesc<KIND>(smem_u32(stages));
+            const uint64_t b_desc0 = kdesc<KIND>(smem_u32(qimg));
             constexpr uint64_t kStageStep = uint64_t(C::kStageBytes >> 4);
             int b = 0, qn = -1, st = 0, acc = 0;
             uint32_t ph = 0, aph = 0;
@@ -599,6 +639,14 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                             if (u < gn)
                                 mma_f16(d_t[u], a_d[u] + uint64_t((kk * 32) >> 4), b_cur + uint64_t((kk * 32) >> 4),
                                         IDESC, kk > 0);
+                } else if (KIND == E4M3_D64) {
+                    // as below, with 64-byte rows: the halves are 8 KB apart, two K = 32 steps
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+                        for (int sub = 0; sub < 2; ++sub)
+                            mma_f8(d_t[0] + uint32_t(sub * SUBC), a_d[0] + uint64_t((sub * 8192 + kk * 32) >> 4),
+                                   b_cur + uint64_t((kk * 32) >> 4), IDESC, kk > 0);
                 } else {
                     // the two 128-row halves of the tile (16 KB apart in the stage) into their own
                     // column blocks, chains interleaved; N = 2H covers both query pieces
@@ -730,7 +778,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             }
             float zs = (za + zb) + (zc + zd);
             if (row < row_end) {
-                if (KIND == E4M3_D128) zs *= sc;
+                if (kScales) zs *= sc;
                 z[row] = zs;
                 if (I) I[row] = 1.f / (1.f + expf(-zs));
             }
@@ -771,7 +819,7 @@ size_t smem_bytes(int B) {
     using C = Cfg<KIND>;
     return 1024 + size_t(C::kStages) * C::kStageBytes + 2 * qimg_bytes<KIND, H>() +
            (C::kStages + 2 + kRel + 2 * kAccMax + 1 + kScaleSlotsMax) * 8 + 16 + 16 + 2 * H * 4 +
-           size_t(B + 1) * 24 + 16 + (KIND == E4M3_D128 ? size_t(C::kStages + acc_tiles<KIND, H>()) * tile_rows<KIND>() * 4 : 0) +
+           size_t(B + 1) * 24 + 16 + (is_e4m3(KIND) ? size_t(C::kStages + acc_tiles<KIND, H>()) * tile_rows<KIND>() * 4 : 0) +
            64;
 }
 
@@ -785,15 +833,16 @@ lsa_status launch(const void *q, const float *w, const void *k, const float *k_s
         return LSA_ERR_CUDA;
     }
     CUtensorMap map;
-    const bool fp8 = KIND == E4M3_D128;
+    const bool fp8 = is_e4m3(KIND);
     const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(n_total)};
     const cuuint64_t strides[1] = {cuuint64_t(d) * (fp8 ? 1 : 2)};
-    const cuuint32_t box[2] = {cuuint32_t(fp8 ? 128 : 64), cuuint32_t(Cfg<KIND>::kBoxRows)};
+    // box: one 128-byte column block (64 bytes for e4m3 d = 64) x kBoxRows rows
+    const cuuint32_t box[2] = {cuuint32_t(fp8 ? d : 64), cuuint32_t(Cfg<KIND>::kBoxRows)};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                      const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     KIND == E4M3_D64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         set_error("lsa_index_score: cuTensorMapEncodeTiled failed (%d)", int(r));
         return LSA_ERR_CUDA;
@@ -807,7 +856,10 @@ lsa_status launch(const void *q, const float *w, const void *k, const float *k_s
     LSA_CUDA(launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, map, static_cast<const uint8_t *>(k),
                         static_cast<const uint16_t *>(q), w, d, seq_off, idx, idx_off, list_cap, B, k_scale, z, I,
                         err));
-    LSA_LAUNCHED(idx ? "scan_tc_listed" : "scan_tc");
+    static const char *kNames[2][4] = {
+        {"scan_tc bf16 d128", "scan_tc bf16 d64", "scan_tc e4m3 d128", "scan_tc e4m3 d64"},
+        {"scan_tc_listed bf16 d128", "scan_tc_listed bf16 d64", "scan_tc_listed e4m3 d128", "scan_tc_listed e4m3 d64"}};
+    LSA_LAUNCHED(kNames[idx ? 1 : 0][KIND]);
     return LSA_OK;
 }
 
@@ -830,8 +882,7 @@ bool index_score_tc_supported(lsa_dtype q_dtype, lsa_dtype k_dtype, int64_t n_to
     if (q_dtype != LSA_BF16 || B > kMaxB) return false;
     if (n_total < (k_dtype == LSA_E4M3 ? tile_rows<E4M3_D128>() : kRows)) return false;
     if (!(H == 16 || H == 32 || H == 64)) return false;
-    if (k_dtype == LSA_BF16) return d == 128 || d == 64;
-    if (k_dtype == LSA_E4M3) return d == 128;
+    if (k_dtype == LSA_BF16 || k_dtype == LSA_E4M3) return d == 128 || d == 64;
     return false;
 }
 
@@ -839,9 +890,12 @@ lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, l
                                  const float *k_scale, const int64_t *seq_off, int64_t n_total,
                                  const int32_t *idx, const int64_t *idx_off, int64_t list_cap, int32_t B,
                                  int32_t H, int32_t d, float *z, float *I, int32_t *err, cudaStream_t st) {
-    if (k_dtype == LSA_E4M3)
+    if (k_dtype == LSA_E4M3 && d == 128)
         return launch_h<E4M3_D128>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err,
                                    st);
+    if (k_dtype == LSA_E4M3)
+        return launch_h<E4M3_D64>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err,
+                                  st);
     if (d == 128)
         return launch_h<BF16_D128>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err,
                                    st);

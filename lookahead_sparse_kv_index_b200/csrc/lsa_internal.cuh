@@ -54,11 +54,12 @@ void clear_error();
             ::lsa::set_error("launch of %s failed: %s", name, cudaGetErrorString(e_)); \
             return LSA_ERR_CUDA;                                                       \
         }                                                                              \
-        ::lsa::count_launch();                                                         \
+        ::lsa::count_launch(name);                                                     \
     } while (0)
 
-// Per-thread kernel launch counter (read by the decode context).
-void count_launch();
+// Per-thread kernel launch counter (read by the decode context) and the name of
+// the last kernel launched (lsa_last_kernel).  `name` must be a static string.
+void count_launch(const char *name);
 int64_t launch_count();
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

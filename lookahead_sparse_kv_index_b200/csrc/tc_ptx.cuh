@@ -90,6 +90,20 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// Row gather by TMA: four rows y0..y3 of a 2-D tensor map whose box is one
+// row high, each `box[0]` elements from column x, land as four consecutive box
+// rows at dst (the map's swizzle applied as for a tiled load); completion
+// counted on `bar`.  A row outside the map reads the fill value (zeros).
+__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y0, int y1,
+                                            int y2, int y3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
+          "r"(y2), "r"(y3)
+        : "memory");
+}
+
 // Contiguous bulk copy global -> shared (16-byte aligned, size % 16 == 0).
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile(
@@ -214,6 +228,21 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
     d |= uint64_t(1024 >> 4) << 32;                // stride byte offset: 8 rows x 128 B
     d |= uint64_t(1) << 46;                        // descriptor version for tcgen05
     d |= uint64_t(2) << 61;                        // swizzle mode: 128 B
+    return d;
+}
+
+// Shared-memory matrix descriptor, K-major operand with the 64-byte swizzle:
+// rows of 64 bytes, 8-row atoms of 512 bytes stacked with a 512-byte stride;
+// 16-byte chunk c of row r sits at chunk c ^ ((r / 2) % 4) (the swizzle acts on
+// the absolute shared-memory address, so atoms must be 512-byte aligned).
+// `addr` may be advanced by 32 bytes inside an atom row to select a K slice.
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t addr) {
+    uint64_t d = 0;
+    d |= uint64_t((addr >> 4) & 0x3FFFu);         // start address >> 4
+    d |= uint64_t(1) << 16;                        // leading byte offset (unused for this layout)
+    d |= uint64_t(512 >> 4) << 32;                 // stride byte offset: 8 rows x 64 B
+    d |= uint64_t(1) << 46;                        // descriptor version for tcgen05
+    d |= uint64_t(4) << 61;                        // swizzle mode: 64 B
     return d;
 }
 

@@ -31,7 +31,7 @@ N_STAGES = 6
 
 # every symbol include/lsa.h declares
 EXPORTS = [
-    "lsa_version", "lsa_last_error", "lsa_status_name", "lsa_index_score",
+    "lsa_version", "lsa_last_error", "lsa_last_kernel", "lsa_status_name", "lsa_index_score",
     "lsa_select_workspace_size", "lsa_select_noalloc_max_entries", "lsa_select_noalloc",
     "lsa_select", "lsa_topk", "lsa_gather", "lsa_sparse_attn_workspace_size", "lsa_sparse_attn",
     "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
@@ -74,6 +74,7 @@ def _sig(name, res, args):
 _sig("lsa_version", i32, [])
 _sig("lsa_struct_size", i64, [i32])
 _sig("lsa_last_error", ctypes.c_char_p, [])
+_sig("lsa_last_kernel", ctypes.c_char_p, [])
 _sig("lsa_status_name", ctypes.c_char_p, [i32])
 _sig("lsa_index_score", i32, [P, i32, P, P, i32, P, P, i64, P, P, i64, i32, i32, i32, P, P, i32, P, P])
 SCORE_CUDA_CORE = 1
@@ -124,6 +125,11 @@ def _check(status, where):
 
 def version() -> int:
     return int(_L.lsa_version())
+
+
+def last_kernel() -> str:
+    """Name of the last kernel this thread launched through the library."""
+    return _L.lsa_last_kernel().decode()
 
 
 # ------------------------------------------------------------------ stages

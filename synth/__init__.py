@@ -264,6 +264,87 @@ def small_ragged(seed: int = 5, key_dtype: str = "bf16", lengths=(1000, 4133, 25
                    topk=topk, Hq=Hq, D=D)
 
 
+# Indexer-only sweep (B in 1..32, N in 8K..256K entries per sequence, H in {16, 32, 64}, d in {64, 128},
+# bf16 or e4m3 keys): 12.5% of the entries in planted chunks plus the ~1% background leakage the gates are
+# calibrated for, i.e. about 13.5% kept, the pages' average KV footprint.
+SWEEP_PLANTED = 0.125
+SWEEP_B = (1, 2, 4, 8, 16, 32)
+SWEEP_N = (8192, 16384, 32768, 65536, 131072, 262144)
+SWEEP_H = (16, 32, 64)
+SWEEP_D = (64, 128)
+SWEEP_DTYPES = ("bf16", "e4m3")
+
+
+def sweep_seed(B: int, N: int, H: int, d: int, key_dtype: str) -> int:
+    """The sweep's seed stream (4 + point number) of one grid point."""
+    i = ((((SWEEP_B.index(B) * len(SWEEP_N) + SWEEP_N.index(N)) * len(SWEEP_H) + SWEEP_H.index(H)) * len(SWEEP_D)
+          + SWEEP_D.index(d)) * len(SWEEP_DTYPES) + SWEEP_DTYPES.index(key_dtype))
+    return 4 + i
+
+
+def sweep(B: int, N: int, H: int, d: int, key_dtype: str, seed: int | None = None, with_cold: bool = False,
+          **kw) -> Workload:
+    """One point of the indexer-only sweep, generated on the CPU (for parity tests): B sequences of N
+    entries, 12.5% planted chunks."""
+    if seed is None:
+        seed = sweep_seed(B, N, H, d, key_dtype) if B in SWEEP_B and N in SWEEP_N else 4
+    return planted(f"sweep_B{B}_N{N}_H{H}_d{d}_{key_dtype}", seed, [N] * B, H, d, key_dtype,
+                   [SWEEP_PLANTED] * B, with_cold=with_cold, **kw)
+
+
+def sweep_device(B: int, N: int, H: int, d: int, key_dtype: str, seed: int, device: str = "cuda") -> dict:
+    """The same planted-chunk recipe as `planted`, drawn directly on `device` with a seeded device generator
+    (a different random stream from the CPU generator's, same distributions and structure): indexer keys,
+    row scales (e4m3), queries, gates and CSR offsets as device tensors, for timing sweeps whose hundreds of
+    points would take minutes to draw on the host.  Pure data generation, like the rest of this module."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    n = B * N
+    k = torch.randn(n, d, generator=g, device=device) / math.sqrt(d)
+    u = torch.randn(B, d, generator=g, device=device, dtype=torch.float64)
+    u = (u / u.norm(dim=1, keepdim=True)).to(torch.float32)
+    n_chunks = (N + CHUNK - 1) // CHUNK
+    n_plant = int(round(SWEEP_PLANTED * n_chunks))
+    for b in range(B):
+        chosen = torch.randperm(n_chunks, generator=g, device=device)[:n_plant]
+        rows = (chosen[:, None] * CHUNK + torch.arange(CHUNK, device=device)[None, :]).flatten()
+        rows = rows[rows < N] + b * N
+        m = rows.numel()
+        norms = (torch.randn(m, d, generator=g, device=device) / math.sqrt(d)).norm(dim=1, keepdim=True)
+        v = torch.randn(m, d, generator=g, device=device)
+        v = v - (v @ u[b])[:, None] * u[b][None, :]
+        v = v / v.norm(dim=1, keepdim=True)
+        k[rows] = norms * (0.6 * u[b][None, :] + 0.8 * v)
+    r = torch.randn(B, H, d, generator=g, device=device) / math.sqrt(d)
+    r[:, : H // 2] += u[:, None, :]
+    w = torch.from_numpy(np.tile(gate_weights(H, GATE_GAMMA[(H, d)]), (B, 1))).to(device)
+    if key_dtype == "e4m3":
+        amax = k.abs().amax(dim=1)
+        scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+        keys = (k / scale[:, None]).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+        k_scale = scale.contiguous()
+    else:
+        keys = k.to(torch.bfloat16).view(torch.int16)
+        k_scale = None
+    del k
+    seq_off = torch.arange(B + 1, dtype=torch.int64, device=device) * N
+    return dict(keys=keys.contiguous(), k_scale=k_scale, q=r.to(torch.bfloat16).view(torch.int16).contiguous(),
+                w=w.contiguous(), seq_off=seq_off, n_total=n, B=B, N=N, H=H, d=d, key_dtype=key_dtype)
+
+
+def sweep_fetch_rows(n_pool: int, n_rows: int, layout: str, seed: int) -> np.ndarray:
+    """Sorted entry indices of n_rows selected rows out of a pool of n_pool: `runs` takes whole contiguous
+    64-entry chunks (the pages' critical chunks), `scattered` single rows uniformly at random."""
+    g = torch.Generator().manual_seed(seed)
+    if layout == "runs":
+        n_chunks = n_pool // CHUNK
+        take = (n_rows + CHUNK - 1) // CHUNK
+        chosen = torch.randperm(n_chunks, generator=g)[:take]
+        rows = (chosen[:, None] * CHUNK + torch.arange(CHUNK)[None, :]).flatten()[:n_rows]
+    else:
+        rows = torch.randperm(n_pool, generator=g)[:n_rows]
+    return np.sort(rows.numpy()).astype(np.int32)
+
+
 WORKLOADS = {
     "tiny": tiny,
     "ctx128k": ctx128k,

@@ -44,6 +44,10 @@ def test_index_score_full_matches_oracle(lsa, name, tc):
     wl = SCORE_CASES[name]()
     dev = synth.to_torch(wl, pin_cold=False)
     z, I = gpu_full_scores(wl, dev, lsa, tc=tc)
+    if tc and wl.q_dtype == "bf16":   # every bf16-query case here has a shape the tensor cores run
+        assert lsa.last_kernel() == f"scan_tc {wl.key_dtype} d{wl.d}"
+    elif not tc:
+        assert lsa.last_kernel() == "score_cuda_core"
     z_ref, I_ref = oracle.index_score(wl.q, wl.q_dtype, wl.w, wl.keys, wl.key_dtype, wl.k_scale, wl.seq_off,
                                       wl.H, wl.d)
     assert np.abs(z - z_ref).max() <= Z_TOL
@@ -330,6 +334,16 @@ ATTN_CASES = [
 
 @pytest.mark.parametrize("case", ATTN_CASES, ids=lambda c: f"{c[0]}-B{c[1]}-H{c[2]}-D{c[3]}-k{c[4]}")
 def test_sparse_attn_matches_oracle(lsa, case):
+    _attn_case(lsa, case)
+
+
+def test_sparse_attn_padding_holes(lsa):
+    """Padding entries (-1, and any other negative index) scattered through the row lists, so that chunks
+    start with padding, hold a single selected row, or none: the tensor-core path against the oracle."""
+    _attn_case(lsa, ("bf16", 3, 128, 512, 640, 5000, False), holes=True)
+
+
+def _attn_case(lsa, case, holes=False):
     dt, B, Hq, D, k, n_rows, separate = case
     g = torch.Generator().manual_seed(11)
     stride = 2 * D if separate else D
@@ -342,6 +356,13 @@ def test_sparse_attn_matches_oracle(lsa, case):
     for b in range(B):
         c = min(counts[b], n_rows)
         rows[b, :c] = np.sort(rng.choice(n_rows, size=c, replace=False))
+    if holes:
+        rows[0, rng.random(k) < 0.4] = -1        # sequence 0: 40% holes anywhere
+        rows[0, :5] = -1                          # chunk 0 starts with padding
+        rows[0, 128:256] = -1                     # chunk 1: a single selected row
+        rows[0, 200] = 17
+        rows[0, 256:384] = -1                     # chunk 2: nothing selected
+        rows[1, 1::2] = -3                        # sequence 1: every other entry another negative value
     out = torch.empty((B, Hq, D), dtype=torch.float32 if dt == "f32" else torch.int16, device="cuda")
     lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
     ws = torch.empty(lsa.sparse_attn_workspace_size(B, Hq, D, k), dtype=torch.uint8, device="cuda")
@@ -350,6 +371,8 @@ def test_sparse_attn_matches_oracle(lsa, case):
     lsa.sparse_attn(synth.raw_to_torch(Q), dt, synth.raw_to_torch(kv), stride, 0, v_off,
                     torch.from_numpy(rows).cuda(), B, Hq, D, k, scale, out, lse, ws)
     torch.cuda.synchronize()
+    assert lsa.last_kernel().startswith("attn_combine")
+    rows = np.where(rows < 0, -1, rows)   # every negative index is padding
     out_ref, lse_ref = oracle.sparse_attn(Q, dt, kv, dt, stride, 0, v_off, rows.astype(np.int64), scale)
     o = out.cpu().numpy()
     o = oracle.decode(o.view(np.uint16), "bf16") if dt == "bf16" else o.astype(np.float64)
