@@ -84,6 +84,12 @@ struct lsa_ctx {
     const float *ks_layer[lsa::kMaxUnionLayers] = {};
     float *z_layers = nullptr;    // [n_layers, n_total] full-scan scores (n_layers >= 2)
     float *zk_layers = nullptr;   // [n_layers, kept_capacity] listed scores (n_layers >= 2)
+    // compacted kept keys (and e4m3 row scales) per layer, in kept-list order, written at each refresh; the
+    // listed re-score streams them with the full tensor-core scan (when the shape runs on the tensor cores)
+    bool compact = false;
+    void *kc[lsa::kMaxUnionLayers] = {};
+    float *sc[lsa::kMaxUnionLayers] = {};
+    int64_t sc_len = 0;
     // merged attention set: window and HCA rows live in the arena after the hot buffer
     bool merged = false;
     int64_t win_base = 0, hca_base = 0, row_cap = 0;
@@ -133,6 +139,10 @@ void free_all(lsa_ctx *c) {
                     c->zk_layers};
     for (void *b : bufs)
         if (b) cudaFree(b);
+    for (int l = 0; l < lsa::kMaxUnionLayers; ++l) {
+        if (c->kc[l]) cudaFree(c->kc[l]);
+        if (c->sc[l]) cudaFree(c->sc[l]);
+    }
     for (auto &sg : c->stage) {
         for (void *b : {sg.q, sg.Q, sg.out, static_cast<void *>(sg.w), static_cast<void *>(sg.lse)})
             if (b) cudaFree(b);
@@ -250,6 +260,11 @@ lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w,
                                  c->slot_of, c->owner, c->kept_slot, c->fetched, c->fetch_ws, c->err, c->ev_assign,
                                  c->side));
         }
+        if (c->compact)
+            for (int l = 0; l < c->n_layers; ++l)
+                LSA_TRY(launch_gather_keys(c->k_layer[l], int64_t(p.d) * int64_t(elem_size(p.k_dtype)), c->ks_layer[l],
+                                           c->seq_off_d, c->kept_idx, c->kept_off, p.B, cap, c->kc[l], c->sc[l],
+                                           c->side));
         tg.done();
         LSA_CUDA(cudaEventRecord(c->ev_gather, c->side));
         // the top-k writes hot slots: with the cache it needs the slot assignment first
@@ -261,7 +276,19 @@ lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w,
         LSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
     } else {
         StageTimer tr(c, LSA_STAGE_RESCORE, st);
-        if (c->n_layers == 1) {
+        const bool compact = c->compact && aligned16(q);   // the tensor-core scan reads q with 16-byte loads
+        if (compact) {
+            // the kept keys in kept-list order: z lands at the kept position
+            const float *zl[kMaxUnionLayers];
+            for (int l = 0; l < c->n_layers; ++l) {
+                float *z_l = c->n_layers == 1 ? c->z_kept : c->zk_layers + size_t(l) * cap;
+                LSA_TRY(launch_index_score_tc_axis(static_cast<const char *>(q) + l * q_layer, w + l * w_layer,
+                                                   c->kc[l], p.k_dtype, c->sc[l], c->sc_len, c->kept_off, cap, cap,
+                                                   p.B, p.H, p.d, z_l, c->err, st));
+                zl[l] = z_l;
+            }
+            if (c->n_layers > 1) LSA_TRY(launch_union(zl, c->n_layers, cap, c->z_kept, st));
+        } else if (c->n_layers == 1) {
             LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
                                        p.n_total, c->kept_idx, c->kept_off, cap, p.B, p.H, p.d, c->z_kept,
                                        nullptr, 0, c->err, st));
@@ -456,6 +483,14 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
         LSA_ALLOC(c->hca_off_d, size_t(p.B + 1) * 8);
         LSA_ALLOC(c->attn_rows, size_t(p.B) * row_cap * 4);
     }
+    // the compacted kept keys, when the listed re-score runs on the tensor cores
+    c->compact = index_score_tc_supported(p.q_dtype, p.k_dtype, cap, p.B, p.H, p.d);
+    c->sc_len = int64_t(align_up(size_t(cap), 4)) + 8;
+    if (c->compact)
+        for (int l = 0; l < n_layers; ++l) {
+            LSA_ALLOC(c->kc[l], size_t(cap) * p.d * elem_size(p.k_dtype));
+            if (p.k_dtype == LSA_E4M3) LSA_ALLOC(c->sc[l], size_t(c->sc_len) * 4);
+        }
     LSA_ALLOC(c->topk_idx, size_t(p.B) * p.topk * 4);
     LSA_ALLOC(c->topk_pos, size_t(p.B) * p.topk * 4);
     LSA_ALLOC(c->topk_cnt, size_t(p.B) * 4);
@@ -500,6 +535,10 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
         if (ce == cudaSuccess) ce = cudaMemset(c->slot_of, 0xFF, size_t(p.n_total > 0 ? p.n_total : 1) * 4);
         if (ce == cudaSuccess) ce = cudaMemset(c->owner, 0xFF, size_t(cap) * 4);
         if (ce == cudaSuccess) ce = cudaMemset(c->fetched, 0, 16);
+        for (int l = 0; l < n_layers && c->compact; ++l) {
+            if (ce == cudaSuccess) ce = cudaMemset(c->kc[l], 0, size_t(cap) * p.d * elem_size(p.k_dtype));
+            if (ce == cudaSuccess && c->sc[l]) ce = cudaMemset(c->sc[l], 0, size_t(c->sc_len) * 4);
+        }
         if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking);
         if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking);
         if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_sel, cudaEventDisableTiming);

@@ -254,49 +254,77 @@ __device__ __forceinline__ void build_query(const uint16_t *__restrict__ qb, con
     } else {
         // d / 16 threads per head (8 for d = 128, 4 for d = 64), thread g of a head owns channels
         // 16g .. 16g+15 (one 16-byte chunk of each piece): the head's max is a 3- or 2-step shuffle and
-        // each thread converts 16 channels
+        // each thread converts 16 channels.  Two heads per thread per iteration, both heads' loads issued
+        // before any arithmetic (one global round trip for the 8-warp build of 64 heads)
         constexpr int DK = KIND == E4M3_D64 ? 64 : 128;
         constexpr int TPH = DK / 16;   // threads per head
         constexpr int LOG_TPH = TPH == 8 ? 3 : 2;
         const int tid = wi * 32 + lane, nthr = nw * 32;
         const int g = tid & (TPH - 1);
+        const int hstride = nthr >> LOG_TPH;   // heads per round
         // every lane of a warp takes the same trip count (32 / TPH heads per warp, H a multiple of 16)
-        for (int j = tid >> LOG_TPH; j < H; j += nthr >> LOG_TPH) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(qb + j * DK + 16 * g);
-            const uint4 ra = src[0], rb = src[1];
-            const float wj = wb[j];
-            const uint32_t wds[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-            float v[16];
+        for (int j0 = tid >> LOG_TPH; j0 < H; j0 += 2 * hstride) {
+            uint4 ra[2], rb[2];
+            float wj[2];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                v[2 * c] = __uint_as_float(wds[c] << 16);
-                v[2 * c + 1] = __uint_as_float(wds[c] & 0xFFFF0000u);
+            for (int h = 0; h < 2; ++h) {
+                const int j = j0 + h * hstride;
+                if (j < H) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(qb + j * DK + 16 * g);
+                    ra[h] = src[0];
+                    rb[h] = src[1];
+                    wj[h] = wb[j];
+                } else {
+                    ra[h] = rb[h] = make_uint4(0u, 0u, 0u, 0u);
+                    wj[h] = 0.f;
+                }
             }
-            float m = 0.f;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) m = fmaxf(m, fabsf(v[c]));
+            for (int h = 0; h < 2; ++h) {
+                const int j = j0 + h * hstride;   // uniform across the TPH threads of a head
+                const uint32_t wds[8] = {ra[h].x, ra[h].y, ra[h].z, ra[h].w, rb[h].x, rb[h].y, rb[h].z, rb[h].w};
+                float v[16];
 #pragma unroll
-            for (int o = TPH / 2; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            const int e = m > 0.f ? 8 - frexp_exponent(m) : 0;   // m 2^e in [128, 256)
-            uint32_t p1w[4] = {0u, 0u, 0u, 0u}, p2w[4] = {0u, 0u, 0u, 0u};
+                for (int c = 0; c < 8; ++c) {
+                    v[2 * c] = __uint_as_float(wds[c] << 16);
+                    v[2 * c + 1] = __uint_as_float(wds[c] & 0xFFFF0000u);
+                }
+                float m = 0.f;
 #pragma unroll
-            for (int c = 0; c < 16; c += 2) {   // two channels per conversion (.x -> low byte)
-                const float2 sv = make_float2(scale_pow2(v[c], e), scale_pow2(v[c + 1], e));
-                const __nv_fp8x2_storage_t p1 = __nv_cvt_float2_to_fp8x2(sv, __NV_SATFINITE, __NV_E4M3);
-                const float2 h1 = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(p1, __NV_E4M3)));
-                const __nv_fp8x2_storage_t p2 =
-                    __nv_cvt_float2_to_fp8x2(make_float2(sv.x - h1.x, sv.y - h1.y), __NV_SATFINITE, __NV_E4M3);
-                p1w[c >> 2] |= uint32_t(p1) << (8 * (c & 3));
-                p2w[c >> 2] |= uint32_t(p2) << (8 * (c & 3));
+                for (int c = 0; c < 16; ++c) m = fmaxf(m, fabsf(v[c]));
+#pragma unroll
+                for (int o = TPH / 2; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                const int e = m > 0.f ? 8 - frexp_exponent(m) : 0;   // m 2^e in [128, 256)
+                uint32_t p1w[4] = {0u, 0u, 0u, 0u}, p2w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                for (int c = 0; c < 16; c += 2) {   // two channels per conversion (.x -> low byte)
+                    const float2 sv = make_float2(scale_pow2(v[c], e), scale_pow2(v[c + 1], e));
+                    const __nv_fp8x2_storage_t p1 = __nv_cvt_float2_to_fp8x2(sv, __NV_SATFINITE, __NV_E4M3);
+                    const float2 h1 = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(p1, __NV_E4M3)));
+                    const __nv_fp8x2_storage_t p2 =
+                        __nv_cvt_float2_to_fp8x2(make_float2(sv.x - h1.x, sv.y - h1.y), __NV_SATFINITE, __NV_E4M3);
+                    p1w[c >> 2] |= uint32_t(p1) << (8 * (c & 3));
+                    p2w[c >> 2] |= uint32_t(p2) << (8 * (c & 3));
+                }
+                if (j < H) {
+                    // the query operand in the keys' layout: row j (piece 1) and row H + j (piece 2); H is a
+                    // multiple of 8, so both rows have the same swizzle phase
+                    const int off =
+                        DK == 128 ? j * 128 + ((g ^ (j & 7)) << 4) : j * 64 + ((g ^ ((j >> 1) & 3)) << 4);
+                    *reinterpret_cast<uint4 *>(slot + off) = make_uint4(p1w[0], p1w[1], p1w[2], p1w[3]);
+                    *reinterpret_cast<uint4 *>(slot + H * DK + off) = make_uint4(p2w[0], p2w[1], p2w[2], p2w[3]);
+                    if (g == 0) wsm[j] = ldexpf(wj[h], -e);
+                }
             }
-            // the query operand in the keys' layout: row j (piece 1) and row H + j (piece 2); H is a
-            // multiple of 8, so both rows have the same swizzle phase
-            const int off = DK == 128 ? j * 128 + ((g ^ (j & 7)) << 4) : j * 64 + ((g ^ ((j >> 1) & 3)) << 4);
-            *reinterpret_cast<uint4 *>(slot + off) = make_uint4(p1w[0], p1w[1], p1w[2], p1w[3]);
-            *reinterpret_cast<uint4 *>(slot + H * DK + off) = make_uint4(p2w[0], p2w[1], p2w[2], p2w[3]);
-            if (g == 0) wsm[j] = ldexpf(wj, -e);
         }
     }
+}
+
+// Whether the row scales of a tile (rows row0 .. row0+nvalid-1) travel by one bulk copy: the aligned
+// superset [row0 & ~3, (row0 + nvalid + 3) & ~3) of 16-byte-aligned scales inside the array's scale_len
+// entries.  Otherwise the producer copies them 4 bytes at a time.
+__device__ __forceinline__ bool scales_bulk(int64_t row0, int64_t nvalid, int64_t scale_len, const float *k_scale) {
+    return (reinterpret_cast<uintptr_t>(k_scale) & 15) == 0 && ((row0 + nvalid + 3) & ~int64_t(3)) <= scale_len;
 }
 
 // Sequence and rows of tile t; `b` is a cursor that only moves forward.
@@ -317,7 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kbytes,
         const uint16_t *__restrict__ q, const float *__restrict__ w, int d, const int64_t *__restrict__ seq_off,
         const int32_t *__restrict__ idx, const int64_t *__restrict__ idx_off, int64_t list_cap, int B,
-        const float *__restrict__ k_scale, float *__restrict__ z, float *__restrict__ I, int32_t *err) {
+        const float *__restrict__ k_scale, int64_t scale_len, int64_t axis_cap, float *__restrict__ z,
+        float *__restrict__ I, int32_t *err) {
     using C = Cfg<KIND>;
     constexpr int S = C::kStages;
     constexpr int QIMG = qimg_bytes<KIND, H>();
@@ -350,6 +379,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     // j released its accumulator, which it does after reading the scales.
     constexpr bool kScales = is_e4m3(KIND);
     constexpr int RS = S + KACC;
+    // a scale slot holds a tile's row scales from an aligned start: up to 3 leading and 4 trailing extra
+    constexpr int SS = TR + 8;
     static_assert(!kScales || RS <= kScaleSlotsMax, "row-scale ring");
 
     extern __shared__ uint8_t smem_raw[];
@@ -380,13 +411,16 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     volatile int *abort_v = abort_flag;
 
     // tile axis: the entries (full mode) or the list positions (listed mode); all offsets are
-    // loaded at once, the tile prefix is then summed from shared memory
+    // loaded at once, the tile prefix is then summed from shared memory.  Full mode over an axis an earlier
+    // kernel produced (axis_cap > 0: the rows of a compacted key array, their offsets clamped to its
+    // capacity) waits for that kernel first, like the listed mode
     {
-        if (LISTED) pdl_wait();   // the list offsets come from an earlier kernel
+        if (LISTED || axis_cap > 0) pdl_wait();
         const int64_t *axis = LISTED ? idx_off : seq_off;
+        const int64_t acap = LISTED ? list_cap : axis_cap;
         for (int b = threadIdx.x; b <= B; b += kThreads) {
             int64_t a = axis[b];
-            if (LISTED && a > list_cap) a = list_cap;
+            if (acap > 0 && a > acap) a = acap;
             s_seq[b] = a;
             s_base[b] = seq_off[b];
         }
@@ -458,14 +492,15 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             if (!kScales) return;
             const int slot = int(j % RS);
             const int64_t nvalid = (row_end - row0) < TR ? (row_end - row0) : TR;
-            if ((row0 & 3) == 0 && (nvalid & 3) == 0 && (reinterpret_cast<uintptr_t>(k_scale) & 15) == 0) {
+            const int64_t a0 = row0 & ~int64_t(3), a1 = (row0 + nvalid + 3) & ~int64_t(3);
+            if (scales_bulk(row0, nvalid, scale_len, k_scale)) {
                 if (lane == 0) {   // the barrier's only arrival (no per-lane arrivals next to the MMA's reads)
-                    mbar_arrive_expect_tx(&sfull[slot], uint32_t(nvalid * 4));
-                    bulk_load(s_scale + slot * TR, k_scale + row0, uint32_t(nvalid * 4), &sfull[slot]);
+                    mbar_arrive_expect_tx(&sfull[slot], uint32_t((a1 - a0) * 4));
+                    bulk_load(s_scale + slot * SS, k_scale + a0, uint32_t((a1 - a0) * 4), &sfull[slot]);
                 }
                 return;
             }
-            const uint32_t dst = smem_u32(s_scale + slot * TR);
+            const uint32_t dst = smem_u32(s_scale + slot * SS);
 #pragma unroll
             for (int k = 0; k < TR / 32; ++k) {
                 const int r = lane + 32 * k;
@@ -568,7 +603,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                     for (int c = 0; c < CPR; ++c)
                         cp_async_16(stage_u32 + stage_chunk_off<KIND>(r, c), src + c * 16, valid ? 16u : 0u);
                     if (kScales)
-                        cp_async_4(smem_u32(s_scale + int((t - t0) % RS) * TR + r), k_scale + e, valid ? 4u : 0u);
+                        cp_async_4(smem_u32(s_scale + int((t - t0) % RS) * SS + r), k_scale + e, valid ? 4u : 0u);
                 }
                 // each lane's arrival fires when its copies so far have landed: the stage is signalled as
                 // soon as its own rows are in, while the next tile's gathers are already being issued
@@ -735,7 +770,12 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             if (kScales) ok = ok && mbar_wait(&sfull[i % RS], uint32_t((i / RS) & 1), abort_v, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
             tc_fence_after();
-            const float sc = kScales ? s_scale[int(i % RS) * TR + sub * kRows + quarter * 32 + lane] : 1.f;
+            // the tile's scales start at row0's offset from its aligned start when they came by bulk copy
+            const int soff = (!LISTED && kScales && scales_bulk(row0, (row_end - row0) < TR ? (row_end - row0) : TR,
+                                                                scale_len, k_scale))
+                                 ? int(row0 & 3)
+                                 : 0;
+            const float sc = kScales ? s_scale[int(i % RS) * SS + soff + sub * kRows + quarter * 32 + lane] : 1.f;
             const uint32_t taddr =
                 tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * TILEC + sub * SUBC);
             float za = 0.f, zb = 0.f, zc = 0.f, zd = 0.f;   // four short dependency chains
@@ -819,14 +859,30 @@ size_t smem_bytes(int B) {
     using C = Cfg<KIND>;
     return 1024 + size_t(C::kStages) * C::kStageBytes + 2 * qimg_bytes<KIND, H>() +
            (C::kStages + 2 + kRel + 2 * kAccMax + 1 + kScaleSlotsMax) * 8 + 16 + 16 + 2 * H * 4 +
-           size_t(B + 1) * 24 + 16 + (is_e4m3(KIND) ? size_t(C::kStages + acc_tiles<KIND, H>()) * tile_rows<KIND>() * 4 : 0) +
+           size_t(B + 1) * 24 + 16 +
+           (is_e4m3(KIND) ? size_t(C::kStages + acc_tiles<KIND, H>()) * (tile_rows<KIND>() + 8) * 4 : 0) +
            64;
 }
 
+struct ScanArgs {
+    const void *q;
+    const float *w;
+    const void *k;
+    const float *k_scale;
+    const int64_t *seq_off;   // the tile axis of a full scan (sequence offsets, or a device-produced axis)
+    int64_t n_total;          // rows of the key array
+    const int32_t *idx;       // listed mode: entry lists (NULL: full mode)
+    const int64_t *idx_off;
+    int64_t list_cap;
+    int B, d;
+    float *z, *I;
+    int32_t *err;
+    int64_t axis_cap;         // full mode over a device-produced axis: its capacity (0: seq_off is constant)
+    int64_t scale_len;        // entries of k_scale
+};
+
 template <int KIND, int H>
-lsa_status launch(const void *q, const float *w, const void *k, const float *k_scale, const int64_t *seq_off,
-                  int64_t n_total, const int32_t *idx, const int64_t *idx_off, int64_t list_cap, int B, int d,
-                  float *z, float *I, int32_t *err, cudaStream_t st) {
+lsa_status launch(const ScanArgs &a, cudaStream_t st) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) {
         set_error("lsa_index_score: cuTensorMapEncodeTiled is unavailable");
@@ -834,44 +890,49 @@ lsa_status launch(const void *q, const float *w, const void *k, const float *k_s
     }
     CUtensorMap map;
     const bool fp8 = is_e4m3(KIND);
-    const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(n_total)};
-    const cuuint64_t strides[1] = {cuuint64_t(d) * (fp8 ? 1 : 2)};
+    const cuuint64_t dims[2] = {cuuint64_t(a.d), cuuint64_t(a.n_total)};
+    const cuuint64_t strides[1] = {cuuint64_t(a.d) * (fp8 ? 1 : 2)};
     // box: one 128-byte column block (64 bytes for e4m3 d = 64) x kBoxRows rows
-    const cuuint32_t box[2] = {cuuint32_t(fp8 ? d : 64), cuuint32_t(Cfg<KIND>::kBoxRows)};
+    const cuuint32_t box[2] = {cuuint32_t(fp8 ? a.d : 64), cuuint32_t(Cfg<KIND>::kBoxRows)};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                     const_cast<void *>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     const_cast<void *>(a.k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      KIND == E4M3_D64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         set_error("lsa_index_score: cuTensorMapEncodeTiled failed (%d)", int(r));
         return LSA_ERR_CUDA;
     }
-    const size_t smem = smem_bytes<KIND, H>(B);
-    auto kern = idx ? scan_tc<KIND, H, true> : scan_tc<KIND, H, false>;
+    const size_t smem = smem_bytes<KIND, H>(a.B);
+    auto kern = a.idx ? scan_tc<KIND, H, true> : scan_tc<KIND, H, false>;
     LSA_CUDA(ensure_smem(kern, smem));
-    const int64_t axis = idx ? list_cap : n_total;
-    const int64_t max_tiles = (axis + tile_rows<KIND>() - 1) / tile_rows<KIND>() + B;
+    const int64_t axis = a.idx ? a.list_cap : (a.axis_cap > 0 ? a.axis_cap : a.n_total);
+    const int64_t max_tiles = (axis + tile_rows<KIND>() - 1) / tile_rows<KIND>() + a.B;
     const int grid = int(max_tiles < sm_count() ? max_tiles : sm_count());
-    LSA_CUDA(launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, map, static_cast<const uint8_t *>(k),
-                        static_cast<const uint16_t *>(q), w, d, seq_off, idx, idx_off, list_cap, B, k_scale, z, I,
-                        err));
+    LSA_CUDA(launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, map, static_cast<const uint8_t *>(a.k),
+                        static_cast<const uint16_t *>(a.q), a.w, a.d, a.seq_off, a.idx, a.idx_off, a.list_cap, a.B,
+                        a.k_scale, a.scale_len, a.axis_cap, a.z, a.I, a.err));
     static const char *kNames[2][4] = {
         {"scan_tc bf16 d128", "scan_tc bf16 d64", "scan_tc e4m3 d128", "scan_tc e4m3 d64"},
         {"scan_tc_listed bf16 d128", "scan_tc_listed bf16 d64", "scan_tc_listed e4m3 d128", "scan_tc_listed e4m3 d64"}};
-    LSA_LAUNCHED(kNames[idx ? 1 : 0][KIND]);
+    LSA_LAUNCHED(kNames[a.idx ? 1 : 0][KIND]);
     return LSA_OK;
 }
 
 template <int KIND>
-lsa_status launch_h(int H, const void *q, const float *w, const void *k, const float *k_scale,
-                    const int64_t *seq_off, int64_t n_total, const int32_t *idx, const int64_t *idx_off,
-                    int64_t list_cap, int B, int d, float *z, float *I, int32_t *err, cudaStream_t st) {
+lsa_status launch_h(int H, const ScanArgs &a, cudaStream_t st) {
     switch (H) {
-    case 16: return launch<KIND, 16>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err, st);
-    case 32: return launch<KIND, 32>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err, st);
-    default: return launch<KIND, 64>(q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err, st);
+    case 16: return launch<KIND, 16>(a, st);
+    case 32: return launch<KIND, 32>(a, st);
+    default: return launch<KIND, 64>(a, st);
     }
+}
+
+lsa_status launch_kind(lsa_dtype k_dtype, int H, const ScanArgs &a, cudaStream_t st) {
+    if (k_dtype == LSA_E4M3 && a.d == 128) return launch_h<E4M3_D128>(H, a, st);
+    if (k_dtype == LSA_E4M3) return launch_h<E4M3_D64>(H, a, st);
+    if (a.d == 128) return launch_h<BF16_D128>(H, a, st);
+    return launch_h<BF16_D64>(H, a, st);
 }
 
 }  // namespace
@@ -890,16 +951,17 @@ lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, l
                                  const float *k_scale, const int64_t *seq_off, int64_t n_total,
                                  const int32_t *idx, const int64_t *idx_off, int64_t list_cap, int32_t B,
                                  int32_t H, int32_t d, float *z, float *I, int32_t *err, cudaStream_t st) {
-    if (k_dtype == LSA_E4M3 && d == 128)
-        return launch_h<E4M3_D128>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err,
-                                   st);
-    if (k_dtype == LSA_E4M3)
-        return launch_h<E4M3_D64>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err,
-                                  st);
-    if (d == 128)
-        return launch_h<BF16_D128>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err,
-                                   st);
-    return launch_h<BF16_D64>(H, q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err, st);
+    const ScanArgs a{q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err, 0, n_total};
+    return launch_kind(k_dtype, H, a, st);
+}
+
+lsa_status launch_index_score_tc_axis(const void *q, const float *w, const void *k, lsa_dtype k_dtype,
+                                      const float *k_scale, int64_t scale_len, const int64_t *axis_off,
+                                      int64_t axis_cap, int64_t n_rows, int32_t B, int32_t H, int32_t d, float *z,
+                                      int32_t *err, cudaStream_t st) {
+    const ScanArgs a{q,  w,        k,    k_scale, axis_off, n_rows, nullptr, nullptr, 0, B, d, z, nullptr,
+                     err, axis_cap, scale_len};
+    return launch_kind(k_dtype, H, a, st);
 }
 
 }  // namespace lsa

@@ -92,6 +92,18 @@ lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, l
                                  const float *k_scale, const int64_t *seq_off, int64_t n_total,
                                  const int32_t *idx, const int64_t *idx_off, int64_t list_cap, int32_t B,
                                  int32_t H, int32_t d, float *z, float *I, int32_t *err, cudaStream_t st);
+// Full tensor-core scan over a device-produced row axis: rows axis_off[b] .. axis_off[b+1] (clamped to
+// axis_cap) of the key array k [n_rows, d] belong to sequence b; z is written per row.  Used on a compacted
+// copy of the kept keys (rows in kept-list order), so z lands at the kept position.
+lsa_status launch_index_score_tc_axis(const void *q, const float *w, const void *k, lsa_dtype k_dtype,
+                                      const float *k_scale, int64_t scale_len, const int64_t *axis_off,
+                                      int64_t axis_cap, int64_t n_rows, int32_t B, int32_t H, int32_t d, float *z,
+                                      int32_t *err, cudaStream_t st);
+// Copies the key rows (and e4m3 row scales) of the kept entries into kept-list order:
+// kc[p] = k[seq_off[b] + kept_idx[p]] for p < min(kept_off[B], cap).
+lsa_status launch_gather_keys(const void *k, int64_t row_bytes, const float *k_scale, const int64_t *seq_off,
+                              const int32_t *kept_idx, const int64_t *kept_off, int32_t B, int64_t cap, void *kc,
+                              float *sc, cudaStream_t st);
 lsa_status launch_select(const float *z, const int64_t *seq_off, int64_t n_total, int32_t B,
                          int32_t *kept_idx, int64_t capacity, int64_t *kept_off, uint32_t *mask,
                          void *workspace, int32_t *err, cudaStream_t st);

@@ -215,6 +215,31 @@ def test_topk_stage_exact(lsa, k, ties):
             assert ((pos[b][:c] >= ko[b]) & (pos[b][:c] < ko[b + 1])).all()
 
 
+@pytest.mark.parametrize("k", [64, 2048, 4096])
+def test_topk_clustered_scores_stage_exact(lsa, k):
+    """Scores shaped like a kept set of the 500K context: ~14K kept per sequence, chunk-correlated values in
+    a narrow band, runs of exactly equal scores at and around the k-th, and one sequence whose scores are all
+    equal: the candidate path and its fallbacks against the oracle's sorted top-k."""
+    rng = np.random.default_rng(k)
+    lens = [14400, 14000, 15000, 30000, 9000]
+    seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    n = int(seq_off[-1])
+    chunk_mean = np.repeat(rng.uniform(0.05, 0.3, size=(n + 63) // 64), 64)[:n]
+    z = (chunk_mean + 0.01 * rng.normal(size=n)).astype(np.float32)
+    z[rng.random(n) < 0.1] = -1.0                                    # ~10% not kept
+    s3 = slice(seq_off[3], seq_off[4])
+    z[s3] = np.round(z[s3] * 64) / 64                                # many exact ties
+    z[seq_off[4]:] = 0.125                                           # all equal
+    kept, ko, _ = oracle.select(z.astype(np.float64), seq_off)
+    b_of = np.repeat(np.arange(len(lens)), np.diff(ko))
+    zk = z[seq_off[:-1][b_of] + kept].astype(np.float64)
+    ref_idx, ref_cnt = oracle.topk(zk, kept, ko, k)
+    for by_entry, zin in ((1, z), (0, zk.astype(np.float32))):
+        idx, pos, cnt = _topk_gpu(lsa, zin, by_entry, seq_off, kept, ko, k)
+        assert np.array_equal(cnt, ref_cnt)
+        assert np.array_equal(idx, ref_idx)
+
+
 def test_topk_respects_kept_capacity(lsa):
     seq_off = np.array([0, 100, 300], np.int64)
     z = np.linspace(1, 2, 300).astype(np.float32)
