@@ -66,7 +66,8 @@ def parse_args():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--hot-frac", type=float, default=0.2)
-    ap.add_argument("--only", choices=["scan", "union", "encoder", "merged"], default=None,
+    ap.add_argument("--lookahead", type=int, default=16, help="--only lookahead: the lookahead distance L")
+    ap.add_argument("--only", choices=["scan", "union", "encoder", "merged", "lookahead"], default=None,
                     help="run one stage alone (W + K launches), for profiling; prints its mean time. encoder: the indexer query encoder h -> (q, w). merged: decode with the recent window and HCA rows merged into the attention set. "
                          "union: the OR-mode union of three indexer layers (three full scans, the union, select)")
     return ap.parse_args()
@@ -676,6 +677,119 @@ def run_only_encoder(args):
     return 0
 
 
+def run_only_lookahead(args):
+    """Decode windows with and without lookahead, from a warm cache and from a cold one.  Warm: the hot
+    buffer caches rows across refreshes (a refresh fetches a few hundred new rows).  Cold: the cache is
+    emptied before each window's refresh (lookahead 0) or prediction step (lookahead L), so every kept row
+    (~57 MB at 500K) crosses the host link, as for a new request or a topic shift.  With lookahead the fetch
+    runs on the side stream under the window's last L steps.  Same loop as the headline (tau-step windows, 3
+    context replicas, CUDA graphs); prints ms per window for the four cases and the cold fetch's rate."""
+    import torch
+
+    import synth
+    from lookahead_sparse_kv_index_b200 import lsa
+
+    wl = synth.WORKLOADS[args.config]()
+    dev = synth.to_torch(wl)
+    keys = [dev["keys"]] + [dev["keys"].clone() for _ in range(REPLICAS - 1)]
+    # a cold prediction keeps the current set resident beside the whole next set: twice the hot buffer
+    cap = max(wl.topk, int(min(1.0, 2 * args.hot_frac) * wl.n_total))
+    tau, L = wl.tau, args.lookahead
+    steps_in = [wl.step_inputs(t) for t in range(tau)]
+    q_d = [synth.raw_to_torch(s_[0]) for s_ in steps_in]
+    w_d = [torch.from_numpy(np.ascontiguousarray(s_[1])).cuda() for s_ in steps_in]
+    Q_d = [synth.raw_to_torch(s_[2]) for s_ in steps_in]
+    q_ref = [synth.raw_to_torch(wl.step_inputs(tau * (w + 1))[0]) for w in range(8)]
+    odt = torch.int16 if wl.attn_dtype == "bf16" else torch.float32
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=odt, device="cuda")
+    lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device="cuda")
+    res = {}
+    for la in (0, L):
+        ctxs = [lsa.Context(B=wl.B, H=wl.H, d=wl.d, q_dtype=wl.q_dtype, k_dtype=wl.key_dtype, Hq=wl.Hq, D=wl.D,
+                            attn_dtype=wl.attn_dtype, topk=wl.topk, seq_off_host=wl.seq_off, keys=keys[r],
+                            k_scale=dev["k_scale"], cold_host=dev["cold"], row_bytes=wl.row_bytes,
+                            kv_row_stride=wl.row_stride, k_off=wl.k_off, v_off=wl.v_off, kept_capacity=cap,
+                            tau=tau, scale=wl.scale, lookahead=la) for r in range(REPLICAS)]
+        # the refreshing / predicting step's query changes every window, so the kept set moves
+        qs = [q_d[0].clone()] + q_d[1:]
+        if la:
+            qs[tau - la] = qs[tau - la].clone()
+        qv = qs[tau - la] if la else qs[0]
+        counter = [0]
+        t_next = [0] * REPLICAS
+
+        for mode in ("warm", "cold"):
+            def window(w):
+                r = w % REPLICAS
+                ctx = ctxs[r]
+                for _ in range(tau):
+                    t = t_next[r]
+                    t_next[r] += 1
+                    fetch_step = (t % tau == 0) if la == 0 else ((t + la) % tau == 0)
+                    if fetch_step:
+                        qv.copy_(q_ref[counter[0] % len(q_ref)], non_blocking=True)
+                        counter[0] += 1
+                        if mode == "cold":
+                            ctx.flush_cache()
+                    ctx.step(t, qs[t % tau], w_d[t % tau], Q_d[t % tau], out, lse)
+
+            for w in range(2 * REPLICAS + args.warmup):
+                window(w)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for w in range(args.steps):
+                window(w)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+            # one more window per context with stage timing (eager): the fetch's own time on the side stream
+            for c in ctxs:
+                c.reset_counters()
+                c.set_timing(True)
+            fetched = []
+            for w in range(REPLICAS):
+                window(w)
+                torch.cuda.synchronize()
+                fetched.append(ctxs[w % REPLICAS].fetched())
+            st = {}
+            for c in ctxs:
+                for k, (msk, calls) in c.stage_times().items():
+                    a = st.setdefault(k, [0.0, 0])
+                    a[0] += msk
+                    a[1] += calls
+                c.set_timing(False)
+            g = st.get("gather", [0.0, 0])
+            fetch_ms = g[0] / g[1] if g[1] else None
+            rows = float(np.mean(fetched))
+            errs = [int(lsa.device_view(c.view().err, 1, torch.int32).item()) for c in ctxs]
+            res[f"lookahead{la}_{mode}"] = {"kept_capacity": cap,
+                "ms_per_window": ms, "decode_steps_per_s": tau / (ms / 1e3), "fetched_rows_per_window": rows,
+                "fetch_ms_side_stream": fetch_ms,
+                "fetch_GBps": rows * wl.row_bytes / (fetch_ms / 1e3) / 1e9 if fetch_ms else None,
+                "device_errors": errs}
+        for c in ctxs:
+            c.close()
+        torch.cuda.synchronize()
+    # the host link's own rate in this run (pinned copy, copy engine)
+    hsrc = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    ddst = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ddst.copy_(hsrc, non_blocking=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        ddst.copy_(hsrc, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    h2d = 3 * (256 << 20) / (e0.elapsed_time(e1) / 1e3) / 1e9
+    for k in res:
+        if res[k]["fetch_GBps"]:
+            res[k]["fetch_frac_of_pinned_copy"] = res[k]["fetch_GBps"] / h2d
+    print(json.dumps({"only": "lookahead", "config": args.config, "tau": tau, "lookahead": L,
+                      "windows_timed": args.steps, "pinned_h2d_copy_GBps": h2d, **res}), flush=True)
+    return 0 if all(e == 0 for r in res.values() for e in r["device_errors"]) else 1
+
+
 def run_only_merged(args):
     """Decode windows with the always-resident context merged into the attention set: a recent window of
     8K tokens (2048 entries) and the HCA rows (one per 128 tokens) per sequence, against the same decode
@@ -895,6 +1009,8 @@ def main():
         return run_only_encoder(args)
     if args.only == "merged":
         return run_only_merged(args)
+    if args.only == "lookahead":
+        return run_only_lookahead(args)
     return run_cuda(args)
 
 

@@ -365,6 +365,15 @@ typedef struct lsa_params {
     const void *const *k_dev_layers;    /* HOST array [n_layers-1] of DEVICE key pointers of layers
                                            1 .. n_layers-1 (layer 0 is k_dev); same dtype and shape */
     const float *const *k_scale_layers; /* HOST array [n_layers-1] of their E4M3 row scales (else NULL) */
+    /* Lookahead (blog page: critical chunks fetched from the cold pool "just in time"; section 2.1
+     * "Dynamic Fetching"): 0 refreshes at the first step of every window, its fetch on the step's critical
+     * path.  L in [1, tau): the kept set of window r >= 1 (steps r*tau .. r*tau + tau-1) is predicted at
+     * step r*tau - L with that step's indexer query, after the step's own work; its rows are fetched on the
+     * context's side stream while steps r*tau - L .. r*tau - 1 still attend window r-1's set (the fetch never
+     * evicts a row that set uses), and at step r*tau the new set becomes current and is re-ranked with that
+     * step's query.  Window 0 refreshes at its first step.  Needs full_fetch = 0; the hot buffer must hold
+     * both sets' rows (LSA_ERR_CAPACITY otherwise). */
+    int32_t lookahead;
 } lsa_params;
 
 typedef struct lsa_ctx lsa_ctx;
@@ -444,6 +453,11 @@ lsa_status lsa_ctx_set_timing(lsa_ctx *ctx, int32_t enable);
 lsa_status lsa_ctx_stage_times(lsa_ctx *ctx, double *ms, int64_t *calls);
 lsa_status lsa_ctx_reset_counters(lsa_ctx *ctx);
 int64_t lsa_ctx_launches(lsa_ctx *ctx);
+
+/* Empties the hot-buffer cache (enqueued on `stream`): afterwards no entry counts as resident, so the next
+ * refresh or prediction fetches every kept row from the cold pool (a cold start, e.g. a new request or a
+ * topic shift).  The current kept set's rows stay in place for the steps that still read them. */
+lsa_status lsa_ctx_flush_cache(lsa_ctx *ctx, void *stream);
 
 /* ------------------------------------------------------------------------
  * lsa_selftest_bounded_wait -- checks, on the GPU, the expiry path of the

@@ -12,6 +12,15 @@
 // Other steps: listed re-score of the kept set with the step's indexer query
 // -> top-k -> attention.  The host never waits inside a step.
 //
+// Lookahead (lsa_params.lookahead = L >= 1): window r >= 1's kept set is
+// predicted at step r tau - L with that step's indexer query -- after that
+// step's own work, a full scan and the selection into a second kept-set buffer
+// -- and fetched on the side stream (the cache never evicting a slot the
+// current set uses) while steps r tau - L .. r tau - 1 still attend window
+// r - 1's set; at step r tau the new set becomes current and the step re-ranks
+// it with its own query.  The side-stream work is enqueued outside the step
+// graphs (a captured fork must rejoin inside its graph).
+//
 // Options.  Several indexer layers (section 2.4 "Optimal Configuration"): each
 // scan runs once per layer with that layer's keys and (q, w), and the union
 // score max_l z_l (union.cu) feeds select and the top-k.  Merged attention set
@@ -34,18 +43,23 @@
 
 #include "lsa_internal.cuh"
 
+// Step kinds: a refresh (scan, select, fetch, top-k over the scan's scores, attention), a listed step
+// (re-score of the current kept set, top-k, attention), and with lookahead a predicting step (a listed step,
+// then the scan and selection of the next window's set into the other kept-set buffer).
+enum StepKind { kRefresh = 0, kListed = 1, kPredict = 2, kKinds = 3 };
+
 struct GraphKey {
-    bool refresh;
+    int kind, set;
     const void *q, *w, *Q;
     void *out;
     float *lse;
     bool operator==(const GraphKey &o) const {
-        return refresh == o.refresh && q == o.q && w == o.w && Q == o.Q && out == o.out && lse == o.lse;
+        return kind == o.kind && set == o.set && q == o.q && w == o.w && Q == o.Q && out == o.out && lse == o.lse;
     }
 };
 struct GraphKeyHash {
     size_t operator()(const GraphKey &k) const {
-        size_t h = k.refresh;
+        size_t h = size_t(k.kind) * 2 + size_t(k.set);
         for (const void *p : {k.q, k.w, k.Q, static_cast<const void *>(k.out), static_cast<const void *>(k.lse)})
             h = h * 1000003u ^ std::hash<const void *>()(p);
         return h;
@@ -66,15 +80,24 @@ struct lsa_ctx {
     int64_t *seq_off_d = nullptr;
     float *z = nullptr;
     float *z_kept = nullptr;
-    int32_t *kept_idx = nullptr;
-    int64_t *kept_off = nullptr;
+    // kept sets: the current one (cur) and, with lookahead, the next window's, written while cur is in use
+    struct KeptSet {
+        int32_t *kept_idx = nullptr;
+        int64_t *kept_off = nullptr;
+        int32_t *kept_slot = nullptr;   // [cap] hot slot of each kept position
+        void *kc[lsa::kMaxUnionLayers] = {};    // compacted kept keys per layer (kept-list order)
+        float *sc[lsa::kMaxUnionLayers] = {};   // their e4m3 row scales
+    } ks[2];
+    int cur = 0, n_sets = 1;
+    int lookahead = 0;
+    bool predicted = false;   // the other set holds a predicted set whose fetch was enqueued
+    cudaEvent_t ev_pred = nullptr, ev_pend = nullptr;
     int32_t *slot_of = nullptr;
     void *hot = nullptr;
     int32_t *topk_idx = nullptr, *topk_pos = nullptr, *topk_cnt = nullptr;
     int32_t *err = nullptr;
     // hot-buffer cache (incremental fetch)
     int32_t *owner = nullptr;       // [cap] entry held by each slot, or -1
-    int32_t *kept_slot = nullptr;   // [cap] hot slot of each kept position
     int64_t *fetched = nullptr;     // rows fetched by the last refresh
     void *fetch_ws = nullptr;
     cudaEvent_t ev_assign = nullptr;
@@ -87,8 +110,6 @@ struct lsa_ctx {
     // compacted kept keys (and e4m3 row scales) per layer, in kept-list order, written at each refresh; the
     // listed re-score streams them with the full tensor-core scan (when the shape runs on the tensor cores)
     bool compact = false;
-    void *kc[lsa::kMaxUnionLayers] = {};
-    float *sc[lsa::kMaxUnionLayers] = {};
     int64_t sc_len = 0;
     // merged attention set: window and HCA rows live in the arena after the hot buffer
     bool merged = false;
@@ -123,7 +144,7 @@ struct lsa_ctx {
     int64_t launches = 0;
     // graphs
     bool use_graphs = true;
-    bool eager_done[2] = {false, false};
+    bool eager_done[kKinds * 2] = {};
     cudaStream_t cap = nullptr;
     std::unordered_map<GraphKey, GraphEntry, GraphKeyHash> graphs;
 };
@@ -133,16 +154,23 @@ namespace {
 using namespace lsa;
 
 void free_all(lsa_ctx *c) {
-    void *bufs[] = {c->seq_off_d, c->z, c->z_kept, c->kept_idx, c->kept_off, c->slot_of, c->hot,
+    void *bufs[] = {c->seq_off_d, c->z, c->z_kept, c->slot_of, c->hot,
                     c->topk_idx, c->topk_pos, c->topk_cnt, c->err, c->sel_ws, c->attn_ws,
-                    c->owner, c->kept_slot, c->fetched, c->fetch_ws, c->hca_off_d, c->attn_rows, c->z_layers,
+                    c->owner, c->fetched, c->fetch_ws, c->hca_off_d, c->attn_rows, c->z_layers,
                     c->zk_layers};
     for (void *b : bufs)
         if (b) cudaFree(b);
-    for (int l = 0; l < lsa::kMaxUnionLayers; ++l) {
-        if (c->kc[l]) cudaFree(c->kc[l]);
-        if (c->sc[l]) cudaFree(c->sc[l]);
+    for (auto &k : c->ks) {
+        for (void *b : {static_cast<void *>(k.kept_idx), static_cast<void *>(k.kept_off),
+                        static_cast<void *>(k.kept_slot)})
+            if (b) cudaFree(b);
+        for (int l = 0; l < lsa::kMaxUnionLayers; ++l) {
+            if (k.kc[l]) cudaFree(k.kc[l]);
+            if (k.sc[l]) cudaFree(k.sc[l]);
+        }
     }
+    if (c->ev_pred) cudaEventDestroy(c->ev_pred);
+    if (c->ev_pend) cudaEventDestroy(c->ev_pend);
     for (auto &sg : c->stage) {
         for (void *b : {sg.q, sg.Q, sg.out, static_cast<void *>(sg.w), static_cast<void *>(sg.lse)})
             if (b) cudaFree(b);
@@ -163,6 +191,7 @@ void free_all(lsa_ctx *c) {
 }
 
 constexpr size_t kMaxGraphs = 256;
+constexpr int kPredictFetchCtas = 32;
 
 // The device address of page-locked host memory mapped for the device, else nullptr.
 void *mapped_host(const void *p) {
@@ -221,97 +250,107 @@ lsa_status alloc(T **p, size_t bytes) {
     return LSA_OK;
 }
 
-lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w, const void *Q, void *out,
-                        float *lse, cudaStream_t st) {
+// Full scan(s) of every entry with (q, w), the layers' union, and the selection into kept set `set`.
+lsa_status enqueue_scan_select(lsa_ctx *c, const void *q, const float *w, int set, cudaStream_t st) {
     const lsa_params &p = c->p;
-    const int64_t cap = p.kept_capacity;
     const size_t q_layer = size_t(p.B) * p.H * p.d * elem_size(p.q_dtype);   // bytes of one layer's q
     const size_t w_layer = size_t(p.B) * p.H;                                 // floats of one layer's w
-    if (refresh) {
-        StageTimer ts(c, LSA_STAGE_SCORE, st);
-        if (c->n_layers == 1) {
-            LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
-                                       p.n_total, nullptr, nullptr, 0, p.B, p.H, p.d, c->z, nullptr, 0,
-                                       c->err, st));
-        } else {
-            const float *zl[kMaxUnionLayers];
-            for (int l = 0; l < c->n_layers; ++l) {
-                float *z_l = c->z_layers + size_t(l) * p.n_total;
-                LSA_TRY(launch_index_score(static_cast<const char *>(q) + l * q_layer, p.q_dtype, w + l * w_layer,
-                                           c->k_layer[l], p.k_dtype, c->ks_layer[l], c->seq_off_d, p.n_total,
-                                           nullptr, nullptr, 0, p.B, p.H, p.d, z_l, nullptr, 0, c->err, st));
-                zl[l] = z_l;
-            }
-            LSA_TRY(launch_union(zl, c->n_layers, p.n_total, c->z, st));
-        }
-        ts.done();
-        StageTimer tsel(c, LSA_STAGE_SELECT, st);
-        LSA_TRY(launch_select(c->z, c->seq_off_d, p.n_total, p.B, c->kept_idx, cap, c->kept_off,
-                              nullptr, c->sel_ws, c->err, st));
-        tsel.done();
-        LSA_CUDA(cudaEventRecord(c->ev_sel, st));
-        LSA_CUDA(cudaStreamWaitEvent(c->side, c->ev_sel, 0));
-        StageTimer tg(c, LSA_STAGE_GATHER, c->side);
-        if (p.full_fetch) {
-            LSA_TRY(launch_gather(c->cold_dev, p.row_bytes, c->seq_off_d, p.n_total, c->kept_idx, c->kept_off, p.B,
-                                  c->hot, cap, c->slot_of, c->err, c->side));
-        } else {
-            LSA_TRY(launch_fetch(c->cold_dev, p.row_bytes, c->seq_off_d, c->kept_idx, c->kept_off, p.B, c->hot, cap,
-                                 c->slot_of, c->owner, c->kept_slot, c->fetched, c->fetch_ws, c->err, c->ev_assign,
-                                 c->side));
-        }
-        if (c->compact)
-            for (int l = 0; l < c->n_layers; ++l)
-                LSA_TRY(launch_gather_keys(c->k_layer[l], int64_t(p.d) * int64_t(elem_size(p.k_dtype)), c->ks_layer[l],
-                                           c->seq_off_d, c->kept_idx, c->kept_off, p.B, cap, c->kc[l], c->sc[l],
-                                           c->side));
-        tg.done();
-        LSA_CUDA(cudaEventRecord(c->ev_gather, c->side));
-        // the top-k writes hot slots: with the cache it needs the slot assignment first
-        if (!p.full_fetch) LSA_CUDA(cudaStreamWaitEvent(st, c->ev_assign, 0));
-        StageTimer tk(c, LSA_STAGE_TOPK, st);
-        LSA_TRY(launch_topk(c->z, 1, c->seq_off_d, c->kept_idx, c->kept_off, p.B, p.topk, cap,
-                            p.full_fetch ? nullptr : c->kept_slot, c->topk_idx, c->topk_pos, c->topk_cnt, st));
-        tk.done();
-        LSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
+    StageTimer ts(c, LSA_STAGE_SCORE, st);
+    if (c->n_layers == 1) {
+        LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d, p.n_total,
+                                   nullptr, nullptr, 0, p.B, p.H, p.d, c->z, nullptr, 0, c->err, st));
     } else {
-        StageTimer tr(c, LSA_STAGE_RESCORE, st);
-        const bool compact = c->compact && aligned16(q);   // the tensor-core scan reads q with 16-byte loads
-        if (compact) {
-            // the kept keys in kept-list order: z lands at the kept position
-            const float *zl[kMaxUnionLayers];
-            for (int l = 0; l < c->n_layers; ++l) {
-                float *z_l = c->n_layers == 1 ? c->z_kept : c->zk_layers + size_t(l) * cap;
-                LSA_TRY(launch_index_score_tc_axis(static_cast<const char *>(q) + l * q_layer, w + l * w_layer,
-                                                   c->kc[l], p.k_dtype, c->sc[l], c->sc_len, c->kept_off, cap, cap,
-                                                   p.B, p.H, p.d, z_l, c->err, st));
-                zl[l] = z_l;
-            }
-            if (c->n_layers > 1) LSA_TRY(launch_union(zl, c->n_layers, cap, c->z_kept, st));
-        } else if (c->n_layers == 1) {
-            LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
-                                       p.n_total, c->kept_idx, c->kept_off, cap, p.B, p.H, p.d, c->z_kept,
-                                       nullptr, 0, c->err, st));
-        } else {
-            // every layer re-scores the kept set; the ranking score is their union (positions past the
-            // kept total hold stale values that the top-k never reads)
-            const float *zl[kMaxUnionLayers];
-            for (int l = 0; l < c->n_layers; ++l) {
-                float *z_l = c->zk_layers + size_t(l) * cap;
-                LSA_TRY(launch_index_score(static_cast<const char *>(q) + l * q_layer, p.q_dtype, w + l * w_layer,
-                                           c->k_layer[l], p.k_dtype, c->ks_layer[l], c->seq_off_d, p.n_total,
-                                           c->kept_idx, c->kept_off, cap, p.B, p.H, p.d, z_l, nullptr, 0, c->err,
-                                           st));
-                zl[l] = z_l;
-            }
-            LSA_TRY(launch_union(zl, c->n_layers, cap, c->z_kept, st));
+        const float *zl[kMaxUnionLayers];
+        for (int l = 0; l < c->n_layers; ++l) {
+            float *z_l = c->z_layers + size_t(l) * p.n_total;
+            LSA_TRY(launch_index_score(static_cast<const char *>(q) + l * q_layer, p.q_dtype, w + l * w_layer,
+                                       c->k_layer[l], p.k_dtype, c->ks_layer[l], c->seq_off_d, p.n_total, nullptr,
+                                       nullptr, 0, p.B, p.H, p.d, z_l, nullptr, 0, c->err, st));
+            zl[l] = z_l;
         }
-        tr.done();
-        StageTimer tk(c, LSA_STAGE_TOPK, st);
-        LSA_TRY(launch_topk(c->z_kept, 0, c->seq_off_d, c->kept_idx, c->kept_off, p.B, p.topk, cap,
-                            p.full_fetch ? nullptr : c->kept_slot, c->topk_idx, c->topk_pos, c->topk_cnt, st));
-        tk.done();
+        LSA_TRY(launch_union(zl, c->n_layers, p.n_total, c->z, st));
     }
+    ts.done();
+    StageTimer tsel(c, LSA_STAGE_SELECT, st);
+    LSA_TRY(launch_select(c->z, c->seq_off_d, p.n_total, p.B, c->ks[set].kept_idx, p.kept_capacity,
+                          c->ks[set].kept_off, nullptr, c->sel_ws, c->err, st));
+    tsel.done();
+    return LSA_OK;
+}
+
+// The cold-pool fetch of kept set `set` (the cache never evicting the slots of kept set `protect`, or none
+// when protect < 0), then the compaction of its keys; on the side stream.
+lsa_status enqueue_fetch(lsa_ctx *c, int set, int protect, cudaStream_t side) {
+    const lsa_params &p = c->p;
+    const int64_t cap = p.kept_capacity;
+    auto &k = c->ks[set];
+    StageTimer tg(c, LSA_STAGE_GATHER, side);
+    if (p.full_fetch) {
+        LSA_TRY(launch_gather(c->cold_dev, p.row_bytes, c->seq_off_d, p.n_total, k.kept_idx, k.kept_off, p.B, c->hot,
+                              cap, c->slot_of, c->err, side));
+    } else {
+        LSA_TRY(launch_fetch(c->cold_dev, p.row_bytes, c->seq_off_d, k.kept_idx, k.kept_off, p.B, c->hot, cap,
+                             c->slot_of, c->owner, k.kept_slot, c->fetched, c->fetch_ws, c->err, c->ev_assign, side,
+                             protect >= 0 ? c->ks[protect].kept_slot : nullptr,
+                             protect >= 0 ? c->ks[protect].kept_off : nullptr,
+                             // under running decode steps the host-link copy takes few SMs (32 CTAs keep ~1 MB of
+                             // zero-copy reads in flight, far more than the link's bandwidth-delay product)
+                             protect >= 0 ? kPredictFetchCtas : 0));
+    }
+    if (c->compact)
+        for (int l = 0; l < c->n_layers; ++l)
+            LSA_TRY(launch_gather_keys(c->k_layer[l], int64_t(p.d) * int64_t(elem_size(p.k_dtype)), c->ks_layer[l],
+                                       c->seq_off_d, k.kept_idx, k.kept_off, p.B, cap, k.kc[l], k.sc[l], side));
+    tg.done();
+    return LSA_OK;
+}
+
+// Re-score of kept set `set` with this step's (q, w), the layers' union, then the top-k.
+lsa_status enqueue_rescore_topk(lsa_ctx *c, const void *q, const float *w, int set, cudaStream_t st) {
+    const lsa_params &p = c->p;
+    const int64_t cap = p.kept_capacity;
+    const size_t q_layer = size_t(p.B) * p.H * p.d * elem_size(p.q_dtype);
+    const size_t w_layer = size_t(p.B) * p.H;
+    auto &k = c->ks[set];
+    StageTimer tr(c, LSA_STAGE_RESCORE, st);
+    const bool compact = c->compact && aligned16(q);   // the tensor-core scan reads q with 16-byte loads
+    if (compact) {
+        // the kept keys in kept-list order: z lands at the kept position
+        const float *zl[kMaxUnionLayers];
+        for (int l = 0; l < c->n_layers; ++l) {
+            float *z_l = c->n_layers == 1 ? c->z_kept : c->zk_layers + size_t(l) * cap;
+            LSA_TRY(launch_index_score_tc_axis(static_cast<const char *>(q) + l * q_layer, w + l * w_layer, k.kc[l],
+                                               p.k_dtype, k.sc[l], c->sc_len, k.kept_off, cap, cap, p.B, p.H, p.d,
+                                               z_l, c->err, st));
+            zl[l] = z_l;
+        }
+        if (c->n_layers > 1) LSA_TRY(launch_union(zl, c->n_layers, cap, c->z_kept, st));
+    } else if (c->n_layers == 1) {
+        LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d, p.n_total,
+                                   k.kept_idx, k.kept_off, cap, p.B, p.H, p.d, c->z_kept, nullptr, 0, c->err, st));
+    } else {
+        // every layer re-scores the kept set; the ranking score is their union (positions past the
+        // kept total hold stale values that the top-k never reads)
+        const float *zl[kMaxUnionLayers];
+        for (int l = 0; l < c->n_layers; ++l) {
+            float *z_l = c->zk_layers + size_t(l) * cap;
+            LSA_TRY(launch_index_score(static_cast<const char *>(q) + l * q_layer, p.q_dtype, w + l * w_layer,
+                                       c->k_layer[l], p.k_dtype, c->ks_layer[l], c->seq_off_d, p.n_total,
+                                       k.kept_idx, k.kept_off, cap, p.B, p.H, p.d, z_l, nullptr, 0, c->err, st));
+            zl[l] = z_l;
+        }
+        LSA_TRY(launch_union(zl, c->n_layers, cap, c->z_kept, st));
+    }
+    tr.done();
+    StageTimer tk(c, LSA_STAGE_TOPK, st);
+    LSA_TRY(launch_topk(c->z_kept, 0, c->seq_off_d, k.kept_idx, k.kept_off, p.B, p.topk, cap,
+                        p.full_fetch ? nullptr : k.kept_slot, c->topk_idx, c->topk_pos, c->topk_cnt, st));
+    tk.done();
+    return LSA_OK;
+}
+
+lsa_status enqueue_attention(lsa_ctx *c, const void *Q, void *out, float *lse, cudaStream_t st) {
+    const lsa_params &p = c->p;
     StageTimer ta(c, LSA_STAGE_ATTN, st);
     if (c->merged) {
         LSA_TRY(launch_merge_rows(c->topk_idx, c->topk_pos, c->topk_cnt, c->seq_off_d, p.B, p.topk, p.window,
@@ -320,18 +359,45 @@ lsa_status enqueue_step(lsa_ctx *c, bool refresh, const void *q, const float *w,
         LSA_TRY(launch_sparse_attn(Q, p.attn_dtype, c->hot, p.kv_row_stride, p.k_off, p.v_off, c->attn_rows, p.B,
                                    p.Hq, p.D, int32_t(c->row_cap), c->scale, out, lse, c->attn_ws, c->err, st));
     } else {
-        LSA_TRY(launch_sparse_attn(Q, p.attn_dtype, c->hot, p.kv_row_stride, p.k_off, p.v_off, c->topk_pos,
-                                   p.B, p.Hq, p.D, p.topk, c->scale, out, lse, c->attn_ws, c->err, st));
+        LSA_TRY(launch_sparse_attn(Q, p.attn_dtype, c->hot, p.kv_row_stride, p.k_off, p.v_off, c->topk_pos, p.B,
+                                   p.Hq, p.D, p.topk, c->scale, out, lse, c->attn_ws, c->err, st));
     }
     ta.done();
     return LSA_OK;
 }
 
-lsa_status run_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const void *Q, void *out,
-                    float *lse, cudaStream_t st) {
-    const bool refresh = (t % c->tau) == 0 || !c->refreshed;
-    if (c->use_graphs && !c->timing && c->eager_done[refresh]) {
-        const GraphKey key{refresh, q, w, Q, out, lse};
+// The kernels of one step of kind `kind` on kept set `set` (a predicting step also scans and selects into
+// the other set; its fetch is enqueued by run_step, outside any graph).
+lsa_status enqueue_step(lsa_ctx *c, int kind, int set, const void *q, const float *w, const void *Q, void *out,
+                        float *lse, cudaStream_t st) {
+    const lsa_params &p = c->p;
+    if (kind == kRefresh) {
+        LSA_TRY(enqueue_scan_select(c, q, w, set, st));
+        LSA_CUDA(cudaEventRecord(c->ev_sel, st));
+        LSA_CUDA(cudaStreamWaitEvent(c->side, c->ev_sel, 0));
+        LSA_TRY(enqueue_fetch(c, set, -1, c->side));
+        LSA_CUDA(cudaEventRecord(c->ev_gather, c->side));
+        // the top-k writes hot slots: with the cache it needs the slot assignment first
+        if (!p.full_fetch) LSA_CUDA(cudaStreamWaitEvent(st, c->ev_assign, 0));
+        StageTimer tk(c, LSA_STAGE_TOPK, st);
+        LSA_TRY(launch_topk(c->z, 1, c->seq_off_d, c->ks[set].kept_idx, c->ks[set].kept_off, p.B, p.topk,
+                            p.kept_capacity, p.full_fetch ? nullptr : c->ks[set].kept_slot, c->topk_idx, c->topk_pos,
+                            c->topk_cnt, st));
+        tk.done();
+        LSA_CUDA(cudaStreamWaitEvent(st, c->ev_gather, 0));
+        return enqueue_attention(c, Q, out, lse, st);
+    }
+    LSA_TRY(enqueue_rescore_topk(c, q, w, set, st));
+    LSA_TRY(enqueue_attention(c, Q, out, lse, st));
+    if (kind == kPredict) LSA_TRY(enqueue_scan_select(c, q, w, set ^ 1, st));
+    return LSA_OK;
+}
+
+lsa_status launch_step(lsa_ctx *c, int kind, int set, const void *q, const float *w, const void *Q, void *out,
+                       float *lse, cudaStream_t st) {
+    const int slot = kind * 2 + set;
+    if (c->use_graphs && !c->timing && c->eager_done[slot]) {
+        const GraphKey key{kind, set, q, w, Q, out, lse};
         auto it = c->graphs.find(key);
         if (it == c->graphs.end()) {
             if (c->graphs.size() >= kMaxGraphs) {
@@ -340,7 +406,7 @@ lsa_status run_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const 
             }
             LSA_CUDA(cudaStreamBeginCapture(c->cap, cudaStreamCaptureModeThreadLocal));
             const int64_t l0 = launch_count();
-            const lsa_status s = enqueue_step(c, refresh, q, w, Q, out, lse, c->cap);
+            const lsa_status s = enqueue_step(c, kind, set, q, w, Q, out, lse, c->cap);
             cudaGraph_t g = nullptr;
             const cudaError_t e = cudaStreamEndCapture(c->cap, &g);
             if (s != LSA_OK || e != cudaSuccess) {
@@ -363,11 +429,49 @@ lsa_status run_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const 
         c->launches += it->second.kernels;
     } else {
         const int64_t l0 = launch_count();
-        LSA_TRY(enqueue_step(c, refresh, q, w, Q, out, lse, st));
+        LSA_TRY(enqueue_step(c, kind, set, q, w, Q, out, lse, st));
         c->launches += launch_count() - l0;
-        c->eager_done[refresh] = true;
+        c->eager_done[slot] = true;
     }
-    if (refresh) c->refreshed = true;
+    return LSA_OK;
+}
+
+lsa_status run_step(lsa_ctx *c, int64_t t, const void *q, const float *w, const void *Q, void *out,
+                    float *lse, cudaStream_t st) {
+    const int L = c->lookahead;
+    int kind;
+    if (!c->refreshed) {
+        kind = kRefresh;
+    } else if (L == 0) {
+        kind = (t % c->tau) == 0 ? kRefresh : kListed;
+    } else if (t % c->tau == 0) {
+        // window start: the predicted set becomes current once its fetch has landed; without a prediction
+        // (the caller skipped its step) the window refreshes here
+        kind = c->predicted ? kListed : kRefresh;
+        if (c->predicted) {
+            LSA_CUDA(cudaStreamWaitEvent(st, c->ev_pend, 0));
+            c->cur ^= 1;
+            c->predicted = false;
+        }
+    } else {
+        kind = (t + L) % c->tau == 0 ? kPredict : kListed;
+    }
+    const int set = c->cur;
+    LSA_TRY(launch_step(c, kind, set, q, w, Q, out, lse, st));
+    if (kind == kRefresh) {
+        c->refreshed = true;
+        c->predicted = false;
+    } else if (kind == kPredict) {
+        // the next window's fetch and key compaction run on the side stream while this window's
+        // remaining steps run; the window's first step waits for them
+        LSA_CUDA(cudaEventRecord(c->ev_pred, st));
+        LSA_CUDA(cudaStreamWaitEvent(c->side, c->ev_pred, 0));
+        const int64_t l0 = launch_count();
+        LSA_TRY(enqueue_fetch(c, set ^ 1, set, c->side));
+        c->launches += launch_count() - l0;
+        LSA_CUDA(cudaEventRecord(c->ev_pend, c->side));
+        c->predicted = true;
+    }
     return LSA_OK;
 }
 
@@ -402,6 +506,11 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     for (int b = 0; b < p.B; ++b)
         LSA_CHECK_ARG(so[b + 1] >= so[b], "lsa_ctx_create: seq_off must be non-decreasing");
     LSA_CHECK_ARG(p.window >= 0, "lsa_ctx_create: window < 0");
+    const int tau = p.tau ? p.tau : 64;
+    LSA_CHECK_ARG(p.lookahead >= 0 && p.lookahead < tau, "lsa_ctx_create: lookahead=%d must lie in [0, tau)",
+                  p.lookahead);
+    LSA_CHECK_SUPPORTED(p.lookahead == 0 || !p.full_fetch,
+                        "lsa_ctx_create: lookahead needs the cached hot buffer (full_fetch = 0)");
     const int n_layers = p.n_layers <= 1 ? 1 : p.n_layers;
     LSA_CHECK_ARG(n_layers <= kMaxUnionLayers, "lsa_ctx_create: n_layers=%d > %d", p.n_layers, kMaxUnionLayers);
     if (n_layers > 1) {
@@ -440,7 +549,9 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     c->p = p;
     c->seq_off_h.assign(so, so + p.B + 1);
     c->p.seq_off_host = c->seq_off_h.data();
-    c->tau = p.tau ? p.tau : 64;
+    c->tau = tau;
+    c->lookahead = p.lookahead;
+    c->n_sets = p.lookahead > 0 ? 2 : 1;
     c->scale = p.scale > 0.f ? p.scale : 1.f / std::sqrt(float(p.D));
     c->cold_dev = attr.devicePointer;
     cudaGetDevice(&c->device);
@@ -471,8 +582,11 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     LSA_ALLOC(c->seq_off_d, size_t(p.B + 1) * 8);
     LSA_ALLOC(c->z, size_t(p.n_total) * 4);
     LSA_ALLOC(c->z_kept, size_t(cap) * 4);
-    LSA_ALLOC(c->kept_idx, size_t(cap) * 4);
-    LSA_ALLOC(c->kept_off, size_t(p.B + 1) * 8);
+    for (int k = 0; k < c->n_sets; ++k) {
+        LSA_ALLOC(c->ks[k].kept_idx, size_t(cap) * 4);
+        LSA_ALLOC(c->ks[k].kept_off, size_t(p.B + 1) * 8);
+        LSA_ALLOC(c->ks[k].kept_slot, size_t(cap) * 4);
+    }
     LSA_ALLOC(c->slot_of, size_t(p.n_total) * 4);
     LSA_ALLOC(c->hot, size_t(arena_rows) * p.row_bytes);
     if (n_layers > 1) {
@@ -487,10 +601,11 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     c->compact = index_score_tc_supported(p.q_dtype, p.k_dtype, cap, p.B, p.H, p.d);
     c->sc_len = int64_t(align_up(size_t(cap), 4)) + 8;
     if (c->compact)
-        for (int l = 0; l < n_layers; ++l) {
-            LSA_ALLOC(c->kc[l], size_t(cap) * p.d * elem_size(p.k_dtype));
-            if (p.k_dtype == LSA_E4M3) LSA_ALLOC(c->sc[l], size_t(c->sc_len) * 4);
-        }
+        for (int k = 0; k < c->n_sets; ++k)
+            for (int l = 0; l < n_layers; ++l) {
+                LSA_ALLOC(c->ks[k].kc[l], size_t(cap) * p.d * elem_size(p.k_dtype));
+                if (p.k_dtype == LSA_E4M3) LSA_ALLOC(c->ks[k].sc[l], size_t(c->sc_len) * 4);
+            }
     LSA_ALLOC(c->topk_idx, size_t(p.B) * p.topk * 4);
     LSA_ALLOC(c->topk_pos, size_t(p.B) * p.topk * 4);
     LSA_ALLOC(c->topk_cnt, size_t(p.B) * 4);
@@ -498,7 +613,6 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     LSA_ALLOC(c->sel_ws, c->sel_ws_bytes);
     LSA_ALLOC(c->attn_ws, c->attn_ws_bytes);
     LSA_ALLOC(c->owner, size_t(cap) * 4);
-    LSA_ALLOC(c->kept_slot, size_t(cap) * 4);
     LSA_ALLOC(c->fetched, 16);
     LSA_ALLOC(c->fetch_ws, fetch_workspace(cap));
     for (auto &sg : c->stage) {
@@ -535,15 +649,23 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
         if (ce == cudaSuccess) ce = cudaMemset(c->slot_of, 0xFF, size_t(p.n_total > 0 ? p.n_total : 1) * 4);
         if (ce == cudaSuccess) ce = cudaMemset(c->owner, 0xFF, size_t(cap) * 4);
         if (ce == cudaSuccess) ce = cudaMemset(c->fetched, 0, 16);
-        for (int l = 0; l < n_layers && c->compact; ++l) {
-            if (ce == cudaSuccess) ce = cudaMemset(c->kc[l], 0, size_t(cap) * p.d * elem_size(p.k_dtype));
-            if (ce == cudaSuccess && c->sc[l]) ce = cudaMemset(c->sc[l], 0, size_t(c->sc_len) * 4);
+        for (int k = 0; k < c->n_sets; ++k) {
+            // an empty kept set: no position, no slot
+            if (ce == cudaSuccess) ce = cudaMemset(c->ks[k].kept_off, 0, size_t(p.B + 1) * 8);
+            if (ce == cudaSuccess) ce = cudaMemset(c->ks[k].kept_slot, 0xFF, size_t(cap) * 4);
+            for (int l = 0; l < n_layers && c->compact; ++l) {
+                if (ce == cudaSuccess)
+                    ce = cudaMemset(c->ks[k].kc[l], 0, size_t(cap) * p.d * elem_size(p.k_dtype));
+                if (ce == cudaSuccess && c->ks[k].sc[l]) ce = cudaMemset(c->ks[k].sc[l], 0, size_t(c->sc_len) * 4);
+            }
         }
         if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking);
         if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking);
         if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_sel, cudaEventDisableTiming);
         if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_gather, cudaEventDisableTiming);
         if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_assign, cudaEventDisableTiming);
+        if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_pred, cudaEventDisableTiming);
+        if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&c->ev_pend, cudaEventDisableTiming);
         if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->h2d, cudaStreamNonBlocking);
         if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&c->d2h, cudaStreamNonBlocking);
         for (auto &sg : c->stage)
@@ -627,15 +749,15 @@ lsa_status lsa_ctx_get_view(lsa_ctx *c, lsa_ctx_view *v) {
     LSA_CHECK_ARG(c && v, "lsa_ctx_get_view: ctx and view required");
     v->z = c->z;
     v->z_kept = c->z_kept;
-    v->kept_idx = c->kept_idx;
-    v->kept_off = c->kept_off;
+    v->kept_idx = c->ks[c->cur].kept_idx;
+    v->kept_off = c->ks[c->cur].kept_off;
     v->slot_of = c->slot_of;
     v->hot = c->hot;
     v->topk_idx = c->topk_idx;
     v->topk_pos = c->topk_pos;
     v->topk_cnt = c->topk_cnt;
     v->err = c->err;
-    v->kept_slot = c->p.full_fetch ? nullptr : c->kept_slot;
+    v->kept_slot = c->p.full_fetch ? nullptr : c->ks[c->cur].kept_slot;
     v->owner = c->p.full_fetch ? nullptr : c->owner;
     v->fetched = c->fetched;
     v->attn_rows = c->attn_rows;
@@ -694,5 +816,18 @@ lsa_status lsa_ctx_reset_counters(lsa_ctx *c) {
 }
 
 int64_t lsa_ctx_launches(lsa_ctx *c) { return c ? c->launches : -1; }
+
+lsa_status lsa_ctx_flush_cache(lsa_ctx *c, void *stream) {
+    clear_error();
+    LSA_CHECK_ARG(c, "lsa_ctx_flush_cache: ctx required");
+    const lsa_params &p = c->p;
+    cudaStream_t st = as_stream(stream);
+    // no entry resident and no slot owned: the next refresh (or prediction) fetches every kept row; the
+    // current kept set's rows stay where they are (its steps keep reading them, and a prediction's fetch
+    // never evicts its slots)
+    LSA_CUDA(cudaMemsetAsync(c->slot_of, 0xFF, size_t(p.n_total > 0 ? p.n_total : 1) * 4, st));
+    LSA_CUDA(cudaMemsetAsync(c->owner, 0xFF, size_t(p.kept_capacity) * 4, st));
+    return LSA_OK;
+}
 
 }  // extern "C"

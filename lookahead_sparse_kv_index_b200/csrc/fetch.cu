@@ -20,6 +20,12 @@
 // warp-aggregated atomics, so slot placement may differ between runs; nothing
 // computed depends on it.  A kept list longer than the hot buffer raises
 // LSA_ERR_CAPACITY and is truncated, like lsa_gather.
+//
+// Lookahead (the next window's kept set fetched while the current window's
+// steps still attend the current set): the slots of a protected kept list
+// (the current set's kept_slot) are marked used too, so the fetch never
+// evicts a row the running steps read; entries left without a free slot
+// raise LSA_ERR_CAPACITY.
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -43,11 +49,19 @@ __global__ void __launch_bounds__(kThreads)
 fetch_mark(const int64_t *__restrict__ seq_off, const int32_t *__restrict__ kept_idx,
            const int64_t *__restrict__ kept_off, int B, int64_t cap, const int32_t *__restrict__ slot_of,
            int32_t *__restrict__ kept_slot, uint8_t *__restrict__ used, int32_t *__restrict__ new_list,
-           int32_t *__restrict__ counts, int32_t *err) {
+           int32_t *__restrict__ counts, const int32_t *__restrict__ prot_slot, const int64_t *__restrict__ prot_off,
+           int32_t *err) {
     const int64_t total = kept_off[B];
     const int64_t n = total < cap ? total : cap;
     if (total > cap && blockIdx.x == 0 && threadIdx.x == 0) raise_err(err, LSA_ERR_CAPACITY);
     const int64_t stride = int64_t(gridDim.x) * kThreads;
+    if (prot_slot) {   // slots the running steps still read
+        const int64_t pt = prot_off[B] < cap ? prot_off[B] : cap;
+        for (int64_t p = int64_t(blockIdx.x) * kThreads + threadIdx.x; p < pt; p += stride) {
+            const int32_t s = prot_slot[p];
+            if (s >= 0 && s < cap) used[s] = 1;
+        }
+    }
     for (int64_t p0 = int64_t(blockIdx.x) * kThreads; p0 < n; p0 += stride) {   // uniform per warp
         const int64_t p = p0 + threadIdx.x;
         bool is_new = false;
@@ -78,10 +92,14 @@ fetch_assign(const int64_t *__restrict__ seq_off, const int32_t *__restrict__ ke
              const int64_t *__restrict__ kept_off, int B, const int32_t *__restrict__ new_list,
              const int32_t *__restrict__ free_list, const int32_t *__restrict__ counts,
              int32_t *__restrict__ kept_slot, int32_t *__restrict__ slot_of, int32_t *__restrict__ owner,
-             int64_t *__restrict__ fetched) {
-    // free >= new whenever the kept list fits the hot buffer; the clamp keeps every slot index in range
+             int64_t *__restrict__ fetched, int32_t *err) {
+    // free >= new whenever the kept list (with the protected one) fits the hot buffer; the clamp keeps every
+    // slot index in range, and an entry left without a slot is a capacity error
     const int n_new = min(counts[0], counts[1]);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *fetched = n_new;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *fetched = n_new;
+        if (counts[0] > counts[1]) raise_err(err, LSA_ERR_CAPACITY);
+    }
     for (int i = blockIdx.x * kThreads + threadIdx.x; i < n_new; i += gridDim.x * kThreads) {
         const int32_t p = new_list[i];
         const int32_t s = free_list[i];
@@ -154,7 +172,8 @@ size_t fetch_workspace(int64_t cap) {
 lsa_status launch_fetch(const void *cold_dev, int64_t row_bytes, const int64_t *seq_off, const int32_t *kept_idx,
                         const int64_t *kept_off, int32_t B, void *hot, int64_t cap, int32_t *slot_of,
                         int32_t *owner, int32_t *kept_slot, int64_t *fetched, void *workspace, int32_t *err,
-                        cudaEvent_t assigned, cudaStream_t st) {
+                        cudaEvent_t assigned, cudaStream_t st, const int32_t *prot_slot, const int64_t *prot_off,
+                        int row_ctas) {
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint8_t *used = ws;
     int32_t *new_list = reinterpret_cast<int32_t *>(ws + align_up(size_t(cap), 256));
@@ -164,15 +183,16 @@ lsa_status launch_fetch(const void *cold_dev, int64_t row_bytes, const int64_t *
     LSA_CUDA(cudaMemsetAsync(counts, 0, 8, st));
     const int blocks = sm_count() * 4;
     fetch_mark<<<blocks, kThreads, 0, st>>>(seq_off, kept_idx, kept_off, B, cap, slot_of, kept_slot, used, new_list,
-                                            counts, err);
+                                            counts, prot_slot, prot_off, err);
     LSA_LAUNCHED("fetch_mark");
     fetch_free<<<blocks, kThreads, 0, st>>>(cap, used, free_list, counts);
     LSA_LAUNCHED("fetch_free");
     fetch_assign<<<blocks, kThreads, 0, st>>>(seq_off, kept_idx, kept_off, B, new_list, free_list, counts, kept_slot,
-                                              slot_of, owner, fetched);
+                                              slot_of, owner, fetched, err);
     LSA_LAUNCHED("fetch_assign");
     if (assigned) LSA_CUDA(cudaEventRecord(assigned, st));
-    fetch_rows<<<sm_count() * 8, kThreads, 0, st>>>(static_cast<const uint4 *>(cold_dev), row_bytes / 16, seq_off,
+    fetch_rows<<<row_ctas > 0 ? row_ctas : sm_count() * 8, kThreads, 0, st>>>(static_cast<const uint4 *>(cold_dev),
+                                                                             row_bytes / 16, seq_off,
                                                     kept_idx, kept_off, B, new_list, counts, kept_slot,
                                                     static_cast<uint4 *>(hot));
     LSA_LAUNCHED("fetch_rows");

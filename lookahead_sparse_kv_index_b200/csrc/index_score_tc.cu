@@ -13,18 +13,19 @@
 //     operand and gate weights in one of two smem slots (the first two are
 //     built by the epilogue warps while the first keys load; no separate
 //     preparation kernel);
-//   * warp 1: tcgen05.mma, M = 128 entries per instruction, into a ring of
-//     TMEM accumulators.  bf16 keys: N = H heads, the MMAs of two tiles issued
-//     interleaved.  e4m3 keys: N = 2H (both query pieces), the two 128-entry
-//     halves of a tile issued interleaved.  Issuing an MMA and passing a tile
-//     boundary both cost the single issuing thread far more than the small
-//     MMAs take on the tensor core, so the layout keeps MMAs per byte and
-//     tiles per byte low: 8 MMAs per 32 KB of keys in both cases;
+//   * warp 1: tcgen05.mma, M = 128 entries per instruction, N = H heads, into
+//     a ring of TMEM accumulators.  bf16 keys: the MMAs of two tiles issued
+//     interleaved, 8 per 32 KB of keys.  e4m3 keys: the two query pieces are
+//     further K steps over the same key slices, so the accumulator receives
+//     their sum (16 MMAs per 32 KB, the two 128-entry halves of a tile issued
+//     interleaved): one accumulator column per head, which halves what the
+//     epilogue reads from TMEM per key byte against a layout with the pieces
+//     side by side along N -- those TMEM reads, not the MMAs, paced that
+//     layout's tiles;
 //   * warps 2-9: two epilogue warpgroups (alternate tiles for bf16 keys, the
 //     two halves of every tile for e4m3 keys), one TMEM lane (= one entry)
-//     per thread: the two pieces' products added (e4m3), ReLU, gate weights,
-//     head sum in registers, one coalesced fp32 store per entry; the row
-//     scale is fetched one tile ahead.
+//     per thread: ReLU, gate weights, head sum in registers, one coalesced
+//     fp32 store per entry; the row scale comes from shared memory.
 // bf16 keys use kind::f16 (bf16 x bf16).  e4m3 keys use kind::f8f6f4 against
 // an exact two-piece e4m3 split of the bf16 query, so the keys go from HBM to
 // the tensor core untouched; the per-row key scale and the per-head
@@ -60,14 +61,14 @@ template <int KIND>
 struct Cfg;
 // Per key type: a tile is kSub sub-tiles of 128 rows (one MMA row block each);
 // a stage holds one tile, loaded as kBoxes TMA boxes of 128 bytes x kBoxRows
-// rows; the query operand has kPieces x H rows (N of the MMA).
+// rows; the query operand has H rows (N of the MMA), of d elements (bf16) or
+// two e4m3 pieces of d elements each, piece 2's rows after piece 1's (e4m3).
 template <>
 struct Cfg<BF16_D128> {
     static constexpr int kSub = 1;
     static constexpr int kStageBytes = 32768;   // 128 rows x 128 bf16
     static constexpr int kBoxes = 2;            // two 64-element (128-byte) column boxes
     static constexpr int kBoxRows = 128;
-    static constexpr int kPieces = 1;
     static constexpr int kQBytesPerHead = 256;
     static constexpr int kStages = 5;
 };
@@ -77,7 +78,6 @@ struct Cfg<BF16_D64> {
     static constexpr int kStageBytes = 16384;
     static constexpr int kBoxes = 1;
     static constexpr int kBoxRows = 128;
-    static constexpr int kPieces = 1;
     static constexpr int kQBytesPerHead = 128;
     static constexpr int kStages = 8;
 };
@@ -87,9 +87,8 @@ struct Cfg<E4M3_D128> {
     static constexpr int kStageBytes = 32768;   // 256 rows x 128 e4m3
     static constexpr int kBoxes = 1;
     static constexpr int kBoxRows = 256;
-    static constexpr int kPieces = 2;           // both query pieces in one N = 2H operand
     static constexpr int kQBytesPerHead = 256;  // two e4m3 pieces x 128
-    static constexpr int kStages = 4;           // at most twice the tile accumulators (2)
+    static constexpr int kStages = 5;           // 160 KB of keys in flight per SM, as for bf16 keys
 };
 // e4m3 keys with d = 64: 64-byte rows in the 64-byte-swizzled K-major layout (the
 // 128-byte swizzle needs 128-byte rows); 256-row tiles of 16 KB, each sub-tile
@@ -101,9 +100,8 @@ struct Cfg<E4M3_D64> {
     static constexpr int kStageBytes = 16384;   // 256 rows x 64 e4m3
     static constexpr int kBoxes = 1;
     static constexpr int kBoxRows = 256;
-    static constexpr int kPieces = 2;
     static constexpr int kQBytesPerHead = 128;  // two e4m3 pieces x 64
-    static constexpr int kStages = 8;           // a multiple of the tile accumulators (2, 4 or 8)
+    static constexpr int kStages = 10;          // 160 KB of keys in flight per SM, as for bf16 keys
 };
 
 // Key row bytes, and where 16-byte chunk c of row r of a stage sits: the TMA
@@ -130,7 +128,8 @@ constexpr int kEpiWarps = 8;
 constexpr int kRel = 8;               // query-slot release barriers, by sequence ordinal mod kRel
 constexpr int kRows = 128;            // rows of one MMA (M) and of a sub-tile
 constexpr int kAccMax = 8;            // TMEM accumulator stages at most
-constexpr int kScaleSlotsMax = 16;    // row-scale ring slots at most (stages + accumulators)
+constexpr int kScaleSlotsMax = 24;    // row-scale ring slots at most (stages + accumulators)
+constexpr int kDoneMax = 24;          // tile-completion barriers at most (per accumulator + per stage)
 constexpr int kMaxB = 512;            // sequences per launch on this path
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
 
@@ -138,12 +137,11 @@ template <int KIND>
 __host__ __device__ constexpr int tile_rows() {
     return kRows * Cfg<KIND>::kSub;
 }
-// TMEM columns of one sub-tile's accumulator (fp32, one per head and query
-// piece: e4m3 keys give columns [0, H) for piece 1 and [H, 2H) for piece 2,
-// added by the epilogue before the ReLU) and of one tile's.
+// TMEM columns of one sub-tile's accumulator (fp32, one per head: with e4m3
+// keys the two query pieces accumulate into the same column) and of one tile's.
 template <int KIND, int H>
 __host__ __device__ constexpr int sub_cols() {
-    return H * Cfg<KIND>::kPieces;
+    return H;
 }
 template <int KIND, int H>
 __host__ __device__ constexpr int tile_cols() {
@@ -358,20 +356,18 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     constexpr uint32_t NCOL = tmem_cols(KACC * TILEC);
     static_assert(G >= 1 && G <= KACC / 2, "the epilogue must own accumulators while a group is issued");
     static_assert(S >= G, "a group waits for G filled stages");
-    // One commit per tile tells both the epilogue (accumulator ready) and the producer (stage free)
-    // that the tile's MMAs completed.  A parity wait is only unambiguous while the barrier cannot
-    // complete a second phase past the one waited for.  Per accumulator (S <= KACC): the next tile
-    // on the same accumulator needs this tile's epilogue release, and the producer's wait for tile
-    // j - S sees no other tile of that accumulator before j.  With more stages than accumulators
-    // (e4m3 keys: 4 stages, 2 accumulators) tile j - S + KACC shares the accumulator and could
-    // complete while a slow producer (listed gathers) has not yet polled for tile j - S: there the
-    // barrier is per stage, whose next use is the producer's own load; the epilogue's wait stays
-    // unambiguous because tile i + S needs every epilogue warp's release of tile i + S - KACC >= i.
+    // The epilogue warpgroups take alternate tiles (each warp has two tile times for one tile: a
+    // warpgroup's wait / TMEM load / arithmetic chain per tile paced the kernel when both warpgroups
+    // worked on every tile).  The MMA commits each tile's completion to a barrier per accumulator
+    // (the epilogue waits there: the next phase is the tile KACC later, whose MMA needs this tile's
+    // release by the waiting warpgroup itself).  A parity wait is only unambiguous while the barrier
+    // cannot complete a second phase past the one waited for: the producer's wait for tile j - S may
+    // share that barrier when S <= KACC (its next phase, tile j - S + KACC >= j, needs the producer's
+    // own load of tile j); with more stages than accumulators tile j - S + KACC could complete before a
+    // slow producer polls, so the MMA also commits to a barrier per stage, whose next phase is again
+    // the producer's own load.
     constexpr bool kStageDone = S > KACC;
-    constexpr int NDONE = kStageDone ? S : KACC;
-    static_assert(NDONE <= kAccMax, "completion barriers");
-    static_assert(!kStageDone || (S % KACC == 0 && C::kSub == 2),
-                  "per-stage completion needs every epilogue warp on every tile, in order");
+    static_assert(KACC + (kStageDone ? S : 0) <= kDoneMax, "completion barriers");
     // e4m3 keys: the per-row scales of each tile go to a shared-memory ring by cp.async (the
     // producer warp), never through a register load of an epilogue warp, whose wait on its TMEM
     // loads would otherwise also wait for that HBM load.  Slot j % RS holds tile j's scales; it is
@@ -390,10 +386,11 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
     uint64_t *full = reinterpret_cast<uint64_t *>(qimg + 2 * QIMG);  // [S] stage loaded
     uint64_t *qfull = full + S;                                   // [2] query slot built
     uint64_t *qrel = qfull + 2;                                   // [kRel] by sequence ordinal
-    // [NDONE] the MMAs of a tile completed (per accumulator, or per stage when S > KACC): its
-    // accumulator is ready and its stage is free
+    // the MMAs of a tile completed: [KACC] its accumulator is ready (and, with S <= KACC, its stage
+    // free); then, with S > KACC, [S] its stage is free
     uint64_t *tdone = qrel + kRel;
-    uint64_t *tempty = tdone + kAccMax;                           // [KACC] accumulator read by the epilogue
+    uint64_t *tfree = tdone + KACC;
+    uint64_t *tempty = tdone + kDoneMax;                          // [KACC] accumulator read by the epilogue
     uint64_t *drain = tempty + kAccMax;
     uint64_t *sfull = drain + 1;                                  // [RS] row scales of a tile landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfull + kScaleSlotsMax);
@@ -448,8 +445,11 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         for (int s = 0; s < 2; ++s) mbar_init(&qfull[s], 1);
         for (int s = 0; s < kRel; ++s) mbar_init(&qrel[s], 1 + kEpiWarps);
         // an accumulator is released by the warps that read it: one warpgroup per 128-row sub-tile
-        for (int s = 0; s < NDONE; ++s) mbar_init(&tdone[s], 1);
-        for (int s = 0; s < KACC; ++s) mbar_init(&tempty[s], 4 * C::kSub);
+        for (int s = 0; s < KACC; ++s) mbar_init(&tdone[s], 1);
+        if (kStageDone)
+            for (int s = 0; s < S; ++s) mbar_init(&tfree[s], 1);
+        // an accumulator is released by the four warps of the warpgroup that read it
+        for (int s = 0; s < KACC; ++s) mbar_init(&tempty[s], 4);
         mbar_init(drain, 1);
         // full mode: one arrival (the bulk copy's expect_tx, or lane 0 after the copies landed); listed
         // mode: one cp.async-tracked arrival per producer lane
@@ -475,8 +475,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         // builds the query operand of a new sequence (ordinal o) into slot o & 1
         // local tile j may be loaded once the MMA of tile j - S (same stage) has completed
         // completion barrier and parity of local tile i
-        auto done_bar = [&](int64_t i) -> uint64_t * { return &tdone[int(i % NDONE)]; };
-        auto done_par = [&](int64_t i) -> uint32_t { return uint32_t((i / NDONE) & 1); };
+        auto done_bar = [&](int64_t i) -> uint64_t * { return kStageDone ? &tfree[int(i % S)] : &tdone[int(i % KACC)]; };
+        auto done_par = [&](int64_t i) -> uint32_t { return uint32_t((i / (kStageDone ? S : KACC)) & 1); };
         auto stage_free_test = [&](int64_t j) -> bool {
             return j < S || mbar_test_wait(done_bar(j - S), done_par(j - S));
         };
@@ -641,7 +641,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 const int gn = int(gend - t < G ? gend - t : G);
                 uint64_t a_d[G];
                 uint32_t d_t[G];
-                int done_of[G];   // completion barrier of each tile of the group
+                int acc_of[G], st_of[G];   // accumulator and stage of each tile of the group
 #pragma unroll
                 for (int u = 0; u < G; ++u) {
                     if (u >= gn) break;
@@ -649,7 +649,8 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                     if (!mbar_wait(&full[st], ph, abort_v, kWaitLimitNs)) { ok = false; break; }
                     a_d[u] = a_cur;
                     d_t[u] = tmem_base + uint32_t(acc * TILEC);
-                    done_of[u] = kStageDone ? st : acc;
+                    acc_of[u] = acc;
+                    st_of[u] = st;
                     a_cur += kStageStep;
                     if (++st == S) { st = 0; ph ^= 1; a_cur = a_desc0; }
                     if (++acc == KACC) { acc = 0; aph ^= 1; }
@@ -675,27 +676,35 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                                 mma_f16(d_t[u], a_d[u] + uint64_t((kk * 32) >> 4), b_cur + uint64_t((kk * 32) >> 4),
                                         IDESC, kk > 0);
                 } else if (KIND == E4M3_D64) {
-                    // as below, with 64-byte rows: the halves are 8 KB apart, two K = 32 steps
-#pragma unroll
-                    for (int kk = 0; kk < 2; ++kk)
-#pragma unroll
-                        for (int sub = 0; sub < 2; ++sub)
-                            mma_f8(d_t[0] + uint32_t(sub * SUBC), a_d[0] + uint64_t((sub * 8192 + kk * 32) >> 4),
-                                   b_cur + uint64_t((kk * 32) >> 4), IDESC, kk > 0);
-                } else {
-                    // the two 128-row halves of the tile (16 KB apart in the stage) into their own
-                    // column blocks, chains interleaved; N = 2H covers both query pieces
+                    // as below, with 64-byte rows: the halves are 8 KB apart; K steps 0-1 piece 1, 2-3
+                    // piece 2 (its rows H*64 bytes after piece 1's) over the same two key slices
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
                         for (int sub = 0; sub < 2; ++sub)
-                            mma_f8(d_t[0] + uint32_t(sub * SUBC), a_d[0] + uint64_t((sub * 16384 + kk * 32) >> 4),
-                                   b_cur + uint64_t((kk * 32) >> 4), IDESC, kk > 0);
+                            mma_f8(d_t[0] + uint32_t(sub * SUBC),
+                                   a_d[0] + uint64_t((sub * 8192 + (kk & 1) * 32) >> 4),
+                                   b_cur + uint64_t(((kk >> 1) * (H * 64) + (kk & 1) * 32) >> 4), IDESC, kk > 0);
+                } else {
+                    // the two 128-row halves of the tile (16 KB apart in the stage) into their own
+                    // accumulators, chains interleaved; K steps 0-3 take query piece 1, 4-7 piece 2 (its rows
+                    // H*128 bytes after piece 1's) over the same four key slices: the accumulator holds
+                    // (p1 + p2) . k = q 2^e . k
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+                        for (int sub = 0; sub < 2; ++sub)
+                            mma_f8(d_t[0] + uint32_t(sub * SUBC),
+                                   a_d[0] + uint64_t((sub * 16384 + (kk & 3) * 32) >> 4),
+                                   b_cur + uint64_t(((kk >> 2) * (H * 128) + (kk & 3) * 32) >> 4), IDESC, kk > 0);
                 }
                 issued = true;
 #pragma unroll
                 for (int u = 0; u < G; ++u)
-                    if (u < gn) mma_commit(&tdone[done_of[u]]);   // accumulator ready, stage free
+                    if (u < gn) {
+                        mma_commit(&tdone[acc_of[u]]);                  // accumulator ready
+                        if (kStageDone) mma_commit(&tfree[st_of[u]]);   // stage free
+                    }
                 if (t == gend) mma_commit(&qrel[qn % kRel]);      // this sequence's operand is no longer read
             }
             if (issued) {
@@ -710,11 +719,9 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
         const int ew = warp - 2;              // 0..7
         const int grp = ew >> 2;              // warpgroup
         const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
-        // 128-row tiles: the warpgroups take alternate tiles; 256-row tiles: every tile, warpgroup g
-        // its sub-tile g
-        constexpr int kStep = C::kSub == 2 ? 1 : kEpiGroups;
-        const int sub = C::kSub == 2 ? grp : 0;
-        const int64_t tfirst = C::kSub == 2 ? t0 : t0 + grp;
+        // the warpgroups take alternate tiles, every sub-tile of a tile (one TMEM round trip)
+        constexpr int kStep = kEpiGroups;
+        const int64_t tfirst = t0 + grp;
         int b = 0, cur = -1, ord = -1, released = 0;
         int64_t row0, row_end;
         // a sequence ordinal this warp will not read again frees its slot (1 of the 8 epilogue arrivals)
@@ -763,9 +770,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                 if (!__all_sync(0xffffffffu, ok)) break;
             }
             const float *wq = wsm + (ord & 1) * H;
-            const int64_t row = row0 + sub * kRows + quarter * 32 + lane;   // entry (full) or list position
-            ok = kStageDone ? mbar_wait(&tdone[int(i % S)], uint32_t((i / S) & 1), abort_v, kWaitLimitNs)
-                            : mbar_wait(&tdone[acc], aph, abort_v, kWaitLimitNs);
+            ok = mbar_wait(&tdone[acc], aph, abort_v, kWaitLimitNs);
             // the row scales landed long before (loaded with the keys); read before the release
             if (kScales) ok = ok && mbar_wait(&sfull[i % RS], uint32_t((i / RS) & 1), abort_v, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) break;   // keep the warp converged for tcgen05.ld
@@ -775,19 +780,24 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                                                                 scale_len, k_scale))
                                  ? int(row0 & 3)
                                  : 0;
-            const float sc = kScales ? s_scale[int(i % RS) * SS + soff + sub * kRows + quarter * 32 + lane] : 1.f;
-            const uint32_t taddr =
-                tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * TILEC + sub * SUBC);
-            float za = 0.f, zb = 0.f, zc = 0.f, zd = 0.f;   // four short dependency chains
-            if (C::kPieces == 1) {
+            const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * TILEC);
+            // the sub-tiles one after the other through the same registers (a whole 256-row tile's row,
+            // 2 H columns, does not fit beside the rest in the 168 registers of a 320-thread CTA); the
+            // accumulator is released once the last sub-tile's columns are in registers
+#pragma unroll
+            for (int sub = 0; sub < C::kSub; ++sub) {
                 uint32_t r[H];
 #pragma unroll
                 for (int c = 0; c < H / 16; ++c)
-                    tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[c * 16]));
+                    tmem_ld_32x32b_x16(taddr + sub * SUBC + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[c * 16]));
                 tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[acc]);
+                const float sc = kScales ? s_scale[int(i % RS) * SS + soff + sub * kRows + quarter * 32 + lane] : 1.f;
+                if (sub == C::kSub - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[acc]);
+                }
+                float za = 0.f, zb = 0.f, zc = 0.f, zd = 0.f;   // four short dependency chains
 #pragma unroll
                 for (int j = 0; j < H; j += 4) {
                     const float4 wv = *reinterpret_cast<const float4 *>(wq + j);
@@ -796,31 +806,13 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                     zc = fmaf(wv.z, fmaxf(__uint_as_float(r[j + 2]), 0.f), zc);
                     zd = fmaf(wv.w, fmaxf(__uint_as_float(r[j + 3]), 0.f), zd);
                 }
-            } else {
-                // both pieces' columns in one round trip, so that the accumulator is released
-                // before any arithmetic (only two tile accumulators fit in TMEM)
-                uint32_t r[2 * H];
-#pragma unroll
-                for (int c = 0; c < 2 * H / 16; ++c)
-                    tmem_ld_32x32b_x16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[c * 16]));
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[acc]);
-#pragma unroll
-                for (int j = 0; j < H; j += 4) {
-                    const float4 wv = *reinterpret_cast<const float4 *>(wq + j);
-                    za = fmaf(wv.x, fmaxf(__uint_as_float(r[j]) + __uint_as_float(r[H + j]), 0.f), za);
-                    zb = fmaf(wv.y, fmaxf(__uint_as_float(r[j + 1]) + __uint_as_float(r[H + j + 1]), 0.f), zb);
-                    zc = fmaf(wv.z, fmaxf(__uint_as_float(r[j + 2]) + __uint_as_float(r[H + j + 2]), 0.f), zc);
-                    zd = fmaf(wv.w, fmaxf(__uint_as_float(r[j + 3]) + __uint_as_float(r[H + j + 3]), 0.f), zd);
+                float zs = (za + zb) + (zc + zd);
+                const int64_t row = row0 + sub * kRows + quarter * 32 + lane;   // entry (full) or list position
+                if (row < row_end) {
+                    if (kScales) zs *= sc;
+                    z[row] = zs;
+                    if (I) I[row] = 1.f / (1.f + expf(-zs));
                 }
-            }
-            float zs = (za + zb) + (zc + zd);
-            if (row < row_end) {
-                if (kScales) zs *= sc;
-                z[row] = zs;
-                if (I) I[row] = 1.f / (1.f + expf(-zs));
             }
         }
         release_to(nord);   // every sequence of the range
@@ -858,7 +850,7 @@ template <int KIND, int H>
 size_t smem_bytes(int B) {
     using C = Cfg<KIND>;
     return 1024 + size_t(C::kStages) * C::kStageBytes + 2 * qimg_bytes<KIND, H>() +
-           (C::kStages + 2 + kRel + 2 * kAccMax + 1 + kScaleSlotsMax) * 8 + 16 + 16 + 2 * H * 4 +
+           (C::kStages + 2 + kRel + kDoneMax + kAccMax + 1 + kScaleSlotsMax) * 8 + 16 + 16 + 2 * H * 4 +
            size_t(B + 1) * 24 + 16 +
            (is_e4m3(KIND) ? size_t(C::kStages + acc_tiles<KIND, H>()) * (tile_rows<KIND>() + 8) * 4 : 0) +
            64;

@@ -36,10 +36,13 @@ void clear_error();
         }                                     \
     } while (0)
 
+// (a failed call's error is also taken off the runtime's last-error slot, so that it is not reported
+// again by the next launch check)
 #define LSA_CUDA(call)                                                              \
     do {                                                                            \
         cudaError_t e_ = (call);                                                    \
         if (e_ != cudaSuccess) {                                                    \
+            cudaGetLastError();                                                     \
             ::lsa::set_error("%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), \
                              __FILE__, __LINE__);                                   \
             return LSA_ERR_CUDA;                                                    \
@@ -116,7 +119,8 @@ size_t fetch_workspace(int64_t cap);
 lsa_status launch_fetch(const void *cold_dev, int64_t row_bytes, const int64_t *seq_off, const int32_t *kept_idx,
                         const int64_t *kept_off, int32_t B, void *hot, int64_t cap, int32_t *slot_of,
                         int32_t *owner, int32_t *kept_slot, int64_t *fetched, void *workspace, int32_t *err,
-                        cudaEvent_t assigned, cudaStream_t st);
+                        cudaEvent_t assigned, cudaStream_t st, const int32_t *prot_slot = nullptr,
+                        const int64_t *prot_off = nullptr, int row_ctas = 0);
 lsa_status launch_gather(const void *cold_dev, int64_t row_bytes, const int64_t *seq_off,
                          int64_t n_total, const int32_t *kept_idx, const int64_t *kept_off,
                          int32_t B, void *hot, int64_t hot_capacity, int32_t *slot_of,

@@ -37,7 +37,7 @@ EXPORTS = [
     "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
     "lsa_ctx_set_graphs", "lsa_ctx_set_timing", "lsa_ctx_stage_times", "lsa_ctx_reset_counters",
     "lsa_ctx_launches", "lsa_selftest_bounded_wait", "lsa_index_union", "lsa_query_encode",
-    "lsa_attn_set_merge", "lsa_struct_size",
+    "lsa_attn_set_merge", "lsa_struct_size", "lsa_ctx_flush_cache",
 ]
 
 
@@ -55,7 +55,7 @@ class Params(ctypes.Structure):
         ("n_total", i64), ("seq_off_host", P), ("k_dev", P), ("k_scale_dev", P), ("cold_host", P),
         ("row_bytes", i64), ("kv_row_stride", i64), ("k_off", i64), ("v_off", i64), ("kept_capacity", i64),
         ("full_fetch", i32), ("window", i32), ("hca_rows", P), ("hca_off_host", P),
-        ("n_layers", i32), ("k_dev_layers", P), ("k_scale_layers", P),
+        ("n_layers", i32), ("k_dev_layers", P), ("k_scale_layers", P), ("lookahead", i32),
     ]
 
 
@@ -96,6 +96,7 @@ _sig("lsa_ctx_set_timing", i32, [P, i32])
 _sig("lsa_ctx_stage_times", i32, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)])
 _sig("lsa_ctx_reset_counters", i32, [P])
 _sig("lsa_ctx_launches", i64, [P])
+_sig("lsa_ctx_flush_cache", i32, [P, P])
 _sig("lsa_selftest_bounded_wait", i32, [i64, P, P, P])
 _sig("lsa_index_union", i32, [ctypes.POINTER(P), i32, i64, P, P])
 _sig("lsa_query_encode", i32, [P, i32, i32, P, i32, P, i32, i32, P, P, i32, P, P, P])
@@ -231,11 +232,12 @@ class Context:
 
     def __init__(self, *, B, H, d, q_dtype, k_dtype, Hq, D, attn_dtype, topk, seq_off_host, keys, k_scale,
                  cold_host, row_bytes, kv_row_stride, k_off, v_off, kept_capacity, tau=64, scale=0.0,
-                 full_fetch=False, window=0, hca_rows=None, hca_off_host=None, layers=None):
+                 full_fetch=False, window=0, hca_rows=None, hca_off_host=None, layers=None, lookahead=0):
         """window / hca_rows / hca_off_host: the always-resident context merged into the attention set
         (see lsa_attn_set_merge); hca_rows is a host or device tensor of HCA rows in the cold-pool row format.
         layers: [(keys, k_scale), ...] of indexer layers 1 .. L-1 (layer 0 is keys / k_scale) for the OR-mode
-        union in the cadence; steps then take q [L, B, H, d] and w [L, B, H]."""
+        union in the cadence; steps then take q [L, B, H, d] and w [L, B, H].
+        lookahead: predict each window's kept set this many steps ahead and fetch it meanwhile (see lsa.h)."""
         self._seq_off = torch.as_tensor(seq_off_host, dtype=torch.int64).contiguous()
         self._hca_off = None if hca_off_host is None else torch.as_tensor(hca_off_host, dtype=torch.int64).contiguous()
         n_total = int(self._seq_off[-1])
@@ -244,6 +246,7 @@ class Context:
                              _ptr(cold_host), row_bytes, kv_row_stride, k_off, v_off, kept_capacity,
                              int(bool(full_fetch)), int(window), _ptr(hca_rows),
                              None if self._hca_off is None else self._hca_off.data_ptr())
+        self.params.lookahead = int(lookahead)
         self.n_layers = 1
         if layers:
             self.n_layers = 1 + len(layers)
@@ -300,6 +303,10 @@ class Context:
 
     def launches(self) -> int:
         return int(_L.lsa_ctx_launches(self.handle))
+
+    def flush_cache(self, stream=None):
+        """Empty the hot-buffer cache: the next refresh or prediction fetches every kept row."""
+        _check(_L.lsa_ctx_flush_cache(self.handle, _stream(stream)), "lsa_ctx_flush_cache")
 
     def fetched(self) -> int:
         """Rows the last refresh fetched from the cold pool (synchronises the device)."""

@@ -87,7 +87,7 @@ def decoded(raw: np.ndarray, dtype: str) -> np.ndarray:
     return oracle.decode(raw, dtype)
 
 
-def make_context(wl, dev, lsa, kept_capacity=None, tau=64, full_fetch=False):
+def make_context(wl, dev, lsa, kept_capacity=None, tau=64, full_fetch=False, lookahead=0):
     cap = kept_capacity or max(64, int(0.4 * wl.n_total) + 64)
     if wl.n_total <= 65536:
         cap = kept_capacity or wl.n_total + 64   # small cases may keep more than half the entries
@@ -95,33 +95,40 @@ def make_context(wl, dev, lsa, kept_capacity=None, tau=64, full_fetch=False):
                        attn_dtype=wl.attn_dtype, topk=wl.topk, seq_off_host=wl.seq_off, keys=dev["keys"],
                        k_scale=dev["k_scale"], cold_host=dev["cold"], row_bytes=wl.row_bytes,
                        kv_row_stride=wl.row_stride, k_off=wl.k_off, v_off=wl.v_off, kept_capacity=cap, tau=tau,
-                       scale=wl.scale, full_fetch=full_fetch)
+                       scale=wl.scale, full_fetch=full_fetch, lookahead=lookahead)
 
 
 def check_hot_cache(ctx, wl, lsa, gpu):
-    """The hot buffer after a refresh: every kept entry's row sits in its slot byte for byte,
-    slot_of and owner are inverse maps, and the top-k slots are the chosen entries' slots."""
+    """The hot buffer after a step: every kept entry's row sits in the slot its kept position names (the slot
+    the attention reads), byte for byte, each in its own slot; the top-k slots are those of the chosen
+    entries; slot_of and owner are inverse maps and every resident row is valid.  (After a cache flush with
+    lookahead, the current set's rows stay in their slots while slot_of forgets them.)"""
     v = ctx.view()
     cap = ctx.kept_capacity
     slot_of = lsa.device_view(v.slot_of, wl.n_total, torch.int32).cpu().numpy()
     hot = lsa.device_view(v.hot, cap * ctx.row_bytes, torch.uint8).cpu().numpy().reshape(cap, ctx.row_bytes)
     cold = np.ascontiguousarray(wl.cold).view(np.uint8).reshape(wl.n_total, ctx.row_bytes)
-    b_of = np.repeat(np.arange(wl.B), np.diff(gpu["kept_off"]))[: len(gpu["kept_idx"])]
+    nk = len(gpu["kept_idx"])
+    b_of = np.repeat(np.arange(wl.B), np.diff(gpu["kept_off"]))[:nk]
     ent = wl.seq_off[:-1][b_of] + gpu["kept_idx"]
-    slots = slot_of[ent]
+    if v.kept_slot:
+        slots = lsa.device_view(v.kept_slot, nk, torch.int32).cpu().numpy()
+    else:                                    # every kept row fetched into kept order
+        slots = slot_of[ent]
     assert (slots >= 0).all()
     assert len(np.unique(slots)) == len(slots)
     assert np.array_equal(hot[slots], cold[ent])
     if v.owner:
         owner = lsa.device_view(v.owner, cap, torch.int32).cpu().numpy()
-        assert np.array_equal(owner[slots], ent)
         res = np.nonzero(slot_of >= 0)[0]
         assert np.array_equal(owner[slot_of[res]], res)
         assert np.array_equal(hot[slot_of[res]], cold[res])   # rows kept resident stay valid
     for b in range(wl.B):
         c = gpu["topk_cnt"][b]
-        e = wl.seq_off[b] + gpu["topk_idx"][b][:c]
-        assert np.array_equal(gpu["topk_pos"][b][:c], slot_of[e])
+        lo, hi = gpu["kept_off"][b], min(gpu["kept_off"][b + 1], nk)
+        pos = lo + np.searchsorted(gpu["kept_idx"][lo:hi], gpu["topk_idx"][b][:c])
+        assert np.array_equal(gpu["kept_idx"][pos], gpu["topk_idx"][b][:c])
+        assert np.array_equal(gpu["topk_pos"][b][:c], slots[pos])
 
 
 def read_ctx(ctx, wl, lsa):
@@ -192,13 +199,16 @@ def check_decode_step(wl, t, q_t, w_t, Q_t, gpu, out_gpu, lse_gpu, z_refresh, re
     return report
 
 
-def run_decode_and_check(wl, steps, tau, lsa, kept_capacity=None, full_fetch=False):
-    """Drive the context and the oracle decoder over `steps`; check every listed step."""
+def run_decode_and_check(wl, steps, tau, lsa, kept_capacity=None, full_fetch=False, lookahead=0, flush_at=()):
+    """Drive the context and the oracle decoder over `steps` (plus every window's first step and, with
+    lookahead, every prediction step: both sides skip the same steps); check every step in `steps`.
+    flush_at: steps before which the hot-buffer cache is emptied (a cold start)."""
     from oracle.stepper import OracleDecoder
 
     dev = synth.to_torch(wl)
-    ctx = make_context(wl, dev, lsa, kept_capacity=kept_capacity, tau=tau, full_fetch=full_fetch)
-    dec = OracleDecoder(wl, tau=tau)
+    ctx = make_context(wl, dev, lsa, kept_capacity=kept_capacity, tau=tau, full_fetch=full_fetch,
+                       lookahead=lookahead)
+    dec = OracleDecoder(wl, tau=tau, lookahead=lookahead)
     out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.float32 if wl.attn_dtype == "f32" else torch.int16,
                       device="cuda")
     lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device="cuda")
@@ -206,14 +216,16 @@ def run_decode_and_check(wl, steps, tau, lsa, kept_capacity=None, full_fetch=Fal
     z_refresh = None
     last = max(steps)
     for t in range(last + 1):
-        if t not in steps and t % tau != 0:
+        predict = lookahead > 0 and t % tau != 0 and (t + lookahead) % tau == 0
+        if t not in steps and t % tau != 0 and not predict:
             continue
+        if t in flush_at:
+            ctx.flush_cache()
         q_t, w_t, Q_t = wl.step_inputs(t)
         ctx.step(t, synth.raw_to_torch(q_t), torch.from_numpy(w_t).cuda(), synth.raw_to_torch(Q_t), out, lse)
         torch.cuda.synchronize()
         res_o = dec.step(t, q_t, w_t, Q_t)
-        if "z" in res_o:
-            z_refresh = res_o["z"]
+        z_refresh = res_o["z_sel"]   # the scores the current kept set was selected on
         if t in steps:
             gpu = read_ctx(ctx, wl, lsa)
             assert gpu["err"] == 0

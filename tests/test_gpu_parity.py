@@ -459,6 +459,25 @@ def test_hot_cache_fetches_only_new_rows(lsa):
         ctx.close()
 
 
+@pytest.mark.parametrize("key_dtype", ["bf16", "e4m3"])
+def test_decode_lookahead_matches_oracle(lsa, key_dtype):
+    """Lookahead L = 3, tau = 8, every step of three windows: window 1's set predicted at step 5 and fetched
+    while steps 5-7 attend window 0's set, current from step 8; the cache emptied before the prediction at
+    step 13, so its fetch brings every kept row (a cold start) while steps 13-15 still read theirs."""
+    wl = synth.small_ragged(key_dtype=key_dtype)
+    reps = run_decode_and_check(wl, list(range(24)), 8, lsa, lookahead=3, flush_at=(13,))
+    assert len(reps) == 24
+    assert max(r["attn_rel"] for r in reps) <= ATTN_TOL["bf16"]
+
+
+def test_decode_lookahead_skipped_prediction_refreshes(lsa):
+    """A run that skips window 2's prediction step (13) refreshes at step 16, like the plain cadence."""
+    wl = synth.small_ragged(key_dtype="e4m3")
+    steps = [t for t in range(20) if t != 13]
+    reps = run_decode_and_check(wl, steps, 8, lsa, lookahead=3)
+    assert len(reps) == len(steps)
+
+
 def test_decode_step_host_equals_device(lsa):
     wl = synth.small_ragged(key_dtype="e4m3")
     from gpu_cases import make_context
@@ -553,6 +572,14 @@ def test_decode_full_size(lsa, name):
     wl = synth.WORKLOADS[name]()
     reps = run_decode_and_check(wl, [0, 1, 63], 64, lsa, kept_capacity=int(0.2 * wl.n_total))
     print(name, reps)
+
+
+def test_decode_lookahead_full_size(lsa):
+    """The 500K-token context with lookahead 16: window 1 predicted at step 48 and current from step 64."""
+    wl = synth.ctx500k()
+    reps = run_decode_and_check(wl, [0, 47, 48, 49, 63, 64, 65], 64, lsa, kept_capacity=int(0.2 * wl.n_total),
+                                lookahead=16)
+    assert len(reps) == 7
 
 
 def test_decode_ragged_serving_batch(lsa):

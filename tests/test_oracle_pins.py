@@ -453,6 +453,39 @@ def test_decoder_tau_cadence_and_kept_superset():
     assert "z" in r4                                       # refresh again at t = tau
 
 
+def test_decoder_lookahead_cadence():
+    """Lookahead L = 2, tau = 4: steps 0-3 run exactly the plain cadence's window 0 (steps 2 and 3 still use
+    its kept set); step 2 predicts window 1's set, which equals a plain refresh given step 2's query; step 4
+    makes it current without a refresh and ranks it by the listed scores of step 4's query; a run that skips
+    the prediction step (6) refreshes at 8 like the plain cadence; a run whose first step is a prediction step
+    only refreshes there."""
+    wl = synth.small_ragged(lengths=(300, 700), topk=64, Hq=4, D=64)
+    tau, L = 4, 2
+    la = OracleDecoder(wl, tau=tau, lookahead=L)
+    plain = OracleDecoder(wl, tau=tau)
+    res = {t: la.step(t, *wl.step_inputs(t)) for t in (0, 1, 2, 3, 4, 5, 8)}   # step 6 skipped
+    for t in range(4):
+        r = plain.step(t, *wl.step_inputs(t))
+        for key in ("kept_idx", "kept_off", "topk_idx", "topk_cnt", "out", "lse"):
+            assert np.array_equal(res[t][key], r[key]), (t, key)
+    assert "z_pred" in res[2] and all("z_pred" not in res[t] for t in (0, 1, 3, 4, 5, 8))
+    q2, w2, _ = wl.step_inputs(2)
+    q4, w4, Q4 = wl.step_inputs(4)
+    ref = OracleDecoder(wl, tau=tau).step(0, q2, w2, Q4)          # a refresh from step 2's query
+    assert np.array_equal(res[4]["kept_idx"], ref["kept_idx"])
+    assert np.array_equal(res[4]["kept_off"], ref["kept_off"])
+    assert "z" not in res[4] and np.array_equal(res[4]["z_sel"], res[2]["z_pred"])
+    zk4 = oracle.index_score_list(q4, wl.q_dtype, w4, wl.keys, wl.key_dtype, wl.k_scale, wl.seq_off,
+                                  ref["kept_idx"], ref["kept_off"], wl.H, wl.d)
+    tk4, _ = oracle.topk(zk4, ref["kept_idx"], ref["kept_off"], wl.topk)
+    assert np.array_equal(res[4]["topk_idx"], tk4)
+    assert np.array_equal(res[5]["kept_idx"], res[4]["kept_idx"])   # the window keeps its set
+    r8 = OracleDecoder(wl, tau=tau).step(8, *wl.step_inputs(8))     # no prediction ran: a refresh at 8
+    assert "z" in res[8] and np.array_equal(res[8]["kept_idx"], r8["kept_idx"])
+    first = OracleDecoder(wl, tau=tau, lookahead=L).step(2, *wl.step_inputs(2))
+    assert "z" in first and "z_pred" not in first
+
+
 def test_layered_decoder_reduces_to_one_layer_and_keeps_the_or():
     """Three copies of one indexer layer give exactly the one-layer decode (the union of equal scores is
     that score); with three different layers every layer's own kept set lies inside the union's, and the
