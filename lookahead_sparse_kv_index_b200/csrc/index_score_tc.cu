@@ -13,19 +13,20 @@
 //     operand and gate weights in one of two smem slots (the first two are
 //     built by the epilogue warps while the first keys load; no separate
 //     preparation kernel);
-//   * warp 1: tcgen05.mma, M = 128 entries per instruction, N = H heads, into
-//     a ring of TMEM accumulators.  bf16 keys: the MMAs of two tiles issued
-//     interleaved, 8 per 32 KB of keys.  e4m3 keys: the two query pieces are
-//     further K steps over the same key slices, so the accumulator receives
-//     their sum (16 MMAs per 32 KB, the two 128-entry halves of a tile issued
-//     interleaved): one accumulator column per head, which halves what the
-//     epilogue reads from TMEM per key byte against a layout with the pieces
-//     side by side along N -- those TMEM reads, not the MMAs, paced that
-//     layout's tiles;
-//   * warps 2-9: two epilogue warpgroups (alternate tiles for bf16 keys, the
-//     two halves of every tile for e4m3 keys), one TMEM lane (= one entry)
-//     per thread: ReLU, gate weights, head sum in registers, one coalesced
-//     fp32 store per entry; the row scale comes from shared memory.
+//   * warp 1: tcgen05.mma, M = 128 entries per instruction, into a ring of
+//     TMEM accumulators.  bf16 keys: N = H heads, the MMAs of two tiles issued
+//     interleaved.  e4m3 keys: N = 2H (both query pieces side by side), the
+//     two 128-entry halves of a tile issued interleaved.  Here an MMA costs the
+//     tensor pipe about 50 cycles whatever its N (32 to 128), so the layout
+//     keeps MMAs per byte low: 8 per 32 KB of keys in both cases (putting the
+//     e4m3 pieces along K instead doubles them, and the MMAs then pace the
+//     scan);
+//   * warps 2-9: two epilogue warpgroups taking alternate tiles (a warpgroup's
+//     per-tile chain of barrier wait, TMEM loads and arithmetic paced the scan
+//     when both worked on every tile), one TMEM lane (= one entry) per thread:
+//     the two pieces' products added (e4m3), ReLU, gate weights, head sum in
+//     registers, one coalesced fp32 store per entry; the row scale comes from
+//     shared memory.
 // bf16 keys use kind::f16 (bf16 x bf16).  e4m3 keys use kind::f8f6f4 against
 // an exact two-piece e4m3 split of the bf16 query, so the keys go from HBM to
 // the tensor core untouched; the per-row key scale and the per-head
@@ -137,11 +138,12 @@ template <int KIND>
 __host__ __device__ constexpr int tile_rows() {
     return kRows * Cfg<KIND>::kSub;
 }
-// TMEM columns of one sub-tile's accumulator (fp32, one per head: with e4m3
-// keys the two query pieces accumulate into the same column) and of one tile's.
+// TMEM columns of one sub-tile's accumulator (fp32, one per head and query
+// piece: e4m3 keys give columns [0, H) for piece 1 and [H, 2H) for piece 2,
+// added by the epilogue before the ReLU) and of one tile's.
 template <int KIND, int H>
 __host__ __device__ constexpr int sub_cols() {
-    return H;
+    return is_e4m3(KIND) ? 2 * H : H;
 }
 template <int KIND, int H>
 __host__ __device__ constexpr int tile_cols() {
@@ -676,27 +678,23 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                                 mma_f16(d_t[u], a_d[u] + uint64_t((kk * 32) >> 4), b_cur + uint64_t((kk * 32) >> 4),
                                         IDESC, kk > 0);
                 } else if (KIND == E4M3_D64) {
-                    // as below, with 64-byte rows: the halves are 8 KB apart; K steps 0-1 piece 1, 2-3
-                    // piece 2 (its rows H*64 bytes after piece 1's) over the same two key slices
+                    // as below, with 64-byte rows: the halves are 8 KB apart, two K = 32 steps
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+                        for (int sub = 0; sub < 2; ++sub)
+                            mma_f8(d_t[0] + uint32_t(sub * SUBC), a_d[0] + uint64_t((sub * 8192 + kk * 32) >> 4),
+                                   b_cur + uint64_t((kk * 32) >> 4), IDESC, kk > 0);
+                } else {
+                    // the two 128-row halves of the tile (16 KB apart in the stage) into their own column
+                    // blocks, chains interleaved; N = 2H covers both query pieces (piece 2's rows follow
+                    // piece 1's in the operand)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
                         for (int sub = 0; sub < 2; ++sub)
-                            mma_f8(d_t[0] + uint32_t(sub * SUBC),
-                                   a_d[0] + uint64_t((sub * 8192 + (kk & 1) * 32) >> 4),
-                                   b_cur + uint64_t(((kk >> 1) * (H * 64) + (kk & 1) * 32) >> 4), IDESC, kk > 0);
-                } else {
-                    // the two 128-row halves of the tile (16 KB apart in the stage) into their own
-                    // accumulators, chains interleaved; K steps 0-3 take query piece 1, 4-7 piece 2 (its rows
-                    // H*128 bytes after piece 1's) over the same four key slices: the accumulator holds
-                    // (p1 + p2) . k = q 2^e . k
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-#pragma unroll
-                        for (int sub = 0; sub < 2; ++sub)
-                            mma_f8(d_t[0] + uint32_t(sub * SUBC),
-                                   a_d[0] + uint64_t((sub * 16384 + (kk & 3) * 32) >> 4),
-                                   b_cur + uint64_t(((kk >> 2) * (H * 128) + (kk & 3) * 32) >> 4), IDESC, kk > 0);
+                            mma_f8(d_t[0] + uint32_t(sub * SUBC), a_d[0] + uint64_t((sub * 16384 + kk * 32) >> 4),
+                                   b_cur + uint64_t((kk * 32) >> 4), IDESC, kk > 0);
                 }
                 issued = true;
 #pragma unroll
@@ -781,30 +779,44 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                                  ? int(row0 & 3)
                                  : 0;
             const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * TILEC);
-            // the sub-tiles one after the other through the same registers (a whole 256-row tile's row,
-            // 2 H columns, does not fit beside the rest in the 168 registers of a 320-thread CTA); the
-            // accumulator is released once the last sub-tile's columns are in registers
+            // the sub-tiles one after the other, each in chunks of up to 32 heads (both pieces' columns of a
+            // chunk per TMEM round trip) through the same registers: a whole tile's row does not fit beside
+            // the rest in the 168 registers of a 320-thread CTA; the accumulator is released once the last
+            // chunk is in registers
+            constexpr int HC = H < 32 ? H : 32;   // heads per chunk
+            constexpr int NP = is_e4m3(KIND) ? 2 : 1;
 #pragma unroll
             for (int sub = 0; sub < C::kSub; ++sub) {
-                uint32_t r[H];
-#pragma unroll
-                for (int c = 0; c < H / 16; ++c)
-                    tmem_ld_32x32b_x16(taddr + sub * SUBC + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[c * 16]));
-                tmem_ld_wait();
                 const float sc = kScales ? s_scale[int(i % RS) * SS + soff + sub * kRows + quarter * 32 + lane] : 1.f;
-                if (sub == C::kSub - 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[acc]);
-                }
                 float za = 0.f, zb = 0.f, zc = 0.f, zd = 0.f;   // four short dependency chains
 #pragma unroll
-                for (int j = 0; j < H; j += 4) {
-                    const float4 wv = *reinterpret_cast<const float4 *>(wq + j);
-                    za = fmaf(wv.x, fmaxf(__uint_as_float(r[j]), 0.f), za);
-                    zb = fmaf(wv.y, fmaxf(__uint_as_float(r[j + 1]), 0.f), zb);
-                    zc = fmaf(wv.z, fmaxf(__uint_as_float(r[j + 2]), 0.f), zc);
-                    zd = fmaf(wv.w, fmaxf(__uint_as_float(r[j + 3]), 0.f), zd);
+                for (int h0 = 0; h0 < H; h0 += HC) {
+                    uint32_t r[NP][HC];
+#pragma unroll
+                    for (int pc = 0; pc < NP; ++pc)
+#pragma unroll
+                        for (int c = 0; c < HC / 16; ++c)
+                            tmem_ld_32x32b_x16(taddr + sub * SUBC + pc * H + h0 + c * 16,
+                                               *reinterpret_cast<uint32_t(*)[16]>(&r[pc][c * 16]));
+                    tmem_ld_wait();
+                    if (sub == C::kSub - 1 && h0 + HC == H) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[acc]);
+                    }
+#pragma unroll
+                    for (int j = 0; j < HC; j += 4) {
+                        const float4 wv = *reinterpret_cast<const float4 *>(wq + h0 + j);
+                        float v[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            v[e] = NP == 2 ? __uint_as_float(r[0][j + e]) + __uint_as_float(r[NP - 1][j + e])
+                                           : __uint_as_float(r[0][j + e]);
+                        za = fmaf(wv.x, fmaxf(v[0], 0.f), za);
+                        zb = fmaf(wv.y, fmaxf(v[1], 0.f), zb);
+                        zc = fmaf(wv.z, fmaxf(v[2], 0.f), zc);
+                        zd = fmaf(wv.w, fmaxf(v[3], 0.f), zd);
+                    }
                 }
                 float zs = (za + zb) + (zc + zd);
                 const int64_t row = row0 + sub * kRows + quarter * 32 + lane;   // entry (full) or list position
