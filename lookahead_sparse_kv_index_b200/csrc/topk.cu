@@ -1,17 +1,28 @@
 // Fine-grained top-k inside the kept set ("FlashMemory-DeepSeek-V4 ...
 // Lookahead Sparse Attention", gist.science technical summary, section 2.1
-// "Tiered Selection").
+// "Tiered Selection"): the k largest scores of a sequence's kept entries, ties
+// to the lower kept-list position, returned in kept-list (= ascending entry)
+// order.
 //
-// One CTA of 1024 threads per sequence.  Scores map to an order-preserving
-// 32-bit key (larger z -> larger key, -0.0 folded onto +0.0).  A most-
-// significant-digit radix select (passes of 11 bits, below the bits every key
-// shares) finds the digits of the k-th largest key and how many entries sharing
-// them must be taken; an ordered pass then takes every key above and the
-// lowest-index entries at the threshold, and compacts them in kept-list order,
-// which is ascending entry order.  A few tens of thousands of kept entries per
-// sequence fit in shared memory, so every pass works there and the only
-// synchronisation is the CTA's own barrier (a cluster of CTAs spent most of its
-// time in cluster-wide barriers at this size).
+// One CTA of 1024 threads per sequence; scores map to an order-preserving
+// 32-bit key (larger z -> larger key, -0.0 folded onto +0.0) staged in shared
+// memory.  With one CTA per sequence the kernel is bound by instruction issue
+// and by shared-memory atomics (kept scores cluster in few histogram bins), so
+// the common case touches every key only twice after staging, with no atomics:
+//   1. 64 keys sampled at evenly spaced positions give two pivots lo <= hi that
+//      bracket the k-th largest with high probability (a margin of 2.5 binomial
+//      standard deviations around its expected sample rank);
+//   2. one pass counts the keys above hi and copies the keys in [lo, hi] (about
+//      a fifth of them) to a list, one region per warp, appended by ballots;
+//   3. if the bracket holds (fewer than k above hi, at least k up to lo), a
+//      most-significant-digit radix select (12-bit digits, below the bits that lo
+//      and hi share) over the list alone finds the threshold key interval and how
+//      many keys in it are taken; otherwise the same radix select runs over every
+//      key (the exact fallback);
+//   4. one ordered pass takes every key above the threshold interval and the
+//      lowest-position keys inside it: warp w owns a contiguous segment, and
+//      ballots give each taken key its output slot, the warps' offsets coming
+//      from the list (or, on the fallback, from one counting pass).
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -25,79 +36,42 @@ __device__ __forceinline__ uint32_t order_key(float z) {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kStageKeys = 40960;   // keys staged in shared memory (160 KB)
+constexpr int kStageKeys = 32768;   // keys staged in shared memory (128 KB)
 constexpr int kMaxK = 4096;          // the largest k (the entry points check it); positions of the chosen in smem
-constexpr int kDigit = 11;
-constexpr int kBins = 1 << kDigit;   // 2048: two bins per thread
+constexpr int kListW = 256;          // listed keys per warp
+constexpr int kList = kListW * kWarps;   // 8192 (32 KB)
+constexpr int kDigit = 12;
+constexpr int kBins = 1 << kDigit;   // 4096: four per thread
+constexpr int kSamples = 64;         // two per lane of warp 0
+constexpr size_t kSmemBytes = size_t(kStageKeys + 4 + kMaxK + kList + kBins) * 4;
 
-// Exclusive block-wide prefix sum of v (kThreads threads); *total receives the sum.
-__device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int s = s_warp[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, s, o);
-            if (lane >= o) s += y;
-        }
-        s_warp[lane] = s;
-    }
-    __syncthreads();
-    const int res = (warp ? s_warp[warp - 1] : 0) + x - v;
-    *total = s_warp[kWarps - 1];
-    return res;   // s_warp is rewritten only after the caller's next barrier
-}
-
-// Exclusive block-wide prefix sum of a 64-bit value (two counters packed as hi:lo 32-bit halves).
-__device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t *s_warp64) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint64_t x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) s_warp64[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        uint64_t t = s_warp64[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint64_t y = __shfl_up_sync(0xffffffffu, t, o);
-            if (lane >= o) t += y;
-        }
-        s_warp64[lane] = t;
-    }
-    __syncthreads();
-    return (warp ? s_warp64[warp - 1] : 0) + x - v;
-}
+// A compile-time flag for code specialised on where the keys live.
+template <bool V>
+struct Flag {
+    static constexpr bool value = V;
+};
 
 __global__ void __launch_bounds__(kThreads, 1)
 topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restrict__ seq_off,
             const int32_t *__restrict__ kept_idx, const int64_t *__restrict__ kept_off, int64_t kept_cap, int k,
             const int32_t *__restrict__ pos_map, int32_t *__restrict__ topk_idx, int32_t *__restrict__ topk_pos,
             int32_t *__restrict__ topk_cnt) {
-    extern __shared__ uint32_t s_keys[];   // [kStageKeys] keys, then [kMaxK] positions of the chosen
-    int *s_pos = reinterpret_cast<int *>(s_keys + kStageKeys);
-    __shared__ int s_hist[kBins];
+    // [kStageKeys + 4] keys | [kMaxK] positions of the chosen | [kList] listed keys | [kBins] histogram
+    extern __shared__ __align__(16) uint32_t s_keys[];
+    int *s_pos = reinterpret_cast<int *>(s_keys + kStageKeys + 4);
+    uint32_t *s_list = reinterpret_cast<uint32_t *>(s_pos + kMaxK);
+    int *s_hist = reinterpret_cast<int *>(s_list + kList);
     __shared__ int s_warp[kWarps];
-    __shared__ uint64_t s_warp64[kWarps];
-    __shared__ uint32_t s_red[2][kWarps];
-    __shared__ uint32_t s_want;
-    __shared__ int s_kr, s_done;
+    __shared__ int s_chi[kWarps], s_cnt[kWarps];   // per warp: keys above hi, keys listed
+    __shared__ int s_red[2][kWarps];
+    __shared__ uint32_t s_lo, s_hi, s_want;
+    __shared__ int s_kr, s_done, s_binc;
 
     pdl_launch_dependents();   // attention may stage its queries meanwhile
     pdl_wait();                // scores come from the preceding scan
     const int b = blockIdx.x;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t = int(threadIdx.x), lane = t & 31, warp = t >> 5;
+    const uint32_t full = 0xffffffffu, lt = (1u << lane) - 1u;
     const int64_t p0 = kept_off[b];
     int64_t n64 = kept_off[b + 1] - p0;
     if (p0 >= kept_cap) n64 = 0;
@@ -108,126 +82,298 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
     int32_t *out_pos = topk_pos ? topk_pos + int64_t(b) * k : nullptr;
 
     if (n <= k) {   // everything kept is chosen
-        for (int i = threadIdx.x; i < k; i += kThreads) {
+        for (int i = t; i < k; i += kThreads) {
             out_idx[i] = i < n ? kept_idx[p0 + i] : -1;
             if (out_pos) out_pos[i] = i < n ? (pos_map ? pos_map[p0 + i] : int32_t(p0 + i)) : -1;
         }
-        if (threadIdx.x == 0) topk_cnt[b] = n;
+        if (t == 0) topk_cnt[b] = n;
         return;
     }
     const int64_t sbase = z_by_entry ? seq_off[b] : 0;
     const bool staged = n <= kStageKeys;
-    auto load_key = [&](int i) -> uint32_t {   // i: position in the sequence's kept list
+    auto load_z = [&](int i) -> float {   // i: position in the sequence's kept list
         const int64_t p = p0 + i;
-        return order_key(z_by_entry ? z[sbase + kept_idx[p]] : z[p]);
+        return z_by_entry ? z[sbase + kept_idx[p]] : z[p];
     };
-    // each thread owns the contiguous run [lo, hi) of positions (the ordered take needs runs)
-    const int per = (n + kThreads - 1) / kThreads;
-    const int lo = min(n, int(threadIdx.x) * per), hi = min(n, lo + per);
+    const float *zs = z + p0;
+    // listed scores are staged with 16-byte loads from their first 16-byte boundary (`head` scores in); the
+    // staged copy is shifted by `aoff` so that those vectors land on 16-byte boundaries too
+    const bool vec = !z_by_entry && staged;
+    const int head = vec ? min(n, int((4 - ((reinterpret_cast<uintptr_t>(zs) >> 2) & 3)) & 3)) : 0;
+    const int aoff = (4 - head) & 3;
+    uint32_t *sk = s_keys + aoff;   // the key of position i is sk[i]
+    // the key of position i, with the branch on where keys live taken at compile time
+    auto key_of = [&](auto where, int i) -> uint32_t {
+        if constexpr (decltype(where)::value) return sk[i];
+        else return order_key(load_z(i));
+    };
+    auto specialised = [&](auto &&f) {
+        if (staged) f(Flag<true>{});
+        else f(Flag<false>{});
+    };
 
-    // stage the keys (coalesced: consecutive threads, consecutive positions), min / max on the way
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-    for (int i0 = int(threadIdx.x); i0 < n; i0 += 8 * kThreads) {
-        uint32_t v[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * kThreads;
-            v[u] = i < n ? load_key(i) : 0u;
+    for (int q = 0; q < kBins / kThreads; ++q) s_hist[t + q * kThreads] = 0;   // readers re-zero their bins
+    for (int j = t; j < k; j += kThreads) s_pos[j] = -1;   // a slot left unfilled yields -1, not a stray read
+
+    if (warp == 0) {
+        // 1. the sample, ranked by warp 0 alone while the other warps stage: the sample at descending index
+        // i has gt <= i < gt + eq
+        const uint32_t a = order_key(load_z(int((int64_t(2 * lane + 1) * n) / (2 * kSamples))));
+        const uint32_t c = order_key(load_z(int((int64_t(2 * (lane + 32) + 1) * n) / (2 * kSamples))));
+        int gta = 0, eqa = 0, gtc = 0, eqc = 0;
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+            const uint32_t x = __shfl_sync(full, a, j), y = __shfl_sync(full, c, j);
+            gta += int(x > a) + int(y > a);
+            eqa += int(x == a) + int(y == a);
+            gtc += int(x > c) + int(y > c);
+            eqc += int(x == c) + int(y == c);
         }
+        // the k-th largest is expected at sample index r = 64 k / n, with binomial spread
+        const float frac = float(k) / float(n);
+        const float r = float(kSamples) * frac;
+        const int margin = int(ceilf(2.5f * sqrtf(r * (1.f - frac)))) + 1;
+        const int i_hi = int(r) - margin, i_lo = int(r) + margin;
+        auto at = [&](int i, uint32_t *dst) {
+            if (gta <= i && i < gta + eqa) *dst = a;   // equal samples write equal values
+            if (gtc <= i && i < gtc + eqc) *dst = c;
+        };
+        if (i_hi >= 0) at(i_hi, &s_hi);
+        else if (lane == 0) s_hi = 0xFFFFFFFFu;
+        if (i_lo < kSamples) at(i_lo, &s_lo);
+        else if (lane == 0) s_lo = 0u;
+    } else if (vec) {
+        // warps 1.. stage
+        const int ts = t - 32, ns = kThreads - 32;
+        const int nv = (n - head) >> 2;
+        const float4 *z4 = reinterpret_cast<const float4 *>(zs + head);
+        for (int j0 = ts; j0 < nv; j0 += 4 * ns) {
+            float4 v[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * kThreads;
-            if (i < n) {
-                if (staged) s_keys[i] = v[u];
-                kmin = min(kmin, v[u]);
-                kmax = max(kmax, v[u]);
+            for (int u = 0; u < 4; ++u)
+                if (j0 + u * ns < nv) v[u] = z4[j0 + u * ns];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = j0 + u * ns;
+                if (j < nv)
+                    *reinterpret_cast<uint4 *>(sk + head + 4 * j) =
+                        make_uint4(order_key(v[u].x), order_key(v[u].y), order_key(v[u].z), order_key(v[u].w));
             }
         }
-    }
+        // the scores before the first boundary (threads 32..35) and after the last whole vector (36..39)
+        if (ts < 8) {
+            const int i = ts < 4 ? ts : head + 4 * nv + ts - 4;
+            if (ts < 4 ? i < head : i < n) sk[i] = order_key(zs[i]);
+        }
+    } else if (staged) {
+        const int ts = t - 32, ns = kThreads - 32;
+        for (int i0 = ts; i0 < n; i0 += 8 * ns) {
+            float v[8];
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+            for (int u = 0; u < 8; ++u)
+                if (i0 + u * ns < n) v[u] = load_z(i0 + u * ns);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (i0 + u * ns < n) sk[i0 + u * ns] = order_key(v[u]);
+        }
     }
-    if (lane == 0) { s_red[0][warp] = kmin; s_red[1][warp] = kmax; }
-    __syncthreads();   // also publishes the staged keys
-    uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
-#pragma unroll 4
-    for (int w = 0; w < kWarps; ++w) { gmin = min(gmin, s_red[0][w]); gmax = max(gmax, s_red[1][w]); }
-    auto key = [&](int i) -> uint32_t { return staged ? s_keys[i] : load_key(i); };
+    __syncthreads();   // publishes the staged keys and the pivots
 
-    const uint32_t diff = gmin ^ gmax;
-    int top = diff ? 31 - __clz(diff) : -1;   // bits above `top` are shared by every key
-    uint32_t hmask = top >= 31 ? 0u : (top >= 0 ? ~((2u << top) - 1u) : 0xFFFFFFFFu);
-    uint32_t want = gmin & hmask;
-    int kr = k;
-    s_hist[threadIdx.x] = 0;   // each pass's reader zeroes its bins for the next pass
-    s_hist[threadIdx.x + kThreads] = 0;
+    // 2. keys above hi (counted) and in [lo, hi] (listed); warp w owns positions [w_lo, w_hi)
+    uint32_t lo = s_lo, hi = s_hi;
+    const int seg = ((n + kThreads - 1) / kThreads) * 32;
+    const int w_lo = min(n, warp * seg), w_hi = min(n, w_lo + seg);
+    uint32_t *reg = s_list + warp * kListW;
+    int nlist;
+    {
+        const uint32_t span = hi - lo;
+        int c_hi = 0, cnt = 0;
+        specialised([&](auto where) {
+            for (int q0 = w_lo; q0 < w_hi; q0 += 4 * 32) {   // warp-uniform trip count
+                uint32_t u[4], m[4];
+                bool v[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int p = q0 + 32 * q + lane;
+                    v[q] = p < w_hi;
+                    u[q] = v[q] ? key_of(where, p) : 0u;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    c_hi += int(v[q] && u[q] > hi);
+                    m[q] = __ballot_sync(full, v[q] && u[q] - lo <= span);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int slot = cnt + __popc(m[q] & lt);
+                    if (((m[q] >> lane) & 1u) && slot < kListW) reg[slot] = u[q];
+                    cnt += __popc(m[q]);
+                }
+            }
+        });
+        c_hi = __reduce_add_sync(full, c_hi);
+        if (lane == 0) { s_chi[warp] = c_hi; s_cnt[warp] = cnt; }
+        nlist = min(cnt, kListW);
+    }
     __syncthreads();
+    const int n_hi = __reduce_add_sync(full, s_chi[lane]);
+    const int n_in = __reduce_add_sync(full, s_cnt[lane]);
+    const bool bracket = !__any_sync(full, s_cnt[lane] > kListW) && n_hi < k && n_hi + n_in >= k;   // uniform
+
+    // 3. radix select over the list (or every key): the kr-th largest key among those whose bits under
+    // hmask equal want
+    int kr, top, binc;
+    if (bracket) {
+        kr = k - n_hi;
+        const uint32_t diff = lo ^ hi;
+        top = diff ? 31 - __clz(diff) : -1;   // bits above `top` are shared by every listed key
+        binc = n_in;
+    } else {
+        lo = 0u;
+        hi = 0xFFFFFFFFu;
+        kr = k;
+        top = 31;
+        binc = n;
+    }
+    uint32_t hmask = top >= 31 ? 0u : (top >= 0 ? ~((2u << top) - 1u) : 0xFFFFFFFFu);
+    uint32_t want = lo & hmask;
     while (top >= 0) {
         const int width = top + 1 < kDigit ? top + 1 : kDigit;
         const int shift = top + 1 - width;
         const uint32_t dmask = (1u << width) - 1u;
-        for (int i = lo; i < hi; ++i) {
-            const uint32_t u = key(i);
-            if ((u & hmask) == want) atomicAdd(&s_hist[(u >> shift) & dmask], 1);
+        if (bracket) {
+            for (int j = lane; j < nlist; j += 32) {
+                const uint32_t u = reg[j];
+                if ((u & hmask) == want) atomicAdd(&s_hist[(u >> shift) & dmask], 1);
+            }
+        } else {
+            specialised([&](auto where) {
+                for (int p = t; p < n; p += kThreads) {
+                    const uint32_t u = key_of(where, p);
+                    if ((u & hmask) == want) atomicAdd(&s_hist[(u >> shift) & dmask], 1);
+                }
+            });
         }
         __syncthreads();
-        {   // thread t owns bins 2047 - 2t and 2046 - 2t (descending key order); suffix counts by a block scan
-            const int bh = kBins - 1 - 2 * int(threadIdx.x);
-            const int h0 = s_hist[bh], h1 = s_hist[bh - 1];
-            s_hist[bh] = 0;   // only this thread reads these two bins
-            s_hist[bh - 1] = 0;
-            int tot;
-            int above = block_excl_scan(h0 + h1, s_warp, &tot);   // entries in bins above bh
-            if (above < kr && above + h0 >= kr) {
-                s_want = want | (uint32_t(bh) << shift);
-                s_kr = kr - above;
-                s_done = (above + h0 == kr);
-            } else if (above + h0 < kr && above + h0 + h1 >= kr) {
-                s_want = want | (uint32_t(bh - 1) << shift);
-                s_kr = kr - above - h0;
-                s_done = (above + h0 + h1 == kr);
+        {   // thread t owns bins 4095 - 4t .. 4092 - 4t (descending key order).  The warp sums locate the warp
+            // whose bins hold the kr-th key; that warp alone scans its lanes.
+            const int bh = kBins - 1 - 4 * t;
+            int h[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                h[q] = s_hist[bh - q];
+                s_hist[bh - q] = 0;   // only this thread reads these bins
+            }
+            const int mine = h[0] + h[1] + h[2] + h[3];
+            const int wsum = __reduce_add_sync(full, mine);
+            if (lane == 0) s_warp[warp] = wsum;
+            __syncthreads();
+            const int above_w = __reduce_add_sync(full, lane < warp ? s_warp[lane] : 0);
+            if (above_w < kr && above_w + wsum >= kr) {   // warp-uniform
+                int x = mine;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(full, x, o);
+                    if (lane >= o) x += y;
+                }
+                int above = above_w + x - mine;   // keys in bins above bh
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (above < kr && above + h[q] >= kr) {
+                        s_want = want | (uint32_t(bh - q) << shift);
+                        s_kr = kr - above;
+                        s_done = (above + h[q] == kr);
+                        s_binc = h[q];
+                    }
+                    above += h[q];
+                }
             }
         }
         __syncthreads();
         want = s_want;
         kr = s_kr;
+        binc = s_binc;
         hmask |= dmask << shift;
         top = shift - 1;
         if (s_done) break;   // uniform: read after the barrier, rewritten only after the next barrier
     }
-    // ordered take: keys whose resolved bits exceed `want`, then the first kr equal to it (in kept-list
-    // order).  One scan of the packed counts (equal : above) gives both this thread's rank among the
-    // equal keys and the number of keys above before it.
-    int n_eq = 0, n_above = 0;
-    for (int i = lo; i < hi; ++i) {
-        const uint32_t u = key(i) & hmask;
-        n_eq += u == want;
-        n_above += u > want;
-    }
-    const uint64_t pre = block_excl_scan64((uint64_t(n_eq) << 32) | uint32_t(n_above), s_warp64);
-    const int eq_rank = int(pre >> 32);
-    int out = int(uint32_t(pre)) + min(eq_rank, kr);
-    // the take records the position of each output slot; the entry indices are then fetched with
-    // independent loads, two slots per thread (a dependent load per taken key serialised the tail)
-    int r = eq_rank;
-    for (int i = lo; i < hi; ++i) {
-        const uint32_t u = key(i) & hmask;
-        bool t = u > want;
-        if (u == want) { t = r < kr; ++r; }
-        if (t) {
-            if (out < k) s_pos[out] = i;
-            ++out;
+    // the threshold interval: keys in [e_lo, e_hi] are equal at the resolved bits (binc of them, kr taken);
+    // keys above e_hi are all taken
+    const uint32_t e_lo = max(want, lo), e_hi = min(want | ~hmask, hi), espan = e_hi - e_lo;
+    const bool all_eq = kr == binc;   // uniform
+
+    // 4. ordered take.  Keys above and inside the interval in the warps before this one:
+    int a_w = 0, e_w = 0;
+    if (bracket) {
+        for (int j = lane; j < nlist; j += 32) {
+            const uint32_t u = reg[j];
+            a_w += int(u > e_hi);
+            e_w += int(u - e_lo <= espan);
         }
+        a_w = __reduce_add_sync(full, a_w) + s_chi[warp];
+    } else {
+        specialised([&](auto where) {
+            for (int p = w_lo + lane; p < w_hi; p += 32) {
+                const uint32_t u = key_of(where, p);
+                a_w += int(u > e_hi);
+                e_w += int(u - e_lo <= espan);
+            }
+        });
+        a_w = __reduce_add_sync(full, a_w);
     }
+    e_w = __reduce_add_sync(full, e_w);
+    if (lane == 0) { s_red[0][warp] = a_w; s_red[1][warp] = e_w; }
     __syncthreads();
-    for (int j = threadIdx.x; j < k; j += kThreads) {
-        const int64_t p = p0 + s_pos[j];
-        out_idx[j] = kept_idx[p];
-        if (out_pos) out_pos[j] = pos_map ? pos_map[p] : int32_t(p);
+    int a_run = __reduce_add_sync(full, lane < warp ? s_red[0][lane] : 0);
+    int e_run = __reduce_add_sync(full, lane < warp ? s_red[1][lane] : 0);
+    if (all_eq) a_run += e_run;   // one running count of taken keys
+    // a taken key with `a` keys above and `e` inside the interval before it goes to slot a + min(e, kr)
+    specialised([&](auto where) {
+        for (int q0 = w_lo; q0 < w_hi; q0 += 4 * 32) {   // warp-uniform trip count
+            uint32_t u[4], ba[4], be[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int p = q0 + 32 * q + lane;
+                u[q] = p < w_hi ? key_of(where, p) : 0u;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const bool v = q0 + 32 * q + lane < w_hi;
+                ba[q] = __ballot_sync(full, v && u[q] > e_hi);
+                be[q] = __ballot_sync(full, v && u[q] - e_lo <= espan);
+            }
+            if (all_eq) {   // every key inside the interval is taken: a_run counts both kinds
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t bt = ba[q] | be[q];
+                    const int slot = a_run + __popc(bt & lt);
+                    if (((bt >> lane) & 1u) && slot < k) s_pos[slot] = q0 + 32 * q + lane;
+                    a_run += __popc(bt);
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int eb = e_run + __popc(be[q] & lt);
+                    const int slot = a_run + __popc(ba[q] & lt) + min(eb, kr);
+                    const bool take = ((ba[q] >> lane) & 1u) || (((be[q] >> lane) & 1u) && eb < kr);
+                    if (take && slot < k) s_pos[slot] = q0 + 32 * q + lane;
+                    a_run += __popc(ba[q]);
+                    e_run += __popc(be[q]);
+                }
+            }
+        }
+    });
+    __syncthreads();
+    // the entry indices of the chosen positions, fetched with independent loads
+    for (int j = t; j < k; j += kThreads) {
+        const int i = s_pos[j];
+        const bool ok = 0 <= i && i < n;
+        const int64_t p = p0 + (ok ? i : 0);
+        out_idx[j] = ok ? kept_idx[p] : -1;
+        if (out_pos) out_pos[j] = !ok ? -1 : (pos_map ? pos_map[p] : int32_t(p));
     }
-    if (threadIdx.x == 0) topk_cnt[b] = k;
+    if (t == 0) topk_cnt[b] = k;
 }
 
 }  // namespace
@@ -236,7 +382,7 @@ lsa_status launch_topk(const float *z, int32_t z_by_entry, const int64_t *seq_of
                        const int32_t *kept_idx, const int64_t *kept_off, int32_t B, int32_t k,
                        int64_t kept_cap, const int32_t *pos_map, int32_t *topk_idx, int32_t *topk_pos,
                        int32_t *topk_cnt, cudaStream_t st) {
-    const size_t smem = size_t(kStageKeys) * 4 + size_t(kMaxK) * 4;
+    const size_t smem = kSmemBytes;
     LSA_CUDA(ensure_smem(topk_select, smem));
     LSA_CUDA(launch_pdl(topk_select, dim3(B), dim3(kThreads), smem, st, z, z_by_entry, seq_off, kept_idx, kept_off,
                         kept_cap, k, pos_map, topk_idx, topk_pos, topk_cnt));
