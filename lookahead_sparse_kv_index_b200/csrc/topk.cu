@@ -15,10 +15,12 @@
 //   2. one pass counts the keys above hi and copies the keys in [lo, hi] (about
 //      a fifth of them) to a list, one region per warp, appended by ballots;
 //   3. if the bracket holds (fewer than k above hi, at least k up to lo), a
-//      most-significant-digit radix select (12-bit digits, below the bits that lo
-//      and hi share) over the list alone finds the threshold key interval and how
-//      many keys in it are taken; otherwise the same radix select runs over every
-//      key (the exact fallback);
+//      radix-style select over the list alone narrows the key interval [lo, hi]
+//      to the one holding the k-th largest: each pass splits the interval into
+//      4096 equal bins (of a power-of-two width), counts the listed keys per bin
+//      and keeps the bin holding it, until the bin holds only keys that are all
+//      taken or one key value; otherwise the same select runs over every key,
+//      from the whole key range (the exact fallback);
 //   4. one ordered pass takes every key above the threshold interval and the
 //      lowest-position keys inside it: warp w owns a contiguous segment, and
 //      ballots give each taken key its output slot, the warps' offsets coming
@@ -64,7 +66,7 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
     __shared__ int s_warp[kWarps];
     __shared__ int s_chi[kWarps], s_cnt[kWarps];   // per warp: keys above hi, keys listed
     __shared__ int s_red[2][kWarps];
-    __shared__ uint32_t s_lo, s_hi, s_want;
+    __shared__ uint32_t s_lo, s_hi, s_ilo, s_ihi;
     __shared__ int s_kr, s_done, s_binc;
 
     pdl_launch_dependents();   // attention may stage its queries meanwhile
@@ -221,37 +223,34 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
     const int n_in = __reduce_add_sync(full, s_cnt[lane]);
     const bool bracket = !__any_sync(full, s_cnt[lane] > kListW) && n_hi < k && n_hi + n_in >= k;   // uniform
 
-    // 3. radix select over the list (or every key): the kr-th largest key among those whose bits under
-    // hmask equal want
-    int kr, top, binc;
+    // 3. select over the list (or every key): [ilo, ihi] holds the kr-th largest of the source's keys in it
+    int kr, binc;   // binc: the source's keys in [ilo, ihi]
+    uint32_t ilo, ihi;
     if (bracket) {
         kr = k - n_hi;
-        const uint32_t diff = lo ^ hi;
-        top = diff ? 31 - __clz(diff) : -1;   // bits above `top` are shared by every listed key
+        ilo = lo;
+        ihi = hi;
         binc = n_in;
     } else {
-        lo = 0u;
-        hi = 0xFFFFFFFFu;
         kr = k;
-        top = 31;
+        ilo = 0u;
+        ihi = 0xFFFFFFFFu;
         binc = n;
     }
-    uint32_t hmask = top >= 31 ? 0u : (top >= 0 ? ~((2u << top) - 1u) : 0xFFFFFFFFu);
-    uint32_t want = lo & hmask;
-    while (top >= 0) {
-        const int width = top + 1 < kDigit ? top + 1 : kDigit;
-        const int shift = top + 1 - width;
-        const uint32_t dmask = (1u << width) - 1u;
+    while (ilo != ihi) {   // uniform
+        const uint32_t span = ihi - ilo;
+        const int bits = 32 - __clz(span);
+        const int sh = bits > kDigit ? bits - kDigit : 0;   // 4096 bins of 2^sh key values cover the interval
         if (bracket) {
             for (int j = lane; j < nlist; j += 32) {
-                const uint32_t u = reg[j];
-                if ((u & hmask) == want) atomicAdd(&s_hist[(u >> shift) & dmask], 1);
+                const uint32_t u = reg[j] - ilo;
+                if (u <= span) atomicAdd(&s_hist[u >> sh], 1);
             }
         } else {
             specialised([&](auto where) {
                 for (int p = t; p < n; p += kThreads) {
-                    const uint32_t u = key_of(where, p);
-                    if ((u & hmask) == want) atomicAdd(&s_hist[(u >> shift) & dmask], 1);
+                    const uint32_t u = key_of(where, p) - ilo;
+                    if (u <= span) atomicAdd(&s_hist[u >> sh], 1);
                 }
             });
         }
@@ -281,7 +280,9 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     if (above < kr && above + h[q] >= kr) {
-                        s_want = want | (uint32_t(bh - q) << shift);
+                        const uint32_t blo = ilo + (uint32_t(bh - q) << sh), wmax = (1u << sh) - 1u;
+                        s_ilo = blo;
+                        s_ihi = ihi - blo < wmax ? ihi : blo + wmax;
                         s_kr = kr - above;
                         s_done = (above + h[q] == kr);
                         s_binc = h[q];
@@ -291,16 +292,15 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
             }
         }
         __syncthreads();
-        want = s_want;
+        ilo = s_ilo;
+        ihi = s_ihi;
         kr = s_kr;
         binc = s_binc;
-        hmask |= dmask << shift;
-        top = shift - 1;
         if (s_done) break;   // uniform: read after the barrier, rewritten only after the next barrier
     }
-    // the threshold interval: keys in [e_lo, e_hi] are equal at the resolved bits (binc of them, kr taken);
-    // keys above e_hi are all taken
-    const uint32_t e_lo = max(want, lo), e_hi = min(want | ~hmask, hi), espan = e_hi - e_lo;
+    // keys in [e_lo, e_hi] (binc of them) are the candidates at the threshold, kr of them taken; keys above
+    // e_hi are all taken
+    const uint32_t e_lo = ilo, e_hi = ihi, espan = e_hi - e_lo;
     const bool all_eq = kr == binc;   // uniform
 
     // 4. ordered take.  Keys above and inside the interval in the warps before this one:
@@ -337,21 +337,22 @@ topk_select(const float *__restrict__ z, int z_by_entry, const int64_t *__restri
                 const int p = q0 + 32 * q + lane;
                 u[q] = p < w_hi ? key_of(where, p) : 0u;
             }
+            if (all_eq) {   // every key from e_lo up is taken: a_run counts both kinds
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const bool v = q0 + 32 * q + lane < w_hi;
-                ba[q] = __ballot_sync(full, v && u[q] > e_hi);
-                be[q] = __ballot_sync(full, v && u[q] - e_lo <= espan);
-            }
-            if (all_eq) {   // every key inside the interval is taken: a_run counts both kinds
+                for (int q = 0; q < 4; ++q) ba[q] = __ballot_sync(full, q0 + 32 * q + lane < w_hi && u[q] >= e_lo);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t bt = ba[q] | be[q];
-                    const int slot = a_run + __popc(bt & lt);
-                    if (((bt >> lane) & 1u) && slot < k) s_pos[slot] = q0 + 32 * q + lane;
-                    a_run += __popc(bt);
+                    const int slot = a_run + __popc(ba[q] & lt);
+                    if (((ba[q] >> lane) & 1u) && slot < k) s_pos[slot] = q0 + 32 * q + lane;
+                    a_run += __popc(ba[q]);
                 }
             } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const bool v = q0 + 32 * q + lane < w_hi;
+                    ba[q] = __ballot_sync(full, v && u[q] > e_hi);
+                    be[q] = __ballot_sync(full, v && u[q] - e_lo <= espan);
+                }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int eb = e_run + __popc(be[q] & lt);

@@ -240,6 +240,29 @@ def test_topk_clustered_scores_stage_exact(lsa, k):
         assert np.array_equal(idx, ref_idx)
 
 
+@pytest.mark.parametrize("sampled", ["low", "high"])
+def test_topk_unrepresentative_sample_falls_back_exactly(lsa, sampled):
+    """The scores at the evenly spaced positions the kernel samples are made the smallest (or largest) of their
+    sequence, so the pivots drawn from them miss the k-th largest (too many keys above the upper pivot, too few
+    from the lower one up, or too many between them) and the exact full-range select must run."""
+    k = 2048
+    lens = [12800, 6400, 25600]
+    seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    rng = np.random.default_rng(7 if sampled == "low" else 8)
+    z = rng.uniform(1.0, 2.0, size=int(seq_off[-1])).astype(np.float32)
+    for b, n in enumerate(lens):
+        pos = (np.arange(64) * 2 + 1) * n // 128             # the sampled kept positions (every entry is kept)
+        z[seq_off[b] + pos] = 1e-3 if sampled == "low" else 50.0 + rng.random(64)
+    kept, ko, _ = oracle.select(z.astype(np.float64), seq_off)
+    assert np.array_equal(np.diff(ko), lens)
+    zk = z.astype(np.float64)
+    ref_idx, ref_cnt = oracle.topk(zk, kept, ko, k)
+    for by_entry in (1, 0):
+        idx, pos, cnt = _topk_gpu(lsa, z, by_entry, seq_off, kept, ko, k)
+        assert np.array_equal(cnt, ref_cnt)
+        assert np.array_equal(idx, ref_idx)
+
+
 def test_topk_respects_kept_capacity(lsa):
     seq_off = np.array([0, 100, 300], np.int64)
     z = np.linspace(1, 2, 300).astype(np.float32)
