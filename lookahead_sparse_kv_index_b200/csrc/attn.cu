@@ -180,24 +180,21 @@ __device__ __forceinline__ void put4(T *out, int64_t i, float4 a, float inv) {
 //   lse = M + log L;  a chunk with m_c = -inf (no selected row) has weight 0 and
 // its o is never read into the sum.
 // The kernel is a chain of dependent L2 round trips unless the loads go out
-// together.  Up to 16 chunks: every thread issues its four columns of every
-// chunk at once; the (m, l) of the chunks, the same for the whole block, go
-// through shared memory meanwhile.
-template <typename T, typename TP>
+// together.  Up to kMax (16) chunks: every thread issues its four columns
+// of every chunk at once; meanwhile warp 0 turns the chunks' (m, l), the same
+// for the whole block, into the weights w_c and 1 / L in shared memory.
+template <typename T, typename TP, int kMax>
 __global__ void __launch_bounds__(128, 4)   // 4 CTAs per SM: the whole grid (Hq x B) resident at once
-attn_combine16(const TP *__restrict__ part_o, const float *__restrict__ part_ml, int nchunks, int Hq, int D,
-               T *__restrict__ out, float *__restrict__ lse) {
-    constexpr int kMax = 16;
+attn_combine_few(const TP *__restrict__ part_o, const float *__restrict__ part_ml, int nchunks, int Hq, int D,
+                 T *__restrict__ out, float *__restrict__ lse) {
+    static_assert(kMax <= 32, "warp 0 holds one chunk per lane");
     using PR = Raw4<TP>;
-    __shared__ float2 s_ml[kMax];
+    __shared__ float s_w[kMax];
+    __shared__ float s_inv;
     pdl_wait();   // partials come from the preceding kernel
     const int h = blockIdx.x, b = blockIdx.y;
     const int64_t p0 = int64_t(b) * nchunks * Hq + h;   // partial index of chunk 0; chunk c adds c * Hq
     const int64_t ob = (int64_t(b) * Hq + h) * D;
-    if (threadIdx.x < kMax)
-        s_ml[threadIdx.x] = int(threadIdx.x) < nchunks
-                                ? reinterpret_cast<const float2 *>(part_ml)[p0 + int64_t(threadIdx.x) * Hq]
-                                : make_float2(-INFINITY, 0.f);
     const int64_t cstride = int64_t(Hq) * D;
     for (int col0 = 0; col0 < D; col0 += 4 * int(blockDim.x)) {   // uniform trip count: barrier inside
         const int col = col0 + 4 * int(threadIdx.x);
@@ -206,24 +203,95 @@ attn_combine16(const TP *__restrict__ part_o, const float *__restrict__ part_ml,
         const TP *base = part_o + p0 * D + col;
 #pragma unroll
         for (int u = 0; u < kMax; ++u) v[u] = (act && u < nchunks) ? PR::load(base, int64_t(u) * cstride) : PR::zero();
-        __syncthreads();
-        float M = -INFINITY;
+        if (col0 == 0 && threadIdx.x < 32) {
+            const int c = int(threadIdx.x);
+            const float2 x = c < kMax && c < nchunks ? reinterpret_cast<const float2 *>(part_ml)[p0 + int64_t(c) * Hq]
+                                                     : make_float2(-INFINITY, 0.f);
+            float M = x.x;
 #pragma unroll
-        for (int u = 0; u < kMax; ++u) M = fmaxf(M, s_ml[u].x);
-        float L = 0.f;
+            for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            // an empty chunk (m = -inf, or past nchunks) has weight 0 and its o is never read into the sum
+            const float w = x.x == -INFINITY ? 0.f : expf(x.x - M);
+            float L = x.y * w;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+            if (c < kMax) s_w[c] = w;
+            if (c == 0) {
+                s_inv = M == -INFINITY ? 0.f : 1.f / L;
+                if (lse) lse[int64_t(b) * Hq + h] = M == -INFINITY ? -INFINITY : M + logf(L);
+            }
+        }
+        __syncthreads();
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int u = 0; u < kMax; ++u) {
-            const float2 x = s_ml[u];
-            if (x.x == -INFINITY) continue;   // empty chunk (or u >= nchunks): its o is never read
-            const float w = expf(x.x - M);
-            L = fmaf(x.y, w, L);
+            const float w = s_w[u];
+            if (w == 0.f) continue;   // empty chunk (or u >= nchunks), or a weight below the float range
             const float4 o = PR::f(v[u]);
             a.x = fmaf(w, o.x, a.x); a.y = fmaf(w, o.y, a.y);
             a.z = fmaf(w, o.z, a.z); a.w = fmaf(w, o.w, a.w);
         }
-        if (act) put4(out, ob + col, a, M == -INFINITY ? 0.f : 1.f / L);
-        if (col == 0 && lse) lse[int64_t(b) * Hq + h] = M == -INFINITY ? -INFINITY : M + logf(L);
+        if (act) put4(out, ob + col, a, s_inv);
+    }
+}
+
+// 17..32 chunks of bf16 partials at the tensor-core shape (Hq x D fixed): the
+// same scheme with two columns per thread and 256 threads, so that the 32
+// chunks' values in flight fit in 64 registers (four CTAs per SM keep the whole
+// grid resident; at four columns per thread the values spilled and the spill
+// serialised the loads).  The chunk stride is a compile-time constant, so every
+// load addresses off one base register.
+template <typename T, int kHqC, int kDC>
+__global__ void __launch_bounds__(256, 4)
+attn_combine32(const uint16_t *__restrict__ part_o, const float *__restrict__ part_ml, int nchunks,
+               T *__restrict__ out, float *__restrict__ lse) {
+    constexpr int kMax = 32, Hq = kHqC, D = kDC;
+    __shared__ float s_w[kMax];
+    __shared__ float s_inv;
+    pdl_wait();   // partials come from the preceding kernel
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int64_t p0 = int64_t(b) * nchunks * Hq + h;   // partial index of chunk 0; chunk c adds c * Hq
+    const int64_t ob = (int64_t(b) * Hq + h) * D;
+    constexpr int64_t cstride = int64_t(Hq) * D;
+    for (int col0 = 0; col0 < D; col0 += 2 * int(blockDim.x)) {   // uniform trip count: barrier inside
+        const int col = col0 + 2 * int(threadIdx.x);
+        const bool act = col < D;
+        uint32_t v[kMax];
+        const uint16_t *base = part_o + p0 * D + col;
+#pragma unroll
+        for (int u = 0; u < kMax; ++u)
+            v[u] = (act && u < nchunks) ? *reinterpret_cast<const uint32_t *>(base + u * cstride) : 0u;
+        if (col0 == 0 && threadIdx.x < 32) {
+            const int c = int(threadIdx.x);
+            const float2 x = c < nchunks ? reinterpret_cast<const float2 *>(part_ml)[p0 + int64_t(c) * Hq]
+                                         : make_float2(-INFINITY, 0.f);
+            float M = x.x;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            // an empty chunk (m = -inf, or past nchunks) has weight 0 and its o is never read into the sum
+            const float w = x.x == -INFINITY ? 0.f : expf(x.x - M);
+            float L = x.y * w;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+            s_w[c] = w;
+            if (c == 0) {
+                s_inv = M == -INFINITY ? 0.f : 1.f / L;
+                if (lse) lse[int64_t(b) * Hq + h] = M == -INFINITY ? -INFINITY : M + logf(L);
+            }
+        }
+        __syncthreads();
+        float ax = 0.f, ay = 0.f;
+#pragma unroll
+        for (int u = 0; u < kMax; ++u) {
+            const float w = s_w[u];
+            if (w == 0.f) continue;   // empty chunk (or u >= nchunks), or a weight below the float range
+            ax = fmaf(w, __uint_as_float(v[u] << 16), ax);
+            ay = fmaf(w, __uint_as_float(v[u] & 0xFFFF0000u), ay);
+        }
+        if (act) {
+            Elem<T>::put(out, ob + col, ax * s_inv);
+            Elem<T>::put(out, ob + col + 1, ay * s_inv);
+        }
     }
 }
 
@@ -277,7 +345,15 @@ attn_combine(const TP *__restrict__ part_o, const float *__restrict__ part_ml, i
 template <typename T, typename TP>
 lsa_status launch_combine(const TP *part_o, const float *part_ml, int nchunks, int B, int Hq, int D, void *out,
                           float *lse, cudaStream_t st) {
-    auto kern = nchunks <= 16 ? attn_combine16<T, TP> : attn_combine<T, TP>;
+    if constexpr (sizeof(TP) == 2) {
+        if (nchunks > 16 && nchunks <= 32 && Hq == 128 && D == 512) {   // two columns per thread
+            LSA_CUDA(launch_pdl(attn_combine32<T, 128, 512>, dim3(Hq, B), dim3(256), 0, st, part_o, part_ml, nchunks,
+                                static_cast<T *>(out), lse));
+            LSA_LAUNCHED("attn_combine32");
+            return LSA_OK;
+        }
+    }
+    auto kern = nchunks <= 16 ? attn_combine_few<T, TP, 16> : attn_combine<T, TP>;
     LSA_CUDA(launch_pdl(kern, dim3(Hq, B), dim3(128), 0, st, part_o, part_ml, nchunks, Hq, D, static_cast<T *>(out),
                         lse));
     LSA_LAUNCHED("attn_combine");
