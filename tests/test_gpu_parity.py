@@ -263,6 +263,27 @@ def test_topk_unrepresentative_sample_falls_back_exactly(lsa, sampled):
         assert np.array_equal(idx, ref_idx)
 
 
+def test_topk_run_of_high_scores_in_one_segment(lsa):
+    """A contiguous run of 200 top scores inside one warp's segment of kept positions (far more keys above the
+    upper pivot in one segment than elsewhere), with distinct top scores in one sequence and equal ones plus
+    ties at the k-th score in the other."""
+    k = 2048
+    lens = [14400, 14400]
+    seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    rng = np.random.default_rng(11)
+    z = rng.uniform(0.1, 1.0, size=int(seq_off[-1])).astype(np.float32)
+    z[1000:1200] = 100.0 + rng.random(200).astype(np.float32)      # sequence 0: distinct top scores
+    z[seq_off[1] + 1000:seq_off[1] + 1200] = 100.0                  # sequence 1: all equal
+    z[seq_off[1]:] = np.round(z[seq_off[1]:] * 16) / 16              # ... and ties at the k-th
+    kept, ko, _ = oracle.select(z.astype(np.float64), seq_off)
+    zk = z.astype(np.float64)
+    ref_idx, ref_cnt = oracle.topk(zk, kept, ko, k)
+    for by_entry in (1, 0):
+        idx, pos, cnt = _topk_gpu(lsa, z, by_entry, seq_off, kept, ko, k)
+        assert np.array_equal(cnt, ref_cnt)
+        assert np.array_equal(idx, ref_idx)
+
+
 def test_topk_respects_kept_capacity(lsa):
     seq_off = np.array([0, 100, 300], np.int64)
     z = np.linspace(1, 2, 300).astype(np.float32)
