@@ -140,6 +140,33 @@ lsa_status lsa_select(const float *z, const int64_t *seq_off, int64_t n_total, i
                       void *workspace, size_t ws_bytes, int32_t *err, void *stream);
 
 /* ------------------------------------------------------------------------
+ * lsa_index_score_select -- the full index scan and the threshold selection in
+ * one call (section 2.1, "Scoring Mechanism" then "Dynamic Fetching"): the
+ * z of lsa_index_score in full mode (every entry) and the kept lists of
+ * lsa_select, bit for bit (same z, same decision z >= 0, same order).
+ *
+ * On the tensor-core path (the shapes lsa_index_score runs on tcgen05) the
+ * selection is fused into the scan: its epilogue takes the z >= 0 ballots of
+ * the rows it has just scored, so z is written once and not read again; two
+ * short kernels then place the kept entries.  Any other shape runs the
+ * CUDA-core scan and lsa_select's kernels.
+ *
+ * Arguments as lsa_index_score (full mode: no list, no I output, no flags) and
+ * lsa_select (kept_idx, capacity, kept_off: kept_off[B] is the true total even
+ * when it exceeds capacity, then *err = LSA_ERR_CAPACITY; no mask output).
+ * workspace device scratch of at least
+ *           lsa_index_score_select_workspace_size(n_total, B) bytes, 16-byte
+ *           aligned; contents need not be initialised.
+ * ---------------------------------------------------------------------- */
+size_t lsa_index_score_select_workspace_size(int64_t n_total, int32_t B);
+lsa_status lsa_index_score_select(const void *q, lsa_dtype q_dtype, const float *w,
+                                  const void *k, lsa_dtype k_dtype, const float *k_scale,
+                                  const int64_t *seq_off, int64_t n_total, int32_t B, int32_t H,
+                                  int32_t d, float *z, int32_t *kept_idx, int64_t capacity,
+                                  int64_t *kept_off, void *workspace, size_t ws_bytes,
+                                  int32_t *err, void *stream);
+
+/* ------------------------------------------------------------------------
  * lsa_select_noalloc -- lsa_select without a caller workspace.  The pages
  * have no counterpart: this is a calling convention for callers that cannot
  * allocate device memory when they select (a stream capture that forbids

@@ -131,6 +131,40 @@ lsa_status lsa_select(const float *z, const int64_t *seq_off, int64_t n_total, i
                          as_stream(stream));
 }
 
+size_t lsa_index_score_select_workspace_size(int64_t n_total, int32_t B) {
+    return index_score_select_workspace(n_total, B < 1 ? 1 : B);
+}
+
+lsa_status lsa_index_score_select(const void *q, lsa_dtype q_dtype, const float *w, const void *k,
+                                  lsa_dtype k_dtype, const float *k_scale, const int64_t *seq_off,
+                                  int64_t n_total, int32_t B, int32_t H, int32_t d, float *z, int32_t *kept_idx,
+                                  int64_t capacity, int64_t *kept_off, void *workspace, size_t ws_bytes,
+                                  int32_t *err, void *stream) {
+    clear_error();
+    LSA_CHECK_ARG(q && w && k && seq_off && z && kept_off && workspace,
+                  "lsa_index_score_select: q, w, k, seq_off, z, kept_off and workspace are required");
+    LSA_CHECK_ARG(B >= 1 && H >= 1 && d >= 1, "lsa_index_score_select: B=%d H=%d d=%d must be positive", B, H, d);
+    LSA_CHECK_ARG(n_total >= 0 && n_total < (int64_t(1) << 31),
+                  "lsa_index_score_select: n_total=%lld out of range", (long long)n_total);
+    LSA_CHECK_ARG(valid_dtype(q_dtype) && valid_dtype(k_dtype), "lsa_index_score_select: unknown dtype");
+    LSA_CHECK_SUPPORTED(q_dtype == LSA_F32 || q_dtype == LSA_BF16, "lsa_index_score_select: q must be F32 or BF16");
+    LSA_CHECK_ARG((k_dtype == LSA_E4M3) == (k_scale != nullptr),
+                  "lsa_index_score_select: k_scale is required for E4M3 keys and only for them");
+    LSA_CHECK_SUPPORTED(H <= 64, "lsa_index_score_select: H=%d > 64", H);
+    LSA_CHECK_SUPPORTED(d == 32 || d == 64 || d == 128, "lsa_index_score_select: d=%d not in {32,64,128}", d);
+    LSA_CHECK_ARG((d * elem_size(k_dtype)) % 16 == 0 && aligned16(k),
+                  "lsa_index_score_select: key rows must be 16-byte aligned");
+    LSA_CHECK_ARG(capacity >= 0 && (kept_idx || capacity == 0), "lsa_index_score_select: bad capacity / kept_idx");
+    LSA_CHECK_ARG(ws_bytes >= index_score_select_workspace(n_total, B) && aligned16(workspace),
+                  "lsa_index_score_select: workspace of %zu bytes < %zu", ws_bytes,
+                  index_score_select_workspace(n_total, B));
+    cudaStream_t st = as_stream(stream);
+    if (n_total == 0)
+        return launch_select(z, seq_off, n_total, B, kept_idx, capacity, kept_off, nullptr, workspace, err, st);
+    return launch_index_score_select(q, q_dtype, w, k, k_dtype, k_scale, seq_off, n_total, B, H, d, z, kept_idx,
+                                     capacity, kept_off, workspace, err, st);
+}
+
 lsa_status lsa_topk(const float *z, int32_t z_by_entry, const int64_t *seq_off,
                     const int32_t *kept_idx, const int64_t *kept_off, int64_t kept_capacity,
                     int32_t B, int32_t k, int32_t *topk_idx, int32_t *topk_pos,

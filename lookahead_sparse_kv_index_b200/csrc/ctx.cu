@@ -257,8 +257,14 @@ lsa_status enqueue_scan_select(lsa_ctx *c, const void *q, const float *w, int se
     const size_t w_layer = size_t(p.B) * p.H;                                 // floats of one layer's w
     StageTimer ts(c, LSA_STAGE_SCORE, st);
     if (c->n_layers == 1) {
-        LSA_TRY(launch_index_score(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d, p.n_total,
-                                   nullptr, nullptr, 0, p.B, p.H, p.d, c->z, nullptr, 0, c->err, st));
+        // one indexer layer: the scan with the selection fused into it (the select stage is then empty)
+        LSA_TRY(launch_index_score_select(q, p.q_dtype, w, p.k_dev, p.k_dtype, p.k_scale_dev, c->seq_off_d,
+                                          p.n_total, p.B, p.H, p.d, c->z, c->ks[set].kept_idx, p.kept_capacity,
+                                          c->ks[set].kept_off, c->sel_ws, c->err, st));
+        ts.done();
+        StageTimer tsel(c, LSA_STAGE_SELECT, st);
+        tsel.done();
+        return LSA_OK;
     } else {
         const float *zl[kMaxUnionLayers];
         for (int l = 0; l < c->n_layers; ++l) {
@@ -559,7 +565,7 @@ lsa_status lsa_ctx_create(const lsa_params *pp, lsa_ctx **out) {
     const int64_t cap = p.kept_capacity;
     const size_t qbytes = size_t(p.B) * p.H * p.d * elem_size(p.q_dtype);
     const size_t Qbytes = size_t(p.B) * p.Hq * p.D * elem_size(p.attn_dtype);
-    c->sel_ws_bytes = lsa_select_workspace_size(p.n_total);
+    c->sel_ws_bytes = index_score_select_workspace(p.n_total, p.B);   // covers lsa_select's layout too
     c->attn_ws_bytes = sparse_attn_workspace(p.B, p.Hq, p.D, int32_t(row_cap));
     c->merged = merged;
     c->n_layers = n_layers;

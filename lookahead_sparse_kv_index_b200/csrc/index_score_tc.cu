@@ -340,13 +340,14 @@ __device__ __forceinline__ void tile_info(const int64_t *s_toff, const int64_t *
 // LISTED = true:  entries idx[idx_off[b] ..] of each sequence (rows gathered
 //                 by the producer warp with cp.async); z is written at the list
 //                 position.
-template <int KIND, int H, bool LISTED>
+// SEL (full mode only): the selection's ballots fused into the epilogue (sel_bits, sel_cnt).
+template <int KIND, int H, bool LISTED, bool SEL = false>
 __global__ void __launch_bounds__(kThreads, 1)
 scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kbytes,
         const uint16_t *__restrict__ q, const float *__restrict__ w, int d, const int64_t *__restrict__ seq_off,
         const int32_t *__restrict__ idx, const int64_t *__restrict__ idx_off, int64_t list_cap, int B,
         const float *__restrict__ k_scale, int64_t scale_len, int64_t axis_cap, float *__restrict__ z,
-        float *__restrict__ I, int32_t *err) {
+        float *__restrict__ I, uint32_t *__restrict__ sel_bits, int32_t *__restrict__ sel_cnt, int32_t *err) {
     using C = Cfg<KIND>;
     constexpr int S = C::kStages;
     constexpr int QIMG = qimg_bytes<KIND, H>();
@@ -785,6 +786,7 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
             // chunk is in registers
             constexpr int HC = H < 32 ? H : 32;   // heads per chunk
             constexpr int NP = is_e4m3(KIND) ? 2 : 1;
+            [[maybe_unused]] int kept = 0;   // fused selection: this warp's kept rows of the tile
 #pragma unroll
             for (int sub = 0; sub < C::kSub; ++sub) {
                 const float sc = kScales ? s_scale[int(i % RS) * SS + soff + sub * kRows + quarter * 32 + lane] : 1.f;
@@ -819,13 +821,25 @@ scan_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ kb
                     }
                 }
                 float zs = (za + zb) + (zc + zd);
+                if constexpr (SEL)
+                    if (kScales) zs *= sc;
                 const int64_t row = row0 + sub * kRows + quarter * 32 + lane;   // entry (full) or list position
                 if (row < row_end) {
-                    if (kScales) zs *= sc;
+                    if constexpr (!SEL)
+                        if (kScales) zs *= sc;
                     z[row] = zs;
                     if (I) I[row] = 1.f / (1.f + expf(-zs));
                 }
+                if constexpr (SEL) {
+                    // fused selection (I >= 0.5 <=> z >= 0): bit `lane` of word 4 sub + quarter of tile t is
+                    // row row0 + 128 sub + 32 quarter + lane
+                    const uint32_t word = __ballot_sync(0xffffffffu, row < row_end && zs >= 0.f);
+                    if (lane == 0) sel_bits[t * (4 * C::kSub) + 4 * sub + quarter] = word;
+                    kept += __popc(word);
+                }
             }
+            if constexpr (SEL)
+                if (lane == 0) sel_cnt[t * 4 + quarter] = kept;
         }
         release_to(nord);   // every sequence of the range
     }
@@ -883,6 +897,8 @@ struct ScanArgs {
     int32_t *err;
     int64_t axis_cap;         // full mode over a device-produced axis: its capacity (0: seq_off is constant)
     int64_t scale_len;        // entries of k_scale
+    uint32_t *sel_bits = nullptr;   // fused selection (full mode): per tile, one ballot word per 32 rows
+    int32_t *sel_cnt = nullptr;     // ... and the kept rows of each of its 4 row quarters
 };
 
 template <int KIND, int H>
@@ -908,14 +924,14 @@ lsa_status launch(const ScanArgs &a, cudaStream_t st) {
         return LSA_ERR_CUDA;
     }
     const size_t smem = smem_bytes<KIND, H>(a.B);
-    auto kern = a.idx ? scan_tc<KIND, H, true> : scan_tc<KIND, H, false>;
+    auto kern = a.idx ? scan_tc<KIND, H, true> : (a.sel_bits ? scan_tc<KIND, H, false, true> : scan_tc<KIND, H, false>);
     LSA_CUDA(ensure_smem(kern, smem));
     const int64_t axis = a.idx ? a.list_cap : (a.axis_cap > 0 ? a.axis_cap : a.n_total);
     const int64_t max_tiles = (axis + tile_rows<KIND>() - 1) / tile_rows<KIND>() + a.B;
     const int grid = int(max_tiles < sm_count() ? max_tiles : sm_count());
     LSA_CUDA(launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, map, static_cast<const uint8_t *>(a.k),
                         static_cast<const uint16_t *>(a.q), a.w, a.d, a.seq_off, a.idx, a.idx_off, a.list_cap, a.B,
-                        a.k_scale, a.scale_len, a.axis_cap, a.z, a.I, a.err));
+                        a.k_scale, a.scale_len, a.axis_cap, a.z, a.I, a.sel_bits, a.sel_cnt, a.err));
     static const char *kNames[2][4] = {
         {"scan_tc bf16 d128", "scan_tc bf16 d64", "scan_tc e4m3 d128", "scan_tc e4m3 d64"},
         {"scan_tc_listed bf16 d128", "scan_tc_listed bf16 d64", "scan_tc_listed e4m3 d128", "scan_tc_listed e4m3 d64"}};
@@ -956,6 +972,20 @@ lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, l
                                  const int32_t *idx, const int64_t *idx_off, int64_t list_cap, int32_t B,
                                  int32_t H, int32_t d, float *z, float *I, int32_t *err, cudaStream_t st) {
     const ScanArgs a{q, w, k, k_scale, seq_off, n_total, idx, idx_off, list_cap, B, d, z, I, err, 0, n_total};
+    return launch_kind(k_dtype, H, a, st);
+}
+
+int index_score_tc_tile_rows(lsa_dtype k_dtype) {
+    return k_dtype == LSA_E4M3 ? tile_rows<E4M3_D128>() : tile_rows<BF16_D128>();
+}
+
+lsa_status launch_index_score_tc_select(const void *q, const float *w, const void *k, lsa_dtype k_dtype,
+                                        const float *k_scale, const int64_t *seq_off, int64_t n_total, int32_t B,
+                                        int32_t H, int32_t d, float *z, uint32_t *sel_bits, int32_t *sel_cnt,
+                                        int32_t *err, cudaStream_t st) {
+    ScanArgs a{q, w, k, k_scale, seq_off, n_total, nullptr, nullptr, 0, B, d, z, nullptr, err, 0, n_total};
+    a.sel_bits = sel_bits;
+    a.sel_cnt = sel_cnt;
     return launch_kind(k_dtype, H, a, st);
 }
 

@@ -98,6 +98,22 @@ lsa_status launch_index_score_tc(const void *q, const float *w, const void *k, l
 // Full tensor-core scan over a device-produced row axis: rows axis_off[b] .. axis_off[b+1] (clamped to
 // axis_cap) of the key array k [n_rows, d] belong to sequence b; z is written per row.  Used on a compacted
 // copy of the kept keys (rows in kept-list order), so z lands at the kept position.
+// The full tensor-core scan that also writes the z >= 0 ballots of each scan tile (TR / 32 words) and the
+// kept count of each quarter of the tile, for the fused selection; TR = index_score_tc_tile_rows.
+int index_score_tc_tile_rows(lsa_dtype k_dtype);
+lsa_status launch_index_score_tc_select(const void *q, const float *w, const void *k, lsa_dtype k_dtype,
+                                        const float *k_scale, const int64_t *seq_off, int64_t n_total, int32_t B,
+                                        int32_t H, int32_t d, float *z, uint32_t *sel_bits, int32_t *sel_cnt,
+                                        int32_t *err, cudaStream_t st);
+// Full scan + selection: fused on the tensor-core path, else the CUDA-core scan and lsa_select's kernels.
+// workspace: index_score_select_workspace(n_total, B) bytes (covers both).
+size_t select_tiles_workspace(int64_t n_total, int32_t B);
+size_t index_score_select_workspace(int64_t n_total, int32_t B);
+lsa_status launch_index_score_select(const void *q, lsa_dtype q_dtype, const float *w, const void *k,
+                                     lsa_dtype k_dtype, const float *k_scale, const int64_t *seq_off,
+                                     int64_t n_total, int32_t B, int32_t H, int32_t d, float *z, int32_t *kept_idx,
+                                     int64_t capacity, int64_t *kept_off, void *workspace, int32_t *err,
+                                     cudaStream_t st);
 lsa_status launch_index_score_tc_axis(const void *q, const float *w, const void *k, lsa_dtype k_dtype,
                                       const float *k_scale, int64_t scale_len, const int64_t *axis_off,
                                       int64_t axis_cap, int64_t n_rows, int32_t B, int32_t H, int32_t d, float *z,

@@ -37,7 +37,8 @@ EXPORTS = [
     "lsa_ctx_create", "lsa_ctx_destroy", "lsa_decode_step", "lsa_decode_step_host", "lsa_ctx_get_view",
     "lsa_ctx_set_graphs", "lsa_ctx_set_timing", "lsa_ctx_stage_times", "lsa_ctx_reset_counters",
     "lsa_ctx_launches", "lsa_selftest_bounded_wait", "lsa_index_union", "lsa_query_encode",
-    "lsa_attn_set_merge", "lsa_struct_size", "lsa_ctx_flush_cache",
+    "lsa_attn_set_merge", "lsa_struct_size", "lsa_ctx_flush_cache", "lsa_index_score_select_workspace_size",
+    "lsa_index_score_select",
 ]
 
 
@@ -79,6 +80,8 @@ _sig("lsa_status_name", ctypes.c_char_p, [i32])
 _sig("lsa_index_score", i32, [P, i32, P, P, i32, P, P, i64, P, P, i64, i32, i32, i32, P, P, i32, P, P])
 SCORE_CUDA_CORE = 1
 _sig("lsa_select_workspace_size", sz, [i64])
+_sig("lsa_index_score_select_workspace_size", sz, [i64, i32])
+_sig("lsa_index_score_select", i32, [P, i32, P, P, i32, P, P, i64, i32, i32, i32, P, P, i64, P, P, sz, P, P])
 _sig("lsa_select", i32, [P, P, i64, i32, P, i64, P, P, P, sz, P, P])
 _sig("lsa_select_noalloc_max_entries", i64, [])
 _sig("lsa_select_noalloc", i32, [P, P, i64, i32, P, i64, P, P, P, P])
@@ -147,6 +150,20 @@ def index_score(q, q_dtype, w, k, k_dtype, k_scale, seq_off, n_total, H, d, z, I
 
 def select_workspace_size(n_total) -> int:
     return int(_L.lsa_select_workspace_size(n_total))
+
+
+def index_score_select_workspace_size(n_total, B) -> int:
+    return int(_L.lsa_index_score_select_workspace_size(n_total, B))
+
+
+def index_score_select(q, q_dtype, w, k, k_dtype, k_scale, seq_off, n_total, H, d, z, kept_idx, capacity, kept_off,
+                       workspace, err=None, stream=None):
+    """Full index scan and threshold selection in one call (fused on the tensor-core path; see lsa.h)."""
+    B = seq_off.numel() - 1
+    _check(_L.lsa_index_score_select(_ptr(q), DTYPE[q_dtype], _ptr(w), _ptr(k), DTYPE[k_dtype], _ptr(k_scale),
+                                     _ptr(seq_off), n_total, B, H, d, _ptr(z), _ptr(kept_idx), capacity,
+                                     _ptr(kept_off), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _ptr(err), _stream(stream)), "lsa_index_score_select")
 
 
 def select(z, seq_off, n_total, kept_idx, capacity, kept_off, mask, workspace, err, stream=None):

@@ -170,6 +170,72 @@ def test_select_capacity_overflow(lsa):
     assert np.array_equal(kept, k_ref[:cap])
 
 
+# ------------------------------------------------- scan + select, fused
+
+def _score_select_gpu(lsa, wl, dev, capacity=None):
+    n = wl.n_total
+    B = len(wl.seq_off) - 1
+    cap = n if capacity is None else capacity
+    z = torch.full((max(n, 1) + 64,), 77.0, dtype=torch.float32, device="cuda")
+    kept_idx = torch.full((max(cap, 1) + 16,), -7, dtype=torch.int32, device="cuda")
+    kept_off = torch.full((B + 1,), -7, dtype=torch.int64, device="cuda")
+    ws = torch.full((lsa.index_score_select_workspace_size(n, B),), 0xA5, dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lsa.index_score_select(dev["q"], wl.q_dtype, dev["w"], dev["keys"], wl.key_dtype, dev["k_scale"], dev["seq_off"],
+                           n, wl.H, wl.d, z, kept_idx, cap, kept_off, ws, err=err)
+    torch.cuda.synchronize()
+    kernel = lsa.last_kernel()
+    kept = kept_idx.cpu().numpy()
+    assert (kept[cap:] == -7).all(), "selection wrote past the capacity"
+    assert (z[n:].cpu().numpy() == 77.0).all(), "scan wrote past the entry axis"
+    return z[:n].cpu().numpy(), kept, kept_off.cpu().numpy(), int(err.item()), kernel
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_bf16", "ragged_e4m3", "ragged_e4m3_d64_h16", "ragged_bf16_d64_h32",
+                                  "ragged_bf16_h16", "ragged_e4m3_h32"])
+def test_index_score_select_fused_matches_stages(lsa, name):
+    """The fused scan + select gives the full scan's z bit for bit and, on those scores, the oracle's kept lists
+    (sequences of every length modulo the tile: empty, 1, one tile, a ragged tail)."""
+    wl = SCORE_CASES[name]()
+    dev = synth.to_torch(wl, pin_cold=False)
+    z, kept, ko, err, kernel = _score_select_gpu(lsa, wl, dev)
+    assert err == 0
+    if wl.q_dtype == "bf16":   # the tensor-core shapes: the selection comes from the scan's ballots
+        assert kernel == "select_tiles_scatter"
+    z_sep, _ = gpu_full_scores(wl, dev, lsa, want_I=False, tc=True)
+    assert np.array_equal(z.view(np.uint32), z_sep.view(np.uint32))
+    k_ref, ko_ref, _ = oracle.select(z.astype(np.float64), wl.seq_off)
+    assert np.array_equal(ko, ko_ref)
+    assert np.array_equal(kept[:len(k_ref)], k_ref)
+
+
+def test_index_score_select_fused_capacity_overflow(lsa):
+    wl = synth.small_ragged(key_dtype="e4m3", lengths=(5000, 300, 0, 129))
+    dev = synth.to_torch(wl, pin_cold=False)
+    z, kept_full, ko_full, err, _ = _score_select_gpu(lsa, wl, dev)
+    assert err == 0
+    total = int(ko_full[-1])
+    cap = total // 2
+    z2, kept, ko, err, _ = _score_select_gpu(lsa, wl, dev, capacity=cap)
+    assert err == 3                                       # LSA_ERR_CAPACITY
+    assert np.array_equal(ko, ko_full)                    # true offsets even past capacity
+    assert np.array_equal(kept[:cap], kept_full[:cap])
+
+
+def test_index_score_select_fused_full_size_500k(lsa):
+    """The 500K-token batch (4 x 131072 e4m3 entries): the fused kept lists against the oracle's selection of the
+    same scores, and equal to lsa_select's."""
+    wl = synth.ctx500k(with_cold=False)
+    dev = synth.to_torch(wl, pin_cold=False)
+    z, kept, ko, err, kernel = _score_select_gpu(lsa, wl, dev)
+    assert err == 0 and kernel == "select_tiles_scatter"
+    k_ref, ko_ref, _ = oracle.select(z.astype(np.float64), wl.seq_off)
+    assert np.array_equal(ko, ko_ref)
+    assert np.array_equal(kept[:len(k_ref)], k_ref)
+    kept2, ko2, _, err2 = gpu_select(z, wl.seq_off, lsa)
+    assert err2 == 0 and np.array_equal(ko2, ko) and np.array_equal(kept2[:len(k_ref)], k_ref)
+
+
 # ----------------------------------------------------------------- top-k
 
 def _topk_gpu(lsa, z, z_by_entry, seq_off, kept, ko, k, cap=None):
