@@ -106,8 +106,8 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
     uint64_t *kv_full = qfull + kQSlices;        // [kD / 64] column blocks of the rows
     uint64_t *s_full = kv_full + kD / 64;
     uint64_t *p_full = s_full + 1;
-    uint64_t *o_full = p_full + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_full + 1);
+    uint64_t *o_full = p_full + 1;               // [2]: O columns 0..255 and 256..511 done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_full + 2);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     int *s_nvalid = abort_flag + 1;
     uint32_t *s_valid = reinterpret_cast<uint32_t *>(s_nvalid + 1);   // [2] bit j % 32 of word j / 32: row j selected
@@ -128,7 +128,8 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
         for (int kb = 0; kb < kD / 64; ++kb) mbar_init(&kv_full[kb], 32 * kSoftWarps);
         mbar_init(s_full, 1);
         mbar_init(p_full, kSoftWarps);
-        mbar_init(o_full, 1);
+        mbar_init(&o_full[0], 1);
+        mbar_init(&o_full[1], 1);
         fence_mbar_init();
     }
     if (warp == kMmaWarp) {
@@ -258,11 +259,11 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
-            // ---- O: each half converts its 256 columns, 64-column blocks staged in the (now free) Q
-            // buffer, each in its own 16 KB buffer, one TMA store per block
-            ok = mbar_wait(o_full, 0, abort_v, kWaitLimitNs);
-            // the block loop below synchronises these 256 threads: agree on one outcome first
-            if (named_barrier_and(1, 32 * kSoftWarps, ok)) {
+            // ---- O: each half converts its 256 columns as soon as their MMAs are done, 64-column blocks
+            // staged in the (now free) Q buffer, each in its own 16 KB buffer, one TMA store per block
+            ok = mbar_wait(&o_full[half], 0, abort_v, kWaitLimitNs);
+            // the block loop below synchronises the 128 threads of this half: agree on one outcome first
+            if (named_barrier_and(2 + half, 128, ok)) {
                 tc_fence_after();
                 l = s_sum[2 * head] + s_sum[2 * head + 1];
 #pragma unroll 1
@@ -330,13 +331,14 @@ attn_tc(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtens
                     tc_fence_after();
                     const uint32_t p_u32 = smem_u32(ps);
 #pragma unroll
-                    for (int half = 0; half < 2; ++half)
+                    for (int half = 0; half < 2; ++half) {
 #pragma unroll
                         for (int kk = 0; kk < kRowsPerCta / 16; ++kk)
                             mma_f16(tmem + half * 256, desc_sw128(p_u32 + kk * 32),
                                     desc_sw128_mn(kv_u32 + half * 4 * kKvBlock + kk * 2048, kKvBlock), IDESC_O,
                                     kk != 0);
-                    mma_commit(o_full);
+                        mma_commit(&o_full[half]);   // this half's epilogue may start
+                    }
                 }
             }
             if (!ok) {
@@ -378,7 +380,7 @@ EncodeTiledFn encode_fn() {
 }
 
 constexpr size_t kSmemBytes = 1024 + size_t(kKvBytes) + size_t(kQSlices) * kQStageBytes +
-                              (kQSlices + kD / 64 + 3) * 8 + 16 + 16 + 4 * kHq * 4 + 16 + kRowsPerCta * 4 + 64;
+                              (kQSlices + kD / 64 + 4) * 8 + 16 + 16 + 4 * kHq * 4 + 16 + kRowsPerCta * 4 + 64;
 
 }  // namespace
 
