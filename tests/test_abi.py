@@ -93,6 +93,34 @@ def test_other_entry_points_reject_bad_arguments(lsa):
     assert L.lsa_index_union(arr, 3, 10, big, None) == 1                      # a layer without scores
 
 
+def _score_select(lsa, **kw):
+    big = 1 << 20
+    a = dict(q=big, qd=1, w=big, k=big, kd=1, ks=None, so=big, n=1000, B=2, H=64, d=128, z=big, kept=big, cap=1000,
+             ko=big, ws=big, wsb=1 << 30)
+    a.update(kw)
+    return lsa.lib.lsa_index_score_select(a["q"], a["qd"], a["w"], a["k"], a["kd"], a["ks"], a["so"], a["n"], a["B"],
+                                          a["H"], a["d"], a["z"], a["kept"], a["cap"], a["ko"], a["ws"], a["wsb"],
+                                          None, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(z=None), 1), (dict(ko=None), 1), (dict(ws=None), 1), (dict(B=0), 1),
+    (dict(H=65), 5), (dict(d=96), 5), (dict(kd=2), 1), (dict(ks=1 << 20), 1), (dict(qd=2), 5),
+    (dict(n=-1), 1), (dict(cap=-1), 1), (dict(kept=None), 1), (dict(wsb=16), 1), (dict(ws=(1 << 20) + 8), 1),
+])
+def test_index_score_select_rejects_bad_arguments(lsa, kw, status):
+    assert _score_select(lsa, **kw) == status
+    assert lsa.lib.lsa_last_error() != b""
+
+
+def test_index_score_select_workspace_covers_both_paths(lsa):
+    for n, B in [(1, 1), (1000, 3), (4 * 131072, 4), (2_200_000, 64)]:
+        ws = lsa.index_score_select_workspace_size(n, B)
+        assert ws >= lsa.select_workspace_size(n)          # the CUDA-core scan + lsa_select fallback
+        # the fused path: per scan tile of >= 128 rows, 8 ballot words, 4 counts, base, first row, sequence
+        assert ws >= ((n + 127) // 128 + B) * (32 + 16 + 8 + 8 + 4)
+
+
 def test_struct_mirrors_match_the_header(lsa):
     assert lsa.lib.lsa_struct_size(0) == ctypes.sizeof(lsa.Params)
     assert lsa.lib.lsa_struct_size(1) == ctypes.sizeof(lsa.View)
